@@ -1,0 +1,359 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself -- a closed form, a brute-force construction, a textbook routine or a
+figure printed on the pages.  No GPU needed."""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import shampoo4_oracle as O
+from pinlib import (coupled_newton_inverse_root, jacobi_eigh, random_orthogonal,
+                    spd_with_spectrum)
+
+EPS0 = 1e-300   # "eps -> 0" for the fp64 limits
+
+
+def _converged_state(S: np.ndarray, eps: float, iters: int = 400):
+    """Run quant-off refreshes with S fixed until the subspace iteration has
+    converged; returns (U, lam)."""
+    f = O.Factor(S.shape[0], S.astype(np.float32))
+    for _ in range(iters):
+        O.refresh_factor(f, eps, 0, quant=False)
+    return f.U64, f.lam
+
+
+# ---------------------------------------------------------------- codec (P7)
+
+def test_codebook_is_signed_square_of_linear_grid():
+    cb = O.codebook_f64()
+    y = np.linspace(-1.0, 1.0, 16)           # the linear grid, independently
+    assert np.allclose(cb, np.sign(y) * y * y, rtol=0, atol=1e-15)
+    assert cb[0] == -1.0 and cb[-1] == 1.0
+    assert np.all(np.diff(cb) > 0)
+    assert not np.any(cb == 0.0)             # 16 levels, no exact zero
+    t = O.thresholds_f32()
+    assert t[7] == 0.0 and np.all(np.diff(t) > 0)
+
+
+def test_codebook_points_roundtrip_exactly():
+    rng = np.random.default_rng(1)
+    cb32 = O.codebook_f32()
+    for k in (-20, -3, 0, 5):
+        j = rng.integers(0, 16, size=640)
+        j[::64] = 15                         # absmax element = +2^k in every block
+        x = (cb32[j] * np.float32(2.0 ** k)).astype(np.float32)
+        codes, scales = O.quantize(x)
+        assert np.all(scales == np.float32(2.0 ** k))
+        assert np.array_equal(O.unpack_nibbles(codes, x.size), j.astype(np.uint8))
+        assert np.array_equal(O.dequantize(codes, scales, x.size), x)
+
+
+def test_quantizer_is_nearest_level_rounding_near_every_threshold():
+    # Brute force: 2^16 consecutive fp32 bit patterns around each threshold.
+    # The count rule must agree with nearest-codebook-level rounding (fp64
+    # distances) except exactly on a threshold, where it takes the lower code.
+    t = O.thresholds_f32()
+    cb = O.codebook_f64()
+    vals = []
+    for tk in t:
+        if tk == 0.0:
+            base = np.arange(-32768, 32768, dtype=np.int64)
+            pos = base[base >= 0].astype(np.uint32).view(np.float32)
+            neg = (-base[base > 0]).astype(np.uint32).view(np.float32) * np.float32(-1)
+            vals.append(pos); vals.append(neg)
+        else:
+            b = np.array([tk], np.float32).view(np.uint32)[0].astype(np.int64)
+            vals.append((b + np.arange(-32768, 32768)).astype(np.uint32).view(np.float32))
+    v = np.concatenate(vals).astype(np.float32)
+    v = v[np.abs(v) <= 1.0]
+    nblk = (v.size + 62) // 63
+    x = np.zeros(nblk * 64, np.float32)
+    x.reshape(nblk, 64)[:, 0] = 1.0          # absmax 1 -> v = x exactly
+    flat = x.reshape(nblk, 64)[:, 1:].ravel()
+    flat[:v.size] = v
+    x.reshape(nblk, 64)[:, 1:] = flat.reshape(nblk, 63)
+    codes, scales = O.quantize(x)
+    assert np.all(scales == 1.0)
+    got = O.unpack_nibbles(codes, x.size).reshape(nblk, 64)[:, 1:].ravel()[:v.size]
+    # Nearest level, computed exactly: level j is nearest iff v lies between
+    # the exact midpoints (a_{j-1}+a_j)/450 and (a_j+a_{j+1})/450 with
+    # a_j = (2j-15)|2j-15| integers; 450 v is exact in fp64.
+    a = np.array([(2 * j - 15) * abs(2 * j - 15) for j in range(16)], np.float64)
+    assert np.array_equal(a / 225, cb)
+    w = 450.0 * v.astype(np.float64)
+    nearest = np.sum(w[:, None] > (a[:-1] + a[1:])[None, :], axis=1)
+    on_thr = np.isin(v, t)
+    assert np.array_equal(got[~on_thr], nearest[~on_thr])
+    for k, tk in enumerate(t):
+        assert np.all(got[v == tk] == k)
+
+
+def test_quantizer_error_bound_and_absmax_exact():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal(64 * 257 + 13).astype(np.float32)
+    codes, scales = O.quantize(x)
+    xr = O.dequantize(codes, scales, x.size)
+    cb = O.codebook_f64()
+    half_gap = np.max(np.diff(cb)) / 2          # 28/225
+    assert abs(half_gap - 28 / 225) < 1e-15
+    s = np.repeat(scales, 64)[:x.size].astype(np.float64)
+    err = np.abs(x.astype(np.float64) - xr.astype(np.float64))
+    assert np.all(err <= half_gap * s * (1 + 1e-6) + 1e-30)
+    c = O.unpack_nibbles(codes, x.size)
+    for b in range(scales.size):
+        blk = slice(64 * b, min(64 * b + 64, x.size))
+        i = np.argmax(np.abs(x[blk]))
+        assert c[blk][i] in (0, 15)
+        assert abs(xr[blk][i]) == scales[b]
+
+
+def test_quantizer_zero_block_ragged_tail_and_packing():
+    x = np.zeros(64 + 65, np.float32)
+    x[64:] = np.linspace(-1, 1, 65, dtype=np.float32)
+    codes, scales = O.quantize(x)
+    assert codes.size == (x.size + 1) // 2 and scales.size == 3
+    assert scales[0] == 0.0 and scales[2] == 1.0       # ragged last block of 1
+    assert np.all(O.dequantize(codes, scales, x.size)[:64] == 0.0)
+    # one element per 2 nibbles, even index low; padded high nibble is 0
+    c = O.unpack_nibbles(codes, x.size)
+    assert codes[-1] >> 4 == 0
+    assert np.array_equal(codes[:-1], c[0:-1:2] | (c[1::2] << 4))
+
+
+def test_quantizer_nonfinite_rule():
+    x = np.ones(192, np.float32)
+    x[3] = np.nan
+    x[64 + 5] = np.inf
+    codes, scales = O.quantize(x)
+    assert np.isnan(scales[0]) and scales[1] == np.inf and scales[2] == 1.0
+    c = O.unpack_nibbles(codes, x.size)
+    assert np.all(c[:64] == 0)                 # NaN scale: every comparison fails
+    assert c[64 + 5] == 0                      # inf / inf = NaN
+    assert np.all(np.delete(c[64:128], 5) == 7)   # 1 / inf = +0 -> code 7
+
+
+# ------------------------------------------------------------ stats (EMA)
+
+def test_ema_stats_closed_form_and_sides():
+    G = np.zeros((3, 5), np.float32)
+    G[0, 1] = 2.0
+    G[2, 4] = -1.0
+    beta = float(np.float32(0.95))
+    SL = np.zeros((3, 3), np.float32)
+    SR = np.zeros((5, 5), np.float32)
+    for _ in range(7):
+        SL = O.ema_stats(SL, G, beta, "L")
+        SR = O.ema_stats(SR, G, beta, "R")
+    w = 1 - beta ** 7                          # geometric series sum (1-b) b^i
+    eL = np.zeros((3, 3)); eL[0, 0] = 4 * w; eL[2, 2] = w
+    eR = np.zeros((5, 5)); eR[1, 1] = 4 * w; eR[4, 4] = w
+    assert np.allclose(SL, eL, rtol=1e-6, atol=0)
+    assert np.allclose(SR, eR, rtol=1e-6, atol=0)
+
+
+# ------------------------------------------------------------ Bjorck (P4)
+
+def test_bjorck_closed_form_on_svd():
+    rng = np.random.default_rng(3)
+    d = 12
+    Q1, Q2 = random_orthogonal(d, rng), random_orthogonal(d, rng)
+    s = rng.uniform(0.2, 2.0, d)
+    U = (Q1 * s) @ Q2.T
+    got = O.bjorck(U, 1)
+    want = (Q1 * (s * (1.5 - 0.5 * s * s))) @ Q2.T
+    assert np.allclose(got, want, rtol=0, atol=1e-13)
+
+
+def test_bjorck_orthogonality_residual_decreases_on_dequantized_basis():
+    rng = np.random.default_rng(4)
+    d = 96
+    Q = random_orthogonal(d, rng).astype(np.float32)
+    codes, scales = O.quantize(Q.ravel())
+    U = O.dequantize(codes, scales, d * d).reshape(d, d).astype(np.float64)
+    res = [np.linalg.norm(U.T @ U - np.eye(d))]
+    for _ in range(5):
+        U = O.bjorck(U, 1)
+        res.append(np.linalg.norm(U.T @ U - np.eye(d)))
+    assert res[0] > 1e-2
+    assert all(b < a for a, b in zip(res[:3], res[1:4]))
+    assert res[-1] < 1e-12
+
+
+# ----------------------------------------------------- eigenpairs (P5, P8)
+
+def test_subspace_iteration_converges_to_jacobi_eigenpairs():
+    rng = np.random.default_rng(5)
+    d = 20
+    lam_true = 0.7 ** np.arange(d)              # distinct, ratio 0.7
+    S = spd_with_spectrum(lam_true, rng).astype(np.float32)
+    U, lam = _converged_state(S, EPS0, iters=300)
+    S64 = S.astype(np.float64)
+    lj, Vj = jacobi_eigh(S64)
+    assert np.allclose(lam, lj, rtol=1e-10, atol=1e-14)
+    assert np.linalg.norm(S64 @ U - U * lam[None, :]) <= 1e-10 * np.linalg.norm(S64)
+    # columns equal Jacobi's eigenvectors up to sign
+    cos = np.abs(np.sum(U * Vj, axis=0))
+    assert np.all(np.abs(cos - 1) < 1e-9)
+    # third opinion: LAPACK eigh
+    le = np.linalg.eigvalsh(S64)[::-1]
+    assert np.allclose(lam, le, rtol=1e-10, atol=1e-14)
+
+
+def test_subspace_step_is_the_qr_factor_with_positive_diagonal():
+    rng = np.random.default_rng(8)
+    d = 9
+    G = rng.standard_normal((d, 4))
+    S = (G @ G.T).astype(np.float32)             # rank 4: zero eigenvalues
+    U = random_orthogonal(d, rng)
+    eps = 1e-3
+    Q, lam = O.subspace_step(S, U, eps)
+    Y = (S.astype(np.float64) + eps * np.eye(d)) @ U
+    R = Q.T @ Y                                  # Y = Q R  =>  R = Q^T Y
+    assert np.allclose(Q.T @ Q, np.eye(d), atol=1e-13)
+    assert np.allclose(np.tril(R, -1), 0, atol=1e-12)
+    assert np.all(np.diag(R) > 0)
+    assert np.all(lam >= 0)
+    assert np.allclose(lam, np.maximum(np.diag(Q.T @ S.astype(np.float64) @ Q), 0), atol=1e-14)
+
+
+def test_diagonal_statistic_with_identity_start_is_exact():
+    lam_star = np.array([3.0, 0.5, 0.25, 2.0, 1e-3], np.float32)
+    S = np.diag(lam_star).astype(np.float32)
+    Q, lam = O.subspace_step(S, np.eye(5), 1e-6)
+    assert np.array_equal(Q, np.eye(5))
+    assert np.array_equal(lam, lam_star.astype(np.float64))
+    # and the step D = diag(mu_L) G diag(mu_R) exactly (quant off)
+    orc = O.Shampoo4Oracle([(5, 3)], quant=False)
+    for f, d in zip(orc.factors, (5, 3)):
+        f.S = np.diag(lam_star[:d]).astype(np.float32)
+    orc.refresh_roots()
+    G = np.arange(15, dtype=np.float32).reshape(5, 3) - 7
+    D = orc.precondition([G])[0]
+    muL = (lam_star[:5].astype(np.float64) + orc.eps) ** -0.25
+    muR = (lam_star[:3].astype(np.float64) + orc.eps) ** -0.25
+    want = (muL[:, None] * G.astype(np.float64) * muR[None, :]).astype(np.float32)
+    assert np.array_equal(D, want)
+
+
+# ----------------------------------------------------------- root (P6)
+
+def test_root_matches_coupled_newton_and_fourth_power():
+    rng = np.random.default_rng(6)
+    d = 16
+    lam_true = np.geomspace(2.0, 1e-4, d)
+    S = spd_with_spectrum(lam_true, rng).astype(np.float32)
+    eps = 1e-6
+    U, lam = _converged_state(S, eps, iters=600)
+    P = O.root_from_basis(U, lam, eps)
+    A = S.astype(np.float64) + eps * np.eye(d)
+    X = coupled_newton_inverse_root(A, 4)
+    assert np.linalg.norm(P - X) <= 1e-10 * np.linalg.norm(X)
+    P4 = np.linalg.matrix_power(P, 4)
+    assert np.linalg.norm(P4 @ A - np.eye(d)) < 1e-9
+
+
+# -------------------------------------- Kronecker identity and bound (P1)
+
+@pytest.mark.parametrize("m,n", [(2, 3), (3, 2), (4, 4), (2, 2)])
+def test_update_equals_kronecker_preconditioner_on_vec(m, n):
+    rng = np.random.default_rng(10 * m + n)
+    orc = O.Shampoo4Oracle([(m, n)], eps=1e-6, quant=False)
+    for _ in range(6):
+        orc.update_stats([rng.standard_normal((m, n)).astype(np.float32)])
+    for _ in range(300):
+        orc.refresh_roots()
+    G = rng.standard_normal((m, n)).astype(np.float32)
+    D = orc.precondition([G])[0].astype(np.float64)
+    PL = O.factor_root(orc.factors[0], orc.eps, False)
+    PR = O.factor_root(orc.factors[1], orc.eps, False)
+    vec = lambda X: X.reshape(-1, order="F")           # column-major vec
+    assert np.allclose(vec(D), np.kron(PR, PL) @ vec(G.astype(np.float64)),
+                       rtol=1e-6, atol=1e-7)           # D is stored fp32
+    # The page's route: (R^(1/2) kron L^(1/2))^(-1/2) acting on vec(G), with
+    # the eps-shifted factors, built from LAPACK eigh on the full mn x mn
+    # matrix -- no use of the oracle's own eigen machinery.
+    def sqrtm(A):
+        w, V = np.linalg.eigh(A)
+        return (V * np.sqrt(w)) @ V.T
+    Le = orc.factors[0].S.astype(np.float64) + orc.eps * np.eye(m)
+    Re = orc.factors[1].S.astype(np.float64) + orc.eps * np.eye(n)
+    K = np.kron(sqrtm(Re), sqrtm(Le))
+    w, V = np.linalg.eigh(K)
+    Kmh = (V * w ** -0.5) @ V.T
+    assert np.allclose(vec(D), Kmh @ vec(G.astype(np.float64)), rtol=2e-6, atol=1e-6)
+
+
+# ------------------------------------------------------ homogeneity (P2)
+
+def test_step_is_homogeneous_of_degree_zero():
+    rng = np.random.default_rng(7)
+    G = rng.standard_normal((6, 6)).astype(np.float32)
+    outs, codes = [], []
+    for scale, quant in ((1, False), (2, False), (1, True), (2, True)):
+        orc = O.Shampoo4Oracle([(6, 6)], eps=EPS0, quant=quant)
+        D = orc.step(1, [G * np.float32(scale)], refresh_every=1)[0]
+        outs.append(D.astype(np.float64))
+        codes.append([f.codes for f in orc.factors] if quant else None)
+    assert np.linalg.norm(outs[0] - outs[1]) <= 1e-12 * np.linalg.norm(outs[0])
+    for a, b in zip(codes[2], codes[3]):
+        assert np.array_equal(a, b)
+    assert np.linalg.norm(outs[2] - outs[3]) <= 1e-6 * np.linalg.norm(outs[2])
+
+
+# ------------------------------------------------------ partition (a1)
+
+def test_partition_counts_for_the_workload_shapes():
+    from bit_quantized_shampoo_b200.workloads import WORKLOADS
+    b5 = O.partition(WORKLOADS[5].shapes, 1024)
+    # 4096 x 11008 -> 4 row chunks x (10 full + one 768) = 44 blocks, x8;
+    # 4096 x 4096 -> 16 blocks, x8.
+    assert len(b5) == 4 * 11 * 8 + 16 * 8 == 480
+    dims = [d for b in b5 for d in (b.m, b.n)]
+    assert dims.count(1024) == 928 and dims.count(768) == 32
+    b4 = O.partition(WORKLOADS[4].shapes, 1024)
+    # per layer: 768x2304 -> 1024+1024+256; 768x768 -> 1; 768x3072 -> 3;
+    # 3072x768 -> 3 row chunks.
+    assert len(b4) == 12 * (3 + 1 + 3 + 3)
+    assert sorted({(b.m, b.n) for b in b4}) == [(768, 256), (768, 768), (768, 1024), (1024, 768)]
+    b1 = O.partition(WORKLOADS[1].shapes, 1024)
+    assert [(b.m, b.n) for b in b1] == [(128, 128)]
+    # a ragged tail is kept, not rebalanced
+    assert [(b.r0, b.m) for b in O.partition([(2500, 10)], 1024)] == [(0, 1024), (1024, 1024), (2048, 452)]
+
+
+# ------------------------------------------------------ cost model (P9)
+
+def _golden_costs():
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "shampoo_cost_model.txt")
+    out = {}
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        k, v, tol, _ = [p.strip() for p in line.split("|")]
+        out[k] = (float(v), float(tol))
+    return out
+
+
+def test_cost_model_reproduces_the_pages_figures():
+    from bit_quantized_shampoo_b200 import costmodel as C
+    g = _golden_costs()
+    got = {
+        "full_matrix_entries_1024x1024": C.full_matrix_entries(1024, 1024),
+        "full_matrix_bytes_fp32_1024x1024": 4 * C.full_matrix_entries(1024, 1024),
+        "full_matrix_root_flops_1024x1024": C.full_matrix_root_flops(1024, 1024),
+        "kron_floats_1024x1024": C.kronecker_floats(1024, 1024),
+        "kron_bytes_fp32_1024x1024": 4 * C.kronecker_floats(1024, 1024),
+        "kron_root_flops_1024x1024": C.kronecker_root_flops(1024, 1024),
+        "overhead_4096x4096_B1e6": C.overhead_ratio(4096, 4096, 1e6),
+        "overhead_2048x2048_B4096": C.overhead_ratio(2048, 2048, 4096),
+        "accumulator_floats_4096x11008": C.kronecker_floats(4096, 11008),
+        "adam_floats_4096x11008": C.adam_floats(4096, 11008),
+        "blocked_floats_per_param": C.kronecker_floats(1024, 1024) / (1024 * 1024),
+        "cached_roots_floats_per_param": 2 * C.kronecker_floats(512, 512) / (512 * 512),
+    }
+    assert set(got) == set(g)
+    for k, (v, tol) in g.items():
+        assert abs(got[k] - v) <= tol * abs(v) + 1e-12, (k, got[k], v)
+    # the per-step term is the sum of its four parts
+    assert C.step_flops(300, 70) == C.stats_flops(300, 70) + C.apply_flops(300, 70)
