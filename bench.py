@@ -1,0 +1,360 @@
+"""Throughput of the 4-bit Shampoo preconditioner step on B200.
+
+One step = update_stats + refresh_roots + precondition over every tile of the
+workload (default: the Llama-style layer set, 8 x 4096x11008 + 8 x 4096x4096
+cut into 480 tiles of at most 1024 x 1024, 960 factors), with the gradients
+already resident in HBM.  Prints one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 1..5] [--precision tf32|fp32]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own copy of
+the workload (tiles are independent; no data-path collective), so per-GPU
+work is fixed as N grows ("weak" scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "precond steps/sec & 1024² root refreshes/sec; quant HBM GB/s; TC util"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=5)
+    ap.add_argument("--precision", default="tf32", choices=["tf32", "fp32"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-codec", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.samples.append([p.strip() for p in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if len(s) > 5 + i and s[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ peaks
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0}, "fallback"
+
+
+# B200: 148 SMs; per SM and clock 128 fp32 FMA lanes and 64 fp64 FMA lanes.
+def alu_peak_tflops(kind: str, mhz: float) -> float:
+    lanes = 128 if kind == "fp32" else 64
+    return 148 * lanes * 2 * mhz * 1e6 / 1e12
+
+
+# Which unit bounds each stage in the current kernels.
+STAGE_BOUND = {
+    "stats_gemm": "alu_fp32", "bjorck_gram": "alu_fp32", "bjorck_update": "alu_fp32",
+    "subspace": "alu_fp32", "rayleigh_gemm": "alu_fp32", "roots": "alu_fp32",
+    "apply_left": "alu_fp32", "apply_right": "alu_fp32",
+    "qr_gram": "alu_fp64", "qr_syrk": "alu_fp64", "qr_solve_update": "alu_fp64",
+    "qr_potrf": "alu_fp64", "qr_trsm_panel": "alu_fp64", "qr_solve_panel": "alu_fp64",
+    "rayleigh": "alu_fp64",
+    "requant": "hbm", "precond_dequant": "hbm", "basis": "hbm", "stats_scan": "hbm",
+    "refresh_scan": "hbm", "qr_convert": "hbm", "precond_mu": "hbm",
+}
+
+
+def workload_shapes(wid):
+    from bit_quantized_shampoo_b200.workloads import WORKLOADS
+    return WORKLOADS[wid]
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+def cpu_sample(w, nblocks_sample: int, seed_step: int = 1):
+    """Time the oracle on a bounded sample of tiles; returns (seconds per tile,
+    tiles in the workload, description, threads)."""
+    from oracle import shampoo4_oracle as O
+    from bit_quantized_shampoo_b200.workloads import gradient
+    blocks = O.partition(w.shapes, w.max_block)
+    rng = np.random.default_rng(7)
+    pick = sorted(set([len(blocks) - 1] + list(rng.choice(len(blocks), size=min(nblocks_sample, len(blocks)),
+                                                            replace=False)[:max(0, nblocks_sample - 1)])))
+    grads = {}
+    t_total = 0.0
+    for k in pick:
+        b = blocks[k]
+        if b.param not in grads:
+            grads[b.param] = gradient(w, b.param, seed_step)
+        g = grads[b.param][b.r0:b.r0 + b.m, b.c0:b.c0 + b.n].copy()
+        fl = O.Factor(b.m, np.zeros((b.m, b.m), np.float32))
+        fr = O.Factor(b.n, np.zeros((b.n, b.n), np.float32))
+        for f, side in ((fl, "L"), (fr, "R")):        # untimed: a first basis
+            f.S = O.ema_stats(f.S, g, w.beta, side)
+            O.refresh_factor(f, w.eps, w.bjorck_iters)
+        t0 = time.perf_counter()
+        fl.S = O.ema_stats(fl.S, g, w.beta, "L")
+        fr.S = O.ema_stats(fr.S, g, w.beta, "R")
+        O.refresh_factor(fl, w.eps, w.bjorck_iters)
+        O.refresh_factor(fr, w.eps, w.bjorck_iters)
+        O.apply_roots(O.factor_root(fl, w.eps), g, O.factor_root(fr, w.eps))
+        t_total += time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    desc = (f"{len(pick)} of {len(blocks)} tiles (stats + warm refresh with Bjorck of both factors + "
+            f"precondition), per-tile time extrapolated to the whole workload")
+    return t_total / len(pick), len(blocks), desc, threads
+
+
+# ------------------------------------------------------------------ main
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = workload_shapes(args.workload)
+    per_tile = []
+    desc = threads = None
+    for i in range(args.warmup + args.steps):
+        t, nblocks, desc, threads = cpu_sample(w, 1, seed_step=1 + i)
+        if i >= args.warmup:
+            per_tile.append(t)
+    tile_s = float(np.mean(per_tile))
+    value = 1.0 / (tile_s * nblocks)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "tiles": nblocks},
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from bit_quantized_shampoo_b200 import api, _lib as L
+    from bit_quantized_shampoo_b200.workloads import gradient
+    import ctypes as C
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+
+    w = workload_shapes(args.workload)
+    shapes = list(w.shapes)
+    # inputs: seeded host draws, copied to pinned host memory and to HBM
+    host_g = [torch.from_numpy(gradient(w, i, 1)).pin_memory() for i in range(len(shapes))]
+    dev_g = [h.to(dev, non_blocking=False) for h in host_g]
+    dev_out = [torch.empty(s, dtype=torch.float32, device=dev) for s in shapes]
+    host_out = [torch.empty(s, dtype=torch.float32).pin_memory() for s in shapes]
+    sh = api.Shampoo4(shapes, beta=w.beta, eps=w.eps, max_block=w.max_block, bjorck_iters=w.bjorck_iters,
+                      precision=args.precision, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        sh.update_stats(dev_g)
+        sh.refresh_roots()
+        sh.precondition(dev_g, out=dev_out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    L.call("shampoo4_timing_enable", sh._h, 1)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * args.steps / (ms / 1e3)
+
+    # per-stage times measured live over the timed region
+    stages = {}
+    launches = 0
+    for s in range(22):
+        t_ms, n, fl, by = C.c_double(), C.c_int64(), C.c_double(), C.c_double()
+        L.call("shampoo4_timing_read", sh._h, s, C.byref(t_ms), C.byref(n), C.byref(fl), C.byref(by))
+        name = L.lib().shampoo4_stage_name(s).decode()
+        if n.value:
+            stages[name] = {"ms": t_ms.value / args.steps, "launches": n.value // args.steps,
+                            "flops": fl.value / args.steps, "bytes": by.value / args.steps}
+            launches += n.value
+    L.call("shampoo4_timing_enable", sh._h, 0)
+
+    pk, pk_src = peaks()
+    clocks = clk.summary()
+    dom = max(stages, key=lambda k: stages[k]["ms"])
+    ds = stages[dom]
+    bound = STAGE_BOUND.get(dom, "alu_fp32")
+    if bound == "hbm":
+        achieved = ds["bytes"] / (ds["ms"] / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s"}
+    else:
+        achieved = ds["flops"] / (ds["ms"] / 1e3) / 1e12
+        peak = alu_peak_tflops("fp32" if bound == "alu_fp32" else "fp64", pk.get("sm_max_mhz", 1965.0))
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = dom
+    roof["peak_source"] = pk_src if bound == "hbm" else "derived: 148 SMs x lanes x 2 x max SM clock"
+    roof["per_launch"] = {"launches_per_step": ds["launches"], "ms_per_launch": ds["ms"] / max(1, ds["launches"])}
+
+    line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": args.precision if args.precision == "fp32" else "tf32",
+            "data": "synthetic",
+            "config": {"workload": w.name, "tiles": sh.nblocks, "factors": sh.nfactors,
+                       "steps_per_refresh": 1, "l2": "inputs larger than L2 (2 GB of G, 4 GB of statistics)"},
+            "root_refreshes_per_s": value * sh.nfactors,
+            "gpu_launches": launches,
+            "clocks": clocks, "roofline": roof,
+            "stages_ms": {k: round(v["ms"], 4) for k, v in sorted(stages.items(), key=lambda kv: -kv[1]["ms"])}}
+
+    # end to end through the public API with host buffers
+    if not args.no_e2e:
+        torch.cuda.synchronize()
+        k = max(1, min(args.steps, 3))
+        e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2.record(stream)
+        for _ in range(k):
+            for h, d in zip(host_g, dev_g):
+                d.copy_(h, non_blocking=True)
+            step()
+            for d, h in zip(dev_out, host_out):
+                h.copy_(d, non_blocking=True)
+        e3.record(stream)
+        torch.cuda.synchronize()
+        ems = e2.elapsed_time(e3)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        bi = sum(h.numel() * 4 for h in host_g)
+        bo = sum(h.numel() * 4 for h in host_out)
+        line["e2e"] = {"value": world * k / (ems / 1e3), "unit": "steps/s", "h2d_bytes_per_step": bi,
+                       "d2h_bytes_per_step": bo}
+
+    # stand-alone codec bandwidth on eigenvector-shaped tensors of the workload's size
+    if not args.no_codec:
+        n_elem = sum(int(b[3]) ** 2 + int(b[4]) ** 2 for b in (sh.block_info(k) for k in range(sh.nblocks)))
+        g = torch.Generator(device=dev).manual_seed(3)
+        x = torch.randn(n_elem, device=dev, generator=g) * (1.0 / 32)
+        codes = torch.empty((n_elem + 1) // 2, dtype=torch.uint8, device=dev)
+        scales = torch.empty((n_elem + 63) // 64, dtype=torch.float32, device=dev)
+        y = torch.empty_like(x)
+        for _ in range(3):
+            api.quant4_pack([x], [codes], [scales])
+            api.quant4_unpack([codes], [scales], [n_elem], [y])
+        torch.cuda.synchronize()
+        reps = 5
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        for _ in range(reps):
+            api.quant4_pack([x], [codes], [scales])
+        ev[1].record(stream)
+        for _ in range(reps):
+            api.quant4_unpack([codes], [scales], [n_elem], [y])
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        bpe = 4.0 + 0.5 + 4.0 / 64
+        pack_gbs = bpe * n_elem * reps / (ev[0].elapsed_time(ev[1]) / 1e3) / 1e9
+        unpack_gbs = bpe * n_elem * reps / (ev[1].elapsed_time(ev[2]) / 1e3) / 1e9
+        line["codec"] = {"elements": n_elem, "pack_gbs": pack_gbs, "unpack_gbs": unpack_gbs,
+                         "pack_frac": pack_gbs / pk["hbm_gbs"], "unpack_frac": unpack_gbs / pk["hbm_gbs"],
+                         "peak_gbs": pk["hbm_gbs"], "peak_source": pk_src}
+        del x, y, codes, scales
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        tile_s, nb, desc, threads = cpu_sample(w, 4)
+        v = 1.0 / (tile_s * nb)
+        line["cpu_baseline"] = {"value": v, "unit": "steps/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,161 @@
+"""Thin PyTorch-facing wrapper of the shampoo4 C ABI.
+
+PyTorch provides the device memory (state, workspace, outputs) and the CUDA
+stream; every arithmetic step runs in libshampoo4.so.  Tensors must be CUDA
+float32 (gradients, outputs) or uint8 (codes).
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import torch
+
+from . import _lib as L
+
+
+def _stream(stream=None) -> C.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(t: torch.Tensor, dtype, name: str):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == dtype):
+        raise TypeError(f"{name} must be a CUDA {dtype} tensor")
+
+
+def _row_major_2d(t: torch.Tensor, name: str) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be 2-D with unit column stride")
+    return t.stride(0)
+
+
+class Shampoo4:
+    """One handle: a fixed list of 2-D parameter shapes and their state."""
+
+    def __init__(self, shapes, beta=0.95, eps=1e-6, max_block=1024, bjorck_iters=5,
+                 precision="tf32", device=None, reset=True):
+        self.shapes = [(int(r), int(c)) for r, c in shapes]
+        cfg = L.Config(beta, eps, max_block, 64, bjorck_iters,
+                       L.PREC_FP32 if precision == "fp32" else L.PREC_TF32)
+        params = (L.Param * len(self.shapes))(*[L.Param(r, c) for r, c in self.shapes])
+        h = C.c_void_p()
+        L.call("shampoo4_init", C.byref(cfg), params, len(self.shapes), C.byref(h))
+        self._h = h
+        self.config = cfg
+        st, ws = C.c_size_t(), C.c_size_t()
+        L.call("shampoo4_sizes", h, C.byref(st), C.byref(ws))
+        self.state_bytes, self.workspace_bytes = st.value, ws.value
+        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.state = torch.empty(max(self.state_bytes, 256), dtype=torch.uint8, device=self.device)
+        self.workspace = torch.empty(max(self.workspace_bytes, 256), dtype=torch.uint8, device=self.device)
+        nb, nf = C.c_int32(), C.c_int32()
+        L.call("shampoo4_counts", h, C.byref(nb), C.byref(nf))
+        self.nblocks, self.nfactors = nb.value, nf.value
+        self.bind(reset=reset)
+
+    def bind(self, reset=True, stream=None):
+        L.call("shampoo4_bind", self._h, C.c_void_p(self.state.data_ptr()),
+               C.c_void_p(self.workspace.data_ptr()), 1 if reset else 0, _stream(stream))
+
+    def set_has_basis(self, flag: bool):
+        L.call("shampoo4_set_has_basis", self._h, 1 if flag else 0)
+
+    def _ptrs(self, mats, name):
+        if len(mats) != len(self.shapes):
+            raise ValueError(f"expected {len(self.shapes)} {name}")
+        lds = []
+        for m, (r, c) in zip(mats, self.shapes):
+            _need_cuda(m, torch.float32, name)
+            if tuple(m.shape) != (r, c):
+                raise ValueError(f"{name}: shape {tuple(m.shape)} != {(r, c)}")
+            lds.append(_row_major_2d(m, name))
+        return L.ptr_array([m.data_ptr() for m in mats]), L.i64_array(lds)
+
+    def update_stats(self, grads, stream=None):
+        p, ld = self._ptrs(grads, "grads")
+        L.call("shampoo4_update_stats", self._h, p, ld, _stream(stream))
+
+    def refresh_roots(self, stream=None):
+        L.call("shampoo4_refresh_roots", self._h, _stream(stream))
+
+    def precondition(self, grads, out=None, stream=None):
+        if out is None:
+            out = [torch.empty(s, dtype=torch.float32, device=self.device) for s in self.shapes]
+        p, ld = self._ptrs(grads, "grads")
+        q, ldo = self._ptrs(out, "out")
+        L.call("shampoo4_precondition", self._h, p, ld, q, ldo, _stream(stream))
+        return out
+
+    def status_flags(self, stream=None) -> int:
+        f = C.c_uint32()
+        L.call("shampoo4_get_status_flags", self._h, C.byref(f), _stream(stream))
+        return f.value
+
+    def block_info(self, k):
+        p, m, n = C.c_int32(), C.c_int32(), C.c_int32()
+        r0, c0 = C.c_int64(), C.c_int64()
+        L.call("shampoo4_block_info", self._h, k, C.byref(p), C.byref(r0), C.byref(c0), C.byref(m), C.byref(n))
+        return p.value, r0.value, c0.value, m.value, n.value
+
+    def factor_views(self, f):
+        """(S, codes, scales, lambda) as tensor views into the state buffer."""
+        oS, oc, os_, ol = C.c_size_t(), C.c_size_t(), C.c_size_t(), C.c_size_t()
+        d = C.c_int32()
+        L.call("shampoo4_factor_layout", self._h, f, C.byref(oS), C.byref(oc), C.byref(os_), C.byref(ol), C.byref(d))
+        d = d.value
+        n = d * d
+        st = self.state
+        S = st[oS.value:oS.value + 4 * n].view(torch.float32).view(d, d)
+        codes = st[oc.value:oc.value + (n + 1) // 2]
+        scales = st[os_.value:os_.value + 4 * ((n + 63) // 64)].view(torch.float32)
+        lam = st[ol.value:ol.value + 4 * d].view(torch.float32)
+        return S, codes, scales, lam
+
+    def debug_q(self, f):
+        off = C.c_size_t()
+        L.call("shampoo4_debug_q_offset", self._h, f, C.byref(off))
+        d = self.factor_views(f)[0].shape[0]
+        return self.workspace[off.value:off.value + 4 * d * d].view(torch.float32).view(d, d)
+
+    def close(self):
+        if getattr(self, "_h", None):
+            L.lib().shampoo4_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def quant4_pack(xs, codes=None, scales=None, stream=None):
+    """Quantize a list of fp32 CUDA tensors (flattened)."""
+    xs = [x.contiguous() for x in xs]
+    ns = [x.numel() for x in xs]
+    for x in xs:
+        _need_cuda(x, torch.float32, "x")
+    if codes is None:
+        codes = [torch.empty((n + 1) // 2, dtype=torch.uint8, device=x.device) for x, n in zip(xs, ns)]
+    if scales is None:
+        scales = [torch.empty((n + 63) // 64, dtype=torch.float32, device=x.device) for x, n in zip(xs, ns)]
+    L.call("quant4_pack", L.ptr_array([x.data_ptr() for x in xs]), L.i64_array(ns), len(xs),
+           L.ptr_array([c.data_ptr() for c in codes]), L.ptr_array([s.data_ptr() for s in scales]),
+           _stream(stream))
+    return codes, scales
+
+
+def quant4_unpack(codes, scales, ns, out=None, stream=None):
+    if out is None:
+        out = [torch.empty(n, dtype=torch.float32, device=c.device) for c, n in zip(codes, ns)]
+    L.call("quant4_unpack", L.ptr_array([c.data_ptr() for c in codes]),
+           L.ptr_array([s.data_ptr() for s in scales]), L.i64_array(ns), len(codes),
+           L.ptr_array([o.data_ptr() for o in out]), _stream(stream))
+    return out
+
+
+def quant4_tables():
+    cb = (C.c_float * 16)()
+    th = (C.c_float * 15)()
+    L.call("quant4_tables", cb, th)
+    return list(cb), list(th)

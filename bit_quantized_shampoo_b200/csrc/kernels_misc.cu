@@ -1,0 +1,241 @@
+// Small batched kernels of the refresh and precondition programs: blocked
+// Cholesky panels and triangular solves (fp64), basis initialization,
+// Rayleigh quotients, root weights, non-finite scans and conversions.
+#include "quant4.cuh"
+#include "plan.h"
+
+namespace s4 {
+
+constexpr int kPanel = 64;     // Cholesky / triangular-solve panel width
+
+// ---- Cholesky of a jb x jb diagonal block, lower, in place ---------------
+__global__ void __launch_bounds__(256) k_potrf(const PotrfDesc* __restrict__ descs) {
+  const PotrfDesc& g = descs[blockIdx.x];
+  const int jb = g.jb;
+  if (jb <= 0) return;
+  __shared__ double L[kPanel][kPanel + 1];
+  __shared__ int bad;
+  for (int e = threadIdx.x; e < jb * jb; e += blockDim.x) {
+    int r = e / jb, c = e % jb;
+    L[r][c] = (c <= r) ? g.A[int64_t(r) * g.ld + c] : 0.0;
+  }
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  for (int c = 0; c < jb; ++c) {
+    if (threadIdx.x == 0) {
+      double p = L[c][c];
+      if (!(p > 0.0) || !isfinite(p)) { bad = 1; p = 1.0; }
+      L[c][c] = sqrt(p);
+    }
+    __syncthreads();
+    double piv = L[c][c];
+    for (int r = c + 1 + threadIdx.x; r < jb; r += blockDim.x) L[r][c] /= piv;
+    __syncthreads();
+    const int w = jb - c - 1;                 // trailing (w x w) lower triangle
+    for (int e = threadIdx.x; e < w * w; e += blockDim.x) {
+      int r = c + 1 + e / w, s = c + 1 + e % w;
+      if (s <= r) L[r][s] -= L[r][c] * L[s][c];
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < jb * jb; e += blockDim.x) {
+    int r = e / jb, c = e % jb;
+    if (c <= r) g.A[int64_t(r) * g.ld + c] = L[r][c];
+  }
+  if (threadIdx.x == 0 && bad) {
+    *g.fail = 1u;
+    atomicOr(g.gflags, SHAMPOO4_FLAG_REFRESH_FAILED);
+  }
+}
+
+shampoo4_status launch_potrf(const PotrfDesc* d_desc, int count, cudaStream_t st) {
+  if (count <= 0) return SHAMPOO4_OK;
+  k_potrf<<<count, 256, 0, st>>>(d_desc);
+  S4_CUDA(cudaGetLastError());
+  return SHAMPOO4_OK;
+}
+
+// ---- X[r, 0:jb] <- X[r, 0:jb] L^-T, one warp per row --------------------
+constexpr int kTrsmRowsPerCta = 64;
+__global__ void __launch_bounds__(256) k_trsm(const TrsmDesc* __restrict__ descs) {
+  const TrsmDesc& g = descs[blockIdx.y];
+  const int jb = g.jb;
+  const int row0 = blockIdx.x * kTrsmRowsPerCta;
+  if (jb <= 0 || row0 >= g.rows) return;
+  __shared__ double L[kPanel][kPanel + 1];
+  for (int e = threadIdx.x; e < jb * jb; e += blockDim.x) {
+    int r = e / jb, c = e % jb;
+    L[r][c] = (c <= r) ? g.L[int64_t(r) * g.ldl + c] : 0.0;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int row_end = min(g.rows, row0 + kTrsmRowsPerCta);
+  for (int r = row0 + warp; r < row_end; r += 8) {
+    double* x = g.X + int64_t(r) * g.ldx;
+    double x0 = lane < jb ? x[lane] : 0.0;
+    double x1 = lane + 32 < jb ? x[lane + 32] : 0.0;
+    for (int c = 0; c < jb; ++c) {
+      // x_c is final once columns < c are applied; divide by L[c][c]
+      double xc = __shfl_sync(0xffffffffu, c < 32 ? x0 : x1, c & 31);
+      xc /= L[c][c];
+      if (c < 32) { if (lane == c) x0 = xc; } else { if (lane + 32 == c) x1 = xc; }
+      if (lane > c && lane < jb) x0 -= xc * L[lane][c];
+      if (lane + 32 > c && lane + 32 < jb) x1 -= xc * L[lane + 32][c];
+    }
+    if (lane < jb) x[lane] = x0;
+    if (lane + 32 < jb) x[lane + 32] = x1;
+  }
+}
+
+shampoo4_status launch_trsm(const TrsmDesc* d_desc, int count, int max_rows, cudaStream_t st) {
+  if (count <= 0 || max_rows <= 0) return SHAMPOO4_OK;
+  for (int base = 0; base < count; base += 65535) {
+    int c = count - base < 65535 ? count - base : 65535;
+    dim3 grid((max_rows + kTrsmRowsPerCta - 1) / kTrsmRowsPerCta, c);
+    k_trsm<<<grid, 256, 0, st>>>(d_desc + base);
+    S4_CUDA(cudaGetLastError());
+  }
+  return SHAMPOO4_OK;
+}
+
+// ---- U = dequant(codes, scales) or I ------------------------------------
+__global__ void __launch_bounds__(256) k_basis(const BasisDesc* __restrict__ descs) {
+  const BasisDesc& g = descs[blockIdx.y];
+  __shared__ float level[16];
+  if (threadIdx.x < 16) level[threadIdx.x] = level_f32(threadIdx.x);
+  __syncthreads();
+  const int64_t n = int64_t(g.d) * g.d;
+  const int64_t e0 = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  if (e0 >= n) return;
+  float v[8];
+  if (g.identity) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      int64_t i = e0 + e;
+      v[e] = (i / g.d == i % g.d) ? 1.0f : 0.0f;
+    }
+  } else {
+    uint32_t packed = 0;
+    const int64_t nbytes = (n + 1) >> 1;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if ((e0 >> 1) + k < nbytes) packed |= uint32_t(g.codes[(e0 >> 1) + k]) << (8 * k);
+    dequantize8(packed, g.scales[e0 / kQuantBlock], level, v);
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    if (e0 + e < n) g.U[e0 + e] = v[e];
+}
+
+shampoo4_status launch_basis(const BasisDesc* d_desc, int count, int64_t max_elems, cudaStream_t st) {
+  if (count <= 0 || max_elems <= 0) return SHAMPOO4_OK;
+  int64_t ctas = (max_elems + 256 * 8 - 1) / (256 * 8);
+  for (int base = 0; base < count; base += 65535) {
+    int c = count - base < 65535 ? count - base : 65535;
+    k_basis<<<dim3(unsigned(ctas), c), 256, 0, st>>>(d_desc + base);
+    S4_CUDA(cudaGetLastError());
+  }
+  return SHAMPOO4_OK;
+}
+
+// ---- lambda_i = max(q_i . (S q)_i, 0) -----------------------------------
+__global__ void __launch_bounds__(256) k_rayleigh(const RayleighDesc* __restrict__ descs) {
+  const RayleighDesc& g = descs[blockIdx.y];
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= g.d) return;
+  if (g.skip && *g.skip) return;
+  double acc = 0.0;
+  for (int r = 0; r < g.d; ++r)
+    acc += double(g.Q[int64_t(r) * g.d + i]) * double(g.T[int64_t(r) * g.d + i]);
+  g.lam[i] = float(acc > 0.0 ? acc : 0.0);
+}
+
+shampoo4_status launch_rayleigh(const RayleighDesc* d_desc, int count, int max_d, cudaStream_t st) {
+  if (count <= 0 || max_d <= 0) return SHAMPOO4_OK;
+  for (int base = 0; base < count; base += 65535) {
+    int c = count - base < 65535 ? count - base : 65535;
+    k_rayleigh<<<dim3((max_d + 255) / 256, c), 256, 0, st>>>(d_desc + base);
+    S4_CUDA(cudaGetLastError());
+  }
+  return SHAMPOO4_OK;
+}
+
+// ---- mu_i = (lambda_i + eps)^(-1/4), evaluated in fp64 -------------------
+__global__ void __launch_bounds__(256) k_mu(const MuDesc* __restrict__ descs, float eps) {
+  const MuDesc& g = descs[blockIdx.y];
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= g.d) return;
+  double x = double(g.lam[i]) + double(eps);
+  g.mu[i] = float(1.0 / sqrt(sqrt(x)));
+}
+
+shampoo4_status launch_mu(const MuDesc* d_desc, int count, int max_d, float eps, cudaStream_t st) {
+  if (count <= 0 || max_d <= 0) return SHAMPOO4_OK;
+  for (int base = 0; base < count; base += 65535) {
+    int c = count - base < 65535 ? count - base : 65535;
+    k_mu<<<dim3((max_d + 255) / 256, c), 256, 0, st>>>(d_desc + base, eps);
+    S4_CUDA(cudaGetLastError());
+  }
+  return SHAMPOO4_OK;
+}
+
+// ---- non-finite scan -------------------------------------------------------
+__global__ void __launch_bounds__(256)
+k_scan(const ScanDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, int nparams,
+       uint32_t* __restrict__ gflags) {
+  const ScanDesc& g = descs[blockIdx.y];
+  const int64_t n = int64_t(g.rows) * g.cols;
+  int64_t ld = g.ld;
+  const float* X = g.X;
+  if (g.ref.tab >= 0) {
+    const PtrEntry& e = tabs[g.ref.tab * nparams + g.ref.param];
+    ld = e.ld;
+    X = e.ptr + g.ref.r0 * e.ld + g.ref.c0;
+  }
+  bool bad = false;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    int64_t r = e / g.cols, c = e % g.cols;
+    float v = X[r * ld + c];
+    bad |= !isfinite(v);
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) {
+    *g.flag = 1u;
+    atomicOr(gflags, g.bit);
+  }
+}
+
+shampoo4_status launch_scan(const ScanDesc* d_desc, int count, int64_t max_elems,
+                            const PtrEntry* tabs, int nparams, uint32_t* flags, cudaStream_t st) {
+  if (count <= 0 || max_elems <= 0) return SHAMPOO4_OK;
+  int64_t ctas = (max_elems + 256 * 8 - 1) / (256 * 8);
+  if (ctas > 1024) ctas = 1024;
+  for (int base = 0; base < count; base += 65535) {
+    int c = count - base < 65535 ? count - base : 65535;
+    k_scan<<<dim3(unsigned(ctas), c), 256, 0, st>>>(d_desc + base, tabs, nparams, flags);
+    S4_CUDA(cudaGetLastError());
+  }
+  return SHAMPOO4_OK;
+}
+
+// ---- fp64 -> fp32 ----------------------------------------------------------
+__global__ void __launch_bounds__(256) k_convert(const ConvertDesc* __restrict__ descs) {
+  const ConvertDesc& g = descs[blockIdx.y];
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < g.n;
+       e += int64_t(gridDim.x) * blockDim.x)
+    g.dst[e] = float(g.src[e]);
+}
+
+shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st) {
+  if (count <= 0 || max_elems <= 0) return SHAMPOO4_OK;
+  int64_t ctas = (max_elems + 1023) / 1024;
+  if (ctas > 1024) ctas = 1024;
+  for (int base = 0; base < count; base += 65535) {
+    int c = count - base < 65535 ? count - base : 65535;
+    k_convert<<<dim3(unsigned(ctas), c), 256, 0, st>>>(d_desc + base);
+    S4_CUDA(cudaGetLastError());
+  }
+  return SHAMPOO4_OK;
+}
+
+}  // namespace s4

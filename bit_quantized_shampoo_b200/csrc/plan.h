@@ -1,0 +1,149 @@
+// Device descriptors and launchers of the shampoo4 library.
+//
+// The host planner turns a handle's tile partition into a fixed list of
+// launches per API call (a "program"); every launch processes a whole batch
+// of problems -- one per tile or per factor -- described by an array of
+// descriptors that lives in the workspace.  The descriptors are written once
+// at bind time; only the per-call gradient and output addresses change, and
+// those sit in two small pointer tables that descriptors refer to by index.
+#pragma once
+#include "common.cuh"
+
+namespace s4 {
+
+// A per-call operand: either an absolute address (tab < 0) or parameter
+// `param` of pointer table `tab` (0 = gradients, 1 = outputs), offset by
+// (r0, c0) with that table's leading dimension.
+struct PtrEntry {
+  const float* ptr;
+  int64_t ld;
+};
+
+struct OperandRef {
+  int32_t tab;
+  int32_t param;
+  int64_t r0, c0;
+};
+
+// ---- fp32-output batched GEMM --------------------------------------------
+// C = alpha * op(A) op(B) + beta * Cin, op(X) = X or X^T (row-major storage).
+// kscale (optional) multiplies op(A)[i,k] by kscale[k]; skip (optional)
+// suppresses the whole problem when *skip != 0.  mode selects arithmetic.
+enum GemmMode : int32_t { kModeTF32 = 0, kModeFP32 = 1 };
+
+struct GemmF32Desc {
+  int32_t M, N, K;
+  int32_t ta, tb;
+  int32_t mode;
+  int32_t symmetric;          // output known symmetric: only tiles on or below
+                              // the diagonal are computed, then mirrored
+  int32_t pad_;
+  float alpha, beta;
+  const float* A; int64_t lda;
+  const float* B; int64_t ldb;
+  float* C; int64_t ldc;
+  const float* Cin; int64_t ldcin;
+  const float* kscale;
+  const uint32_t* skip;
+  OperandRef a_ref, b_ref, c_ref;
+};
+
+// ---- fp64-accumulating batched GEMM (QR of the subspace step) --------------
+struct GemmF64Desc {
+  int32_t M, N, K;
+  int32_t ta, tb;
+  int32_t lower_only;         // skip tiles strictly above the diagonal
+  int32_t a_f64, b_f64, c_f64, cin_f64;
+  double alpha, beta;
+  const void* A; int64_t lda;
+  const void* B; int64_t ldb;
+  void* C; int64_t ldc;
+  const void* Cin; int64_t ldcin;
+  const uint32_t* skip;
+};
+
+// Cholesky of one jb x jb diagonal block (lower, in place).
+struct PotrfDesc {
+  double* A; int64_t ld;
+  int32_t jb; int32_t pad_;
+  uint32_t* fail;             // set to 1 on a non-positive or non-finite pivot
+  uint32_t* gflags;           // ... and SHAMPOO4_FLAG_REFRESH_FAILED ORed here
+};
+
+// X[r, 0:jb] <- X[r, 0:jb] * L^-T for r < rows, L the jb x jb lower block.
+struct TrsmDesc {
+  const double* L; int64_t ldl;
+  double* X; int64_t ldx;
+  int32_t jb, rows;
+};
+
+// Initial basis of a refresh: U = dequant(codes, scales) or the identity.
+struct BasisDesc {
+  const uint8_t* codes;
+  const float* scales;
+  float* U;
+  int32_t d;
+  int32_t identity;
+};
+
+// lambda_i = max(sum_r Q[r,i] T[r,i], 0), T = S Q; written only if *skip==0.
+struct RayleighDesc {
+  const float* Q;
+  const float* T;
+  float* lam;
+  int32_t d; int32_t pad_;
+  const uint32_t* skip;
+};
+
+// mu_i = (lambda_i + eps)^(-1/4)
+struct MuDesc {
+  const float* lam;
+  float* mu;
+  int32_t d; int32_t pad_;
+};
+
+// Scan a matrix (absolute or per-call) for NaN/Inf; on one, set *flag = 1
+// and OR `bit` into the global flag word.
+struct ScanDesc {
+  const float* X; int64_t ld;
+  int32_t rows, cols;
+  OperandRef ref;
+  uint32_t* flag;
+  uint32_t bit; int32_t pad_;
+};
+
+struct ConvertDesc {
+  const double* src;
+  float* dst;
+  int64_t n;
+};
+
+struct ClearDesc {
+  uint32_t* p;
+  int64_t n;
+};
+
+// ---- launchers (each enqueues one launch over `count` descriptors) -------
+shampoo4_status launch_gemm_f32(const GemmF32Desc* d_desc, int count, int max_tiles,
+                                const PtrEntry* tabs, int nparams, cudaStream_t st);
+shampoo4_status launch_gemm_f64(const GemmF64Desc* d_desc, int count, int max_tiles,
+                                cudaStream_t st);
+shampoo4_status launch_potrf(const PotrfDesc* d_desc, int count, cudaStream_t st);
+shampoo4_status launch_trsm(const TrsmDesc* d_desc, int count, int max_rows, cudaStream_t st);
+shampoo4_status launch_basis(const BasisDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
+shampoo4_status launch_rayleigh(const RayleighDesc* d_desc, int count, int max_d, cudaStream_t st);
+shampoo4_status launch_mu(const MuDesc* d_desc, int count, int max_d, float eps, cudaStream_t st);
+shampoo4_status launch_scan(const ScanDesc* d_desc, int count, int64_t max_elems,
+                            const PtrEntry* tabs, int nparams, uint32_t* flags, cudaStream_t st);
+shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
+shampoo4_status launch_clear(const ClearDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
+
+// Codec launchers (quant4.cu).  `skip` (optional, per tensor) suppresses a
+// tensor when *skip[i] != 0.
+shampoo4_status launch_pack(const float* const* x, const int64_t* n, int32_t count,
+                            uint8_t* const* codes, float* const* scales, cudaStream_t st,
+                            const uint32_t* const* skip = nullptr);
+shampoo4_status launch_unpack(const uint8_t* const* codes, const float* const* scales,
+                              const int64_t* n, int32_t count, float* const* x, cudaStream_t st);
+
+}  // namespace s4

@@ -1,0 +1,245 @@
+// Stand-alone 4-bit codec: quant4_pack / quant4_unpack over batches of fp32
+// tensors ("4-bit Shampoo for Memory-Efficient Network Training", abstract:
+// block-wise linear square quantization).
+//
+// Memory-bound.  One CTA of 256 threads covers 4096 consecutive elements of
+// one tensor (64 quantization blocks); each thread owns two groups of 8
+// elements (two 32-byte loads in flight), 8 consecutive lanes own one block.
+#include "quant4.cuh"
+#include "plan.h"
+
+namespace s4 {
+
+constexpr int kCodecThreads = 256;
+constexpr int kCodecGroupsPerThread = 2;
+constexpr int kCodecEltsPerCta = kCodecThreads * 8 * kCodecGroupsPerThread;   // 4096
+constexpr int kCodecMaxBatch = 64;
+
+struct PackTensor {
+  const float* x;
+  uint8_t* codes;
+  float* scales;
+  int64_t n;
+  int64_t cta_begin;
+  const uint32_t* skip;   // optional: tensor left untouched when *skip != 0
+  int32_t vec_x;          // x is 16-byte aligned: 128-bit loads
+  int32_t vec_codes;      // codes is 4-byte aligned: 32-bit stores
+};
+struct PackBatch {
+  int32_t count;
+  PackTensor t[kCodecMaxBatch];
+};
+
+struct UnpackTensor {
+  const uint8_t* codes;
+  const float* scales;
+  float* x;
+  int64_t n;
+  int64_t cta_begin;
+  int32_t vec_x;
+  int32_t vec_codes;
+};
+struct UnpackBatch {
+  int32_t count;
+  UnpackTensor t[kCodecMaxBatch];
+};
+
+template <class B>
+__device__ __forceinline__ int find_tensor(const B& b, int64_t cta) {
+  int lo = 0, hi = b.count - 1;
+  while (lo < hi) {                    // last tensor with cta_begin <= cta
+    int mid = (lo + hi + 1) >> 1;
+    if (b.t[mid].cta_begin <= cta) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Quantize the 8 elements starting at element e0 of tensor t (all lanes of
+// the warp call this together; lanes past the end contribute zeros).
+__device__ __forceinline__ void pack_group(const PackTensor& t, int64_t e0, const float* thr) {
+  float v[8];
+  uint32_t valid = 0;
+  if (t.vec_x && e0 + 8 <= t.n) {
+    const float4* p = reinterpret_cast<const float4*>(t.x + e0);
+    float4 a = __ldg(p), b = __ldg(p + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    valid = 0xffu;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      bool ok = e0 + e < t.n;
+      v[e] = ok ? __ldg(t.x + e0 + e) : 0.0f;
+      valid |= ok ? (1u << e) : 0u;
+    }
+  }
+  float s;
+  uint32_t packed = quantize8(v, valid, thr, &s);
+  if ((threadIdx.x & 7) == 0 && e0 < t.n) t.scales[e0 / kQuantBlock] = s;
+  if (valid == 0) return;
+  int64_t byte0 = e0 >> 1;
+  if (t.vec_codes && valid == 0xffu) {
+    *reinterpret_cast<uint32_t*>(t.codes + byte0) = packed;
+  } else {
+    int64_t nbytes = (t.n + 1) >> 1;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (byte0 + k < nbytes) t.codes[byte0 + k] = uint8_t(packed >> (8 * k));
+  }
+}
+
+__global__ void __launch_bounds__(kCodecThreads)
+k_quant4_pack(const __grid_constant__ PackBatch b) {
+  __shared__ CodecSmem sm;
+  codec_smem_init(sm);
+  __syncthreads();
+  const PackTensor& t = b.t[find_tensor(b, blockIdx.x)];
+  if (t.skip && *t.skip) return;
+  int64_t e_base = (int64_t(blockIdx.x) - t.cta_begin) * kCodecEltsPerCta;
+#pragma unroll
+  for (int g = 0; g < kCodecGroupsPerThread; ++g) {
+    int64_t e0 = e_base + (int64_t(g) * kCodecThreads + threadIdx.x) * 8;
+    pack_group(t, e0, sm.thr);
+  }
+}
+
+__device__ __forceinline__ void unpack_group(const UnpackTensor& t, int64_t e0, const float* level) {
+  if (e0 >= t.n) return;
+  float s = __ldg(t.scales + e0 / kQuantBlock);
+  int64_t byte0 = e0 >> 1;
+  uint32_t packed;
+  bool full = e0 + 8 <= t.n;
+  if (t.vec_codes && full) {
+    packed = __ldg(reinterpret_cast<const uint32_t*>(t.codes + byte0));
+  } else {
+    packed = 0;
+    int64_t nbytes = (t.n + 1) >> 1;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (byte0 + k < nbytes) packed |= uint32_t(__ldg(t.codes + byte0 + k)) << (8 * k);
+  }
+  float v[8];
+  dequantize8(packed, s, level, v);
+  if (t.vec_x && full) {
+    float4* p = reinterpret_cast<float4*>(t.x + e0);
+    p[0] = make_float4(v[0], v[1], v[2], v[3]);
+    p[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (e0 + e < t.n) t.x[e0 + e] = v[e];
+  }
+}
+
+__global__ void __launch_bounds__(kCodecThreads)
+k_quant4_unpack(const __grid_constant__ UnpackBatch b) {
+  __shared__ CodecSmem sm;
+  codec_smem_init(sm);
+  __syncthreads();
+  const UnpackTensor& t = b.t[find_tensor(b, blockIdx.x)];
+  int64_t e_base = (int64_t(blockIdx.x) - t.cta_begin) * kCodecEltsPerCta;
+#pragma unroll
+  for (int g = 0; g < kCodecGroupsPerThread; ++g) {
+    int64_t e0 = e_base + (int64_t(g) * kCodecThreads + threadIdx.x) * 8;
+    unpack_group(t, e0, sm.level);
+  }
+}
+
+// Host launchers, shared with the optimizer's own requantization.
+shampoo4_status launch_pack(const float* const* x, const int64_t* n, int32_t count,
+                            uint8_t* const* codes, float* const* scales, cudaStream_t st,
+                            const uint32_t* const* skip) {
+  for (int32_t base = 0; base < count; base += kCodecMaxBatch) {
+    PackBatch b;
+    b.count = 0;
+    int64_t ctas = 0;
+    for (int32_t i = base; i < count && i < base + kCodecMaxBatch; ++i) {
+      if (n[i] == 0) continue;
+      PackTensor& t = b.t[b.count++];
+      t.x = x[i]; t.codes = codes[i]; t.scales = scales[i]; t.n = n[i];
+      t.cta_begin = ctas;
+      t.skip = skip ? skip[i] : nullptr;
+      t.vec_x = aligned(x[i], 16);
+      t.vec_codes = aligned(codes[i], 4);
+      ctas += (n[i] + kCodecEltsPerCta - 1) / kCodecEltsPerCta;
+    }
+    if (b.count == 0) continue;
+    if (ctas > 0x7fffffffLL) return SHAMPOO4_ERR_INVALID_ARG;
+    k_quant4_pack<<<unsigned(ctas), kCodecThreads, 0, st>>>(b);
+    S4_CUDA(cudaGetLastError());
+  }
+  return SHAMPOO4_OK;
+}
+
+shampoo4_status launch_unpack(const uint8_t* const* codes, const float* const* scales,
+                              const int64_t* n, int32_t count, float* const* x, cudaStream_t st) {
+  for (int32_t base = 0; base < count; base += kCodecMaxBatch) {
+    UnpackBatch b;
+    b.count = 0;
+    int64_t ctas = 0;
+    for (int32_t i = base; i < count && i < base + kCodecMaxBatch; ++i) {
+      if (n[i] == 0) continue;
+      UnpackTensor& t = b.t[b.count++];
+      t.codes = codes[i]; t.scales = scales[i]; t.x = x[i]; t.n = n[i];
+      t.cta_begin = ctas;
+      t.vec_x = aligned(x[i], 16);
+      t.vec_codes = aligned(codes[i], 4);
+      ctas += (n[i] + kCodecEltsPerCta - 1) / kCodecEltsPerCta;
+    }
+    if (b.count == 0) continue;
+    if (ctas > 0x7fffffffLL) return SHAMPOO4_ERR_INVALID_ARG;
+    k_quant4_unpack<<<unsigned(ctas), kCodecThreads, 0, st>>>(b);
+    S4_CUDA(cudaGetLastError());
+  }
+  return SHAMPOO4_OK;
+}
+
+}  // namespace s4
+
+// ------------------------------------------------------------------ C ABI
+
+static shampoo4_status check_codec_args(const void* const* a, const void* const* b,
+                                        const void* const* c, const int64_t* n, int32_t count) {
+  if (count < 0) return SHAMPOO4_ERR_INVALID_ARG;
+  if (count == 0) return SHAMPOO4_OK;
+  if (!a || !b || !c || !n) return SHAMPOO4_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < count; ++i) {
+    if (n[i] < 0) return SHAMPOO4_ERR_INVALID_ARG;
+    if (n[i] == 0) continue;
+    if (!a[i] || !b[i] || !c[i]) return SHAMPOO4_ERR_INVALID_ARG;
+  }
+  return SHAMPOO4_OK;
+}
+
+extern "C" shampoo4_status quant4_pack(const float* const* d_x, const int64_t* n, int32_t count,
+                                       uint8_t* const* d_codes, float* const* d_scales,
+                                       shampoo4_stream_t stream) {
+  S4_TRY(check_codec_args(reinterpret_cast<const void* const*>(d_x),
+                          reinterpret_cast<const void* const*>(d_codes),
+                          reinterpret_cast<const void* const*>(d_scales), n, count));
+  for (int32_t i = 0; i < count; ++i)
+    if (n[i] > 0 && (!s4::aligned(d_x[i], 4) || !s4::aligned(d_scales[i], 4)))
+      return SHAMPOO4_ERR_INVALID_ARG;
+  if (count == 0) return SHAMPOO4_OK;
+  return s4::launch_pack(d_x, n, count, d_codes, d_scales, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" shampoo4_status quant4_unpack(const uint8_t* const* d_codes, const float* const* d_scales,
+                                         const int64_t* n, int32_t count, float* const* d_x,
+                                         shampoo4_stream_t stream) {
+  S4_TRY(check_codec_args(reinterpret_cast<const void* const*>(d_codes),
+                          reinterpret_cast<const void* const*>(d_scales),
+                          reinterpret_cast<const void* const*>(d_x), n, count));
+  for (int32_t i = 0; i < count; ++i)
+    if (n[i] > 0 && (!s4::aligned(d_x[i], 4) || !s4::aligned(d_scales[i], 4)))
+      return SHAMPOO4_ERR_INVALID_ARG;
+  if (count == 0) return SHAMPOO4_OK;
+  return s4::launch_unpack(d_codes, d_scales, n, count, d_x, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" shampoo4_status quant4_tables(float codebook[16], float thresholds[15]) {
+  if (!codebook || !thresholds) return SHAMPOO4_ERR_INVALID_ARG;
+  for (int j = 0; j < 16; ++j) codebook[j] = s4::level_f32(j);
+  for (int k = 0; k < 15; ++k) thresholds[k] = s4::threshold_f32(k);
+  return SHAMPOO4_OK;
+}

@@ -1,0 +1,102 @@
+// Device-side pieces of the block-wise linear square 4-bit codec
+// ("4-bit Shampoo for Memory-Efficient Network Training", abstract: linear
+// square quantization, block-wise, of the eigenvector matrix).
+//
+// Layout: a block is 64 consecutive elements; 8 consecutive lanes of a warp
+// own one block, 8 elements each, so the block's absmax is a 3-step
+// xor-shuffle inside each 8-lane segment.
+#pragma once
+#include "common.cuh"
+
+namespace s4 {
+
+// Thresholds t_0..t_14 in shared memory (indexed by a per-lane position).
+struct CodecSmem {
+  float thr[16];
+  float level[16];
+};
+
+__device__ __forceinline__ void codec_smem_init(CodecSmem& sm) {
+  if (threadIdx.x < 16) {
+    int j = threadIdx.x;
+    sm.level[j] = level_f32(j);
+    sm.thr[j] = j < 15 ? threshold_f32(j) : __int_as_float(0x7f800000);
+  }
+}
+
+// code = number of thresholds strictly below v (t sorted ascending), by a
+// 4-step binary search.  NaN compares false everywhere and gives 0.
+__device__ __forceinline__ uint32_t code_of(float v, const float* thr) {
+  uint32_t c = (v > thr[7]) ? 8u : 0u;
+  c += (v > thr[c + 3]) ? 4u : 0u;
+  c += (v > thr[c + 1]) ? 2u : 0u;
+  c += (v > thr[c]) ? 1u : 0u;
+  return c;
+}
+
+// IEEE round-to-nearest x / s for a block that shares one divisor s.
+// Markstein's correction (P. Markstein, "Computation of elementary functions
+// on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990):
+// with r = RN(1/s) and q0 = RN(x r) within an ulp of x/s, the residual
+// e = x - s q0 is exact under an FMA and RN(q0 + e r) is the correctly
+// rounded quotient, provided nothing underflows.  Callers pass a normal,
+// finite s; operands or quotients below 2^-100 (where the residual could
+// underflow) take the plain IEEE division instead.
+__device__ __forceinline__ float div_rn_shared(float x, float s, float r) {
+  float q0 = x * r;
+  if (fabsf(x) < 0x1p-100f || fabsf(q0) < 0x1p-100f) return __fdiv_rn(x, s);
+  float e = fmaf(-q0, s, x);
+  return fmaf(e, r, q0);
+}
+
+// Quantize 8 values owned by this lane; the 8 lanes of the block are the
+// aligned 8-lane segment of the warp that contains this lane.  All 32 lanes
+// of the warp must call it together.  Returns the 8 codes packed as 4 bytes
+// (element 0 in the low nibble of byte 0) and the block scale in *scale.
+// Lanes whose elements lie past the end pass zeros and a valid mask of 0
+// for those elements; their codes are forced to 0.
+__device__ __forceinline__ uint32_t quantize8(const float (&v)[8], uint32_t valid_mask,
+                                              const float* thr, float* scale) {
+  float m = 0.0f;
+  uint32_t has_nan = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    float a = fabsf(v[e]);
+    has_nan |= (a != a) ? 1u : 0u;
+    m = fmaxf(m, a);                 // fmaxf ignores NaN; tracked separately
+  }
+#pragma unroll
+  for (int off = 4; off >= 1; off >>= 1) {
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    has_nan |= __shfl_xor_sync(0xffffffffu, has_nan, off);
+  }
+  float s = has_nan ? __int_as_float(0x7fc00000) : m;
+  *scale = s;
+  uint32_t packed = 0;
+  if (s == 0.0f) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      packed |= ((valid_mask >> e) & 1u ? 7u : 0u) << (4 * e);
+    return packed;
+  }
+  // s normal and finite: shared-reciprocal division; otherwise (NaN, Inf,
+  // subnormal) the plain IEEE division.
+  bool fast = (s >= 1.17549435e-38f) && (s <= 3.0e38f);
+  float r = fast ? __frcp_rn(s) : 0.0f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    float q = fast ? div_rn_shared(v[e], s, r) : __fdiv_rn(v[e], s);
+    uint32_t c = code_of(q, thr);
+    c = ((valid_mask >> e) & 1u) ? c : 0u;
+    packed |= c << (4 * e);
+  }
+  return packed;
+}
+
+__device__ __forceinline__ void dequantize8(uint32_t packed, float s, const float* level,
+                                            float (&out)[8]) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) out[e] = level[(packed >> (4 * e)) & 0xFu] * s;
+}
+
+}  // namespace s4

@@ -1,0 +1,221 @@
+/*
+ * shampoo4.h -- C ABI of the B200 4-bit Shampoo preconditioner library.
+ *
+ * The library runs the per-layer preconditioner step of 4-bit Shampoo
+ * ("4-bit Shampoo for Memory-Efficient Network Training", Wang, Zhou, Li,
+ * Huang -- abstract) on one GPU:
+ *
+ *   update_stats    L <- beta L + (1-beta) G G^T,  R <- beta R + (1-beta) G^T G
+ *                   ("Shampoo -- Second-Order Optimizer", sections "Kronecker
+ *                   factorization" and "Pitfalls": EMA with decay beta)
+ *   refresh_roots   per factor: dequantize the 4-bit eigenvector matrix U,
+ *                   Bjorck-rectify it (U <- 1.5 U - 0.5 U U^T U, t times),
+ *                   one subspace-iteration step Y = (S + eps I) U, Y = QR,
+ *                   Rayleigh eigenvalues lambda_i = max(q_i^T S q_i, 0), and
+ *                   requantize Q to 4-bit codes with per-64 scales
+ *   precondition    P = U diag((lambda + eps)^(-1/4)) U^T per factor
+ *                   ("Computing the inverse fourth root") and
+ *                   D = P_L G P_R per block ("Kronecker factorization")
+ *
+ * Weights are cut into tiles of at most max_block x max_block, each with its
+ * own pair of factors ("Blocked and distributed variants").
+ *
+ * Conventions shared by every entry point
+ *  - All device buffers are allocated and owned by the caller; the library
+ *    never allocates device memory.  It owns only host-side planning data
+ *    (and one small pinned host staging buffer per handle).
+ *  - Calls that take a stream are asynchronous on it; none synchronizes
+ *    except shampoo4_get_status_flags.  All calls on one handle must be
+ *    ordered on the same stream (or by the caller's own events).
+ *  - Matrices are fp32, row-major, with a leading dimension in elements.
+ *  - Argument errors are returned synchronously before anything is enqueued.
+ *    Errors found on the device (non-finite input, a failed factorization)
+ *    are latched in a flag word inside the workspace and read back with
+ *    shampoo4_get_status_flags.
+ *  - Arrays of device pointers ("d_grads", "d_x", ...) are HOST arrays whose
+ *    elements are device addresses.
+ *  - A handle is not thread-safe; distinct handles are independent.
+ */
+#ifndef SHAMPOO4_H
+#define SHAMPOO4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st* shampoo4_stream_t;
+
+typedef enum {
+  SHAMPOO4_OK = 0,
+  SHAMPOO4_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or config  */
+  SHAMPOO4_ERR_CUDA = 2,         /* a CUDA launch or copy failed            */
+  SHAMPOO4_ERR_NOT_READY = 3,    /* precondition before the first refresh,
+                                    or a compute call before shampoo4_bind  */
+  SHAMPOO4_ERR_NONFINITE = 4,    /* reported through the status flags       */
+  SHAMPOO4_ERR_WORKSPACE = 5,    /* workspace smaller than shampoo4_sizes   */
+  SHAMPOO4_ERR_UNSUPPORTED = 6,  /* no device of compute capability 10.x    */
+  SHAMPOO4_ERR_TIMEOUT = 7       /* reserved for bounded device waits       */
+} shampoo4_status;
+
+/* Arithmetic of the dense products.
+ *  TF32: operands rounded to TF32 (round to nearest), fp32 accumulation.
+ *  FP32: fp32-accurate products.
+ * The subspace product (S + eps I) U and the Rayleigh product S Q are always
+ * fp32-accurate: they must resolve eigenvalues near eps, far below TF32's
+ * resolution of the largest one.  The QR of the subspace step always runs
+ * its Gram matrix, Cholesky factor and triangular solve in fp64. */
+typedef enum { SHAMPOO4_PREC_TF32 = 0, SHAMPOO4_PREC_FP32 = 1 } shampoo4_precision;
+
+typedef struct {
+  float beta;            /* EMA decay of the statistics, 0 <= beta < 1     */
+  float eps;             /* added to eigenvalues in the root, and the shift
+                            of the subspace step (S + eps I) U; > 0        */
+  int32_t max_block;     /* tile edge b; 1 <= b <= 1024                    */
+  int32_t quant_block;   /* elements per quantization scale; must be 64    */
+  int32_t bjorck_iters;  /* Bjorck rectification steps per refresh, 0..16  */
+  int32_t precision;     /* shampoo4_precision                             */
+} shampoo4_config;
+
+typedef struct { int64_t rows, cols; } shampoo4_param;   /* 2-D weights only;
+                            reshape convolutions to out x (in*kh*kw)        */
+
+typedef struct shampoo4_ctx* shampoo4_handle;
+
+/* Status flag bits (shampoo4_get_status_flags). */
+#define SHAMPOO4_FLAG_NONFINITE_GRAD   0x1u  /* update_stats saw NaN/Inf in G;
+                                               S was left unchanged         */
+#define SHAMPOO4_FLAG_REFRESH_FAILED   0x2u  /* a factor's QR broke down; its
+                                               previous codes and lambda were
+                                               kept (stale-root fallback)   */
+#define SHAMPOO4_FLAG_NONFINITE_STATE  0x4u  /* a statistic held NaN/Inf at
+                                               refresh; that factor kept its
+                                               previous basis               */
+
+/* Plan a set of parameters.  Host only: validates the config and shapes,
+ * partitions every weight into greedy tiles of at most max_block (ragged
+ * last tile), and lays out state and workspace.  *out receives a handle that
+ * must be released with shampoo4_destroy.  Touches no device; shampoo4_bind
+ * needs a device of compute capability 10.x (ERR_UNSUPPORTED otherwise). */
+shampoo4_status shampoo4_init(const shampoo4_config* cfg, const shampoo4_param* params,
+                              int32_t nparams, shampoo4_handle* out);
+
+/* Bytes of device memory the caller must provide: the persistent optimizer
+ * state (kept between steps, checkpointable) and the scratch workspace
+ * (contents need not persist between calls, but the same buffer must be
+ * passed to bind and used for the handle's lifetime). */
+shampoo4_status shampoo4_sizes(shampoo4_handle h, size_t* state_bytes, size_t* workspace_bytes);
+
+/* Attach caller-owned device buffers (256-byte aligned).  reset != 0 zeroes
+ * the statistics and marks every factor as having no basis yet (the first
+ * refresh then starts from U = I); reset == 0 adopts the buffer contents as
+ * they are (resume from a checkpoint; the caller states with has_basis
+ * whether it already holds a basis, see shampoo4_set_has_basis). */
+shampoo4_status shampoo4_bind(shampoo4_handle h, void* d_state, void* d_workspace,
+                              int32_t reset, shampoo4_stream_t stream);
+
+/* Declare whether the bound state already holds eigenvector codes (after a
+ * resume from a checkpoint taken after a refresh). */
+shampoo4_status shampoo4_set_has_basis(shampoo4_handle h, int32_t has_basis);
+
+/* S_L <- beta S_L + (1-beta) G_b G_b^T and S_R <- beta S_R + (1-beta) G_b^T G_b
+ * for every tile G_b of every parameter.  d_grads[p] is the device address of
+ * parameter p's gradient (rows x cols, row-major, leading dimension ld[p] >=
+ * cols, 4-byte aligned).  A non-finite value anywhere in a tile leaves that
+ * tile's two statistics unchanged and sets SHAMPOO4_FLAG_NONFINITE_GRAD. */
+shampoo4_status shampoo4_update_stats(shampoo4_handle h, const float* const* d_grads,
+                                      const int64_t* ld, shampoo4_stream_t stream);
+
+/* Recompute every factor's 4-bit eigenvector codes, scales and eigenvalues
+ * from its statistic (dequantize, Bjorck, subspace step, QR, Rayleigh,
+ * requantize).  The first refresh after a reset starts from U = I. */
+shampoo4_status shampoo4_refresh_roots(shampoo4_handle h, shampoo4_stream_t stream);
+
+/* D = P_L G_b P_R for every tile, written into d_out[p] (same shape as the
+ * gradient, leading dimension ld_out[p] >= cols).  d_out must not overlap
+ * d_grads.  Returns ERR_NOT_READY before the first refresh. */
+shampoo4_status shampoo4_precondition(shampoo4_handle h, const float* const* d_grads,
+                                      const int64_t* ld, float* const* d_out,
+                                      const int64_t* ld_out, shampoo4_stream_t stream);
+
+/* Synchronize the stream, return the latched flag bits and clear them. */
+shampoo4_status shampoo4_get_status_flags(shampoo4_handle h, uint32_t* flags,
+                                          shampoo4_stream_t stream);
+
+/* Counts of the plan. */
+shampoo4_status shampoo4_counts(shampoo4_handle h, int32_t* nblocks, int32_t* nfactors);
+
+/* Tile k of the plan: parameter index, first row and column, size m x n.
+ * Tile k owns factor 2k (L, dimension m) and factor 2k+1 (R, dimension n). */
+shampoo4_status shampoo4_block_info(shampoo4_handle h, int32_t block, int32_t* param,
+                                    int64_t* r0, int64_t* c0, int32_t* m, int32_t* n);
+
+/* Byte offsets inside the state buffer of one factor's statistic S (fp32
+ * d x d, row-major, dense), codes (uint8, ceil(d*d/2), two per byte, element
+ * 2i in the low nibble), scales (fp32, ceil(d*d/64)) and eigenvalues (fp32,
+ * d); *dim receives d.  Any pointer may be NULL. */
+shampoo4_status shampoo4_factor_layout(shampoo4_handle h, int32_t factor, size_t* off_S,
+                                       size_t* off_codes, size_t* off_scales,
+                                       size_t* off_lambda, int32_t* dim);
+
+/* Byte offset inside the workspace of the fp32 d x d orthonormal Q that the
+ * last refresh quantized for this factor (valid until the next call that uses
+ * the workspace).  For tests and diagnostics. */
+shampoo4_status shampoo4_debug_q_offset(shampoo4_handle h, int32_t factor, size_t* off_q);
+
+/* Stages of the three programs, for the optional launch timing below. */
+typedef enum {
+  SHAMPOO4_STAGE_STATS_SCAN = 0, SHAMPOO4_STAGE_STATS_GEMM, SHAMPOO4_STAGE_REFRESH_SCAN,
+  SHAMPOO4_STAGE_BASIS, SHAMPOO4_STAGE_BJORCK_GRAM, SHAMPOO4_STAGE_BJORCK_UPDATE,
+  SHAMPOO4_STAGE_SUBSPACE, SHAMPOO4_STAGE_QR_GRAM, SHAMPOO4_STAGE_QR_POTRF,
+  SHAMPOO4_STAGE_QR_TRSM_PANEL, SHAMPOO4_STAGE_QR_SYRK, SHAMPOO4_STAGE_QR_SOLVE_UPDATE,
+  SHAMPOO4_STAGE_QR_SOLVE_PANEL, SHAMPOO4_STAGE_QR_CONVERT, SHAMPOO4_STAGE_RAYLEIGH_GEMM,
+  SHAMPOO4_STAGE_RAYLEIGH, SHAMPOO4_STAGE_REQUANT, SHAMPOO4_STAGE_PRECOND_DEQUANT,
+  SHAMPOO4_STAGE_PRECOND_MU, SHAMPOO4_STAGE_ROOTS, SHAMPOO4_STAGE_APPLY_LEFT,
+  SHAMPOO4_STAGE_APPLY_RIGHT, SHAMPOO4_STAGE_COUNT
+} shampoo4_stage;
+
+/* Launch timing, for diagnostics and roofline figures.  While enabled, every
+ * kernel launch of the handle is bracketed by a pair of CUDA events on the
+ * call's stream.  Enabling or disabling clears the totals. */
+shampoo4_status shampoo4_timing_enable(shampoo4_handle h, int32_t enable);
+
+/* Totals for one stage since timing was enabled: device milliseconds,
+ * launches, and the algorithmic flops and bytes of those launches (flops
+ * 2 M N K per product, M (M+1) K when only one triangle of a symmetric
+ * output is needed).  Synchronizes on the recorded events. */
+shampoo4_status shampoo4_timing_read(shampoo4_handle h, int32_t stage, double* ms,
+                                     int64_t* launches, double* flops, double* bytes);
+const char* shampoo4_stage_name(int32_t stage);
+
+/* Block-wise linear square 4-bit quantization of `count` fp32 tensors.
+ * For tensor i: n[i] elements at d_x[i] (4-byte aligned), ceil(n[i]/2) code
+ * bytes to d_codes[i], ceil(n[i]/64) scales to d_scales[i].
+ * Per block of 64 consecutive elements: scale = max |x| (NaN if the block
+ * holds a NaN, +Inf if it holds an infinity), v = x / scale (IEEE division),
+ * code = number of the 15 thresholds t_k strictly below v, where t_k is the
+ * fp32-rounded midpoint of adjacent levels of the codebook
+ * cb_j = sgn(y) y^2, y = (2j-15)/15; an all-zero block gets code 7.
+ * Element 2i goes to the low nibble of byte i; a padded nibble is 0. */
+shampoo4_status quant4_pack(const float* const* d_x, const int64_t* n, int32_t count,
+                            uint8_t* const* d_codes, float* const* d_scales,
+                            shampoo4_stream_t stream);
+
+/* Inverse of quant4_pack: x = fp32(cb_code) * scale (one fp32 multiply). */
+shampoo4_status quant4_unpack(const uint8_t* const* d_codes, const float* const* d_scales,
+                              const int64_t* n, int32_t count, float* const* d_x,
+                              shampoo4_stream_t stream);
+
+/* The 16 codebook levels and 15 thresholds the codec uses (host copy). */
+shampoo4_status quant4_tables(float codebook[16], float thresholds[15]);
+
+void shampoo4_destroy(shampoo4_handle h);
+const char* shampoo4_status_string(shampoo4_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SHAMPOO4_H */

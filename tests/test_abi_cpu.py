@@ -1,0 +1,111 @@
+"""Host-side checks of the C ABI, no GPU: the library loads, exports every
+entry point the header declares, plans tiles like the oracle, and rejects bad
+arguments before touching a device."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+from bit_quantized_shampoo_b200 import _lib as L
+from bit_quantized_shampoo_b200.workloads import WORKLOADS
+from oracle import shampoo4_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "shampoo4.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b((?:shampoo4|quant4)_[a-z_]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_entry_point():
+    lib = L.lib()
+    names = _declared()
+    assert len(names) >= 17
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_codec_tables_match_the_oracle_definition():
+    cb = (C.c_float * 16)()
+    th = (C.c_float * 15)()
+    L.call("quant4_tables", cb, th)
+    assert np.array_equal(np.array(cb, np.float32), O.codebook_f32())
+    assert np.array_equal(np.array(th, np.float32), O.thresholds_f32())
+
+
+def _init(shapes, **kw):
+    cfg = L.Config(kw.get("beta", 0.95), kw.get("eps", 1e-6), kw.get("max_block", 1024), kw.get("qb", 64),
+                   kw.get("bj", 5), kw.get("prec", 0))
+    params = (L.Param * len(shapes))(*[L.Param(r, c) for r, c in shapes])
+    h = C.c_void_p()
+    st = L.lib().shampoo4_init(C.byref(cfg), params, len(shapes), C.byref(h))
+    return st, h
+
+
+@pytest.mark.parametrize("wid", [1, 2, 3, 4, 5])
+def test_plan_matches_oracle_partition(wid):
+    w = WORKLOADS[wid]
+    st, h = _init(w.shapes, max_block=w.max_block)
+    assert st == 0
+    try:
+        nb, nf = C.c_int32(), C.c_int32()
+        L.call("shampoo4_counts", h, C.byref(nb), C.byref(nf))
+        blocks = O.partition(w.shapes, w.max_block)
+        assert nb.value == len(blocks) and nf.value == 2 * len(blocks)
+        p, m, n = C.c_int32(), C.c_int32(), C.c_int32()
+        r0, c0 = C.c_int64(), C.c_int64()
+        for k, b in enumerate(blocks):
+            L.call("shampoo4_block_info", h, k, C.byref(p), C.byref(r0), C.byref(c0), C.byref(m), C.byref(n))
+            assert (p.value, r0.value, c0.value, m.value, n.value) == (b.param, b.r0, b.c0, b.m, b.n)
+        # state layout: every factor's pieces are disjoint, 256-aligned and inside the state
+        sb, wb = C.c_size_t(), C.c_size_t()
+        L.call("shampoo4_sizes", h, C.byref(sb), C.byref(wb))
+        spans = []
+        for f in range(nf.value):
+            o = [C.c_size_t() for _ in range(4)]
+            d = C.c_int32()
+            L.call("shampoo4_factor_layout", h, f, *[C.byref(x) for x in o], C.byref(d))
+            b = blocks[f // 2]
+            assert d.value == (b.m if f % 2 == 0 else b.n)
+            dd = d.value * d.value
+            sizes = [4 * dd, (dd + 1) // 2, 4 * ((dd + 63) // 64), 4 * d.value]
+            for off, sz in zip(o, sizes):
+                assert off.value % 256 == 0
+                spans.append((off.value, off.value + sz))
+        spans.sort()
+        assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+        assert spans[-1][1] <= sb.value
+        assert wb.value > 0
+    finally:
+        L.lib().shampoo4_destroy(h)
+
+
+def test_init_rejects_bad_configs():
+    bad = [dict(beta=1.0), dict(beta=-0.1), dict(eps=0.0), dict(max_block=0), dict(max_block=2048),
+           dict(qb=32), dict(bj=-1), dict(bj=17), dict(prec=2)]
+    for kw in bad:
+        st, h = _init([(8, 8)], **kw)
+        assert st == 1, kw
+    st, h = _init([(0, 8)])
+    assert st == 1
+
+
+def test_calls_before_bind_are_not_ready_and_null_handles_invalid():
+    st, h = _init([(8, 8)])
+    assert st == 0
+    try:
+        lib = L.lib()
+        assert lib.shampoo4_refresh_roots(h, None) == 3
+        g = L.ptr_array([0])
+        assert lib.shampoo4_update_stats(h, g, L.i64_array([8]), None) == 3
+        assert lib.shampoo4_refresh_roots(None, None) == 1
+        assert lib.shampoo4_block_info(h, 5, None, None, None, None, None) == 1
+        assert lib.quant4_pack(None, None, -1, None, None, None) == 1
+        assert lib.quant4_pack(None, None, 0, None, None, None) == 0
+        assert lib.shampoo4_status_string(3)
+    finally:
+        L.lib().shampoo4_destroy(h)

@@ -1,0 +1,110 @@
+"""quant4_pack / quant4_unpack on the GPU against the oracle codec: codes and
+scales bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import shampoo4_oracle as O
+from gpu_helpers import cuda_f32
+
+pytestmark = pytest.mark.gpu
+
+
+def _api():
+    from bit_quantized_shampoo_b200 import api
+    return api
+
+
+def _check(xs):
+    api = _api()
+    tx = [cuda_f32(x) for x in xs]
+    codes, scales = api.quant4_pack(tx)
+    torch.cuda.synchronize()
+    for x, c, s in zip(xs, codes, scales):
+        oc, os_ = O.quantize(x)
+        gc, gs = c.cpu().numpy(), s.cpu().numpy()
+        assert np.array_equal(gc, oc), (x.size, np.nonzero(gc != oc)[0][:8])
+        assert np.array_equal(gs.view(np.uint32), os_.view(np.uint32)) or \
+            np.array_equal(np.isnan(gs), np.isnan(os_)) and np.array_equal(gs[~np.isnan(gs)], os_[~np.isnan(os_)])
+    back = api.quant4_unpack(codes, scales, [x.size for x in xs])
+    torch.cuda.synchronize()
+    for x, c, s, b in zip(xs, codes, scales, back):
+        ref = O.dequantize(c.cpu().numpy(), s.cpu().numpy(), x.size)
+        got = b.cpu().numpy()
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)) or \
+            (np.array_equal(np.isnan(got), np.isnan(ref)) and np.array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)]))
+
+
+def test_ragged_sizes_one_batch():
+    rng = np.random.default_rng(11)
+    sizes = [1, 2, 7, 8, 63, 64, 65, 127, 128, 4095, 4096, 4097, 8193, 100003, 1 << 18]
+    _check([rng.standard_normal(n).astype(np.float32) for n in sizes])
+
+
+def test_eigenvector_shaped_inputs():
+    from bit_quantized_shampoo_b200.workloads import u_like
+    xs = [u_like(d, 100 + d)[0].ravel() for d in (64, 147, 576, 768, 1024)]
+    _check(xs)
+
+
+def test_special_values():
+    rng = np.random.default_rng(12)
+    t = O.thresholds_f32()
+    blocks = []
+    blocks.append(np.zeros(64, np.float32))                                   # zero block
+    blocks.append((rng.standard_normal(64) * 1e-39).astype(np.float32))      # subnormal scale
+    b = (rng.standard_normal(64) * 1e-30).astype(np.float32); b[0] = 1.0     # tiny quotients
+    blocks.append(b)
+    b = np.concatenate([t, -t, [1.0], np.zeros(64 - 31)]).astype(np.float32)  # exact ties, absmax 1
+    blocks.append(b[:64])
+    b = rng.standard_normal(64).astype(np.float32); b[5] = -np.abs(b).max(); b[9] = -b[5]   # +-absmax tie
+    blocks.append(b)
+    b = np.ones(64, np.float32); b[3] = np.nan; blocks.append(b)
+    b = np.ones(64, np.float32); b[4] = np.inf; b[7] = -np.inf; blocks.append(b)
+    b = (rng.standard_normal(64) * 3e38).astype(np.float32); blocks.append(b)   # near overflow
+    b = (rng.standard_normal(64)).astype(np.float32) * np.float32(2.0 ** -126); blocks.append(b)
+    _check([np.concatenate(blocks).astype(np.float32)])
+    _check(blocks)
+
+
+def test_shared_divisor_division_matches_ieee_over_exponent_range():
+    rng = np.random.default_rng(13)
+    xs = []
+    for e in range(-140, 120, 7):
+        x = rng.standard_normal(64 * 97).astype(np.float32) * np.float32(2.0 ** e)
+        m = rng.integers(-60, 1, size=x.size).astype(np.float32)
+        xs.append((x * np.exp2(m)).astype(np.float32))
+    _check(xs)
+
+
+def test_misaligned_pointers():
+    api = _api()
+    rng = np.random.default_rng(14)
+    n = 1000
+    x = rng.standard_normal(n + 3).astype(np.float32)
+    tx = cuda_f32(x)[1:n + 1]                      # 4-byte but not 16-byte aligned
+    cbuf = torch.empty(n // 2 + 3, dtype=torch.uint8, device="cuda")
+    sbuf = torch.empty((n + 63) // 64 + 1, dtype=torch.float32, device="cuda")
+    codes, scales = api.quant4_pack([tx], codes=[cbuf[1:1 + n // 2]], scales=[sbuf[1:]])
+    torch.cuda.synchronize()
+    oc, os_ = O.quantize(x[1:n + 1])
+    assert np.array_equal(codes[0].cpu().numpy(), oc)
+    assert np.array_equal(scales[0].cpu().numpy()[:os_.size], os_)
+
+
+def test_large_tensor_sampled():
+    api = _api()
+    n = (1 << 27) + 37                            # 512 MiB of fp32, ragged tail
+    g = torch.Generator(device="cuda").manual_seed(5)
+    x = torch.randn(n, device="cuda", generator=g)
+    codes, scales = api.quant4_pack([x])
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(15)
+    nb = (n + 63) // 64
+    for b in list(rng.integers(0, nb, 64)) + [nb - 1]:
+        lo, hi = 64 * int(b), min(64 * int(b) + 64, n)
+        xb = x[lo:hi].cpu().numpy()
+        oc, os_ = O.quantize(xb)
+        assert scales[0][int(b)].item() == os_[0]
+        gc = codes[0][lo // 2:(hi + 1) // 2].cpu().numpy()
+        assert np.array_equal(gc, oc)

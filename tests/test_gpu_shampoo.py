@@ -1,0 +1,130 @@
+"""Stage parity of the preconditioner step on the GPU against the oracle,
+with the library's incoming state injected into the oracle before each
+stage."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import shampoo4_oracle as O
+from gpu_helpers import basis_root, cuda_f32, gpu_factor, oracle_from_gpu, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+# relative Frobenius bounds of the dense stages (stats, precondition)
+TOL = {"tf32": 2e-3, "fp32": 1e-5}
+
+SHAPE_SETS = {
+    "square128": [(128, 128)],
+    "ragged": [(64, 147), (200, 130), (96, 576)],
+    "multi_tile": [(300, 260)],
+}
+
+
+def _grads(shapes, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return [(rng.standard_normal(s) * scale).astype(np.float32) for s in shapes]
+
+
+def _mk(shapes, precision, **kw):
+    from bit_quantized_shampoo_b200 import api
+    return api.Shampoo4(shapes, precision=precision, **kw)
+
+
+@pytest.mark.parametrize("precision", ["tf32", "fp32"])
+@pytest.mark.parametrize("which", list(SHAPE_SETS))
+def test_update_stats(which, precision):
+    shapes = SHAPE_SETS[which]
+    sh = _mk(shapes, precision)
+    orc = O.Shampoo4Oracle(shapes, beta=float(np.float32(0.95)))
+    for step in range(3):
+        gs = _grads(shapes, 100 + step)
+        sh.update_stats([cuda_f32(g) for g in gs])
+        orc.update_stats(gs)
+    torch.cuda.synchronize()
+    worst = 0.0
+    for f in range(sh.nfactors):
+        S = sh.factor_views(f)[0].cpu().numpy()
+        assert np.array_equal(S, S.T)                     # mirrored symmetric output
+        worst = max(worst, rel_fro(S, orc.factors[f].S))
+    print(f"stats {which} {precision}: worst rel {worst:.3e}")
+    assert worst <= TOL[precision]
+    assert sh.status_flags() == 0
+
+
+@pytest.mark.parametrize("precision", ["tf32", "fp32"])
+@pytest.mark.parametrize("which", list(SHAPE_SETS))
+def test_refresh_and_precondition(which, precision):
+    shapes = SHAPE_SETS[which]
+    sh = _mk(shapes, precision)
+    eps = float(np.float32(1e-6))
+    report = []
+    for rnd in range(2):                       # first refresh (U = I), then a warm one
+        for step in range(2):
+            gs = _grads(shapes, 200 + 10 * rnd + step)
+            sh.update_stats([cuda_f32(g) for g in gs])
+        torch.cuda.synchronize()
+        orc = oracle_from_gpu(sh, shapes, has_basis=(rnd > 0))
+        orc.refresh_roots()
+        sh.refresh_roots()
+        torch.cuda.synchronize()
+        assert sh.status_flags() == 0
+        for f in range(sh.nfactors):
+            d = orc.factors[f].d
+            Qg = sh.debug_q(f).cpu().numpy().astype(np.float64)
+            g = gpu_factor(sh, f)
+            # (i) requantized codes: bit-exact with the oracle quantizer on the GPU's Q
+            oc, os_ = O.quantize(Qg.astype(np.float32).ravel())
+            assert np.array_equal(g.codes, oc) and np.array_equal(g.scales, os_)
+            # (ii) orthonormality of the GPU's Q
+            orth = np.linalg.norm(Qg.T @ Qg - np.eye(d)) / np.sqrt(d)
+            assert orth <= 1e-5, orth
+            # (iii) eigenvalues and (iv) basis-invariant root against the oracle
+            Qo, lo = orc.factors[f].q_last, orc.factors[f].lam.astype(np.float64)
+            lg = g.lam.astype(np.float64)
+            big = lo > 1e3 * eps
+            lam_err = np.max(np.abs(lg[big] - lo[big]) / lo[big]) if big.any() else 0.0
+            root_err = rel_fro(basis_root(Qg, lo, eps), basis_root(Qo, lo, eps))
+            report.append((rnd, f, d, orth, lam_err, root_err))
+        # precondition with the GPU's state injected into the oracle
+        orc2 = oracle_from_gpu(sh, shapes, has_basis=True)
+        gs = _grads(shapes, 300 + rnd)
+        out = sh.precondition([cuda_f32(g) for g in gs])
+        torch.cuda.synchronize()
+        want = orc2.precondition(gs)
+        for o, w in zip(out, want):
+            e = rel_fro(o.cpu().numpy(), w)
+            report.append((rnd, "D", w.shape, e))
+            assert e <= TOL[precision], e
+    for r in report:
+        print("refresh", which, precision, r)
+    worst_lam = max(r[4] for r in report if len(r) == 6)
+    worst_root = max(r[5] for r in report if len(r) == 6)
+    print(f"refresh {which} {precision}: worst lambda {worst_lam:.3e} root {worst_root:.3e}")
+    assert worst_lam < 5e-2 and worst_root < 5e-2
+
+
+def test_precondition_before_refresh_is_not_ready():
+    from bit_quantized_shampoo_b200._lib import Shampoo4Error
+    sh = _mk([(64, 64)], "tf32")
+    g = [cuda_f32(_grads([(64, 64)], 1)[0])]
+    with pytest.raises(Shampoo4Error) as e:
+        sh.precondition(g)
+    assert e.value.status == 3
+
+
+def test_nonfinite_gradient_leaves_statistics_unchanged():
+    from bit_quantized_shampoo_b200._lib import FLAG_NONFINITE_GRAD
+    shapes = [(64, 80), (32, 32)]
+    sh = _mk(shapes, "fp32")
+    gs = _grads(shapes, 5)
+    sh.update_stats([cuda_f32(g) for g in gs])
+    torch.cuda.synchronize()
+    before = [sh.factor_views(f)[0].cpu().numpy().copy() for f in range(sh.nfactors)]
+    bad = [g.copy() for g in gs]
+    bad[0][3, 7] = np.nan
+    sh.update_stats([cuda_f32(g) for g in bad])
+    flags = sh.status_flags()
+    assert flags & FLAG_NONFINITE_GRAD
+    after = [sh.factor_views(f)[0].cpu().numpy() for f in range(sh.nfactors)]
+    assert np.array_equal(after[0], before[0]) and np.array_equal(after[1], before[1])
+    assert not np.array_equal(after[2], before[2])        # the clean parameter still updated
