@@ -61,6 +61,9 @@ _SIGS = {
     "quant4_unpack": [C.POINTER(C.c_void_p), C.POINTER(C.c_void_p), c_i64_p, C.c_int32,
                       C.POINTER(C.c_void_p), C.c_void_p],
     "quant4_tables": [c_f32_p, c_f32_p],
+    "shampoo4_timing_enable": [C.c_void_p, C.c_int32],
+    "shampoo4_timing_read": [C.c_void_p, C.c_int32, C.POINTER(C.c_double), c_i64_p, C.POINTER(C.c_double),
+                             C.POINTER(C.c_double)],
 }
 
 
@@ -76,6 +79,8 @@ def lib() -> C.CDLL:
             f.restype = C.c_int
         L.shampoo4_destroy.argtypes = [C.c_void_p]
         L.shampoo4_destroy.restype = None
+        L.shampoo4_stage_name.argtypes = [C.c_int32]
+        L.shampoo4_stage_name.restype = C.c_char_p
         L.shampoo4_status_string.argtypes = [C.c_int]
         L.shampoo4_status_string.restype = C.c_char_p
         _lib = L

@@ -33,6 +33,21 @@ __host__ __device__ constexpr float threshold_f32(int k) {
 
 constexpr int kQuantBlock = 64;
 
+// Round to the nearest TF32 number (ties away from zero).
+__device__ __forceinline__ float tf32_rn(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+// Store the TF32 split of v: h[i] = RN(v) and, if l, l[i] = RN(v - h[i]).
+__device__ __forceinline__ void put_split(float v, float* h, float* l, int64_t i) {
+  if (!h) return;
+  const float hv = tf32_rn(v);
+  h[i] = hv;
+  if (l) l[i] = tf32_rn(v - hv);
+}
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

@@ -1,0 +1,383 @@
+// Tensor-core batched GEMM for sm_100a: tcgen05.mma (kind::tf32) with the
+// accumulator in tensor memory, operands staged in shared memory by TMA.
+//
+//   C = alpha * op(A) op(B) + beta * Cin        (one CTA per 128 x BN tile)
+//
+// Operands are fp32 matrices in global memory whose values are already
+// TF32 numbers (the kernels that write them round to nearest), so the
+// tensor core's use of the top 19 bits loses nothing.  In split mode each
+// operand comes as a high and a low TF32 part and three products per K step
+// (hi*hi + hi*lo + lo*hi) give fp32-accurate results.
+//
+// Shared memory tiles use the 128-byte swizzle.  An operand whose contraction
+// index is contiguous in memory ("K-major") is loaded as one TMA box of
+// 32 x rows; one whose row index is contiguous ("MN-major") as boxes of
+// 32 x 32, one per 32 rows.  The MMA reads both forms through its matrix
+// descriptors, so no operand is ever transposed.
+//
+// Warp roles (192 threads): warp 0 issues the TMA loads, warp 1 owns the
+// tensor memory and issues the MMAs, warps 2..5 drain the accumulator
+// (warp w reads TMEM lanes 32*(w%4) .. +31, one output row per thread).
+// Every wait on an mbarrier is bounded in time; on expiry the CTA raises
+// SHAMPOO4_FLAG_TIMEOUT, drains what it issued and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include "tc.h"
+
+namespace s4 {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 32;                  // fp32 elements per row of a 128-byte swizzle atom
+constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false after ~2 s without the phase completing.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = now_ns();
+  for (;;) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try(bar, parity)) return true;
+    if (now_ns() - t0 > kWaitNs) return false;
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((addr >> 4) & 0x3FFF);
+  d |= uint64_t((lbo >> 4) & 0x3FFF) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFF) << 32;
+  d |= uint64_t(1) << 46;                 // descriptor version for tcgen05
+  d |= uint64_t(2) << 61;                 // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor: dense, fp32 accumulator, TF32 A and B.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16) |
+         (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float rn_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+template <int BN, bool SPLIT>
+struct TcCfg {
+  static constexpr int kATile = kBM * kBK * 4;                  // bytes
+  static constexpr int kBTile = BN * kBK * 4;
+  static constexpr int kStage = (kATile + kBTile) * (SPLIT ? 2 : 1);
+  static constexpr int kStages = SPLIT ? 3 : 4;
+  static constexpr int kSmem = kStage * kStages + 1024;         // + alignment slack
+  static constexpr int kTmemCols = BN;                          // 128 or 256: a power of two
+};
+
+// Issue the loads of one operand tile (rows mn0.. of the problem, K block k0).
+__device__ __forceinline__ void load_operand(const CUtensorMap* map, const TcOperand& op, int rows, int mn0,
+                                             int k0, uint32_t dst, uint64_t* bar) {
+  if (!op.mn_major) {
+    tma_load_2d(dst, map, op.col0 + k0, op.row0 + mn0, bar);          // box {32 (K), rows}
+  } else {
+    for (int g = 0; g < rows / 32; ++g)                                // boxes {32 (MN), 32 (K)}
+      tma_load_2d(dst + g * 4096, map, op.col0 + mn0 + 32 * g, op.row0 + k0, bar);
+  }
+}
+
+__device__ __forceinline__ uint64_t operand_desc(const TcOperand& op, uint32_t base, int kk) {
+  // K-major: rows of 128 B, 8-row groups 1024 B apart; a K step of 8 is 32 B.
+  // MN-major: 32-row MN groups 4096 B apart, 8-row K groups 1024 B apart.
+  return op.mn_major ? smem_desc(base + kk * 1024, 4096, 1024) : smem_desc(base + kk * 32, 16, 1024);
+}
+
+template <int BN, bool SPLIT>
+__global__ void __launch_bounds__(192, 1)
+k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, int nparams,
+          uint32_t* __restrict__ gflags) {
+  using Cfg = TcCfg<BN, SPLIT>;
+  const TcGemmDesc& g = descs[blockIdx.y];
+  const int tiles_n = (g.N + BN - 1) / BN;
+  const int tiles_m = (g.M + kBM - 1) / kBM;
+  if (int(blockIdx.x) >= tiles_m * tiles_n) return;
+  const int tm = blockIdx.x / tiles_n, tn = blockIdx.x % tiles_n;
+  const int m0 = tm * kBM, n0 = tn * BN;
+  if (g.symmetric && n0 >= m0 + kBM) return;             // wholly above the diagonal
+  if (g.skip && *g.skip) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t full_bar[Cfg::kStages], empty_bar[Cfg::kStages], done_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&done_bar, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                 "r"(Cfg::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = tmem_slot;
+  const int kblocks = (g.K + kBK - 1) / kBK;
+
+  if (warp == 0) {
+    if (lane == 0) {                                        // ---- TMA producer
+      int issued = 0;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % Cfg::kStages;
+        if (kb >= Cfg::kStages && !mbar_wait(&empty_bar[s], ((kb / Cfg::kStages) - 1) & 1)) {
+          atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+          abort_flag = 1;
+          break;
+        }
+        if (*(volatile int*)&abort_flag) break;
+        const uint32_t st = smem_u32(smem + s * Cfg::kStage);
+        mbar_expect_tx(&full_bar[s], Cfg::kStage);
+        const int k0 = kb * kBK;
+        load_operand(g.a.hi, g.a, kBM, m0, k0, st, &full_bar[s]);
+        load_operand(g.b.hi, g.b, BN, n0, k0, st + Cfg::kATile, &full_bar[s]);
+        if (SPLIT) {
+          load_operand(g.a.lo, g.a, kBM, m0, k0, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+          load_operand(g.b.lo, g.b, BN, n0, k0, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+        }
+        issued = kb + 1;
+      }
+      // Whatever happened, the loads issued last must land before the CTA
+      // exits: wait (bounded) for the final phases of the live stages.
+      for (int kb = issued - Cfg::kStages < 0 ? 0 : issued - Cfg::kStages; kb < issued; ++kb)
+        if (!mbar_wait(&full_bar[kb % Cfg::kStages], (kb / Cfg::kStages) & 1)) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {                                        // ---- MMA issuer
+      const uint32_t idesc = idesc_tf32(kBM, BN, g.a.mn_major, g.b.mn_major);
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % Cfg::kStages;
+        if (!mbar_wait(&full_bar[s], (kb / Cfg::kStages) & 1)) {
+          atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+          abort_flag = 1;
+          break;
+        }
+        if (*(volatile int*)&abort_flag) break;
+        fence_after_sync();
+        const uint32_t st = smem_u32(smem + s * Cfg::kStage);
+        const uint32_t a_hi = st, b_hi = st + Cfg::kATile;
+        const uint32_t a_lo = st + Cfg::kATile + Cfg::kBTile, b_lo = a_lo + Cfg::kATile;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 8; ++kk) {
+          const uint32_t acc = (kb | kk) != 0;
+          mma_tf32(tmem, operand_desc(g.a, a_hi, kk), operand_desc(g.b, b_hi, kk), idesc, acc);
+          if (SPLIT) {
+            mma_tf32(tmem, operand_desc(g.a, a_hi, kk), operand_desc(g.b, b_lo, kk), idesc, 1);
+            mma_tf32(tmem, operand_desc(g.a, a_lo, kk), operand_desc(g.b, b_hi, kk), idesc, 1);
+          }
+        }
+        mma_commit(&empty_bar[s]);                          // stage free once these MMAs finish
+      }
+      mma_commit(&done_bar);                                // accumulator complete
+    }
+  } else {                                                  // ---- epilogue, warps 2..5
+    const int q = warp & 3;                                 // TMEM lane quarter = 32-row slab
+    const bool ok = mbar_wait(&done_bar, 0);
+    if (!ok) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+    fence_after_sync();
+    if (ok && !*(volatile int*)&abort_flag) {
+      int64_t ldc = g.ldc;
+      float* C = g.C;
+      if (g.c_ref.tab >= 0) {
+        const PtrEntry& e = tabs[g.c_ref.tab * nparams + g.c_ref.param];
+        ldc = e.ld;
+        C = const_cast<float*>(e.ptr) + g.c_ref.r0 * e.ld + g.c_ref.c0;
+      }
+      // The pipeline buffers are idle now: each warp stages its 32 x 32
+      // chunks there (row pitch 33 floats, conflict-free both ways).
+      float* stg = reinterpret_cast<float*>(smem) + q * (32 * 33);
+      const int row0 = m0 + 32 * q;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        if (n0 + c0 >= g.N) break;                          // warp-uniform
+        uint32_t r[32];
+        tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(c0), r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(r[j]);
+        __syncwarp();
+        // direct store: lane = column, coalesced along the row
+        const int col = n0 + c0 + lane;
+        for (int rr = 0; rr < 32; ++rr) {
+          const int row = row0 + rr;
+          if (row >= g.M) break;
+          if (col >= g.N || (g.symmetric && col > row)) continue;
+          float v = g.alpha * stg[rr * 33 + lane];
+          if (g.beta != 0.0f) v = fmaf(g.beta, g.Cin[int64_t(row) * g.ldcin + col], v);
+          stg[rr * 33 + lane] = v;
+          if (C) C[int64_t(row) * ldc + col] = g.out_round ? rn_tf32(v) : v;
+          if (g.Chi) {
+            const float h = rn_tf32(v);
+            g.Chi[int64_t(row) * g.ldh + col] = h;
+            if (g.Clo) g.Clo[int64_t(row) * g.ldh + col] = rn_tf32(v - h);
+          }
+        }
+        __syncwarp();
+        // mirror store of the strictly-lower part: lane = row, coalesced
+        // along the transposed row
+        if (g.symmetric && n0 + c0 < row0 + 32) {
+          const int row = row0 + lane;
+          for (int j = 0; j < 32; ++j) {
+            const int c = n0 + c0 + j;
+            if (c >= g.N) break;
+            if (row >= g.M || c >= row) continue;
+            const float v = stg[lane * 33 + j];
+            if (C) C[int64_t(c) * ldc + row] = g.out_round ? rn_tf32(v) : v;
+            if (g.Chi) {
+              const float h = rn_tf32(v);
+              g.Chi[int64_t(c) * g.ldh + row] = h;
+              if (g.Clo) g.Clo[int64_t(c) * g.ldh + row] = rn_tf32(v - h);
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(Cfg::kTmemCols)
+                 : "memory");
+  }
+}
+
+template <int BN, bool SPLIT>
+shampoo4_status launch_tc_impl(const TcGemmDesc* d_desc, int count, int max_tiles, const PtrEntry* tabs,
+                               int nparams, uint32_t* gflags, cudaStream_t st) {
+  using Cfg = TcCfg<BN, SPLIT>;
+  static bool configured = false;
+  if (!configured) {
+    S4_CUDA(cudaFuncSetAttribute(k_gemm_tc<BN, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem));
+    configured = true;
+  }
+  for (int base = 0; base < count; base += 65535) {
+    const int c = count - base < 65535 ? count - base : 65535;
+    k_gemm_tc<BN, SPLIT><<<dim3(unsigned(max_tiles), unsigned(c)), 192, Cfg::kSmem, st>>>(d_desc + base, tabs,
+                                                                                        nparams, gflags);
+    S4_CUDA(cudaGetLastError());
+  }
+  return SHAMPOO4_OK;
+}
+
+}  // namespace
+
+int tc_block_n(int split) { return split ? 128 : 256; }
+
+shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split,
+                               const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st) {
+  if (count <= 0 || max_tiles <= 0) return SHAMPOO4_OK;
+  return split ? launch_tc_impl<128, true>(d_desc, count, max_tiles, tabs, nparams, gflags, st)
+               : launch_tc_impl<256, false>(d_desc, count, max_tiles, tabs, nparams, gflags, st);
+}
+
+// ---------------------------------------------------------------- host side
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+}
+
+shampoo4_status tc_encode_map(CUtensorMap* out, const float* base, int64_t rows, int64_t cols, int64_t ld,
+                              int box_rows) {
+  if (!g_encode) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return SHAMPOO4_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  if ((ld * 4) % 16 != 0 || (reinterpret_cast<uintptr_t>(base) % 16) != 0) return SHAMPOO4_ERR_INVALID_ARG;
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(ld) * 4};
+  cuuint32_t box[2] = {32u, cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SHAMPOO4_OK : SHAMPOO4_ERR_CUDA;
+}
+
+}  // namespace s4

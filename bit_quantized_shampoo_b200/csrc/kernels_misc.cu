@@ -123,8 +123,13 @@ __global__ void __launch_bounds__(256) k_basis(const BasisDesc* __restrict__ des
     dequantize8(packed, g.scales[e0 / kQuantBlock], level, v);
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e)
-    if (e0 + e < n) g.U[e0 + e] = v[e];
+  for (int e = 0; e < 8; ++e) {
+    const int64_t i = e0 + e;
+    if (i >= n) break;
+    if (g.U) g.U[i] = v[e];
+    put_split(v[e], g.Uh, g.Ul, i);
+    if (g.Vh) put_split(v[e] * g.mu[i % g.d], g.Vh, g.Vl, i);
+  }
 }
 
 shampoo4_status launch_basis(const BasisDesc* d_desc, int count, int64_t max_elems, cudaStream_t st) {
@@ -198,6 +203,7 @@ k_scan(const ScanDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, in
     int64_t r = e / g.cols, c = e % g.cols;
     float v = X[r * ld + c];
     bad |= !isfinite(v);
+    put_split(v, g.oh, g.ol, e);
   }
   if (__syncthreads_or(bad) && threadIdx.x == 0) {
     *g.flag = 1u;
@@ -218,12 +224,40 @@ shampoo4_status launch_scan(const ScanDesc* d_desc, int count, int64_t max_elems
   return SHAMPOO4_OK;
 }
 
+// ---- shifted Gram diagonal ------------------------------------------------
+__global__ void __launch_bounds__(256) k_shift(const ShiftDesc* __restrict__ descs) {
+  const ShiftDesc& g = descs[blockIdx.x];
+  if (g.skip && *g.skip) return;
+  __shared__ double part[256];
+  double t = 0.0;
+  for (int i = threadIdx.x; i < g.d; i += blockDim.x) t += g.W[int64_t(i) * g.ld + i];
+  part[threadIdx.x] = t;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+    __syncthreads();
+  }
+  const double d = double(g.d);
+  const double s = 11.0 * (2.0 * d * d + d) * 0x1p-53 * part[0];
+  for (int i = threadIdx.x; i < g.d; i += blockDim.x) g.W[int64_t(i) * g.ld + i] += s;
+}
+
+shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st) {
+  if (count <= 0) return SHAMPOO4_OK;
+  k_shift<<<count, 256, 0, st>>>(d_desc);
+  S4_CUDA(cudaGetLastError());
+  return SHAMPOO4_OK;
+}
+
 // ---- fp64 -> fp32 ----------------------------------------------------------
 __global__ void __launch_bounds__(256) k_convert(const ConvertDesc* __restrict__ descs) {
   const ConvertDesc& g = descs[blockIdx.y];
   for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < g.n;
-       e += int64_t(gridDim.x) * blockDim.x)
-    g.dst[e] = float(g.src[e]);
+       e += int64_t(gridDim.x) * blockDim.x) {
+    const float v = float(g.src[e]);
+    g.dst[e] = v;
+    put_split(v, g.dh, g.dl, e);
+  }
 }
 
 shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st) {

@@ -77,11 +77,16 @@ struct TrsmDesc {
   int32_t jb, rows;
 };
 
-// Initial basis of a refresh: U = dequant(codes, scales) or the identity.
+// A basis from the state: U = dequant(codes, scales), or the identity.
+// Outputs, each optional: U (fp32), its TF32 split (Uh, Ul), and the TF32
+// split of U diag(mu) (Vh, Vl; column j scaled by mu[j]).
 struct BasisDesc {
   const uint8_t* codes;
   const float* scales;
   float* U;
+  float* Uh; float* Ul;
+  const float* mu;
+  float* Vh; float* Vl;
   int32_t d;
   int32_t identity;
 };
@@ -112,6 +117,18 @@ struct ScanDesc {
   uint32_t bit; int32_t pad_;
 };
 
+// W <- W + s I with s = 11 (2 d^2 + d) 2^-53 trace(W): the shift of the
+// first pass of shifted Cholesky-QR (Fukaya, Kannan, Nakatsukasa, Zhang,
+// Yamamoto, "Shifted Cholesky QR for computing the QR factorization of
+// ill-conditioned matrices", SIAM J. Sci. Comput. 42(1), 2020), with the
+// Frobenius norm standing in for the spectral norm (a larger, still valid
+// shift).
+struct ShiftDesc {
+  double* W; int64_t ld;
+  int32_t d; int32_t pad_;
+  const uint32_t* skip;
+};
+
 struct ConvertDesc {
   const double* src;
   float* dst;
@@ -135,6 +152,7 @@ shampoo4_status launch_rayleigh(const RayleighDesc* d_desc, int count, int max_d
 shampoo4_status launch_mu(const MuDesc* d_desc, int count, int max_d, float eps, cudaStream_t st);
 shampoo4_status launch_scan(const ScanDesc* d_desc, int count, int64_t max_elems,
                             const PtrEntry* tabs, int nparams, uint32_t* flags, cudaStream_t st);
+shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_clear(const ClearDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 

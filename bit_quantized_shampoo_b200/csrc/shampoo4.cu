@@ -20,7 +20,7 @@ using namespace s4;
 
 namespace {
 
-enum class Kind { GemmF32, GemmF64, Potrf, Trsm, Basis, Rayleigh, Mu, Scan, Convert, Pack };
+enum class Kind { GemmF32, GemmF64, Potrf, Trsm, Basis, Rayleigh, Mu, Scan, Convert, Pack, Shift };
 
 struct Launch {
   Kind kind;
@@ -262,7 +262,7 @@ void build_stats(Builder& b) {
 // Cholesky-QR pass: X (fp32, d x d) -> Q (fp32) through fp64 Gram W = X^T X,
 // blocked right-looking Cholesky W = L L^T and a blocked solve Q L^T = X.
 void build_cholqr_pass(Builder& b, std::vector<Launch>& prog, const std::vector<size_t>& x_off,
-                       const std::vector<size_t>& q_off) {
+                       const std::vector<size_t>& q_off, bool shifted) {
   shampoo4_ctx* h = b.h;
   const size_t nf = h->factors.size();
   int dmax = 0;
@@ -281,6 +281,15 @@ void build_cholqr_pass(Builder& b, std::vector<Launch>& prog, const std::vector<
     }
     b.tag = SHAMPOO4_STAGE_QR_GRAM;
     emit_gemm64(b, prog, g);
+  }
+  if (shifted) {
+    std::vector<ShiftDesc> sd;
+    for (size_t i = 0; i < nf; ++i) {
+      const FactorPlan& f = h->factors[i];
+      sd.push_back({b.wd(f.ws_W64), f.d, f.d, 0, b.fail(i)});
+    }
+    b.tag = SHAMPOO4_STAGE_QR_GRAM;
+    b.emit(prog, Kind::Shift, sd, 0);
   }
   for (int j = 0; j < dmax; j += kPanelW) {
     std::vector<PotrfDesc> po;
@@ -438,9 +447,12 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
     b.tag = SHAMPOO4_STAGE_SUBSPACE;
     emit_gemm32(b, prog, g);
   }
-  // CholeskyQR2: pass 1 on Y (in `other`) -> Q1 into `cur`; pass 2 -> Q in `other`.
-  build_cholqr_pass(b, prog, other, cur);
-  build_cholqr_pass(b, prog, cur, other);
+  // Shifted CholeskyQR3: a shifted pass on Y (in `other`) -> Q0 into `cur`,
+  // then two plain passes cur -> other -> cur.  Q ends in `cur`.
+  build_cholqr_pass(b, prog, other, cur, true);
+  build_cholqr_pass(b, prog, cur, other, false);
+  build_cholqr_pass(b, prog, other, cur, false);
+  std::swap(cur, other);                    // from here on Q is `other`
   for (size_t i = 0; i < nf; ++i) (first ? h->factors[i].ws_q_first : h->factors[i].ws_q_next) = other[i];
   // Rayleigh quotients: T = S Q (fp32-accurate), lambda_i = max(q_i . t_i, 0).
   {
@@ -583,6 +595,9 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
         break;
       case Kind::Scan:
         S4_TRY(launch_scan(static_cast<const ScanDesc*>(d), L.count, L.extent, tabs, np, gflags, st));
+        break;
+      case Kind::Shift:
+        S4_TRY(launch_shift(static_cast<const ShiftDesc*>(d), L.count, st));
         break;
       case Kind::Convert:
         S4_TRY(launch_convert(static_cast<const ConvertDesc*>(d), L.count, L.extent, st));

@@ -1,0 +1,49 @@
+// Descriptors of the tensor-core GEMM (gemm_tc.cu).
+#pragma once
+#include <cuda.h>
+#include "plan.h"
+
+namespace s4 {
+
+// One operand of a tensor-core product: TMA tensor maps of its TF32 value
+// (hi) and, in split mode, of its TF32 residual (lo).  mn_major = 0 when the
+// contraction index is contiguous in memory (map box 32 x rows), 1 when the
+// row index of op(X) is (map box 32 x 32).  (row0, col0) offset the tile
+// coordinates inside the mapped matrix.
+struct TcOperand {
+  const CUtensorMap* hi;
+  const CUtensorMap* lo;
+  int32_t mn_major;
+  int32_t row0, col0;
+  int32_t pad_;
+};
+
+// C = alpha * op(A) op(B) + beta * Cin for one problem.  Outputs, each
+// optional: C (fp32, rounded to TF32 when out_round), and the TF32 split
+// Chi = RN(v), Clo = RN(v - Chi) with leading dimension ldh.  symmetric:
+// only tiles touching the lower triangle run and every element below the
+// diagonal is also written to its mirror position.  skip: problem skipped
+// when *skip != 0.  c_ref: C taken from the per-call pointer tables.
+struct TcGemmDesc {
+  int32_t M, N, K;
+  int32_t symmetric;
+  int32_t out_round;
+  int32_t pad_;
+  float alpha, beta;
+  TcOperand a, b;
+  float* C; int64_t ldc;
+  float* Chi; float* Clo; int64_t ldh;
+  const float* Cin; int64_t ldcin;
+  const uint32_t* skip;
+  OperandRef c_ref;
+};
+
+int tc_block_n(int split);
+shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split,
+                               const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st);
+// Encode a 2-D fp32 tensor map (rows x cols, leading dimension ld elements),
+// 128-byte swizzle, box 32 (contiguous) x box_rows, zero fill out of bounds.
+shampoo4_status tc_encode_map(CUtensorMap* out, const float* base, int64_t rows, int64_t cols, int64_t ld,
+                              int box_rows);
+
+}  // namespace s4

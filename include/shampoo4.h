@@ -94,6 +94,9 @@ typedef struct shampoo4_ctx* shampoo4_handle;
 #define SHAMPOO4_FLAG_NONFINITE_STATE  0x4u  /* a statistic held NaN/Inf at
                                                refresh; that factor kept its
                                                previous basis               */
+#define SHAMPOO4_FLAG_TIMEOUT          0x8u  /* a kernel's bounded wait on one
+                                               of its own pipeline barriers
+                                               expired; its output is invalid */
 
 /* Plan a set of parameters.  Host only: validates the config and shapes,
  * partitions every weight into greedy tiles of at most max_block (ragged
