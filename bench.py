@@ -260,6 +260,7 @@ def main():
                             "flops": fl.value / args.steps, "bytes": by.value / args.steps}
             launches += n.value
     L.call("shampoo4_timing_enable", sh._h, 0)
+    status = sh.status_flags()
 
     pk, pk_src = peaks()
     clocks = clk.summary()
@@ -286,6 +287,7 @@ def main():
             "config": {"workload": w.name, "tiles": sh.nblocks, "factors": sh.nfactors,
                        "steps_per_refresh": 1, "l2": "inputs larger than L2 (2 GB of G, 4 GB of statistics)"},
             "root_refreshes_per_s": value * sh.nfactors,
+            "status_flags": status,
             "gpu_launches": launches,
             "clocks": clocks, "roofline": roof,
             "stages_ms": {k: round(v["ms"], 4) for k, v in sorted(stages.items(), key=lambda kv: -kv[1]["ms"])}}

@@ -23,6 +23,8 @@ STATUS_NAMES = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_CUDA", 3: "ERR_NOT_READY"
 FLAG_NONFINITE_GRAD = 0x1
 FLAG_REFRESH_FAILED = 0x2
 FLAG_NONFINITE_STATE = 0x4
+FLAG_TIMEOUT = 0x8
+FLAG_QR_FALLBACK = 0x10
 PREC_TF32 = 0
 PREC_FP32 = 1
 

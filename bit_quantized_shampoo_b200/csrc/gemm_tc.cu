@@ -76,14 +76,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor, sm_100 version field.  layout: 2 =
+// 128-byte swizzle (16-byte atoms), 1 = 128-byte swizzle with 32-byte atoms
+// (the only swizzled form the MMA accepts for MN-major 32-bit operands).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
   uint64_t d = 0;
   d |= uint64_t((addr >> 4) & 0x3FFF);
   d |= uint64_t((lbo >> 4) & 0x3FFF) << 16;
   d |= uint64_t((sbo >> 4) & 0x3FFF) << 32;
   d |= uint64_t(1) << 46;                 // descriptor version for tcgen05
-  d |= uint64_t(2) << 61;                 // SWIZZLE_128B
+  d |= uint64_t(layout & 7) << 61;
   return d;
 }
 
@@ -128,12 +130,12 @@ __device__ __forceinline__ float rn_tf32(float x) {
   return __uint_as_float(r);
 }
 
-template <int BN, bool SPLIT>
+template <int BN, bool SPLIT, int STAGES>
 struct TcCfg {
   static constexpr int kATile = kBM * kBK * 4;                  // bytes
   static constexpr int kBTile = BN * kBK * 4;
   static constexpr int kStage = (kATile + kBTile) * (SPLIT ? 2 : 1);
-  static constexpr int kStages = SPLIT ? 3 : 4;
+  static constexpr int kStages = STAGES;
   static constexpr int kSmem = kStage * kStages + 1024;         // + alignment slack
   static constexpr int kTmemCols = BN;                          // 128 or 256: a power of two
 };
@@ -150,16 +152,18 @@ __device__ __forceinline__ void load_operand(const CUtensorMap* map, const TcOpe
 }
 
 __device__ __forceinline__ uint64_t operand_desc(const TcOperand& op, uint32_t base, int kk) {
-  // K-major: rows of 128 B, 8-row groups 1024 B apart; a K step of 8 is 32 B.
-  // MN-major: 32-row MN groups 4096 B apart, 8-row K groups 1024 B apart.
-  return op.mn_major ? smem_desc(base + kk * 1024, 4096, 1024) : smem_desc(base + kk * 32, 16, 1024);
+  // K-major (128 B swizzle): rows of 128 B, 8-row groups 1024 B apart; a K
+  // step of 8 is 32 B along the row.
+  // MN-major (128 B swizzle, 32 B atoms): 32-wide MN groups 4096 B apart,
+  // 4-row K groups 512 B apart; a K step of 8 rows is 1024 B.
+  return op.mn_major ? smem_desc(base + kk * 1024, 4096, 512, 1) : smem_desc(base + kk * 32, 16, 1024, 2);
 }
 
-template <int BN, bool SPLIT>
-__global__ void __launch_bounds__(192, 1)
+template <int BN, bool SPLIT, int STAGES>
+__global__ void __launch_bounds__(192, STAGES <= 2 ? 2 : 1)
 k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, int nparams,
           uint32_t* __restrict__ gflags) {
-  using Cfg = TcCfg<BN, SPLIT>;
+  using Cfg = TcCfg<BN, SPLIT, STAGES>;
   const TcGemmDesc& g = descs[blockIdx.y];
   const int tiles_n = (g.N + BN - 1) / BN;
   const int tiles_m = (g.M + kBM - 1) / kBM;
@@ -199,6 +203,12 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
 
   if (warp == 0) {
     if (lane == 0) {                                        // ---- TMA producer
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(g.a.hi)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(g.b.hi)) : "memory");
+      if (SPLIT) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(g.a.lo)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(g.b.lo)) : "memory");
+      }
       int issued = 0;
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % Cfg::kStages;
@@ -277,15 +287,25 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
 #pragma unroll
         for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(r[j]);
         __syncwarp();
-        // direct store: lane = column, coalesced along the row
+        // direct store: lane = column, coalesced along the row.  All 32
+        // loads of Cin are issued before any use so their latencies overlap.
         const int col = n0 + c0 + lane;
+        const bool col_ok = col < g.N;
+        float cin[32];
+        if (g.beta != 0.0f) {
+#pragma unroll
+          for (int rr = 0; rr < 32; ++rr) {
+            const int row = row0 + rr;
+            cin[rr] = (col_ok && row < g.M) ? __ldg(g.Cin + int64_t(row) * g.ldcin + col) : 0.0f;
+          }
+        }
+#pragma unroll
         for (int rr = 0; rr < 32; ++rr) {
           const int row = row0 + rr;
-          if (row >= g.M) break;
-          if (col >= g.N || (g.symmetric && col > row)) continue;
           float v = g.alpha * stg[rr * 33 + lane];
-          if (g.beta != 0.0f) v = fmaf(g.beta, g.Cin[int64_t(row) * g.ldcin + col], v);
+          if (g.beta != 0.0f) v = fmaf(g.beta, cin[rr], v);
           stg[rr * 33 + lane] = v;
+          if (!col_ok || row >= g.M || (g.symmetric && col > row)) continue;
           if (C) C[int64_t(row) * ldc + col] = g.out_round ? rn_tf32(v) : v;
           if (g.Chi) {
             const float h = rn_tf32(v);
@@ -324,19 +344,20 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
   }
 }
 
-template <int BN, bool SPLIT>
+template <int BN, bool SPLIT, int STAGES>
 shampoo4_status launch_tc_impl(const TcGemmDesc* d_desc, int count, int max_tiles, const PtrEntry* tabs,
                                int nparams, uint32_t* gflags, cudaStream_t st) {
-  using Cfg = TcCfg<BN, SPLIT>;
+  using Cfg = TcCfg<BN, SPLIT, STAGES>;
   static bool configured = false;
   if (!configured) {
-    S4_CUDA(cudaFuncSetAttribute(k_gemm_tc<BN, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem));
+    S4_CUDA(cudaFuncSetAttribute(k_gemm_tc<BN, SPLIT, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg::kSmem));
     configured = true;
   }
   for (int base = 0; base < count; base += 65535) {
     const int c = count - base < 65535 ? count - base : 65535;
-    k_gemm_tc<BN, SPLIT><<<dim3(unsigned(max_tiles), unsigned(c)), 192, Cfg::kSmem, st>>>(d_desc + base, tabs,
-                                                                                        nparams, gflags);
+    k_gemm_tc<BN, SPLIT, STAGES><<<dim3(unsigned(max_tiles), unsigned(c)), 192, Cfg::kSmem, st>>>(
+        d_desc + base, tabs, nparams, gflags);
     S4_CUDA(cudaGetLastError());
   }
   return SHAMPOO4_OK;
@@ -346,11 +367,15 @@ shampoo4_status launch_tc_impl(const TcGemmDesc* d_desc, int count, int max_tile
 
 int tc_block_n(int split) { return split ? 128 : 256; }
 
-shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split,
+shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split, int bn,
                                const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st) {
   if (count <= 0 || max_tiles <= 0) return SHAMPOO4_OK;
-  return split ? launch_tc_impl<128, true>(d_desc, count, max_tiles, tabs, nparams, gflags, st)
-               : launch_tc_impl<256, false>(d_desc, count, max_tiles, tabs, nparams, gflags, st);
+  // TF32: two 2-stage CTAs per SM, so one tile's epilogue overlaps the
+  // other's main loop.  Split mode: one 3-stage CTA per SM, or two 2-stage
+  // CTAs with 64-wide tiles for the narrow panel updates.
+  if (!split) return launch_tc_impl<256, false, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, st);
+  if (bn == 64) return launch_tc_impl<64, true, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, st);
+  return launch_tc_impl<128, true, 3>(d_desc, count, max_tiles, tabs, nparams, gflags, st);
 }
 
 // ---------------------------------------------------------------- host side
@@ -360,7 +385,7 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 }
 
 shampoo4_status tc_encode_map(CUtensorMap* out, const float* base, int64_t rows, int64_t cols, int64_t ld,
-                              int box_rows) {
+                              int box_rows, int mn_major) {
   if (!g_encode) {
     cudaDriverEntryPointQueryResult q;
     void* fn = nullptr;
@@ -375,7 +400,8 @@ shampoo4_status tc_encode_map(CUtensorMap* out, const float* base, int64_t rows,
   cuuint32_t box[2] = {32u, cuuint32_t(box_rows)};
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = g_encode(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? SHAMPOO4_OK : SHAMPOO4_ERR_CUDA;
 }

@@ -68,6 +68,7 @@ struct PotrfDesc {
   int32_t jb; int32_t pad_;
   uint32_t* fail;             // set to 1 on a non-positive or non-finite pivot
   uint32_t* gflags;           // ... and SHAMPOO4_FLAG_REFRESH_FAILED ORed here
+  const uint32_t* skip;       // optional: block skipped when *skip != 0
 };
 
 // X[r, 0:jb] <- X[r, 0:jb] * L^-T for r < rows, L the jb x jb lower block.
@@ -75,6 +76,7 @@ struct TrsmDesc {
   const double* L; int64_t ldl;
   double* X; int64_t ldx;
   int32_t jb, rows;
+  const uint32_t* skip;       // optional
 };
 
 // A basis from the state: U = dequant(codes, scales), or the identity.
@@ -115,6 +117,7 @@ struct ScanDesc {
   OperandRef ref;
   uint32_t* flag;
   uint32_t bit; int32_t pad_;
+  float* oh; float* ol;       // optional dense TF32 split of the matrix
 };
 
 // W <- W + s I with s = 11 (2 d^2 + d) 2^-53 trace(W): the shift of the
@@ -129,10 +132,54 @@ struct ShiftDesc {
   const uint32_t* skip;
 };
 
+// ---- fp32-storage pieces of the tensor-core Cholesky-QR ------------------
+// Cholesky of the jb x jb diagonal block of an fp32 matrix, lower, in place,
+// carried out in fp64.
+// On a breakdown: *fail = 1, *clear = 0 (if set), gflags |= REFRESH_FAILED
+// (if set).  Skipped when *fail is already set.
+struct PotrfDescF {
+  float* A; int64_t ld;
+  int32_t jb; int32_t pad_;
+  uint32_t* fail;
+  uint32_t* gflags;
+  uint32_t* clear;
+  float* oh; float* ol;       // optional TF32 split of the factor (same ld)
+};
+
+// X[r, 0:jb] <- Xin[r, 0:jb] L^-T (Xin = X when null), fp64 inside; also
+// stores the TF32 split of the result into (oh, ol) with leading dimension
+// ldo, and, when zero_pad, zeros in columns jb..63 of the split.
+struct TrsmDescF {
+  const float* L; int64_t ldl;
+  const float* Xin;
+  float* X; int64_t ldx;
+  float* oh; float* ol; int64_t ldo;
+  int32_t jb, rows;
+  int32_t zero_pad; int32_t pad_;
+  const uint32_t* skip;
+};
+
+// W <- W + coef * trace(W) * I (the shift of the first Cholesky-QR pass).
+struct ShiftDescF {
+  float* W; int64_t ld;
+  int32_t d; float coef;
+  const uint32_t* skip;
+};
+
+// (h, l) = TF32 split of x, elementwise over n.
+struct SplitDesc {
+  const float* x;
+  float* h; float* l;
+  int64_t n;
+};
+
+// dst = fp32(src); optionally also the TF32 split (dh, dl).
 struct ConvertDesc {
   const double* src;
   float* dst;
+  float* dh; float* dl;
   int64_t n;
+  const uint32_t* skip;       // optional
 };
 
 struct ClearDesc {
@@ -153,6 +200,10 @@ shampoo4_status launch_mu(const MuDesc* d_desc, int count, int max_d, float eps,
 shampoo4_status launch_scan(const ScanDesc* d_desc, int count, int64_t max_elems,
                             const PtrEntry* tabs, int nparams, uint32_t* flags, cudaStream_t st);
 shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st);
+shampoo4_status launch_potrf_f(const PotrfDescF* d_desc, int count, cudaStream_t st);
+shampoo4_status launch_trsm_f(const TrsmDescF* d_desc, int count, int max_rows, cudaStream_t st);
+shampoo4_status launch_shift_f(const ShiftDescF* d_desc, int count, cudaStream_t st);
+shampoo4_status launch_split(const SplitDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_clear(const ClearDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 

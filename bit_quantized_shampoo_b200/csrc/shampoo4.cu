@@ -5,22 +5,31 @@
 //          distributed variants": each tile preconditioned independently,
 //          greedy chunks from index 0, ragged last chunk) and lays out the
 //          caller-owned state and workspace.
-// bind     writes every descriptor of every program into the workspace once;
-//          a program is the fixed list of batched launches of one API call.
+// bind     writes every descriptor and TMA tensor map of every program into
+//          the workspace once; a program is the fixed list of batched
+//          launches of one API call.
 // calls    upload the per-call gradient/output addresses if they changed,
 //          then replay their program on the caller's stream.
+//
+// Kernel choice: a factor whose dimension is a multiple of 4 (rows 16-byte
+// aligned, as TMA needs) runs its products on the tensor cores (gemm_tc.cu);
+// a tile whose both sides are multiples of 4 does too.  The rest use the
+// CUDA-core kernels (gemm_simt.cu).  Both produce the same state.
 #include <algorithm>
 #include <cstring>
+#include <map>
 #include <new>
+#include <tuple>
 #include <vector>
 
-#include "plan.h"
+#include "tc.h"
 
 using namespace s4;
 
 namespace {
 
-enum class Kind { GemmF32, GemmF64, Potrf, Trsm, Basis, Rayleigh, Mu, Scan, Convert, Pack, Shift };
+enum class Kind { GemmF32, GemmF64, Potrf, Trsm, Basis, Rayleigh, Mu, Scan, Convert, Pack, Shift, GemmTC, GemmTCSplit,
+                  GemmTCSplit64, PotrfF, TrsmF, ShiftF, Split };
 
 struct Launch {
   Kind kind;
@@ -41,13 +50,25 @@ struct BlockPlan {
   int32_t param;
   int64_t r0, c0;
   int32_t m, n;
+  bool tc;
+  size_t ws_Gh, ws_Gl, ws_Bh, ws_Bl;   // tensor-core path: G split, apply intermediate split
+  size_t ws_tmp;                       // CUDA-core path: apply intermediate
 };
 
+// Per-factor workspace.  Tensor-core factors: fp32/TF32-split triplets
+// X[0], X[1], Z (m = fp32, h/l = TF32 split), a split Gram or Cholesky
+// factor Th/Tl, the split of S (Sh/Sl), the fp32 Gram/Cholesky matrix W,
+// and fp64 W and Q for the QR fallback.  CUDA-core factors: U, T, Y fp32
+// and fp64 W and Q for the Cholesky-QR.  Both: mu.
 struct FactorPlan {
   int32_t block, side, d;
-  size_t st_S, st_codes, st_scales, st_lam;          // state offsets
-  size_t ws_U, ws_T, ws_Y, ws_W64, ws_Q64, ws_mu;   // workspace offsets
-  size_t ws_q_first, ws_q_next;                      // where each refresh program leaves Q
+  bool tc;
+  size_t st_S, st_codes, st_scales, st_lam;
+  size_t ws_mu;
+  size_t ws_W64, ws_Q64, ws_U, ws_T, ws_Y;
+  size_t ws_Xm[2], ws_Xh[2], ws_Xl[2], ws_Th, ws_Tl, ws_Sh, ws_Sl, ws_W;
+  size_t ws_Zm, ws_Zh, ws_Zl;
+  size_t ws_q_first, ws_q_next;
 };
 
 constexpr size_t kAlign = 256;
@@ -62,10 +83,13 @@ struct shampoo4_ctx {
   std::vector<FactorPlan> factors;
   size_t state_bytes = 0, ws_bytes = 0;
   // workspace regions
-  size_t ws_flags = 0, ws_tabs = 0, ws_fail = 0, ws_bflag = 0, ws_desc = 0, ws_desc_bytes = 0;
+  size_t ws_flags = 0, ws_tabs = 0, ws_fail = 0, ws_bflag = 0, ws_maps = 0, ws_nmaps = 0;
+  size_t ws_tcbad = 0, ws_tcgood = 0;
+  size_t ws_desc = 0, ws_desc_bytes = 0;
   // programs
   std::vector<Launch> prog_stats, prog_refresh_first, prog_refresh, prog_precond;
-  std::vector<uint8_t> arena;      // host image of the descriptor region
+  std::vector<uint8_t> arena;            // host image of the descriptor region
+  std::vector<CUtensorMap> maps;         // host image of the tensor-map region
   // bound buffers
   uint8_t* d_state = nullptr;
   uint8_t* d_ws = nullptr;
@@ -106,12 +130,18 @@ size_t take(size_t& cursor, size_t bytes) {
   return at;
 }
 
+bool tc_dim(int d) { return d % 4 == 0; }
+
 shampoo4_status plan(shampoo4_ctx* h) {
   for (size_t p = 0; p < h->params.size(); ++p) {
     const shampoo4_param& q = h->params[p];
     for (auto rc : chunks(q.rows, h->cfg.max_block))
-      for (auto cc : chunks(q.cols, h->cfg.max_block))
-        h->blocks.push_back({int32_t(p), rc.first, cc.first, rc.second, cc.second});
+      for (auto cc : chunks(q.cols, h->cfg.max_block)) {
+        BlockPlan b{};
+        b.param = int32_t(p); b.r0 = rc.first; b.c0 = cc.first; b.m = rc.second; b.n = cc.second;
+        b.tc = tc_dim(b.m) && tc_dim(b.n);
+        h->blocks.push_back(b);
+      }
   }
   if (h->blocks.size() > (1u << 30)) return SHAMPOO4_ERR_INVALID_ARG;
   size_t st = 0;
@@ -121,6 +151,7 @@ shampoo4_status plan(shampoo4_ctx* h) {
       f.block = int32_t(k);
       f.side = side;
       f.d = side == 0 ? h->blocks[k].m : h->blocks[k].n;
+      f.tc = tc_dim(f.d);
       size_t dd = size_t(f.d) * f.d;
       f.st_S = take(st, 4 * dd);
       f.st_codes = take(st, (dd + 1) / 2);
@@ -135,18 +166,49 @@ shampoo4_status plan(shampoo4_ctx* h) {
   h->ws_flags = take(ws, 16);
   h->ws_tabs = take(ws, sizeof(PtrEntry) * 2 * h->params.size());
   h->ws_fail = take(ws, 4 * h->factors.size());
+  h->ws_tcbad = take(ws, 4 * h->factors.size());
+  h->ws_tcgood = take(ws, 4 * h->factors.size());
   h->ws_bflag = take(ws, 4 * h->blocks.size());
   for (FactorPlan& f : h->factors) {
     size_t dd = size_t(f.d) * f.d;
-    f.ws_U = take(ws, 4 * dd);
-    f.ws_T = take(ws, 4 * dd);
-    f.ws_Y = take(ws, 4 * dd);
-    f.ws_W64 = take(ws, 8 * dd);
-    f.ws_Q64 = take(ws, 8 * dd);
     f.ws_mu = take(ws, 4 * size_t(f.d));
+    if (f.tc) {
+      for (int i = 0; i < 2; ++i) {
+        f.ws_Xm[i] = take(ws, 4 * dd);
+        f.ws_Xh[i] = take(ws, 4 * dd);
+        f.ws_Xl[i] = take(ws, 4 * dd);
+      }
+      f.ws_Th = take(ws, 4 * dd);
+      f.ws_Tl = take(ws, 4 * dd);
+      f.ws_Sh = take(ws, 4 * dd);
+      f.ws_Sl = take(ws, 4 * dd);
+      f.ws_W = take(ws, 4 * dd);
+      f.ws_Zm = take(ws, 4 * dd);
+      f.ws_Zh = take(ws, 4 * dd);
+      f.ws_Zl = take(ws, 4 * dd);
+      f.ws_W64 = take(ws, 8 * dd);            // fp64 fallback of the QR
+      f.ws_Q64 = take(ws, 8 * dd);
+    } else {
+      f.ws_W64 = take(ws, 8 * dd);
+      f.ws_Q64 = take(ws, 8 * dd);
+      f.ws_U = take(ws, 4 * dd);
+      f.ws_T = take(ws, 4 * dd);
+      f.ws_Y = take(ws, 4 * dd);
+    }
   }
-  h->ws_desc = align_up(ws, kAlign);
-  h->ws_bytes = h->ws_desc;     // descriptor bytes are added by build_programs
+  for (BlockPlan& b : h->blocks) {
+    size_t mn = size_t(b.m) * b.n;
+    if (!b.tc) {
+      b.ws_tmp = take(ws, 4 * mn);
+      continue;
+    }
+    b.ws_Gh = take(ws, 4 * mn);
+    b.ws_Gl = take(ws, 4 * mn);
+    b.ws_Bh = take(ws, 4 * mn);
+    b.ws_Bl = take(ws, 4 * mn);
+  }
+  h->ws_maps = align_up(ws, kAlign);
+  h->ws_bytes = h->ws_maps;     // maps and descriptors are added by init
   return SHAMPOO4_OK;
 }
 
@@ -157,6 +219,10 @@ struct Builder {
   std::vector<uint8_t>& arena;
   uint8_t* ws;        // device workspace base (descriptors point into it)
   uint8_t* stb;       // device state base
+  bool encode;        // false: only count tensor maps (sizing pass)
+  int tag = 0;        // stage label applied to the launches emitted next
+  shampoo4_status err = SHAMPOO4_OK;
+  std::map<std::tuple<uintptr_t, int, int, int, int>, size_t> map_index;
 
   template <class D>
   size_t put(const std::vector<D>& v) {
@@ -165,7 +231,6 @@ struct Builder {
     if (!v.empty()) std::memcpy(arena.data() + at, v.data(), sizeof(D) * v.size());
     return at;
   }
-  int tag = 0;          // stage label applied to the launches emitted next
   template <class D>
   void emit(std::vector<Launch>& prog, Kind k, const std::vector<D>& v, int64_t extent,
             double flops = 0, double bytes = 0) {
@@ -186,7 +251,41 @@ struct Builder {
   float* sf(size_t off) const { return reinterpret_cast<float*>(stb + off); }
   uint8_t* sb(size_t off) const { return stb + off; }
   uint32_t* fail(size_t fi) const { return wu(h->ws_fail) + fi; }
+  uint32_t* tcbad(size_t fi) const { return wu(h->ws_tcbad) + fi; }
+  uint32_t* tcgood(size_t fi) const { return wu(h->ws_tcgood) + fi; }
   uint32_t* gflags() const { return wu(h->ws_flags); }
+
+  // Device address of the tensor map of a dense d0 x d1 workspace matrix.
+  const CUtensorMap* map(const float* base, int rows, int cols, int box_rows, int mn_major) {
+    auto key = std::make_tuple(reinterpret_cast<uintptr_t>(base), rows, cols, box_rows, mn_major);
+    auto it = map_index.find(key);
+    size_t idx;
+    if (it != map_index.end()) {
+      idx = it->second;
+    } else {
+      idx = h->maps.size();
+      h->maps.emplace_back();
+      map_index[key] = idx;
+      if (encode) {
+        shampoo4_status s = tc_encode_map(&h->maps.back(), base, rows, cols, cols, box_rows, mn_major);
+        if (s != SHAMPOO4_OK) err = s;
+      }
+    }
+    return reinterpret_cast<const CUtensorMap*>(ws + h->ws_maps + idx * sizeof(CUtensorMap));
+  }
+  // Operand of a tensor-core product from a dense rows x cols matrix held as
+  // a TF32 split (hi, lo).  as_a: the A operand (tile rows 128), else B.
+  // trans: op(X) = X^T.  K-major iff the contraction index is contiguous.
+  TcOperand operand(const float* hi, const float* lo, int rows, int cols, bool as_a, bool trans, bool split,
+                    int bn = 0) {
+    TcOperand o{};
+    const bool k_major = as_a ? !trans : trans;
+    o.mn_major = k_major ? 0 : 1;
+    const int box = k_major ? (as_a ? 128 : (bn ? bn : tc_block_n(split))) : 32;
+    o.hi = map(hi, rows, cols, box, o.mn_major);
+    o.lo = split ? map(lo, rows, cols, box, o.mn_major) : nullptr;
+    return o;
+  }
 };
 
 int tiles128(int M, int N) { return ((M + 127) / 128) * ((N + 127) / 128); }
@@ -200,6 +299,17 @@ GemmF32Desc gemm32(int M, int N, int K, int ta, int tb, int mode, float alpha, f
   return g;
 }
 
+TcGemmDesc gemmtc(int M, int N, int K, float alpha, float beta) {
+  TcGemmDesc g{};
+  g.M = M; g.N = N; g.K = K; g.alpha = alpha; g.beta = beta;
+  g.c_ref.tab = -1;
+  return g;
+}
+
+double product_flops(int M, int N, int K, bool symmetric) {
+  return symmetric ? double(M) * (M + 1) * K : 2.0 * M * N * K;
+}
+
 // Algorithmic flops of a product: 2 M N K, or M (M+1) K for an output known
 // to be symmetric (only one triangle is needed).
 void emit_gemm32(Builder& b, std::vector<Launch>& prog, const std::vector<GemmF32Desc>& v) {
@@ -207,7 +317,7 @@ void emit_gemm32(Builder& b, std::vector<Launch>& prog, const std::vector<GemmF3
   double fl = 0;
   for (auto& g : v) {
     mt = std::max(mt, tiles128(g.M, g.N));
-    fl += g.symmetric ? double(g.M) * (g.M + 1) * g.K : 2.0 * g.M * g.N * g.K;
+    fl += product_flops(g.M, g.N, g.K, g.symmetric);
   }
   b.emit(prog, Kind::GemmF32, v, mt, fl);
 }
@@ -220,75 +330,122 @@ void emit_gemm64(Builder& b, std::vector<Launch>& prog, const std::vector<GemmF6
   }
   b.emit(prog, Kind::GemmF64, v, mt, fl);
 }
+void emit_gemmtc(Builder& b, std::vector<Launch>& prog, const std::vector<TcGemmDesc>& v, bool split,
+                 int bn_override = 0) {
+  const int bn = bn_override ? bn_override : tc_block_n(split);
+  int mt = 0;
+  double fl = 0;
+  for (auto& g : v) {
+    mt = std::max(mt, ((g.M + 127) / 128) * ((g.N + bn - 1) / bn));
+    fl += product_flops(g.M, g.N, g.K, g.symmetric);
+  }
+  b.emit(prog, !split ? Kind::GemmTC : (bn == 64 ? Kind::GemmTCSplit64 : Kind::GemmTCSplit), v, mt, fl);
+}
 
 int mode_of(const shampoo4_config& c) { return c.precision == SHAMPOO4_PREC_FP32 ? kModeFP32 : kModeTF32; }
+bool split_of(const shampoo4_config& c) { return c.precision == SHAMPOO4_PREC_FP32; }
 
-void build_stats(Builder& b) {
+// Scan (and, for tensor-core tiles, split) the per-call gradients.
+void build_grad_copy(Builder& b, std::vector<Launch>& prog, int tag, bool with_flags) {
   shampoo4_ctx* h = b.h;
+  const bool split = split_of(h->cfg);
   std::vector<ScanDesc> scan;
-  std::vector<GemmF32Desc> g;
   int64_t max_elems = 0;
-  double bytes_scan = 0;
-  const float beta = h->cfg.beta, omb = 1.0f - h->cfg.beta;
+  double bytes = 0;
   for (size_t k = 0; k < h->blocks.size(); ++k) {
     const BlockPlan& bp = h->blocks[k];
+    if (!with_flags && !bp.tc) continue;
     ScanDesc s{};
     s.rows = bp.m; s.cols = bp.n;
     s.ref = {0, bp.param, bp.r0, bp.c0};
     s.flag = b.wu(h->ws_bflag) + k;
-    s.bit = SHAMPOO4_FLAG_NONFINITE_GRAD;
+    s.bit = with_flags ? SHAMPOO4_FLAG_NONFINITE_GRAD : 0u;
+    if (bp.tc) {
+      s.oh = b.wf(bp.ws_Gh);
+      s.ol = split ? b.wf(bp.ws_Gl) : nullptr;
+    }
     scan.push_back(s);
     max_elems = std::max<int64_t>(max_elems, int64_t(bp.m) * bp.n);
-    bytes_scan += 4.0 * bp.m * bp.n;
+    bytes += (4.0 + (bp.tc ? (split ? 8.0 : 4.0) : 0.0)) * bp.m * bp.n;
+  }
+  b.tag = tag;
+  b.emit(prog, Kind::Scan, scan, max_elems, 0, bytes);
+}
+
+void build_stats(Builder& b) {
+  shampoo4_ctx* h = b.h;
+  const bool split = split_of(h->cfg);
+  build_grad_copy(b, h->prog_stats, SHAMPOO4_STAGE_STATS_SCAN, true);
+  std::vector<GemmF32Desc> g;
+  std::vector<TcGemmDesc> t;
+  const float beta = h->cfg.beta, omb = 1.0f - h->cfg.beta;
+  for (size_t k = 0; k < h->blocks.size(); ++k) {
+    const BlockPlan& bp = h->blocks[k];
+    uint32_t* skip = b.wu(h->ws_bflag) + k;
     for (int side = 0; side < 2; ++side) {
       const FactorPlan& f = h->factors[2 * k + side];
-      GemmF32Desc d = side == 0 ? gemm32(bp.m, bp.m, bp.n, 0, 1, mode_of(h->cfg), omb, beta)
-                                : gemm32(bp.n, bp.n, bp.m, 1, 0, mode_of(h->cfg), omb, beta);
-      d.a_ref = {0, bp.param, bp.r0, bp.c0};
-      d.b_ref = d.a_ref;
-      d.C = b.sf(f.st_S); d.ldc = f.d;
-      d.Cin = d.C; d.ldcin = f.d;
-      d.symmetric = 1;
-      d.skip = s.flag;
-      g.push_back(d);
+      const int d = f.d, kk = side == 0 ? bp.n : bp.m;
+      if (bp.tc) {
+        // L: A = G (K-major), B = G^T as op(B)[k,j] = G[j,k] (K-major).
+        // R: A = G^T (MN-major), B = G (MN-major).
+        TcGemmDesc x = gemmtc(d, d, kk, omb, beta);
+        x.a = b.operand(b.wf(bp.ws_Gh), b.wf(bp.ws_Gl), bp.m, bp.n, true, side == 1, split);
+        x.b = b.operand(b.wf(bp.ws_Gh), b.wf(bp.ws_Gl), bp.m, bp.n, false, side == 0, split);
+        x.C = b.sf(f.st_S); x.ldc = d;
+        x.Cin = x.C; x.ldcin = d;
+        x.symmetric = 1;
+        x.skip = skip;
+        t.push_back(x);
+      } else {
+        GemmF32Desc x = side == 0 ? gemm32(d, d, kk, 0, 1, mode_of(h->cfg), omb, beta)
+                                  : gemm32(d, d, kk, 1, 0, mode_of(h->cfg), omb, beta);
+        x.a_ref = {0, bp.param, bp.r0, bp.c0};
+        x.b_ref = x.a_ref;
+        x.C = b.sf(f.st_S); x.ldc = d;
+        x.Cin = x.C; x.ldcin = d;
+        x.symmetric = 1;
+        x.skip = skip;
+        g.push_back(x);
+      }
     }
   }
-  b.tag = SHAMPOO4_STAGE_STATS_SCAN;
-  b.emit(h->prog_stats, Kind::Scan, scan, max_elems, 0, bytes_scan);
   b.tag = SHAMPOO4_STAGE_STATS_GEMM;
+  emit_gemmtc(b, h->prog_stats, t, split);
   emit_gemm32(b, h->prog_stats, g);
 }
 
-// Cholesky-QR pass: X (fp32, d x d) -> Q (fp32) through fp64 Gram W = X^T X,
-// blocked right-looking Cholesky W = L L^T and a blocked solve Q L^T = X.
-void build_cholqr_pass(Builder& b, std::vector<Launch>& prog, const std::vector<size_t>& x_off,
-                       const std::vector<size_t>& q_off, bool shifted) {
+// fp64 Cholesky-QR pass over the factors with use[i]: X (fp32, d x d) -> Q
+// (fp32) through the fp64 Gram W = X^T X (+ shift), blocked right-looking
+// Cholesky W = L L^T and a blocked solve Q L^T = X, all on CUDA cores.
+// qh/ql (optional) receive the TF32 split of Q.  skip[i]: per-factor flag
+// that suppresses the pass.  Used by the CUDA-core factors, and by the
+// tensor-core factors whose fp32 factorization broke down.
+void build_cholqr_pass(Builder& b, std::vector<Launch>& prog, const std::vector<char>& use,
+                       const std::vector<const float*>& X, const std::vector<float*>& Q,
+                       const std::vector<float*>& qh, const std::vector<float*>& ql,
+                       const std::vector<const uint32_t*>& skip, bool shifted) {
   shampoo4_ctx* h = b.h;
   const size_t nf = h->factors.size();
   int dmax = 0;
-  for (auto& f : h->factors) dmax = std::max(dmax, f.d);
+  for (size_t i = 0; i < nf; ++i) if (use[i]) dmax = std::max(dmax, h->factors[i].d);
+  if (dmax == 0) return;
   {
     std::vector<GemmF64Desc> g;
+    std::vector<ShiftDesc> sd;
     for (size_t i = 0; i < nf; ++i) {
+      if (!use[i]) continue;
       const FactorPlan& f = h->factors[i];
       GemmF64Desc d{};
       d.M = d.N = d.K = f.d; d.ta = 1; d.tb = 0; d.lower_only = 1;
-      d.A = b.wf(x_off[i]); d.lda = f.d; d.B = d.A; d.ldb = f.d;
+      d.A = X[i]; d.lda = f.d; d.B = d.A; d.ldb = f.d;
       d.C = b.wd(f.ws_W64); d.ldc = f.d; d.c_f64 = 1;
       d.alpha = 1.0; d.beta = 0.0;
-      d.skip = b.fail(i);
+      d.skip = skip[i];
       g.push_back(d);
+      if (shifted) sd.push_back({b.wd(f.ws_W64), f.d, f.d, 0, skip[i]});
     }
     b.tag = SHAMPOO4_STAGE_QR_GRAM;
     emit_gemm64(b, prog, g);
-  }
-  if (shifted) {
-    std::vector<ShiftDesc> sd;
-    for (size_t i = 0; i < nf; ++i) {
-      const FactorPlan& f = h->factors[i];
-      sd.push_back({b.wd(f.ws_W64), f.d, f.d, 0, b.fail(i)});
-    }
-    b.tag = SHAMPOO4_STAGE_QR_GRAM;
     b.emit(prog, Kind::Shift, sd, 0);
   }
   for (int j = 0; j < dmax; j += kPanelW) {
@@ -299,16 +456,16 @@ void build_cholqr_pass(Builder& b, std::vector<Launch>& prog, const std::vector<
     double fl_po = 0, fl_tr = 0;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
-      if (j >= f.d) continue;
+      if (!use[i] || j >= f.d) continue;
       const int jb = std::min(kPanelW, f.d - j);
       double* W = b.wd(f.ws_W64);
       const int64_t ld = f.d;
-      po.push_back({W + j * ld + j, ld, jb, 0, b.fail(i), b.gflags()});
+      po.push_back({W + j * ld + j, ld, jb, 0, b.fail(i), b.gflags(), skip[i]});
       fl_po += double(jb) * jb * jb / 3.0;
       const int rest = f.d - j - jb;
       if (rest > 0) {
         fl_tr += double(rest) * jb * jb;
-        tr.push_back({W + j * ld + j, ld, W + (j + jb) * ld + j, ld, jb, rest});
+        tr.push_back({W + j * ld + j, ld, W + (j + jb) * ld + j, ld, jb, rest, skip[i]});
         max_rows = std::max(max_rows, rest);
         GemmF64Desc d{};
         d.M = d.N = rest; d.K = jb; d.ta = 0; d.tb = 1; d.lower_only = 1;
@@ -316,6 +473,7 @@ void build_cholqr_pass(Builder& b, std::vector<Launch>& prog, const std::vector<
         d.A = W + (j + jb) * ld + j; d.lda = ld; d.B = d.A; d.ldb = ld;
         d.C = W + (j + jb) * ld + (j + jb); d.ldc = ld; d.Cin = d.C; d.ldcin = ld;
         d.alpha = -1.0; d.beta = 1.0;
+        d.skip = skip[i];
         sy.push_back(d);
       }
     }
@@ -326,29 +484,28 @@ void build_cholqr_pass(Builder& b, std::vector<Launch>& prog, const std::vector<
     b.tag = SHAMPOO4_STAGE_QR_SYRK;
     emit_gemm64(b, prog, sy);
   }
-  // Solve Q L^T = X by column panels.
-  for (int j = 0; j < dmax; j += kPanelW) {
+  for (int j = 0; j < dmax; j += kPanelW) {          // solve Q L^T = X by column panels
     std::vector<GemmF64Desc> up;
     std::vector<TrsmDesc> tr;
     int max_rows = 0;
     double fl_tr = 0;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
-      if (j >= f.d) continue;
+      if (!use[i] || j >= f.d) continue;
       const int jb = std::min(kPanelW, f.d - j);
       const int64_t ld = f.d;
       fl_tr += double(f.d) * jb * jb;
       double* W = b.wd(f.ws_W64);
-      double* Q = b.wd(f.ws_Q64);
+      double* Qd = b.wd(f.ws_Q64);
       GemmF64Desc d{};
       d.M = f.d; d.N = jb; d.K = j; d.ta = 0; d.tb = 1;
       d.a_f64 = 1; d.b_f64 = 1; d.c_f64 = 1; d.cin_f64 = 0;
-      d.A = Q; d.lda = ld; d.B = W + j * ld; d.ldb = ld;
-      d.C = Q + j; d.ldc = ld; d.Cin = b.wf(x_off[i]) + j; d.ldcin = ld;
+      d.A = Qd; d.lda = ld; d.B = W + j * ld; d.ldb = ld;
+      d.C = Qd + j; d.ldc = ld; d.Cin = X[i] + j; d.ldcin = ld;
       d.alpha = -1.0; d.beta = 1.0;
-      d.skip = b.fail(i);
+      d.skip = skip[i];
       up.push_back(d);
-      tr.push_back({W + j * ld + j, ld, Q + j, ld, jb, f.d});
+      tr.push_back({W + j * ld + j, ld, Qd + j, ld, jb, f.d, skip[i]});
       max_rows = std::max(max_rows, f.d);
     }
     b.tag = SHAMPOO4_STAGE_QR_SOLVE_UPDATE;
@@ -361,18 +518,151 @@ void build_cholqr_pass(Builder& b, std::vector<Launch>& prog, const std::vector<
   double bytes_cv = 0;
   for (size_t i = 0; i < nf; ++i) {
     const FactorPlan& f = h->factors[i];
+    if (!use[i]) continue;
     int64_t n = int64_t(f.d) * f.d;
-    cv.push_back({b.wd(f.ws_Q64), b.wf(q_off[i]), n});
-    bytes_cv += 12.0 * double(n);
+    cv.push_back({b.wd(f.ws_Q64), Q[i], qh[i], ql[i], n, skip[i]});
     max_elems = std::max(max_elems, n);
+    bytes_cv += (12.0 + (qh[i] ? 4.0 : 0.0) + (ql[i] ? 4.0 : 0.0)) * double(n);
   }
   b.tag = SHAMPOO4_STAGE_QR_CONVERT;
   b.emit(prog, Kind::Convert, cv, max_elems, 0, bytes_cv);
 }
 
+// Cholesky-QR pass over the tensor-core factors, fp32-accurate throughout:
+// X -> Q.  Gram W = X^T X on the tensor cores (3xTF32), optional shift
+// W += 1e-5 trace(W) I, blocked right-looking Cholesky W = L L^T (64-wide
+// diagonal blocks and panel solves on CUDA cores in fp64, trailing updates
+// on the tensor cores), then Q L^T = X by column panels (updates on the
+// tensor cores, panel solves on CUDA cores).  Three such passes, the first
+// shifted, form shifted Cholesky-QR3 (Fukaya et al., SIAM J. Sci. Comput.
+// 2020).  The shift only has to exceed the error of the fp32-accurate Gram
+// (about 2e-6 ||X||_F^2); the first pass then leaves Q0 with a condition
+// number near sqrt(shift) / sigma_min(X), and the second pass succeeds when
+// that is below about 1e3.  Factors beyond that break down in a Cholesky
+// panel and are redone in fp64 from the intact Y.
+constexpr float kTcShift = 1e-5f;
+
+struct Triplet { float* m; float* h; float* l; };
+
+void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Triplet>& X,
+                     const std::vector<Triplet>& Q, bool shifted) {
+  shampoo4_ctx* h = b.h;
+  const size_t nf = h->factors.size();
+  int dmax = 0;
+  for (auto& f : h->factors) if (f.tc) dmax = std::max(dmax, f.d);
+  if (dmax == 0) return;
+  {
+    std::vector<TcGemmDesc> g;
+    std::vector<ShiftDescF> sd;
+    for (size_t i = 0; i < nf; ++i) {
+      const FactorPlan& f = h->factors[i];
+      if (!f.tc) continue;
+      const int d = f.d;
+      TcGemmDesc w = gemmtc(d, d, d, 1.0f, 0.0f);
+      w.a = b.operand(X[i].h, X[i].l, d, d, true, true, true);
+      w.b = b.operand(X[i].h, X[i].l, d, d, false, false, true);
+      w.C = b.wf(f.ws_W); w.ldc = d;
+      w.symmetric = 1;
+      w.skip = b.tcbad(i);
+      g.push_back(w);
+      if (shifted) sd.push_back({b.wf(f.ws_W), d, d, kTcShift, b.tcbad(i)});
+    }
+    b.tag = SHAMPOO4_STAGE_QR_GRAM;
+    emit_gemmtc(b, prog, g, true);
+    b.emit(prog, Kind::ShiftF, sd, 0);
+  }
+  // Cholesky, left-looking by 64-wide panels.  For panel J:
+  //   W[j:, J] -= L[j:, <J] L[J, <J]^T      (tensor cores, one tall product)
+  //   L[J, J]   = chol(W[J, J])              (CUDA cores, fp64 inside)
+  //   L[j+jb:, J] = W[j+jb:, J] L[J, J]^-T   (CUDA cores, fp64 inside)
+  // The panels also leave the TF32 split of L in (Th, Tl), which the later
+  // updates and the triangular solve read.
+  for (int j = 0; j < dmax; j += kPanelW) {
+    std::vector<TcGemmDesc> up;
+    std::vector<PotrfDescF> po;
+    std::vector<TrsmDescF> tr;
+    int max_rows = 0;
+    double fl_po = 0, fl_tr = 0;
+    for (size_t i = 0; i < nf; ++i) {
+      const FactorPlan& f = h->factors[i];
+      if (!f.tc || j >= f.d) continue;
+      const int d = f.d, jb = std::min(kPanelW, d - j), rest = d - j - jb;
+      float* W = b.wf(f.ws_W);
+      float* Th = b.wf(f.ws_Th);
+      float* Tl = b.wf(f.ws_Tl);
+      if (j > 0) {
+        TcGemmDesc u = gemmtc(d - j, jb, j, -1.0f, 1.0f);
+        u.a = b.operand(Th, Tl, d, d, true, false, true);
+        u.b = b.operand(Th, Tl, d, d, false, true, true, 64);
+        u.a.row0 = u.b.row0 = j;
+        u.C = W + int64_t(j) * d + j; u.ldc = d;
+        u.Cin = u.C; u.ldcin = d;
+        u.skip = b.tcbad(i);
+        up.push_back(u);
+      }
+      po.push_back({W + int64_t(j) * d + j, d, jb, 0, b.tcbad(i), b.gflags(), b.tcgood(i),
+                    Th + int64_t(j) * d + j, Tl + int64_t(j) * d + j});
+      fl_po += double(jb) * jb * jb / 3.0;
+      if (rest <= 0) continue;
+      TrsmDescF t{};
+      t.L = W + int64_t(j) * d + j; t.ldl = d;
+      t.X = W + int64_t(j + jb) * d + j; t.ldx = d;
+      t.oh = Th + int64_t(j + jb) * d + j; t.ol = Tl + int64_t(j + jb) * d + j; t.ldo = d;
+      t.jb = jb; t.rows = rest; t.zero_pad = 0;
+      t.skip = b.tcbad(i);
+      tr.push_back(t);
+      fl_tr += double(rest) * jb * jb;
+      max_rows = std::max(max_rows, rest);
+    }
+    b.tag = SHAMPOO4_STAGE_QR_SYRK;
+    emit_gemmtc(b, prog, up, true, 64);
+    b.tag = SHAMPOO4_STAGE_QR_POTRF;
+    b.emit(prog, Kind::PotrfF, po, 0, fl_po);
+    b.tag = SHAMPOO4_STAGE_QR_TRSM_PANEL;
+    b.emit(prog, Kind::TrsmF, tr, max_rows, fl_tr);
+  }
+  for (int j = 0; j < dmax; j += kPanelW) {          // solve Q L^T = X
+    std::vector<TcGemmDesc> up;
+    std::vector<TrsmDescF> tr;
+    int max_rows = 0;
+    double fl_tr = 0;
+    for (size_t i = 0; i < nf; ++i) {
+      const FactorPlan& f = h->factors[i];
+      if (!f.tc || j >= f.d) continue;
+      const int d = f.d, jb = std::min(kPanelW, d - j);
+      float* W = b.wf(f.ws_W);
+      if (j > 0) {                                    // Q[:, J] = X[:, J] - Q[:, <J] L[J, <J]^T
+        TcGemmDesc u = gemmtc(d, jb, j, -1.0f, 1.0f);
+        u.a = b.operand(Q[i].h, Q[i].l, d, d, true, false, true);
+        u.b = b.operand(b.wf(f.ws_Th), b.wf(f.ws_Tl), d, d, false, true, true, 64);
+        u.b.row0 = j;
+        u.C = Q[i].m + j; u.ldc = d;
+        u.Cin = X[i].m + j; u.ldcin = d;
+        u.skip = b.tcbad(i);
+        up.push_back(u);
+      }
+      TrsmDescF t{};
+      t.L = W + int64_t(j) * d + j; t.ldl = d;
+      t.Xin = j == 0 ? X[i].m : nullptr;
+      t.X = Q[i].m + j; t.ldx = d;
+      t.oh = Q[i].h + j; t.ol = Q[i].l + j; t.ldo = d;
+      t.jb = jb; t.rows = d; t.zero_pad = 0;
+      t.skip = b.tcbad(i);
+      tr.push_back(t);
+      fl_tr += double(d) * jb * jb;
+      max_rows = std::max(max_rows, d);
+    }
+    b.tag = SHAMPOO4_STAGE_QR_SOLVE_UPDATE;
+    emit_gemmtc(b, prog, up, true, 64);
+    b.tag = SHAMPOO4_STAGE_QR_SOLVE_PANEL;
+    b.emit(prog, Kind::TrsmF, tr, max_rows, fl_tr);
+  }
+}
+
 void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
   shampoo4_ctx* h = b.h;
   const size_t nf = h->factors.size();
+  const bool split = split_of(h->cfg);
   int dmax = 0;
   int64_t emax = 0;
   double sum_dd = 0;
@@ -381,10 +671,9 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
     emax = std::max<int64_t>(emax, int64_t(f.d) * f.d);
     sum_dd += double(f.d) * f.d;
   }
-  const double bytes_scan = 4.0 * sum_dd, fl_rq = 2.0 * sum_dd;
-  const double bytes_bd = first ? 4.0 * sum_dd : 4.5625 * sum_dd;
-  {  // non-finite statistic -> keep the factor's previous basis
+  {  // non-finite statistic -> keep the factor's previous basis; split S
     std::vector<ScanDesc> scan;
+    double bytes = 0;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
       ScanDesc s{};
@@ -392,94 +681,207 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
       s.ref.tab = -1;
       s.flag = b.fail(i);
       s.bit = SHAMPOO4_FLAG_NONFINITE_STATE;
+      if (f.tc) { s.oh = b.wf(f.ws_Sh); s.ol = b.wf(f.ws_Sl); }
       scan.push_back(s);
+      bytes += (f.tc ? 12.0 : 4.0) * double(f.d) * f.d;
     }
     b.tag = SHAMPOO4_STAGE_REFRESH_SCAN;
-    b.emit(prog, Kind::Scan, scan, emax, 0, bytes_scan);
+    b.emit(prog, Kind::Scan, scan, emax, 0, bytes);
   }
+  // cur/oth: index of the current and the other triplet (tensor-core
+  // factors) or buffer offsets (CUDA-core factors).
+  std::vector<int> cur(nf, 0);
+  std::vector<size_t> ucur(nf), uoth(nf);
+  for (size_t i = 0; i < nf; ++i) { ucur[i] = h->factors[i].ws_U; uoth[i] = h->factors[i].ws_Y; }
   {
     std::vector<BasisDesc> bd;
+    double bytes = 0;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
-      bd.push_back({b.sb(f.st_codes), b.sf(f.st_scales), b.wf(f.ws_U), f.d, first ? 1 : 0});
+      BasisDesc x{};
+      x.codes = b.sb(f.st_codes); x.scales = b.sf(f.st_scales);
+      x.d = f.d; x.identity = first ? 1 : 0;
+      if (f.tc) { x.U = b.wf(f.ws_Xm[0]); x.Uh = b.wf(f.ws_Xh[0]); x.Ul = b.wf(f.ws_Xl[0]); }
+      else x.U = b.wf(f.ws_U);
+      bd.push_back(x);
+      bytes += (first ? 0.0 : 0.5625) * double(f.d) * f.d + (f.tc ? 12.0 : 4.0) * double(f.d) * f.d;
     }
     b.tag = SHAMPOO4_STAGE_BASIS;
-    b.emit(prog, Kind::Basis, bd, emax, 0, bytes_bd);
+    b.emit(prog, Kind::Basis, bd, emax, 0, bytes);
   }
-  // Bjorck rectification U <- 1.5 U - 0.5 U (U^T U), ping-ponging U and Y.
-  std::vector<size_t> cur(nf), other(nf);
-  for (size_t i = 0; i < nf; ++i) { cur[i] = h->factors[i].ws_U; other[i] = h->factors[i].ws_Y; }
+  // Bjorck rectification U <- 1.5 U - 0.5 U (U^T U).
   const int iters = first ? 0 : h->cfg.bjorck_iters;
   for (int it = 0; it < iters; ++it) {
     std::vector<GemmF32Desc> gram, upd;
+    std::vector<TcGemmDesc> tgram, tupd;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
-      GemmF32Desc g = gemm32(f.d, f.d, f.d, 1, 0, mode_of(h->cfg), 1.0f, 0.0f);
-      g.A = g.B = b.wf(cur[i]); g.lda = g.ldb = f.d;
-      g.C = b.wf(f.ws_T); g.ldc = f.d;
-      g.symmetric = 1;
-      gram.push_back(g);
-      GemmF32Desc u = gemm32(f.d, f.d, f.d, 0, 0, mode_of(h->cfg), -0.5f, 1.5f);
-      u.A = b.wf(cur[i]); u.lda = f.d;
-      u.B = b.wf(f.ws_T); u.ldb = f.d;
-      u.C = b.wf(other[i]); u.ldc = f.d;
-      u.Cin = b.wf(cur[i]); u.ldcin = f.d;
-      upd.push_back(u);
+      const int d = f.d;
+      if (f.tc) {
+        const int c = cur[i], o = 1 - c;
+        TcGemmDesc g = gemmtc(d, d, d, 1.0f, 0.0f);          // T = U^T U
+        g.a = b.operand(b.wf(f.ws_Xh[c]), b.wf(f.ws_Xl[c]), d, d, true, true, split);
+        g.b = b.operand(b.wf(f.ws_Xh[c]), b.wf(f.ws_Xl[c]), d, d, false, false, split);
+        g.Chi = b.wf(f.ws_Th); g.Clo = b.wf(f.ws_Tl); g.ldh = d;
+        g.symmetric = 1;
+        tgram.push_back(g);
+        TcGemmDesc u = gemmtc(d, d, d, -0.5f, 1.5f);         // U' = 1.5 U - 0.5 U T
+        u.a = b.operand(b.wf(f.ws_Xh[c]), b.wf(f.ws_Xl[c]), d, d, true, false, split);
+        u.b = b.operand(b.wf(f.ws_Th), b.wf(f.ws_Tl), d, d, false, true, split);   // T symmetric
+        u.Cin = b.wf(f.ws_Xm[c]); u.ldcin = d;
+        u.C = b.wf(f.ws_Xm[o]); u.ldc = d;
+        u.Chi = b.wf(f.ws_Xh[o]); u.Clo = b.wf(f.ws_Xl[o]); u.ldh = d;
+        tupd.push_back(u);
+        cur[i] = o;
+      } else {
+        GemmF32Desc g = gemm32(d, d, d, 1, 0, mode_of(h->cfg), 1.0f, 0.0f);
+        g.A = g.B = b.wf(ucur[i]); g.lda = g.ldb = d;
+        g.C = b.wf(f.ws_T); g.ldc = d;
+        g.symmetric = 1;
+        gram.push_back(g);
+        GemmF32Desc u = gemm32(d, d, d, 0, 0, mode_of(h->cfg), -0.5f, 1.5f);
+        u.A = b.wf(ucur[i]); u.lda = d;
+        u.B = b.wf(f.ws_T); u.ldb = d;
+        u.C = b.wf(uoth[i]); u.ldc = d;
+        u.Cin = b.wf(ucur[i]); u.ldcin = d;
+        upd.push_back(u);
+        std::swap(ucur[i], uoth[i]);
+      }
     }
     b.tag = SHAMPOO4_STAGE_BJORCK_GRAM;
+    emit_gemmtc(b, prog, tgram, split);
     emit_gemm32(b, prog, gram);
     b.tag = SHAMPOO4_STAGE_BJORCK_UPDATE;
+    emit_gemmtc(b, prog, tupd, split);
     emit_gemm32(b, prog, upd);
-    std::swap(cur, other);
   }
-  // Subspace step Y = (S + eps I) U = S U + eps U, fp32-accurate.
+  // Subspace step Y = (S + eps I) U = S U + eps U, always fp32-accurate.
+  std::vector<const float*> Yx(nf);
+  std::vector<float*> Q0(nf), Q1(nf), Qf(nf), Qh(nf, nullptr), Ql(nf, nullptr), none(nf, nullptr);
   {
     std::vector<GemmF32Desc> g;
+    std::vector<TcGemmDesc> t;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
-      GemmF32Desc y = gemm32(f.d, f.d, f.d, 0, 0, kModeFP32, 1.0f, h->cfg.eps);
-      y.A = b.sf(f.st_S); y.lda = f.d;
-      y.B = b.wf(cur[i]); y.ldb = f.d;
-      y.C = b.wf(other[i]); y.ldc = f.d;
-      y.Cin = b.wf(cur[i]); y.ldcin = f.d;
-      g.push_back(y);
+      const int d = f.d;
+      if (f.tc) {
+        const int c = cur[i], o = 1 - c;
+        TcGemmDesc y = gemmtc(d, d, d, 1.0f, h->cfg.eps);
+        y.a = b.operand(b.wf(f.ws_Sh), b.wf(f.ws_Sl), d, d, true, false, true);
+        y.b = b.operand(b.wf(f.ws_Xh[c]), b.wf(f.ws_Xl[c]), d, d, false, false, true);
+        y.Cin = b.wf(f.ws_Xm[c]); y.ldcin = d;
+        y.C = b.wf(f.ws_Xm[o]); y.ldc = d;
+        y.Chi = b.wf(f.ws_Xh[o]); y.Clo = b.wf(f.ws_Xl[o]); y.ldh = d;
+        t.push_back(y);
+        // shifted CholeskyQR3: Y (X[o]) -> Q0 (X[c]) -> Q1 (X[o]) -> Q (X[c] + split)
+        Yx[i] = b.wf(f.ws_Xm[o]);
+        Q0[i] = b.wf(f.ws_Xm[c]);
+        Q1[i] = b.wf(f.ws_Xm[o]);
+        Qf[i] = b.wf(f.ws_Xm[c]);
+        Qh[i] = b.wf(f.ws_Xh[c]);
+        Ql[i] = b.wf(f.ws_Xl[c]);
+      } else {
+        GemmF32Desc y = gemm32(d, d, d, 0, 0, kModeFP32, 1.0f, h->cfg.eps);
+        y.A = b.sf(f.st_S); y.lda = d;
+        y.B = b.wf(ucur[i]); y.ldb = d;
+        y.C = b.wf(uoth[i]); y.ldc = d;
+        y.Cin = b.wf(ucur[i]); y.ldcin = d;
+        g.push_back(y);
+        Yx[i] = b.wf(uoth[i]);
+        Q0[i] = b.wf(ucur[i]);
+        Q1[i] = b.wf(uoth[i]);
+        Qf[i] = b.wf(ucur[i]);
+      }
     }
     b.tag = SHAMPOO4_STAGE_SUBSPACE;
+    emit_gemmtc(b, prog, t, true);
     emit_gemm32(b, prog, g);
   }
-  // Shifted CholeskyQR3: a shifted pass on Y (in `other`) -> Q0 into `cur`,
-  // then two plain passes cur -> other -> cur.  Q ends in `cur`.
-  build_cholqr_pass(b, prog, other, cur, true);
-  build_cholqr_pass(b, prog, cur, other, false);
-  build_cholqr_pass(b, prog, other, cur, false);
-  std::swap(cur, other);                    // from here on Q is `other`
-  for (size_t i = 0; i < nf; ++i) (first ? h->factors[i].ws_q_first : h->factors[i].ws_q_next) = other[i];
+  {
+    // Tensor-core factors: Y stays in X[o]; fp32 shifted Cholesky-QR3
+    // Y -> X[c] -> Z -> X[c].  A factor whose fp32 Cholesky breaks down
+    // (tcbad) redoes the three passes in fp64 from the intact Y; the others
+    // skip that work (tcgood).  CUDA-core factors run the fp64 passes only.
+    std::vector<Triplet> Xy(nf), Xc(nf), Xz(nf);
+    std::vector<char> use_simt(nf, 0), use_fb(nf, 0);
+    std::vector<const uint32_t*> sk(nf);
+    std::vector<const float*> a1(nf), a2(nf), a3(nf);
+    std::vector<float*> o1(nf), o2(nf), o3(nf), q3h(nf, nullptr), q3l(nf, nullptr);
+    for (size_t i = 0; i < nf; ++i) {
+      const FactorPlan& f = h->factors[i];
+      if (f.tc) {
+        const int c = cur[i], o = 1 - c;
+        Xy[i] = {b.wf(f.ws_Xm[o]), b.wf(f.ws_Xh[o]), b.wf(f.ws_Xl[o])};
+        Xc[i] = {b.wf(f.ws_Xm[c]), b.wf(f.ws_Xh[c]), b.wf(f.ws_Xl[c])};
+        Xz[i] = {b.wf(f.ws_Zm), b.wf(f.ws_Zh), b.wf(f.ws_Zl)};
+        use_fb[i] = 1;
+        sk[i] = b.tcgood(i);
+        a1[i] = Xy[i].m; o1[i] = Xc[i].m;
+        a2[i] = Xc[i].m; o2[i] = Xz[i].m;
+        a3[i] = Xz[i].m; o3[i] = Xc[i].m;
+        q3h[i] = Xc[i].h; q3l[i] = Xc[i].l;
+        Qf[i] = Xc[i].m; Qh[i] = Xc[i].h; Ql[i] = Xc[i].l;
+        Q1[i] = Xz[i].m;                                  // free after the QR
+      } else {
+        use_simt[i] = 1;
+        sk[i] = b.fail(i);
+        a1[i] = Yx[i]; o1[i] = Q0[i];
+        a2[i] = Q0[i]; o2[i] = Q1[i];
+        a3[i] = Q1[i]; o3[i] = Qf[i];
+      }
+    }
+    build_cholqr_tc(b, prog, Xy, Xc, true);
+    build_cholqr_tc(b, prog, Xc, Xz, false);
+    build_cholqr_tc(b, prog, Xz, Xc, false);
+    std::vector<char> use_any(nf);
+    for (size_t i = 0; i < nf; ++i) use_any[i] = use_simt[i] || use_fb[i];
+    build_cholqr_pass(b, prog, use_any, a1, o1, none, none, sk, true);
+    build_cholqr_pass(b, prog, use_any, a2, o2, none, none, sk, false);
+    build_cholqr_pass(b, prog, use_any, a3, o3, q3h, q3l, sk, false);
+  }
+  for (size_t i = 0; i < nf; ++i) {
+    const size_t off = size_t(reinterpret_cast<uint8_t*>(Qf[i]) - b.ws);
+    (first ? h->factors[i].ws_q_first : h->factors[i].ws_q_next) = off;
+  }
   // Rayleigh quotients: T = S Q (fp32-accurate), lambda_i = max(q_i . t_i, 0).
   {
     std::vector<GemmF32Desc> g;
+    std::vector<TcGemmDesc> t;
     std::vector<RayleighDesc> rq;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
-      GemmF32Desc t = gemm32(f.d, f.d, f.d, 0, 0, kModeFP32, 1.0f, 0.0f);
-      t.A = b.sf(f.st_S); t.lda = f.d;
-      t.B = b.wf(other[i]); t.ldb = f.d;
-      t.C = b.wf(f.ws_T); t.ldc = f.d;
-      g.push_back(t);
-      rq.push_back({b.wf(other[i]), b.wf(f.ws_T), b.sf(f.st_lam), f.d, 0, b.fail(i)});
+      const int d = f.d;
+      float* T;
+      if (f.tc) {
+        T = Q1[i];                                         // free again
+        TcGemmDesc x = gemmtc(d, d, d, 1.0f, 0.0f);
+        x.a = b.operand(b.wf(f.ws_Sh), b.wf(f.ws_Sl), d, d, true, false, true);
+        x.b = b.operand(Qh[i], Ql[i], d, d, false, false, true);
+        x.C = T; x.ldc = d;
+        t.push_back(x);
+      } else {
+        T = b.wf(f.ws_T);
+        GemmF32Desc x = gemm32(d, d, d, 0, 0, kModeFP32, 1.0f, 0.0f);
+        x.A = b.sf(f.st_S); x.lda = d;
+        x.B = Qf[i]; x.ldb = d;
+        x.C = T; x.ldc = d;
+        g.push_back(x);
+      }
+      rq.push_back({Qf[i], T, b.sf(f.st_lam), d, 0, b.fail(i)});
     }
     b.tag = SHAMPOO4_STAGE_RAYLEIGH_GEMM;
+    emit_gemmtc(b, prog, t, true);
     emit_gemm32(b, prog, g);
     b.tag = SHAMPOO4_STAGE_RAYLEIGH;
-    b.emit(prog, Kind::Rayleigh, rq, dmax, fl_rq);
+    b.emit(prog, Kind::Rayleigh, rq, dmax, 2.0 * sum_dd);
   }
-  // Requantize Q into the state (skipped for failed factors).
-  {
+  {  // requantize Q into the state (skipped for failed factors)
     Launch L{};
     L.kind = Kind::Pack;
     L.tag = SHAMPOO4_STAGE_REQUANT;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
-      L.px.push_back(b.wf(other[i]));
+      L.px.push_back(Qf[i]);
       L.pn.push_back(int64_t(f.d) * f.d);
       L.pcodes.push_back(b.sb(f.st_codes));
       L.pscales.push_back(b.sf(f.st_scales));
@@ -494,6 +896,7 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
 void build_precondition(Builder& b) {
   shampoo4_ctx* h = b.h;
   const size_t nf = h->factors.size();
+  const bool split = split_of(h->cfg);
   int dmax = 0;
   int64_t emax = 0;
   double sum_dd = 0;
@@ -502,48 +905,89 @@ void build_precondition(Builder& b) {
     emax = std::max<int64_t>(emax, int64_t(f.d) * f.d);
     sum_dd += double(f.d) * f.d;
   }
-  const double bytes_bd = 4.5625 * sum_dd;
   std::vector<BasisDesc> bd;
   std::vector<MuDesc> mu;
   std::vector<GemmF32Desc> roots;
+  std::vector<TcGemmDesc> troots;
+  std::vector<float*> Pm(nf);                  // fp32 root of each factor
+  double bytes_bd = 0;
   for (size_t i = 0; i < nf; ++i) {
     const FactorPlan& f = h->factors[i];
-    bd.push_back({b.sb(f.st_codes), b.sf(f.st_scales), b.wf(f.ws_Y), f.d, 0});
-    mu.push_back({b.sf(f.st_lam), b.wf(f.ws_mu), f.d, 0});
-    // P = (U diag(mu)) U^T
-    GemmF32Desc g = gemm32(f.d, f.d, f.d, 0, 1, mode_of(h->cfg), 1.0f, 0.0f);
-    g.A = b.wf(f.ws_Y); g.lda = f.d; g.kscale = b.wf(f.ws_mu);
-    g.B = b.wf(f.ws_Y); g.ldb = f.d;
-    g.C = b.wf(f.ws_U); g.ldc = f.d;
-    g.symmetric = 1;
-    roots.push_back(g);
+    const int d = f.d;
+    mu.push_back({b.sf(f.st_lam), b.wf(f.ws_mu), d, 0});
+    BasisDesc x{};
+    x.codes = b.sb(f.st_codes); x.scales = b.sf(f.st_scales); x.d = d; x.identity = 0;
+    if (f.tc) {
+      // U -> X[0] split, U diag(mu) -> X[1] split; P = (U mu) U^T -> Th/Tl (+ fp32 in X[1].m)
+      x.Uh = b.wf(f.ws_Xh[0]); x.Ul = split ? b.wf(f.ws_Xl[0]) : nullptr;
+      x.mu = b.wf(f.ws_mu);
+      x.Vh = b.wf(f.ws_Xh[1]); x.Vl = split ? b.wf(f.ws_Xl[1]) : nullptr;
+      TcGemmDesc g = gemmtc(d, d, d, 1.0f, 0.0f);
+      g.a = b.operand(b.wf(f.ws_Xh[1]), b.wf(f.ws_Xl[1]), d, d, true, false, split);
+      g.b = b.operand(b.wf(f.ws_Xh[0]), b.wf(f.ws_Xl[0]), d, d, false, true, split);
+      g.C = b.wf(f.ws_Xm[1]); g.ldc = d;
+      g.Chi = b.wf(f.ws_Th); g.Clo = split ? b.wf(f.ws_Tl) : nullptr; g.ldh = d;
+      g.symmetric = 1;
+      troots.push_back(g);
+      Pm[i] = b.wf(f.ws_Xm[1]);
+      bytes_bd += (0.5625 + (split ? 16.0 : 8.0)) * double(d) * d;
+    } else {
+      x.U = b.wf(f.ws_Y);
+      GemmF32Desc g = gemm32(d, d, d, 0, 1, mode_of(h->cfg), 1.0f, 0.0f);
+      g.A = b.wf(f.ws_Y); g.lda = d; g.kscale = b.wf(f.ws_mu);
+      g.B = b.wf(f.ws_Y); g.ldb = d;
+      g.C = b.wf(f.ws_U); g.ldc = d;
+      g.symmetric = 1;
+      roots.push_back(g);
+      Pm[i] = b.wf(f.ws_U);
+      bytes_bd += 4.5625 * double(d) * d;
+    }
+    bd.push_back(x);
   }
-  b.tag = SHAMPOO4_STAGE_PRECOND_DEQUANT;
-  b.emit(h->prog_precond, Kind::Basis, bd, emax, 0, bytes_bd);
   b.tag = SHAMPOO4_STAGE_PRECOND_MU;
   b.emit(h->prog_precond, Kind::Mu, mu, dmax);
+  b.tag = SHAMPOO4_STAGE_PRECOND_DEQUANT;
+  b.emit(h->prog_precond, Kind::Basis, bd, emax, 0, bytes_bd);
   b.tag = SHAMPOO4_STAGE_ROOTS;
+  emit_gemmtc(b, h->prog_precond, troots, split);
   emit_gemm32(b, h->prog_precond, roots);
+  build_grad_copy(b, h->prog_precond, SHAMPOO4_STAGE_STATS_SCAN, false);
   std::vector<GemmF32Desc> left, right;
+  std::vector<TcGemmDesc> tleft, tright;
   for (size_t k = 0; k < h->blocks.size(); ++k) {
     const BlockPlan& bp = h->blocks[k];
     const FactorPlan& fl = h->factors[2 * k];
     const FactorPlan& fr = h->factors[2 * k + 1];
-    float* tmp = b.wf(bp.m >= bp.n ? fl.ws_T : fr.ws_T);   // m x n fits in max(m,n)^2
-    GemmF32Desc l = gemm32(bp.m, bp.n, bp.m, 0, 0, mode_of(h->cfg), 1.0f, 0.0f);
-    l.A = b.wf(fl.ws_U); l.lda = bp.m;
-    l.b_ref = {0, bp.param, bp.r0, bp.c0};
-    l.C = tmp; l.ldc = bp.n;
-    left.push_back(l);
-    GemmF32Desc r = gemm32(bp.m, bp.n, bp.n, 0, 0, mode_of(h->cfg), 1.0f, 0.0f);
-    r.A = tmp; r.lda = bp.n;
-    r.B = b.wf(fr.ws_U); r.ldb = bp.n;
-    r.c_ref = {1, bp.param, bp.r0, bp.c0};
-    right.push_back(r);
+    if (bp.tc) {
+      TcGemmDesc l = gemmtc(bp.m, bp.n, bp.m, 1.0f, 0.0f);       // B = P_L G
+      l.a = b.operand(b.wf(fl.ws_Th), b.wf(fl.ws_Tl), bp.m, bp.m, true, false, split);
+      l.b = b.operand(b.wf(bp.ws_Gh), b.wf(bp.ws_Gl), bp.m, bp.n, false, false, split);
+      l.Chi = b.wf(bp.ws_Bh); l.Clo = split ? b.wf(bp.ws_Bl) : nullptr; l.ldh = bp.n;
+      tleft.push_back(l);
+      TcGemmDesc r = gemmtc(bp.m, bp.n, bp.n, 1.0f, 0.0f);       // D = B P_R
+      r.a = b.operand(b.wf(bp.ws_Bh), b.wf(bp.ws_Bl), bp.m, bp.n, true, false, split);
+      r.b = b.operand(b.wf(fr.ws_Th), b.wf(fr.ws_Tl), bp.n, bp.n, false, true, split);  // P_R symmetric
+      r.c_ref = {1, bp.param, bp.r0, bp.c0};
+      tright.push_back(r);
+    } else {
+      float* tmp = b.wf(bp.ws_tmp);
+      GemmF32Desc l = gemm32(bp.m, bp.n, bp.m, 0, 0, mode_of(h->cfg), 1.0f, 0.0f);
+      l.A = Pm[2 * k]; l.lda = bp.m;
+      l.b_ref = {0, bp.param, bp.r0, bp.c0};
+      l.C = tmp; l.ldc = bp.n;
+      left.push_back(l);
+      GemmF32Desc r = gemm32(bp.m, bp.n, bp.n, 0, 0, mode_of(h->cfg), 1.0f, 0.0f);
+      r.A = tmp; r.lda = bp.n;
+      r.B = Pm[2 * k + 1]; r.ldb = bp.n;
+      r.c_ref = {1, bp.param, bp.r0, bp.c0};
+      right.push_back(r);
+    }
   }
   b.tag = SHAMPOO4_STAGE_APPLY_LEFT;
+  emit_gemmtc(b, h->prog_precond, tleft, split);
   emit_gemm32(b, h->prog_precond, left);
   b.tag = SHAMPOO4_STAGE_APPLY_RIGHT;
+  emit_gemmtc(b, h->prog_precond, tright, split);
   emit_gemm32(b, h->prog_precond, right);
 }
 
@@ -595,6 +1039,25 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
         break;
       case Kind::Scan:
         S4_TRY(launch_scan(static_cast<const ScanDesc*>(d), L.count, L.extent, tabs, np, gflags, st));
+        break;
+      case Kind::GemmTC:
+      case Kind::GemmTCSplit:
+      case Kind::GemmTCSplit64:
+        S4_TRY(launch_gemm_tc(static_cast<const TcGemmDesc*>(d), L.count, int(L.extent),
+                              L.kind == Kind::GemmTC ? 0 : 1, L.kind == Kind::GemmTCSplit64 ? 64 : 0, tabs, np,
+                              gflags, st));
+        break;
+      case Kind::PotrfF:
+        S4_TRY(launch_potrf_f(static_cast<const PotrfDescF*>(d), L.count, st));
+        break;
+      case Kind::TrsmF:
+        S4_TRY(launch_trsm_f(static_cast<const TrsmDescF*>(d), L.count, int(L.extent), st));
+        break;
+      case Kind::ShiftF:
+        S4_TRY(launch_shift_f(static_cast<const ShiftDescF*>(d), L.count, st));
+        break;
+      case Kind::Split:
+        S4_TRY(launch_split(static_cast<const SplitDesc*>(d), L.count, L.extent, st));
         break;
       case Kind::Shift:
         S4_TRY(launch_shift(static_cast<const ShiftDesc*>(d), L.count, st));
@@ -687,17 +1150,21 @@ extern "C" shampoo4_status shampoo4_init(const shampoo4_config* cfg, const shamp
   h->params.assign(params, params + nparams);
   shampoo4_status s = plan(h);
   if (s != SHAMPOO4_OK) { delete h; return s; }
-  // Descriptor bytes: build the programs once against a null base to size
-  // the arena; bind rebuilds them with the real addresses.
-  Builder b{h, h->arena, nullptr, nullptr};
+  // Tensor-map and descriptor bytes: build the programs once against a null
+  // base (maps counted, not encoded) to size both regions; bind rebuilds
+  // them with the real addresses.
+  Builder b{h, h->arena, nullptr, nullptr, false};
   build_stats(b);
   build_refresh(b, h->prog_refresh_first, true);
   build_refresh(b, h->prog_refresh, false);
   build_precondition(b);
+  h->ws_nmaps = h->maps.size();
+  h->ws_desc = align_up(h->ws_maps + h->ws_nmaps * sizeof(CUtensorMap), kAlign);
   h->ws_desc_bytes = align_up(h->arena.size(), kAlign);
   h->ws_bytes = h->ws_desc + h->ws_desc_bytes;
   h->prog_stats.clear(); h->prog_refresh_first.clear(); h->prog_refresh.clear(); h->prog_precond.clear();
   h->arena.clear();
+  h->maps.clear();
   *out = h;
   return SHAMPOO4_OK;
 }
@@ -728,14 +1195,20 @@ extern "C" shampoo4_status shampoo4_bind(shampoo4_handle h, void* d_state, void*
   h->d_ws = static_cast<uint8_t*>(d_workspace);
   h->prog_stats.clear(); h->prog_refresh_first.clear(); h->prog_refresh.clear(); h->prog_precond.clear();
   h->arena.clear();
-  Builder b{h, h->arena, h->d_ws, h->d_state};
+  h->maps.clear();
+  Builder b{h, h->arena, h->d_ws, h->d_state, true};
   build_stats(b);
   build_refresh(b, h->prog_refresh_first, true);
   build_refresh(b, h->prog_refresh, false);
   build_precondition(b);
-  if (align_up(h->arena.size(), kAlign) != h->ws_desc_bytes) return SHAMPOO4_ERR_WORKSPACE;
+  if (b.err != SHAMPOO4_OK) return b.err;
+  if (align_up(h->arena.size(), kAlign) != h->ws_desc_bytes || h->maps.size() != h->ws_nmaps)
+    return SHAMPOO4_ERR_WORKSPACE;
+  S4_CUDA(cudaMemsetAsync(h->d_ws, 0, h->ws_maps, st));
+  if (!h->maps.empty())
+    S4_CUDA(cudaMemcpyAsync(h->d_ws + h->ws_maps, h->maps.data(), h->maps.size() * sizeof(CUtensorMap),
+                            cudaMemcpyHostToDevice, st));
   S4_CUDA(cudaMemcpyAsync(h->d_ws + h->ws_desc, h->arena.data(), h->arena.size(), cudaMemcpyHostToDevice, st));
-  S4_CUDA(cudaMemsetAsync(h->d_ws, 0, h->ws_desc, st));
   if (reset) {
     S4_CUDA(cudaMemsetAsync(h->d_state, 0, h->state_bytes, st));
     h->has_basis = false;
@@ -768,6 +1241,8 @@ extern "C" shampoo4_status shampoo4_refresh_roots(shampoo4_handle h, shampoo4_st
   if (!h->bound) return SHAMPOO4_ERR_NOT_READY;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_fail, 0, 4 * h->factors.size(), st));
+  S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_tcbad, 0, 4 * h->factors.size(), st));
+  S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_tcgood, 1, 4 * h->factors.size(), st));
   const bool first = !h->has_basis;
   S4_TRY(run(h, first ? h->prog_refresh_first : h->prog_refresh, st));
   h->last_refresh_first = first;

@@ -38,12 +38,15 @@ struct TcGemmDesc {
   OperandRef c_ref;
 };
 
+// Tile width N of the kernel instance: 256 (TF32), 128 (split), or 64
+// (split, narrow products).
 int tc_block_n(int split);
-shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split,
+shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split, int bn,
                                const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st);
 // Encode a 2-D fp32 tensor map (rows x cols, leading dimension ld elements),
-// 128-byte swizzle, box 32 (contiguous) x box_rows, zero fill out of bounds.
+// box 32 (contiguous) x box_rows, zero fill out of bounds; 128-byte swizzle,
+// with 32-byte atoms for an operand read MN-major.
 shampoo4_status tc_encode_map(CUtensorMap* out, const float* base, int64_t rows, int64_t cols, int64_t ld,
-                              int box_rows);
+                              int box_rows, int mn_major);
 
 }  // namespace s4

@@ -97,6 +97,10 @@ typedef struct shampoo4_ctx* shampoo4_handle;
 #define SHAMPOO4_FLAG_TIMEOUT          0x8u  /* a kernel's bounded wait on one
                                                of its own pipeline barriers
                                                expired; its output is invalid */
+#define SHAMPOO4_FLAG_QR_FALLBACK      0x10u /* informational: the fp32 QR of
+                                               some factor's subspace step was
+                                               too ill-conditioned and was
+                                               redone in fp64                */
 
 /* Plan a set of parameters.  Host only: validates the config and shapes,
  * partitions every weight into greedy tiles of at most max_block (ragged

@@ -67,7 +67,12 @@ def test_refresh_and_precondition(which, precision):
         orc.refresh_roots()
         sh.refresh_roots()
         torch.cuda.synchronize()
-        assert sh.status_flags() == 0
+        flags = sh.status_flags()
+        # well-conditioned statistics stay on the fp32 tensor-core QR; the
+        # rank-deficient ones (lambda_max / eps ~ 1e7 and more) may need the
+        # fp64 redo, which is reported but is not an error
+        allowed = 0x10 if which == "ragged" else 0
+        assert flags & ~allowed == 0, flags
         for f in range(sh.nfactors):
             d = orc.factors[f].d
             Qg = sh.debug_q(f).cpu().numpy().astype(np.float64)
@@ -81,8 +86,15 @@ def test_refresh_and_precondition(which, precision):
             # (iii) eigenvalues and (iv) basis-invariant root against the oracle
             Qo, lo = orc.factors[f].q_last, orc.factors[f].lam.astype(np.float64)
             lg = g.lam.astype(np.float64)
+            # lambda_i = q_i^T S q_i comes from an fp32-accurate product S Q
+            # (3xTF32: each product carries a relative error of about
+            # u = 2^-21), so its error is absolute, about u * lambda_max, on
+            # top of the stage tolerance: the excess over that bound is
+            # reported relative to lambda_i.
             big = lo > 1e3 * eps
-            lam_err = np.max(np.abs(lg[big] - lo[big]) / lo[big]) if big.any() else 0.0
+            slack = 16 * 2.0 ** -21 * lo.max()
+            excess = np.maximum(np.abs(lg - lo) - slack, 0.0)
+            lam_err = np.max(excess[big] / lo[big]) if big.any() else 0.0
             # The basis-invariant root is only determined to the arithmetic's
             # resolution: the subspace product carries an absolute error of
             # about u32 * lambda_max per column, so eigen-directions are pinned
