@@ -142,91 +142,96 @@ __device__ __forceinline__ double ld_any(const void* p, bool f64, int64_t idx) {
   return f64 ? static_cast<const double*>(p)[idx] : double(static_cast<const float*>(p)[idx]);
 }
 
+// Work items (tile, problem) looped over by a fixed grid, so that a launch
+// whose problems are all skipped (the fp64 fallback of the QR) costs only
+// its flag reads.
 __global__ void __launch_bounds__(kF64Threads)
-k_gemm_f64(const GemmF64Desc* __restrict__ descs) {
-  const GemmF64Desc& g = descs[blockIdx.y];
-  if (g.M <= 0 || g.N <= 0) return;
-  const int tiles_m = (g.M + kF64Tile - 1) / kF64Tile;
-  const int tiles_n = (g.N + kF64Tile - 1) / kF64Tile;
-  if (int(blockIdx.x) >= tiles_m * tiles_n) return;
-  const int tm = blockIdx.x / tiles_n, tn = blockIdx.x % tiles_n;
-  if (g.lower_only && tn > tm) return;
-  if (g.skip && *g.skip) return;
-  const int m0 = tm * kF64Tile, n0 = tn * kF64Tile;
+k_gemm_f64(const GemmF64Desc* __restrict__ descs, int count, int max_tiles) {
   __shared__ double As[kF64BK][kF64Tile + 1];
   __shared__ double Bs[kF64BK][kF64Tile + 1];
   const int tid = threadIdx.x;
   const int tx = tid % 16, ty = tid / 16;
-  double acc[4][4];
+  for (int w = blockIdx.x; w < count * max_tiles; w += gridDim.x) {
+    const GemmF64Desc& g = descs[w / max_tiles];
+    const int t = w % max_tiles;
+    if (g.M <= 0 || g.N <= 0) continue;
+    const int tiles_m = (g.M + kF64Tile - 1) / kF64Tile;
+    const int tiles_n = (g.N + kF64Tile - 1) / kF64Tile;
+    if (t >= tiles_m * tiles_n) continue;
+    const int tm = t / tiles_n, tn = t % tiles_n;
+    if (g.lower_only && tn > tm) continue;
+    if (g.skip && *g.skip) continue;
+    const int m0 = tm * kF64Tile, n0 = tn * kF64Tile;
+    double acc[4][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-  const bool af = g.a_f64, bf = g.b_f64;
-  for (int k0 = 0; k0 < g.K; k0 += kF64BK) {
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    const bool af = g.a_f64, bf = g.b_f64;
+    for (int k0 = 0; k0 < g.K; k0 += kF64BK) {
+      __syncthreads();
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      int e = tid + r * kF64Threads;          // 0..1023 over a 64 x 16 tile
-      int i, kk;
-      if (!g.ta) { i = e / kF64BK; kk = e % kF64BK; }
-      else       { kk = e / kF64Tile; i = e % kF64Tile; }
-      int gi = m0 + i, gk = k0 + kk;
-      double v = 0.0;
-      if (gi < g.M && gk < g.K)
-        v = g.ta ? ld_any(g.A, af, int64_t(gk) * g.lda + gi) : ld_any(g.A, af, int64_t(gi) * g.lda + gk);
-      As[kk][i] = v;
+      for (int r = 0; r < 4; ++r) {
+        int e = tid + r * kF64Threads;          // 0..1023 over a 64 x 16 tile
+        int i, kk;
+        if (!g.ta) { i = e / kF64BK; kk = e % kF64BK; }
+        else       { kk = e / kF64Tile; i = e % kF64Tile; }
+        int gi = m0 + i, gk = k0 + kk;
+        double v = 0.0;
+        if (gi < g.M && gk < g.K)
+          v = g.ta ? ld_any(g.A, af, int64_t(gk) * g.lda + gi) : ld_any(g.A, af, int64_t(gi) * g.lda + gk);
+        As[kk][i] = v;
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        int e = tid + r * kF64Threads;
+        int j, kk;
+        if (!g.tb) { kk = e / kF64Tile; j = e % kF64Tile; }
+        else       { j = e / kF64BK; kk = e % kF64BK; }
+        int gj = n0 + j, gk = k0 + kk;
+        double v = 0.0;
+        if (gj < g.N && gk < g.K)
+          v = g.tb ? ld_any(g.B, bf, int64_t(gj) * g.ldb + gk) : ld_any(g.B, bf, int64_t(gk) * g.ldb + gj);
+        Bs[kk][j] = v;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int kk = 0; kk < kF64BK; ++kk) {
+        double a[4], b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx + 16 * j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+      }
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      int e = tid + r * kF64Threads;
-      int j, kk;
-      if (!g.tb) { kk = e / kF64Tile; j = e % kF64Tile; }
-      else       { j = e / kF64BK; kk = e % kF64BK; }
-      int gj = n0 + j, gk = k0 + kk;
-      double v = 0.0;
-      if (gj < g.N && gk < g.K)
-        v = g.tb ? ld_any(g.B, bf, int64_t(gj) * g.ldb + gk) : ld_any(g.B, bf, int64_t(gk) * g.ldb + gj);
-      Bs[kk][j] = v;
-    }
-    __syncthreads();
+    for (int i = 0; i < 4; ++i) {
+      int gi = m0 + ty + 16 * i;
+      if (gi >= g.M) continue;
 #pragma unroll
-    for (int kk = 0; kk < kF64BK; ++kk) {
-      double a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx + 16 * j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    int gi = m0 + ty + 16 * i;
-    if (gi >= g.M) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      int gj = n0 + tx + 16 * j;
-      if (gj >= g.N) continue;
-      double v = g.alpha * acc[i][j];
-      if (g.beta != 0.0) v = fma(g.beta, ld_any(g.Cin, g.cin_f64, int64_t(gi) * g.ldcin + gj), v);
-      int64_t o = int64_t(gi) * g.ldc + gj;
-      if (g.c_f64) static_cast<double*>(g.C)[o] = v;
-      else static_cast<float*>(g.C)[o] = float(v);
+      for (int j = 0; j < 4; ++j) {
+        int gj = n0 + tx + 16 * j;
+        if (gj >= g.N) continue;
+        double v = g.alpha * acc[i][j];
+        if (g.beta != 0.0) v = fma(g.beta, ld_any(g.Cin, g.cin_f64, int64_t(gi) * g.ldcin + gj), v);
+        int64_t o = int64_t(gi) * g.ldc + gj;
+        if (g.c_f64) static_cast<double*>(g.C)[o] = v;
+        else static_cast<float*>(g.C)[o] = float(v);
+      }
     }
   }
 }
 
 shampoo4_status launch_gemm_f64(const GemmF64Desc* d_desc, int count, int max_tiles, cudaStream_t st) {
-  for (int base = 0; base < count; base += 65535) {
-    int c = count - base < 65535 ? count - base : 65535;
-    if (max_tiles <= 0) break;
-    k_gemm_f64<<<dim3(unsigned(max_tiles), unsigned(c)), kF64Threads, 0, st>>>(d_desc + base);
-    S4_CUDA(cudaGetLastError());
-  }
+  if (count <= 0 || max_tiles <= 0) return SHAMPOO4_OK;
+  const int64_t items = int64_t(count) * max_tiles;
+  const unsigned ctas = unsigned(items < 148 * 8 ? items : 148 * 8);
+  k_gemm_f64<<<ctas, kF64Threads, 0, st>>>(d_desc, count, max_tiles);
+  S4_CUDA(cudaGetLastError());
   return SHAMPOO4_OK;
 }
 

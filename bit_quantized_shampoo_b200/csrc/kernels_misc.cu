@@ -57,44 +57,48 @@ shampoo4_status launch_potrf(const PotrfDesc* d_desc, int count, cudaStream_t st
 
 // ---- X[r, 0:jb] <- X[r, 0:jb] L^-T, one warp per row --------------------
 constexpr int kTrsmRowsPerCta = 64;
-__global__ void __launch_bounds__(256) k_trsm(const TrsmDesc* __restrict__ descs) {
-  const TrsmDesc& g = descs[blockIdx.y];
-  const int jb = g.jb;
-  const int row0 = blockIdx.x * kTrsmRowsPerCta;
-  if (jb <= 0 || row0 >= g.rows || (g.skip && *g.skip)) return;
+constexpr unsigned kWorkCtas = 148 * 8;     // grid of the work-item loops
+
+// Work items (row chunk, problem), looped over by a fixed grid so that a
+// launch whose problems are all skipped costs only its flag reads.
+__global__ void __launch_bounds__(256) k_trsm(const TrsmDesc* __restrict__ descs, int count, int chunks) {
   __shared__ double L[kPanel][kPanel + 1];
-  for (int e = threadIdx.x; e < jb * jb; e += blockDim.x) {
-    int r = e / jb, c = e % jb;
-    L[r][c] = (c <= r) ? g.L[int64_t(r) * g.ldl + c] : 0.0;
-  }
-  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int row_end = min(g.rows, row0 + kTrsmRowsPerCta);
-  for (int r = row0 + warp; r < row_end; r += 8) {
-    double* x = g.X + int64_t(r) * g.ldx;
-    double x0 = lane < jb ? x[lane] : 0.0;
-    double x1 = lane + 32 < jb ? x[lane + 32] : 0.0;
-    for (int c = 0; c < jb; ++c) {
-      // x_c is final once columns < c are applied; divide by L[c][c]
-      double xc = __shfl_sync(0xffffffffu, c < 32 ? x0 : x1, c & 31);
-      xc /= L[c][c];
-      if (c < 32) { if (lane == c) x0 = xc; } else { if (lane + 32 == c) x1 = xc; }
-      if (lane > c && lane < jb) x0 -= xc * L[lane][c];
-      if (lane + 32 > c && lane + 32 < jb) x1 -= xc * L[lane + 32][c];
+  for (int w = blockIdx.x; w < count * chunks; w += gridDim.x) {
+    const TrsmDesc& g = descs[w / chunks];
+    const int jb = g.jb;
+    const int row0 = (w % chunks) * kTrsmRowsPerCta;
+    if (jb <= 0 || row0 >= g.rows || (g.skip && *g.skip)) continue;
+    __syncthreads();                           // previous item done with L
+    for (int e = threadIdx.x; e < jb * jb; e += blockDim.x) {
+      int r = e / jb, c = e % jb;
+      L[r][c] = (c <= r) ? g.L[int64_t(r) * g.ldl + c] : 0.0;
     }
-    if (lane < jb) x[lane] = x0;
-    if (lane + 32 < jb) x[lane + 32] = x1;
+    __syncthreads();
+    const int row_end = min(g.rows, row0 + kTrsmRowsPerCta);
+    for (int r = row0 + warp; r < row_end; r += 8) {
+      double* x = g.X + int64_t(r) * g.ldx;
+      double x0 = lane < jb ? x[lane] : 0.0;
+      double x1 = lane + 32 < jb ? x[lane + 32] : 0.0;
+      for (int c = 0; c < jb; ++c) {
+        double xc = __shfl_sync(0xffffffffu, c < 32 ? x0 : x1, c & 31);
+        xc /= L[c][c];
+        if (c < 32) { if (lane == c) x0 = xc; } else { if (lane + 32 == c) x1 = xc; }
+        if (lane > c && lane < jb) x0 -= xc * L[lane][c];
+        if (lane + 32 > c && lane + 32 < jb) x1 -= xc * L[lane + 32][c];
+      }
+      if (lane < jb) x[lane] = x0;
+      if (lane + 32 < jb) x[lane + 32] = x1;
+    }
   }
 }
 
 shampoo4_status launch_trsm(const TrsmDesc* d_desc, int count, int max_rows, cudaStream_t st) {
   if (count <= 0 || max_rows <= 0) return SHAMPOO4_OK;
-  for (int base = 0; base < count; base += 65535) {
-    int c = count - base < 65535 ? count - base : 65535;
-    dim3 grid((max_rows + kTrsmRowsPerCta - 1) / kTrsmRowsPerCta, c);
-    k_trsm<<<grid, 256, 0, st>>>(d_desc + base);
-    S4_CUDA(cudaGetLastError());
-  }
+  const int chunks = (max_rows + kTrsmRowsPerCta - 1) / kTrsmRowsPerCta;
+  const int64_t items = int64_t(count) * chunks;
+  k_trsm<<<unsigned(items < kWorkCtas ? items : kWorkCtas), 256, 0, st>>>(d_desc, count, chunks);
+  S4_CUDA(cudaGetLastError());
   return SHAMPOO4_OK;
 }
 
@@ -104,19 +108,14 @@ __global__ void __launch_bounds__(256) k_basis(const BasisDesc* __restrict__ des
   __shared__ float level[16];
   if (threadIdx.x < 16) level[threadIdx.x] = level_f32(threadIdx.x);
   __syncthreads();
-  const int64_t n = int64_t(g.d) * g.d;
-  const int64_t e0 = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  const int n = g.d * g.d;                       // d <= 1024: fits in 32 bits
+  const int e0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
   if (e0 >= n) return;
+  int row = e0 / g.d, col = e0 - row * g.d;
   float v[8];
-  if (g.identity) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      int64_t i = e0 + e;
-      v[e] = (i / g.d == i % g.d) ? 1.0f : 0.0f;
-    }
-  } else {
+  if (!g.identity) {
     uint32_t packed = 0;
-    const int64_t nbytes = (n + 1) >> 1;
+    const int nbytes = (n + 1) >> 1;
 #pragma unroll
     for (int k = 0; k < 4; ++k)
       if ((e0 >> 1) + k < nbytes) packed |= uint32_t(g.codes[(e0 >> 1) + k]) << (8 * k);
@@ -124,11 +123,13 @@ __global__ void __launch_bounds__(256) k_basis(const BasisDesc* __restrict__ des
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    const int64_t i = e0 + e;
+    const int i = e0 + e;
     if (i >= n) break;
-    if (g.U) g.U[i] = v[e];
-    put_split(v[e], g.Uh, g.Ul, i);
-    if (g.Vh) put_split(v[e] * g.mu[i % g.d], g.Vh, g.Vl, i);
+    const float x = g.identity ? (row == col ? 1.0f : 0.0f) : v[e];
+    if (g.U) g.U[i] = x;
+    put_split(x, g.Uh, g.Ul, i);
+    if (g.Vh) put_split(x * g.mu[col], g.Vh, g.Vl, i);
+    if (++col == g.d) { col = 0; ++row; }
   }
 }
 
@@ -189,7 +190,6 @@ __global__ void __launch_bounds__(256)
 k_scan(const ScanDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, int nparams,
        uint32_t* __restrict__ gflags) {
   const ScanDesc& g = descs[blockIdx.y];
-  const int64_t n = int64_t(g.rows) * g.cols;
   int64_t ld = g.ld;
   const float* X = g.X;
   if (g.ref.tab >= 0) {
@@ -198,12 +198,14 @@ k_scan(const ScanDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, in
     X = e.ptr + g.ref.r0 * e.ld + g.ref.c0;
   }
   bool bad = false;
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
-       e += int64_t(gridDim.x) * blockDim.x) {
-    int64_t r = e / g.cols, c = e % g.cols;
-    float v = X[r * ld + c];
-    bad |= !isfinite(v);
-    put_split(v, g.oh, g.ol, e);
+  for (int r = blockIdx.x; r < g.rows; r += gridDim.x) {      // rows, coalesced columns
+    const float* xr = X + int64_t(r) * ld;
+    const int64_t o = int64_t(r) * g.cols;
+    for (int c = threadIdx.x; c < g.cols; c += blockDim.x) {
+      const float v = xr[c];
+      bad |= !isfinite(v);
+      put_split(v, g.oh, g.ol, o + c);
+    }
   }
   if (__syncthreads_or(bad) && threadIdx.x == 0) {
     *g.flag = 1u;
@@ -211,20 +213,19 @@ k_scan(const ScanDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, in
   }
 }
 
-shampoo4_status launch_scan(const ScanDesc* d_desc, int count, int64_t max_elems,
+shampoo4_status launch_scan(const ScanDesc* d_desc, int count, int64_t max_rows,
                             const PtrEntry* tabs, int nparams, uint32_t* flags, cudaStream_t st) {
-  if (count <= 0 || max_elems <= 0) return SHAMPOO4_OK;
-  int64_t ctas = (max_elems + 256 * 8 - 1) / (256 * 8);
-  if (ctas > 1024) ctas = 1024;
+  if (count <= 0 || max_rows <= 0) return SHAMPOO4_OK;
+  const unsigned ctas = unsigned(max_rows < 128 ? max_rows : 128);
   for (int base = 0; base < count; base += 65535) {
     int c = count - base < 65535 ? count - base : 65535;
-    k_scan<<<dim3(unsigned(ctas), c), 256, 0, st>>>(d_desc + base, tabs, nparams, flags);
+    k_scan<<<dim3(ctas, c), 256, 0, st>>>(d_desc + base, tabs, nparams, flags);
     S4_CUDA(cudaGetLastError());
   }
   return SHAMPOO4_OK;
 }
 
-// ---- shifted Gram diagonal ------------------------------------------------
+// ---- shifted Gram diagonal (fp64) -----------------------------------------
 __global__ void __launch_bounds__(256) k_shift(const ShiftDesc* __restrict__ descs) {
   const ShiftDesc& g = descs[blockIdx.x];
   if (g.skip && *g.skip) return;
@@ -250,11 +251,17 @@ shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st
 }
 
 // ---- fp32-storage Cholesky panel (fp64 inside) ------------------------------
+// Factor the jb x jb diagonal block, then (if requested) invert the factor:
+// thread c forms column c of L^-1 by forward substitution.
+constexpr int kPotrfFSmem = 2 * kPanel * (kPanel + 1) * 8;
+
 __global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ descs) {
   const PotrfDescF& g = descs[blockIdx.x];
   const int jb = g.jb;
   if (jb <= 0 || *g.fail) return;
-  __shared__ double L[kPanel][kPanel + 1];
+  extern __shared__ double sm_potrf[];
+  double (*L)[kPanel + 1] = reinterpret_cast<double (*)[kPanel + 1]>(sm_potrf);
+  double (*Li)[kPanel + 1] = reinterpret_cast<double (*)[kPanel + 1]>(sm_potrf + kPanel * (kPanel + 1));
   __shared__ int bad;
   for (int e = threadIdx.x; e < jb * jb; e += blockDim.x) {
     int r = e / jb, c = e % jb;
@@ -287,6 +294,25 @@ __global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ 
       put_split(v, g.oh, g.ol, int64_t(r) * g.ld + c);
     }
   }
+  if (g.ih) {
+    if (threadIdx.x < kPanel) {
+      const int c = threadIdx.x;
+      for (int r = 0; r < kPanel; ++r) Li[r][c] = 0.0;
+      if (c < jb) {
+        Li[c][c] = 1.0 / L[c][c];
+        for (int r = c + 1; r < jb; ++r) {
+          double acc = 0.0;
+          for (int k = c; k < r; ++k) acc = fma(L[r][k], Li[k][c], acc);
+          Li[r][c] = -acc / L[r][r];
+        }
+      }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < kPanel * kPanel; e += blockDim.x) {
+      const int r = e / kPanel, c = e % kPanel;
+      put_split(float(Li[r][c]), g.ih, g.il, e);
+    }
+  }
   if (threadIdx.x == 0 && bad) {
     *g.fail = 1u;
     if (g.clear) {                        // fp32 attempt: fall back to fp64
@@ -300,73 +326,13 @@ __global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ 
 
 shampoo4_status launch_potrf_f(const PotrfDescF* d_desc, int count, cudaStream_t st) {
   if (count <= 0) return SHAMPOO4_OK;
-  k_potrf_f<<<count, 256, 0, st>>>(d_desc);
+  static bool configured = false;
+  if (!configured) {
+    S4_CUDA(cudaFuncSetAttribute(k_potrf_f, cudaFuncAttributeMaxDynamicSharedMemorySize, kPotrfFSmem));
+    configured = true;
+  }
+  k_potrf_f<<<count, 256, kPotrfFSmem, st>>>(d_desc);
   S4_CUDA(cudaGetLastError());
-  return SHAMPOO4_OK;
-}
-
-__global__ void __launch_bounds__(256) k_trsm_f(const TrsmDescF* __restrict__ descs) {
-  const TrsmDescF& g = descs[blockIdx.y];
-  const int jb = g.jb;
-  const int row0 = blockIdx.x * kTrsmRowsPerCta;
-  if (jb <= 0 || row0 >= g.rows) return;
-  if (g.skip && *g.skip) return;
-  __shared__ double L[kPanel][kPanel + 1];
-  __shared__ double rdiag[kPanel];
-  for (int e = threadIdx.x; e < jb * jb; e += blockDim.x) {
-    int r = e / jb, c = e % jb;
-    L[r][c] = (c <= r) ? double(g.L[int64_t(r) * g.ldl + c]) : 0.0;
-  }
-  __syncthreads();
-  if (threadIdx.x < jb) rdiag[threadIdx.x] = 1.0 / L[threadIdx.x][threadIdx.x];
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int row_end = min(g.rows, row0 + kTrsmRowsPerCta);
-  const float* in = g.Xin ? g.Xin : g.X;
-  // two rows per warp at a time: their dependency chains interleave
-  for (int ra = row0 + 2 * warp; ra < row_end; ra += 16) {
-    const int rb = ra + 1;
-    const bool hb = rb < row_end;
-    const float* xa = in + int64_t(ra) * g.ldx;
-    const float* xb = in + int64_t(hb ? rb : ra) * g.ldx;
-    double a0 = lane < jb ? double(xa[lane]) : 0.0;
-    double a1 = lane + 32 < jb ? double(xa[lane + 32]) : 0.0;
-    double b0 = lane < jb ? double(xb[lane]) : 0.0;
-    double b1 = lane + 32 < jb ? double(xb[lane + 32]) : 0.0;
-    for (int c = 0; c < jb; ++c) {
-      const bool lo = c < 32;
-      double ac = __shfl_sync(0xffffffffu, lo ? a0 : a1, c & 31) * rdiag[c];
-      double bc = __shfl_sync(0xffffffffu, lo ? b0 : b1, c & 31) * rdiag[c];
-      if (lo) { if (lane == c) { a0 = ac; b0 = bc; } } else { if (lane + 32 == c) { a1 = ac; b1 = bc; } }
-      if (lane > c && lane < jb) { const double l = L[lane][c]; a0 -= ac * l; b0 -= bc * l; }
-      if (lane + 32 > c && lane + 32 < jb) { const double l = L[lane + 32][c]; a1 -= ac * l; b1 -= bc * l; }
-    }
-    for (int k = 0; k < 2; ++k) {
-      const int r = k == 0 ? ra : rb;
-      if (k == 1 && !hb) break;
-      const float f0 = float(k == 0 ? a0 : b0), f1 = float(k == 0 ? a1 : b1);
-      float* xo = g.X + int64_t(r) * g.ldx;
-      if (lane < jb) xo[lane] = f0;
-      if (lane + 32 < jb) xo[lane + 32] = f1;
-      if (g.oh) {
-        const int64_t o = int64_t(r) * g.ldo;
-        if (lane < jb) put_split(f0, g.oh, g.ol, o + lane);
-        else if (g.zero_pad) put_split(0.0f, g.oh, g.ol, o + lane);
-        if (lane + 32 < jb) put_split(f1, g.oh, g.ol, o + lane + 32);
-        else if (g.zero_pad) put_split(0.0f, g.oh, g.ol, o + lane + 32);
-      }
-    }
-  }
-}
-
-shampoo4_status launch_trsm_f(const TrsmDescF* d_desc, int count, int max_rows, cudaStream_t st) {
-  if (count <= 0 || max_rows <= 0) return SHAMPOO4_OK;
-  for (int base = 0; base < count; base += 65535) {
-    int c = count - base < 65535 ? count - base : 65535;
-    dim3 grid((max_rows + kTrsmRowsPerCta - 1) / kTrsmRowsPerCta, c);
-    k_trsm_f<<<grid, 256, 0, st>>>(d_desc + base);
-    S4_CUDA(cudaGetLastError());
-  }
   return SHAMPOO4_OK;
 }
 
@@ -413,26 +379,27 @@ shampoo4_status launch_split(const SplitDesc* d_desc, int count, int64_t max_ele
 }
 
 // ---- fp64 -> fp32 ----------------------------------------------------------
-__global__ void __launch_bounds__(256) k_convert(const ConvertDesc* __restrict__ descs) {
-  const ConvertDesc& g = descs[blockIdx.y];
-  if (g.skip && *g.skip) return;
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < g.n;
-       e += int64_t(gridDim.x) * blockDim.x) {
-    const float v = float(g.src[e]);
-    g.dst[e] = v;
-    put_split(v, g.dh, g.dl, e);
+constexpr int64_t kConvertChunk = 1 << 16;
+__global__ void __launch_bounds__(256) k_convert(const ConvertDesc* __restrict__ descs, int count, int chunks) {
+  for (int w = blockIdx.x; w < count * chunks; w += gridDim.x) {
+    const ConvertDesc& g = descs[w / chunks];
+    const int64_t lo = int64_t(w % chunks) * kConvertChunk;
+    if (lo >= g.n || (g.skip && *g.skip)) continue;
+    const int64_t hi = lo + kConvertChunk < g.n ? lo + kConvertChunk : g.n;
+    for (int64_t e = lo + threadIdx.x; e < hi; e += blockDim.x) {
+      const float v = float(g.src[e]);
+      g.dst[e] = v;
+      put_split(v, g.dh, g.dl, e);
+    }
   }
 }
 
 shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st) {
   if (count <= 0 || max_elems <= 0) return SHAMPOO4_OK;
-  int64_t ctas = (max_elems + 1023) / 1024;
-  if (ctas > 1024) ctas = 1024;
-  for (int base = 0; base < count; base += 65535) {
-    int c = count - base < 65535 ? count - base : 65535;
-    k_convert<<<dim3(unsigned(ctas), c), 256, 0, st>>>(d_desc + base);
-    S4_CUDA(cudaGetLastError());
-  }
+  const int chunks = int((max_elems + kConvertChunk - 1) / kConvertChunk);
+  const int64_t items = int64_t(count) * chunks;
+  k_convert<<<unsigned(items < kWorkCtas ? items : kWorkCtas), 256, 0, st>>>(d_desc, count, chunks);
+  S4_CUDA(cudaGetLastError());
   return SHAMPOO4_OK;
 }
 

@@ -144,19 +144,8 @@ struct PotrfDescF {
   uint32_t* gflags;
   uint32_t* clear;
   float* oh; float* ol;       // optional TF32 split of the factor (same ld)
-};
-
-// X[r, 0:jb] <- Xin[r, 0:jb] L^-T (Xin = X when null), fp64 inside; also
-// stores the TF32 split of the result into (oh, ol) with leading dimension
-// ldo, and, when zero_pad, zeros in columns jb..63 of the split.
-struct TrsmDescF {
-  const float* L; int64_t ldl;
-  const float* Xin;
-  float* X; int64_t ldx;
-  float* oh; float* ol; int64_t ldo;
-  int32_t jb, rows;
-  int32_t zero_pad; int32_t pad_;
-  const uint32_t* skip;
+  float* ih; float* il;       // optional TF32 split of the inverse factor,
+                              // 64 x 64 with leading dimension 64, zero-padded
 };
 
 // W <- W + coef * trace(W) * I (the shift of the first Cholesky-QR pass).
@@ -197,11 +186,10 @@ shampoo4_status launch_trsm(const TrsmDesc* d_desc, int count, int max_rows, cud
 shampoo4_status launch_basis(const BasisDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_rayleigh(const RayleighDesc* d_desc, int count, int max_d, cudaStream_t st);
 shampoo4_status launch_mu(const MuDesc* d_desc, int count, int max_d, float eps, cudaStream_t st);
-shampoo4_status launch_scan(const ScanDesc* d_desc, int count, int64_t max_elems,
+shampoo4_status launch_scan(const ScanDesc* d_desc, int count, int64_t max_rows,
                             const PtrEntry* tabs, int nparams, uint32_t* flags, cudaStream_t st);
 shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_potrf_f(const PotrfDescF* d_desc, int count, cudaStream_t st);
-shampoo4_status launch_trsm_f(const TrsmDescF* d_desc, int count, int max_rows, cudaStream_t st);
 shampoo4_status launch_shift_f(const ShiftDescF* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_split(const SplitDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);

@@ -29,7 +29,7 @@ using namespace s4;
 namespace {
 
 enum class Kind { GemmF32, GemmF64, Potrf, Trsm, Basis, Rayleigh, Mu, Scan, Convert, Pack, Shift, GemmTC, GemmTCSplit,
-                  GemmTCSplit64, PotrfF, TrsmF, ShiftF, Split };
+                  GemmTCSplit64, PotrfF, ShiftF, Split };
 
 struct Launch {
   Kind kind;
@@ -68,6 +68,7 @@ struct FactorPlan {
   size_t ws_W64, ws_Q64, ws_U, ws_T, ws_Y;
   size_t ws_Xm[2], ws_Xh[2], ws_Xl[2], ws_Th, ws_Tl, ws_Sh, ws_Sl, ws_W;
   size_t ws_Zm, ws_Zh, ws_Zl;
+  size_t ws_Ih, ws_Il, ws_Ph, ws_Pl;     // d x 64: inverse diagonal blocks, panel temporary
   size_t ws_q_first, ws_q_next;
 };
 
@@ -186,6 +187,13 @@ shampoo4_status plan(shampoo4_ctx* h) {
       f.ws_Zm = take(ws, 4 * dd);
       f.ws_Zh = take(ws, 4 * dd);
       f.ws_Zl = take(ws, 4 * dd);
+      // the inverse blocks are written 64 x 64 (zero-padded): rows up to a
+      // multiple of 64
+      const size_t dpad = align_up(size_t(f.d), kPanelW);
+      f.ws_Ih = take(ws, 4 * dpad * kPanelW);
+      f.ws_Il = take(ws, 4 * dpad * kPanelW);
+      f.ws_Ph = take(ws, 4 * size_t(f.d) * kPanelW);
+      f.ws_Pl = take(ws, 4 * size_t(f.d) * kPanelW);
       f.ws_W64 = take(ws, 8 * dd);            // fp64 fallback of the QR
       f.ws_Q64 = take(ws, 8 * dd);
     } else {
@@ -365,7 +373,7 @@ void build_grad_copy(Builder& b, std::vector<Launch>& prog, int tag, bool with_f
       s.ol = split ? b.wf(bp.ws_Gl) : nullptr;
     }
     scan.push_back(s);
-    max_elems = std::max<int64_t>(max_elems, int64_t(bp.m) * bp.n);
+    max_elems = std::max<int64_t>(max_elems, int64_t(bp.m));     // rows
     bytes += (4.0 + (bp.tc ? (split ? 8.0 : 4.0) : 0.0)) * bp.m * bp.n;
   }
   b.tag = tag;
@@ -544,6 +552,8 @@ constexpr float kTcShift = 1e-5f;
 
 struct Triplet { float* m; float* h; float* l; };
 
+int dpad_of(int d) { return (d + kPanelW - 1) / kPanelW * kPanelW; }
+
 void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Triplet>& X,
                      const std::vector<Triplet>& Q, bool shifted) {
   shampoo4_ctx* h = b.h;
@@ -552,6 +562,7 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
   for (auto& f : h->factors) if (f.tc) dmax = std::max(dmax, f.d);
   if (dmax == 0) return;
   {
+    // Gram W = X^T X (fp32 into W, its TF32 split into Th/Tl), optional shift
     std::vector<TcGemmDesc> g;
     std::vector<ShiftDescF> sd;
     for (size_t i = 0; i < nf; ++i) {
@@ -562,6 +573,7 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
       w.a = b.operand(X[i].h, X[i].l, d, d, true, true, true);
       w.b = b.operand(X[i].h, X[i].l, d, d, false, false, true);
       w.C = b.wf(f.ws_W); w.ldc = d;
+      w.Chi = b.wf(f.ws_Th); w.Clo = b.wf(f.ws_Tl); w.ldh = d;
       w.symmetric = 1;
       w.skip = b.tcbad(i);
       g.push_back(w);
@@ -572,17 +584,17 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
     b.emit(prog, Kind::ShiftF, sd, 0);
   }
   // Cholesky, left-looking by 64-wide panels.  For panel J:
-  //   W[j:, J] -= L[j:, <J] L[J, <J]^T      (tensor cores, one tall product)
-  //   L[J, J]   = chol(W[J, J])              (CUDA cores, fp64 inside)
-  //   L[j+jb:, J] = W[j+jb:, J] L[J, J]^-T   (CUDA cores, fp64 inside)
-  // The panels also leave the TF32 split of L in (Th, Tl), which the later
-  // updates and the triangular solve read.
+  //   W[j:, J] -= L[j:, <J] L[J, <J]^T      tensor cores (also refreshes the
+  //                                          TF32 split of that column block)
+  //   L[J, J] = chol(W[J, J]), L[J, J]^-1     CUDA cores, fp64 inside
+  //   L[j+jb:, J] = W[j+jb:, J] L[J, J]^-T    tensor cores
+  // (Th, Tl) ends up holding the TF32 split of L; (Ih, Il) rows J hold the
+  // split of L[J, J]^-1 for the solve.  A diagonal-shift pass may leave the
+  // split of W's diagonal in Th/Tl only until the panel overwrites it.
   for (int j = 0; j < dmax; j += kPanelW) {
-    std::vector<TcGemmDesc> up;
+    std::vector<TcGemmDesc> up, l21;
     std::vector<PotrfDescF> po;
-    std::vector<TrsmDescF> tr;
-    int max_rows = 0;
-    double fl_po = 0, fl_tr = 0;
+    double fl_po = 0;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
       if (!f.tc || j >= f.d) continue;
@@ -596,66 +608,66 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
         u.b = b.operand(Th, Tl, d, d, false, true, true, 64);
         u.a.row0 = u.b.row0 = j;
         u.C = W + int64_t(j) * d + j; u.ldc = d;
+        u.Chi = Th + int64_t(j) * d + j; u.Clo = Tl + int64_t(j) * d + j; u.ldh = d;
         u.Cin = u.C; u.ldcin = d;
         u.skip = b.tcbad(i);
         up.push_back(u);
       }
       po.push_back({W + int64_t(j) * d + j, d, jb, 0, b.tcbad(i), b.gflags(), b.tcgood(i),
-                    Th + int64_t(j) * d + j, Tl + int64_t(j) * d + j});
-      fl_po += double(jb) * jb * jb / 3.0;
+                    Th + int64_t(j) * d + j, Tl + int64_t(j) * d + j,
+                    b.wf(f.ws_Ih) + int64_t(j) * kPanelW, b.wf(f.ws_Il) + int64_t(j) * kPanelW});
+      fl_po += 2.0 * double(jb) * jb * jb / 3.0;
       if (rest <= 0) continue;
-      TrsmDescF t{};
-      t.L = W + int64_t(j) * d + j; t.ldl = d;
-      t.X = W + int64_t(j + jb) * d + j; t.ldx = d;
-      t.oh = Th + int64_t(j + jb) * d + j; t.ol = Tl + int64_t(j + jb) * d + j; t.ldo = d;
-      t.jb = jb; t.rows = rest; t.zero_pad = 0;
+      TcGemmDesc t = gemmtc(rest, jb, jb, 1.0f, 0.0f);     // L21 = W21 L11^-T (in the split, in place)
+      t.a = b.operand(Th, Tl, d, d, true, false, true);
+      t.a.row0 = j + jb; t.a.col0 = j;
+      t.b = b.operand(b.wf(f.ws_Ih), b.wf(f.ws_Il), dpad_of(d), kPanelW, false, true, true, 64);
+      t.b.row0 = j;
+      t.Chi = Th + int64_t(j + jb) * d + j; t.Clo = Tl + int64_t(j + jb) * d + j; t.ldh = d;
       t.skip = b.tcbad(i);
-      tr.push_back(t);
-      fl_tr += double(rest) * jb * jb;
-      max_rows = std::max(max_rows, rest);
+      l21.push_back(t);
     }
     b.tag = SHAMPOO4_STAGE_QR_SYRK;
     emit_gemmtc(b, prog, up, true, 64);
     b.tag = SHAMPOO4_STAGE_QR_POTRF;
     b.emit(prog, Kind::PotrfF, po, 0, fl_po);
     b.tag = SHAMPOO4_STAGE_QR_TRSM_PANEL;
-    b.emit(prog, Kind::TrsmF, tr, max_rows, fl_tr);
+    emit_gemmtc(b, prog, l21, true, 64);
   }
-  for (int j = 0; j < dmax; j += kPanelW) {          // solve Q L^T = X
-    std::vector<TcGemmDesc> up;
-    std::vector<TrsmDescF> tr;
-    int max_rows = 0;
-    double fl_tr = 0;
+  // Solve Q L^T = X by 64-wide column panels:
+  //   T = X[:, J] - Q[:, <J] L[J, <J]^T      tensor cores, TF32 split into P
+  //   Q[:, J] = T L[J, J]^-T                  tensor cores
+  for (int j = 0; j < dmax; j += kPanelW) {
+    std::vector<TcGemmDesc> up, qp;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
       if (!f.tc || j >= f.d) continue;
       const int d = f.d, jb = std::min(kPanelW, d - j);
-      float* W = b.wf(f.ws_W);
-      if (j > 0) {                                    // Q[:, J] = X[:, J] - Q[:, <J] L[J, <J]^T
+      TcGemmDesc q = gemmtc(d, jb, jb, 1.0f, 0.0f);
+      if (j > 0) {
         TcGemmDesc u = gemmtc(d, jb, j, -1.0f, 1.0f);
         u.a = b.operand(Q[i].h, Q[i].l, d, d, true, false, true);
         u.b = b.operand(b.wf(f.ws_Th), b.wf(f.ws_Tl), d, d, false, true, true, 64);
         u.b.row0 = j;
-        u.C = Q[i].m + j; u.ldc = d;
+        u.Chi = b.wf(f.ws_Ph); u.Clo = b.wf(f.ws_Pl); u.ldh = kPanelW;
         u.Cin = X[i].m + j; u.ldcin = d;
         u.skip = b.tcbad(i);
         up.push_back(u);
+        q.a = b.operand(b.wf(f.ws_Ph), b.wf(f.ws_Pl), d, kPanelW, true, false, true);
+      } else {
+        q.a = b.operand(X[i].h, X[i].l, d, d, true, false, true);   // T = X[:, 0:jb]
       }
-      TrsmDescF t{};
-      t.L = W + int64_t(j) * d + j; t.ldl = d;
-      t.Xin = j == 0 ? X[i].m : nullptr;
-      t.X = Q[i].m + j; t.ldx = d;
-      t.oh = Q[i].h + j; t.ol = Q[i].l + j; t.ldo = d;
-      t.jb = jb; t.rows = d; t.zero_pad = 0;
-      t.skip = b.tcbad(i);
-      tr.push_back(t);
-      fl_tr += double(d) * jb * jb;
-      max_rows = std::max(max_rows, d);
+      q.b = b.operand(b.wf(f.ws_Ih), b.wf(f.ws_Il), dpad_of(d), kPanelW, false, true, true, 64);
+      q.b.row0 = j;
+      q.C = Q[i].m + j; q.ldc = d;
+      q.Chi = Q[i].h + j; q.Clo = Q[i].l + j; q.ldh = d;
+      q.skip = b.tcbad(i);
+      qp.push_back(q);
     }
     b.tag = SHAMPOO4_STAGE_QR_SOLVE_UPDATE;
     emit_gemmtc(b, prog, up, true, 64);
     b.tag = SHAMPOO4_STAGE_QR_SOLVE_PANEL;
-    b.emit(prog, Kind::TrsmF, tr, max_rows, fl_tr);
+    emit_gemmtc(b, prog, qp, true, 64);
   }
 }
 
@@ -686,7 +698,7 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
       bytes += (f.tc ? 12.0 : 4.0) * double(f.d) * f.d;
     }
     b.tag = SHAMPOO4_STAGE_REFRESH_SCAN;
-    b.emit(prog, Kind::Scan, scan, emax, 0, bytes);
+    b.emit(prog, Kind::Scan, scan, dmax, 0, bytes);
   }
   // cur/oth: index of the current and the other triplet (tensor-core
   // factors) or buffer offsets (CUDA-core factors).
@@ -1049,9 +1061,6 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
         break;
       case Kind::PotrfF:
         S4_TRY(launch_potrf_f(static_cast<const PotrfDescF*>(d), L.count, st));
-        break;
-      case Kind::TrsmF:
-        S4_TRY(launch_trsm_f(static_cast<const TrsmDescF*>(d), L.count, int(L.extent), st));
         break;
       case Kind::ShiftF:
         S4_TRY(launch_shift_f(static_cast<const ShiftDescF*>(d), L.count, st));
