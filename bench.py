@@ -6,7 +6,13 @@ cut into 480 tiles of at most 1024 x 1024, 960 factors), with the gradients
 already resident in HBM.  Prints one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 1..5] [--precision tf32|fp32]
+                    [--workload 1..5] [--precision tf32|fp32] [--shapes RxC,...]
+
+--shapes replaces the workload's parameter list (its hyper-parameters and
+gradient distribution stay), e.g. ``--shapes 4096x4096`` for a small case
+with the same 1024 x 1024 factors as the default workload.  The timed steps
+run inside an NVTX push/pop range named "timed", so a profiler can select
+exactly their launches (ncu --nvtx --nvtx-include "timed/").
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own copy of
 the workload (tiles are independent; no data-path collective), so per-GPU
@@ -42,6 +48,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-codec", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--shapes", default=None, help="comma-separated RxC list replacing the workload's shapes")
     return ap.parse_args()
 
 
@@ -146,9 +153,16 @@ def stage_roofline(name, st, pk, pk_src, sustained=True):
     return r
 
 
-def workload_shapes(wid):
+def workload_shapes(wid, shapes=None):
+    import dataclasses
     from bit_quantized_shampoo_b200.workloads import WORKLOADS
-    return WORKLOADS[wid]
+    w = WORKLOADS[wid]
+    if shapes:
+        dims = tuple(tuple(int(v) for v in item.lower().split("x")) for item in shapes.split(","))
+        if not dims or any(len(d) != 2 or min(d) < 1 for d in dims):
+            raise SystemExit(f"--shapes: expected RxC[,RxC...], got {shapes!r}")
+        w = dataclasses.replace(w, shapes=dims, name=f"{w.name}; shapes replaced by {shapes}")
+    return w
 
 
 # ------------------------------------------------------------------ CPU oracle leg
@@ -194,7 +208,7 @@ def cpu_sample(w, nblocks_sample: int, seed_step: int = 1):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    w = workload_shapes(args.workload)
+    w = workload_shapes(args.workload, args.shapes)
     per_tile = []
     desc = threads = None
     for i in range(args.warmup + args.steps):
@@ -234,7 +248,7 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
 
-    w = workload_shapes(args.workload)
+    w = workload_shapes(args.workload, args.shapes)
     shapes = list(w.shapes)
     # inputs: seeded host draws, copied to pinned host memory and to HBM
     host_g = [torch.from_numpy(gradient(w, i, 1)).pin_memory() for i in range(len(shapes))]
@@ -259,10 +273,12 @@ def main():
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
+        torch.cuda.nvtx.range_push("timed")
         e0.record(stream)
         for _ in range(args.steps):
             step()
         e1.record(stream)
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -290,6 +306,8 @@ def main():
 
     pk, pk_src = peaks()
     clocks = clk.summary()
+    g_bytes = sum(r * c for r, c in shapes) * 4
+    stat_bytes = sum(int(b[3]) ** 2 + int(b[4]) ** 2 for b in (sh.block_info(k) for k in range(sh.nblocks))) * 4
     ranked = sorted(stages, key=lambda k: -stages[k]["ms"])
     dom = next(k for k in ranked if STAGE_BOUND.get(k, "latency") != "latency")
     roof = stage_roofline(dom, stages[dom], pk, pk_src)
@@ -301,7 +319,9 @@ def main():
             "vs_baseline": None, "dtype": args.precision if args.precision == "fp32" else "tf32",
             "data": "synthetic",
             "config": {"workload": w.name, "tiles": sh.nblocks, "factors": sh.nfactors,
-                       "steps_per_refresh": 1, "l2": "inputs larger than L2 (2 GB of G, 4 GB of statistics)"},
+                       "steps_per_refresh": 1,
+                       "l2": (f"inputs larger than L2 ({g_bytes / 1e9:.2f} GB of G, {stat_bytes / 1e9:.2f} GB "
+                              f"of fp32 statistics; L2 is 0.126 GB)")},
             "root_refreshes_per_s": value * sh.nfactors,
             "status_flags": status,
             "gpu_launches": launches,

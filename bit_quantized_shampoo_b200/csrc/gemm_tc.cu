@@ -124,6 +124,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 1-D bulk copies (TMA, no tensor map): global -> shared completing on an
+// mbarrier, shared -> global in per-thread bulk groups, and an L2 prefetch.
+// Addresses and sizes are multiples of 16 bytes.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 __device__ __forceinline__ float rn_tf32(float x) {
   uint32_t r;
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -137,6 +157,14 @@ struct TcCfg {
   static constexpr int kStage = (kATile + kBTile) * (SPLIT ? 2 : 1);
   static constexpr int kStages = STAGES;
   static constexpr int kSmem = kStage * kStages + 1024;         // + alignment slack
+  // Epilogue staging, carved out of the pipeline buffers once the main loop
+  // is over: per warp two Cin buffers and three output buffers of 32 rows,
+  // row pitch 36 floats (16-byte aligned rows, conflict-free 16-byte
+  // accesses by lane = row).
+  static constexpr int kPitch = 36;
+  static constexpr int kRowBuf = 32 * kPitch * 4;
+  static constexpr int kEpiWarp = 5 * kRowBuf;
+  static_assert(4 * kEpiWarp <= kStage * kStages, "epilogue staging fits the pipeline buffers");
   static constexpr int kTmemCols = BN;                          // 128 or 256: a power of two
 };
 
@@ -159,6 +187,52 @@ __device__ __forceinline__ uint64_t operand_desc(const TcOperand& op, uint32_t b
   return op.mn_major ? smem_desc(base + kk * 1024, 4096, 512, 1) : smem_desc(base + kk * 32, 16, 1024, 2);
 }
 
+// Output fields of one problem, held in registers by the epilogue warps.
+struct EpiArgs {
+  int M, N, symmetric, out_round;
+  float alpha, beta;
+  float* C; int64_t ldc;
+  float* Chi; float* Clo; int64_t ldh;
+  const float* Cin; int64_t ldcin;
+
+  __device__ __forceinline__ void load(const TcGemmDesc& g, const PtrEntry* tabs, int nparams) {
+    M = g.M; N = g.N; symmetric = g.symmetric; out_round = g.out_round;
+    alpha = g.alpha; beta = g.beta;
+    C = g.C; ldc = g.ldc;
+    if (g.c_ref.tab >= 0) {
+      const PtrEntry& t = tabs[g.c_ref.tab * nparams + g.c_ref.param];
+      ldc = t.ld;
+      C = const_cast<float*>(t.ptr) + g.c_ref.r0 * t.ld + g.c_ref.c0;
+    }
+    Chi = g.Chi; Clo = g.Clo; ldh = g.ldh;
+    Cin = g.Cin; ldcin = g.ldcin;
+  }
+  // One element to every requested output: C (optionally TF32-rounded) and
+  // the TF32 split (Chi, Clo).
+  __device__ __forceinline__ void put(int64_t r, int c, float v) const {
+    if (C) C[r * ldc + c] = out_round ? rn_tf32(v) : v;
+    if (Chi) {
+      const float h = rn_tf32(v);
+      Chi[r * ldh + c] = h;
+      if (Clo) Clo[r * ldh + c] = rn_tf32(v - h);
+    }
+  }
+  __device__ __forceinline__ void put4(int64_t r, int c, float a, float b, float x, float y) const {
+    if (C) {
+      const float4 o = out_round ? make_float4(rn_tf32(a), rn_tf32(b), rn_tf32(x), rn_tf32(y))
+                                 : make_float4(a, b, x, y);
+      *reinterpret_cast<float4*>(C + r * ldc + c) = o;
+    }
+    if (Chi) {
+      const float4 h = make_float4(rn_tf32(a), rn_tf32(b), rn_tf32(x), rn_tf32(y));
+      *reinterpret_cast<float4*>(Chi + r * ldh + c) = h;
+      if (Clo)
+        *reinterpret_cast<float4*>(Clo + r * ldh + c) =
+            make_float4(rn_tf32(a - h.x), rn_tf32(b - h.y), rn_tf32(x - h.z), rn_tf32(y - h.w));
+    }
+  }
+};
+
 template <int BN, bool SPLIT, int STAGES>
 __global__ void __launch_bounds__(192, STAGES <= 2 ? 2 : 1)
 k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, int nparams,
@@ -176,6 +250,7 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t full_bar[Cfg::kStages], empty_bar[Cfg::kStages], done_bar;
+  __shared__ uint64_t cin_bar[4][2];                      // epilogue Cin buffers, per warp
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -186,6 +261,10 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&done_bar, 1);
+    for (int w = 0; w < 4; ++w) {
+      mbar_init(&cin_bar[w][0], 1);
+      mbar_init(&cin_bar[w][1], 1);
+    }
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -203,11 +282,22 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
 
   if (warp == 0) {
     if (lane == 0) {                                        // ---- TMA producer
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(g.a.hi)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(g.b.hi)) : "memory");
+      // Register copies: after every asm statement with a "memory" clobber a
+      // field read through `g` would be fetched from global memory again,
+      // several hundred cycles on the path of each issue.
+      const TcOperand ga = g.a, gb = g.b;
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(ga.hi)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(gb.hi)) : "memory");
+      // Bring the tile of Cin into L2 while the main loop runs.
+      if (g.beta != 0.0f && ((reinterpret_cast<uintptr_t>(g.Cin) | uintptr_t(g.ldcin * 4)) & 15) == 0 &&
+          (g.N & 3) == 0) {
+        const uint32_t bytes = uint32_t(min(BN, g.N - n0)) * 4u;
+        const int rows = min(kBM, g.M - m0);
+        for (int r = 0; r < rows; ++r) bulk_prefetch_l2(g.Cin + int64_t(m0 + r) * g.ldcin + n0, bytes);
+      }
       if (SPLIT) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(g.a.lo)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(g.b.lo)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(ga.lo)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(gb.lo)) : "memory");
       }
       int issued = 0;
       for (int kb = 0; kb < kblocks; ++kb) {
@@ -221,11 +311,11 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
         const uint32_t st = smem_u32(smem + s * Cfg::kStage);
         mbar_expect_tx(&full_bar[s], Cfg::kStage);
         const int k0 = kb * kBK;
-        load_operand(g.a.hi, g.a, kBM, m0, k0, st, &full_bar[s]);
-        load_operand(g.b.hi, g.b, BN, n0, k0, st + Cfg::kATile, &full_bar[s]);
+        load_operand(ga.hi, ga, kBM, m0, k0, st, &full_bar[s]);
+        load_operand(gb.hi, gb, BN, n0, k0, st + Cfg::kATile, &full_bar[s]);
         if (SPLIT) {
-          load_operand(g.a.lo, g.a, kBM, m0, k0, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
-          load_operand(g.b.lo, g.b, BN, n0, k0, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+          load_operand(ga.lo, ga, kBM, m0, k0, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+          load_operand(gb.lo, gb, BN, n0, k0, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
         }
         issued = kb + 1;
       }
@@ -236,7 +326,8 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
     }
   } else if (warp == 1) {
     if (lane == 0) {                                        // ---- MMA issuer
-      const uint32_t idesc = idesc_tf32(kBM, BN, g.a.mn_major, g.b.mn_major);
+      const TcOperand ga = g.a, gb = g.b;                   // registers, as in the producer
+      const uint32_t idesc = idesc_tf32(kBM, BN, ga.mn_major, gb.mn_major);
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % Cfg::kStages;
         if (!mbar_wait(&full_bar[s], (kb / Cfg::kStages) & 1)) {
@@ -252,10 +343,10 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
 #pragma unroll
         for (int kk = 0; kk < kBK / 8; ++kk) {
           const uint32_t acc = (kb | kk) != 0;
-          mma_tf32(tmem, operand_desc(g.a, a_hi, kk), operand_desc(g.b, b_hi, kk), idesc, acc);
+          mma_tf32(tmem, operand_desc(ga, a_hi, kk), operand_desc(gb, b_hi, kk), idesc, acc);
           if (SPLIT) {
-            mma_tf32(tmem, operand_desc(g.a, a_hi, kk), operand_desc(g.b, b_lo, kk), idesc, 1);
-            mma_tf32(tmem, operand_desc(g.a, a_lo, kk), operand_desc(g.b, b_hi, kk), idesc, 1);
+            mma_tf32(tmem, operand_desc(ga, a_hi, kk), operand_desc(gb, b_lo, kk), idesc, 1);
+            mma_tf32(tmem, operand_desc(ga, a_lo, kk), operand_desc(gb, b_hi, kk), idesc, 1);
           }
         }
         mma_commit(&empty_bar[s]);                          // stage free once these MMAs finish
@@ -268,70 +359,145 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
     if (!ok) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
     fence_after_sync();
     if (ok && !*(volatile int*)&abort_flag) {
-      int64_t ldc = g.ldc;
-      float* C = g.C;
-      if (g.c_ref.tab >= 0) {
-        const PtrEntry& e = tabs[g.c_ref.tab * nparams + g.c_ref.param];
-        ldc = e.ld;
-        C = const_cast<float*>(e.ptr) + g.c_ref.r0 * e.ld + g.c_ref.c0;
-      }
-      // The pipeline buffers are idle now: each warp stages its 32 x 32
-      // chunks there (row pitch 33 floats, conflict-free both ways).
-      float* stg = reinterpret_cast<float*>(smem) + q * (32 * 33);
-      const int row0 = m0 + 32 * q;
+      EpiArgs e;
+      e.load(g, tabs, nparams);
+      // Lane l of warp q holds accumulator row 32 q + l (TMEM lane), 32
+      // columns per load.  When bases and leading dimensions are 16-byte
+      // aligned, Cin comes in and the outputs go out as one 1-D bulk copy
+      // per row segment (128 bytes), staged in this warp's rows of the idle
+      // pipeline buffers; otherwise each lane loads and stores its row
+      // directly.  The mirror of a symmetric product writes column segments,
+      // contiguous across the lanes.
+      const int rbase = m0 + 32 * q;
+      const int row = rbase + lane;
+      const bool row_ok = row < e.M;
+      const int nrows = min(32, e.M - rbase);
+      const int ncols = min(BN, e.N - n0);
+      const int nchunks = ncols > 0 ? (ncols + 31) / 32 : 0;
+      const bool cin_bulk = e.beta != 0.0f &&
+                            ((reinterpret_cast<uintptr_t>(e.Cin) | uintptr_t(e.ldcin * 4)) & 15) == 0 &&
+                            (e.N & 3) == 0;
+      const bool out_bulk = ((reinterpret_cast<uintptr_t>(e.C) | uintptr_t(e.ldc * 4) |
+                              reinterpret_cast<uintptr_t>(e.Chi) | reinterpret_cast<uintptr_t>(e.Clo) |
+                              uintptr_t(e.ldh * 4)) & 15) == 0 &&
+                            (e.N & 3) == 0;
+      const bool out_vec = out_bulk;                        // same alignment conditions
+      uint8_t* wbuf = smem + q * Cfg::kEpiWarp;
+      const uint32_t wsm = smem_u32(wbuf);
+      const uint32_t my_row = uint32_t(lane * Cfg::kPitch * 4);
+      int issued = -1, consumed = -1;                       // Cin chunks
+      auto issue_cin = [&](int i) {
+        const int cb = n0 + 32 * i;
+        const uint32_t bytes = uint32_t(min(32, e.N - cb)) * 4u;
+        uint64_t* bar = &cin_bar[q][i & 1];
+        if (lane == 0) mbar_expect_tx(bar, bytes * uint32_t(nrows));
+        __syncwarp();
+        if (row_ok) bulk_load(wsm + (i & 1) * Cfg::kRowBuf + my_row, e.Cin + int64_t(row) * e.ldcin + cb, bytes, bar);
+        issued = i;
+      };
+      if (nrows > 0 && nchunks > 0) {
+        if (cin_bulk) issue_cin(0);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        if (n0 + c0 >= g.N) break;                          // warp-uniform
-        uint32_t r[32];
-        tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(c0), r);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __uint_as_float(r[j]);
-        __syncwarp();
-        // direct store: lane = column, coalesced along the row.  All 32
-        // loads of Cin are issued before any use so their latencies overlap.
-        const int col = n0 + c0 + lane;
-        const bool col_ok = col < g.N;
-        float cin[32];
-        if (g.beta != 0.0f) {
-#pragma unroll
-          for (int rr = 0; rr < 32; ++rr) {
-            const int row = row0 + rr;
-            cin[rr] = (col_ok && row < g.M) ? __ldg(g.Cin + int64_t(row) * g.ldcin + col) : 0.0f;
+        for (int i = 0; i < nchunks; ++i) {
+          const int c0 = 32 * i, cb = n0 + c0;
+          if (cin_bulk && i + 1 < nchunks) {
+            // buffer (i + 1) & 1 was last read, through the generic proxy, in chunk i - 1
+            fence_proxy_async();
+            __syncwarp();
+            issue_cin(i + 1);
           }
-        }
+          uint32_t r[32];
+          tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(c0), r);
+          float v[32];
 #pragma unroll
-        for (int rr = 0; rr < 32; ++rr) {
-          const int row = row0 + rr;
-          float v = g.alpha * stg[rr * 33 + lane];
-          if (g.beta != 0.0f) v = fmaf(g.beta, cin[rr], v);
-          stg[rr * 33 + lane] = v;
-          if (!col_ok || row >= g.M || (g.symmetric && col > row)) continue;
-          if (C) C[int64_t(row) * ldc + col] = g.out_round ? rn_tf32(v) : v;
-          if (g.Chi) {
-            const float h = rn_tf32(v);
-            g.Chi[int64_t(row) * g.ldh + col] = h;
-            if (g.Clo) g.Clo[int64_t(row) * g.ldh + col] = rn_tf32(v - h);
+          for (int j = 0; j < 32; ++j) v[j] = e.alpha * __uint_as_float(r[j]);
+          if (e.beta != 0.0f) {
+            if (cin_bulk) {
+              if (!mbar_wait(&cin_bar[q][i & 1], (i >> 1) & 1)) {
+                atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+                break;
+              }
+              consumed = i;
+              if (row_ok) {
+                const float4* src = reinterpret_cast<const float4*>(wbuf + (i & 1) * Cfg::kRowBuf + my_row);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                  if (cb + 4 * t >= e.N) break;
+                  const float4 x = src[t];
+                  v[4 * t + 0] = fmaf(e.beta, x.x, v[4 * t + 0]);
+                  v[4 * t + 1] = fmaf(e.beta, x.y, v[4 * t + 1]);
+                  v[4 * t + 2] = fmaf(e.beta, x.z, v[4 * t + 2]);
+                  v[4 * t + 3] = fmaf(e.beta, x.w, v[4 * t + 3]);
+                }
+              }
+            } else if (row_ok) {
+              const float* src = e.Cin + int64_t(row) * e.ldcin + cb;
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (cb + j < e.N) v[j] = fmaf(e.beta, __ldg(src + j), v[j]);
+            }
           }
-        }
-        __syncwarp();
-        // mirror store of the strictly-lower part: lane = row, coalesced
-        // along the transposed row
-        if (g.symmetric && n0 + c0 < row0 + 32) {
-          const int row = row0 + lane;
-          for (int j = 0; j < 32; ++j) {
-            const int c = n0 + c0 + j;
-            if (c >= g.N) break;
-            if (row >= g.M || c >= row) continue;
-            const float v = stg[lane * 33 + j];
-            if (C) C[int64_t(c) * ldc + row] = g.out_round ? rn_tf32(v) : v;
-            if (g.Chi) {
-              const float h = rn_tf32(v);
-              g.Chi[int64_t(c) * g.ldh + row] = h;
-              if (g.Clo) g.Clo[int64_t(c) * g.ldh + row] = rn_tf32(v - h);
+          // row segment: columns cb.. of this lane's row (only col <= row
+          // when the product is symmetric)
+          const bool below = !e.symmetric || cb + 31 < rbase;   // whole chunk left of every row
+          if (out_bulk && below) {
+            if (row_ok) {
+              bulk_wait_read();                             // staging rows free again
+              float4* oc = reinterpret_cast<float4*>(wbuf + 2 * Cfg::kRowBuf + my_row);
+              float4* oh = reinterpret_cast<float4*>(wbuf + 3 * Cfg::kRowBuf + my_row);
+              float4* ol = reinterpret_cast<float4*>(wbuf + 4 * Cfg::kRowBuf + my_row);
+#pragma unroll
+              for (int t = 0; t < 8; ++t) {
+                if (cb + 4 * t >= e.N) break;
+                const float a = v[4 * t], b = v[4 * t + 1], x = v[4 * t + 2], y = v[4 * t + 3];
+                const float4 h = make_float4(rn_tf32(a), rn_tf32(b), rn_tf32(x), rn_tf32(y));
+                oc[t] = e.out_round ? h : make_float4(a, b, x, y);
+                oh[t] = h;
+                ol[t] = make_float4(rn_tf32(a - h.x), rn_tf32(b - h.y), rn_tf32(x - h.z), rn_tf32(y - h.w));
+              }
+              fence_proxy_async();                          // staged rows visible to the bulk copies
+              const uint32_t bytes = uint32_t(min(32, e.N - cb)) * 4u;
+              if (e.C) bulk_store(e.C + int64_t(row) * e.ldc + cb, wsm + 2 * Cfg::kRowBuf + my_row, bytes);
+              if (e.Chi) bulk_store(e.Chi + int64_t(row) * e.ldh + cb, wsm + 3 * Cfg::kRowBuf + my_row, bytes);
+              if (e.Clo) bulk_store(e.Clo + int64_t(row) * e.ldh + cb, wsm + 4 * Cfg::kRowBuf + my_row, bytes);
+              bulk_commit();
+            }
+          } else if (row_ok) {
+            if (out_vec) {
+#pragma unroll
+              for (int t = 0; t < 8; ++t) {
+                const int c = cb + 4 * t;
+                if (c >= e.N) break;
+                if (!e.symmetric || c + 3 <= row) {
+                  e.put4(int64_t(row), c, v[4 * t + 0], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
+                } else {
+#pragma unroll
+                  for (int u = 0; u < 4; ++u)
+                    if (c + u <= row) e.put(int64_t(row), c + u, v[4 * t + u]);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int c = cb + j;
+                if (c < e.N && (!e.symmetric || c <= row)) e.put(int64_t(row), c, v[j]);
+              }
+            }
+          }
+          // mirror of the strictly-lower part: element (row, c) also at (c, row)
+          if (e.symmetric && cb < rbase + 32) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int c = cb + j;
+              if (row_ok && c < e.N && c < row) e.put(int64_t(c), row, v[j]);
             }
           }
         }
-        __syncwarp();
+        // Before the buffers are released: this lane's bulk stores done, and
+        // (after an abort) every Cin copy that was issued has landed.
+        bulk_wait_all();
+        for (int i = consumed + 1; i <= issued; ++i)
+          if (!mbar_wait(&cin_bar[q][i & 1], (i >> 1) & 1)) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
       }
     }
   }

@@ -196,10 +196,11 @@ shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max
 shampoo4_status launch_clear(const ClearDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 
 // Codec launchers (quant4.cu).  `skip` (optional, per tensor) suppresses a
-// tensor when *skip[i] != 0.
+// tensor when *skip[i] != 0.  `launched` (optional) receives the number of
+// kernels issued (one per batch of up to 64 non-empty tensors).
 shampoo4_status launch_pack(const float* const* x, const int64_t* n, int32_t count,
                             uint8_t* const* codes, float* const* scales, cudaStream_t st,
-                            const uint32_t* const* skip = nullptr);
+                            const uint32_t* const* skip = nullptr, int* launched = nullptr);
 shampoo4_status launch_unpack(const uint8_t* const* codes, const float* const* scales,
                               const int64_t* n, int32_t count, float* const* x, cudaStream_t st);
 

@@ -148,7 +148,8 @@ k_quant4_unpack(const __grid_constant__ UnpackBatch b) {
 // Host launchers, shared with the optimizer's own requantization.
 shampoo4_status launch_pack(const float* const* x, const int64_t* n, int32_t count,
                             uint8_t* const* codes, float* const* scales, cudaStream_t st,
-                            const uint32_t* const* skip) {
+                            const uint32_t* const* skip, int* launched) {
+  if (launched) *launched = 0;
   for (int32_t base = 0; base < count; base += kCodecMaxBatch) {
     PackBatch b;
     b.count = 0;
@@ -167,6 +168,7 @@ shampoo4_status launch_pack(const float* const* x, const int64_t* n, int32_t cou
     if (ctas > 0x7fffffffLL) return SHAMPOO4_ERR_INVALID_ARG;
     k_quant4_pack<<<unsigned(ctas), kCodecThreads, 0, st>>>(b);
     S4_CUDA(cudaGetLastError());
+    if (launched) ++*launched;
   }
   return SHAMPOO4_OK;
 }

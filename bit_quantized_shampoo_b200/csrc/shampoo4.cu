@@ -105,7 +105,7 @@ struct shampoo4_ctx {
   cudaEvent_t tab_event = nullptr;
   bool tab_event_pending = false;
   // optional per-launch timing (diagnostics)
-  struct Rec { int tag; cudaEvent_t e0, e1; double flops, bytes; };
+  struct Rec { int tag; cudaEvent_t e0, e1; double flops, bytes; int kernels; };
   bool timing = false;
   std::vector<cudaEvent_t> ev_pool;
   std::vector<Rec> recs;
@@ -1020,7 +1020,7 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
   uint32_t* gflags = reinterpret_cast<uint32_t*>(h->d_ws + h->ws_flags);
   for (const Launch& L : prog) {
     const void* d = h->d_ws + h->ws_desc + L.desc_off;
-    shampoo4_ctx::Rec rec{L.tag, nullptr, nullptr, L.flops, L.bytes};
+    shampoo4_ctx::Rec rec{L.tag, nullptr, nullptr, L.flops, L.bytes, 1};
     if (h->timing) {
       rec.e0 = take_event(h);
       rec.e1 = take_event(h);
@@ -1076,7 +1076,7 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
         break;
       case Kind::Pack:
         S4_TRY(launch_pack(L.px.data(), L.pn.data(), L.count, L.pcodes.data(), L.pscales.data(), st,
-                           L.pskip.data()));
+                           L.pskip.data(), &rec.kernels));
         break;
     }
     if (h->timing) {
@@ -1095,7 +1095,7 @@ shampoo4_status collect_timing(shampoo4_ctx* h) {
     h->t_ms[r.tag] += ms;
     h->t_flops[r.tag] += r.flops;
     h->t_bytes[r.tag] += r.bytes;
-    h->t_launches[r.tag] += 1;
+    h->t_launches[r.tag] += r.kernels;
     h->ev_pool.push_back(r.e0);
     h->ev_pool.push_back(r.e1);
   }

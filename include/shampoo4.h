@@ -64,10 +64,14 @@ typedef enum {
 /* Arithmetic of the dense products.
  *  TF32: operands rounded to TF32 (round to nearest), fp32 accumulation.
  *  FP32: fp32-accurate products.
- * The subspace product (S + eps I) U and the Rayleigh product S Q are always
- * fp32-accurate: they must resolve eigenvalues near eps, far below TF32's
- * resolution of the largest one.  The QR of the subspace step always runs
- * its Gram matrix, Cholesky factor and triangular solve in fp64. */
+ * The subspace product (S + eps I) U, the Rayleigh product S Q and every
+ * product of the QR are always fp32-accurate: they must resolve eigenvalues
+ * near eps, far below TF32's resolution of the largest one.  The QR is a
+ * shifted Cholesky-QR3 (Fukaya et al., SIAM J. Sci. Comput. 2020) whose
+ * products run on the tensor cores as 3xTF32 with 64x64 Cholesky blocks in
+ * fp64; a factor whose fp32 Cholesky breaks down is redone in fp64 on the
+ * CUDA cores (SHAMPOO4_FLAG_QR_FALLBACK).  Factors whose edge is not a
+ * multiple of 4 take the fp64 QR directly. */
 typedef enum { SHAMPOO4_PREC_TF32 = 0, SHAMPOO4_PREC_FP32 = 1 } shampoo4_precision;
 
 typedef struct {
