@@ -63,6 +63,8 @@ _SIGS = {
     "quant4_unpack": [C.POINTER(C.c_void_p), C.POINTER(C.c_void_p), c_i64_p, C.c_int32,
                       C.POINTER(C.c_void_p), C.c_void_p],
     "quant4_tables": [c_f32_p, c_f32_p],
+    "shampoo4_update_stats_noalloc": [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_int64,
+                                      C.c_float, C.c_void_p, C.c_void_p],
     "shampoo4_timing_enable": [C.c_void_p, C.c_int32],
     "shampoo4_timing_read": [C.c_void_p, C.c_int32, C.POINTER(C.c_double), c_i64_p, C.POINTER(C.c_double),
                              C.POINTER(C.c_double)],

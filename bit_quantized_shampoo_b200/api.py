@@ -154,6 +154,25 @@ def quant4_unpack(codes, scales, ns, out=None, stream=None):
     return out
 
 
+def update_stats_noalloc(L_, R_, G, beta, flags=None, stream=None):
+    """shampoo4_update_stats_noalloc on caller-owned CUDA tensors: L_ (m x m)
+    and R_ (n x n) fp32 contiguous, G (m x n) fp32 with unit column stride,
+    flags an optional int32/uint32 device word.  Marshalling only; the
+    library allocates nothing."""
+    _need_cuda(G, torch.float32, "G")
+    _need_cuda(L_, torch.float32, "L")
+    _need_cuda(R_, torch.float32, "R")
+    m, n = G.shape
+    ldg = _row_major_2d(G, "G")
+    if tuple(L_.shape) != (m, m) or not L_.is_contiguous():
+        raise ValueError("L must be a contiguous m x m tensor")
+    if tuple(R_.shape) != (n, n) or not R_.is_contiguous():
+        raise ValueError("R must be a contiguous n x n tensor")
+    fp = C.c_void_p(flags.data_ptr()) if flags is not None else C.c_void_p()
+    L.call("shampoo4_update_stats_noalloc", C.c_void_p(L_.data_ptr()), C.c_void_p(R_.data_ptr()),
+           C.c_void_p(G.data_ptr()), m, n, ldg, float(beta), fp, _stream(stream))
+
+
 def quant4_tables():
     cb = (C.c_float * 16)()
     th = (C.c_float * 15)()

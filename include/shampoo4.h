@@ -223,6 +223,32 @@ shampoo4_status quant4_unpack(const uint8_t* const* d_codes, const float* const*
 /* The 16 codebook levels and 15 thresholds the codec uses (host copy). */
 shampoo4_status quant4_tables(float codebook[16], float thresholds[15]);
 
+/* Statistics update of ONE tile with no handle, no workspace and no device
+ * allocation (no counterpart in the 4-bit Shampoo paper: an interface for
+ * callers that cannot allocate device memory at the point of the call, such
+ * as a hook running while a caching allocator holds its lock, or a process
+ * whose device memory is fully reserved by another allocator).
+ *   L <- beta L + (1 - beta) G G^T     (m x m, row-major, ld m)
+ *   R <- beta R + (1 - beta) G^T G     (n x n, row-major, ld n)
+ * G: m x n row-major device matrix, leading dimension ldg >= n.  The products
+ * are TF32 (operands rounded to TF32, round to nearest; fp32 sums), like
+ * shampoo4_update_stats with SHAMPOO4_PREC_TF32; L and R come out exactly
+ * symmetric.  A gradient holding a NaN or an infinity leaves L and R
+ * unchanged and ORs SHAMPOO4_FLAG_NONFINITE_GRAD into *d_flags (a device
+ * word the caller owns and zeroes; optional, may be NULL).
+ * Limits: m, n <= 1024 and m * n <= 2^18 (262144); larger tiles return
+ * SHAMPOO4_ERR_WORKSPACE before touching the device.  Pointers 4-byte aligned;
+ * other bad arguments return SHAMPOO4_ERR_INVALID_ARG.
+ * Scratch is a fixed 1 MiB + 4 KiB device array inside the library (one per
+ * device); every call resets what must start at zero.  Calls that overlap
+ * (different streams or unordered host threads) share it and race: order
+ * them.  The first call on a device looks the array up and may load the
+ * module; make it before any stream capture.  Everything is enqueued on
+ * `stream`; nothing is allocated or freed. */
+shampoo4_status shampoo4_update_stats_noalloc(float* d_L, float* d_R, const float* d_G, int32_t m,
+                                              int32_t n, int64_t ldg, float beta, uint32_t* d_flags,
+                                              shampoo4_stream_t stream);
+
 void shampoo4_destroy(shampoo4_handle h);
 const char* shampoo4_status_string(shampoo4_status s);
 
