@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-codec", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--shapes", default=None, help="comma-separated RxC list replacing the workload's shapes")
+    ap.add_argument("--grad-sets", type=int, default=2,
+                    help="seeded gradient sets the steps cycle through (1 = the same gradient every step)")
     return ap.parse_args()
 
 
@@ -250,19 +252,27 @@ def main():
 
     w = workload_shapes(args.workload, args.shapes)
     shapes = list(w.shapes)
-    # inputs: seeded host draws, copied to pinned host memory and to HBM
-    host_g = [torch.from_numpy(gradient(w, i, 1)).pin_memory() for i in range(len(shapes))]
-    dev_g = [h.to(dev, non_blocking=False) for h in host_g]
+    # inputs: seeded host draws (one set per gradient step seed), copied to
+    # pinned host memory and to HBM; step t uses set t mod grad_sets
+    nsets = max(1, args.grad_sets)
+    host_sets = [[torch.from_numpy(gradient(w, i, 1 + s)).pin_memory() for i in range(len(shapes))]
+                 for s in range(nsets)]
+    dev_sets = [[h.to(dev, non_blocking=False) for h in hs] for hs in host_sets]
+    host_g = host_sets[0]
     dev_out = [torch.empty(s, dtype=torch.float32, device=dev) for s in shapes]
     host_out = [torch.empty(s, dtype=torch.float32).pin_memory() for s in shapes]
     sh = api.Shampoo4(shapes, beta=w.beta, eps=w.eps, max_block=w.max_block, bjorck_iters=w.bjorck_iters,
                       precision=args.precision, device=dev)
     stream = torch.cuda.current_stream()
 
+    counter = [0]
+
     def step():
-        sh.update_stats(dev_g)
+        g = dev_sets[counter[0] % nsets]
+        counter[0] += 1
+        sh.update_stats(g)
         sh.refresh_roots()
-        sh.precondition(dev_g, out=dev_out)
+        sh.precondition(g, out=dev_out)
 
     for _ in range(args.warmup):
         step()
@@ -320,6 +330,7 @@ def main():
             "data": "synthetic",
             "config": {"workload": w.name, "tiles": sh.nblocks, "factors": sh.nfactors,
                        "steps_per_refresh": 1,
+                       "gradients": f"{nsets} seeded set(s), step t uses set t mod {nsets}",
                        "l2": (f"inputs larger than L2 ({g_bytes / 1e9:.2f} GB of G, {stat_bytes / 1e9:.2f} GB "
                               f"of fp32 statistics; L2 is 0.126 GB)")},
             "root_refreshes_per_s": value * sh.nfactors,
@@ -335,7 +346,8 @@ def main():
         e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e2.record(stream)
         for _ in range(k):
-            for h, d in zip(host_g, dev_g):
+            s = counter[0] % nsets
+            for h, d in zip(host_sets[s], dev_sets[s]):
                 d.copy_(h, non_blocking=True)
             step()
             for d, h in zip(dev_out, host_out):

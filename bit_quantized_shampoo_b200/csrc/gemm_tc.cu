@@ -194,6 +194,7 @@ struct EpiArgs {
   float* C; int64_t ldc;
   float* Chi; float* Clo; int64_t ldh;
   const float* Cin; int64_t ldcin;
+  unsigned long long* devsq;
 
   __device__ __forceinline__ void load(const TcGemmDesc& g, const PtrEntry* tabs, int nparams) {
     M = g.M; N = g.N; symmetric = g.symmetric; out_round = g.out_round;
@@ -206,6 +207,7 @@ struct EpiArgs {
     }
     Chi = g.Chi; Clo = g.Clo; ldh = g.ldh;
     Cin = g.Cin; ldcin = g.ldcin;
+    devsq = g.devsq;
   }
   // One element to every requested output: C (optionally TF32-rounded) and
   // the TF32 split (Chi, Clo).
@@ -386,6 +388,7 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
       const uint32_t wsm = smem_u32(wbuf);
       const uint32_t my_row = uint32_t(lane * Cfg::kPitch * 4);
       int issued = -1, consumed = -1;                       // Cin chunks
+      unsigned long long dev_fine = 0;                      // deviation sum, plan.h units
       auto issue_cin = [&](int i) {
         const int cb = n0 + 32 * i;
         const uint32_t bytes = uint32_t(min(32, e.N - cb)) * 4u;
@@ -435,6 +438,16 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
 #pragma unroll
               for (int j = 0; j < 32; ++j)
                 if (cb + j < e.N) v[j] = fmaf(e.beta, __ldg(src + j), v[j]);
+            }
+          }
+          if (e.devsq && row_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int c = cb + j;
+              if (c >= e.N || c == row || (e.symmetric && c > row)) continue;
+              const float q = v[j] * v[j];
+              const unsigned long long w = (e.symmetric && c < row) ? 2ull : 1ull;
+              dev_fine += w * static_cast<unsigned long long>(fminf(q, kDevFineClamp) * kDevFineUnit);
             }
           }
           // row segment: columns cb.. of this lane's row (only col <= row
@@ -492,6 +505,11 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
               if (row_ok && c < e.N && c < row) e.put(int64_t(c), row, v[j]);
             }
           }
+        }
+        if (e.devsq) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) dev_fine += __shfl_xor_sync(0xffffffffu, dev_fine, o);
+          if (lane == 0 && dev_fine) atomicAdd(e.devsq, dev_fine);
         }
         // Before the buffers are released: this lane's bulk stores done, and
         // (after an abort) every Cin copy that was issued has landed.

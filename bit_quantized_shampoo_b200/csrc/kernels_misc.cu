@@ -258,7 +258,7 @@ constexpr int kPotrfFSmem = 2 * kPanel * (kPanel + 1) * 8;
 __global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ descs) {
   const PotrfDescF& g = descs[blockIdx.x];
   const int jb = g.jb;
-  if (jb <= 0 || *g.fail) return;
+  if (jb <= 0 || *g.fail || (g.skip && *g.skip)) return;
   extern __shared__ double sm_potrf[];
   double (*L)[kPanel + 1] = reinterpret_cast<double (*)[kPanel + 1]>(sm_potrf);
   double (*Li)[kPanel + 1] = reinterpret_cast<double (*)[kPanel + 1]>(sm_potrf + kPanel * (kPanel + 1));
@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ 
   for (int c = 0; c < jb; ++c) {
     if (threadIdx.x == 0) {
       double p = L[c][c];
-      if (!(p > 0.0) || !isfinite(p)) { bad = 1; p = 1.0; }
+      if (!(p > double(g.min_pivot)) || !isfinite(p)) { bad = 1; p = 1.0; }
       L[c][c] = sqrt(p);
     }
     __syncthreads();
@@ -339,17 +339,64 @@ shampoo4_status launch_potrf_f(const PotrfDescF* d_desc, int count, cudaStream_t
 __global__ void __launch_bounds__(256) k_shift_f(const ShiftDescF* __restrict__ descs) {
   const ShiftDescF& g = descs[blockIdx.x];
   if (g.skip && *g.skip) return;
-  __shared__ double part[256];
-  double t = 0.0;
-  for (int i = threadIdx.x; i < g.d; i += blockDim.x) t += double(g.W[int64_t(i) * g.ld + i]);
-  part[threadIdx.x] = t;
-  __syncthreads();
-  for (int w = 128; w > 0; w >>= 1) {
-    if (threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
-    __syncthreads();
+  for (int i = threadIdx.x; i < g.d; i += blockDim.x) {
+    float* w = g.W + int64_t(i) * g.ld + i;
+    *w = fmaf(g.coef, *w, *w);
   }
-  const float s = float(double(g.coef) * part[0]);
-  for (int i = threadIdx.x; i < g.d; i += blockDim.x) g.W[int64_t(i) * g.ld + i] += s;
+}
+
+// ---- exact Gram diagonal ------------------------------------------------------
+__global__ void __launch_bounds__(256) k_diag(const DiagDesc* __restrict__ descs) {
+  const DiagDesc& g = descs[blockIdx.y];
+  if (g.skip && *g.skip) return;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  unsigned long long t = 0;
+  if (i < g.d) {
+    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+    const float* x = g.X + i;
+    int k = 0;
+    for (; k + 4 <= g.d; k += 4) {
+      const double a = x[int64_t(k) * g.d], b = x[int64_t(k + 1) * g.d];
+      const double c = x[int64_t(k + 2) * g.d], e = x[int64_t(k + 3) * g.d];
+      s0 = fma(a, a, s0); s1 = fma(b, b, s1); s2 = fma(c, c, s2); s3 = fma(e, e, s3);
+    }
+    for (; k < g.d; ++k) { const double a = x[int64_t(k) * g.d]; s0 = fma(a, a, s0); }
+    const float w = float((s0 + s1) + (s2 + s3));
+    g.W[int64_t(i) * g.ldw + i] = w;
+    if (g.devsq) {
+      const float q = (w - 1.0f) * (w - 1.0f);
+      t = static_cast<unsigned long long>(fminf(q, kDevFineClamp) * kDevFineUnit);
+    }
+  }
+  if (g.devsq) {
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if ((threadIdx.x & 31) == 0 && t) atomicAdd(g.devsq, t);
+  }
+}
+
+shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaStream_t st) {
+  if (count <= 0 || max_d <= 0) return SHAMPOO4_OK;
+  for (int base = 0; base < count; base += 65535) {
+    const int c = count - base < 65535 ? count - base : 65535;
+    k_diag<<<dim3(unsigned((max_d + 255) / 256), unsigned(c)), 256, 0, st>>>(d_desc + base);
+    S4_CUDA(cudaGetLastError());
+  }
+  return SHAMPOO4_OK;
+}
+
+// ---- last-pass gate -----------------------------------------------------------
+__global__ void __launch_bounds__(256) k_gate(const GateDesc* __restrict__ descs, int count) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= count) return;
+  const GateDesc& g = descs[i];
+  *g.out = (*g.bad != 0u || *g.devsq <= g.thr) ? 1u : 0u;
+}
+
+shampoo4_status launch_gate(const GateDesc* d_desc, int count, cudaStream_t st) {
+  if (count <= 0) return SHAMPOO4_OK;
+  k_gate<<<unsigned((count + 255) / 256), 256, 0, st>>>(d_desc, count);
+  S4_CUDA(cudaGetLastError());
+  return SHAMPOO4_OK;
 }
 
 shampoo4_status launch_shift_f(const ShiftDescF* d_desc, int count, cudaStream_t st) {

@@ -146,9 +146,16 @@ struct PotrfDescF {
   float* oh; float* ol;       // optional TF32 split of the factor (same ld)
   float* ih; float* il;       // optional TF32 split of the inverse factor,
                               // 64 x 64 with leading dimension 64, zero-padded
+  const uint32_t* skip;       // optional: block skipped when *skip != 0
+  float min_pivot;            // a pivot (Schur-complement diagonal) at or
+                              // below this counts as a breakdown; 0 = only
+                              // non-positive or non-finite pivots do
+  int32_t pad2_;
 };
 
-// W <- W + coef * trace(W) * I (the shift of the first Cholesky-QR pass).
+// W_ii <- W_ii (1 + coef) for i < d: the shift of the first Cholesky-QR
+// pass, applied to the column-equilibrated Gram (D^-1 W D^-1 + coef I with
+// D = diag(W)^1/2), i.e. a shift of coef times each column's squared norm.
 struct ShiftDescF {
   float* W; int64_t ld;
   int32_t d; float coef;
@@ -176,6 +183,35 @@ struct ClearDesc {
   int64_t n;
 };
 
+// W_ii <- sum_k X[k, i]^2 (fp64 sums, one thread per column, rounded once
+// to fp32) for i < d, X row-major d x d.  The tensor cores' accumulation
+// truncates, so a Gram's diagonal -- a sum of positive terms -- comes out
+// low by about 1e-8 K relative; this restores it.  devsq (optional, two
+// words): adds the diagonal's share of sum (W_ij - delta_ij)^2, as the GEMM
+// epilogue does for the off-diagonal part (see kDevFineUnit).
+struct DiagDesc {
+  const float* X;
+  float* W; int64_t ldw;
+  int32_t d; int32_t pad_;
+  unsigned long long* devsq;
+  const uint32_t* skip;
+};
+
+// Deviation sum sum_ij min((W_ij - delta_ij)^2, 2^-20) of a Gram, in units
+// of 2^-60: an exact integer sum, independent of the order of additions.
+constexpr float kDevFineClamp = 0x1p-20f, kDevFineUnit = 0x1p60f;
+
+// Decision before the last Cholesky-QR pass of a factor, from the Gram of
+// its input Q: out = 1 (skip the pass) when *bad != 0 or *devsq <= thr (Q
+// already orthonormal to the arithmetic's floor), else 0.
+struct GateDesc {
+  const unsigned long long* devsq;
+  const uint32_t* bad;
+  uint32_t* out;
+  unsigned long long thr;
+};
+
+
 // ---- launchers (each enqueues one launch over `count` descriptors) -------
 shampoo4_status launch_gemm_f32(const GemmF32Desc* d_desc, int count, int max_tiles,
                                 const PtrEntry* tabs, int nparams, cudaStream_t st);
@@ -194,6 +230,8 @@ shampoo4_status launch_shift_f(const ShiftDescF* d_desc, int count, cudaStream_t
 shampoo4_status launch_split(const SplitDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_clear(const ClearDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
+shampoo4_status launch_gate(const GateDesc* d_desc, int count, cudaStream_t st);
+shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaStream_t st);
 
 // Codec launchers (quant4.cu).  `skip` (optional, per tensor) suppresses a
 // tensor when *skip[i] != 0.  `launched` (optional) receives the number of

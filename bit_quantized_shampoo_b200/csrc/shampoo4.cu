@@ -16,6 +16,7 @@
 // a tile whose both sides are multiples of 4 does too.  The rest use the
 // CUDA-core kernels (gemm_simt.cu).  Both produce the same state.
 #include <algorithm>
+#include <cmath>
 #include <cstring>
 #include <map>
 #include <new>
@@ -29,7 +30,7 @@ using namespace s4;
 namespace {
 
 enum class Kind { GemmF32, GemmF64, Potrf, Trsm, Basis, Rayleigh, Mu, Scan, Convert, Pack, Shift, GemmTC, GemmTCSplit,
-                  GemmTCSplit64, PotrfF, ShiftF, Split };
+                  GemmTCSplit64, PotrfF, ShiftF, Split, Gate, Diag };
 
 struct Launch {
   Kind kind;
@@ -85,7 +86,7 @@ struct shampoo4_ctx {
   size_t state_bytes = 0, ws_bytes = 0;
   // workspace regions
   size_t ws_flags = 0, ws_tabs = 0, ws_fail = 0, ws_bflag = 0, ws_maps = 0, ws_nmaps = 0;
-  size_t ws_tcbad = 0, ws_tcgood = 0;
+  size_t ws_tcbad = 0, ws_tcgood = 0, ws_devsq = 0, ws_skip3 = 0;
   size_t ws_desc = 0, ws_desc_bytes = 0;
   // programs
   std::vector<Launch> prog_stats, prog_refresh_first, prog_refresh, prog_precond;
@@ -169,6 +170,8 @@ shampoo4_status plan(shampoo4_ctx* h) {
   h->ws_fail = take(ws, 4 * h->factors.size());
   h->ws_tcbad = take(ws, 4 * h->factors.size());
   h->ws_tcgood = take(ws, 4 * h->factors.size());
+  h->ws_devsq = take(ws, 8 * h->factors.size());
+  h->ws_skip3 = take(ws, 4 * h->factors.size());
   h->ws_bflag = take(ws, 4 * h->blocks.size());
   for (FactorPlan& f : h->factors) {
     size_t dd = size_t(f.d) * f.d;
@@ -261,6 +264,10 @@ struct Builder {
   uint32_t* fail(size_t fi) const { return wu(h->ws_fail) + fi; }
   uint32_t* tcbad(size_t fi) const { return wu(h->ws_tcbad) + fi; }
   uint32_t* tcgood(size_t fi) const { return wu(h->ws_tcgood) + fi; }
+  unsigned long long* devsq(size_t fi) const {
+    return reinterpret_cast<unsigned long long*>(ws + h->ws_devsq) + fi;
+  }
+  uint32_t* skip3(size_t fi) const { return wu(h->ws_skip3) + fi; }
   uint32_t* gflags() const { return wu(h->ws_flags); }
 
   // Device address of the tensor map of a dense d0 x d1 workspace matrix.
@@ -537,25 +544,44 @@ void build_cholqr_pass(Builder& b, std::vector<Launch>& prog, const std::vector<
 }
 
 // Cholesky-QR pass over the tensor-core factors, fp32-accurate throughout:
-// X -> Q.  Gram W = X^T X on the tensor cores (3xTF32), optional shift
-// W += 1e-5 trace(W) I, blocked right-looking Cholesky W = L L^T (64-wide
-// diagonal blocks and panel solves on CUDA cores in fp64, trailing updates
-// on the tensor cores), then Q L^T = X by column panels (updates on the
-// tensor cores, panel solves on CUDA cores).  Three such passes, the first
-// shifted, form shifted Cholesky-QR3 (Fukaya et al., SIAM J. Sci. Comput.
-// 2020).  The shift only has to exceed the error of the fp32-accurate Gram
-// (about 2e-6 ||X||_F^2); the first pass then leaves Q0 with a condition
-// number near sqrt(shift) / sigma_min(X), and the second pass succeeds when
-// that is below about 1e3.  Factors beyond that break down in a Cholesky
-// panel and are redone in fp64 from the intact Y.
+// X -> Q.  Gram W = X^T X on the tensor cores (3xTF32), optional shift,
+// left-looking blocked Cholesky W = L L^T (64-wide diagonal blocks in fp64
+// on CUDA cores, panel products on the tensor cores), then Q L^T = X by
+// column panels.  Up to three such passes, the first shifted, form shifted
+// Cholesky-QR3 (Fukaya et al., SIAM J. Sci. Comput. 2020).
+//
+// The shift is taken in the column-equilibrated frame: Cholesky-QR of X and
+// of X D^-1 (D = column norms) give the same Q and, in floating point, the
+// same rounding behaviour, so the conditioning that matters is that of
+// X D^-1 (unit columns, ||X D^-1||_F^2 = d).  The shift 1e-5 d there (1e-5 d
+// W_ii on the diagonal of W) exceeds the error of the fp32-accurate Gram
+// (about 2e-6 d in that frame); the first pass then leaves Q0 with a
+// condition number near sqrt(1e-5 d) / sigma_min(X D^-1), and the second
+// pass succeeds when that is below about 1e3.  Factors beyond that break
+// down in a Cholesky panel and are redone in fp64 from the intact Y.
+//
+// A warm subspace step (U from the previous refresh) has Y = (S + eps I) U
+// with nearly orthogonal columns of very different lengths: X D^-1 is close
+// to orthonormal, and two passes already reach the orthogonality floor of
+// this arithmetic (||Q^T Q - I||_F / sqrt(d) near 1.1e-7 sqrt(d), set by
+// the unbiased rounding of the off-diagonal sums).  So the third pass is
+// gated per factor: its Gram also measures ||Q^T Q - I||_F of the second
+// pass's output; its Cholesky and solve run only when that exceeds
+// kLastPassTol sqrt(d) * sqrt(d) (a cold first refresh needs them).  In that
+// pass a Cholesky pivot at or below kLastPassPivot -- a column of the
+// (unit-column) input nearly in the span of the previous ones, so that the
+// pass cannot be trusted -- counts as a breakdown, and the factor is redone
+// in fp64.
 constexpr float kTcShift = 1e-5f;
+constexpr double kLastPassTol = 2e-7;
+constexpr float kLastPassPivot = 1e-2f;
 
 struct Triplet { float* m; float* h; float* l; };
 
 int dpad_of(int d) { return (d + kPanelW - 1) / kPanelW * kPanelW; }
 
 void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Triplet>& X,
-                     const std::vector<Triplet>& Q, bool shifted) {
+                     const std::vector<Triplet>& Q, bool shifted, bool gated = false) {
   shampoo4_ctx* h = b.h;
   const size_t nf = h->factors.size();
   int dmax = 0;
@@ -565,11 +591,19 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
     // Gram W = X^T X (fp32 into W, its TF32 split into Th/Tl), optional shift
     std::vector<TcGemmDesc> g;
     std::vector<ShiftDescF> sd;
+    std::vector<GateDesc> gd;
+    std::vector<DiagDesc> dg;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
       if (!f.tc) continue;
       const int d = f.d;
       TcGemmDesc w = gemmtc(d, d, d, 1.0f, 0.0f);
+      if (gated) {
+        w.devsq = b.devsq(i);
+        const double tol = kLastPassTol * std::sqrt(double(d));        // on ||Q^T Q - I||_F / sqrt(d)
+        const double thr = std::min(tol * tol * d * double(kDevFineUnit), 0x1p62);
+        gd.push_back({b.devsq(i), b.tcbad(i), b.skip3(i), static_cast<unsigned long long>(thr)});
+      }
       w.a = b.operand(X[i].h, X[i].l, d, d, true, true, true);
       w.b = b.operand(X[i].h, X[i].l, d, d, false, false, true);
       w.C = b.wf(f.ws_W); w.ldc = d;
@@ -577,12 +611,19 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
       w.symmetric = 1;
       w.skip = b.tcbad(i);
       g.push_back(w);
-      if (shifted) sd.push_back({b.wf(f.ws_W), d, d, kTcShift, b.tcbad(i)});
+      dg.push_back({X[i].m, b.wf(f.ws_W), d, d, 0, gated ? b.devsq(i) : nullptr, b.tcbad(i)});
+      if (shifted) sd.push_back({b.wf(f.ws_W), d, d, kTcShift * float(d), b.tcbad(i)});
     }
     b.tag = SHAMPOO4_STAGE_QR_GRAM;
     emit_gemmtc(b, prog, g, true);
+    b.emit(prog, Kind::Diag, dg, dmax, 0, 4.0 * [&] { double s = 0; for (auto& x : dg) s += double(x.d) * x.d; return s; }());
     b.emit(prog, Kind::ShiftF, sd, 0);
+    b.tag = SHAMPOO4_STAGE_QR_CONVERT;
+    b.emit(prog, Kind::Gate, gd, 0);
   }
+  // the rest of the pass: skipped for a broken-down factor, and for a
+  // factor the gate passed
+  auto skip_of = [&](size_t i) -> const uint32_t* { return gated ? b.skip3(i) : b.tcbad(i); };
   // Cholesky, left-looking by 64-wide panels.  For panel J:
   //   W[j:, J] -= L[j:, <J] L[J, <J]^T      tensor cores (also refreshes the
   //                                          TF32 split of that column block)
@@ -610,12 +651,13 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
         u.C = W + int64_t(j) * d + j; u.ldc = d;
         u.Chi = Th + int64_t(j) * d + j; u.Clo = Tl + int64_t(j) * d + j; u.ldh = d;
         u.Cin = u.C; u.ldcin = d;
-        u.skip = b.tcbad(i);
+        u.skip = skip_of(i);
         up.push_back(u);
       }
       po.push_back({W + int64_t(j) * d + j, d, jb, 0, b.tcbad(i), b.gflags(), b.tcgood(i),
                     Th + int64_t(j) * d + j, Tl + int64_t(j) * d + j,
-                    b.wf(f.ws_Ih) + int64_t(j) * kPanelW, b.wf(f.ws_Il) + int64_t(j) * kPanelW});
+                    b.wf(f.ws_Ih) + int64_t(j) * kPanelW, b.wf(f.ws_Il) + int64_t(j) * kPanelW,
+                    gated ? b.skip3(i) : nullptr, gated ? kLastPassPivot : 0.0f, 0});
       fl_po += 2.0 * double(jb) * jb * jb / 3.0;
       if (rest <= 0) continue;
       TcGemmDesc t = gemmtc(rest, jb, jb, 1.0f, 0.0f);     // L21 = W21 L11^-T (in the split, in place)
@@ -624,7 +666,7 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
       t.b = b.operand(b.wf(f.ws_Ih), b.wf(f.ws_Il), dpad_of(d), kPanelW, false, true, true, 64);
       t.b.row0 = j;
       t.Chi = Th + int64_t(j + jb) * d + j; t.Clo = Tl + int64_t(j + jb) * d + j; t.ldh = d;
-      t.skip = b.tcbad(i);
+      t.skip = skip_of(i);
       l21.push_back(t);
     }
     b.tag = SHAMPOO4_STAGE_QR_SYRK;
@@ -651,7 +693,7 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
         u.b.row0 = j;
         u.Chi = b.wf(f.ws_Ph); u.Clo = b.wf(f.ws_Pl); u.ldh = kPanelW;
         u.Cin = X[i].m + j; u.ldcin = d;
-        u.skip = b.tcbad(i);
+        u.skip = skip_of(i);
         up.push_back(u);
         q.a = b.operand(b.wf(f.ws_Ph), b.wf(f.ws_Pl), d, kPanelW, true, false, true);
       } else {
@@ -661,7 +703,7 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
       q.b.row0 = j;
       q.C = Q[i].m + j; q.ldc = d;
       q.Chi = Q[i].h + j; q.Clo = Q[i].l + j; q.ldh = d;
-      q.skip = b.tcbad(i);
+      q.skip = skip_of(i);
       qp.push_back(q);
     }
     b.tag = SHAMPOO4_STAGE_QR_SOLVE_UPDATE;
@@ -810,10 +852,13 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
     emit_gemm32(b, prog, g);
   }
   {
-    // Tensor-core factors: Y stays in X[o]; fp32 shifted Cholesky-QR3
-    // Y -> X[c] -> Z -> X[c].  A factor whose fp32 Cholesky breaks down
-    // (tcbad) redoes the three passes in fp64 from the intact Y; the others
-    // skip that work (tcgood).  CUDA-core factors run the fp64 passes only.
+    // Tensor-core factors: Y stays in X[o]; fp32 shifted Cholesky-QR
+    // Y -> Z -> X[c], then the gated third pass in place on X[c] (its Gram
+    // and diagonal read X[c] first; panel J of the solve reads only column
+    // block J of the input and the already-rewritten blocks before it).  A
+    // factor whose fp32 Cholesky breaks down (tcbad) redoes three passes in
+    // fp64 from the intact Y; the others skip that work (tcgood).  CUDA-core
+    // factors run the fp64 passes only.
     std::vector<Triplet> Xy(nf), Xc(nf), Xz(nf);
     std::vector<char> use_simt(nf, 0), use_fb(nf, 0);
     std::vector<const uint32_t*> sk(nf);
@@ -842,9 +887,9 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
         a3[i] = Q1[i]; o3[i] = Qf[i];
       }
     }
-    build_cholqr_tc(b, prog, Xy, Xc, true);
-    build_cholqr_tc(b, prog, Xc, Xz, false);
+    build_cholqr_tc(b, prog, Xy, Xz, true);
     build_cholqr_tc(b, prog, Xz, Xc, false);
+    build_cholqr_tc(b, prog, Xc, Xc, false, true);
     std::vector<char> use_any(nf);
     for (size_t i = 0; i < nf; ++i) use_any[i] = use_simt[i] || use_fb[i];
     build_cholqr_pass(b, prog, use_any, a1, o1, none, none, sk, true);
@@ -1068,6 +1113,12 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
       case Kind::Split:
         S4_TRY(launch_split(static_cast<const SplitDesc*>(d), L.count, L.extent, st));
         break;
+      case Kind::Gate:
+        S4_TRY(launch_gate(static_cast<const GateDesc*>(d), L.count, st));
+        break;
+      case Kind::Diag:
+        S4_TRY(launch_diag(static_cast<const DiagDesc*>(d), L.count, int(L.extent), st));
+        break;
       case Kind::Shift:
         S4_TRY(launch_shift(static_cast<const ShiftDesc*>(d), L.count, st));
         break;
@@ -1252,6 +1303,7 @@ extern "C" shampoo4_status shampoo4_refresh_roots(shampoo4_handle h, shampoo4_st
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_fail, 0, 4 * h->factors.size(), st));
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_tcbad, 0, 4 * h->factors.size(), st));
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_tcgood, 1, 4 * h->factors.size(), st));
+  S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_devsq, 0, 8 * h->factors.size(), st));
   const bool first = !h->has_basis;
   S4_TRY(run(h, first ? h->prog_refresh_first : h->prog_refresh, st));
   h->last_refresh_first = first;

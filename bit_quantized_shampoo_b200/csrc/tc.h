@@ -36,6 +36,10 @@ struct TcGemmDesc {
   const float* Cin; int64_t ldcin;
   const uint32_t* skip;
   OperandRef c_ref;
+  // optional: the off-diagonal share (strictly-lower elements counted twice
+  // when symmetric) of the deviation sum of plan.h; the diagonal's share
+  // comes from the diagonal kernel
+  unsigned long long* devsq;
 };
 
 // Tile width N of the kernel instance: 256 (TF32), 128 (split), or 64
