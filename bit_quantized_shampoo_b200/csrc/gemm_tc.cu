@@ -165,7 +165,15 @@ struct TcCfg {
   static constexpr int kRowBuf = 32 * kPitch * 4;
   static constexpr int kEpiWarp = 5 * kRowBuf;
   static_assert(4 * kEpiWarp <= kStage * kStages, "epilogue staging fits the pipeline buffers");
-  static constexpr int kTmemCols = BN;                          // 128 or 256: a power of two
+  // The tensor cores' fp32 accumulation truncates: a long sum drifts low
+  // (about 1e-8 K relative when its terms share a sign) and its rounding
+  // noise grows with the accumulator's magnitude.  The fp32-accurate
+  // instances therefore keep kAcc accumulators, k-block kb going to
+  // accumulator kb mod kAcc, and add them in the epilogue with
+  // round-to-nearest: the drift drops kAcc-fold, the noise about
+  // sqrt(kAcc)-fold.
+  static constexpr int kAcc = SPLIT ? 4 : 1;
+  static constexpr int kTmemCols = BN * kAcc;                   // 256 or 512: a power of two
 };
 
 // Issue the loads of one operand tile (rows mn0.. of the problem, K block k0).
@@ -344,11 +352,13 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
         const uint32_t a_lo = st + Cfg::kATile + Cfg::kBTile, b_lo = a_lo + Cfg::kATile;
 #pragma unroll
         for (int kk = 0; kk < kBK / 8; ++kk) {
-          const uint32_t acc = (kb | kk) != 0;
-          mma_tf32(tmem, operand_desc(ga, a_hi, kk), operand_desc(gb, b_hi, kk), idesc, acc);
+          // first MMA into accumulator kb mod kAcc overwrites it
+          const uint32_t acc = (kb >= Cfg::kAcc || kk != 0) ? 1u : 0u;
+          const uint32_t dt = tmem + uint32_t((kb % Cfg::kAcc) * BN);
+          mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(gb, b_hi, kk), idesc, acc);
           if (SPLIT) {
-            mma_tf32(tmem, operand_desc(ga, a_hi, kk), operand_desc(gb, b_lo, kk), idesc, 1);
-            mma_tf32(tmem, operand_desc(ga, a_lo, kk), operand_desc(gb, b_hi, kk), idesc, 1);
+            mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(gb, b_lo, kk), idesc, 1);
+            mma_tf32(dt, operand_desc(ga, a_lo, kk), operand_desc(gb, b_hi, kk), idesc, 1);
           }
         }
         mma_commit(&empty_bar[s]);                          // stage free once these MMAs finish
@@ -372,6 +382,7 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
       // contiguous across the lanes.
       const int rbase = m0 + 32 * q;
       const int row = rbase + lane;
+      const int nacc = kblocks < Cfg::kAcc ? kblocks : Cfg::kAcc;   // accumulators written
       const bool row_ok = row < e.M;
       const int nrows = min(32, e.M - rbase);
       const int ncols = min(BN, e.N - n0);
@@ -413,7 +424,14 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
           tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(c0), r);
           float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = e.alpha * __uint_as_float(r[j]);
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          for (int a = 1; a < nacc; ++a) {                  // the other accumulators, added with RN
+            tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(a * BN + c0), r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += __uint_as_float(r[j]);
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= e.alpha;
           if (e.beta != 0.0f) {
             if (cin_bulk) {
               if (!mbar_wait(&cin_bar[q][i & 1], (i >> 1) & 1)) {

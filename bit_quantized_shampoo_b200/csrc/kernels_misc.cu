@@ -384,6 +384,40 @@ shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaSt
   return SHAMPOO4_OK;
 }
 
+// ---- exact diagonal of a product of split operands --------------------------
+__global__ void __launch_bounds__(256) k_rowdiag(const RowDiagDesc* __restrict__ descs) {
+  const RowDiagDesc& g = descs[blockIdx.y];
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (i >= g.d) return;                                    // warp-uniform
+  const int64_t r = int64_t(i) * g.ld;
+  double s = 0.0;
+  for (int k = lane; k < g.d; k += 32) {
+    const double a = double(g.ah[r + k]) + (g.al ? double(g.al[r + k]) : 0.0);
+    const double b = double(g.bh[r + k]) + (g.bl ? double(g.bl[r + k]) : 0.0);
+    s = fma(a, b, s);
+  }
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) {
+    const float v = float(s);
+    if (g.C) g.C[r + i] = v;
+    if (g.Chi) {
+      const float hv = tf32_rn(v);
+      g.Chi[r + i] = hv;
+      if (g.Clo) g.Clo[r + i] = tf32_rn(v - hv);
+    }
+  }
+}
+
+shampoo4_status launch_rowdiag(const RowDiagDesc* d_desc, int count, int max_d, cudaStream_t st) {
+  if (count <= 0 || max_d <= 0) return SHAMPOO4_OK;
+  for (int base = 0; base < count; base += 65535) {
+    const int c = count - base < 65535 ? count - base : 65535;
+    k_rowdiag<<<dim3(unsigned((max_d + 7) / 8), unsigned(c)), 256, 0, st>>>(d_desc + base);
+    S4_CUDA(cudaGetLastError());
+  }
+  return SHAMPOO4_OK;
+}
+
 // ---- last-pass gate -----------------------------------------------------------
 __global__ void __launch_bounds__(256) k_gate(const GateDesc* __restrict__ descs, int count) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;

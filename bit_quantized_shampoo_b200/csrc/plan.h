@@ -197,6 +197,20 @@ struct DiagDesc {
   const uint32_t* skip;
 };
 
+// Diagonal of a product C = A B^T of two split operands with the same rows:
+// C_ii = sum_k (ah + al)_ik (bh + bl)_ik in fp64 over the d columns, rounded
+// once to fp32 into C, and its TF32 split into (Chi, Clo) (each optional).
+// A sum of positive terms -- the diagonal of U diag(mu) U^T -- comes out of
+// the tensor cores' truncating accumulation low by about 1e-8 K relative;
+// this rewrites it.  One warp per row.
+struct RowDiagDesc {
+  const float* ah; const float* al;
+  const float* bh; const float* bl;
+  int64_t ld;                 // of the operands and of C / Chi / Clo
+  int32_t d; int32_t pad_;
+  float* C; float* Chi; float* Clo;
+};
+
 // Deviation sum sum_ij min((W_ij - delta_ij)^2, 2^-20) of a Gram, in units
 // of 2^-60: an exact integer sum, independent of the order of additions.
 constexpr float kDevFineClamp = 0x1p-20f, kDevFineUnit = 0x1p60f;
@@ -232,6 +246,7 @@ shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max
 shampoo4_status launch_clear(const ClearDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_gate(const GateDesc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaStream_t st);
+shampoo4_status launch_rowdiag(const RowDiagDesc* d_desc, int count, int max_d, cudaStream_t st);
 
 // Codec launchers (quant4.cu).  `skip` (optional, per tensor) suppresses a
 // tensor when *skip[i] != 0.  `launched` (optional) receives the number of

@@ -30,7 +30,7 @@ using namespace s4;
 namespace {
 
 enum class Kind { GemmF32, GemmF64, Potrf, Trsm, Basis, Rayleigh, Mu, Scan, Convert, Pack, Shift, GemmTC, GemmTCSplit,
-                  GemmTCSplit64, PotrfF, ShiftF, Split, Gate, Diag };
+                  GemmTCSplit64, PotrfF, ShiftF, Split, Gate, Diag, RowDiag };
 
 struct Launch {
   Kind kind;
@@ -966,6 +966,7 @@ void build_precondition(Builder& b) {
   std::vector<MuDesc> mu;
   std::vector<GemmF32Desc> roots;
   std::vector<TcGemmDesc> troots;
+  std::vector<RowDiagDesc> rdiag;              // exact diagonal of the fp32-accurate roots
   std::vector<float*> Pm(nf);                  // fp32 root of each factor
   double bytes_bd = 0;
   for (size_t i = 0; i < nf; ++i) {
@@ -986,6 +987,9 @@ void build_precondition(Builder& b) {
       g.Chi = b.wf(f.ws_Th); g.Clo = split ? b.wf(f.ws_Tl) : nullptr; g.ldh = d;
       g.symmetric = 1;
       troots.push_back(g);
+      if (split)
+        rdiag.push_back({b.wf(f.ws_Xh[1]), b.wf(f.ws_Xl[1]), b.wf(f.ws_Xh[0]), b.wf(f.ws_Xl[0]), d, d, 0,
+                         b.wf(f.ws_Xm[1]), b.wf(f.ws_Th), b.wf(f.ws_Tl)});
       Pm[i] = b.wf(f.ws_Xm[1]);
       bytes_bd += (0.5625 + (split ? 16.0 : 8.0)) * double(d) * d;
     } else {
@@ -1007,6 +1011,7 @@ void build_precondition(Builder& b) {
   b.emit(h->prog_precond, Kind::Basis, bd, emax, 0, bytes_bd);
   b.tag = SHAMPOO4_STAGE_ROOTS;
   emit_gemmtc(b, h->prog_precond, troots, split);
+  b.emit(h->prog_precond, Kind::RowDiag, rdiag, dmax, 0, 16.0 * sum_dd);
   emit_gemm32(b, h->prog_precond, roots);
   build_grad_copy(b, h->prog_precond, SHAMPOO4_STAGE_STATS_SCAN, false);
   std::vector<GemmF32Desc> left, right;
@@ -1118,6 +1123,9 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
         break;
       case Kind::Diag:
         S4_TRY(launch_diag(static_cast<const DiagDesc*>(d), L.count, int(L.extent), st));
+        break;
+      case Kind::RowDiag:
+        S4_TRY(launch_rowdiag(static_cast<const RowDiagDesc*>(d), L.count, int(L.extent), st));
         break;
       case Kind::Shift:
         S4_TRY(launch_shift(static_cast<const ShiftDesc*>(d), L.count, st));
