@@ -103,42 +103,76 @@ shampoo4_status launch_trsm(const TrsmDesc* d_desc, int count, int max_rows, cud
 }
 
 // ---- U = dequant(codes, scales) or I ------------------------------------
+// One CTA per row, each thread four consecutive columns: one 16-bit load of
+// codes, one scale (a 64-element block never splits a group of four), and
+// 16-byte stores of every output, so each warp writes 512 contiguous bytes.
+// Rows whose length is not a multiple of 4 take the element-wise path.
 __global__ void __launch_bounds__(256) k_basis(const BasisDesc* __restrict__ descs) {
   const BasisDesc& g = descs[blockIdx.y];
+  const int d = g.d, r = blockIdx.x;
+  if (r >= d) return;                                      // CTA-uniform
   __shared__ float level[16];
   if (threadIdx.x < 16) level[threadIdx.x] = level_f32(threadIdx.x);
   __syncthreads();
-  const int n = g.d * g.d;                       // d <= 1024: fits in 32 bits
-  const int e0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
-  if (e0 >= n) return;
-  int row = e0 / g.d, col = e0 - row * g.d;
-  float v[8];
-  if (!g.identity) {
-    uint32_t packed = 0;
-    const int nbytes = (n + 1) >> 1;
+  const int c0 = threadIdx.x * 4;
+  if (c0 >= d) return;
+  const int64_t e0 = int64_t(r) * d + c0;
+  if ((d & 3) == 0) {
+    float v[4];
+    if (g.identity) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      if ((e0 >> 1) + k < nbytes) packed |= uint32_t(g.codes[(e0 >> 1) + k]) << (8 * k);
-    dequantize8(packed, g.scales[e0 / kQuantBlock], level, v);
+      for (int k = 0; k < 4; ++k) v[k] = (r == c0 + k) ? 1.0f : 0.0f;
+    } else {
+      const uint32_t packed = *reinterpret_cast<const uint16_t*>(g.codes + (e0 >> 1));
+      const float sc = g.scales[e0 / kQuantBlock];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) v[k] = level[(packed >> (4 * k)) & 15u] * sc;
+    }
+    if (g.U) *reinterpret_cast<float4*>(g.U + e0) = make_float4(v[0], v[1], v[2], v[3]);
+    if (g.Uh) {
+      const float4 h = make_float4(tf32_rn(v[0]), tf32_rn(v[1]), tf32_rn(v[2]), tf32_rn(v[3]));
+      *reinterpret_cast<float4*>(g.Uh + e0) = h;
+      if (g.Ul)
+        *reinterpret_cast<float4*>(g.Ul + e0) =
+            make_float4(tf32_rn(v[0] - h.x), tf32_rn(v[1] - h.y), tf32_rn(v[2] - h.z), tf32_rn(v[3] - h.w));
+    }
+    if (g.Vh) {
+      const float4 m = *reinterpret_cast<const float4*>(g.mu + c0);
+      const float w0 = v[0] * m.x, w1 = v[1] * m.y, w2 = v[2] * m.z, w3 = v[3] * m.w;
+      const float4 h = make_float4(tf32_rn(w0), tf32_rn(w1), tf32_rn(w2), tf32_rn(w3));
+      *reinterpret_cast<float4*>(g.Vh + e0) = h;
+      if (g.Vl)
+        *reinterpret_cast<float4*>(g.Vl + e0) =
+            make_float4(tf32_rn(w0 - h.x), tf32_rn(w1 - h.y), tf32_rn(w2 - h.z), tf32_rn(w3 - h.w));
+    }
+    return;
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int i = e0 + e;
-    if (i >= n) break;
-    const float x = g.identity ? (row == col ? 1.0f : 0.0f) : v[e];
-    if (g.U) g.U[i] = x;
-    put_split(x, g.Uh, g.Ul, i);
-    if (g.Vh) put_split(x * g.mu[col], g.Vh, g.Vl, i);
-    if (++col == g.d) { col = 0; ++row; }
+  for (int k = 0; k < 4; ++k) {
+    const int c = c0 + k;
+    if (c >= d) break;
+    const int64_t e = e0 + k;
+    float x;
+    if (g.identity) {
+      x = (r == c) ? 1.0f : 0.0f;
+    } else {
+      const uint32_t byte = g.codes[e >> 1];
+      x = level[(e & 1) ? (byte >> 4) : (byte & 15u)] * g.scales[e / kQuantBlock];
+    }
+    if (g.U) g.U[e] = x;
+    put_split(x, g.Uh, g.Ul, e);
+    if (g.Vh) put_split(x * g.mu[c], g.Vh, g.Vl, e);
   }
 }
 
 shampoo4_status launch_basis(const BasisDesc* d_desc, int count, int64_t max_elems, cudaStream_t st) {
   if (count <= 0 || max_elems <= 0) return SHAMPOO4_OK;
-  int64_t ctas = (max_elems + 256 * 8 - 1) / (256 * 8);
+  int64_t max_d = 1;
+  while (max_d * max_d < max_elems) ++max_d;               // extent is the largest d * d
+  if (max_d > 1024) return SHAMPOO4_ERR_INVALID_ARG;
   for (int base = 0; base < count; base += 65535) {
     int c = count - base < 65535 ? count - base : 65535;
-    k_basis<<<dim3(unsigned(ctas), c), 256, 0, st>>>(d_desc + base);
+    k_basis<<<dim3(unsigned(max_d), c), 256, 0, st>>>(d_desc + base);
     S4_CUDA(cudaGetLastError());
   }
   return SHAMPOO4_OK;
