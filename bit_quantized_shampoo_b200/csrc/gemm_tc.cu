@@ -124,25 +124,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// 1-D bulk copies (TMA, no tensor map): global -> shared completing on an
-// mbarrier, shared -> global in per-thread bulk groups, and an L2 prefetch.
-// Addresses and sizes are multiples of 16 bytes.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-               ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
+// 16-byte asynchronous copies global -> shared (cp.async groups).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ float rn_tf32(float x) {
   uint32_t r;
@@ -158,12 +146,12 @@ struct TcCfg {
   static constexpr int kStages = STAGES;
   static constexpr int kSmem = kStage * kStages + 1024;         // + alignment slack
   // Epilogue staging, carved out of the pipeline buffers once the main loop
-  // is over: per warp two Cin buffers and three output buffers of 32 rows,
-  // row pitch 36 floats (16-byte aligned rows, conflict-free 16-byte
-  // accesses by lane = row).
+  // is over: per warp two Cin buffers and one transposing output buffer of
+  // 32 rows, row pitch 36 floats (16-byte aligned rows, conflict-free
+  // 16-byte accesses both by lane = row and by 8 lanes along a row).
   static constexpr int kPitch = 36;
   static constexpr int kRowBuf = 32 * kPitch * 4;
-  static constexpr int kEpiWarp = 5 * kRowBuf;
+  static constexpr int kEpiWarp = 3 * kRowBuf;
   static_assert(4 * kEpiWarp <= kStage * kStages, "epilogue staging fits the pipeline buffers");
   // The tensor cores' fp32 accumulation truncates: a long sum drifts low
   // (about 1e-8 K relative when its terms share a sign) and its rounding
@@ -260,7 +248,6 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t full_bar[Cfg::kStages], empty_bar[Cfg::kStages], done_bar;
-  __shared__ uint64_t cin_bar[4][2];                      // epilogue Cin buffers, per warp
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -271,10 +258,6 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&done_bar, 1);
-    for (int w = 0; w < 4; ++w) {
-      mbar_init(&cin_bar[w][0], 1);
-      mbar_init(&cin_bar[w][1], 1);
-    }
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -298,13 +281,6 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
       const TcOperand ga = g.a, gb = g.b;
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(ga.hi)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(gb.hi)) : "memory");
-      // Bring the tile of Cin into L2 while the main loop runs.
-      if (g.beta != 0.0f && ((reinterpret_cast<uintptr_t>(g.Cin) | uintptr_t(g.ldcin * 4)) & 15) == 0 &&
-          (g.N & 3) == 0) {
-        const uint32_t bytes = uint32_t(min(BN, g.N - n0)) * 4u;
-        const int rows = min(kBM, g.M - m0);
-        for (int r = 0; r < rows; ++r) bulk_prefetch_l2(g.Cin + int64_t(m0 + r) * g.ldcin + n0, bytes);
-      }
       if (SPLIT) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(ga.lo)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(gb.lo)) : "memory");
@@ -375,11 +351,12 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
       e.load(g, tabs, nparams);
       // Lane l of warp q holds accumulator row 32 q + l (TMEM lane), 32
       // columns per load.  When bases and leading dimensions are 16-byte
-      // aligned, Cin comes in and the outputs go out as one 1-D bulk copy
-      // per row segment (128 bytes), staged in this warp's rows of the idle
-      // pipeline buffers; otherwise each lane loads and stores its row
-      // directly.  The mirror of a symmetric product writes column segments,
-      // contiguous across the lanes.
+      // aligned, Cin comes in as one 1-D bulk copy per row segment (128
+      // bytes, double-buffered in this warp's rows of the idle pipeline
+      // buffers) and the outputs go out through a transposing staging row
+      // block, four full 128-byte lines per store instruction; otherwise each
+      // lane loads and stores its row directly.  The mirror of a symmetric
+      // product writes column segments, contiguous across the lanes.
       const int rbase = m0 + 32 * q;
       const int row = rbase + lane;
       const int nacc = kblocks < Cfg::kAcc ? kblocks : Cfg::kAcc;   // accumulators written
@@ -398,16 +375,22 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
       uint8_t* wbuf = smem + q * Cfg::kEpiWarp;
       const uint32_t wsm = smem_u32(wbuf);
       const uint32_t my_row = uint32_t(lane * Cfg::kPitch * 4);
-      int issued = -1, consumed = -1;                       // Cin chunks
       unsigned long long dev_fine = 0;                      // deviation sum, plan.h units
+      // Cin chunk i into buffer i & 1 with 16-byte cp.async pieces, four
+      // full 128-byte rows per warp instruction: lane l copies rows
+      // 4 t + l / 8 (t < 8), columns 4 (l % 8).  One group per chunk.
       auto issue_cin = [&](int i) {
-        const int cb = n0 + 32 * i;
-        const uint32_t bytes = uint32_t(min(32, e.N - cb)) * 4u;
-        uint64_t* bar = &cin_bar[q][i & 1];
-        if (lane == 0) mbar_expect_tx(bar, bytes * uint32_t(nrows));
-        __syncwarp();
-        if (row_ok) bulk_load(wsm + (i & 1) * Cfg::kRowBuf + my_row, e.Cin + int64_t(row) * e.ldcin + cb, bytes, bar);
-        issued = i;
+        const int cb = n0 + 32 * i, sr = lane >> 3, sc = 4 * (lane & 7);
+        if (cb + sc < e.N) {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int rr = 4 * t + sr;
+            if (rbase + rr < e.M)
+              cp_async16(wsm + (i & 1) * Cfg::kRowBuf + uint32_t((rr * Cfg::kPitch + sc) * 4),
+                         e.Cin + int64_t(rbase + rr) * e.ldcin + cb + sc);
+          }
+        }
+        cp_async_commit();
       };
       if (nrows > 0 && nchunks > 0) {
         if (cin_bulk) issue_cin(0);
@@ -415,9 +398,7 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
         for (int i = 0; i < nchunks; ++i) {
           const int c0 = 32 * i, cb = n0 + c0;
           if (cin_bulk && i + 1 < nchunks) {
-            // buffer (i + 1) & 1 was last read, through the generic proxy, in chunk i - 1
-            fence_proxy_async();
-            __syncwarp();
+            __syncwarp();                                   // buffer (i + 1) & 1: chunk i - 1's reads done
             issue_cin(i + 1);
           }
           uint32_t r[32];
@@ -434,11 +415,8 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
           for (int j = 0; j < 32; ++j) v[j] *= e.alpha;
           if (e.beta != 0.0f) {
             if (cin_bulk) {
-              if (!mbar_wait(&cin_bar[q][i & 1], (i >> 1) & 1)) {
-                atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
-                break;
-              }
-              consumed = i;
+              if (i + 1 < nchunks) cp_async_wait<1>(); else cp_async_wait<0>();
+              __syncwarp();                                 // every lane's pieces of chunk i visible
               if (row_ok) {
                 const float4* src = reinterpret_cast<const float4*>(wbuf + (i & 1) * Cfg::kRowBuf + my_row);
 #pragma unroll
@@ -472,27 +450,39 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
           // when the product is symmetric)
           const bool below = !e.symmetric || cb + 31 < rbase;   // whole chunk left of every row
           if (out_bulk && below) {
-            if (row_ok) {
-              bulk_wait_read();                             // staging rows free again
-              float4* oc = reinterpret_cast<float4*>(wbuf + 2 * Cfg::kRowBuf + my_row);
-              float4* oh = reinterpret_cast<float4*>(wbuf + 3 * Cfg::kRowBuf + my_row);
-              float4* ol = reinterpret_cast<float4*>(wbuf + 4 * Cfg::kRowBuf + my_row);
+            // Through this warp's staging rows: each lane writes its row
+            // segment as 16-byte pieces, then every store instruction takes
+            // 4 rows x 128 bytes (lane l: row 4 i + l / 8, columns 4 (l % 8)).
+            float* stage = reinterpret_cast<float*>(wbuf + 2 * Cfg::kRowBuf);
+            const int sr = lane >> 3, sc = 4 * (lane & 7);
+            const bool col_ok = cb + sc < e.N;
+#pragma unroll 1
+            for (int o = 0; o < 3; ++o) {
+              float* out = o == 0 ? e.C : (o == 1 ? e.Chi : e.Clo);
+              if (!out) continue;                             // warp-uniform
+              const int64_t ld = o == 0 ? e.ldc : e.ldh;
+              __syncwarp();                                   // previous output's reads done
 #pragma unroll
               for (int t = 0; t < 8; ++t) {
-                if (cb + 4 * t >= e.N) break;
-                const float a = v[4 * t], b = v[4 * t + 1], x = v[4 * t + 2], y = v[4 * t + 3];
-                const float4 h = make_float4(rn_tf32(a), rn_tf32(b), rn_tf32(x), rn_tf32(y));
-                oc[t] = e.out_round ? h : make_float4(a, b, x, y);
-                oh[t] = h;
-                ol[t] = make_float4(rn_tf32(a - h.x), rn_tf32(b - h.y), rn_tf32(x - h.z), rn_tf32(y - h.w));
+                float4 x = make_float4(v[4 * t], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
+                if (o == 1 || (o == 0 && e.out_round)) {
+                  x = make_float4(rn_tf32(x.x), rn_tf32(x.y), rn_tf32(x.z), rn_tf32(x.w));
+                } else if (o == 2) {
+                  x = make_float4(rn_tf32(x.x - rn_tf32(x.x)), rn_tf32(x.y - rn_tf32(x.y)),
+                                  rn_tf32(x.z - rn_tf32(x.z)), rn_tf32(x.w - rn_tf32(x.w)));
+                }
+                *reinterpret_cast<float4*>(stage + lane * Cfg::kPitch + 4 * t) = x;
               }
-              fence_proxy_async();                          // staged rows visible to the bulk copies
-              const uint32_t bytes = uint32_t(min(32, e.N - cb)) * 4u;
-              if (e.C) bulk_store(e.C + int64_t(row) * e.ldc + cb, wsm + 2 * Cfg::kRowBuf + my_row, bytes);
-              if (e.Chi) bulk_store(e.Chi + int64_t(row) * e.ldh + cb, wsm + 3 * Cfg::kRowBuf + my_row, bytes);
-              if (e.Clo) bulk_store(e.Clo + int64_t(row) * e.ldh + cb, wsm + 4 * Cfg::kRowBuf + my_row, bytes);
-              bulk_commit();
+              __syncwarp();
+#pragma unroll
+              for (int t = 0; t < 8; ++t) {
+                const int rr = 4 * t + sr;
+                if (rbase + rr < e.M && col_ok)
+                  *reinterpret_cast<float4*>(out + int64_t(rbase + rr) * ld + cb + sc) =
+                      *reinterpret_cast<const float4*>(stage + rr * Cfg::kPitch + sc);
+              }
             }
+            __syncwarp();
           } else if (row_ok) {
             if (out_vec) {
 #pragma unroll
@@ -529,11 +519,7 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
           for (int o = 16; o > 0; o >>= 1) dev_fine += __shfl_xor_sync(0xffffffffu, dev_fine, o);
           if (lane == 0 && dev_fine) atomicAdd(e.devsq, dev_fine);
         }
-        // Before the buffers are released: this lane's bulk stores done, and
-        // (after an abort) every Cin copy that was issued has landed.
-        bulk_wait_all();
-        for (int i = consumed + 1; i <= issued; ++i)
-          if (!mbar_wait(&cin_bar[q][i & 1], (i >> 1) & 1)) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+        cp_async_wait<0>();                                 // nothing in flight into the buffers
       }
     }
   }
