@@ -132,6 +132,35 @@ STAGE_BOUND = {
 }
 
 
+# DRAM bytes (read + write) of ONE launch of a stage's tensor-core GEMM per
+# element of the factors it processes, from the ncu capture summarised in
+# profiles/k_gemm_tc_4096x4096_factors.md (32 factors of 1024 x 1024).  A
+# launch over other factors of the same kind moves the same bytes per
+# element.  Valid only for the GEMM source it was taken on: the figure is
+# dropped (traffic = null) when gemm_tc.cu or tc.h has changed since.
+TRAFFIC_SOURCE_SHA = "cc56304ced2846b2"
+TRAFFIC_PER_ELEMENT = {"stats_gemm": 6.587, "bjorck_gram": 10.367, "bjorck_update": 22.917,
+                       "subspace": 32.19, "qr_gram": 18.92}
+
+
+def gemm_source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm_tc.cu", "tc.h"):
+        with open(os.path.join(ROOT, "bit_quantized_shampoo_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def stage_traffic(stage, factor_elems):
+    """Per-launch DRAM traffic of the stage's GEMM for factors totalling
+    factor_elems elements, or None when no capture covers it."""
+    b = TRAFFIC_PER_ELEMENT.get(stage)
+    if b is None or gemm_source_sha() != TRAFFIC_SOURCE_SHA:
+        return None
+    return b * factor_elems
+
+
 def stage_roofline(name, st, pk, pk_src, sustained=True):
     bound = STAGE_BOUND.get(name, "latency")
     ms = st["ms"]
@@ -321,7 +350,11 @@ def main():
     ranked = sorted(stages, key=lambda k: -stages[k]["ms"])
     dom = next(k for k in ranked if STAGE_BOUND.get(k, "latency") != "latency")
     roof = stage_roofline(dom, stages[dom], pk, pk_src)
-    roof["traffic"] = None
+    factor_elems = sum(int(b[3]) ** 2 + int(b[4]) ** 2 for b in (sh.block_info(k) for k in range(sh.nblocks)))
+    roof["traffic"] = stage_traffic(dom, factor_elems)
+    if roof["traffic"] is not None:
+        roof["traffic_note"] = ("dram read+write bytes of one launch of this stage's GEMM, scaled from an ncu capture "
+                                "on 32 factors of 1024x1024 by factor elements")
     others = [stage_roofline(k, stages[k], pk, pk_src) for k in ranked[:8] if k != dom]
 
     line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
