@@ -146,7 +146,9 @@ __device__ __forceinline__ double ld_any(const void* p, bool f64, int64_t idx) {
 // whose problems are all skipped (the fp64 fallback of the QR) costs only
 // its flag reads.
 __global__ void __launch_bounds__(kF64Threads)
-k_gemm_f64(const GemmF64Desc* __restrict__ descs, int count, int max_tiles) {
+k_gemm_f64(const GemmF64Desc* __restrict__ descs, int count, int max_tiles,
+           const uint32_t* __restrict__ guard) {
+  if (guard && *guard == 0u) return;                      // no factor needs this launch
   __shared__ double As[kF64BK][kF64Tile + 1];
   __shared__ double Bs[kF64BK][kF64Tile + 1];
   const int tid = threadIdx.x;
@@ -226,11 +228,12 @@ k_gemm_f64(const GemmF64Desc* __restrict__ descs, int count, int max_tiles) {
   }
 }
 
-shampoo4_status launch_gemm_f64(const GemmF64Desc* d_desc, int count, int max_tiles, cudaStream_t st) {
+shampoo4_status launch_gemm_f64(const GemmF64Desc* d_desc, int count, int max_tiles, cudaStream_t st,
+                                const uint32_t* guard) {
   if (count <= 0 || max_tiles <= 0) return SHAMPOO4_OK;
   const int64_t items = int64_t(count) * max_tiles;
   const unsigned ctas = unsigned(items < 148 * 8 ? items : 148 * 8);
-  k_gemm_f64<<<ctas, kF64Threads, 0, st>>>(d_desc, count, max_tiles);
+  k_gemm_f64<<<ctas, kF64Threads, 0, st>>>(d_desc, count, max_tiles, guard);
   S4_CUDA(cudaGetLastError());
   return SHAMPOO4_OK;
 }

@@ -9,7 +9,8 @@ namespace s4 {
 constexpr int kPanel = 64;     // Cholesky / triangular-solve panel width
 
 // ---- Cholesky of a jb x jb diagonal block, lower, in place ---------------
-__global__ void __launch_bounds__(256) k_potrf(const PotrfDesc* __restrict__ descs) {
+__global__ void __launch_bounds__(256) k_potrf(const PotrfDesc* __restrict__ descs, const uint32_t* __restrict__ guard) {
+  if (guard && *guard == 0u) return;                      // no factor needs this launch
   const PotrfDesc& g = descs[blockIdx.x];
   const int jb = g.jb;
   if (jb <= 0 || (g.skip && *g.skip)) return;
@@ -48,9 +49,9 @@ __global__ void __launch_bounds__(256) k_potrf(const PotrfDesc* __restrict__ des
   }
 }
 
-shampoo4_status launch_potrf(const PotrfDesc* d_desc, int count, cudaStream_t st) {
+shampoo4_status launch_potrf(const PotrfDesc* d_desc, int count, cudaStream_t st, const uint32_t* guard) {
   if (count <= 0) return SHAMPOO4_OK;
-  k_potrf<<<count, 256, 0, st>>>(d_desc);
+  k_potrf<<<count, 256, 0, st>>>(d_desc, guard);
   S4_CUDA(cudaGetLastError());
   return SHAMPOO4_OK;
 }
@@ -61,7 +62,9 @@ constexpr unsigned kWorkCtas = 148 * 8;     // grid of the work-item loops
 
 // Work items (row chunk, problem), looped over by a fixed grid so that a
 // launch whose problems are all skipped costs only its flag reads.
-__global__ void __launch_bounds__(256) k_trsm(const TrsmDesc* __restrict__ descs, int count, int chunks) {
+__global__ void __launch_bounds__(256) k_trsm(const TrsmDesc* __restrict__ descs, int count, int chunks,
+                                              const uint32_t* __restrict__ guard) {
+  if (guard && *guard == 0u) return;                      // no factor needs this launch
   __shared__ double L[kPanel][kPanel + 1];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int w = blockIdx.x; w < count * chunks; w += gridDim.x) {
@@ -93,11 +96,12 @@ __global__ void __launch_bounds__(256) k_trsm(const TrsmDesc* __restrict__ descs
   }
 }
 
-shampoo4_status launch_trsm(const TrsmDesc* d_desc, int count, int max_rows, cudaStream_t st) {
+shampoo4_status launch_trsm(const TrsmDesc* d_desc, int count, int max_rows, cudaStream_t st,
+                            const uint32_t* guard) {
   if (count <= 0 || max_rows <= 0) return SHAMPOO4_OK;
   const int chunks = (max_rows + kTrsmRowsPerCta - 1) / kTrsmRowsPerCta;
   const int64_t items = int64_t(count) * chunks;
-  k_trsm<<<unsigned(items < kWorkCtas ? items : kWorkCtas), 256, 0, st>>>(d_desc, count, chunks);
+  k_trsm<<<unsigned(items < kWorkCtas ? items : kWorkCtas), 256, 0, st>>>(d_desc, count, chunks, guard);
   S4_CUDA(cudaGetLastError());
   return SHAMPOO4_OK;
 }
@@ -260,7 +264,8 @@ shampoo4_status launch_scan(const ScanDesc* d_desc, int count, int64_t max_rows,
 }
 
 // ---- shifted Gram diagonal (fp64) -----------------------------------------
-__global__ void __launch_bounds__(256) k_shift(const ShiftDesc* __restrict__ descs) {
+__global__ void __launch_bounds__(256) k_shift(const ShiftDesc* __restrict__ descs, const uint32_t* __restrict__ guard) {
+  if (guard && *guard == 0u) return;                      // no factor needs this launch
   const ShiftDesc& g = descs[blockIdx.x];
   if (g.skip && *g.skip) return;
   __shared__ double part[256];
@@ -277,9 +282,9 @@ __global__ void __launch_bounds__(256) k_shift(const ShiftDesc* __restrict__ des
   for (int i = threadIdx.x; i < g.d; i += blockDim.x) g.W[int64_t(i) * g.ld + i] += s;
 }
 
-shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st) {
+shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st, const uint32_t* guard) {
   if (count <= 0) return SHAMPOO4_OK;
-  k_shift<<<count, 256, 0, st>>>(d_desc);
+  k_shift<<<count, 256, 0, st>>>(d_desc, guard);
   S4_CUDA(cudaGetLastError());
   return SHAMPOO4_OK;
 }
@@ -351,6 +356,7 @@ __global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ 
     *g.fail = 1u;
     if (g.clear) {                        // fp32 attempt: fall back to fp64
       *g.clear = 0u;
+      if (g.any_fallback) *g.any_fallback = 1u;
       if (g.gflags) atomicOr(g.gflags, SHAMPOO4_FLAG_QR_FALLBACK);
     } else if (g.gflags) {
       atomicOr(g.gflags, SHAMPOO4_FLAG_REFRESH_FAILED);
@@ -495,7 +501,9 @@ shampoo4_status launch_split(const SplitDesc* d_desc, int count, int64_t max_ele
 
 // ---- fp64 -> fp32 ----------------------------------------------------------
 constexpr int64_t kConvertChunk = 1 << 16;
-__global__ void __launch_bounds__(256) k_convert(const ConvertDesc* __restrict__ descs, int count, int chunks) {
+__global__ void __launch_bounds__(256) k_convert(const ConvertDesc* __restrict__ descs, int count, int chunks,
+                                                 const uint32_t* __restrict__ guard) {
+  if (guard && *guard == 0u) return;                      // no factor needs this launch
   for (int w = blockIdx.x; w < count * chunks; w += gridDim.x) {
     const ConvertDesc& g = descs[w / chunks];
     const int64_t lo = int64_t(w % chunks) * kConvertChunk;
@@ -509,11 +517,12 @@ __global__ void __launch_bounds__(256) k_convert(const ConvertDesc* __restrict__
   }
 }
 
-shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st) {
+shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st,
+                               const uint32_t* guard) {
   if (count <= 0 || max_elems <= 0) return SHAMPOO4_OK;
   const int chunks = int((max_elems + kConvertChunk - 1) / kConvertChunk);
   const int64_t items = int64_t(count) * chunks;
-  k_convert<<<unsigned(items < kWorkCtas ? items : kWorkCtas), 256, 0, st>>>(d_desc, count, chunks);
+  k_convert<<<unsigned(items < kWorkCtas ? items : kWorkCtas), 256, 0, st>>>(d_desc, count, chunks, guard);
   S4_CUDA(cudaGetLastError());
   return SHAMPOO4_OK;
 }

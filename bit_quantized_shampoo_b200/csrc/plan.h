@@ -151,6 +151,8 @@ struct PotrfDescF {
                               // below this counts as a breakdown; 0 = only
                               // non-positive or non-finite pivots do
   int32_t pad2_;
+  uint32_t* any_fallback;     // optional: set to 1 when the block sends its
+                              // factor to the fp64 redo (guard of those launches)
 };
 
 // W_ii <- W_ii (1 + coef) for i < d: the shift of the first Cholesky-QR
@@ -229,20 +231,27 @@ struct GateDesc {
 // ---- launchers (each enqueues one launch over `count` descriptors) -------
 shampoo4_status launch_gemm_f32(const GemmF32Desc* d_desc, int count, int max_tiles,
                                 const PtrEntry* tabs, int nparams, cudaStream_t st);
+// guard (optional, one word for the whole launch): the launch does nothing
+// while *guard == 0 -- the fp64 QR passes run only when some factor needs
+// them.
 shampoo4_status launch_gemm_f64(const GemmF64Desc* d_desc, int count, int max_tiles,
-                                cudaStream_t st);
-shampoo4_status launch_potrf(const PotrfDesc* d_desc, int count, cudaStream_t st);
-shampoo4_status launch_trsm(const TrsmDesc* d_desc, int count, int max_rows, cudaStream_t st);
+                                cudaStream_t st, const uint32_t* guard = nullptr);
+shampoo4_status launch_potrf(const PotrfDesc* d_desc, int count, cudaStream_t st,
+                             const uint32_t* guard = nullptr);
+shampoo4_status launch_trsm(const TrsmDesc* d_desc, int count, int max_rows, cudaStream_t st,
+                            const uint32_t* guard = nullptr);
 shampoo4_status launch_basis(const BasisDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_rayleigh(const RayleighDesc* d_desc, int count, int max_d, cudaStream_t st);
 shampoo4_status launch_mu(const MuDesc* d_desc, int count, int max_d, float eps, cudaStream_t st);
 shampoo4_status launch_scan(const ScanDesc* d_desc, int count, int64_t max_rows,
                             const PtrEntry* tabs, int nparams, uint32_t* flags, cudaStream_t st);
-shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st);
+shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st,
+                             const uint32_t* guard = nullptr);
 shampoo4_status launch_potrf_f(const PotrfDescF* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_shift_f(const ShiftDescF* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_split(const SplitDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
-shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
+shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st,
+                               const uint32_t* guard = nullptr);
 shampoo4_status launch_clear(const ClearDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_gate(const GateDesc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaStream_t st);

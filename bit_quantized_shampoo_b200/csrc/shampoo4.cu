@@ -39,6 +39,7 @@ struct Launch {
   int count;
   int64_t extent;      // max tiles / rows / elements, per kind
   double flops = 0, bytes = 0;   // algorithmic work of the launch
+  size_t guard_off = SIZE_MAX;   // workspace word gating the whole launch (fp64 QR passes)
   // Pack launches carry host-side tensor lists instead of descriptors.
   std::vector<const float*> px;
   std::vector<int64_t> pn;
@@ -86,7 +87,8 @@ struct shampoo4_ctx {
   size_t state_bytes = 0, ws_bytes = 0;
   // workspace regions
   size_t ws_flags = 0, ws_tabs = 0, ws_fail = 0, ws_bflag = 0, ws_maps = 0, ws_nmaps = 0;
-  size_t ws_tcbad = 0, ws_tcgood = 0, ws_devsq = 0, ws_skip3 = 0;
+  size_t ws_tcbad = 0, ws_tcgood = 0, ws_devsq = 0, ws_skip3 = 0, ws_fbany = 0;
+  bool any_simt = false;                 // some factor always takes the fp64 QR
   size_t ws_desc = 0, ws_desc_bytes = 0;
   // programs
   std::vector<Launch> prog_stats, prog_refresh_first, prog_refresh, prog_precond;
@@ -154,6 +156,7 @@ shampoo4_status plan(shampoo4_ctx* h) {
       f.side = side;
       f.d = side == 0 ? h->blocks[k].m : h->blocks[k].n;
       f.tc = tc_dim(f.d);
+      if (!f.tc) h->any_simt = true;
       size_t dd = size_t(f.d) * f.d;
       f.st_S = take(st, 4 * dd);
       f.st_codes = take(st, (dd + 1) / 2);
@@ -172,6 +175,7 @@ shampoo4_status plan(shampoo4_ctx* h) {
   h->ws_tcgood = take(ws, 4 * h->factors.size());
   h->ws_devsq = take(ws, 8 * h->factors.size());
   h->ws_skip3 = take(ws, 4 * h->factors.size());
+  h->ws_fbany = take(ws, 4);
   h->ws_bflag = take(ws, 4 * h->blocks.size());
   for (FactorPlan& f : h->factors) {
     size_t dd = size_t(f.d) * f.d;
@@ -232,6 +236,7 @@ struct Builder {
   uint8_t* stb;       // device state base
   bool encode;        // false: only count tensor maps (sizing pass)
   int tag = 0;        // stage label applied to the launches emitted next
+  size_t guard = SIZE_MAX;   // guard word applied to the launches emitted next
   shampoo4_status err = SHAMPOO4_OK;
   std::map<std::tuple<uintptr_t, int, int, int, int>, size_t> map_index;
 
@@ -254,6 +259,7 @@ struct Builder {
     L.extent = extent;
     L.flops = flops;
     L.bytes = bytes;
+    L.guard_off = guard;
     prog.push_back(std::move(L));
   }
   float* wf(size_t off) const { return reinterpret_cast<float*>(ws + off); }
@@ -657,7 +663,7 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
       po.push_back({W + int64_t(j) * d + j, d, jb, 0, b.tcbad(i), b.gflags(), b.tcgood(i),
                     Th + int64_t(j) * d + j, Tl + int64_t(j) * d + j,
                     b.wf(f.ws_Ih) + int64_t(j) * kPanelW, b.wf(f.ws_Il) + int64_t(j) * kPanelW,
-                    gated ? b.skip3(i) : nullptr, gated ? kLastPassPivot : 0.0f, 0});
+                    gated ? b.skip3(i) : nullptr, gated ? kLastPassPivot : 0.0f, 0, b.wu(h->ws_fbany)});
       fl_po += 2.0 * double(jb) * jb * jb / 3.0;
       if (rest <= 0) continue;
       TcGemmDesc t = gemmtc(rest, jb, jb, 1.0f, 0.0f);     // L21 = W21 L11^-T (in the split, in place)
@@ -892,9 +898,13 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
     build_cholqr_tc(b, prog, Xc, Xc, false, true);
     std::vector<char> use_any(nf);
     for (size_t i = 0; i < nf; ++i) use_any[i] = use_simt[i] || use_fb[i];
+    // fp64 passes: the whole launches are skipped unless some factor takes
+    // them (a CUDA-core factor, or a tensor-core factor that broke down)
+    b.guard = h->ws_fbany;
     build_cholqr_pass(b, prog, use_any, a1, o1, none, none, sk, true);
     build_cholqr_pass(b, prog, use_any, a2, o2, none, none, sk, false);
     build_cholqr_pass(b, prog, use_any, a3, o3, q3h, q3l, sk, false);
+    b.guard = SIZE_MAX;
   }
   for (size_t i = 0; i < nf; ++i) {
     const size_t off = size_t(reinterpret_cast<uint8_t*>(Qf[i]) - b.ws);
@@ -1070,6 +1080,8 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
   uint32_t* gflags = reinterpret_cast<uint32_t*>(h->d_ws + h->ws_flags);
   for (const Launch& L : prog) {
     const void* d = h->d_ws + h->ws_desc + L.desc_off;
+    const uint32_t* guard =
+        L.guard_off == SIZE_MAX ? nullptr : reinterpret_cast<const uint32_t*>(h->d_ws + L.guard_off);
     shampoo4_ctx::Rec rec{L.tag, nullptr, nullptr, L.flops, L.bytes, 1};
     if (h->timing) {
       rec.e0 = take_event(h);
@@ -1082,13 +1094,13 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
         S4_TRY(launch_gemm_f32(static_cast<const GemmF32Desc*>(d), L.count, int(L.extent), tabs, np, st));
         break;
       case Kind::GemmF64:
-        S4_TRY(launch_gemm_f64(static_cast<const GemmF64Desc*>(d), L.count, int(L.extent), st));
+        S4_TRY(launch_gemm_f64(static_cast<const GemmF64Desc*>(d), L.count, int(L.extent), st, guard));
         break;
       case Kind::Potrf:
-        S4_TRY(launch_potrf(static_cast<const PotrfDesc*>(d), L.count, st));
+        S4_TRY(launch_potrf(static_cast<const PotrfDesc*>(d), L.count, st, guard));
         break;
       case Kind::Trsm:
-        S4_TRY(launch_trsm(static_cast<const TrsmDesc*>(d), L.count, int(L.extent), st));
+        S4_TRY(launch_trsm(static_cast<const TrsmDesc*>(d), L.count, int(L.extent), st, guard));
         break;
       case Kind::Basis:
         S4_TRY(launch_basis(static_cast<const BasisDesc*>(d), L.count, L.extent, st));
@@ -1128,10 +1140,10 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
         S4_TRY(launch_rowdiag(static_cast<const RowDiagDesc*>(d), L.count, int(L.extent), st));
         break;
       case Kind::Shift:
-        S4_TRY(launch_shift(static_cast<const ShiftDesc*>(d), L.count, st));
+        S4_TRY(launch_shift(static_cast<const ShiftDesc*>(d), L.count, st, guard));
         break;
       case Kind::Convert:
-        S4_TRY(launch_convert(static_cast<const ConvertDesc*>(d), L.count, L.extent, st));
+        S4_TRY(launch_convert(static_cast<const ConvertDesc*>(d), L.count, L.extent, st, guard));
         break;
       case Kind::Pack:
         S4_TRY(launch_pack(L.px.data(), L.pn.data(), L.count, L.pcodes.data(), L.pscales.data(), st,
@@ -1312,6 +1324,7 @@ extern "C" shampoo4_status shampoo4_refresh_roots(shampoo4_handle h, shampoo4_st
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_tcbad, 0, 4 * h->factors.size(), st));
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_tcgood, 1, 4 * h->factors.size(), st));
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_devsq, 0, 8 * h->factors.size(), st));
+  S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_fbany, h->any_simt ? 1 : 0, 4, st));
   const bool first = !h->has_basis;
   S4_TRY(run(h, first ? h->prog_refresh_first : h->prog_refresh, st));
   h->last_refresh_first = first;
