@@ -235,6 +235,25 @@ def cpu_sample(w, nblocks_sample: int, seed_step: int = 1):
     return t_total / len(pick), len(blocks), desc, threads
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(ms, device=None):
+    """The job's time: every rank passes its own elapsed milliseconds and
+    gets the slowest rank's.  Unchanged in a single process."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world, units_per_rank, ms):
+    """Whole-job throughput: every rank processed units_per_rank units (weak
+    scaling, one replica of the workload per rank) in the job's time ms."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 # ------------------------------------------------------------------ main
 def run_reference(args, rank, world):
     if rank != 0:
@@ -321,13 +340,9 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
     ms_per_step = ms / args.steps
-    value = world * args.steps / (ms / 1e3)
+    value = job_rate(world, args.steps, ms)
 
     # per-stage times measured live over the timed region
     stages = {}
@@ -387,14 +402,10 @@ def main():
                 h.copy_(d, non_blocking=True)
         e3.record(stream)
         torch.cuda.synchronize()
-        ems = e2.elapsed_time(e3)
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(e2.elapsed_time(e3), dev)
         bi = sum(h.numel() * 4 for h in host_g)
         bo = sum(h.numel() * 4 for h in host_out)
-        line["e2e"] = {"value": world * k / (ems / 1e3), "unit": "steps/s", "h2d_bytes_per_step": bi,
+        line["e2e"] = {"value": job_rate(world, k, ems), "unit": "steps/s", "h2d_bytes_per_step": bi,
                        "d2h_bytes_per_step": bo}
 
     # stand-alone codec bandwidth on eigenvector-shaped tensors of the workload's size
