@@ -294,65 +294,92 @@ shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st
 // thread c forms column c of L^-1 by forward substitution.
 constexpr int kPotrfFSmem = 2 * kPanel * (kPanel + 1) * 8;
 
+// One 64 x 64 block per CTA, fp64 in shared memory, 256 threads as a
+// 16 x 16 grid (thread (ty, tx) owns rows ty + 16 i and columns tx + 16 j).
+// Both loops keep columns (or rows) unscaled while they are read -- the
+// LDL^T form: A[r][s] -= A[r][c] A[s][c] / A[c][c] -- so that a step reads
+// only values no thread writes in that step, and one barrier per step
+// suffices; the square roots and divisions are applied once at the end.
+// Padding beyond jb is the identity in the factorization and zero in the
+// written inverse.
 __global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ descs) {
   const PotrfDescF& g = descs[blockIdx.x];
   const int jb = g.jb;
   if (jb <= 0 || *g.fail || (g.skip && *g.skip)) return;
   extern __shared__ double sm_potrf[];
-  double (*L)[kPanel + 1] = reinterpret_cast<double (*)[kPanel + 1]>(sm_potrf);
-  double (*Li)[kPanel + 1] = reinterpret_cast<double (*)[kPanel + 1]>(sm_potrf + kPanel * (kPanel + 1));
+  double (*A)[kPanel + 1] = reinterpret_cast<double (*)[kPanel + 1]>(sm_potrf);
+  double (*X)[kPanel + 1] = reinterpret_cast<double (*)[kPanel + 1]>(sm_potrf + kPanel * (kPanel + 1));
   __shared__ int bad;
-  for (int e = threadIdx.x; e < jb * jb; e += blockDim.x) {
-    int r = e / jb, c = e % jb;
-    L[r][c] = (c <= r) ? double(g.A[int64_t(r) * g.ld + c]) : 0.0;
+  const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
+  for (int r = t >> 6; r < kPanel; r += 4) {
+    const int c = t & 63;
+    A[r][c] = (r < jb && c <= r) ? double(g.A[int64_t(r) * g.ld + c]) : (r == c ? 1.0 : 0.0);
+    X[r][c] = (r == c) ? 1.0 : 0.0;
   }
-  if (threadIdx.x == 0) bad = 0;
+  if (t == 0) bad = 0;
   __syncthreads();
+  // factorization: after step c, A[c][c] is the pivot d_c and column c
+  // below it holds L[:, c] sqrt(d_c)
   for (int c = 0; c < jb; ++c) {
-    if (threadIdx.x == 0) {
-      double p = L[c][c];
-      if (!(p > double(g.min_pivot)) || !isfinite(p)) { bad = 1; p = 1.0; }
-      L[c][c] = sqrt(p);
+    double p = A[c][c];
+    if (!(p > double(g.min_pivot)) || !isfinite(p)) {
+      if (t == 0) bad = 1;
+      p = 1.0;
     }
-    __syncthreads();
-    double piv = L[c][c];
-    for (int r = c + 1 + threadIdx.x; r < jb; r += blockDim.x) L[r][c] /= piv;
-    __syncthreads();
-    const int w = jb - c - 1;
-    for (int e = threadIdx.x; e < w * w; e += blockDim.x) {
-      int r = c + 1 + e / w, s = c + 1 + e % w;
-      if (s <= r) L[r][s] -= L[r][c] * L[s][c];
-    }
-    __syncthreads();
-  }
-  for (int e = threadIdx.x; e < jb * jb; e += blockDim.x) {
-    int r = e / jb, c = e % jb;
-    if (c <= r) {
-      const float v = float(L[r][c]);
-      g.A[int64_t(r) * g.ld + c] = v;
-      put_split(v, g.oh, g.ol, int64_t(r) * g.ld + c);
-    }
-  }
-  if (g.ih) {
-    if (threadIdx.x < kPanel) {
-      const int c = threadIdx.x;
-      for (int r = 0; r < kPanel; ++r) Li[r][c] = 0.0;
-      if (c < jb) {
-        Li[c][c] = 1.0 / L[c][c];
-        for (int r = c + 1; r < jb; ++r) {
-          double acc = 0.0;
-          for (int k = c; k < r; ++k) acc = fma(L[r][k], Li[k][c], acc);
-          Li[r][c] = -acc / L[r][r];
-        }
+    const double ip = 1.0 / p;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = ty + 16 * i;
+      if (r <= c || r >= jb) continue;
+      const double arc = A[r][c] * ip;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int s2 = tx + 16 * jj;
+        if (s2 > c && s2 <= r) A[r][s2] = fma(-arc, A[s2][c], A[r][s2]);
       }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < kPanel * kPanel; e += blockDim.x) {
-      const int r = e / kPanel, c = e % kPanel;
-      put_split(float(Li[r][c]), g.ih, g.il, e);
+  }
+  // pivots: breakdown leaves 1 so that nothing below is NaN
+  for (int c = t; c < kPanel; c += blockDim.x) {
+    const double p = A[c][c];
+    if (c < jb && (!(p > double(g.min_pivot)) || !isfinite(p))) A[c][c] = 1.0;
+  }
+  __syncthreads();
+  // inverse of the unit-lower factor U (U[r][k] = A[r][k] / d_k, r > k):
+  // X <- U^-1 by rows, right-looking; then L^-1 = D^-1/2 U^-1
+  for (int k = 0; k < jb; ++k) {
+    const double ik = 1.0 / A[k][k];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = ty + 16 * i;
+      if (r <= k || r >= jb) continue;
+      const double urk = A[r][k] * ik;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int c2 = tx + 16 * jj;
+        if (c2 <= k) X[r][c2] = fma(-urk, X[k][c2], X[r][c2]);
+      }
+    }
+    __syncthreads();
+  }
+  // write L = U D^1/2 (fp32 + split) and L^-1 = D^-1/2 U^-1 (split, zero
+  // outside jb x jb)
+  for (int r = t >> 6; r < kPanel; r += 4) {
+    const int c = t & 63;
+    const double sr = sqrt(A[r][r]);
+    if (r < jb && c <= r) {
+      const double l = (c == r) ? sr : A[r][c] / sqrt(A[c][c]);
+      const float v = float(l);
+      g.A[int64_t(r) * g.ld + c] = v;
+      put_split(v, g.oh, g.ol, int64_t(r) * g.ld + c);
+    }
+    if (g.ih) {
+      const float xi = (r < jb && c <= r) ? float(X[r][c] / sr) : 0.0f;
+      put_split(xi, g.ih, g.il, int64_t(r) * kPanel + c);
     }
   }
-  if (threadIdx.x == 0 && bad) {
+  if (t == 0 && bad) {
     *g.fail = 1u;
     if (g.clear) {                        // fp32 attempt: fall back to fp64
       *g.clear = 0u;
