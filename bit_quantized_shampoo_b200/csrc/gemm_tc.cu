@@ -231,6 +231,192 @@ struct EpiArgs {
   }
 };
 
+// Epilogue of one output tile (rows m0.., columns n0..) by an epilogue warp
+// of TMEM lane quarter q, for the tile's 32-column chunks [i_lo, i_hi):
+// reads the tile's accumulator(s) at TMEM column tacc, stages through this
+// warp's staging rows wbuf (Cfg::kEpiWarp bytes), writes every requested
+// output.
+template <int BN, bool SPLIT, int STAGES>
+__device__ __forceinline__ void epilogue_tile(const TcGemmDesc& g, const PtrEntry* __restrict__ tabs, int nparams,
+                                              int m0, int n0, int kblocks, uint32_t tacc, int q, int lane,
+                                              uint8_t* wbuf, int i_lo = 0, int i_hi = BN / 32) {
+  using Cfg = TcCfg<BN, SPLIT, STAGES>;
+  EpiArgs e;
+  e.load(g, tabs, nparams);
+  // Lane l of warp q holds accumulator row 32 q + l (TMEM lane), 32
+  // columns per load.  When bases and leading dimensions are 16-byte
+  // aligned, Cin comes in by 16-byte cp.async pieces (four full rows per
+  // warp instruction, double-buffered in the staging rows) and the outputs
+  // go out through a transposing staging row block, four full 128-byte
+  // lines per store instruction; otherwise each lane loads and stores its
+  // row directly.  The mirror of a symmetric product writes column
+  // segments, contiguous across the lanes.
+  const int rbase = m0 + 32 * q;
+  const int row = rbase + lane;
+  const int nacc = kblocks < Cfg::kAcc ? kblocks : Cfg::kAcc;   // accumulators written
+  const bool row_ok = row < e.M;
+  const int nrows = min(32, e.M - rbase);
+  const int ncols = min(BN, e.N - n0);
+  const int nchunks = ncols > 0 ? (ncols + 31) / 32 : 0;
+  const int i_end = i_hi < nchunks ? i_hi : nchunks;
+  const bool cin_bulk = e.beta != 0.0f &&
+                        ((reinterpret_cast<uintptr_t>(e.Cin) | uintptr_t(e.ldcin * 4)) & 15) == 0 &&
+                        (e.N & 3) == 0;
+  const bool out_bulk = ((reinterpret_cast<uintptr_t>(e.C) | uintptr_t(e.ldc * 4) |
+                          reinterpret_cast<uintptr_t>(e.Chi) | reinterpret_cast<uintptr_t>(e.Clo) |
+                          uintptr_t(e.ldh * 4)) & 15) == 0 &&
+                        (e.N & 3) == 0;
+  const bool out_vec = out_bulk;                        // same alignment conditions
+  const uint32_t wsm = smem_u32(wbuf);
+  const uint32_t my_row = uint32_t(lane * Cfg::kPitch * 4);
+  unsigned long long dev_fine = 0;                      // deviation sum, plan.h units
+  // Cin chunk i into buffer i & 1 with 16-byte cp.async pieces, four
+  // full 128-byte rows per warp instruction: lane l copies rows
+  // 4 t + l / 8 (t < 8), columns 4 (l % 8).  One group per chunk.
+  auto issue_cin = [&](int i) {
+    const int cb = n0 + 32 * i, sr = lane >> 3, sc = 4 * (lane & 7);
+    if (cb + sc < e.N) {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int rr = 4 * t + sr;
+        if (rbase + rr < e.M)
+          cp_async16(wsm + (i & 1) * Cfg::kRowBuf + uint32_t((rr * Cfg::kPitch + sc) * 4),
+                     e.Cin + int64_t(rbase + rr) * e.ldcin + cb + sc);
+      }
+    }
+    cp_async_commit();
+  };
+  if (nrows > 0 && i_lo < i_end) {
+    if (cin_bulk) issue_cin(i_lo);
+#pragma unroll 1
+    for (int i = i_lo; i < i_end; ++i) {
+      const int c0 = 32 * i, cb = n0 + c0;
+      if (cin_bulk && i + 1 < i_end) {
+        __syncwarp();                                   // buffer (i + 1) & 1: chunk i - 1's reads done
+        issue_cin(i + 1);
+      }
+      uint32_t r[32];
+      tmem_ld32(tacc + (uint32_t(32 * q) << 16) + uint32_t(c0), r);
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+      for (int a = 1; a < nacc; ++a) {                  // the other accumulators, added with RN
+        tmem_ld32(tacc + (uint32_t(32 * q) << 16) + uint32_t(a * BN + c0), r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += __uint_as_float(r[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= e.alpha;
+      if (e.beta != 0.0f) {
+        if (cin_bulk) {
+          if (i + 1 < i_end) cp_async_wait<1>(); else cp_async_wait<0>();
+          __syncwarp();                                 // every lane's pieces of chunk i visible
+          if (row_ok) {
+            const float4* src = reinterpret_cast<const float4*>(wbuf + (i & 1) * Cfg::kRowBuf + my_row);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+              if (cb + 4 * t >= e.N) break;
+              const float4 x = src[t];
+              v[4 * t + 0] = fmaf(e.beta, x.x, v[4 * t + 0]);
+              v[4 * t + 1] = fmaf(e.beta, x.y, v[4 * t + 1]);
+              v[4 * t + 2] = fmaf(e.beta, x.z, v[4 * t + 2]);
+              v[4 * t + 3] = fmaf(e.beta, x.w, v[4 * t + 3]);
+            }
+          }
+        } else if (row_ok) {
+          const float* src = e.Cin + int64_t(row) * e.ldcin + cb;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (cb + j < e.N) v[j] = fmaf(e.beta, __ldg(src + j), v[j]);
+        }
+      }
+      if (e.devsq && row_ok) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int c = cb + j;
+          if (c >= e.N || c == row || (e.symmetric && c > row)) continue;
+          const float q = v[j] * v[j];
+          const unsigned long long w = (e.symmetric && c < row) ? 2ull : 1ull;
+          dev_fine += w * static_cast<unsigned long long>(fminf(q, kDevFineClamp) * kDevFineUnit);
+        }
+      }
+      // row segment: columns cb.. of this lane's row (only col <= row
+      // when the product is symmetric)
+      const bool below = !e.symmetric || cb + 31 < rbase;   // whole chunk left of every row
+      if (out_bulk && below) {
+        // Through this warp's staging rows: each lane writes its row
+        // segment as 16-byte pieces, then every store instruction takes
+        // 4 rows x 128 bytes (lane l: row 4 i + l / 8, columns 4 (l % 8)).
+        float* stage = reinterpret_cast<float*>(wbuf + 2 * Cfg::kRowBuf);
+        const int sr = lane >> 3, sc = 4 * (lane & 7);
+        const bool col_ok = cb + sc < e.N;
+#pragma unroll 1
+        for (int o = 0; o < 3; ++o) {
+          float* out = o == 0 ? e.C : (o == 1 ? e.Chi : e.Clo);
+          if (!out) continue;                             // warp-uniform
+          const int64_t ld = o == 0 ? e.ldc : e.ldh;
+          __syncwarp();                                   // previous output's reads done
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            float4 x = make_float4(v[4 * t], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
+            if (o == 1 || (o == 0 && e.out_round)) {
+              x = make_float4(rn_tf32(x.x), rn_tf32(x.y), rn_tf32(x.z), rn_tf32(x.w));
+            } else if (o == 2) {
+              x = make_float4(rn_tf32(x.x - rn_tf32(x.x)), rn_tf32(x.y - rn_tf32(x.y)),
+                              rn_tf32(x.z - rn_tf32(x.z)), rn_tf32(x.w - rn_tf32(x.w)));
+            }
+            *reinterpret_cast<float4*>(stage + lane * Cfg::kPitch + 4 * t) = x;
+          }
+          __syncwarp();
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int rr = 4 * t + sr;
+            if (rbase + rr < e.M && col_ok)
+              *reinterpret_cast<float4*>(out + int64_t(rbase + rr) * ld + cb + sc) =
+                  *reinterpret_cast<const float4*>(stage + rr * Cfg::kPitch + sc);
+          }
+        }
+        __syncwarp();
+      } else if (row_ok) {
+        if (out_vec) {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int c = cb + 4 * t;
+            if (c >= e.N) break;
+            if (!e.symmetric || c + 3 <= row) {
+              e.put4(int64_t(row), c, v[4 * t + 0], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
+            } else {
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                if (c + u <= row) e.put(int64_t(row), c + u, v[4 * t + u]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int c = cb + j;
+            if (c < e.N && (!e.symmetric || c <= row)) e.put(int64_t(row), c, v[j]);
+          }
+        }
+      }
+      // mirror of the strictly-lower part: element (row, c) also at (c, row)
+      if (e.symmetric && cb < rbase + 32) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int c = cb + j;
+          if (row_ok && c < e.N && c < row) e.put(int64_t(c), row, v[j]);
+        }
+      }
+    }
+    if (e.devsq) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dev_fine += __shfl_xor_sync(0xffffffffu, dev_fine, o);
+      if (lane == 0 && dev_fine) atomicAdd(e.devsq, dev_fine);
+    }
+    cp_async_wait<0>();                                 // nothing in flight into the buffers
+  }
+}
+
 template <int BN, bool SPLIT, int STAGES>
 __global__ void __launch_bounds__(192, STAGES <= 2 ? 2 : 1)
 k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, int nparams,
@@ -347,180 +533,7 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
     if (!ok) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
     fence_after_sync();
     if (ok && !*(volatile int*)&abort_flag) {
-      EpiArgs e;
-      e.load(g, tabs, nparams);
-      // Lane l of warp q holds accumulator row 32 q + l (TMEM lane), 32
-      // columns per load.  When bases and leading dimensions are 16-byte
-      // aligned, Cin comes in as one 1-D bulk copy per row segment (128
-      // bytes, double-buffered in this warp's rows of the idle pipeline
-      // buffers) and the outputs go out through a transposing staging row
-      // block, four full 128-byte lines per store instruction; otherwise each
-      // lane loads and stores its row directly.  The mirror of a symmetric
-      // product writes column segments, contiguous across the lanes.
-      const int rbase = m0 + 32 * q;
-      const int row = rbase + lane;
-      const int nacc = kblocks < Cfg::kAcc ? kblocks : Cfg::kAcc;   // accumulators written
-      const bool row_ok = row < e.M;
-      const int nrows = min(32, e.M - rbase);
-      const int ncols = min(BN, e.N - n0);
-      const int nchunks = ncols > 0 ? (ncols + 31) / 32 : 0;
-      const bool cin_bulk = e.beta != 0.0f &&
-                            ((reinterpret_cast<uintptr_t>(e.Cin) | uintptr_t(e.ldcin * 4)) & 15) == 0 &&
-                            (e.N & 3) == 0;
-      const bool out_bulk = ((reinterpret_cast<uintptr_t>(e.C) | uintptr_t(e.ldc * 4) |
-                              reinterpret_cast<uintptr_t>(e.Chi) | reinterpret_cast<uintptr_t>(e.Clo) |
-                              uintptr_t(e.ldh * 4)) & 15) == 0 &&
-                            (e.N & 3) == 0;
-      const bool out_vec = out_bulk;                        // same alignment conditions
-      uint8_t* wbuf = smem + q * Cfg::kEpiWarp;
-      const uint32_t wsm = smem_u32(wbuf);
-      const uint32_t my_row = uint32_t(lane * Cfg::kPitch * 4);
-      unsigned long long dev_fine = 0;                      // deviation sum, plan.h units
-      // Cin chunk i into buffer i & 1 with 16-byte cp.async pieces, four
-      // full 128-byte rows per warp instruction: lane l copies rows
-      // 4 t + l / 8 (t < 8), columns 4 (l % 8).  One group per chunk.
-      auto issue_cin = [&](int i) {
-        const int cb = n0 + 32 * i, sr = lane >> 3, sc = 4 * (lane & 7);
-        if (cb + sc < e.N) {
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int rr = 4 * t + sr;
-            if (rbase + rr < e.M)
-              cp_async16(wsm + (i & 1) * Cfg::kRowBuf + uint32_t((rr * Cfg::kPitch + sc) * 4),
-                         e.Cin + int64_t(rbase + rr) * e.ldcin + cb + sc);
-          }
-        }
-        cp_async_commit();
-      };
-      if (nrows > 0 && nchunks > 0) {
-        if (cin_bulk) issue_cin(0);
-#pragma unroll 1
-        for (int i = 0; i < nchunks; ++i) {
-          const int c0 = 32 * i, cb = n0 + c0;
-          if (cin_bulk && i + 1 < nchunks) {
-            __syncwarp();                                   // buffer (i + 1) & 1: chunk i - 1's reads done
-            issue_cin(i + 1);
-          }
-          uint32_t r[32];
-          tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(c0), r);
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          for (int a = 1; a < nacc; ++a) {                  // the other accumulators, added with RN
-            tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(a * BN + c0), r);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] += __uint_as_float(r[j]);
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] *= e.alpha;
-          if (e.beta != 0.0f) {
-            if (cin_bulk) {
-              if (i + 1 < nchunks) cp_async_wait<1>(); else cp_async_wait<0>();
-              __syncwarp();                                 // every lane's pieces of chunk i visible
-              if (row_ok) {
-                const float4* src = reinterpret_cast<const float4*>(wbuf + (i & 1) * Cfg::kRowBuf + my_row);
-#pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                  if (cb + 4 * t >= e.N) break;
-                  const float4 x = src[t];
-                  v[4 * t + 0] = fmaf(e.beta, x.x, v[4 * t + 0]);
-                  v[4 * t + 1] = fmaf(e.beta, x.y, v[4 * t + 1]);
-                  v[4 * t + 2] = fmaf(e.beta, x.z, v[4 * t + 2]);
-                  v[4 * t + 3] = fmaf(e.beta, x.w, v[4 * t + 3]);
-                }
-              }
-            } else if (row_ok) {
-              const float* src = e.Cin + int64_t(row) * e.ldcin + cb;
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (cb + j < e.N) v[j] = fmaf(e.beta, __ldg(src + j), v[j]);
-            }
-          }
-          if (e.devsq && row_ok) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int c = cb + j;
-              if (c >= e.N || c == row || (e.symmetric && c > row)) continue;
-              const float q = v[j] * v[j];
-              const unsigned long long w = (e.symmetric && c < row) ? 2ull : 1ull;
-              dev_fine += w * static_cast<unsigned long long>(fminf(q, kDevFineClamp) * kDevFineUnit);
-            }
-          }
-          // row segment: columns cb.. of this lane's row (only col <= row
-          // when the product is symmetric)
-          const bool below = !e.symmetric || cb + 31 < rbase;   // whole chunk left of every row
-          if (out_bulk && below) {
-            // Through this warp's staging rows: each lane writes its row
-            // segment as 16-byte pieces, then every store instruction takes
-            // 4 rows x 128 bytes (lane l: row 4 i + l / 8, columns 4 (l % 8)).
-            float* stage = reinterpret_cast<float*>(wbuf + 2 * Cfg::kRowBuf);
-            const int sr = lane >> 3, sc = 4 * (lane & 7);
-            const bool col_ok = cb + sc < e.N;
-#pragma unroll 1
-            for (int o = 0; o < 3; ++o) {
-              float* out = o == 0 ? e.C : (o == 1 ? e.Chi : e.Clo);
-              if (!out) continue;                             // warp-uniform
-              const int64_t ld = o == 0 ? e.ldc : e.ldh;
-              __syncwarp();                                   // previous output's reads done
-#pragma unroll
-              for (int t = 0; t < 8; ++t) {
-                float4 x = make_float4(v[4 * t], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
-                if (o == 1 || (o == 0 && e.out_round)) {
-                  x = make_float4(rn_tf32(x.x), rn_tf32(x.y), rn_tf32(x.z), rn_tf32(x.w));
-                } else if (o == 2) {
-                  x = make_float4(rn_tf32(x.x - rn_tf32(x.x)), rn_tf32(x.y - rn_tf32(x.y)),
-                                  rn_tf32(x.z - rn_tf32(x.z)), rn_tf32(x.w - rn_tf32(x.w)));
-                }
-                *reinterpret_cast<float4*>(stage + lane * Cfg::kPitch + 4 * t) = x;
-              }
-              __syncwarp();
-#pragma unroll
-              for (int t = 0; t < 8; ++t) {
-                const int rr = 4 * t + sr;
-                if (rbase + rr < e.M && col_ok)
-                  *reinterpret_cast<float4*>(out + int64_t(rbase + rr) * ld + cb + sc) =
-                      *reinterpret_cast<const float4*>(stage + rr * Cfg::kPitch + sc);
-              }
-            }
-            __syncwarp();
-          } else if (row_ok) {
-            if (out_vec) {
-#pragma unroll
-              for (int t = 0; t < 8; ++t) {
-                const int c = cb + 4 * t;
-                if (c >= e.N) break;
-                if (!e.symmetric || c + 3 <= row) {
-                  e.put4(int64_t(row), c, v[4 * t + 0], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
-                } else {
-#pragma unroll
-                  for (int u = 0; u < 4; ++u)
-                    if (c + u <= row) e.put(int64_t(row), c + u, v[4 * t + u]);
-                }
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int c = cb + j;
-                if (c < e.N && (!e.symmetric || c <= row)) e.put(int64_t(row), c, v[j]);
-              }
-            }
-          }
-          // mirror of the strictly-lower part: element (row, c) also at (c, row)
-          if (e.symmetric && cb < rbase + 32) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int c = cb + j;
-              if (row_ok && c < e.N && c < row) e.put(int64_t(c), row, v[j]);
-            }
-          }
-        }
-        if (e.devsq) {
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) dev_fine += __shfl_xor_sync(0xffffffffu, dev_fine, o);
-          if (lane == 0 && dev_fine) atomicAdd(e.devsq, dev_fine);
-        }
-        cp_async_wait<0>();                                 // nothing in flight into the buffers
-      }
+      epilogue_tile<BN, SPLIT, STAGES>(g, tabs, nparams, m0, n0, kblocks, tmem, q, lane, smem + q * Cfg::kEpiWarp);
     }
   }
   fence_before_sync();
@@ -558,9 +571,15 @@ int tc_block_n(int split) { return split ? 128 : 256; }
 shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split, int bn,
                                const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st) {
   if (count <= 0 || max_tiles <= 0) return SHAMPOO4_OK;
-  // TF32: two 2-stage CTAs per SM, so one tile's epilogue overlaps the
-  // other's main loop.  Split mode: one 3-stage CTA per SM, or two 2-stage
-  // CTAs with 64-wide tiles for the narrow panel updates.
+  // One tile per CTA.  TF32: two 2-stage CTAs per SM, so one tile's
+  // epilogue overlaps the other's main loop.  (A persistent form with two
+  // TMEM accumulator sets and eight epilogue warps was measured against it:
+  // faster on single-output products, slower on the symmetric and
+  // multi-output products this library runs.)  Split mode: one 3-stage CTA
+  // per SM with 128-wide tiles (four accumulators fill TMEM), or two 2-stage
+  // CTAs per SM with 64-wide tiles for the narrow panel updates, where the
+  // MMA issue rate of a 64-wide instruction makes a second issuing CTA per
+  // SM worth more than overlap.
   if (!split) return launch_tc_impl<256, false, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, st);
   if (bn == 64) return launch_tc_impl<64, true, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, st);
   return launch_tc_impl<128, true, 3>(d_desc, count, max_tiles, tabs, nparams, gflags, st);
