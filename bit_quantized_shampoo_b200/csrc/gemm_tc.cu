@@ -400,7 +400,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmDesc& g, const PtrEntr
         }
       }
       // mirror of the strictly-lower part: element (row, c) also at (c, row)
-      if (e.symmetric && cb < rbase + 32) {
+      if (e.symmetric == 1 && cb < rbase + 32) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int c = cb + j;

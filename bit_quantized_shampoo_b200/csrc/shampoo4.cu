@@ -599,7 +599,8 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
   for (auto& f : h->factors) if (f.tc) dmax = std::max(dmax, f.d);
   if (dmax == 0) return;
   {
-    // Gram W = X^T X (fp32 into W, its TF32 split into Th/Tl), optional shift
+    // Gram W = X^T X (lower triangle: fp32 into W, its TF32 split into
+    // Th/Tl), optional shift
     std::vector<TcGemmDesc> g;
     std::vector<ShiftDescF> sd;
     std::vector<GateDesc> gd;
@@ -617,9 +618,12 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
       }
       w.a = b.operand(X[i].h, X[i].l, d, d, true, true, true);
       w.b = b.operand(X[i].h, X[i].l, d, d, false, false, true, kSquareBN);
+      // only the lower triangles of W and of its TF32 split are ever read
+      // (Cholesky blocks, panel updates, and the first panel's L21 product,
+      // which takes W21 from the split): no mirror stores
       w.C = b.wf(f.ws_W); w.ldc = d;
       w.Chi = b.wf(f.ws_Th); w.Clo = b.wf(f.ws_Tl); w.ldh = d;
-      w.symmetric = 1;
+      w.symmetric = 2;
       w.skip = b.tcbad(i);
       g.push_back(w);
       dg.push_back({X[i].m, b.wf(f.ws_W), d, d, 0, gated ? b.devsq(i) : nullptr, b.tcbad(i)});
@@ -766,7 +770,13 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
       BasisDesc x{};
       x.codes = b.sb(f.st_codes); x.scales = b.sf(f.st_scales);
       x.d = f.d; x.identity = first ? 1 : 0;
-      if (f.tc) { x.U = b.wf(f.ws_Xm[0]); x.Uh = b.wf(f.ws_Xh[0]); x.Ul = b.wf(f.ws_Xl[0]); }
+      // TF32 Björck reads only U's hi part (and rewrites lo at its last
+      // step); without Björck steps the fp32-accurate subspace product
+      // reads both parts
+      if (f.tc) {
+        x.U = b.wf(f.ws_Xm[0]); x.Uh = b.wf(f.ws_Xh[0]);
+        x.Ul = (split || first || h->cfg.bjorck_iters == 0) ? b.wf(f.ws_Xl[0]) : nullptr;
+      }
       else x.U = b.wf(f.ws_U);
       bd.push_back(x);
       bytes += (first ? 0.0 : 0.5625) * double(f.d) * f.d + (f.tc ? 12.0 : 4.0) * double(f.d) * f.d;
@@ -787,7 +797,8 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
         TcGemmDesc g = gemmtc(d, d, d, 1.0f, 0.0f);          // T = U^T U
         g.a = b.operand(b.wf(f.ws_Xh[c]), b.wf(f.ws_Xl[c]), d, d, true, true, split);
         g.b = b.operand(b.wf(f.ws_Xh[c]), b.wf(f.ws_Xl[c]), d, d, false, false, split);
-        g.Chi = b.wf(f.ws_Th); g.Clo = b.wf(f.ws_Tl); g.ldh = d;
+        // the update reads T's lo part only when fp32-accurate
+        g.Chi = b.wf(f.ws_Th); g.Clo = split ? b.wf(f.ws_Tl) : nullptr; g.ldh = d;
         g.symmetric = 1;
         tgram.push_back(g);
         TcGemmDesc u = gemmtc(d, d, d, -0.5f, 1.5f);         // U' = 1.5 U - 0.5 U T
@@ -795,7 +806,9 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
         u.b = b.operand(b.wf(f.ws_Th), b.wf(f.ws_Tl), d, d, false, true, split);   // T symmetric
         u.Cin = b.wf(f.ws_Xm[c]); u.ldcin = d;
         u.C = b.wf(f.ws_Xm[o]); u.ldc = d;
-        u.Chi = b.wf(f.ws_Xh[o]); u.Clo = b.wf(f.ws_Xl[o]); u.ldh = d;
+        // U's lo part feeds the next Björck products only when fp32-accurate;
+        // the last one always feeds the fp32-accurate subspace product
+        u.Chi = b.wf(f.ws_Xh[o]); u.Clo = (split || it + 1 == iters) ? b.wf(f.ws_Xl[o]) : nullptr; u.ldh = d;
         tupd.push_back(u);
         cur[i] = o;
       } else {

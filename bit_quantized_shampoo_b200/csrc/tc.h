@@ -21,8 +21,9 @@ struct TcOperand {
 // C = alpha * op(A) op(B) + beta * Cin for one problem.  Outputs, each
 // optional: C (fp32, rounded to TF32 when out_round), and the TF32 split
 // Chi = RN(v), Clo = RN(v - Chi) with leading dimension ldh.  symmetric:
-// only tiles touching the lower triangle run and every element below the
-// diagonal is also written to its mirror position.  skip: problem skipped
+// only tiles touching the lower triangle run; 1: every element below the
+// diagonal is also written to its mirror position; 2: only the lower
+// triangle (diagonal included) is written.  skip: problem skipped
 // when *skip != 0.  c_ref: C taken from the per-call pointer tables.
 struct TcGemmDesc {
   int32_t M, N, K;
