@@ -127,7 +127,7 @@ STAGE_BOUND = {
     "apply_left": "tf32", "apply_right": "tf32",
     "subspace": "3xtf32", "rayleigh_gemm": "3xtf32", "qr_gram": "3xtf32", "qr_syrk": "3xtf32",
     "qr_trsm_panel": "3xtf32", "qr_solve_update": "3xtf32", "qr_solve_panel": "3xtf32",
-    "qr_potrf": "latency", "rayleigh": "hbm", "requant": "hbm", "precond_dequant": "hbm",
+    "qr_potrf": "latency", "qr_inverse": "latency", "rayleigh": "hbm", "requant": "hbm", "precond_dequant": "hbm",
     "basis": "hbm", "stats_scan": "hbm", "refresh_scan": "hbm", "qr_convert": "hbm", "precond_mu": "hbm",
 }
 
@@ -347,10 +347,14 @@ def main():
     # per-stage times measured live over the timed region
     stages = {}
     launches = 0
-    for s in range(22):
+    s = 0
+    while True:                                      # every stage the library names
+        name = L.lib().shampoo4_stage_name(s).decode()
+        if name == "unknown":
+            break
         t_ms, n, fl, by = C.c_double(), C.c_int64(), C.c_double(), C.c_double()
         L.call("shampoo4_timing_read", sh._h, s, C.byref(t_ms), C.byref(n), C.byref(fl), C.byref(by))
-        name = L.lib().shampoo4_stage_name(s).decode()
+        s += 1
         if n.value:
             stages[name] = {"ms": t_ms.value / args.steps, "launches": n.value // args.steps,
                             "flops": fl.value / args.steps, "bytes": by.value / args.steps}

@@ -485,6 +485,101 @@ shampoo4_status launch_rowdiag(const RowDiagDesc* d_desc, int count, int max_d, 
   return SHAMPOO4_OK;
 }
 
+// ---- 128 x 128 inverse blocks from 64 x 64 ones -------------------------------
+// Three 64 x 64 fp64 arrays (100 KB: two CTAs per SM): T = C A^-1 first,
+// then A^-1's space takes B^-1 and C's space takes -B^-1 T.
+constexpr int kInvSmem = 3 * 64 * 65 * 8;
+
+__global__ void __launch_bounds__(256) k_inv128(const Inv128Desc* __restrict__ descs) {
+  const Inv128Desc& g = descs[blockIdx.x];
+  if (g.skip && *g.skip) return;
+  extern __shared__ double sm_inv[];
+  double (*Xi)[65] = reinterpret_cast<double (*)[65]>(sm_inv);              // A^-1, then B^-1
+  double (*Cm)[65] = reinterpret_cast<double (*)[65]>(sm_inv + 64 * 65);    // C, then M
+  double (*Tm)[65] = reinterpret_cast<double (*)[65]>(sm_inv + 2 * 64 * 65);
+  const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
+  const int n1 = min(64, g.d - g.j), n2 = max(0, min(64, g.d - g.j - 64));
+  auto out = [&](int r, int c, double v) { put_split(float(v), g.jh, g.jl, int64_t(g.j + r) * 128 + c); };
+  for (int r = t >> 6; r < 64; r += 4) {
+    const int c = t & 63;
+    const int64_t a = int64_t(g.j + r) * 64 + c;
+    Xi[r][c] = double(g.ih[a]) + double(g.il[a]);
+    const int64_t o = int64_t(g.j + 64 + r) * g.d + g.j + c;
+    Cm[r][c] = (r < n2 && c < n1) ? double(g.oh[o]) + double(g.ol[o]) : 0.0;
+  }
+  __syncthreads();
+  // T = C A^-1 (thread (ty, tx): rows ty + 16 i, columns tx + 16 k)
+  {
+    double acc[4][4] = {};
+    for (int kk = 0; kk < 64; ++kk) {
+      double lft[4], rgt[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) lft[i] = Cm[ty + 16 * i][kk];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) rgt[k] = Xi[kk][tx + 16 * k];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[i][k] = fma(lft[i], rgt[k], acc[i][k]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) Tm[ty + 16 * i][tx + 16 * k] = acc[i][k];
+  }
+  // top half of the output: [A^-1 0]
+  for (int e = t; e < 64 * 128; e += blockDim.x) {
+    const int r = e >> 7, c = e & 127;
+    out(r, c, (c < 64 && r < n1 && c < n1) ? Xi[r][c] : 0.0);
+  }
+  __syncthreads();
+  for (int r = t >> 6; r < 64; r += 4) {
+    const int c = t & 63;
+    const int64_t b = int64_t(g.j + 64 + r) * 64 + c;
+    Xi[r][c] = n2 > 0 ? double(g.ih[b]) + double(g.il[b]) : 0.0;
+  }
+  __syncthreads();
+  // M = -B^-1 T into Cm
+  {
+    double acc[4][4] = {};
+    for (int kk = 0; kk < 64; ++kk) {
+      double lft[4], rgt[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) lft[i] = Xi[ty + 16 * i][kk];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) rgt[k] = Tm[kk][tx + 16 * k];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[i][k] = fma(lft[i], rgt[k], acc[i][k]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) Cm[ty + 16 * i][tx + 16 * k] = -acc[i][k];
+  }
+  __syncthreads();
+  // bottom half: [M B^-1]
+  for (int e = t; e < 64 * 128; e += blockDim.x) {
+    const int r = e >> 7, c = e & 127;
+    double v = 0.0;
+    if (r < n2) v = c < 64 ? (c < n1 ? Cm[r][c] : 0.0) : (c - 64 < n2 ? Xi[r][c - 64] : 0.0);
+    out(64 + r, c, v);
+  }
+}
+
+shampoo4_status launch_inv128(const Inv128Desc* d_desc, int count, cudaStream_t st) {
+  if (count <= 0) return SHAMPOO4_OK;
+  static bool configured = false;
+  if (!configured) {
+    S4_CUDA(cudaFuncSetAttribute(k_inv128, cudaFuncAttributeMaxDynamicSharedMemorySize, kInvSmem));
+    configured = true;
+  }
+  k_inv128<<<count, 256, kInvSmem, st>>>(d_desc);
+  S4_CUDA(cudaGetLastError());
+  return SHAMPOO4_OK;
+}
+
 // ---- last-pass gate -----------------------------------------------------------
 __global__ void __launch_bounds__(256) k_gate(const GateDesc* __restrict__ descs, int count) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;

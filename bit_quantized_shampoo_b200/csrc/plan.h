@@ -217,6 +217,22 @@ struct RowDiagDesc {
 // of 2^-60: an exact integer sum, independent of the order of additions.
 constexpr float kDevFineClamp = 0x1p-20f, kDevFineUnit = 0x1p60f;
 
+// Inverse of a 128 x 128 lower-triangular diagonal block of L from the
+// inverses of its two 64 x 64 diagonal blocks:
+//   [A 0; C B]^-1 = [A^-1 0; -B^-1 C A^-1  B^-1],
+// with A^-1, B^-1 the split 64 x 64 blocks (ld 64, zero-padded) at ih/il
+// rows j and j + 64, C = L[j+64 :, j : j+64] from the split factor (oh/ol,
+// ld d).  fp64 inside; out: the TF32 split of the 128 x 128 inverse
+// (ld 128), zero outside the d - j valid rows and columns.  One CTA per
+// block.
+struct Inv128Desc {
+  const float* ih; const float* il;    // 64 x 64 inverse blocks, rows j..
+  const float* oh; const float* ol;    // split of L, ld d
+  float* jh; float* jl;                // 128 x 128 output, rows j..
+  int32_t d, j;
+  const uint32_t* skip;
+};
+
 // Decision before the last Cholesky-QR pass of a factor, from the Gram of
 // its input Q: out = 1 (skip the pass) when *bad != 0 or *devsq <= thr (Q
 // already orthonormal to the arithmetic's floor), else 0.
@@ -254,6 +270,7 @@ shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max
                                const uint32_t* guard = nullptr);
 shampoo4_status launch_clear(const ClearDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_gate(const GateDesc* d_desc, int count, cudaStream_t st);
+shampoo4_status launch_inv128(const Inv128Desc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaStream_t st);
 shampoo4_status launch_rowdiag(const RowDiagDesc* d_desc, int count, int max_d, cudaStream_t st);
 

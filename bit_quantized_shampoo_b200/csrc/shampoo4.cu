@@ -30,7 +30,7 @@ using namespace s4;
 namespace {
 
 enum class Kind { GemmF32, GemmF64, Potrf, Trsm, Basis, Rayleigh, Mu, Scan, Convert, Pack, Shift, GemmTC, GemmTCSplit,
-                  GemmTCSplit64, PotrfF, ShiftF, Split, Gate, Diag, RowDiag };
+                  GemmTCSplit64, PotrfF, ShiftF, Split, Gate, Diag, RowDiag, Inv128 };
 
 struct Launch {
   Kind kind;
@@ -70,12 +70,15 @@ struct FactorPlan {
   size_t ws_W64, ws_Q64, ws_U, ws_T, ws_Y;
   size_t ws_Xm[2], ws_Xh[2], ws_Xl[2], ws_Th, ws_Tl, ws_Sh, ws_Sl, ws_W;
   size_t ws_Zm, ws_Zh, ws_Zl;
-  size_t ws_Ih, ws_Il, ws_Ph, ws_Pl;     // d x 64: inverse diagonal blocks, panel temporary
+  size_t ws_Ih, ws_Il;                   // 64 x 64 inverse diagonal blocks of L (rows to a multiple of 64)
+  size_t ws_Jh, ws_Jl;                   // 128 x 128 inverse diagonal blocks (rows to a multiple of 128)
+  size_t ws_Ph, ws_Pl;                   // d x 128: solve panel temporary
   size_t ws_q_first, ws_q_next;
 };
 
 constexpr size_t kAlign = 256;
-constexpr int kPanelW = 64;
+constexpr int kPanelW = 64;     // Cholesky panel width (64 x 64 diagonal blocks)
+constexpr int kSolveW = 128;    // solve panel width (128 x 128 inverse blocks)
 
 }  // namespace
 
@@ -199,8 +202,11 @@ shampoo4_status plan(shampoo4_ctx* h) {
       const size_t dpad = align_up(size_t(f.d), kPanelW);
       f.ws_Ih = take(ws, 4 * dpad * kPanelW);
       f.ws_Il = take(ws, 4 * dpad * kPanelW);
-      f.ws_Ph = take(ws, 4 * size_t(f.d) * kPanelW);
-      f.ws_Pl = take(ws, 4 * size_t(f.d) * kPanelW);
+      const size_t dpad2 = align_up(size_t(f.d), kSolveW);
+      f.ws_Jh = take(ws, 4 * dpad2 * kSolveW);
+      f.ws_Jl = take(ws, 4 * dpad2 * kSolveW);
+      f.ws_Ph = take(ws, 4 * size_t(f.d) * kSolveW);
+      f.ws_Pl = take(ws, 4 * size_t(f.d) * kSolveW);
       f.ws_W64 = take(ws, 8 * dd);            // fp64 fallback of the QR
       f.ws_Q64 = take(ws, 8 * dd);
     } else {
@@ -691,30 +697,47 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
     b.tag = SHAMPOO4_STAGE_QR_TRSM_PANEL;
     emit_gemmtc(b, prog, l21, true, 64);
   }
-  // Solve Q L^T = X by 64-wide column panels:
+  // Solve Q L^T = X by 128-wide column panels, through the 128 x 128
+  // inverse diagonal blocks assembled from the 64 x 64 ones (k_inv128):
   //   T = X[:, J] - Q[:, <J] L[J, <J]^T      tensor cores, TF32 split into P
   //   Q[:, J] = T L[J, J]^-T                  tensor cores
-  for (int j = 0; j < dmax; j += kPanelW) {
+  // 128-wide products keep the MMA at its 128-column rate (a 64-column
+  // instruction pays about the same issue time for half the work), and the
+  // solve takes half as many steps.
+  {
+    std::vector<Inv128Desc> iv;
+    for (size_t i = 0; i < nf; ++i) {
+      const FactorPlan& f = h->factors[i];
+      if (!f.tc) continue;
+      for (int j = 0; j < f.d; j += kSolveW)
+        iv.push_back({b.wf(f.ws_Ih), b.wf(f.ws_Il), b.wf(f.ws_Th), b.wf(f.ws_Tl), b.wf(f.ws_Jh), b.wf(f.ws_Jl),
+                      f.d, j, skip_of(i)});
+    }
+    b.tag = SHAMPOO4_STAGE_QR_INVERSE;
+    b.emit(prog, Kind::Inv128, iv, 0);
+  }
+  for (int j = 0; j < dmax; j += kSolveW) {
     std::vector<TcGemmDesc> up, qp;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
       if (!f.tc || j >= f.d) continue;
-      const int d = f.d, jb = std::min(kPanelW, d - j);
+      const int d = f.d, jb = std::min(kSolveW, d - j);
       TcGemmDesc q = gemmtc(d, jb, jb, 1.0f, 0.0f);
       if (j > 0) {
         TcGemmDesc u = gemmtc(d, jb, j, -1.0f, 1.0f);
         u.a = b.operand(Q[i].h, Q[i].l, d, d, true, false, true);
-        u.b = b.operand(b.wf(f.ws_Th), b.wf(f.ws_Tl), d, d, false, true, true, 64);
+        u.b = b.operand(b.wf(f.ws_Th), b.wf(f.ws_Tl), d, d, false, true, true, kSolveW);
         u.b.row0 = j;
-        u.Chi = b.wf(f.ws_Ph); u.Clo = b.wf(f.ws_Pl); u.ldh = kPanelW;
+        u.Chi = b.wf(f.ws_Ph); u.Clo = b.wf(f.ws_Pl); u.ldh = kSolveW;
         u.Cin = X[i].m + j; u.ldcin = d;
         u.skip = skip_of(i);
         up.push_back(u);
-        q.a = b.operand(b.wf(f.ws_Ph), b.wf(f.ws_Pl), d, kPanelW, true, false, true);
+        q.a = b.operand(b.wf(f.ws_Ph), b.wf(f.ws_Pl), d, kSolveW, true, false, true);
       } else {
         q.a = b.operand(X[i].h, X[i].l, d, d, true, false, true);   // T = X[:, 0:jb]
       }
-      q.b = b.operand(b.wf(f.ws_Ih), b.wf(f.ws_Il), dpad_of(d), kPanelW, false, true, true, 64);
+      q.b = b.operand(b.wf(f.ws_Jh), b.wf(f.ws_Jl), int(align_up(size_t(d), kSolveW)), kSolveW, false, true, true,
+                      64);
       q.b.row0 = j;
       q.C = Q[i].m + j; q.ldc = d;
       q.Chi = Q[i].h + j; q.Clo = Q[i].l + j; q.ldh = d;
@@ -722,7 +745,8 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
       qp.push_back(q);
     }
     b.tag = SHAMPOO4_STAGE_QR_SOLVE_UPDATE;
-    emit_gemmtc(b, prog, up, true, 64);
+    emit_gemmtc(b, prog, up, true, kSolveW);
+    // the panel product is short (K <= 128): 64-wide tiles, two CTAs per SM
     b.tag = SHAMPOO4_STAGE_QR_SOLVE_PANEL;
     emit_gemmtc(b, prog, qp, true, 64);
   }
@@ -1154,6 +1178,9 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
       case Kind::Diag:
         S4_TRY(launch_diag(static_cast<const DiagDesc*>(d), L.count, int(L.extent), st));
         break;
+      case Kind::Inv128:
+        S4_TRY(launch_inv128(static_cast<const Inv128Desc*>(d), L.count, st));
+        break;
       case Kind::RowDiag:
         S4_TRY(launch_rowdiag(static_cast<const RowDiagDesc*>(d), L.count, int(L.extent), st));
         break;
@@ -1450,7 +1477,7 @@ extern "C" const char* shampoo4_stage_name(int32_t stage) {
       "stats_scan", "stats_gemm", "refresh_scan", "basis", "bjorck_gram", "bjorck_update",
       "subspace", "qr_gram", "qr_potrf", "qr_trsm_panel", "qr_syrk", "qr_solve_update",
       "qr_solve_panel", "qr_convert", "rayleigh_gemm", "rayleigh", "requant", "precond_dequant",
-      "precond_mu", "roots", "apply_left", "apply_right"};
+      "precond_mu", "roots", "apply_left", "apply_right", "qr_inverse"};
   if (stage < 0 || stage >= SHAMPOO4_STAGE_COUNT) return "unknown";
   return names[stage];
 }
