@@ -236,13 +236,37 @@ k_scan(const ScanDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, in
     X = e.ptr + g.ref.r0 * e.ld + g.ref.c0;
   }
   bool bad = false;
-  for (int r = blockIdx.x; r < g.rows; r += gridDim.x) {      // rows, coalesced columns
-    const float* xr = X + int64_t(r) * ld;
-    const int64_t o = int64_t(r) * g.cols;
-    for (int c = threadIdx.x; c < g.cols; c += blockDim.x) {
-      const float v = xr[c];
-      bad |= !isfinite(v);
-      put_split(v, g.oh, g.ol, o + c);
+  const bool vec = ((reinterpret_cast<uintptr_t>(X) | uintptr_t(ld * 4) | reinterpret_cast<uintptr_t>(g.oh) |
+                     reinterpret_cast<uintptr_t>(g.ol)) & 15) == 0 && (g.cols & 3) == 0;
+  if (vec) {
+    // 16-byte pieces over the whole matrix, four independent pieces in
+    // flight per thread
+    const int c4n = g.cols >> 2;
+    const int64_t n4 = int64_t(g.rows) * c4n;
+    const int64_t step = int64_t(gridDim.x) * blockDim.x;
+#pragma unroll 4
+    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n4; e += step) {
+      const int r = int(e / c4n), c = int(e - int64_t(r) * c4n) * 4;
+      const float4 v = *reinterpret_cast<const float4*>(X + int64_t(r) * ld + c);
+      bad |= !isfinite(v.x) || !isfinite(v.y) || !isfinite(v.z) || !isfinite(v.w);
+      if (g.oh) {
+        const float4 h = make_float4(tf32_rn(v.x), tf32_rn(v.y), tf32_rn(v.z), tf32_rn(v.w));
+        const int64_t o = int64_t(r) * g.cols + c;
+        *reinterpret_cast<float4*>(g.oh + o) = h;
+        if (g.ol)
+          *reinterpret_cast<float4*>(g.ol + o) =
+              make_float4(tf32_rn(v.x - h.x), tf32_rn(v.y - h.y), tf32_rn(v.z - h.z), tf32_rn(v.w - h.w));
+      }
+    }
+  } else {
+    for (int r = blockIdx.x; r < g.rows; r += gridDim.x) {    // rows, coalesced columns
+      const float* xr = X + int64_t(r) * ld;
+      const int64_t o = int64_t(r) * g.cols;
+      for (int c = threadIdx.x; c < g.cols; c += blockDim.x) {
+        const float v = xr[c];
+        bad |= !isfinite(v);
+        put_split(v, g.oh, g.ol, o + c);
+      }
     }
   }
   if (__syncthreads_or(bad) && threadIdx.x == 0) {
