@@ -626,24 +626,6 @@ shampoo4_status launch_shift_f(const ShiftDescF* d_desc, int count, cudaStream_t
   return SHAMPOO4_OK;
 }
 
-__global__ void __launch_bounds__(256) k_split(const SplitDesc* __restrict__ descs) {
-  const SplitDesc& g = descs[blockIdx.y];
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < g.n;
-       e += int64_t(gridDim.x) * blockDim.x)
-    put_split(g.x[e], g.h, g.l, e);
-}
-
-shampoo4_status launch_split(const SplitDesc* d_desc, int count, int64_t max_elems, cudaStream_t st) {
-  if (count <= 0 || max_elems <= 0) return SHAMPOO4_OK;
-  int64_t ctas = (max_elems + 1023) / 1024;
-  if (ctas > 1024) ctas = 1024;
-  for (int base = 0; base < count; base += 65535) {
-    int c = count - base < 65535 ? count - base : 65535;
-    k_split<<<dim3(unsigned(ctas), c), 256, 0, st>>>(d_desc + base);
-    S4_CUDA(cudaGetLastError());
-  }
-  return SHAMPOO4_OK;
-}
 
 // ---- fp64 -> fp32 ----------------------------------------------------------
 constexpr int64_t kConvertChunk = 1 << 16;

@@ -164,12 +164,6 @@ struct ShiftDescF {
   const uint32_t* skip;
 };
 
-// (h, l) = TF32 split of x, elementwise over n.
-struct SplitDesc {
-  const float* x;
-  float* h; float* l;
-  int64_t n;
-};
 
 // dst = fp32(src); optionally also the TF32 split (dh, dl).
 struct ConvertDesc {
@@ -180,10 +174,6 @@ struct ConvertDesc {
   const uint32_t* skip;       // optional
 };
 
-struct ClearDesc {
-  uint32_t* p;
-  int64_t n;
-};
 
 // W_ii <- sum_k X[k, i]^2 (fp64 sums, one thread per column, rounded once
 // to fp32) for i < d, X row-major d x d.  The tensor cores' accumulation
@@ -265,10 +255,8 @@ shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st
                              const uint32_t* guard = nullptr);
 shampoo4_status launch_potrf_f(const PotrfDescF* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_shift_f(const ShiftDescF* d_desc, int count, cudaStream_t st);
-shampoo4_status launch_split(const SplitDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st,
                                const uint32_t* guard = nullptr);
-shampoo4_status launch_clear(const ClearDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_gate(const GateDesc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_inv128(const Inv128Desc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaStream_t st);

@@ -30,7 +30,7 @@ using namespace s4;
 namespace {
 
 enum class Kind { GemmF32, GemmF64, Potrf, Trsm, Basis, Rayleigh, Mu, Scan, Convert, Pack, Shift, GemmTC, GemmTCSplit,
-                  GemmTCSplit64, PotrfF, ShiftF, Split, Gate, Diag, RowDiag, Inv128 };
+                  GemmTCSplit64, PotrfF, ShiftF, Gate, Diag, RowDiag, Inv128 };
 
 struct Launch {
   Kind kind;
@@ -1174,9 +1174,6 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
         break;
       case Kind::ShiftF:
         S4_TRY(launch_shift_f(static_cast<const ShiftDescF*>(d), L.count, st));
-        break;
-      case Kind::Split:
-        S4_TRY(launch_split(static_cast<const SplitDesc*>(d), L.count, L.extent, st));
         break;
       case Kind::Gate:
         S4_TRY(launch_gate(static_cast<const GateDesc*>(d), L.count, st));
