@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-codec", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-graft", action="store_true")
     ap.add_argument("--shapes", default=None, help="comma-separated RxC list replacing the workload's shapes")
     ap.add_argument("--grad-sets", type=int, default=2,
                     help="seeded gradient sets the steps cycle through (1 = the same gradient every step)")
@@ -441,6 +442,39 @@ def main():
                          "pack_frac": pack_gbs / pk["hbm_gbs"], "unpack_frac": unpack_gbs / pk["hbm_gbs"],
                          "peak_gbs": pk["hbm_gbs"], "peak_source": pk_src}
         del x, y, codes, scales
+
+    # stand-alone grafted weight update (Adam graft) over the workload's parameters,
+    # fed this step's gradients and directions
+    if not args.no_graft:
+        gen = torch.Generator(device=dev).manual_seed(5)
+        weights = [torch.randn(s, device=dev, generator=gen) * 0.02 for s in shapes]
+        gstate = sh.graft_state("adam")
+        g = dev_sets[0]
+        t = [0]
+
+        def graft():
+            t[0] += 1
+            sh.graft_update(gstate, t[0], 1e-3, g, dev_out, weights, kind="adam")
+
+        for _ in range(3):
+            graft()
+        torch.cuda.synchronize()
+        reps = 5
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(stream)
+        for _ in range(reps):
+            graft()
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        n_elem = sum(r * c for r, c in shapes)
+        gms = ev[0].elapsed_time(ev[1]) / reps
+        bpe = 32.0          # read G, D, W, m, v; write W, m, v (fp32)
+        gbs = bpe * n_elem / (gms / 1e3) / 1e9
+        line["graft"] = {"kind": "adam", "elements": n_elem, "ms": gms, "launches": 2, "bound": "hbm",
+                         "bytes_per_element": bpe, "issued_bytes_per_element": 36.0,
+                         "gbs": gbs, "frac": gbs / pk["hbm_gbs"], "peak_gbs": pk["hbm_gbs"], "peak_source": pk_src,
+                         "status_flags": sh.status_flags()}
+        del weights, gstate
 
     if rank == 0 and world == 1 and not args.no_cpu:
         tile_s, nb, desc, threads = cpu_sample(w, 4)

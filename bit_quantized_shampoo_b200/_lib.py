@@ -25,6 +25,9 @@ FLAG_REFRESH_FAILED = 0x2
 FLAG_NONFINITE_STATE = 0x4
 FLAG_TIMEOUT = 0x8
 FLAG_QR_FALLBACK = 0x10
+FLAG_GRAFT_SKIPPED = 0x20
+GRAFT_SGD = 0
+GRAFT_ADAM = 1
 PREC_TF32 = 0
 PREC_FP32 = 1
 
@@ -32,6 +35,11 @@ PREC_FP32 = 1
 class Config(C.Structure):
     _fields_ = [("beta", C.c_float), ("eps", C.c_float), ("max_block", C.c_int32),
                 ("quant_block", C.c_int32), ("bjorck_iters", C.c_int32), ("precision", C.c_int32)]
+
+
+class GraftConfig(C.Structure):
+    _fields_ = [("kind", C.c_int32), ("beta1", C.c_float), ("beta2", C.c_float),
+                ("adam_eps", C.c_float), ("graft_eps", C.c_float)]
 
 
 class Param(C.Structure):
@@ -65,6 +73,11 @@ _SIGS = {
     "quant4_tables": [c_f32_p, c_f32_p],
     "shampoo4_update_stats_noalloc": [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_int64,
                                       C.c_float, C.c_void_p, C.c_void_p],
+    "shampoo4_graft_state_bytes": [C.c_void_p, C.c_int32, c_size_p],
+    "shampoo4_graft_layout": [C.c_void_p, C.c_int32, C.c_int32, c_size_p, c_size_p],
+    "shampoo4_graft_update": [C.c_void_p, C.POINTER(GraftConfig), C.c_void_p, C.c_int64, C.c_float,
+                              C.POINTER(C.c_void_p), c_i64_p, C.POINTER(C.c_void_p), c_i64_p,
+                              C.POINTER(C.c_void_p), c_i64_p, C.c_void_p],
     "shampoo4_timing_enable": [C.c_void_p, C.c_int32],
     "shampoo4_timing_read": [C.c_void_p, C.c_int32, C.POINTER(C.c_double), c_i64_p, C.POINTER(C.c_double),
                              C.POINTER(C.c_double)],

@@ -86,6 +86,35 @@ class Shampoo4:
         L.call("shampoo4_precondition", self._h, p, ld, q, ldo, _stream(stream))
         return out
 
+    # ---- grafting ("Shampoo -- Second-Order Optimizer", section "Grafting")
+
+    def graft_state(self, kind="adam"):
+        """A zero-filled device buffer for the grafting state (Adam's moments)."""
+        n = C.c_size_t()
+        L.call("shampoo4_graft_state_bytes", self._h, _graft_kind(kind), C.byref(n))
+        return torch.zeros(max(n.value, 256), dtype=torch.uint8, device=self.device)
+
+    def graft_moments(self, state, param):
+        """(m, v) of parameter ``param`` as fp32 views into an Adam state buffer."""
+        om, ov = C.c_size_t(), C.c_size_t()
+        L.call("shampoo4_graft_layout", self._h, L.GRAFT_ADAM, param, C.byref(om), C.byref(ov))
+        r, c = self.shapes[param]
+        n = 4 * r * c
+        return (state[om.value:om.value + n].view(torch.float32).view(r, c),
+                state[ov.value:ov.value + n].view(torch.float32).view(r, c))
+
+    def graft_update(self, state, step, lr, grads, dirs, weights, kind="adam", beta1=0.9, beta2=0.999,
+                     adam_eps=1e-8, graft_eps=1e-16, stream=None):
+        """W <- W - lr * ||d_graft|| / (||D|| + graft_eps) * D per tile, in place
+        on ``weights``; ``dirs`` is this step's precondition output."""
+        cfg = L.GraftConfig(_graft_kind(kind), beta1, beta2, adam_eps, graft_eps)
+        p, ld = self._ptrs(grads, "grads")
+        q, ldq = self._ptrs(dirs, "dirs")
+        w, ldw = self._ptrs(weights, "weights")
+        sp = C.c_void_p(state.data_ptr()) if state is not None else C.c_void_p()
+        L.call("shampoo4_graft_update", self._h, C.byref(cfg), sp, int(step), float(lr), p, ld, q, ldq, w, ldw,
+               _stream(stream))
+
     def status_flags(self, stream=None) -> int:
         f = C.c_uint32()
         L.call("shampoo4_get_status_flags", self._h, C.byref(f), _stream(stream))
@@ -127,6 +156,13 @@ class Shampoo4:
             self.close()
         except Exception:
             pass
+
+
+def _graft_kind(kind):
+    kinds = {"sgd": L.GRAFT_SGD, "adam": L.GRAFT_ADAM}
+    if kind not in kinds:
+        raise ValueError(f"graft kind must be one of {sorted(kinds)}")
+    return kinds[kind]
 
 
 def quant4_pack(xs, codes=None, scales=None, stream=None):

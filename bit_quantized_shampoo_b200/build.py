@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libshampoo4.so")
 
-SOURCES = ["quant4.cu", "gemm_simt.cu", "gemm_tc.cu", "kernels_misc.cu", "shampoo4.cu", "noalloc.cu"]
+SOURCES = ["quant4.cu", "gemm_simt.cu", "gemm_tc.cu", "kernels_misc.cu", "graft.cu", "shampoo4.cu", "noalloc.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-I" + INCLUDE, "-I" + CSRC]

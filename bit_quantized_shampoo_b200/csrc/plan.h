@@ -234,6 +234,44 @@ struct GateDesc {
 };
 
 
+// ---- grafted weight update ("Shampoo -- Second-Order Optimizer", section
+// "Grafting: borrow a step size that already works") ------------------------
+// step_b = lr * ||d_graft_b||_F / (||D_b||_F + graft_eps) * D_b per tile b,
+// W_b <- W_b - step_b; d_graft = G (SGD) or the bias-corrected Adam
+// direction m_hat / (sqrt(v_hat) + adam_eps).  A work item is a band of rows
+// of one tile; the items of a tile are consecutive, and the partial sums of
+// item i sit in parts[2i] (sum d_graft^2) and parts[2i + 1] (sum D^2).
+enum GraftKind : int32_t { kGraftSgd = 0, kGraftAdam = 1 };
+
+struct GraftItem {
+  int32_t param, block;        // parameter, and tile (statistics flag index)
+  int64_t r0, c0;              // band origin within the parameter
+  int32_t rows, cols;
+  int32_t part0, nparts;       // the tile's first item and its item count
+  int64_t m_off, v_off;        // element offsets of the band origin's moments
+  int64_t state_ld;            // moments are dense per parameter: ld = cols
+};
+
+struct GraftArgs {
+  const GraftItem* items;
+  int32_t nitems, nparams;
+  const PtrEntry* tabs;        // [0, np): gradients, [np, 2np): directions,
+                               // [2np, 3np): weights
+  float* state;                // Adam moments (unused for SGD)
+  const uint32_t* bflag;       // per tile: non-finite gradient seen by the
+                               // statistics update of this step
+  double* parts;               // 2 * nitems
+  uint32_t* flags;             // status word
+  int32_t kind;
+  float beta1, beta2, omb1, omb2;       // omb = 1 - beta, in fp32
+  float c1, c2;                         // 1 / (1 - beta^t)
+  float adam_eps;
+  double lr, graft_eps;
+};
+
+// Two launches: moments and per-item norms, then the weight update.
+shampoo4_status launch_graft(const GraftArgs& a, cudaStream_t st);
+
 // ---- launchers (each enqueues one launch over `count` descriptors) -------
 shampoo4_status launch_gemm_f32(const GemmF32Desc* d_desc, int count, int max_tiles,
                                 const PtrEntry* tabs, int nparams, cudaStream_t st);

@@ -119,6 +119,17 @@ struct shampoo4_ctx {
   double t_flops[SHAMPOO4_STAGE_COUNT] = {};
   double t_bytes[SHAMPOO4_STAGE_COUNT] = {};
   int64_t t_launches[SHAMPOO4_STAGE_COUNT] = {};
+  // grafted weight update: bands of tile rows, the moments' layout, and a
+  // per-call pointer table of its own (gradients, directions, weights)
+  std::vector<GraftItem> graft_items;
+  std::vector<size_t> graft_off_m, graft_off_v;   // bytes, per parameter
+  size_t graft_state_bytes = 0;
+  size_t ws_gtab = 0, ws_gitems = 0, ws_gparts = 0;
+  std::vector<PtrEntry> gtab_host;
+  bool gtab_valid = false;
+  PtrEntry* gtab_pinned = nullptr;
+  cudaEvent_t gtab_event = nullptr;
+  bool gtab_event_pending = false;
 };
 
 namespace {
@@ -138,6 +149,50 @@ size_t take(size_t& cursor, size_t bytes) {
 }
 
 bool tc_dim(int d) { return d % 4 == 0; }
+
+// Grafting: each tile is cut into bands of whole rows of at most
+// kGraftBandElems elements (one CTA each); the moments are dense per
+// parameter, m then v, each slice kAlign-aligned.
+constexpr int64_t kGraftBandElems = 65536;
+
+void plan_graft(shampoo4_ctx* h, size_t& ws) {
+  const size_t np = h->params.size();
+  size_t gs = 0;
+  h->graft_off_m.resize(np);
+  h->graft_off_v.resize(np);
+  for (size_t p = 0; p < np; ++p) {
+    const size_t elems = size_t(h->params[p].rows) * size_t(h->params[p].cols);
+    h->graft_off_m[p] = take(gs, 4 * elems);
+    h->graft_off_v[p] = take(gs, 4 * elems);
+  }
+  h->graft_state_bytes = align_up(gs, kAlign);
+  for (size_t k = 0; k < h->blocks.size(); ++k) {
+    const BlockPlan& b = h->blocks[k];
+    const int64_t cols = h->params[b.param].cols;
+    const int32_t band = int32_t(std::max<int64_t>(1, std::min<int64_t>(b.m, kGraftBandElems / b.n)));
+    const int32_t nparts = (b.m + band - 1) / band;
+    const int32_t part0 = int32_t(h->graft_items.size());
+    for (int32_t i = 0; i < nparts; ++i) {
+      GraftItem it{};
+      it.param = b.param;
+      it.block = int32_t(k);
+      it.r0 = b.r0 + int64_t(i) * band;
+      it.c0 = b.c0;
+      it.rows = std::min<int32_t>(band, b.m - i * band);
+      it.cols = b.n;
+      it.part0 = part0;
+      it.nparts = nparts;
+      const int64_t e = it.r0 * cols + it.c0;
+      it.m_off = int64_t(h->graft_off_m[b.param] / 4) + e;
+      it.v_off = int64_t(h->graft_off_v[b.param] / 4) + e;
+      it.state_ld = cols;
+      h->graft_items.push_back(it);
+    }
+  }
+  h->ws_gtab = take(ws, sizeof(PtrEntry) * 3 * np);
+  h->ws_gitems = take(ws, sizeof(GraftItem) * h->graft_items.size());
+  h->ws_gparts = take(ws, 16 * h->graft_items.size());
+}
 
 shampoo4_status plan(shampoo4_ctx* h) {
   for (size_t p = 0; p < h->params.size(); ++p) {
@@ -228,6 +283,7 @@ shampoo4_status plan(shampoo4_ctx* h) {
     b.ws_Bh = take(ws, 4 * mn);
     b.ws_Bl = take(ws, 4 * mn);
   }
+  plan_graft(h, ws);
   h->ws_maps = align_up(ws, kAlign);
   h->ws_bytes = h->ws_maps;     // maps and descriptors are added by init
   return SHAMPOO4_OK;
@@ -1317,8 +1373,11 @@ extern "C" shampoo4_status shampoo4_bind(shampoo4_handle h, void* d_state, void*
     S4_CUDA(cudaHostAlloc(&h->tab_pinned, sizeof(PtrEntry) * 2 * h->params.size() + 64, cudaHostAllocDefault));
     S4_CUDA(cudaHostAlloc(&h->flags_pinned, 64, cudaHostAllocDefault));
     S4_CUDA(cudaEventCreateWithFlags(&h->tab_event, cudaEventDisableTiming));
+    S4_CUDA(cudaHostAlloc(&h->gtab_pinned, sizeof(PtrEntry) * 3 * h->params.size() + 64, cudaHostAllocDefault));
+    S4_CUDA(cudaEventCreateWithFlags(&h->gtab_event, cudaEventDisableTiming));
   }
   if (h->tab_event_pending) S4_CUDA(cudaEventSynchronize(h->tab_event));
+  if (h->gtab_event_pending) S4_CUDA(cudaEventSynchronize(h->gtab_event));
   h->d_state = static_cast<uint8_t*>(d_state);
   h->d_ws = static_cast<uint8_t*>(d_workspace);
   h->prog_stats.clear(); h->prog_refresh_first.clear(); h->prog_refresh.clear(); h->prog_precond.clear();
@@ -1337,12 +1396,16 @@ extern "C" shampoo4_status shampoo4_bind(shampoo4_handle h, void* d_state, void*
     S4_CUDA(cudaMemcpyAsync(h->d_ws + h->ws_maps, h->maps.data(), h->maps.size() * sizeof(CUtensorMap),
                             cudaMemcpyHostToDevice, st));
   S4_CUDA(cudaMemcpyAsync(h->d_ws + h->ws_desc, h->arena.data(), h->arena.size(), cudaMemcpyHostToDevice, st));
+  if (!h->graft_items.empty())
+    S4_CUDA(cudaMemcpyAsync(h->d_ws + h->ws_gitems, h->graft_items.data(),
+                            sizeof(GraftItem) * h->graft_items.size(), cudaMemcpyHostToDevice, st));
   if (reset) {
     S4_CUDA(cudaMemsetAsync(h->d_state, 0, h->state_bytes, st));
     h->has_basis = false;
   }
   S4_CUDA(cudaStreamSynchronize(st));   // the host arena is reused by the next bind
   h->tab_valid = false;
+  h->gtab_valid = false;
   h->bound = true;
   return SHAMPOO4_OK;
 }
@@ -1485,6 +1548,117 @@ extern "C" const char* shampoo4_stage_name(int32_t stage) {
   return names[stage];
 }
 
+// ------------------------------------------------------------- grafting
+
+namespace {
+
+bool graft_config_ok(const shampoo4_graft_config* c) {
+  if (!c) return false;
+  if (c->kind != SHAMPOO4_GRAFT_SGD && c->kind != SHAMPOO4_GRAFT_ADAM) return false;
+  if (!(c->graft_eps >= 0.0f) || !std::isfinite(c->graft_eps)) return false;
+  if (c->kind == SHAMPOO4_GRAFT_ADAM) {
+    if (!(c->beta1 >= 0.0f && c->beta1 < 1.0f) || !(c->beta2 >= 0.0f && c->beta2 < 1.0f)) return false;
+    if (!(c->adam_eps >= 0.0f) || !std::isfinite(c->adam_eps)) return false;
+  }
+  return true;
+}
+
+// [p0, p1) byte range of parameter i's matrix at ptr with leading dimension ld
+std::pair<uintptr_t, uintptr_t> span(const shampoo4_param& q, const float* ptr, int64_t ld) {
+  const uintptr_t a = uintptr_t(ptr);
+  return {a, a + 4 * uintptr_t((q.rows - 1) * ld + q.cols)};
+}
+
+}  // namespace
+
+extern "C" shampoo4_status shampoo4_graft_state_bytes(shampoo4_handle h, int32_t kind, size_t* bytes) {
+  if (!h || !bytes) return SHAMPOO4_ERR_INVALID_ARG;
+  if (kind != SHAMPOO4_GRAFT_SGD && kind != SHAMPOO4_GRAFT_ADAM) return SHAMPOO4_ERR_INVALID_ARG;
+  *bytes = kind == SHAMPOO4_GRAFT_ADAM ? h->graft_state_bytes : 0;
+  return SHAMPOO4_OK;
+}
+
+extern "C" shampoo4_status shampoo4_graft_layout(shampoo4_handle h, int32_t kind, int32_t param,
+                                                 size_t* off_m, size_t* off_v) {
+  if (!h || kind != SHAMPOO4_GRAFT_ADAM || param < 0 || size_t(param) >= h->params.size())
+    return SHAMPOO4_ERR_INVALID_ARG;
+  if (off_m) *off_m = h->graft_off_m[param];
+  if (off_v) *off_v = h->graft_off_v[param];
+  return SHAMPOO4_OK;
+}
+
+extern "C" shampoo4_status shampoo4_graft_update(shampoo4_handle h, const shampoo4_graft_config* cfg,
+                                                 void* d_graft_state, int64_t step, float lr,
+                                                 const float* const* d_grads, const int64_t* ld_grads,
+                                                 const float* const* d_dirs, const int64_t* ld_dirs,
+                                                 float* const* d_weights, const int64_t* ld_weights,
+                                                 shampoo4_stream_t stream) {
+  if (!h) return SHAMPOO4_ERR_INVALID_ARG;
+  if (!h->bound) return SHAMPOO4_ERR_NOT_READY;
+  if (!graft_config_ok(cfg) || !std::isfinite(lr)) return SHAMPOO4_ERR_INVALID_ARG;
+  const bool adam = cfg->kind == SHAMPOO4_GRAFT_ADAM;
+  if (adam && (step < 1 || !d_graft_state || !aligned(d_graft_state, kAlign))) return SHAMPOO4_ERR_INVALID_ARG;
+  S4_TRY(check_matrices(h, d_grads, ld_grads));
+  S4_TRY(check_matrices(h, d_dirs, ld_dirs));
+  S4_TRY(check_matrices(h, const_cast<const float* const*>(d_weights), ld_weights));
+  const size_t np = h->params.size();
+  for (size_t i = 0; i < np; ++i) {
+    const auto w = span(h->params[i], d_weights[i], ld_weights[i]);
+    for (size_t j = 0; j < np; ++j) {
+      const auto g = span(h->params[j], d_grads[j], ld_grads[j]);
+      const auto d = span(h->params[j], d_dirs[j], ld_dirs[j]);
+      if ((w.first < g.second && g.first < w.second) || (w.first < d.second && d.first < w.second))
+        return SHAMPOO4_ERR_INVALID_ARG;
+      if (j != i) {
+        const auto w2 = span(h->params[j], d_weights[j], ld_weights[j]);
+        if (w.first < w2.second && w2.first < w.second) return SHAMPOO4_ERR_INVALID_ARG;
+      }
+    }
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // per-call pointer table, uploaded when it changed
+  std::vector<PtrEntry> want(3 * np);
+  for (size_t p = 0; p < np; ++p) {
+    want[p] = {d_grads[p], ld_grads[p]};
+    want[np + p] = {d_dirs[p], ld_dirs[p]};
+    want[2 * np + p] = {d_weights[p], ld_weights[p]};
+  }
+  if (!h->gtab_valid || std::memcmp(want.data(), h->gtab_host.data(), sizeof(PtrEntry) * 3 * np) != 0) {
+    if (h->gtab_event_pending) S4_CUDA(cudaEventSynchronize(h->gtab_event));
+    std::memcpy(h->gtab_pinned, want.data(), sizeof(PtrEntry) * 3 * np);
+    S4_CUDA(cudaMemcpyAsync(h->d_ws + h->ws_gtab, h->gtab_pinned, sizeof(PtrEntry) * 3 * np,
+                            cudaMemcpyHostToDevice, st));
+    S4_CUDA(cudaEventRecord(h->gtab_event, st));
+    h->gtab_event_pending = true;
+    h->gtab_host = want;
+    h->gtab_valid = true;
+  }
+  GraftArgs a{};
+  a.items = reinterpret_cast<const GraftItem*>(h->d_ws + h->ws_gitems);
+  a.nitems = int32_t(h->graft_items.size());
+  a.nparams = int32_t(np);
+  a.tabs = reinterpret_cast<const PtrEntry*>(h->d_ws + h->ws_gtab);
+  a.state = adam ? static_cast<float*>(d_graft_state) : nullptr;
+  a.bflag = reinterpret_cast<const uint32_t*>(h->d_ws + h->ws_bflag);
+  a.parts = reinterpret_cast<double*>(h->d_ws + h->ws_gparts);
+  a.flags = reinterpret_cast<uint32_t*>(h->d_ws + h->ws_flags);
+  a.kind = adam ? kGraftAdam : kGraftSgd;
+  a.beta1 = cfg->beta1;
+  a.beta2 = cfg->beta2;
+  a.omb1 = 1.0f - cfg->beta1;
+  a.omb2 = 1.0f - cfg->beta2;
+  if (adam) {
+    const double t = double(step);
+    a.c1 = float(1.0 / (1.0 - std::pow(double(cfg->beta1), t)));
+    a.c2 = float(1.0 / (1.0 - std::pow(double(cfg->beta2), t)));
+    if (!std::isfinite(a.c1) || !std::isfinite(a.c2)) return SHAMPOO4_ERR_INVALID_ARG;
+  }
+  a.adam_eps = cfg->adam_eps;
+  a.lr = double(lr);
+  a.graft_eps = double(cfg->graft_eps);
+  return launch_graft(a, st);
+}
+
 extern "C" void shampoo4_destroy(shampoo4_handle h) {
   if (!h) return;
   collect_timing(h);
@@ -1494,6 +1668,11 @@ extern "C" void shampoo4_destroy(shampoo4_handle h) {
     cudaEventDestroy(h->tab_event);
   }
   if (h->tab_pinned) cudaFreeHost(h->tab_pinned);
+  if (h->gtab_event) {
+    cudaEventSynchronize(h->gtab_event);
+    cudaEventDestroy(h->gtab_event);
+  }
+  if (h->gtab_pinned) cudaFreeHost(h->gtab_pinned);
   if (h->flags_pinned) cudaFreeHost(h->flags_pinned);
   delete h;
 }

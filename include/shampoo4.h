@@ -105,6 +105,10 @@ typedef struct shampoo4_ctx* shampoo4_handle;
                                                some factor's subspace step was
                                                too ill-conditioned and was
                                                redone in fp64                */
+#define SHAMPOO4_FLAG_GRAFT_SKIPPED    0x20u /* shampoo4_graft_update: a tile's
+                                               norm ratio was not finite (its
+                                               direction or moments overflowed);
+                                               its weights were left unchanged */
 
 /* Plan a set of parameters.  Host only: validates the config and shapes,
  * partitions every weight into greedy tiles of at most max_block (ragged
@@ -248,6 +252,66 @@ shampoo4_status quant4_tables(float codebook[16], float thresholds[15]);
 shampoo4_status shampoo4_update_stats_noalloc(float* d_L, float* d_R, const float* d_G, int32_t m,
                                               int32_t n, int64_t ldg, float beta, uint32_t* d_flags,
                                               shampoo4_stream_t stream);
+
+/* ---- Grafting and the weight update -------------------------------------
+ * "Shampoo -- Second-Order Optimizer", section "Grafting: borrow a step size
+ * that already works": Shampoo gives each tile's direction D_b (the output of
+ * shampoo4_precondition), a method with a tuned step size gives its norm:
+ *   step_b = lr * ||d_graft_b||_F / (||D_b||_F + graft_eps) * D_b,
+ *   W_b   <- W_b - step_b,
+ * with the Frobenius norms taken per tile of the handle's partition.
+ * d_graft is the grafted method's step without its learning rate:
+ *   SHAMPOO4_GRAFT_SGD   d_graft = G;
+ *   SHAMPOO4_GRAFT_ADAM  Adam (Kingma and Ba, ICLR 2015, Algorithm 1):
+ *     m <- beta1 m + (1 - beta1) G,  v <- beta2 v + (1 - beta2) G^2,
+ *     d_graft = (m / (1 - beta1^t)) / (sqrt(v / (1 - beta2^t)) + adam_eps).
+ * Arithmetic: fp32 elementwise (moments by fused multiply-adds, IEEE square
+ * root and division); the norms are summed in fp64 in a fixed order; the
+ * ratio lr * ||d_graft|| / (||D|| + graft_eps) is formed in fp64, rounded to
+ * fp32 once, and W <- fma(-r, D, W).  A zero denominator gives a zero step. */
+typedef enum { SHAMPOO4_GRAFT_SGD = 0, SHAMPOO4_GRAFT_ADAM = 1 } shampoo4_graft_kind;
+
+typedef struct {
+  int32_t kind;          /* shampoo4_graft_kind                              */
+  float beta1, beta2;    /* Adam moment decays, in [0, 1) (ignored for SGD)   */
+  float adam_eps;        /* Adam's denominator epsilon, >= 0                  */
+  float graft_eps;       /* epsilon of the norm ratio, >= 0                   */
+} shampoo4_graft_config;
+
+/* Bytes of grafting state the caller provides for this handle's parameters:
+ * Adam's two fp32 moments (8 bytes per parameter element; 0 for SGD).  The
+ * buffer is 256-byte aligned and zero-filled by the caller before the first
+ * step; it persists between steps (checkpointable). */
+shampoo4_status shampoo4_graft_state_bytes(shampoo4_handle h, int32_t kind, size_t* bytes);
+
+/* Byte offsets inside the grafting state of parameter p's first and second
+ * moments (fp32, rows x cols, row-major, dense). */
+shampoo4_status shampoo4_graft_layout(shampoo4_handle h, int32_t kind, int32_t param,
+                                      size_t* off_m, size_t* off_v);
+
+/* One grafted weight update of every parameter, enqueued on `stream` (two
+ * kernel launches; no synchronization, no allocation).
+ *   d_grads[p]   the step's gradient (the one passed to this step's
+ *                shampoo4_update_stats), leading dimension ld_grads[p];
+ *   d_dirs[p]    the step's Shampoo direction D (shampoo4_precondition's
+ *                output), leading dimension ld_dirs[p];
+ *   d_weights[p] the weights, updated in place, leading dimension
+ *                ld_weights[p]; they must not overlap any gradient or
+ *                direction;
+ *   step         Adam's 1-based step counter t (bias correction);
+ *   lr           the learning rate (finite).
+ * A tile whose gradient the statistics update of this step flagged as
+ * non-finite (SHAMPOO4_FLAG_NONFINITE_GRAD) is skipped whole: moments and
+ * weights unchanged.  A tile whose ratio is not finite keeps its weights and
+ * raises SHAMPOO4_FLAG_GRAFT_SKIPPED.  Pointers 4-byte aligned (16-byte
+ * aligned rows take the vector path); bad arguments return
+ * SHAMPOO4_ERR_INVALID_ARG, an unbound handle SHAMPOO4_ERR_NOT_READY. */
+shampoo4_status shampoo4_graft_update(shampoo4_handle h, const shampoo4_graft_config* cfg,
+                                      void* d_graft_state, int64_t step, float lr,
+                                      const float* const* d_grads, const int64_t* ld_grads,
+                                      const float* const* d_dirs, const int64_t* ld_dirs,
+                                      float* const* d_weights, const int64_t* ld_weights,
+                                      shampoo4_stream_t stream);
 
 void shampoo4_destroy(shampoo4_handle h);
 const char* shampoo4_status_string(shampoo4_status s);

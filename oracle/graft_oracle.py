@@ -32,8 +32,9 @@ Readings where the page is silent (repeated in the design notes):
   weights   stored fp32; W - step is formed in fp64 and rounded once.
   non-finite  a tile whose gradient holds NaN/Inf is skipped whole: its
             moments and weights stay unchanged (the statistics update leaves
-            such a tile's statistics unchanged too).  A tile whose ratio is
-            not finite keeps its weights (its moments are updated).
+            such a tile's statistics unchanged too).  A tile whose squared
+            norms are not finite, or whose step factor lr * ratio is not
+            finite in fp32, keeps its weights (its moments are updated).
 """
 from __future__ import annotations
 
@@ -104,8 +105,12 @@ class GraftOracle:
             else:
                 dg = np.asarray(g, np.float64)
             D = np.asarray(dirs[b.param], np.float32)[rs, cs]
+            ng2 = float(np.sum(np.asarray(dg, np.float64) ** 2))
+            nd2 = float(np.sum(np.asarray(D, np.float64) ** 2))
+            if not (np.isfinite(ng2) and np.isfinite(nd2)):
+                continue
             r = lr * graft_ratio(dg, D, self.graft_eps)
-            if not np.isfinite(r):
+            if not abs(r) <= float(np.finfo(np.float32).max):
                 continue
             w = np.asarray(weights[b.param], np.float64)[rs, cs]
             out[b.param][rs, cs] = (w - r * np.asarray(D, np.float64)).astype(np.float32)

@@ -109,3 +109,38 @@ def test_calls_before_bind_are_not_ready_and_null_handles_invalid():
         assert lib.shampoo4_status_string(3)
     finally:
         L.lib().shampoo4_destroy(h)
+
+
+def test_graft_state_layout_and_argument_checks():
+    shapes = [(37, 29), (1030, 8), (4, 4)]
+    st, h = _init(shapes, max_block=16)
+    assert st == 0
+    try:
+        lib = L.lib()
+        n = C.c_size_t()
+        L.call("shampoo4_graft_state_bytes", h, L.GRAFT_SGD, C.byref(n))
+        assert n.value == 0
+        L.call("shampoo4_graft_state_bytes", h, L.GRAFT_ADAM, C.byref(n))
+        assert n.value >= sum(8 * r * c for r, c in shapes) and n.value % 256 == 0
+        assert lib.shampoo4_graft_state_bytes(h, 2, C.byref(n)) == 1
+        spans = []
+        for p, (r, c) in enumerate(shapes):
+            om, ov = C.c_size_t(), C.c_size_t()
+            L.call("shampoo4_graft_layout", h, L.GRAFT_ADAM, p, C.byref(om), C.byref(ov))
+            for o in (om.value, ov.value):
+                assert o % 256 == 0
+                spans.append((o, o + 4 * r * c))
+        spans.sort()
+        assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:])) and spans[-1][1] <= n.value
+        assert lib.shampoo4_graft_layout(h, L.GRAFT_ADAM, 3, None, None) == 1
+        assert lib.shampoo4_graft_layout(h, L.GRAFT_SGD, 0, None, None) == 1
+        cfg = L.GraftConfig(L.GRAFT_ADAM, 0.9, 0.999, 1e-8, 1e-16)
+        ptrs = L.ptr_array([256, 512, 768])
+        lds = L.i64_array([c for _, c in shapes])
+        # unbound handle: not ready; null handle: invalid
+        assert lib.shampoo4_graft_update(h, C.byref(cfg), C.c_void_p(256), 1, C.c_float(0.1), ptrs, lds, ptrs, lds,
+                                         ptrs, lds, None) == 3
+        assert lib.shampoo4_graft_update(None, C.byref(cfg), None, 1, C.c_float(0.1), ptrs, lds, ptrs, lds,
+                                         ptrs, lds, None) == 1
+    finally:
+        L.lib().shampoo4_destroy(h)
