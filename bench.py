@@ -139,9 +139,9 @@ STAGE_BOUND = {
 # launch over other factors of the same kind moves the same bytes per
 # element.  Valid only for the GEMM source it was taken on: the figure is
 # dropped (traffic = null) when gemm_tc.cu or tc.h has changed since.
-TRAFFIC_SOURCE_SHA = "cc56304ced2846b2"
-TRAFFIC_PER_ELEMENT = {"stats_gemm": 6.587, "bjorck_gram": 10.367, "bjorck_update": 22.917,
-                       "subspace": 32.19, "qr_gram": 18.92}
+TRAFFIC_SOURCE_SHA = "953e5999e9574e38"
+TRAFFIC_PER_ELEMENT = {"stats_gemm": 6.590, "bjorck_gram": 6.758, "bjorck_update": 19.321,
+                       "subspace": 32.588, "qr_gram": 13.066}
 
 
 def gemm_source_sha():
