@@ -170,6 +170,29 @@ def ema_stats(S: np.ndarray, Gb: np.ndarray, beta: float, side: str) -> np.ndarr
     return s.astype(np.float32)
 
 
+def compressed_stats(f: "Factor", Gb: np.ndarray, beta: float, side: str) -> np.ndarray:
+    """The statistic update when S is kept only as its 4-bit eigenbasis and
+    eigenvalues ("4-bit Shampoo ...", abstract: the preconditioner is stored
+    through its quantized eigenvector matrix): the previous statistic is
+    rebuilt as U diag(lambda) U^T from the dequantized codes (no Bjorck, as
+    for the roots), then S = beta U diag(lambda) U^T + (1 - beta) G G^T.
+    Before the first refresh there is nothing stored: S = (1 - beta) G G^T,
+    the EMA from zero.  fp64, stored fp32.  A gradient holding NaN/Inf
+    leaves the statistic as stored (the rebuilt U diag(lambda) U^T; zero
+    before the first refresh)."""
+    g = np.asarray(Gb, dtype=np.float64)
+    stored = np.zeros((f.d, f.d))
+    if f.has_basis:
+        U = dequantize(f.codes, f.scales, f.d * f.d).reshape(f.d, f.d).astype(np.float64)
+        lam = np.asarray(f.lam, np.float64)
+        stored = (U * lam[None, :]) @ U.T
+    if not np.all(np.isfinite(g)):
+        # a non-finite gradient leaves the statistic as stored
+        return stored.astype(np.float32) if f.has_basis else np.asarray(f.S, np.float32)
+    outer = g @ g.T if side == "L" else g.T @ g
+    return (beta * stored + (1.0 - beta) * outer).astype(np.float32)
+
+
 def bjorck(U: np.ndarray, iters: int) -> np.ndarray:
     """Orthogonality rectification U <- 1.5 U - 0.5 U (U^T U), ``iters`` times."""
     U = np.asarray(U, dtype=np.float64)
@@ -253,12 +276,15 @@ class Shampoo4Oracle:
     """The whole preconditioner step over a list of 2-D parameters."""
 
     def __init__(self, shapes, beta=0.95, eps=1e-6, bjorck_iters=5,
-                 max_block=1024, quant=True):
+                 max_block=1024, quant=True, compressed=False):
         self.shapes = [tuple(s) for s in shapes]
         self.beta = float(beta)
         self.eps = float(eps)
         self.bjorck_iters = int(bjorck_iters)
         self.quant = bool(quant)
+        self.compressed = bool(compressed)
+        if self.compressed and not self.quant:
+            raise ValueError("compressed statistics need the 4-bit basis")
         self.blocks = partition(self.shapes, max_block)
         self.factors: list[Factor] = []
         for b in self.blocks:
@@ -273,8 +299,12 @@ class Shampoo4Oracle:
         for k in range(len(self.blocks)):
             g = self.block_view(grads, k)
             fl, fr = self.factors[2 * k], self.factors[2 * k + 1]
-            fl.S = ema_stats(fl.S, g, self.beta, "L")
-            fr.S = ema_stats(fr.S, g, self.beta, "R")
+            if self.compressed:
+                fl.S = compressed_stats(fl, g, self.beta, "L")
+                fr.S = compressed_stats(fr, g, self.beta, "R")
+            else:
+                fl.S = ema_stats(fl.S, g, self.beta, "L")
+                fr.S = ema_stats(fr.S, g, self.beta, "R")
 
     def refresh_roots(self) -> None:
         for f in self.factors:

@@ -151,6 +151,68 @@ def test_ema_stats_closed_form_and_sides():
     assert np.allclose(SR, eR, rtol=1e-6, atol=0)
 
 
+# ------------------------------------------- compressed statistics (f1)
+
+def _signed_hadamard(d, rng):
+    """A non-symmetric orthogonal matrix whose entries are all +-1/sqrt(d):
+    Sylvester's Hadamard matrix with its columns permuted and sign-flipped.
+    For d = 64 every entry is +-1/8, so each 64-block's absmax is 1/8 and
+    every entry sits exactly on a codebook end level: the 4-bit codes hold
+    it without error."""
+    H = np.array([[1.0]])
+    while H.shape[0] < d:
+        H = np.block([[H, H], [H, -H]])
+    H = H[:, rng.permutation(d)] * rng.choice([-1.0, 1.0], d)[None, :]
+    return H / np.sqrt(d)
+
+
+def test_compressed_update_equals_the_ema_when_the_codes_are_exact():
+    # With a basis the codec stores exactly, U diag(lambda) U^T is the stored
+    # statistic itself, so the compressed update is the plain EMA of it.
+    rng = np.random.default_rng(21)
+    d = 64
+    U = _signed_hadamard(d, rng)
+    assert np.allclose(U.T @ U, np.eye(d), atol=1e-15) and not np.allclose(U, U.T)
+    lam = np.sort(rng.uniform(0.0, 3.0, d))[::-1].astype(np.float32)
+    f = O.Factor(d, np.zeros((d, d), np.float32))
+    f.codes, f.scales = O.quantize(U.astype(np.float32).ravel())
+    assert np.array_equal(O.dequantize(f.codes, f.scales, d * d).reshape(d, d), U.astype(np.float32))
+    f.lam = lam
+    f.has_basis = True
+    S_prev = (U * lam.astype(np.float64)[None, :]) @ U.T           # exact fp64 statistic
+    beta = float(np.float32(0.9))
+    for side, shape in (("L", (d, 40)), ("R", (40, d))):
+        G = rng.standard_normal(shape).astype(np.float32)
+        got = O.compressed_stats(f, G, beta, side)
+        g = G.astype(np.float64)
+        want = beta * S_prev + (1 - beta) * (g @ g.T if side == "L" else g.T @ g)
+        assert np.allclose(got, want, rtol=0, atol=2e-6 * np.abs(want).max()), side
+        # a transposed basis would rebuild a different matrix
+        wrong = (U.T * lam.astype(np.float64)[None, :]) @ U
+        assert not np.allclose(S_prev, wrong, atol=1e-3)
+
+
+def test_compressed_update_first_step_and_nonfinite():
+    rng = np.random.default_rng(22)
+    d = 16
+    f = O.Factor(d, np.zeros((d, d), np.float32))
+    G = rng.standard_normal((d, 24)).astype(np.float32)
+    beta = 0.8
+    # nothing stored yet: the EMA from zero
+    assert np.array_equal(O.compressed_stats(f, G, beta, "L"), O.ema_stats(f.S, G, beta, "L"))
+    # a non-finite gradient leaves the stored statistic: zero before any refresh ...
+    Gn = G.copy()
+    Gn[3, 5] = np.inf
+    assert np.array_equal(O.compressed_stats(f, Gn, beta, "L"), f.S)
+    # ... and the rebuilt U diag(lambda) U^T after one
+    f.S = O.compressed_stats(f, G, beta, "L")
+    O.refresh_factor(f, 1e-6, 5)
+    assert f.has_basis and f.lam.max() > 1.0
+    U = O.dequantize(f.codes, f.scales, d * d).reshape(d, d).astype(np.float64)
+    stored = (U * f.lam.astype(np.float64)[None, :]) @ U.T
+    assert np.allclose(O.compressed_stats(f, Gn, beta, "L"), stored, rtol=0, atol=1e-6 * np.abs(stored).max())
+
+
 # ------------------------------------------------------------ Bjorck (P4)
 
 def test_bjorck_closed_form_on_svd():
