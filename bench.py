@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-codec", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-graft", action="store_true")
+    ap.add_argument("--compressed", action="store_true",
+                    help="keep each statistic only as its 4-bit eigenbasis and eigenvalues")
     ap.add_argument("--shapes", default=None, help="comma-separated RxC list replacing the workload's shapes")
     ap.add_argument("--grad-sets", type=int, default=2,
                     help="seeded gradient sets the steps cycle through (1 = the same gradient every step)")
@@ -130,6 +132,7 @@ STAGE_BOUND = {
     "qr_trsm_panel": "3xtf32", "qr_solve_update": "3xtf32", "qr_solve_panel": "3xtf32",
     "qr_potrf": "latency", "qr_inverse": "latency", "rayleigh": "hbm", "requant": "hbm", "precond_dequant": "hbm",
     "basis": "hbm", "stats_scan": "hbm", "refresh_scan": "hbm", "qr_convert": "hbm", "precond_mu": "hbm",
+    "stats_dequant": "hbm", "stats_rebuild": "tf32",
 }
 
 
@@ -311,7 +314,7 @@ def main():
     dev_out = [torch.empty(s, dtype=torch.float32, device=dev) for s in shapes]
     host_out = [torch.empty(s, dtype=torch.float32).pin_memory() for s in shapes]
     sh = api.Shampoo4(shapes, beta=w.beta, eps=w.eps, max_block=w.max_block, bjorck_iters=w.bjorck_iters,
-                      precision=args.precision, device=dev)
+                      precision=args.precision, device=dev, compressed=args.compressed)
     stream = torch.cuda.current_stream()
 
     counter = [0]
@@ -383,6 +386,8 @@ def main():
             "data": "synthetic",
             "config": {"workload": w.name, "tiles": sh.nblocks, "factors": sh.nfactors,
                        "steps_per_refresh": 1,
+                       "statistics": "compressed (4-bit eigenbasis + eigenvalues)" if args.compressed else "fp32",
+                       "state_bytes": sh.state_bytes, "workspace_bytes": sh.workspace_bytes,
                        "gradients": f"{nsets} seeded set(s), step t uses set t mod {nsets}",
                        "l2": (f"inputs larger than L2 ({g_bytes / 1e9:.2f} GB of G, {stat_bytes / 1e9:.2f} GB "
                               f"of fp32 statistics; L2 is 0.126 GB)")},

@@ -33,10 +33,11 @@ class Shampoo4:
     """One handle: a fixed list of 2-D parameter shapes and their state."""
 
     def __init__(self, shapes, beta=0.95, eps=1e-6, max_block=1024, bjorck_iters=5,
-                 precision="tf32", device=None, reset=True):
+                 precision="tf32", device=None, reset=True, compressed=False):
         self.shapes = [(int(r), int(c)) for r, c in shapes]
+        self.compressed = bool(compressed)
         cfg = L.Config(beta, eps, max_block, 64, bjorck_iters,
-                       L.PREC_FP32 if precision == "fp32" else L.PREC_TF32)
+                       L.PREC_FP32 if precision == "fp32" else L.PREC_TF32, 1 if compressed else 0)
         params = (L.Param * len(self.shapes))(*[L.Param(r, c) for r, c in self.shapes])
         h = C.c_void_p()
         L.call("shampoo4_init", C.byref(cfg), params, len(self.shapes), C.byref(h))
@@ -127,14 +128,20 @@ class Shampoo4:
         return p.value, r0.value, c0.value, m.value, n.value
 
     def factor_views(self, f):
-        """(S, codes, scales, lambda) as tensor views into the state buffer."""
+        """(S, codes, scales, lambda) as tensor views into the state buffer
+        (with compressed statistics, S is the workspace copy the last
+        update_stats rebuilt)."""
         oS, oc, os_, ol = C.c_size_t(), C.c_size_t(), C.c_size_t(), C.c_size_t()
         d = C.c_int32()
         L.call("shampoo4_factor_layout", self._h, f, C.byref(oS), C.byref(oc), C.byref(os_), C.byref(ol), C.byref(d))
         d = d.value
         n = d * d
         st = self.state
-        S = st[oS.value:oS.value + 4 * n].view(torch.float32).view(d, d)
+        if self.compressed:
+            L.call("shampoo4_debug_s_offset", self._h, f, C.byref(oS))
+            S = self.workspace[oS.value:oS.value + 4 * n].view(torch.float32).view(d, d)
+        else:
+            S = st[oS.value:oS.value + 4 * n].view(torch.float32).view(d, d)
         codes = st[oc.value:oc.value + (n + 1) // 2]
         scales = st[os_.value:os_.value + 4 * ((n + 63) // 64)].view(torch.float32)
         lam = st[ol.value:ol.value + 4 * d].view(torch.float32)

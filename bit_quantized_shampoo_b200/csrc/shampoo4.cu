@@ -66,6 +66,7 @@ struct FactorPlan {
   int32_t block, side, d;
   bool tc;
   size_t st_S, st_codes, st_scales, st_lam;
+  size_t ws_S;                           // compressed statistics: S lives here
   size_t ws_mu;
   size_t ws_W64, ws_Q64, ws_U, ws_T, ws_Y;
   size_t ws_Xm[2], ws_Xh[2], ws_Xl[2], ws_Th, ws_Tl, ws_Sh, ws_Sl, ws_W;
@@ -94,7 +95,7 @@ struct shampoo4_ctx {
   bool any_simt = false;                 // some factor always takes the fp64 QR
   size_t ws_desc = 0, ws_desc_bytes = 0;
   // programs
-  std::vector<Launch> prog_stats, prog_refresh_first, prog_refresh, prog_precond;
+  std::vector<Launch> prog_stats, prog_stats_first, prog_refresh_first, prog_refresh, prog_precond;
   std::vector<uint8_t> arena;            // host image of the descriptor region
   std::vector<CUtensorMap> maps;         // host image of the tensor-map region
   // bound buffers
@@ -103,6 +104,7 @@ struct shampoo4_ctx {
   bool bound = false;
   bool has_basis = false;
   bool last_refresh_first = true;
+  bool stats_pending = false;            // compressed statistics: rebuilt S not yet refreshed
   // per-call pointer tables
   std::vector<PtrEntry> tab_host;  // last uploaded (2 * nparams)
   bool tab_valid = false;
@@ -216,7 +218,7 @@ shampoo4_status plan(shampoo4_ctx* h) {
       f.tc = tc_dim(f.d);
       if (!f.tc) h->any_simt = true;
       size_t dd = size_t(f.d) * f.d;
-      f.st_S = take(st, 4 * dd);
+      f.st_S = h->cfg.compressed_stats ? SIZE_MAX : take(st, 4 * dd);
       f.st_codes = take(st, (dd + 1) / 2);
       f.st_scales = take(st, 4 * ((dd + kQuantBlock - 1) / kQuantBlock));
       f.st_lam = take(st, 4 * size_t(f.d));
@@ -237,6 +239,7 @@ shampoo4_status plan(shampoo4_ctx* h) {
   h->ws_bflag = take(ws, 4 * h->blocks.size());
   for (FactorPlan& f : h->factors) {
     size_t dd = size_t(f.d) * f.d;
+    f.ws_S = h->cfg.compressed_stats ? take(ws, 4 * dd) : SIZE_MAX;
     f.ws_mu = take(ws, 4 * size_t(f.d));
     if (f.tc) {
       for (int i = 0; i < 2; ++i) {
@@ -329,6 +332,9 @@ struct Builder {
   uint32_t* wu(size_t off) const { return reinterpret_cast<uint32_t*>(ws + off); }
   float* sf(size_t off) const { return reinterpret_cast<float*>(stb + off); }
   uint8_t* sb(size_t off) const { return stb + off; }
+  // the factor's statistic: in the state, or (compressed statistics) in the
+  // workspace
+  float* S(const FactorPlan& f) const { return f.st_S == SIZE_MAX ? wf(f.ws_S) : sf(f.st_S); }
   uint32_t* fail(size_t fi) const { return wu(h->ws_fail) + fi; }
   uint32_t* tcbad(size_t fi) const { return wu(h->ws_tcbad) + fi; }
   uint32_t* tcgood(size_t fi) const { return wu(h->ws_tcgood) + fi; }
@@ -455,27 +461,87 @@ void build_grad_copy(Builder& b, std::vector<Launch>& prog, int tag, bool with_f
   b.emit(prog, Kind::Scan, scan, max_elems, 0, bytes);
 }
 
-void build_stats(Builder& b) {
+// The statistics update into `prog`.  With compressed statistics and
+// `rebuild`, the stored statistic is first rebuilt in the workspace as
+// U diag(lambda) U^T from the codes (k_basis with lambda as the column
+// scale, then one symmetric product), and the EMA reads it as Cin; without
+// `rebuild` (before the first refresh) the EMA starts from zero.
+void build_stats_into(Builder& b, std::vector<Launch>& prog, bool rebuild) {
   shampoo4_ctx* h = b.h;
   const bool split = split_of(h->cfg);
-  build_grad_copy(b, h->prog_stats, SHAMPOO4_STAGE_STATS_SCAN, true);
+  const bool compressed = h->cfg.compressed_stats != 0;
+  build_grad_copy(b, prog, SHAMPOO4_STAGE_STATS_SCAN, true);
+  if (compressed && rebuild) {
+    std::vector<BasisDesc> bd;
+    std::vector<TcGemmDesc> trec;
+    std::vector<GemmF32Desc> rec;
+    std::vector<RowDiagDesc> rdiag;
+    int dmax = 0;
+    int64_t emax = 0;
+    double bytes_bd = 0, sum_dd = 0;
+    for (const FactorPlan& f : h->factors) {
+      const int d = f.d;
+      dmax = std::max(dmax, d);
+      emax = std::max<int64_t>(emax, int64_t(d) * d);
+      sum_dd += double(d) * d;
+      BasisDesc x{};
+      x.codes = b.sb(f.st_codes); x.scales = b.sf(f.st_scales); x.d = d; x.identity = 0;
+      if (f.tc) {
+        // U -> X[0] split, U diag(lambda) -> X[1] split; S = (U lambda) U^T
+        x.Uh = b.wf(f.ws_Xh[0]); x.Ul = split ? b.wf(f.ws_Xl[0]) : nullptr;
+        x.mu = b.sf(f.st_lam);
+        x.Vh = b.wf(f.ws_Xh[1]); x.Vl = split ? b.wf(f.ws_Xl[1]) : nullptr;
+        TcGemmDesc g = gemmtc(d, d, d, 1.0f, 0.0f);
+        g.a = b.operand(b.wf(f.ws_Xh[1]), b.wf(f.ws_Xl[1]), d, d, true, false, split);
+        g.b = b.operand(b.wf(f.ws_Xh[0]), b.wf(f.ws_Xl[0]), d, d, false, true, split);
+        g.C = b.S(f); g.ldc = d;
+        g.symmetric = 1;                  // exactly symmetric: lower tiles, mirrored
+        trec.push_back(g);
+        if (split)
+          rdiag.push_back({b.wf(f.ws_Xh[1]), b.wf(f.ws_Xl[1]), b.wf(f.ws_Xh[0]), b.wf(f.ws_Xl[0]), d, d, 0,
+                           b.S(f), nullptr, nullptr});
+        bytes_bd += (0.5625 + 4.0 + (split ? 16.0 : 8.0)) * double(d) * d;
+      } else {
+        x.U = b.wf(f.ws_Y);
+        GemmF32Desc g = gemm32(d, d, d, 0, 1, mode_of(h->cfg), 1.0f, 0.0f);
+        g.A = b.wf(f.ws_Y); g.lda = d; g.kscale = b.sf(f.st_lam);
+        g.B = b.wf(f.ws_Y); g.ldb = d;
+        g.C = b.S(f); g.ldc = d;
+        g.symmetric = 1;
+        rec.push_back(g);
+        bytes_bd += (0.5625 + 4.0 + 4.0) * double(d) * d;
+      }
+      bd.push_back(x);
+    }
+    b.tag = SHAMPOO4_STAGE_STATS_DEQUANT;
+    b.emit(prog, Kind::Basis, bd, emax, 0, bytes_bd);
+    b.tag = SHAMPOO4_STAGE_STATS_REBUILD;
+    emit_gemmtc(b, prog, trec, split);
+    b.emit(prog, Kind::RowDiag, rdiag, dmax, 0, 16.0 * sum_dd);
+    emit_gemm32(b, prog, rec);
+  }
   std::vector<GemmF32Desc> g;
   std::vector<TcGemmDesc> t;
-  const float beta = h->cfg.beta, omb = 1.0f - h->cfg.beta;
+  // EMA: S <- beta S + (1 - beta) G G^T; compressed statistics read the
+  // rebuilt S with weight beta, or start from zero
+  const float omb = 1.0f - h->cfg.beta;
+  const float beta = (compressed && !rebuild) ? 0.0f : h->cfg.beta;
   for (size_t k = 0; k < h->blocks.size(); ++k) {
     const BlockPlan& bp = h->blocks[k];
     uint32_t* skip = b.wu(h->ws_bflag) + k;
     for (int side = 0; side < 2; ++side) {
       const FactorPlan& f = h->factors[2 * k + side];
       const int d = f.d, kk = side == 0 ? bp.n : bp.m;
+      float* S = b.S(f);
+      const float* Cin = beta == 0.0f ? nullptr : S;
       if (bp.tc) {
         // L: A = G (K-major), B = G^T as op(B)[k,j] = G[j,k] (K-major).
         // R: A = G^T (MN-major), B = G (MN-major).
         TcGemmDesc x = gemmtc(d, d, kk, omb, beta);
         x.a = b.operand(b.wf(bp.ws_Gh), b.wf(bp.ws_Gl), bp.m, bp.n, true, side == 1, split);
         x.b = b.operand(b.wf(bp.ws_Gh), b.wf(bp.ws_Gl), bp.m, bp.n, false, side == 0, split);
-        x.C = b.sf(f.st_S); x.ldc = d;
-        x.Cin = x.C; x.ldcin = d;
+        x.C = S; x.ldc = d;
+        x.Cin = Cin; x.ldcin = d;
         x.symmetric = 1;
         x.skip = skip;
         t.push_back(x);
@@ -484,8 +550,8 @@ void build_stats(Builder& b) {
                                   : gemm32(d, d, kk, 1, 0, mode_of(h->cfg), omb, beta);
         x.a_ref = {0, bp.param, bp.r0, bp.c0};
         x.b_ref = x.a_ref;
-        x.C = b.sf(f.st_S); x.ldc = d;
-        x.Cin = x.C; x.ldcin = d;
+        x.C = S; x.ldc = d;
+        x.Cin = Cin; x.ldcin = d;
         x.symmetric = 1;
         x.skip = skip;
         g.push_back(x);
@@ -493,8 +559,14 @@ void build_stats(Builder& b) {
     }
   }
   b.tag = SHAMPOO4_STAGE_STATS_GEMM;
-  emit_gemmtc(b, h->prog_stats, t, split);
-  emit_gemm32(b, h->prog_stats, g);
+  emit_gemmtc(b, prog, t, split);
+  emit_gemm32(b, prog, g);
+}
+
+void build_stats(Builder& b) {
+  shampoo4_ctx* h = b.h;
+  build_stats_into(b, h->prog_stats, true);
+  if (h->cfg.compressed_stats) build_stats_into(b, h->prog_stats_first, false);
 }
 
 // fp64 Cholesky-QR pass over the factors with use[i]: X (fp32, d x d) -> Q
@@ -826,7 +898,7 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
       ScanDesc s{};
-      s.X = b.sf(f.st_S); s.ld = f.d; s.rows = s.cols = f.d;
+      s.X = b.S(f); s.ld = f.d; s.rows = s.cols = f.d;
       s.ref.tab = -1;
       s.flag = b.fail(i);
       s.bit = SHAMPOO4_FLAG_NONFINITE_STATE;
@@ -943,7 +1015,7 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
         Ql[i] = b.wf(f.ws_Xl[c]);
       } else {
         GemmF32Desc y = gemm32(d, d, d, 0, 0, kModeFP32, 1.0f, h->cfg.eps);
-        y.A = b.sf(f.st_S); y.lda = d;
+        y.A = b.S(f); y.lda = d;
         y.B = b.wf(ucur[i]); y.ldb = d;
         y.C = b.wf(uoth[i]); y.ldc = d;
         y.Cin = b.wf(ucur[i]); y.ldcin = d;
@@ -1030,7 +1102,7 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
       } else {
         T = b.wf(f.ws_T);
         GemmF32Desc x = gemm32(d, d, d, 0, 0, kModeFP32, 1.0f, 0.0f);
-        x.A = b.sf(f.st_S); x.lda = d;
+        x.A = b.S(f); x.lda = d;
         x.B = Qf[i]; x.ldb = d;
         x.C = T; x.ldc = d;
         g.push_back(x);
@@ -1324,6 +1396,7 @@ extern "C" shampoo4_status shampoo4_init(const shampoo4_config* cfg, const shamp
   if (cfg->bjorck_iters < 0 || cfg->bjorck_iters > 16) return SHAMPOO4_ERR_INVALID_ARG;
   if (cfg->precision != SHAMPOO4_PREC_TF32 && cfg->precision != SHAMPOO4_PREC_FP32)
     return SHAMPOO4_ERR_INVALID_ARG;
+  if (cfg->compressed_stats != 0 && cfg->compressed_stats != 1) return SHAMPOO4_ERR_INVALID_ARG;
   for (int32_t i = 0; i < nparams; ++i)
     if (params[i].rows < 1 || params[i].cols < 1 || params[i].rows > (1LL << 31) ||
         params[i].cols > (1LL << 31))
@@ -1346,7 +1419,8 @@ extern "C" shampoo4_status shampoo4_init(const shampoo4_config* cfg, const shamp
   h->ws_desc = align_up(h->ws_maps + h->ws_nmaps * sizeof(CUtensorMap), kAlign);
   h->ws_desc_bytes = align_up(h->arena.size(), kAlign);
   h->ws_bytes = h->ws_desc + h->ws_desc_bytes;
-  h->prog_stats.clear(); h->prog_refresh_first.clear(); h->prog_refresh.clear(); h->prog_precond.clear();
+  h->prog_stats.clear(); h->prog_stats_first.clear(); h->prog_refresh_first.clear(); h->prog_refresh.clear();
+  h->prog_precond.clear();
   h->arena.clear();
   h->maps.clear();
   *out = h;
@@ -1380,7 +1454,8 @@ extern "C" shampoo4_status shampoo4_bind(shampoo4_handle h, void* d_state, void*
   if (h->gtab_event_pending) S4_CUDA(cudaEventSynchronize(h->gtab_event));
   h->d_state = static_cast<uint8_t*>(d_state);
   h->d_ws = static_cast<uint8_t*>(d_workspace);
-  h->prog_stats.clear(); h->prog_refresh_first.clear(); h->prog_refresh.clear(); h->prog_precond.clear();
+  h->prog_stats.clear(); h->prog_stats_first.clear(); h->prog_refresh_first.clear(); h->prog_refresh.clear();
+  h->prog_precond.clear();
   h->arena.clear();
   h->maps.clear();
   Builder b{h, h->arena, h->d_ws, h->d_state, true};
@@ -1403,6 +1478,7 @@ extern "C" shampoo4_status shampoo4_bind(shampoo4_handle h, void* d_state, void*
     S4_CUDA(cudaMemsetAsync(h->d_state, 0, h->state_bytes, st));
     h->has_basis = false;
   }
+  h->stats_pending = false;
   S4_CUDA(cudaStreamSynchronize(st));   // the host arena is reused by the next bind
   h->tab_valid = false;
   h->gtab_valid = false;
@@ -1422,14 +1498,19 @@ extern "C" shampoo4_status shampoo4_update_stats(shampoo4_handle h, const float*
   if (!h->bound) return SHAMPOO4_ERR_NOT_READY;
   S4_TRY(check_matrices(h, d_grads, ld));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (h->cfg.compressed_stats && h->stats_pending) return SHAMPOO4_ERR_NOT_READY;
   S4_TRY(set_tables(h, d_grads, ld, nullptr, nullptr, st));
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_bflag, 0, 4 * h->blocks.size(), st));
-  return run(h, h->prog_stats, st);
+  const bool rebuild = !h->cfg.compressed_stats || h->has_basis;
+  S4_TRY(run(h, rebuild ? h->prog_stats : h->prog_stats_first, st));
+  h->stats_pending = h->cfg.compressed_stats != 0;
+  return SHAMPOO4_OK;
 }
 
 extern "C" shampoo4_status shampoo4_refresh_roots(shampoo4_handle h, shampoo4_stream_t stream) {
   if (!h) return SHAMPOO4_ERR_INVALID_ARG;
   if (!h->bound) return SHAMPOO4_ERR_NOT_READY;
+  if (h->cfg.compressed_stats && !h->stats_pending) return SHAMPOO4_ERR_NOT_READY;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_fail, 0, 4 * h->factors.size(), st));
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_tcbad, 0, 4 * h->factors.size(), st));
@@ -1440,6 +1521,7 @@ extern "C" shampoo4_status shampoo4_refresh_roots(shampoo4_handle h, shampoo4_st
   S4_TRY(run(h, first ? h->prog_refresh_first : h->prog_refresh, st));
   h->last_refresh_first = first;
   h->has_basis = true;
+  h->stats_pending = false;
   return SHAMPOO4_OK;
 }
 
@@ -1516,6 +1598,13 @@ extern "C" shampoo4_status shampoo4_debug_q_offset(shampoo4_handle h, int32_t fa
   return SHAMPOO4_OK;
 }
 
+extern "C" shampoo4_status shampoo4_debug_s_offset(shampoo4_handle h, int32_t factor, size_t* off_s) {
+  if (!h || !off_s || !h->cfg.compressed_stats || factor < 0 || size_t(factor) >= h->factors.size())
+    return SHAMPOO4_ERR_INVALID_ARG;
+  *off_s = h->factors[factor].ws_S;
+  return SHAMPOO4_OK;
+}
+
 extern "C" shampoo4_status shampoo4_timing_enable(shampoo4_handle h, int32_t enable) {
   if (!h) return SHAMPOO4_ERR_INVALID_ARG;
   S4_TRY(collect_timing(h));
@@ -1543,7 +1632,7 @@ extern "C" const char* shampoo4_stage_name(int32_t stage) {
       "stats_scan", "stats_gemm", "refresh_scan", "basis", "bjorck_gram", "bjorck_update",
       "subspace", "qr_gram", "qr_potrf", "qr_trsm_panel", "qr_syrk", "qr_solve_update",
       "qr_solve_panel", "qr_convert", "rayleigh_gemm", "rayleigh", "requant", "precond_dequant",
-      "precond_mu", "roots", "apply_left", "apply_right", "qr_inverse"};
+      "precond_mu", "roots", "apply_left", "apply_right", "qr_inverse", "stats_dequant", "stats_rebuild"};
   if (stage < 0 || stage >= SHAMPOO4_STAGE_COUNT) return "unknown";
   return names[stage];
 }

@@ -82,6 +82,19 @@ typedef struct {
   int32_t quant_block;   /* elements per quantization scale; must be 64    */
   int32_t bjorck_iters;  /* Bjorck rectification steps per refresh, 0..16  */
   int32_t precision;     /* shampoo4_precision                             */
+  int32_t compressed_stats; /* 0: each factor keeps its fp32 statistic S in
+                            the state.  1: the statistic is kept only as its
+                            4-bit eigenvector codes and eigenvalues ("4-bit
+                            Shampoo ...", abstract: the preconditioner is
+                            stored through its quantized eigenvector
+                            matrix); update_stats rebuilds
+                            S = beta U diag(lambda) U^T + (1-beta) G G^T
+                            (U dequantized, no Bjorck) in the workspace, and
+                            every update_stats must be followed by a
+                            refresh_roots before the next one (the refresh
+                            is what stores the new statistic; otherwise
+                            ERR_NOT_READY).  The state shrinks by 4 d^2
+                            bytes per factor.                               */
 } shampoo4_config;
 
 typedef struct { int64_t rows, cols; } shampoo4_param;   /* 2-D weights only;
@@ -171,7 +184,9 @@ shampoo4_status shampoo4_block_info(shampoo4_handle h, int32_t block, int32_t* p
 /* Byte offsets inside the state buffer of one factor's statistic S (fp32
  * d x d, row-major, dense), codes (uint8, ceil(d*d/2), two per byte, element
  * 2i in the low nibble), scales (fp32, ceil(d*d/64)) and eigenvalues (fp32,
- * d); *dim receives d.  Any pointer may be NULL. */
+ * d); *dim receives d.  Any pointer may be NULL.  With compressed_stats the
+ * statistic is not part of the state: *off_S receives SIZE_MAX (see
+ * shampoo4_debug_s_offset). */
 shampoo4_status shampoo4_factor_layout(shampoo4_handle h, int32_t factor, size_t* off_S,
                                        size_t* off_codes, size_t* off_scales,
                                        size_t* off_lambda, int32_t* dim);
@@ -180,6 +195,12 @@ shampoo4_status shampoo4_factor_layout(shampoo4_handle h, int32_t factor, size_t
  * last refresh quantized for this factor (valid until the next call that uses
  * the workspace).  For tests and diagnostics. */
 shampoo4_status shampoo4_debug_q_offset(shampoo4_handle h, int32_t factor, size_t* off_q);
+
+/* With compressed_stats: byte offset inside the workspace of the fp32 d x d
+ * statistic that the last update_stats rebuilt for this factor (valid until
+ * the next refresh_roots).  ERR_INVALID_ARG without compressed_stats.  For
+ * tests and diagnostics. */
+shampoo4_status shampoo4_debug_s_offset(shampoo4_handle h, int32_t factor, size_t* off_s);
 
 /* Stages of the three programs, for the optional launch timing below. */
 typedef enum {
@@ -190,7 +211,8 @@ typedef enum {
   SHAMPOO4_STAGE_QR_SOLVE_PANEL, SHAMPOO4_STAGE_QR_CONVERT, SHAMPOO4_STAGE_RAYLEIGH_GEMM,
   SHAMPOO4_STAGE_RAYLEIGH, SHAMPOO4_STAGE_REQUANT, SHAMPOO4_STAGE_PRECOND_DEQUANT,
   SHAMPOO4_STAGE_PRECOND_MU, SHAMPOO4_STAGE_ROOTS, SHAMPOO4_STAGE_APPLY_LEFT,
-  SHAMPOO4_STAGE_APPLY_RIGHT, SHAMPOO4_STAGE_QR_INVERSE, SHAMPOO4_STAGE_COUNT
+  SHAMPOO4_STAGE_APPLY_RIGHT, SHAMPOO4_STAGE_QR_INVERSE, SHAMPOO4_STAGE_STATS_DEQUANT,
+  SHAMPOO4_STAGE_STATS_REBUILD, SHAMPOO4_STAGE_COUNT
 } shampoo4_stage;
 
 /* Launch timing, for diagnostics and roofline figures.  While enabled, every

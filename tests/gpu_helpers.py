@@ -46,3 +46,34 @@ def basis_root(Q, lam, eps):
     Q = np.asarray(Q, np.float64)
     mu = (np.asarray(lam, np.float64) + eps) ** -0.25
     return (Q * mu[None, :]) @ Q.T
+
+
+def refresh_errors(sh, orc, eps):
+    """After sh.refresh_roots() and orc.refresh_roots() from the same incoming
+    state: per factor (d, ||Q^T Q - I||_F/sqrt(d), lambda excess, root excess),
+    with the requantized codes checked bit-exact against the oracle quantizer
+    applied to the library's own Q.  The lambda and root excesses are taken
+    over the fp32-accurate arithmetic's resolution, as in the stage tests:
+    about 16 u lambda_max for lambda and u kappa for the basis-invariant root
+    (u = 2^-21), nothing pinned beyond u32 kappa >= 1."""
+    out = []
+    for f in range(sh.nfactors):
+        d = orc.factors[f].d
+        Qg = sh.debug_q(f).cpu().numpy().astype(np.float64)
+        g = gpu_factor(sh, f)
+        oc, os_ = O.quantize(Qg.astype(np.float32).ravel())
+        assert np.array_equal(g.codes, oc) and np.array_equal(g.scales, os_), f
+        orth = float(np.linalg.norm(Qg.T @ Qg - np.eye(d)) / np.sqrt(d))
+        Qo, lo = orc.factors[f].q_last, orc.factors[f].lam.astype(np.float64)
+        lg = g.lam.astype(np.float64)
+        big = lo > 1e3 * eps
+        slack = 16 * 2.0 ** -21 * lo.max()
+        excess = np.maximum(np.abs(lg - lo) - slack, 0.0)
+        lam_err = float(np.max(excess[big] / lo[big])) if big.any() else 0.0
+        kappa = (lo.max() + eps) / (lo.min() + eps)
+        root_err = rel_fro(basis_root(Qg, lo, eps), basis_root(Qo, lo, eps))
+        root_err = max(root_err - 2.0 ** -21 * kappa, 0.0)
+        if 6e-8 * kappa >= 1.0:
+            root_err = 0.0
+        out.append((d, orth, lam_err, root_err))
+    return out

@@ -39,7 +39,7 @@ def test_codec_tables_match_the_oracle_definition():
 
 def _init(shapes, **kw):
     cfg = L.Config(kw.get("beta", 0.95), kw.get("eps", 1e-6), kw.get("max_block", 1024), kw.get("qb", 64),
-                   kw.get("bj", 5), kw.get("prec", 0))
+                   kw.get("bj", 5), kw.get("prec", 0), kw.get("compressed", 0))
     params = (L.Param * len(shapes))(*[L.Param(r, c) for r, c in shapes])
     h = C.c_void_p()
     st = L.lib().shampoo4_init(C.byref(cfg), params, len(shapes), C.byref(h))
@@ -86,7 +86,7 @@ def test_plan_matches_oracle_partition(wid):
 
 def test_init_rejects_bad_configs():
     bad = [dict(beta=1.0), dict(beta=-0.1), dict(eps=0.0), dict(max_block=0), dict(max_block=2048),
-           dict(qb=32), dict(bj=-1), dict(bj=17), dict(prec=2)]
+           dict(qb=32), dict(bj=-1), dict(bj=17), dict(prec=2), dict(compressed=2)]
     for kw in bad:
         st, h = _init([(8, 8)], **kw)
         assert st == 1, kw
@@ -144,3 +144,34 @@ def test_graft_state_layout_and_argument_checks():
                                          ptrs, lds, None) == 1
     finally:
         L.lib().shampoo4_destroy(h)
+
+
+def test_compressed_statistics_leave_the_state_and_move_to_the_workspace():
+    shapes = [(300, 260), (64, 147)]
+    sizes = {}
+    for comp in (0, 1):
+        st, h = _init(shapes, max_block=256, compressed=comp)
+        assert st == 0
+        try:
+            sb, wb = C.c_size_t(), C.c_size_t()
+            L.call("shampoo4_sizes", h, C.byref(sb), C.byref(wb))
+            sizes[comp] = (sb.value, wb.value)
+            nb, nf = C.c_int32(), C.c_int32()
+            L.call("shampoo4_counts", h, C.byref(nb), C.byref(nf))
+            dd = 0
+            for f in range(nf.value):
+                oS, d = C.c_size_t(), C.c_int32()
+                L.call("shampoo4_factor_layout", h, f, C.byref(oS), None, None, None, C.byref(d))
+                dd += d.value * d.value
+                off = C.c_size_t()
+                if comp:
+                    assert oS.value == C.c_size_t(-1).value          # SIZE_MAX: not in the state
+                    L.call("shampoo4_debug_s_offset", h, f, C.byref(off))
+                    assert off.value % 256 == 0 and off.value + 4 * d.value ** 2 <= wb.value
+                else:
+                    assert L.lib().shampoo4_debug_s_offset(h, f, C.byref(off)) == 1
+        finally:
+            L.lib().shampoo4_destroy(h)
+    # the state loses every statistic (4 d^2 bytes per factor); the workspace gains them
+    assert sizes[0][0] - sizes[1][0] >= 4 * dd
+    assert sizes[1][1] - sizes[0][1] >= 4 * dd
