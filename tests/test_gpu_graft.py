@@ -78,7 +78,10 @@ def test_graft_update_matches_oracle(kind, case):
             e = rel_fro(step_g, step_o)
             print(f"{case} {kind} t={t} param {p} {shapes[p]}: step {e:.2e}")
             assert e <= TOL_STEP, (t, p)
-    assert sh.status_flags() == 0
+    # ragged tiles have rank-deficient statistics whose QR may be redone in
+    # fp64 (an informational flag); nothing else may be raised
+    from bit_quantized_shampoo_b200 import _lib
+    assert sh.status_flags() & ~_lib.FLAG_QR_FALLBACK == 0
 
 
 def test_graft_step_norm_per_tile_on_the_gpu():
