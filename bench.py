@@ -397,26 +397,58 @@ def main():
             "clocks": clocks, "roofline": roof, "rooflines_other": others,
             "stages_ms": {k: round(v["ms"], 4) for k, v in sorted(stages.items(), key=lambda kv: -kv[1]["ms"])}}
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: every step copies
+    # its gradients in from pinned host memory and its update out to pinned
+    # host memory.  The copies run on a second stream, double-buffered, so
+    # step t+1's gradients load and step t's update drains while the GPU
+    # computes (the first load and the last drain are exposed).
     if not args.no_e2e:
         torch.cuda.synchronize()
-        k = max(1, min(args.steps, 3))
+        k = max(2, args.steps)
+        copy_s = torch.cuda.Stream(device=dev)
+        gbuf = [dev_sets[0], dev_sets[1] if nsets > 1 else [torch.empty_like(x) for x in dev_sets[0]]]
+        obuf = [dev_out, [torch.empty_like(x) for x in dev_out]]
+        hout = [host_out, [torch.empty(s, dtype=torch.float32).pin_memory() for s in shapes]]
+        loaded = [torch.cuda.Event(), torch.cuda.Event()]
+        done = [torch.cuda.Event(), torch.cuda.Event()]
         e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def load(i):
+            slot = i % 2
+            if i >= 2:
+                copy_s.wait_event(done[slot])              # step i-2 has finished reading this slot
+            with torch.cuda.stream(copy_s):
+                for h, d in zip(host_sets[i % nsets], gbuf[slot]):
+                    d.copy_(h, non_blocking=True)
+            loaded[slot].record(copy_s)
+
         e2.record(stream)
-        for _ in range(k):
-            s = counter[0] % nsets
-            for h, d in zip(host_sets[s], dev_sets[s]):
-                d.copy_(h, non_blocking=True)
-            step()
-            for d, h in zip(dev_out, host_out):
-                h.copy_(d, non_blocking=True)
+        copy_s.wait_event(e2)
+        load(0)
+        for i in range(k):
+            slot = i % 2
+            stream.wait_event(loaded[slot])
+            g = gbuf[slot]
+            sh.update_stats(g)
+            sh.refresh_roots()
+            sh.precondition(g, out=obuf[slot])
+            done[slot].record(stream)
+            if i + 1 < k:
+                load(i + 1)
+            copy_s.wait_event(done[slot])
+            with torch.cuda.stream(copy_s):
+                for d, h in zip(obuf[slot], hout[slot]):
+                    h.copy_(d, non_blocking=True)
+        stream.wait_stream(copy_s)
         e3.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(e2.elapsed_time(e3), dev)
         bi = sum(h.numel() * 4 for h in host_g)
         bo = sum(h.numel() * 4 for h in host_out)
-        line["e2e"] = {"value": job_rate(world, k, ems), "unit": "steps/s", "h2d_bytes_per_step": bi,
-                       "d2h_bytes_per_step": bo}
+        line["e2e"] = {"value": job_rate(world, k, ems), "unit": "steps/s", "steps": k, "h2d_bytes_per_step": bi,
+                       "d2h_bytes_per_step": bo,
+                       "copies": "pinned host buffers, second stream, double-buffered (overlapped with compute)"}
+        del gbuf, obuf, hout
 
     # stand-alone codec bandwidth on eigenvector-shaped tensors of the workload's size
     if not args.no_codec:

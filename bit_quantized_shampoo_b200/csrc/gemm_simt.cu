@@ -101,7 +101,11 @@ k_gemm_f32(const GemmF32Desc* __restrict__ descs, const PtrEntry* __restrict__ t
     }
     __syncthreads();
   }
-  const bool mirror = g.symmetric && tm != tn;
+  // symmetric output: every element below the diagonal is written twice,
+  // at (i, j) and (j, i), from one accumulator -- also inside diagonal tiles,
+  // where a product whose operands are scaled on one side only (kscale)
+  // would otherwise round differently at (i, j) and (j, i)
+  const bool diag_tile = g.symmetric && tm == tn;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     int gi = m0 + ty + 16 * i;
@@ -110,6 +114,8 @@ k_gemm_f32(const GemmF32Desc* __restrict__ descs, const PtrEntry* __restrict__ t
     for (int j = 0; j < 8; ++j) {
       int gj = n0 + tx + 16 * j;
       if (gj >= g.N) continue;
+      if (diag_tile && gj > gi) continue;     // written by its mirror
+      const bool mirror = g.symmetric && gj != gi;
       float v = g.alpha * acc[i][j];
       if (g.beta != 0.0f) v = fmaf(g.beta, g.Cin[int64_t(gi) * g.ldcin + gj], v);
       C[int64_t(gi) * ldc + gj] = v;

@@ -100,7 +100,9 @@ def test_compressed_call_order():
     sh.update_stats(G)                               # stored: the next update may run
     sh.refresh_roots()
     torch.cuda.synchronize()
-    assert sh.status_flags() == 0
+    # a 64-row tile's 96 x 96 statistic is rank-deficient: its QR may be
+    # redone in fp64 (an informational flag); nothing else may be raised
+    assert sh.status_flags() & ~0x10 == 0
 
 
 def test_compressed_nonfinite_gradient_keeps_the_stored_statistic():
