@@ -209,6 +209,10 @@ __global__ void __launch_bounds__(256) k_mu(const MuDesc* __restrict__ descs, fl
   const MuDesc& g = descs[blockIdx.y];
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= g.d) return;
+  if (g.sqrt_mode) {
+    g.mu[i] = float(sqrt(fmax(double(g.lam[i]), 0.0)));
+    return;
+  }
   double x = double(g.lam[i]) + double(eps);
   g.mu[i] = float(1.0 / sqrt(sqrt(x)));
 }

@@ -103,10 +103,12 @@ struct RayleighDesc {
 };
 
 // mu_i = (lambda_i + eps)^(-1/4)
+// mu_i = (lambda_i + eps)^(-1/4) (the root's scale), or, with sqrt_mode,
+// sqrt(max(lambda_i, 0)) (the half scale of a rebuilt U diag(lambda) U^T).
 struct MuDesc {
   const float* lam;
   float* mu;
-  int32_t d; int32_t pad_;
+  int32_t d; int32_t sqrt_mode;
 };
 
 // Scan a matrix (absolute or per-call) for NaN/Inf; on one, set *flag = 1

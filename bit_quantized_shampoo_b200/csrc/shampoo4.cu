@@ -472,6 +472,7 @@ void build_stats_into(Builder& b, std::vector<Launch>& prog, bool rebuild) {
   const bool compressed = h->cfg.compressed_stats != 0;
   build_grad_copy(b, prog, SHAMPOO4_STAGE_STATS_SCAN, true);
   if (compressed && rebuild) {
+    std::vector<MuDesc> half;
     std::vector<BasisDesc> bd;
     std::vector<TcGemmDesc> trec;
     std::vector<GemmF32Desc> rec;
@@ -487,20 +488,22 @@ void build_stats_into(Builder& b, std::vector<Launch>& prog, bool rebuild) {
       BasisDesc x{};
       x.codes = b.sb(f.st_codes); x.scales = b.sf(f.st_scales); x.d = d; x.identity = 0;
       if (f.tc) {
-        // U -> X[0] split, U diag(lambda) -> X[1] split; S = (U lambda) U^T
-        x.Uh = b.wf(f.ws_Xh[0]); x.Ul = split ? b.wf(f.ws_Xl[0]) : nullptr;
-        x.mu = b.sf(f.st_lam);
+        // V = U diag(sqrt(lambda)) -> X[1] split; S = V V^T.  The same
+        // rounded V on both sides keeps S positive semidefinite (up to the
+        // fp32 accumulation), as G G^T is, whatever the operand rounding.
+        half.push_back({b.sf(f.st_lam), b.wf(f.ws_mu), d, 1});
+        x.mu = b.wf(f.ws_mu);
         x.Vh = b.wf(f.ws_Xh[1]); x.Vl = split ? b.wf(f.ws_Xl[1]) : nullptr;
         TcGemmDesc g = gemmtc(d, d, d, 1.0f, 0.0f);
         g.a = b.operand(b.wf(f.ws_Xh[1]), b.wf(f.ws_Xl[1]), d, d, true, false, split);
-        g.b = b.operand(b.wf(f.ws_Xh[0]), b.wf(f.ws_Xl[0]), d, d, false, true, split);
+        g.b = b.operand(b.wf(f.ws_Xh[1]), b.wf(f.ws_Xl[1]), d, d, false, true, split);
         g.C = b.S(f); g.ldc = d;
         g.symmetric = 1;                  // exactly symmetric: lower tiles, mirrored
         trec.push_back(g);
         if (split)
-          rdiag.push_back({b.wf(f.ws_Xh[1]), b.wf(f.ws_Xl[1]), b.wf(f.ws_Xh[0]), b.wf(f.ws_Xl[0]), d, d, 0,
+          rdiag.push_back({b.wf(f.ws_Xh[1]), b.wf(f.ws_Xl[1]), b.wf(f.ws_Xh[1]), b.wf(f.ws_Xl[1]), d, d, 0,
                            b.S(f), nullptr, nullptr});
-        bytes_bd += (0.5625 + 4.0 + (split ? 16.0 : 8.0)) * double(d) * d;
+        bytes_bd += (0.5625 + 4.0 + (split ? 8.0 : 4.0)) * double(d) * d;
       } else {
         x.U = b.wf(f.ws_Y);
         GemmF32Desc g = gemm32(d, d, d, 0, 1, mode_of(h->cfg), 1.0f, 0.0f);
@@ -514,6 +517,7 @@ void build_stats_into(Builder& b, std::vector<Launch>& prog, bool rebuild) {
       bd.push_back(x);
     }
     b.tag = SHAMPOO4_STAGE_STATS_DEQUANT;
+    b.emit(prog, Kind::Mu, half, dmax);
     b.emit(prog, Kind::Basis, bd, emax, 0, bytes_bd);
     b.tag = SHAMPOO4_STAGE_STATS_REBUILD;
     emit_gemmtc(b, prog, trec, split);
