@@ -35,7 +35,7 @@ PREC_FP32 = 1
 class Config(C.Structure):
     _fields_ = [("beta", C.c_float), ("eps", C.c_float), ("max_block", C.c_int32),
                 ("quant_block", C.c_int32), ("bjorck_iters", C.c_int32), ("precision", C.c_int32),
-                ("compressed_stats", C.c_int32)]
+                ("compressed_stats", C.c_int32), ("refresh_rank", C.c_int32), ("refresh_world", C.c_int32)]
 
 
 class GraftConfig(C.Structure):
@@ -68,6 +68,8 @@ _SIGS = {
     "shampoo4_factor_layout": [C.c_void_p, C.c_int32, c_size_p, c_size_p, c_size_p, c_size_p, c_i32_p],
     "shampoo4_debug_q_offset": [C.c_void_p, C.c_int32, c_size_p],
     "shampoo4_debug_s_offset": [C.c_void_p, C.c_int32, c_size_p],
+    "shampoo4_factor_owner": [C.c_void_p, C.c_int32, c_i32_p],
+    "shampoo4_owner_span": [C.c_void_p, C.c_int32, c_size_p, c_size_p],
     "quant4_pack": [C.POINTER(C.c_void_p), c_i64_p, C.c_int32, C.POINTER(C.c_void_p),
                     C.POINTER(C.c_void_p), C.c_void_p],
     "quant4_unpack": [C.POINTER(C.c_void_p), C.POINTER(C.c_void_p), c_i64_p, C.c_int32,

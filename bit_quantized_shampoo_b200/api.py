@@ -33,11 +33,13 @@ class Shampoo4:
     """One handle: a fixed list of 2-D parameter shapes and their state."""
 
     def __init__(self, shapes, beta=0.95, eps=1e-6, max_block=1024, bjorck_iters=5,
-                 precision="tf32", device=None, reset=True, compressed=False):
+                 precision="tf32", device=None, reset=True, compressed=False, refresh_rank=0, refresh_world=1):
         self.shapes = [(int(r), int(c)) for r, c in shapes]
         self.compressed = bool(compressed)
+        self.refresh_rank, self.refresh_world = int(refresh_rank), int(refresh_world)
         cfg = L.Config(beta, eps, max_block, 64, bjorck_iters,
-                       L.PREC_FP32 if precision == "fp32" else L.PREC_TF32, 1 if compressed else 0)
+                       L.PREC_FP32 if precision == "fp32" else L.PREC_TF32, 1 if compressed else 0,
+                       self.refresh_rank, self.refresh_world)
         params = (L.Param * len(self.shapes))(*[L.Param(r, c) for r, c in self.shapes])
         h = C.c_void_p()
         L.call("shampoo4_init", C.byref(cfg), params, len(self.shapes), C.byref(h))
@@ -116,6 +118,30 @@ class Shampoo4:
         L.call("shampoo4_graft_update", self._h, C.byref(cfg), sp, int(step), float(lr), p, ld, q, ldq, w, ldw,
                _stream(stream))
 
+    # ---- refresh sharding ("Shampoo -- Second-Order Optimizer", "Blocked and
+    # distributed variants")
+
+    def owner_spans(self):
+        """[(offset, bytes)] per rank: the state range holding the codes,
+        scales and eigenvalues of the factors that rank refreshes."""
+        out = []
+        for r in range(max(1, self.refresh_world)):
+            off, n = C.c_size_t(), C.c_size_t()
+            L.call("shampoo4_owner_span", self._h, r, C.byref(off), C.byref(n))
+            out.append((off.value, n.value))
+        return out
+
+    def factor_owner(self, f):
+        r = C.c_int32()
+        L.call("shampoo4_factor_owner", self._h, f, C.byref(r))
+        return r.value
+
+    def exchange_roots(self, group=None):
+        """After refresh_roots on every rank: each rank's freshly refreshed
+        span goes to all ranks (one torch.distributed broadcast per rank, on
+        the state buffer in place).  Plumbing only."""
+        exchange_spans(self.state, self.owner_spans(), group)
+
     def status_flags(self, stream=None) -> int:
         f = C.c_uint32()
         L.call("shampoo4_get_status_flags", self._h, C.byref(f), _stream(stream))
@@ -163,6 +189,16 @@ class Shampoo4:
             self.close()
         except Exception:
             pass
+
+
+def exchange_spans(buf, spans, group=None):
+    """Broadcast buf[off:off + n] from rank r to every rank, for each rank's
+    (off, n) in ``spans`` (rank order).  ``buf`` is a 1-D uint8 tensor on the
+    process group's device."""
+    import torch.distributed as dist
+    for r, (off, n) in enumerate(spans):
+        if n:
+            dist.broadcast(buf[off:off + n], src=r, group=group)
 
 
 def _graft_kind(kind):

@@ -105,6 +105,13 @@ struct shampoo4_ctx {
   bool has_basis = false;
   bool last_refresh_first = true;
   bool stats_pending = false;            // compressed statistics: rebuilt S not yet refreshed
+  // refresh sharding: factor f is refreshed by rank owner[f] of world; this
+  // handle's rank keeps statistics and refreshes only its own factors, and
+  // the codes, scales and eigenvalues of rank r's factors form one
+  // contiguous state span [span_off[r], span_off[r] + span_bytes[r])
+  int32_t rank = 0, world = 1;
+  std::vector<int32_t> owner;
+  std::vector<size_t> span_off, span_bytes;
   // per-call pointer tables
   std::vector<PtrEntry> tab_host;  // last uploaded (2 * nparams)
   bool tab_valid = false;
@@ -208,7 +215,6 @@ shampoo4_status plan(shampoo4_ctx* h) {
       }
   }
   if (h->blocks.size() > (1u << 30)) return SHAMPOO4_ERR_INVALID_ARG;
-  size_t st = 0;
   for (size_t k = 0; k < h->blocks.size(); ++k) {
     for (int side = 0; side < 2; ++side) {
       FactorPlan f{};
@@ -216,14 +222,50 @@ shampoo4_status plan(shampoo4_ctx* h) {
       f.side = side;
       f.d = side == 0 ? h->blocks[k].m : h->blocks[k].n;
       f.tc = tc_dim(f.d);
-      if (!f.tc) h->any_simt = true;
-      size_t dd = size_t(f.d) * f.d;
-      f.st_S = h->cfg.compressed_stats ? SIZE_MAX : take(st, 4 * dd);
+      h->factors.push_back(f);
+    }
+  }
+  // owners: longest processing time first on the d^3 refresh cost (ties by
+  // factor index), each factor to the least-loaded rank (ties: lowest rank)
+  const size_t nf = h->factors.size();
+  h->owner.assign(nf, 0);
+  if (h->world > 1) {
+    std::vector<size_t> order(nf);
+    for (size_t i = 0; i < nf; ++i) order[i] = i;
+    auto cost = [&](size_t i) { return double(h->factors[i].d) * h->factors[i].d * h->factors[i].d; };
+    std::stable_sort(order.begin(), order.end(), [&](size_t a, size_t b) { return cost(a) > cost(b); });
+    std::vector<double> load(h->world, 0.0);
+    for (size_t i : order) {
+      int32_t r = 0;
+      for (int32_t q = 1; q < h->world; ++q)
+        if (load[q] < load[r]) r = q;
+      h->owner[i] = r;
+      load[r] += cost(i);
+    }
+  }
+  // state: the codes, scales and eigenvalues grouped by owner, then the fp32
+  // statistics of this rank's factors (none with compressed statistics)
+  size_t st = 0;
+  h->span_off.assign(h->world, 0);
+  h->span_bytes.assign(h->world, 0);
+  for (int32_t r = 0; r < h->world; ++r) {
+    h->span_off[r] = align_up(st, kAlign);
+    st = h->span_off[r];
+    for (size_t i = 0; i < nf; ++i) {
+      if (h->owner[i] != r) continue;
+      FactorPlan& f = h->factors[i];
+      const size_t dd = size_t(f.d) * f.d;
       f.st_codes = take(st, (dd + 1) / 2);
       f.st_scales = take(st, 4 * ((dd + kQuantBlock - 1) / kQuantBlock));
       f.st_lam = take(st, 4 * size_t(f.d));
-      h->factors.push_back(f);
     }
+    h->span_bytes[r] = st - h->span_off[r];
+  }
+  for (size_t i = 0; i < nf; ++i) {
+    FactorPlan& f = h->factors[i];
+    const size_t dd = size_t(f.d) * f.d;
+    f.st_S = (h->cfg.compressed_stats || h->owner[i] != h->rank) ? SIZE_MAX : take(st, 4 * dd);
+    if (!f.tc && h->owner[i] == h->rank) h->any_simt = true;
   }
   h->state_bytes = align_up(st, kAlign);
 
@@ -239,7 +281,7 @@ shampoo4_status plan(shampoo4_ctx* h) {
   h->ws_bflag = take(ws, 4 * h->blocks.size());
   for (FactorPlan& f : h->factors) {
     size_t dd = size_t(f.d) * f.d;
-    f.ws_S = h->cfg.compressed_stats ? take(ws, 4 * dd) : SIZE_MAX;
+    f.ws_S = (h->cfg.compressed_stats && h->owner[&f - h->factors.data()] == h->rank) ? take(ws, 4 * dd) : SIZE_MAX;
     f.ws_mu = take(ws, 4 * size_t(f.d));
     if (f.tc) {
       for (int i = 0; i < 2; ++i) {
@@ -480,7 +522,9 @@ void build_stats_into(Builder& b, std::vector<Launch>& prog, bool rebuild) {
     int dmax = 0;
     int64_t emax = 0;
     double bytes_bd = 0, sum_dd = 0;
-    for (const FactorPlan& f : h->factors) {
+    for (size_t i = 0; i < h->factors.size(); ++i) {
+      const FactorPlan& f = h->factors[i];
+      if (h->owner[i] != h->rank) continue;
       const int d = f.d;
       dmax = std::max(dmax, d);
       emax = std::max<int64_t>(emax, int64_t(d) * d);
@@ -534,6 +578,7 @@ void build_stats_into(Builder& b, std::vector<Launch>& prog, bool rebuild) {
     const BlockPlan& bp = h->blocks[k];
     uint32_t* skip = b.wu(h->ws_bflag) + k;
     for (int side = 0; side < 2; ++side) {
+      if (h->owner[2 * k + side] != h->rank) continue;
       const FactorPlan& f = h->factors[2 * k + side];
       const int d = f.d, kk = side == 0 ? bp.n : bp.m;
       float* S = b.S(f);
@@ -884,7 +929,7 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
   }
 }
 
-void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
+void build_refresh_owned(Builder& b, std::vector<Launch>& prog, bool first) {
   shampoo4_ctx* h = b.h;
   const size_t nf = h->factors.size();
   const bool split = split_of(h->cfg);
@@ -1135,6 +1180,34 @@ void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
     L.count = int(nf);
     prog.push_back(std::move(L));
   }
+}
+
+// The refresh programs cover this rank's factors only: they are built over
+// the owned subset (per-factor scratch words are indexed within it), and the
+// offsets the builder assigns to the subset are copied back.
+void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
+  shampoo4_ctx* h = b.h;
+  if (h->world <= 1) {
+    build_refresh_owned(b, prog, first);
+    return;
+  }
+  std::vector<size_t> idx;
+  std::vector<FactorPlan> mine;
+  for (size_t i = 0; i < h->factors.size(); ++i)
+    if (h->owner[i] == h->rank) {
+      idx.push_back(i);
+      mine.push_back(h->factors[i]);
+    }
+  if (mine.empty()) return;
+  std::vector<FactorPlan> all;
+  all.swap(h->factors);
+  h->factors = mine;
+  build_refresh_owned(b, prog, first);
+  for (size_t j = 0; j < idx.size(); ++j) {
+    all[idx[j]].ws_q_first = h->factors[j].ws_q_first;
+    all[idx[j]].ws_q_next = h->factors[j].ws_q_next;
+  }
+  h->factors.swap(all);
 }
 
 void build_precondition(Builder& b) {
@@ -1401,6 +1474,9 @@ extern "C" shampoo4_status shampoo4_init(const shampoo4_config* cfg, const shamp
   if (cfg->precision != SHAMPOO4_PREC_TF32 && cfg->precision != SHAMPOO4_PREC_FP32)
     return SHAMPOO4_ERR_INVALID_ARG;
   if (cfg->compressed_stats != 0 && cfg->compressed_stats != 1) return SHAMPOO4_ERR_INVALID_ARG;
+  if (cfg->refresh_world < 0 || cfg->refresh_world > 4096) return SHAMPOO4_ERR_INVALID_ARG;
+  if (cfg->refresh_world > 1 && (cfg->refresh_rank < 0 || cfg->refresh_rank >= cfg->refresh_world))
+    return SHAMPOO4_ERR_INVALID_ARG;
   for (int32_t i = 0; i < nparams; ++i)
     if (params[i].rows < 1 || params[i].cols < 1 || params[i].rows > (1LL << 31) ||
         params[i].cols > (1LL << 31))
@@ -1409,6 +1485,8 @@ extern "C" shampoo4_status shampoo4_init(const shampoo4_config* cfg, const shamp
   if (!h) return SHAMPOO4_ERR_INVALID_ARG;
   h->cfg = *cfg;
   h->params.assign(params, params + nparams);
+  h->world = cfg->refresh_world > 1 ? cfg->refresh_world : 1;
+  h->rank = h->world > 1 ? cfg->refresh_rank : 0;
   shampoo4_status s = plan(h);
   if (s != SHAMPOO4_OK) { delete h; return s; }
   // Tensor-map and descriptor bytes: build the programs once against a null
@@ -1599,6 +1677,19 @@ extern "C" shampoo4_status shampoo4_debug_q_offset(shampoo4_handle h, int32_t fa
   if (!h || !off_q || factor < 0 || size_t(factor) >= h->factors.size()) return SHAMPOO4_ERR_INVALID_ARG;
   if (!h->bound) return SHAMPOO4_ERR_NOT_READY;
   *off_q = h->last_refresh_first ? h->factors[factor].ws_q_first : h->factors[factor].ws_q_next;
+  return SHAMPOO4_OK;
+}
+
+extern "C" shampoo4_status shampoo4_factor_owner(shampoo4_handle h, int32_t factor, int32_t* rank) {
+  if (!h || !rank || factor < 0 || size_t(factor) >= h->factors.size()) return SHAMPOO4_ERR_INVALID_ARG;
+  *rank = h->owner[factor];
+  return SHAMPOO4_OK;
+}
+
+extern "C" shampoo4_status shampoo4_owner_span(shampoo4_handle h, int32_t rank, size_t* off, size_t* bytes) {
+  if (!h || rank < 0 || rank >= h->world) return SHAMPOO4_ERR_INVALID_ARG;
+  if (off) *off = h->span_off[rank];
+  if (bytes) *bytes = h->span_bytes[rank];
   return SHAMPOO4_OK;
 }
 

@@ -95,6 +95,22 @@ typedef struct {
                             is what stores the new statistic; otherwise
                             ERR_NOT_READY).  The state shrinks by 4 d^2
                             bytes per factor.                               */
+  int32_t refresh_rank;  /* refresh sharding ("Shampoo -- Second-Order
+                            Optimizer", "Blocked and distributed variants":
+                            the roots of different blocks are computed on
+                            different workers).  With refresh_world > 1 the
+                            factors are dealt to refresh_world ranks by
+                            cost (longest d^3 first, each to the least
+                            loaded rank); this handle keeps the statistics
+                            of, and refreshes, only rank refresh_rank's
+                            factors.  Every rank's codes, scales and
+                            eigenvalues sit in one contiguous state span
+                            (shampoo4_owner_span, the same offsets on every
+                            rank); after refresh_roots the caller copies
+                            each rank's span to the others (a broadcast per
+                            rank) before precondition, which covers every
+                            tile.  0 <= refresh_rank < refresh_world.       */
+  int32_t refresh_world; /* 0 or 1: one rank refreshes every factor.        */
 } shampoo4_config;
 
 typedef struct { int64_t rows, cols; } shampoo4_param;   /* 2-D weights only;
@@ -184,9 +200,9 @@ shampoo4_status shampoo4_block_info(shampoo4_handle h, int32_t block, int32_t* p
 /* Byte offsets inside the state buffer of one factor's statistic S (fp32
  * d x d, row-major, dense), codes (uint8, ceil(d*d/2), two per byte, element
  * 2i in the low nibble), scales (fp32, ceil(d*d/64)) and eigenvalues (fp32,
- * d); *dim receives d.  Any pointer may be NULL.  With compressed_stats the
- * statistic is not part of the state: *off_S receives SIZE_MAX (see
- * shampoo4_debug_s_offset). */
+ * d); *dim receives d.  Any pointer may be NULL.  With compressed_stats, or
+ * for a factor another rank refreshes, the statistic is not part of this
+ * handle's state: *off_S receives SIZE_MAX (see shampoo4_debug_s_offset). */
 shampoo4_status shampoo4_factor_layout(shampoo4_handle h, int32_t factor, size_t* off_S,
                                        size_t* off_codes, size_t* off_scales,
                                        size_t* off_lambda, int32_t* dim);
@@ -201,6 +217,12 @@ shampoo4_status shampoo4_debug_q_offset(shampoo4_handle h, int32_t factor, size_
  * the next refresh_roots).  ERR_INVALID_ARG without compressed_stats.  For
  * tests and diagnostics. */
 shampoo4_status shampoo4_debug_s_offset(shampoo4_handle h, int32_t factor, size_t* off_s);
+
+/* Refresh sharding: the rank that refreshes a factor, and the state byte
+ * range [*off, *off + *bytes) holding the codes, scales and eigenvalues of
+ * every factor that rank refreshes (the same on every rank's handle). */
+shampoo4_status shampoo4_factor_owner(shampoo4_handle h, int32_t factor, int32_t* rank);
+shampoo4_status shampoo4_owner_span(shampoo4_handle h, int32_t rank, size_t* off, size_t* bytes);
 
 /* Stages of the three programs, for the optional launch timing below. */
 typedef enum {
