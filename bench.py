@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--no-graft", action="store_true")
     ap.add_argument("--compressed", action="store_true",
                     help="keep each statistic only as its 4-bit eigenbasis and eigenvalues")
+    ap.add_argument("--shard-refresh", action="store_true",
+                    help="with N ranks: each rank refreshes 1/N of the factors (by cost), then the ranks "
+                         "exchange codes, scales and eigenvalues (one NCCL broadcast per rank); strong scaling")
     ap.add_argument("--shapes", default=None, help="comma-separated RxC list replacing the workload's shapes")
     ap.add_argument("--grad-sets", type=int, default=2,
                     help="seeded gradient sets the steps cycle through (1 = the same gradient every step)")
@@ -313,18 +316,25 @@ def main():
     host_g = host_sets[0]
     dev_out = [torch.empty(s, dtype=torch.float32, device=dev) for s in shapes]
     host_out = [torch.empty(s, dtype=torch.float32).pin_memory() for s in shapes]
+    shard = args.shard_refresh and world > 1
     sh = api.Shampoo4(shapes, beta=w.beta, eps=w.eps, max_block=w.max_block, bjorck_iters=w.bjorck_iters,
-                      precision=args.precision, device=dev, compressed=args.compressed)
+                      precision=args.precision, device=dev, compressed=args.compressed,
+                      refresh_rank=rank if shard else 0, refresh_world=world if shard else 1)
     stream = torch.cuda.current_stream()
 
     counter = [0]
 
+    def one_step(g, out):
+        sh.update_stats(g)
+        sh.refresh_roots()
+        if shard:
+            sh.exchange_roots()
+        sh.precondition(g, out=out)
+
     def step():
         g = dev_sets[counter[0] % nsets]
         counter[0] += 1
-        sh.update_stats(g)
-        sh.refresh_roots()
-        sh.precondition(g, out=dev_out)
+        one_step(g, dev_out)
 
     for _ in range(args.warmup):
         step()
@@ -346,7 +356,9 @@ def main():
         dist.barrier()
     ms = max_over_ranks(e0.elapsed_time(e1), dev)
     ms_per_step = ms / args.steps
-    value = job_rate(world, args.steps, ms)
+    # replicas: every rank runs a whole step; sharded refresh: the ranks run
+    # one step together
+    value = args.steps / (ms / 1e3) if shard else job_rate(world, args.steps, ms)
 
     # per-stage times measured live over the timed region
     stages = {}
@@ -381,12 +393,15 @@ def main():
     others = [stage_roofline(k, stages[k], pk, pk_src) for k in ranked[:8] if k != dom]
 
     line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "strong" if shard else "weak",
             "vs_baseline": None, "dtype": args.precision if args.precision == "fp32" else "tf32",
             "data": "synthetic",
             "config": {"workload": w.name, "tiles": sh.nblocks, "factors": sh.nfactors,
                        "steps_per_refresh": 1,
                        "statistics": "compressed (4-bit eigenbasis + eigenvalues)" if args.compressed else "fp32",
+                       "parallelism": (f"refresh sharded over {world} ranks + NCCL span broadcasts" if shard
+                                       else f"{world} independent replica(s)"),
                        "state_bytes": sh.state_bytes, "workspace_bytes": sh.workspace_bytes,
                        "gradients": f"{nsets} seeded set(s), step t uses set t mod {nsets}",
                        "l2": (f"inputs larger than L2 ({g_bytes / 1e9:.2f} GB of G, {stat_bytes / 1e9:.2f} GB "
@@ -429,9 +444,7 @@ def main():
             slot = i % 2
             stream.wait_event(loaded[slot])
             g = gbuf[slot]
-            sh.update_stats(g)
-            sh.refresh_roots()
-            sh.precondition(g, out=obuf[slot])
+            one_step(g, obuf[slot])
             done[slot].record(stream)
             if i + 1 < k:
                 load(i + 1)
@@ -445,7 +458,8 @@ def main():
         ems = max_over_ranks(e2.elapsed_time(e3), dev)
         bi = sum(h.numel() * 4 for h in host_g)
         bo = sum(h.numel() * 4 for h in host_out)
-        line["e2e"] = {"value": job_rate(world, k, ems), "unit": "steps/s", "steps": k, "h2d_bytes_per_step": bi,
+        line["e2e"] = {"value": k / (ems / 1e3) if shard else job_rate(world, k, ems), "unit": "steps/s", "steps": k,
+                       "h2d_bytes_per_step": bi,
                        "d2h_bytes_per_step": bo,
                        "copies": "pinned host buffers, second stream, double-buffered (overlapped with compute)"}
         del gbuf, obuf, hout
