@@ -51,6 +51,7 @@ def parse():
     ap.add_argument("--no-graft", action="store_true")
     ap.add_argument("--compressed", action="store_true",
                     help="keep each statistic only as its 4-bit eigenbasis and eigenvalues")
+    ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--shard-refresh", action="store_true",
                     help="with N ranks: each rank refreshes 1/N of the factors (by cost), then the ranks "
                          "exchange codes, scales and eigenvalues (one NCCL broadcast per rank); strong scaling")
@@ -463,6 +464,34 @@ def main():
                        "d2h_bytes_per_step": bo,
                        "copies": "pinned host buffers, second stream, double-buffered (overlapped with compute)"}
         del gbuf, obuf, hout
+
+    # the same steps captured once in a CUDA graph (two steps, one per gradient
+    # buffer) and replayed: launch gaps and host work leave the step
+    if not args.no_graph and not shard:
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream(device=dev)
+        graph = torch.cuda.CUDAGraph()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                for i in range(2):
+                    one_step(dev_sets[i % nsets], dev_out)
+        stream.wait_stream(side)
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize()
+        reps = max(1, args.steps // 2)
+        e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e4.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e5.record(stream)
+        torch.cuda.synchronize()
+        gms = max_over_ranks(e4.elapsed_time(e5), dev)
+        line["graph"] = {"value": job_rate(world, 2 * reps, gms), "unit": "steps/s", "steps": 2 * reps,
+                         "ms_per_step": gms / (2 * reps),
+                         "note": "the timed steps captured once in a CUDA graph and replayed"}
+        del graph
 
     # stand-alone codec bandwidth on eigenvector-shaped tensors of the workload's size
     if not args.no_codec:

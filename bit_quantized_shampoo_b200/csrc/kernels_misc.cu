@@ -227,6 +227,29 @@ shampoo4_status launch_mu(const MuDesc* d_desc, int count, int max_d, float eps,
   return SHAMPOO4_OK;
 }
 
+// ---- per-call pointer table --------------------------------------------------
+struct TableArgs {
+  PtrEntry e[kMaxTableEntries];
+  PtrEntry* dst;
+  int32_t n;
+};
+
+__global__ void __launch_bounds__(32) k_set_table(const __grid_constant__ TableArgs a) {
+  for (int i = threadIdx.x; i < a.n; i += 32) a.dst[i] = a.e[i];
+}
+
+shampoo4_status launch_set_table(const PtrEntry* entries, int n, PtrEntry* dst, cudaStream_t st) {
+  if (n < 0 || n > kMaxTableEntries) return SHAMPOO4_ERR_UNSUPPORTED;
+  if (n == 0) return SHAMPOO4_OK;
+  static thread_local TableArgs a;                 // 16 KB: off the host stack
+  for (int i = 0; i < n; ++i) a.e[i] = entries[i];
+  a.dst = dst;
+  a.n = n;
+  k_set_table<<<1, 32, 0, st>>>(a);
+  S4_CUDA(cudaGetLastError());
+  return SHAMPOO4_OK;
+}
+
 // ---- non-finite scan -------------------------------------------------------
 __global__ void __launch_bounds__(256)
 k_scan(const ScanDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, int nparams,

@@ -274,6 +274,14 @@ struct GraftArgs {
 // Two launches: moments and per-item norms, then the weight update.
 shampoo4_status launch_graft(const GraftArgs& a, cudaStream_t st);
 
+// ---- per-call pointer tables, written on the stream ---------------------------
+// The table travels as a kernel parameter and one warp stores it, so setting
+// it is an ordinary stream operation: nothing waits on the host, and a CUDA
+// graph captured around an API call replays the table of that call.
+constexpr int kMaxTableEntries = 1024;     // 16 KB of kernel parameter
+
+shampoo4_status launch_set_table(const PtrEntry* entries, int n, PtrEntry* dst, cudaStream_t st);
+
 // ---- launchers (each enqueues one launch over `count` descriptors) -------
 shampoo4_status launch_gemm_f32(const GemmF32Desc* d_desc, int count, int max_tiles,
                                 const PtrEntry* tabs, int nparams, cudaStream_t st);

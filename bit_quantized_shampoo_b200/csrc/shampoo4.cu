@@ -1427,6 +1427,23 @@ shampoo4_status collect_timing(shampoo4_ctx* h) {
   return SHAMPOO4_OK;
 }
 
+// Write a per-call pointer table into the workspace at `region`: by a
+// one-warp kernel that carries the table as its parameter (a stream
+// operation, capturable), or, beyond kMaxTableEntries entries, by a copy
+// from a pinned host buffer (guarded by an event; not capturable).
+shampoo4_status upload_table(shampoo4_ctx* h, const std::vector<PtrEntry>& t, size_t region, PtrEntry* pinned,
+                             cudaEvent_t ev, bool& ev_pending, bool capturing, cudaStream_t st) {
+  PtrEntry* dst = reinterpret_cast<PtrEntry*>(h->d_ws + region);
+  if (t.size() <= size_t(kMaxTableEntries)) return launch_set_table(t.data(), int(t.size()), dst, st);
+  if (capturing) return SHAMPOO4_ERR_UNSUPPORTED;
+  if (ev_pending) S4_CUDA(cudaEventSynchronize(ev));
+  std::memcpy(pinned, t.data(), sizeof(PtrEntry) * t.size());
+  S4_CUDA(cudaMemcpyAsync(dst, pinned, sizeof(PtrEntry) * t.size(), cudaMemcpyHostToDevice, st));
+  S4_CUDA(cudaEventRecord(ev, st));
+  ev_pending = true;
+  return SHAMPOO4_OK;
+}
+
 // Upload the per-call pointer table when any entry changed.
 shampoo4_status set_tables(shampoo4_ctx* h, const float* const* grads, const int64_t* ld,
                            float* const* outs, const int64_t* ld_out, cudaStream_t st) {
@@ -1436,14 +1453,15 @@ shampoo4_status set_tables(shampoo4_ctx* h, const float* const* grads, const int
     want[p] = {grads[p], ld[p]};
     if (outs) want[np + p] = {outs[p], ld_out[p]};
   }
-  if (h->tab_valid && std::memcmp(want.data(), h->tab_host.data(), sizeof(PtrEntry) * 2 * np) == 0)
+  // while a graph is being captured the table is always written, so that
+  // the graph carries the table of every call it replays
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  S4_CUDA(cudaStreamIsCapturing(st, &cs));
+  const bool capturing = cs != cudaStreamCaptureStatusNone;
+  if (!capturing && h->tab_valid &&
+      std::memcmp(want.data(), h->tab_host.data(), sizeof(PtrEntry) * 2 * np) == 0)
     return SHAMPOO4_OK;
-  if (h->tab_event_pending) S4_CUDA(cudaEventSynchronize(h->tab_event));
-  std::memcpy(h->tab_pinned, want.data(), sizeof(PtrEntry) * 2 * np);
-  S4_CUDA(cudaMemcpyAsync(h->d_ws + h->ws_tabs, h->tab_pinned, sizeof(PtrEntry) * 2 * np,
-                          cudaMemcpyHostToDevice, st));
-  S4_CUDA(cudaEventRecord(h->tab_event, st));
-  h->tab_event_pending = true;
+  S4_TRY(upload_table(h, want, h->ws_tabs, h->tab_pinned, h->tab_event, h->tab_event_pending, capturing, st));
   h->tab_host = want;
   h->tab_valid = true;
   return SHAMPOO4_OK;
@@ -1807,13 +1825,12 @@ extern "C" shampoo4_status shampoo4_graft_update(shampoo4_handle h, const shampo
     want[np + p] = {d_dirs[p], ld_dirs[p]};
     want[2 * np + p] = {d_weights[p], ld_weights[p]};
   }
-  if (!h->gtab_valid || std::memcmp(want.data(), h->gtab_host.data(), sizeof(PtrEntry) * 3 * np) != 0) {
-    if (h->gtab_event_pending) S4_CUDA(cudaEventSynchronize(h->gtab_event));
-    std::memcpy(h->gtab_pinned, want.data(), sizeof(PtrEntry) * 3 * np);
-    S4_CUDA(cudaMemcpyAsync(h->d_ws + h->ws_gtab, h->gtab_pinned, sizeof(PtrEntry) * 3 * np,
-                            cudaMemcpyHostToDevice, st));
-    S4_CUDA(cudaEventRecord(h->gtab_event, st));
-    h->gtab_event_pending = true;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  S4_CUDA(cudaStreamIsCapturing(st, &cs));
+  const bool capturing = cs != cudaStreamCaptureStatusNone;
+  if (capturing || !h->gtab_valid ||
+      std::memcmp(want.data(), h->gtab_host.data(), sizeof(PtrEntry) * 3 * np) != 0) {
+    S4_TRY(upload_table(h, want, h->ws_gtab, h->gtab_pinned, h->gtab_event, h->gtab_event_pending, capturing, st));
     h->gtab_host = want;
     h->gtab_valid = true;
   }
