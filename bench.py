@@ -136,7 +136,7 @@ STAGE_BOUND = {
     "qr_trsm_panel": "3xtf32", "qr_solve_update": "3xtf32", "qr_solve_panel": "3xtf32",
     "qr_potrf": "latency", "qr_inverse": "latency", "rayleigh": "hbm", "requant": "hbm", "precond_dequant": "hbm",
     "basis": "hbm", "stats_scan": "hbm", "refresh_scan": "hbm", "qr_convert": "hbm", "precond_mu": "hbm",
-    "stats_dequant": "hbm", "stats_rebuild": "tf32",
+    "stats_dequant": "hbm", "stats_rebuild": "tf32", "tables": "latency",
 }
 
 

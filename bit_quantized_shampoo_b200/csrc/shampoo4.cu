@@ -1434,7 +1434,21 @@ shampoo4_status collect_timing(shampoo4_ctx* h) {
 shampoo4_status upload_table(shampoo4_ctx* h, const std::vector<PtrEntry>& t, size_t region, PtrEntry* pinned,
                              cudaEvent_t ev, bool& ev_pending, bool capturing, cudaStream_t st) {
   PtrEntry* dst = reinterpret_cast<PtrEntry*>(h->d_ws + region);
-  if (t.size() <= size_t(kMaxTableEntries)) return launch_set_table(t.data(), int(t.size()), dst, st);
+  if (t.size() <= size_t(kMaxTableEntries)) {
+    shampoo4_ctx::Rec rec{SHAMPOO4_STAGE_TABLES, nullptr, nullptr, 0.0, 16.0 * double(t.size()), 1};
+    if (h->timing) {
+      rec.e0 = take_event(h);
+      rec.e1 = take_event(h);
+      if (!rec.e0 || !rec.e1) return SHAMPOO4_ERR_CUDA;
+      S4_CUDA(cudaEventRecord(rec.e0, st));
+    }
+    S4_TRY(launch_set_table(t.data(), int(t.size()), dst, st));
+    if (h->timing) {
+      S4_CUDA(cudaEventRecord(rec.e1, st));
+      h->recs.push_back(rec);
+    }
+    return SHAMPOO4_OK;
+  }
   if (capturing) return SHAMPOO4_ERR_UNSUPPORTED;
   if (ev_pending) S4_CUDA(cudaEventSynchronize(ev));
   std::memcpy(pinned, t.data(), sizeof(PtrEntry) * t.size());
@@ -1745,7 +1759,7 @@ extern "C" const char* shampoo4_stage_name(int32_t stage) {
       "stats_scan", "stats_gemm", "refresh_scan", "basis", "bjorck_gram", "bjorck_update",
       "subspace", "qr_gram", "qr_potrf", "qr_trsm_panel", "qr_syrk", "qr_solve_update",
       "qr_solve_panel", "qr_convert", "rayleigh_gemm", "rayleigh", "requant", "precond_dequant",
-      "precond_mu", "roots", "apply_left", "apply_right", "qr_inverse", "stats_dequant", "stats_rebuild"};
+      "precond_mu", "roots", "apply_left", "apply_right", "qr_inverse", "stats_dequant", "stats_rebuild", "tables"};
   if (stage < 0 || stage >= SHAMPOO4_STAGE_COUNT) return "unknown";
   return names[stage];
 }

@@ -234,7 +234,7 @@ typedef enum {
   SHAMPOO4_STAGE_RAYLEIGH, SHAMPOO4_STAGE_REQUANT, SHAMPOO4_STAGE_PRECOND_DEQUANT,
   SHAMPOO4_STAGE_PRECOND_MU, SHAMPOO4_STAGE_ROOTS, SHAMPOO4_STAGE_APPLY_LEFT,
   SHAMPOO4_STAGE_APPLY_RIGHT, SHAMPOO4_STAGE_QR_INVERSE, SHAMPOO4_STAGE_STATS_DEQUANT,
-  SHAMPOO4_STAGE_STATS_REBUILD, SHAMPOO4_STAGE_COUNT
+  SHAMPOO4_STAGE_STATS_REBUILD, SHAMPOO4_STAGE_TABLES, SHAMPOO4_STAGE_COUNT
 } shampoo4_stage;
 
 /* Launch timing, for diagnostics and roofline figures.  While enabled, every
