@@ -141,11 +141,11 @@ STAGE_BOUND = {
 
 
 # DRAM bytes (read + write) of ONE launch of a stage's tensor-core GEMM per
-# element of the factors it processes, from the ncu capture summarised in
-# profiles/k_gemm_tc_4096x4096_factors.md (32 factors of 1024 x 1024).  A
-# launch over other factors of the same kind moves the same bytes per
-# element.  Valid only for the GEMM source it was taken on: the figure is
-# dropped (traffic = null) when gemm_tc.cu or tc.h has changed since.
+# element of the factors it processes, from an ncu capture of the GEMM on 32
+# factors of 1024 x 1024 (one 4096 x 4096 gradient).  A launch over other
+# factors of the same kind moves the same bytes per element.  Valid only for
+# the GEMM source it was taken on: the figure is dropped (traffic = null) when
+# gemm_tc.cu or tc.h has changed since.
 TRAFFIC_SOURCE_SHA = "953e5999e9574e38"
 TRAFFIC_PER_ELEMENT = {"stats_gemm": 6.590, "bjorck_gram": 6.758, "bjorck_update": 19.321,
                        "subspace": 32.588, "qr_gram": 13.066}
