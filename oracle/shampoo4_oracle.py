@@ -223,6 +223,29 @@ def root_from_basis(U: np.ndarray, lam: np.ndarray, eps: float) -> np.ndarray:
     return (U * mu[None, :]) @ U.T
 
 
+def newton_inverse_root(A: np.ndarray, p: int = 4, iters: int = 40, history=None) -> np.ndarray:
+    """A^(-1/p) for a symmetric positive definite A by the coupled Newton
+    iteration of "Shampoo -- Second-Order Optimizer", section "Computing the
+    inverse fourth root": scale A by c = ||A||_F (an upper bound of the
+    spectral norm, so the spectrum of M lies in (0, 1]), start from X = I and
+    M = A / c, and repeat F = ((p + 1) I - M) / p, X <- X F, M <- F^p M.
+    Then A^(-1/p) = X c^(-1/p).  A fixed number of iterations (a device path
+    has no host test to stop on).  ``history``, if a list, receives (X, M)
+    after every iteration.  fp64."""
+    A = np.asarray(A, dtype=np.float64)
+    d = A.shape[0]
+    c = float(np.linalg.norm(A))
+    I = np.eye(d)
+    X, M = I.copy(), A / c
+    for _ in range(iters):
+        F = ((p + 1) * I - M) / p
+        X = X @ F
+        M = np.linalg.matrix_power(F, p) @ M
+        if history is not None:
+            history.append((X, M))
+    return X * c ** (-1.0 / p)
+
+
 def apply_roots(PL: np.ndarray, Gb: np.ndarray, PR: np.ndarray) -> np.ndarray:
     """D = L^(-1/4) G R^(-1/4) ("Kronecker factorization")."""
     return (np.asarray(PL, np.float64) @ np.asarray(Gb, np.float64)

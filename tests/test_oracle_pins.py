@@ -213,6 +213,44 @@ def test_compressed_update_first_step_and_nonfinite():
     assert np.allclose(O.compressed_stats(f, Gn, beta, "L"), stored, rtol=0, atol=1e-6 * np.abs(stored).max())
 
 
+# ------------------------------------------------ coupled Newton root (f4)
+
+def test_newton_root_of_a_diagonal_is_the_elementwise_root():
+    lam = np.array([1.0, 0.3, 2e-3, 7.5, 1e-4])
+    R = O.newton_inverse_root(np.diag(lam), p=4, iters=40)
+    assert np.allclose(R, np.diag(lam ** -0.25), rtol=1e-12, atol=0)
+
+
+def test_newton_root_matches_the_eigen_form_on_a_known_spectrum():
+    rng = np.random.default_rng(31)
+    d = 24
+    V = random_orthogonal(d, rng)
+    lam = np.geomspace(1.0, 1e-4, d)                      # kappa = 1e4
+    A = (V * lam[None, :]) @ V.T
+    want = (V * (lam ** -0.25)[None, :]) @ V.T
+    got = O.newton_inverse_root(A, p=4, iters=40)
+    assert np.linalg.norm(got - want) <= 1e-10 * np.linalg.norm(want)
+    # p = 2: the inverse square root of the same matrix
+    got2 = O.newton_inverse_root(A, p=2, iters=60)
+    assert np.allclose(got2, (V * (lam ** -0.5)[None, :]) @ V.T, rtol=0, atol=1e-9 * lam.min() ** -0.5)
+
+
+def test_newton_root_coupling_invariant_and_homogeneity():
+    # M_k = X_k^p A / c at every iteration (the coupling the iteration keeps),
+    # and (s A)^(-1/p) = s^(-1/p) A^(-1/p)
+    rng = np.random.default_rng(32)
+    d = 10
+    V = random_orthogonal(d, rng)
+    A = (V * rng.uniform(0.05, 3.0, d)[None, :]) @ V.T
+    c = np.linalg.norm(A)
+    hist = []
+    O.newton_inverse_root(A, p=4, iters=12, history=hist)
+    for X, M in hist:
+        assert np.allclose(M, np.linalg.matrix_power(X, 4) @ A / c, rtol=0, atol=1e-11)
+    R = O.newton_inverse_root(A, p=4, iters=40)
+    assert np.allclose(O.newton_inverse_root(16.0 * A, p=4, iters=40), R / 2.0, rtol=1e-12, atol=1e-14)
+
+
 # ------------------------------------------------------------ Bjorck (P4)
 
 def test_bjorck_closed_form_on_svd():
