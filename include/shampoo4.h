@@ -20,10 +20,22 @@
  * Weights are cut into tiles of at most max_block x max_block, each with its
  * own pair of factors ("Blocked and distributed variants").
  *
+ * Beside the step:
+ *   graft_update    W <- W - lr ||d_graft|| / (||D|| + eps) D per tile, with
+ *                   d_graft the SGD or Adam step ("Grafting: borrow a step
+ *                   size that already works")
+ *   compressed_stats (config) keeps each statistic only as its 4-bit
+ *                   eigenbasis and eigenvalues and rebuilds it per update
+ *   refresh_rank / refresh_world (config) deal the refresh of the factors to
+ *                   several ranks, whose state spans the caller exchanges
+ *   a CUDA graph captured around the step calls replays them: a call
+ *                   enqueues only kernels and memsets on its stream
+ *
  * Conventions shared by every entry point
  *  - All device buffers are allocated and owned by the caller; the library
  *    never allocates device memory.  It owns only host-side planning data
- *    (and one small pinned host staging buffer per handle).
+ *    (and small pinned host staging buffers per handle, used only for
+ *    pointer tables of more than 1024 entries and for the status flags).
  *  - Calls that take a stream are asynchronous on it; none synchronizes
  *    except shampoo4_get_status_flags.  All calls on one handle must be
  *    ordered on the same stream (or by the caller's own events).
