@@ -11,9 +11,9 @@ norm, and the weight moves by
     step_b = lr * ||d_graft_b||_F / (||D_b||_F + graft_eps) * D_b,
     W_b   <- W_b - step_b,
 
-with the norms taken per tile of the blocked partition (the page allows
-"per layer or per block"; the tiles are what is preconditioned
-independently, section "Blocked and distributed variants").
+with the norms taken per tile of the blocked partition (the page lets the
+norms be taken over a whole layer or over one block; the tiles are what is
+preconditioned independently, section "Blocked and distributed variants").
 
 d_graft is the step the grafted method would take, without its learning
 rate:
