@@ -156,7 +156,7 @@ class Shampoo4:
     def factor_views(self, f):
         """(S, codes, scales, lambda) as tensor views into the state buffer
         (with compressed statistics, S is the workspace copy the last
-        update_stats rebuilt)."""
+        update_stats rebuilt; S is None for a factor another rank refreshes)."""
         oS, oc, os_, ol = C.c_size_t(), C.c_size_t(), C.c_size_t(), C.c_size_t()
         d = C.c_int32()
         L.call("shampoo4_factor_layout", self._h, f, C.byref(oS), C.byref(oc), C.byref(os_), C.byref(ol), C.byref(d))
@@ -165,9 +165,11 @@ class Shampoo4:
         st = self.state
         if self.compressed:
             L.call("shampoo4_debug_s_offset", self._h, f, C.byref(oS))
-            S = self.workspace[oS.value:oS.value + 4 * n].view(torch.float32).view(d, d)
+            src = self.workspace
         else:
-            S = st[oS.value:oS.value + 4 * n].view(torch.float32).view(d, d)
+            src = st
+        held = oS.value != C.c_size_t(-1).value
+        S = src[oS.value:oS.value + 4 * n].view(torch.float32).view(d, d) if held else None
         codes = st[oc.value:oc.value + (n + 1) // 2]
         scales = st[os_.value:os_.value + 4 * ((n + 63) // 64)].view(torch.float32)
         lam = st[ol.value:ol.value + 4 * d].view(torch.float32)
