@@ -175,3 +175,20 @@ def test_compressed_statistics_leave_the_state_and_move_to_the_workspace():
     # the state loses every statistic (4 d^2 bytes per factor); the workspace gains them
     assert sizes[0][0] - sizes[1][0] >= 4 * dd
     assert sizes[1][1] - sizes[0][1] >= 4 * dd
+
+
+@pytest.mark.skipif(not (os.path.exists("/usr/bin/gcc") or os.path.exists("/usr/bin/cc")), reason="no C compiler")
+def test_c_program_links_and_plans_through_the_header(tmp_path):
+    """The header compiles as C11 with warnings as errors, the library links
+    by its C names, and the host-only calls behave as documented, from C."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    libdir = os.path.dirname(L.library_path())
+    exe = tmp_path / "abi_host_check"
+    subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "native", "abi_host_check.c"), "-o", str(exe),
+                    "-L", libdir, "-lshampoo4", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "abi ok" in r.stdout
