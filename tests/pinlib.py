@@ -25,7 +25,8 @@ def jacobi_eigh(A: np.ndarray, sweeps: int = 30, tol: float = 1e-15):
                 apq = A[p, q]
                 if apq == 0.0:
                     continue
-                tau = (A[q, q] - A[p, p]) / (2.0 * apq)
+                with np.errstate(over="ignore"):          # a tiny apq: tau = inf, t = 0 below
+                    tau = (A[q, q] - A[p, p]) / (2.0 * apq)
                 if abs(tau) > 1e100:
                     t = 0.5 / tau
                 else:
