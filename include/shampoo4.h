@@ -262,9 +262,15 @@ shampoo4_status shampoo4_timing_read(shampoo4_handle h, int32_t stage, double* m
                                      int64_t* launches, double* flops, double* bytes);
 const char* shampoo4_stage_name(int32_t stage);
 
-/* Block-wise linear square 4-bit quantization of `count` fp32 tensors.
+/* Block-wise linear square 4-bit quantization of `count` fp32 tensors
+ * ("4-bit Shampoo for Memory-Efficient Network Training", abstract: linear
+ * square quantization, block-wise; the level and threshold definitions below
+ * are this library's reading of the name).
  * For tensor i: n[i] elements at d_x[i] (4-byte aligned), ceil(n[i]/2) code
- * bytes to d_codes[i], ceil(n[i]/64) scales to d_scales[i].
+ * bytes to d_codes[i], ceil(n[i]/64) scales to d_scales[i].  Errors: a NULL
+ * array or element pointer, count < 0, n[i] < 0 or a misaligned pointer
+ * return ERR_INVALID_ARG before anything is enqueued; count == 0 and empty
+ * tensors (n[i] == 0) do nothing.
  * Per block of 64 consecutive elements: scale = max |x| (NaN if the block
  * holds a NaN, +Inf if it holds an infinity), v = x / scale (IEEE division),
  * code = number of the 15 thresholds t_k strictly below v, where t_k is the
@@ -275,7 +281,8 @@ shampoo4_status quant4_pack(const float* const* d_x, const int64_t* n, int32_t c
                             uint8_t* const* d_codes, float* const* d_scales,
                             shampoo4_stream_t stream);
 
-/* Inverse of quant4_pack: x = fp32(cb_code) * scale (one fp32 multiply). */
+/* Inverse of quant4_pack: x = fp32(cb_code) * scale (one fp32 multiply),
+ * n[i] fp32 elements to d_x[i]; same argument rules as quant4_pack. */
 shampoo4_status quant4_unpack(const uint8_t* const* d_codes, const float* const* d_scales,
                               const int64_t* n, int32_t count, float* const* d_x,
                               shampoo4_stream_t stream);
