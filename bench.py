@@ -473,7 +473,9 @@ def main():
         graph = torch.cuda.CUDAGraph()
         side.wait_stream(stream)
         with torch.cuda.stream(side):
-            with torch.cuda.graph(graph, stream=side):
+            # thread-local capture: another thread's CUDA calls (a process
+            # group's watchdog, say) do not disturb it
+            with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
                 for i in range(2):
                     one_step(dev_sets[i % nsets], dev_out)
         stream.wait_stream(side)
