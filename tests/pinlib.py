@@ -80,3 +80,34 @@ def random_orthogonal(d: int, rng: np.random.Generator) -> np.ndarray:
 def spd_with_spectrum(lam, rng: np.random.Generator) -> np.ndarray:
     V = random_orthogonal(len(lam), rng)
     return (V * np.asarray(lam)[None, :]) @ V.T
+
+
+def mgs_qr(Y: np.ndarray):
+    """Q with orthonormal columns and R upper triangular with a positive
+    diagonal such that Y = Q R, by modified Gram-Schmidt run twice over each
+    column (Golub & Van Loan, Matrix Computations, "Modified Gram-Schmidt";
+    the second sweep restores orthogonality lost to cancellation).  A route
+    to the QR factor independent of LAPACK's Householder reflections."""
+    Y = np.array(Y, dtype=np.float64, copy=True)
+    d, k = Y.shape
+    Q = np.zeros((d, k))
+    R = np.zeros((k, k))
+    for j in range(k):
+        v = Y[:, j].copy()
+        for _ in range(2):
+            for i in range(j):
+                c = Q[:, i] @ v
+                R[i, j] += c
+                v -= c * Q[:, i]
+        R[j, j] = np.linalg.norm(v)
+        Q[:, j] = v / R[j, j]
+    return Q, R
+
+
+def sylvester_hadamard(d: int) -> np.ndarray:
+    """The d x d Sylvester-Hadamard matrix (d a power of two): entries +-1,
+    H H^T = d I."""
+    H = np.ones((1, 1))
+    while H.shape[0] < d:
+        H = np.block([[H, H], [H, -H]])
+    return H

@@ -7,8 +7,8 @@ import numpy as np
 import pytest
 
 from oracle import shampoo4_oracle as O
-from pinlib import (coupled_newton_inverse_root, jacobi_eigh, random_orthogonal,
-                    spd_with_spectrum)
+from pinlib import (coupled_newton_inverse_root, jacobi_eigh, mgs_qr, random_orthogonal,
+                    spd_with_spectrum, sylvester_hadamard)
 
 EPS0 = 1e-300   # "eps -> 0" for the fp64 limits
 
@@ -309,6 +309,116 @@ def test_bjorck_orthogonality_residual_decreases_on_dequantized_basis():
     assert res[0] > 1e-2
     assert all(b < a for a, b in zip(res[:3], res[1:4]))
     assert res[-1] < 1e-12
+
+
+# ------------------------------------------- warm 4-bit refresh (a3-a8)
+
+def _row_scaled_exact_basis(rng, d, r):
+    """Codes and scales whose dequantization is exactly diag(r) V, with V a
+    signed, row-permuted Sylvester-Hadamard basis H / sqrt(d) (not
+    symmetric).  For d = 64 a quantization block is one row; every entry of
+    a row of H is +-1, so the absmax-normalized values sit exactly on the
+    codebook's end levels and the row's scale carries r_i / sqrt(d)."""
+    H = sylvester_hadamard(d)[rng.permutation(d)] * rng.choice([-1.0, 1.0], d)[None, :]
+    V = H / np.sqrt(d)
+    codes, _ = O.quantize(H.astype(np.float32).ravel())
+    scales = (np.asarray(r, np.float64) / np.sqrt(d)).astype(np.float32)
+    return V, codes, scales
+
+
+def _bjorck_scalar(s, t):
+    """t steps of the scalar map s -> s (1.5 - 0.5 s^2): Bjorck's action on
+    the singular values (one step: U = A diag(s) B^T -> A diag(s (1.5 -
+    0.5 s^2)) B^T)."""
+    for _ in range(t):
+        s = s * (1.5 - 0.5 * s * s)
+    return s
+
+
+def test_warm_refresh_rectifies_the_dequantized_basis_before_the_subspace_step():
+    """"4-bit Shampoo ...", abstract: the dequantized eigenvector matrix has
+    its orthogonality rectified, which is what the inverse fourth root is
+    then built from.  For a stored basis that dequantizes exactly to
+    diag(r) V (V orthogonal), U U^T = diag(r^2), so every Bjorck step only
+    rescales rows: U_t = diag(phi_t(r)) V with phi the scalar map above.
+    The warm refresh must then equal one subspace step from that closed
+    form, Q R = (S + eps I) diag(phi_t(r)) V, taken here by Gram-Schmidt.
+    A refresh that skipped Bjorck, ran a different number of steps, ran it
+    after the QR, transposed the dequantized matrix or dropped the eps shift
+    lands measurably away (checked below, so the pin has teeth)."""
+    rng = np.random.default_rng(21)
+    d, t, eps = 64, 5, 1e-3
+    r = rng.integers(16, 103, d) / 64.0              # row scales in [0.25, 1.6], exact in fp32
+    V, codes, scales = _row_scaled_exact_basis(rng, d, r)
+    lam_s = np.concatenate([rng.uniform(0.05, 1.0, d - 2), [0.0, 0.0]])    # two null directions
+    S = spd_with_spectrum(lam_s, rng).astype(np.float32)
+    S64 = S.astype(np.float64)
+    f = O.Factor(d, S.copy(), codes=codes.copy(), scales=scales.copy(),
+                 lam=np.zeros(d, np.float32), has_basis=True)
+    U0 = O.dequantize(codes, scales, d * d).reshape(d, d).astype(np.float64)
+    assert np.array_equal(U0, r[:, None] / np.sqrt(d) * np.sqrt(d) * V)      # exact diag(r) V
+    O.refresh_factor(f, eps, t)
+
+    def expected(rows, M=V, shift=eps):
+        Q, R = mgs_qr((S64 + shift * np.eye(d)) @ (rows[:, None] * M))
+        return Q
+    Qw = expected(_bjorck_scalar(r, t))
+    assert np.linalg.norm(f.q_last - Qw) <= 1e-9 * np.sqrt(d)
+    lam_w = np.maximum(np.einsum("ij,ij->j", Qw, S64 @ Qw), 0.0)
+    assert np.allclose(f.lam.astype(np.float64), lam_w, rtol=1e-6, atol=1e-9)
+    # the requantized state is the codec applied to that Q
+    c2, s2 = O.quantize(f.q_last.astype(np.float32).ravel())
+    assert np.array_equal(f.codes, c2) and np.array_equal(f.scales, s2)
+    # teeth: each plausible mistake moves Q far beyond the tolerance above
+    wrong = {
+        "no Bjorck": expected(r),
+        "t - 1 steps": expected(_bjorck_scalar(r, t - 1)),
+        "Bjorck after the QR": mgs_qr(expected(r))[0],
+        # dequantized matrix read transposed: U = V^T diag(r), whose Bjorck
+        # steps scale its columns the same way
+        "transposed basis": expected(np.ones(d), M=V.T * _bjorck_scalar(r, t)[None, :]),
+        "no eps shift": expected(_bjorck_scalar(r, t), shift=0.0),
+    }
+    for name, Qx in wrong.items():
+        assert np.linalg.norm(f.q_last - Qx) > 1e-4 * np.sqrt(d), name
+
+
+def test_exactly_stored_orthogonal_basis_passes_the_warm_refresh_unchanged():
+    """An orthogonal basis the codes hold exactly (r = 1 above) is a fixed
+    point of Bjorck; if it is also S's eigenbasis, the subspace step
+    returns it exactly (up to rounding), with the eigenvalues as Rayleigh
+    quotients, and requantization gives back the same codes."""
+    rng = np.random.default_rng(22)
+    d, eps = 64, 1e-6
+    V, codes, scales = _row_scaled_exact_basis(rng, d, np.ones(d))
+    assert np.array_equal(O.bjorck(O.dequantize(codes, scales, d * d).reshape(d, d), 5), V)
+    lam_s = np.geomspace(1.0, 1e-3, d)
+    S = ((V * lam_s[None, :]) @ V.T).astype(np.float32)
+    f = O.Factor(d, S.copy(), codes=codes.copy(), scales=scales.copy(), lam=np.zeros(d, np.float32),
+                 has_basis=True)
+    O.refresh_factor(f, eps, 5)
+    assert np.allclose(f.q_last, V, rtol=0, atol=1e-7)     # S holds fp32-rounded entries
+    assert np.allclose(f.lam, lam_s, rtol=1e-6, atol=1e-7)   # fp32 rounding of S: about 1e-8 absolute
+    assert np.array_equal(f.codes, codes) and np.array_equal(f.scales, scales)
+
+
+def test_warm_refresh_is_homogeneous_with_the_quantizer_on():
+    """[tut] "Where the fourth root comes from": the step is homogeneous of
+    degree 0 in G.  Through a warm 4-bit refresh (eps -> 0) that means the
+    same codes and scales, and eigenvalues scaled by exactly 4 for G -> 2G:
+    every fp64 product scales by a power of two, the quantizer is scale
+    invariant, and Bjorck acts on the same dequantized codes."""
+    rng = np.random.default_rng(23)
+    gs = [rng.standard_normal((12, 20)).astype(np.float32) for _ in range(3)]
+    runs = []
+    for scale in (1, 2):
+        orc = O.Shampoo4Oracle([(12, 20)], eps=EPS0)
+        for t, g in enumerate(gs, 1):
+            orc.step(t, [g * np.float32(scale)], refresh_every=1)
+        runs.append(orc)
+    for fa, fb in zip(runs[0].factors, runs[1].factors):
+        assert np.array_equal(fa.codes, fb.codes) and np.array_equal(fa.scales, fb.scales)
+        assert np.array_equal(fb.lam, np.float32(4) * fa.lam)
 
 
 # ----------------------------------------------------- eigenpairs (P5, P8)
