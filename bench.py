@@ -14,9 +14,22 @@ with the same 1024 x 1024 factors as the default workload.  The timed steps
 run inside an NVTX push/pop range named "timed", so a profiler can select
 exactly their launches (ncu --nvtx --nvtx-include "timed/").
 
-Multi-GPU: one process per GPU (torchrun); every rank runs its own copy of
-the workload (tiles are independent; no data-path collective), so per-GPU
-work is fixed as N grows ("weak" scaling).
+The headline roofline is the whole step's algorithmic work by the formulas
+of the work model (bit_quantized_shampoo_b200.costmodel): statistics
+2mn(m+n) and precondition 2(m^3+n^3) + 2mn(m+n) per tile, refresh
+(4t + 2 + 8/3 + 2) d^3 per factor, amortized over the refresh interval --
+divided by the step time, against the precision-weighted tensor peak
+(Bjorck, statistics, roots and apply at the TF32 rate; the fp32-accurate
+subspace step, QR and Rayleigh product at a third of it).
+
+The four smaller workloads are also timed, each at its own refresh interval
+(``configs`` in the line), after the main workload's handle is released.
+
+Multi-GPU: one process per GPU (torchrun).  By default the ranks share one
+workload and shard its refresh: each rank refreshes the factors it owns (by
+d^3 cost) and the ranks exchange codes, scales and eigenvalues by NCCL
+broadcasts ("strong" scaling).  --replicas instead runs an independent copy
+per rank with no data-path collective ("weak").
 """
 from __future__ import annotations
 
@@ -52,9 +65,13 @@ def parse():
     ap.add_argument("--compressed", action="store_true",
                     help="keep each statistic only as its 4-bit eigenbasis and eigenvalues")
     ap.add_argument("--no-graph", action="store_true")
-    ap.add_argument("--shard-refresh", action="store_true",
-                    help="with N ranks: each rank refreshes 1/N of the factors (by cost), then the ranks "
-                         "exchange codes, scales and eigenvalues (one NCCL broadcast per rank); strong scaling")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with N ranks: N independent copies of the workload (weak scaling) instead of the "
+                         "default sharded refresh, where each rank refreshes 1/N of the factors (by cost) and "
+                         "the ranks exchange codes, scales and eigenvalues (one NCCL broadcast per rank)")
+    ap.add_argument("--no-configs", action="store_true", help="skip timing the four smaller workloads")
+    ap.add_argument("--cpu-tiles", type=int, default=48,
+                    help="tiles of the CPU baseline's sample: every ragged tile, then seeded full ones")
     ap.add_argument("--shapes", default=None, help="comma-separated RxC list replacing the workload's shapes")
     ap.add_argument("--grad-sets", type=int, default=2,
                     help="seeded gradient sets the steps cycle through (1 = the same gradient every step)")
@@ -192,6 +209,54 @@ def stage_roofline(name, st, pk, pk_src, sustained=True):
     return r
 
 
+def step_work(dims, bjorck_iters, refresh_every, precision):
+    """Algorithmic flops of one optimizer step by the work model, split by
+    the arithmetic each part runs in: (flops at the TF32 rate, flops at the
+    3xTF32 rate).  dims: the (m, n) of every tile.  The refresh is amortized
+    over refresh_every steps.  In FP32 mode every product is 3xTF32."""
+    from bit_quantized_shampoo_b200 import costmodel as cm
+    single = triple = 0.0
+    for m, n in dims:
+        single += cm.stats_flops(m, n) + cm.precondition_flops(m, n)
+        for d in (m, n):
+            bj = 4.0 * bjorck_iters * float(d) ** 3
+            single += bj / refresh_every
+            triple += (cm.refresh_flops(d, bjorck_iters) - bj) / refresh_every
+    if precision == "fp32":
+        single, triple = 0.0, single + triple
+    return single, triple
+
+
+def refresh_work(dims, bjorck_iters, precision):
+    """(TF32-rate, 3xTF32-rate) algorithmic flops of one refresh of every factor."""
+    from bit_quantized_shampoo_b200 import costmodel as cm
+    single = triple = 0.0
+    for m, n in dims:
+        for d in (m, n):
+            bj = 4.0 * bjorck_iters * float(d) ** 3
+            single += bj
+            triple += cm.refresh_flops(d, bjorck_iters) - bj
+    if precision == "fp32":
+        single, triple = 0.0, single + triple
+    return single, triple
+
+
+def formula_roofline(work, seconds, pk, pk_src, label, sustained=True):
+    """Achieved = algorithmic flops / time; peak = the same flops over their
+    ideal time at the TF32 rate (single) and a third of it (triple), i.e. the
+    precision-weighted peak; frac = ideal time / time."""
+    single, triple = work
+    bf16 = pk.get("bf16_tflops_sustained" if sustained else "bf16_tflops", 1400.0)
+    tf32 = bf16 * TF32_OVER_BF16
+    ideal = single / (tf32 * 1e12) + triple / (tf32 / 3.0 * 1e12)
+    total = single + triple
+    return {"bound": "tensor", "achieved": total / seconds / 1e12, "peak": total / ideal / 1e12,
+            "unit": "TFLOP/s", "frac": ideal / seconds, "kernel": label,
+            "flops": total, "flops_tf32": single, "flops_3xtf32": triple, "ideal_ms": ideal * 1e3,
+            "peak_source": (f"{pk_src} bf16 {'sustained' if sustained else 'burst'} x 1.1/2.25 (TF32), "
+                            f"a third of that for 3xTF32; weighted by the flops at each")}
+
+
 def workload_shapes(wid, shapes=None):
     import dataclasses
     from bit_quantized_shampoo_b200.workloads import WORKLOADS
@@ -205,18 +270,27 @@ def workload_shapes(wid, shapes=None):
 
 
 # ------------------------------------------------------------------ CPU oracle leg
-def cpu_sample(w, nblocks_sample: int, seed_step: int = 1):
-    """Time the oracle on a bounded sample of tiles; returns (seconds per tile,
-    tiles in the workload, description, threads)."""
+def cpu_tile_sample(w, ntiles: int, seed: int = 7):
+    """The CPU baseline's tiles: every ragged tile (an edge below max_block),
+    then seeded random full tiles up to ntiles in all."""
+    from oracle import shampoo4_oracle as O
+    blocks = O.partition(w.shapes, w.max_block)
+    ragged = [k for k, b in enumerate(blocks) if b.m < w.max_block or b.n < w.max_block]
+    full = [k for k in range(len(blocks)) if k not in set(ragged)]
+    rng = np.random.default_rng(seed)
+    extra = list(rng.permutation(full)[:max(0, ntiles - len(ragged))]) if full else []
+    return blocks, sorted(ragged[:ntiles] + [int(k) for k in extra])
+
+
+def cpu_sample(w, picks, blocks, seed_step: int = 1):
+    """Time the oracle on the given tiles (stats + warm refresh of both
+    factors with Bjorck + precondition; a first, cold refresh is untimed).
+    Returns (seconds per tile, threads)."""
     from oracle import shampoo4_oracle as O
     from bit_quantized_shampoo_b200.workloads import gradient
-    blocks = O.partition(w.shapes, w.max_block)
-    rng = np.random.default_rng(7)
-    pick = sorted(set([len(blocks) - 1] + list(rng.choice(len(blocks), size=min(nblocks_sample, len(blocks)),
-                                                            replace=False)[:max(0, nblocks_sample - 1)])))
     grads = {}
     t_total = 0.0
-    for k in pick:
+    for k in picks:
         b = blocks[k]
         if b.param not in grads:
             grads[b.param] = gradient(w, b.param, seed_step)
@@ -238,9 +312,13 @@ def cpu_sample(w, nblocks_sample: int, seed_step: int = 1):
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
         threads = os.cpu_count() or 1
-    desc = (f"{len(pick)} of {len(blocks)} tiles (stats + warm refresh with Bjorck of both factors + "
-            f"precondition), per-tile time extrapolated to the whole workload")
-    return t_total / len(pick), len(blocks), desc, threads
+    return t_total / max(1, len(picks)), threads
+
+
+def cpu_rate(w, picks, blocks, seed_step=1):
+    """(steps/s extrapolated from the sample's mean per-tile time, threads)."""
+    tile_s, threads = cpu_sample(w, picks, blocks, seed_step)
+    return 1.0 / (tile_s * len(blocks)), threads
 
 
 # ------------------------------------------------------------------ ranks
@@ -264,25 +342,94 @@ def job_rate(world, units_per_rank, ms):
 
 # ------------------------------------------------------------------ main
 def run_reference(args, rank, world):
+    """The oracle as the reference arm, on the host cores: each step times a
+    different slice of 4 tiles of the CPU baseline's sample (every ragged
+    tile plus seeded full ones), extrapolated per tile to the workload."""
     if rank != 0:
         return
     w = workload_shapes(args.workload, args.shapes)
-    per_tile = []
-    desc = threads = None
+    blocks, sample = cpu_tile_sample(w, args.cpu_tiles)
+    per_step = 4
+    rates = []
+    threads = None
     for i in range(args.warmup + args.steps):
-        t, nblocks, desc, threads = cpu_sample(w, 1, seed_step=1 + i)
+        picks = [sample[(per_step * i + j) % len(sample)] for j in range(min(per_step, len(sample)))]
+        v, threads = cpu_rate(w, picks, blocks, seed_step=1 + i)
         if i >= args.warmup:
-            per_tile.append(t)
-    tile_s = float(np.mean(per_tile))
-    value = 1.0 / (tile_s * nblocks)
+            rates.append(v)
+    value = float(len(rates) / np.sum([1.0 / r for r in rates]))      # mean time per step
+    desc = (f"each step: 4 tiles of a {len(sample)}-tile sample (all ragged tiles + seeded full ones) of "
+            f"{len(blocks)}, stats + warm refresh with Bjorck of both factors + precondition; per-tile time "
+            f"extrapolated to the whole workload")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name, "tiles": nblocks},
+            "data": "synthetic", "config": {"workload": w.name, "tiles": len(blocks), "steps_per_refresh": 1},
             "cpu_baseline": {"value": value, "unit": "steps/s", "cores": threads, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def measure_config(wid, dev, args, pk, pk_src, world):
+    """One of the smaller workloads at its own refresh interval T: cycles of
+    T steps (statistics every step, a refresh on the first step of each
+    cycle, precondition every step), gradients resident in HBM, CUDA events
+    on the launching stream.  Also the refresh call alone.  Every rank runs
+    its own copy (no collective); times are the max over ranks."""
+    import torch
+    from bit_quantized_shampoo_b200 import api
+    from bit_quantized_shampoo_b200.workloads import WORKLOADS, gradient
+    w = WORKLOADS[wid]
+    T = w.refresh_every
+    shapes = list(w.shapes)
+    sh = api.Shampoo4(shapes, beta=w.beta, eps=w.eps, max_block=w.max_block, bjorck_iters=w.bjorck_iters,
+                      precision=args.precision, device=dev)
+    sets = [[torch.from_numpy(gradient(w, i, 1 + s)).to(dev) for i in range(len(shapes))] for s in range(2)]
+    out = [torch.empty(s, dtype=torch.float32, device=dev) for s in shapes]
+    stream = torch.cuda.current_stream()
+    t = [0]
+
+    def step():
+        g = sets[t[0] % 2]
+        sh.update_stats(g)
+        if t[0] % T == 0:
+            sh.refresh_roots()
+        sh.precondition(g, out=out)
+        t[0] += 1
+
+    for _ in range(max(3, T)):
+        step()
+    while t[0] % T:
+        step()
+    cycles = max(1, (20 + T - 1) // T) if T > 1 else 20
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(cycles * T):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), dev) / (cycles * T)
+    # the refresh alone
+    reps = 5
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record(stream)
+    for _ in range(reps):
+        sh.refresh_roots()
+    r1.record(stream)
+    torch.cuda.synchronize()
+    rms = max_over_ranks(r0.elapsed_time(r1), dev) / reps
+    dims = [tuple(sh.block_info(k)[3:5]) for k in range(sh.nblocks)]
+    res = {"workload": w.name, "tiles": sh.nblocks, "factors": sh.nfactors, "refresh_every": T,
+           "steps_timed": cycles * T, "ms_per_step": ms, "us_per_step": ms * 1e3,
+           "steps_per_s": world * 1e3 / ms, "refresh_ms": rms, "root_refreshes_per_s": world * sh.nfactors * 1e3 / rms,
+           "status_flags": sh.status_flags(),
+           "roofline": formula_roofline(step_work(dims, w.bjorck_iters, T, args.precision), ms / 1e3, pk, pk_src,
+                                        f"step at T = {T}, algorithmic flops of the work model"),
+           "workspace_bytes": sh.workspace_bytes, "state_bytes": sh.state_bytes}
+    del sh, sets, out
+    return res
 
 
 def main():
@@ -317,7 +464,7 @@ def main():
     host_g = host_sets[0]
     dev_out = [torch.empty(s, dtype=torch.float32, device=dev) for s in shapes]
     host_out = [torch.empty(s, dtype=torch.float32).pin_memory() for s in shapes]
-    shard = args.shard_refresh and world > 1
+    shard = (not args.replicas) and world > 1
     sh = api.Shampoo4(shapes, beta=w.beta, eps=w.eps, max_block=w.max_block, bjorck_iters=w.bjorck_iters,
                       precision=args.precision, device=dev, compressed=args.compressed,
                       refresh_rank=rank if shard else 0, refresh_world=world if shard else 1)
@@ -382,16 +529,31 @@ def main():
     pk, pk_src = peaks()
     clocks = clk.summary()
     g_bytes = sum(r * c for r, c in shapes) * 4
-    stat_bytes = sum(int(b[3]) ** 2 + int(b[4]) ** 2 for b in (sh.block_info(k) for k in range(sh.nblocks))) * 4
+    dims = [tuple(sh.block_info(k)[3:5]) for k in range(sh.nblocks)]
+    stat_bytes = sum(m * m + n * n for m, n in dims) * 4
+    # headline: the whole step by the work model's formulas (refresh on every
+    # step here), against the precision-weighted tensor peak
+    roof = formula_roofline(step_work(dims, w.bjorck_iters, 1, args.precision), ms_per_step / 1e3, pk, pk_src,
+                            "whole step (statistics + refresh + precondition), algorithmic flops of the work model")
+    roof["traffic"] = None
+    roof["traffic_note"] = "no single-kernel DRAM count for a whole step; per-stage GEMM traffic in rooflines_other"
+    refresh_stages = ("refresh_scan", "basis", "bjorck_gram", "bjorck_update", "subspace", "qr_gram", "qr_potrf",
+                      "qr_trsm_panel", "qr_syrk", "qr_solve_update", "qr_solve_panel", "qr_convert", "qr_inverse",
+                      "rayleigh_gemm", "rayleigh", "requant")
+    refresh_ms = sum(stages[k]["ms"] for k in refresh_stages if k in stages)
+    others = [formula_roofline(refresh_work(dims, w.bjorck_iters, args.precision), refresh_ms / 1e3, pk, pk_src,
+                               "refresh of every factor (a3-a8), algorithmic flops of the work model; time = sum of "
+                               "its stages' launch times")]
+    # per stage: the flops each launch's descriptors carry (the implementation's
+    # products, which exceed the work model's count for the QR)
     ranked = sorted(stages, key=lambda k: -stages[k]["ms"])
-    dom = next(k for k in ranked if STAGE_BOUND.get(k, "latency") != "latency")
-    roof = stage_roofline(dom, stages[dom], pk, pk_src)
-    factor_elems = sum(int(b[3]) ** 2 + int(b[4]) ** 2 for b in (sh.block_info(k) for k in range(sh.nblocks)))
-    roof["traffic"] = stage_traffic(dom, factor_elems)
-    if roof["traffic"] is not None:
-        roof["traffic_note"] = ("dram read+write bytes of one launch of this stage's GEMM, scaled from an ncu capture "
-                                "on 32 factors of 1024x1024 by factor elements")
-    others = [stage_roofline(k, stages[k], pk, pk_src) for k in ranked[:8] if k != dom]
+    for k in ranked[:8]:
+        r = stage_roofline(k, stages[k], pk, pk_src)
+        t = stage_traffic(k, sum(m * m + n * n for m, n in dims))
+        if t is not None:
+            r["traffic"] = t
+        r["flops_note"] = "implementation flops of the stage's launches (not the work model's count)"
+        others.append(r)
 
     line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -400,6 +562,7 @@ def main():
             "data": "synthetic",
             "config": {"workload": w.name, "tiles": sh.nblocks, "factors": sh.nfactors,
                        "steps_per_refresh": 1,
+                       "refresh_ms_per_step": refresh_ms,
                        "statistics": "compressed (4-bit eigenbasis + eigenvalues)" if args.compressed else "fp32",
                        "parallelism": (f"refresh sharded over {world} ranks + NCCL span broadcasts" if shard
                                        else f"{world} independent replica(s)"),
@@ -558,10 +721,24 @@ def main():
                          "status_flags": sh.status_flags()}
         del weights, gstate
 
+    # the four smaller workloads, each at its own refresh interval
+    if not args.no_configs and args.shapes is None and args.workload == 5:
+        del sh
+        torch.cuda.empty_cache()
+        line["configs"] = {}
+        for wid in (1, 2, 3, 4):
+            line["configs"][f"c{wid}"] = measure_config(wid, dev, args, pk, pk_src, world)
+            torch.cuda.empty_cache()
+
     if rank == 0 and world == 1 and not args.no_cpu:
-        tile_s, nb, desc, threads = cpu_sample(w, 4)
-        v = 1.0 / (tile_s * nb)
-        line["cpu_baseline"] = {"value": v, "unit": "steps/s", "cores": threads, "kind": "oracle", "sample": desc}
+        blocks, sample = cpu_tile_sample(w, args.cpu_tiles)
+        v, threads = cpu_rate(w, sample, blocks)
+        nrag = sum(1 for k in sample if blocks[k].m < w.max_block or blocks[k].n < w.max_block)
+        line["cpu_baseline"] = {"value": v, "unit": "steps/s", "cores": threads, "kind": "oracle",
+                                "sample": (f"{len(sample)} of {len(blocks)} tiles ({nrag} ragged + "
+                                           f"{len(sample) - nrag} seeded full ones): stats + warm refresh with "
+                                           f"Bjorck of both factors + precondition; mean per-tile time extrapolated "
+                                           f"to the whole workload (extrapolated)")}
 
     if world > 1:
         dist.barrier()

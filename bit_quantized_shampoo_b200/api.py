@@ -33,7 +33,8 @@ class Shampoo4:
     """One handle: a fixed list of 2-D parameter shapes and their state."""
 
     def __init__(self, shapes, beta=0.95, eps=1e-6, max_block=1024, bjorck_iters=5,
-                 precision="tf32", device=None, reset=True, compressed=False, refresh_rank=0, refresh_world=1):
+                 precision="tf32", device=None, reset=True, compressed=False, refresh_rank=0, refresh_world=1,
+                 debug=False):
         self.shapes = [(int(r), int(c)) for r, c in shapes]
         self.compressed = bool(compressed)
         self.refresh_rank, self.refresh_world = int(refresh_rank), int(refresh_world)
@@ -54,6 +55,12 @@ class Shampoo4:
         nb, nf = C.c_int32(), C.c_int32()
         L.call("shampoo4_counts", h, C.byref(nb), C.byref(nf))
         self.nblocks, self.nfactors = nb.value, nf.value
+        self.debug_buffer = None
+        if debug:
+            n = C.c_size_t()
+            L.call("shampoo4_debug_capture_bytes", h, C.byref(n))
+            self.debug_buffer = torch.zeros(max(n.value, 256), dtype=torch.uint8, device=self.device)
+            L.call("shampoo4_debug_capture", h, C.c_void_p(self.debug_buffer.data_ptr()))
         self.bind(reset=reset)
 
     def bind(self, reset=True, stream=None):
@@ -175,11 +182,34 @@ class Shampoo4:
         lam = st[ol.value:ol.value + 4 * d].view(torch.float32)
         return S, codes, scales, lam
 
+    def _dim(self, f):
+        d = C.c_int32()
+        L.call("shampoo4_factor_layout", self._h, f, None, None, None, None, C.byref(d))
+        return d.value
+
     def debug_q(self, f):
+        """The pre-quantization Q of factor f from the last refresh: from the
+        debug capture buffer when the handle has one, else from the workspace
+        (valid until the next call)."""
+        d = self._dim(f)
+        if self.debug_buffer is not None:
+            off = C.c_size_t()
+            L.call("shampoo4_debug_capture_layout", self._h, f, None, C.byref(off))
+            return self.debug_buffer[off.value:off.value + 4 * d * d].view(torch.float32).view(d, d)
         off = C.c_size_t()
         L.call("shampoo4_debug_q_offset", self._h, f, C.byref(off))
-        d = self.factor_views(f)[0].shape[0]
         return self.workspace[off.value:off.value + 4 * d * d].view(torch.float32).view(d, d)
+
+    def debug_rectified(self, f):
+        """The rectified basis (dequantized and Bjorck-rectified; the
+        identity on a first refresh) that entered the last refresh's subspace
+        step for factor f.  Needs a handle made with debug=True."""
+        if self.debug_buffer is None:
+            raise RuntimeError("debug_rectified needs a handle made with debug=True")
+        d = self._dim(f)
+        off = C.c_size_t()
+        L.call("shampoo4_debug_capture_layout", self._h, f, C.byref(off), None)
+        return self.debug_buffer[off.value:off.value + 4 * d * d].view(torch.float32).view(d, d)
 
     def close(self):
         if getattr(self, "_h", None):

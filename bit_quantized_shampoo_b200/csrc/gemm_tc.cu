@@ -18,8 +18,13 @@
 // Warp roles (192 threads): warp 0 issues the TMA loads, warp 1 owns the
 // tensor memory and issues the MMAs, warps 2..5 drain the accumulator
 // (warp w reads TMEM lanes 32*(w%4) .. +31, one output row per thread).
-// Every wait on an mbarrier is bounded in time; on expiry the CTA raises
-// SHAMPOO4_FLAG_TIMEOUT, drains what it issued and exits.
+// Every wait on an mbarrier is bounded in time.  The three waits of the
+// pipeline (the producer's for a free stage, the MMA issuer's for a loaded
+// one, the epilogue's for the finished accumulator) give up after a limit
+// the host passes (2 s unless a diagnostic sets another); on expiry the CTA
+// raises SHAMPOO4_FLAG_TIMEOUT and stops issuing.  Before it exits it still
+// waits, with the 2 s limit, for everything it issued: the producer for its
+// TMA loads, the MMA warp for its MMAs (before it frees tensor memory).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include "tc.h"
@@ -58,14 +63,14 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false after ~2 s without the phase completing.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait: false after about limit_ns without the phase completing.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitNs) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = now_ns();
   for (;;) {
     for (int i = 0; i < 64; ++i)
       if (mbar_try(bar, parity)) return true;
-    if (now_ns() - t0 > kWaitNs) return false;
+    if (now_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -420,7 +425,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmDesc& g, const PtrEntr
 template <int BN, bool SPLIT, int STAGES>
 __global__ void __launch_bounds__(192, STAGES <= 2 ? 2 : 1)
 k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, int nparams,
-          uint32_t* __restrict__ gflags) {
+          uint32_t* __restrict__ gflags, uint64_t wait_ns) {
   using Cfg = TcCfg<BN, SPLIT, STAGES>;
   const TcGemmDesc& g = descs[blockIdx.y];
   const int tiles_n = (g.N + BN - 1) / BN;
@@ -474,7 +479,7 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
       int issued = 0;
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % Cfg::kStages;
-        if (kb >= Cfg::kStages && !mbar_wait(&empty_bar[s], ((kb / Cfg::kStages) - 1) & 1)) {
+        if (kb >= Cfg::kStages && !mbar_wait(&empty_bar[s], ((kb / Cfg::kStages) - 1) & 1, wait_ns)) {
           atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
           abort_flag = 1;
           break;
@@ -492,9 +497,12 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
         issued = kb + 1;
       }
       // Whatever happened, the loads issued last must land before the CTA
-      // exits: wait (bounded) for the final phases of the live stages.
+      // exits: wait for the final phases of the live stages (the 2 s limit,
+      // whatever limit the pipeline waits had).  Every earlier load was
+      // consumed by an MMA before its stage was refilled.
       for (int kb = issued - Cfg::kStages < 0 ? 0 : issued - Cfg::kStages; kb < issued; ++kb)
-        if (!mbar_wait(&full_bar[kb % Cfg::kStages], (kb / Cfg::kStages) & 1)) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+        if (!mbar_wait(&full_bar[kb % Cfg::kStages], (kb / Cfg::kStages) & 1, kWaitNs))
+          atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
     }
   } else if (warp == 1) {
     if (lane == 0) {                                        // ---- MMA issuer
@@ -502,7 +510,7 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
       const uint32_t idesc = idesc_tf32(kBM, BN, ga.mn_major, gb.mn_major);
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % Cfg::kStages;
-        if (!mbar_wait(&full_bar[s], (kb / Cfg::kStages) & 1)) {
+        if (!mbar_wait(&full_bar[s], (kb / Cfg::kStages) & 1, wait_ns)) {
           atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
           abort_flag = 1;
           break;
@@ -526,10 +534,13 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
         mma_commit(&empty_bar[s]);                          // stage free once these MMAs finish
       }
       mma_commit(&done_bar);                                // accumulator complete
+      // every MMA this thread issued completes before tensor memory is
+      // freed below, even when the epilogue gave up waiting for them
+      if (!mbar_wait(&done_bar, 0, kWaitNs)) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
     }
   } else {                                                  // ---- epilogue, warps 2..5
     const int q = warp & 3;                                 // TMEM lane quarter = 32-row slab
-    const bool ok = mbar_wait(&done_bar, 0);
+    const bool ok = mbar_wait(&done_bar, 0, wait_ns);
     if (!ok) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
     fence_after_sync();
     if (ok && !*(volatile int*)&abort_flag) {
@@ -547,7 +558,7 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
 
 template <int BN, bool SPLIT, int STAGES>
 shampoo4_status launch_tc_impl(const TcGemmDesc* d_desc, int count, int max_tiles, const PtrEntry* tabs,
-                               int nparams, uint32_t* gflags, cudaStream_t st) {
+                               int nparams, uint32_t* gflags, uint64_t wait_ns, cudaStream_t st) {
   using Cfg = TcCfg<BN, SPLIT, STAGES>;
   static bool configured = false;
   if (!configured) {
@@ -558,7 +569,7 @@ shampoo4_status launch_tc_impl(const TcGemmDesc* d_desc, int count, int max_tile
   for (int base = 0; base < count; base += 65535) {
     const int c = count - base < 65535 ? count - base : 65535;
     k_gemm_tc<BN, SPLIT, STAGES><<<dim3(unsigned(max_tiles), unsigned(c)), 192, Cfg::kSmem, st>>>(
-        d_desc + base, tabs, nparams, gflags);
+        d_desc + base, tabs, nparams, gflags, wait_ns);
     S4_CUDA(cudaGetLastError());
   }
   return SHAMPOO4_OK;
@@ -569,8 +580,10 @@ shampoo4_status launch_tc_impl(const TcGemmDesc* d_desc, int count, int max_tile
 int tc_block_n(int split) { return split ? 128 : 256; }
 
 shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split, int bn,
-                               const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st) {
+                               const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st,
+                               uint64_t wait_ns) {
   if (count <= 0 || max_tiles <= 0) return SHAMPOO4_OK;
+  if (wait_ns == 0 || wait_ns > kWaitNs) wait_ns = kWaitNs;
   // One tile per CTA.  TF32: two 2-stage CTAs per SM, so one tile's
   // epilogue overlaps the other's main loop.  (A persistent form with two
   // TMEM accumulator sets and eight epilogue warps was measured against it:
@@ -580,9 +593,9 @@ shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tile
   // CTAs per SM with 64-wide tiles for the narrow panel updates, where the
   // MMA issue rate of a 64-wide instruction makes a second issuing CTA per
   // SM worth more than overlap.
-  if (!split) return launch_tc_impl<256, false, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, st);
-  if (bn == 64) return launch_tc_impl<64, true, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, st);
-  return launch_tc_impl<128, true, 3>(d_desc, count, max_tiles, tabs, nparams, gflags, st);
+  if (!split) return launch_tc_impl<256, false, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, wait_ns, st);
+  if (bn == 64) return launch_tc_impl<64, true, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, wait_ns, st);
+  return launch_tc_impl<128, true, 3>(d_desc, count, max_tiles, tabs, nparams, gflags, wait_ns, st);
 }
 
 // ---------------------------------------------------------------- host side

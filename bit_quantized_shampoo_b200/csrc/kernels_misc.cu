@@ -682,4 +682,23 @@ shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max
   return SHAMPOO4_OK;
 }
 
+__global__ void __launch_bounds__(256) k_copy(const CopyDesc* __restrict__ descs, int count, int chunks) {
+  for (int w = blockIdx.x; w < count * chunks; w += gridDim.x) {
+    const CopyDesc& g = descs[w / chunks];
+    const int64_t lo = int64_t(w % chunks) * kConvertChunk;
+    if (lo >= g.n || !g.dst) continue;
+    const int64_t hi = lo + kConvertChunk < g.n ? lo + kConvertChunk : g.n;
+    for (int64_t e = lo + threadIdx.x; e < hi; e += blockDim.x) g.dst[e] = g.src[e];
+  }
+}
+
+shampoo4_status launch_copy(const CopyDesc* d_desc, int count, int64_t max_elems, cudaStream_t st) {
+  if (count <= 0 || max_elems <= 0) return SHAMPOO4_OK;
+  const int chunks = int((max_elems + kConvertChunk - 1) / kConvertChunk);
+  const int64_t items = int64_t(count) * chunks;
+  k_copy<<<unsigned(items < kWorkCtas ? items : kWorkCtas), 256, 0, st>>>(d_desc, count, chunks);
+  S4_CUDA(cudaGetLastError());
+  return SHAMPOO4_OK;
+}
+
 }  // namespace s4

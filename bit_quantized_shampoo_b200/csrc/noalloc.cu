@@ -11,8 +11,12 @@
 // that cudaMalloc -- directly or through a library -- would fail or deadlock.
 //
 // Scratch: one file-scope __device__ array (kNoallocScratchBytes, 1 MiB +
-// 4 KiB, one instance per device), found once per device with
-// cudaGetSymbolAddress while that device is current.  It holds
+// 4 KiB, one instance per device), whose device address every call looks up
+// with cudaGetSymbolAddress while the caller's device is current.  The
+// lookup allocates nothing and is cheap once the module is loaded; doing it
+// on every call (rather than caching it per device ordinal) keeps the
+// address right when a context is torn down and created again, which can
+// move the module.  It holds
 //   - the launch descriptors and the gradient's pointer table, written on
 //     the stream by a one-warp setup kernel at the start of every call;
 //   - two flag words that must start every call at zero (the tile's
@@ -22,14 +26,12 @@
 //     by the scan kernel and read by both products.
 // Overlapping calls (on different streams, or from different host threads
 // without ordering) share that scratch and race; calls must be ordered.
-// The first call on a device performs the symbol lookup and may load the
-// module, so it should come before any stream capture.
+// The first call on a device may load the module, so it should come before
+// any stream capture.
 //
 // The kernels are the library's own: the gradient scan that also writes the
 // TF32 copy, and the CUDA-core fp32-output GEMM in TF32 mode (operands
 // rounded to TF32, exact products, fp32 sums) with a symmetric output.
-#include <mutex>
-
 #include "plan.h"
 
 namespace s4 {
@@ -39,7 +41,6 @@ constexpr int kNoallocMaxEdge = 1024;                     // m, n
 constexpr int64_t kNoallocMaxElems = int64_t(1) << 18;   // m * n (staged gradient copy)
 constexpr size_t kNoallocHeaderBytes = 4096;
 constexpr size_t kNoallocScratchBytes = kNoallocHeaderBytes + size_t(kNoallocMaxElems) * sizeof(float);
-constexpr int kNoallocMaxDevices = 64;
 
 struct alignas(256) NoallocHeader {
   uint32_t flag;                // non-finite gradient: gates both products
@@ -53,9 +54,6 @@ static_assert(sizeof(NoallocHeader) <= kNoallocHeaderBytes, "header fits its slo
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
 
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kNoallocMaxDevices] = {};
-
 // Copy the descriptors into scratch (zeroing the flag words with them).
 __global__ void __launch_bounds__(32) k_noalloc_setup(const __grid_constant__ NoallocHeader h,
                                                       NoallocHeader* __restrict__ dst) {
@@ -64,18 +62,14 @@ __global__ void __launch_bounds__(32) k_noalloc_setup(const __grid_constant__ No
   for (int i = threadIdx.x; i < int(sizeof(NoallocHeader) / 4); i += 32) out[i] = src[i];
 }
 
+// The scratch array's device address in the current device's context.  In
+// host code g_noalloc_scratch names a host-side stand-in, never a device
+// address: only this lookup gives one.
 shampoo4_status noalloc_scratch(uint8_t** out) {
-  int dev = -1;
-  S4_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kNoallocMaxDevices) return SHAMPOO4_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p) return SHAMPOO4_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = static_cast<uint8_t*>(g_noalloc_ptr[dev]);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p) return SHAMPOO4_ERR_CUDA;
+  *out = static_cast<uint8_t*>(p);
   return SHAMPOO4_OK;
 }
 

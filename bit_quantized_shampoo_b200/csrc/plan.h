@@ -177,6 +177,15 @@ struct ConvertDesc {
 };
 
 
+// dst[0, n) = src[0, n): the debug capture of a refresh's intermediate
+// matrices into a caller buffer.
+struct CopyDesc {
+  const float* src;
+  float* dst;
+  int64_t n;
+};
+
+
 // W_ii <- sum_k X[k, i]^2 (fp64 sums, one thread per column, rounded once
 // to fp32) for i < d, X row-major d x d.  The tensor cores' accumulation
 // truncates, so a Gram's diagonal -- a sum of positive terms -- comes out
@@ -306,6 +315,7 @@ shampoo4_status launch_shift_f(const ShiftDescF* d_desc, int count, cudaStream_t
 shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st,
                                const uint32_t* guard = nullptr);
 shampoo4_status launch_gate(const GateDesc* d_desc, int count, cudaStream_t st);
+shampoo4_status launch_copy(const CopyDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_inv128(const Inv128Desc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaStream_t st);
 shampoo4_status launch_rowdiag(const RowDiagDesc* d_desc, int count, int max_d, cudaStream_t st);

@@ -30,7 +30,7 @@ using namespace s4;
 namespace {
 
 enum class Kind { GemmF32, GemmF64, Potrf, Trsm, Basis, Rayleigh, Mu, Scan, Convert, Pack, Shift, GemmTC, GemmTCSplit,
-                  GemmTCSplit64, PotrfF, ShiftF, Gate, Diag, RowDiag, Inv128 };
+                  GemmTCSplit64, PotrfF, ShiftF, Gate, Diag, RowDiag, Inv128, Copy };
 
 struct Launch {
   Kind kind;
@@ -75,6 +75,7 @@ struct FactorPlan {
   size_t ws_Jh, ws_Jl;                   // 128 x 128 inverse diagonal blocks (rows to a multiple of 128)
   size_t ws_Ph, ws_Pl;                   // d x 128: solve panel temporary
   size_t ws_q_first, ws_q_next;
+  size_t dbg_u, dbg_q;                   // debug capture: offsets of the rectified U and of Q
 };
 
 constexpr size_t kAlign = 256;
@@ -93,6 +94,11 @@ struct shampoo4_ctx {
   size_t ws_flags = 0, ws_tabs = 0, ws_fail = 0, ws_bflag = 0, ws_maps = 0, ws_nmaps = 0;
   size_t ws_tcbad = 0, ws_tcgood = 0, ws_devsq = 0, ws_skip3 = 0, ws_fbany = 0;
   bool any_simt = false;                 // some factor always takes the fp64 QR
+  // optional debug capture (shampoo4_debug_capture): every refresh copies
+  // each refreshed factor's rectified basis and pre-quantization Q here
+  uint8_t* d_dbg = nullptr;
+  size_t dbg_bytes = 0;
+  uint64_t wait_ns = 0;                  // tensor-core pipeline wait limit (0: the kernel's default)
   size_t ws_desc = 0, ws_desc_bytes = 0;
   // programs
   std::vector<Launch> prog_stats, prog_stats_first, prog_refresh_first, prog_refresh, prog_precond;
@@ -268,6 +274,13 @@ shampoo4_status plan(shampoo4_ctx* h) {
     if (!f.tc && h->owner[i] == h->rank) h->any_simt = true;
   }
   h->state_bytes = align_up(st, kAlign);
+  size_t dbg = 0;
+  for (FactorPlan& f : h->factors) {
+    const size_t dd = size_t(f.d) * f.d;
+    f.dbg_u = take(dbg, 4 * dd);
+    f.dbg_q = take(dbg, 4 * dd);
+  }
+  h->dbg_bytes = align_up(dbg, kAlign);
 
   size_t ws = 0;
   h->ws_flags = take(ws, 16);
@@ -385,6 +398,7 @@ struct Builder {
   }
   uint32_t* skip3(size_t fi) const { return wu(h->ws_skip3) + fi; }
   uint32_t* gflags() const { return wu(h->ws_flags); }
+  float* dbg(size_t off) const { return h->d_dbg ? reinterpret_cast<float*>(h->d_dbg + off) : nullptr; }
 
   // Device address of the tensor map of a dense d0 x d1 workspace matrix.
   const CUtensorMap* map(const float* base, int rows, int cols, int box_rows, int mn_major) {
@@ -1037,6 +1051,16 @@ void build_refresh_owned(Builder& b, std::vector<Launch>& prog, bool first) {
     emit_gemmtc(b, prog, tupd, split);
     emit_gemm32(b, prog, upd);
   }
+  {  // debug capture of the rectified basis (launch skipped without a capture buffer)
+    std::vector<CopyDesc> cp;
+    for (size_t i = 0; i < nf; ++i) {
+      const FactorPlan& f = h->factors[i];
+      const float* U = f.tc ? b.wf(f.ws_Xm[cur[i]]) : b.wf(ucur[i]);
+      cp.push_back({U, b.dbg(f.dbg_u), int64_t(f.d) * f.d});
+    }
+    b.tag = SHAMPOO4_STAGE_BASIS;
+    b.emit(prog, Kind::Copy, cp, emax, 0, 8.0 * sum_dd);
+  }
   // Subspace step Y = (S + eps I) U = S U + eps U, always fp32-accurate.
   std::vector<const float*> Yx(nf);
   std::vector<float*> Q0(nf), Q1(nf), Qf(nf), Qh(nf, nullptr), Ql(nf, nullptr), none(nf, nullptr);
@@ -1131,6 +1155,13 @@ void build_refresh_owned(Builder& b, std::vector<Launch>& prog, bool first) {
   for (size_t i = 0; i < nf; ++i) {
     const size_t off = size_t(reinterpret_cast<uint8_t*>(Qf[i]) - b.ws);
     (first ? h->factors[i].ws_q_first : h->factors[i].ws_q_next) = off;
+  }
+  {  // debug capture of the pre-quantization Q
+    std::vector<CopyDesc> cp;
+    for (size_t i = 0; i < nf; ++i)
+      cp.push_back({Qf[i], b.dbg(h->factors[i].dbg_q), int64_t(h->factors[i].d) * h->factors[i].d});
+    b.tag = SHAMPOO4_STAGE_QR_CONVERT;
+    b.emit(prog, Kind::Copy, cp, emax, 0, 8.0 * sum_dd);
   }
   // Rayleigh quotients: T = S Q (fp32-accurate), lambda_i = max(q_i . t_i, 0).
   {
@@ -1372,7 +1403,7 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
       case Kind::GemmTCSplit64:
         S4_TRY(launch_gemm_tc(static_cast<const TcGemmDesc*>(d), L.count, int(L.extent),
                               L.kind == Kind::GemmTC ? 0 : 1, L.kind == Kind::GemmTCSplit64 ? 64 : 0, tabs, np,
-                              gflags, st));
+                              gflags, st, h->wait_ns));
         break;
       case Kind::PotrfF:
         S4_TRY(launch_potrf_f(static_cast<const PotrfDescF*>(d), L.count, st));
@@ -1397,6 +1428,9 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
         break;
       case Kind::Convert:
         S4_TRY(launch_convert(static_cast<const ConvertDesc*>(d), L.count, L.extent, st, guard));
+        break;
+      case Kind::Copy:
+        if (h->d_dbg) S4_TRY(launch_copy(static_cast<const CopyDesc*>(d), L.count, L.extent, st));
         break;
       case Kind::Pack:
         S4_TRY(launch_pack(L.px.data(), L.pn.data(), L.count, L.pcodes.data(), L.pscales.data(), st,
@@ -1729,6 +1763,34 @@ extern "C" shampoo4_status shampoo4_debug_s_offset(shampoo4_handle h, int32_t fa
   if (!h || !off_s || !h->cfg.compressed_stats || factor < 0 || size_t(factor) >= h->factors.size())
     return SHAMPOO4_ERR_INVALID_ARG;
   *off_s = h->factors[factor].ws_S;
+  return SHAMPOO4_OK;
+}
+
+extern "C" shampoo4_status shampoo4_debug_capture_bytes(shampoo4_handle h, size_t* bytes) {
+  if (!h || !bytes) return SHAMPOO4_ERR_INVALID_ARG;
+  *bytes = h->dbg_bytes;
+  return SHAMPOO4_OK;
+}
+
+extern "C" shampoo4_status shampoo4_debug_capture(shampoo4_handle h, void* d_buf) {
+  if (!h) return SHAMPOO4_ERR_INVALID_ARG;
+  if (d_buf && !aligned(d_buf, kAlign)) return SHAMPOO4_ERR_INVALID_ARG;
+  h->d_dbg = static_cast<uint8_t*>(d_buf);
+  h->bound = false;                       // the refresh programs carry the buffer's addresses: bind again
+  return SHAMPOO4_OK;
+}
+
+extern "C" shampoo4_status shampoo4_debug_capture_layout(shampoo4_handle h, int32_t factor, size_t* off_u,
+                                                         size_t* off_q) {
+  if (!h || factor < 0 || size_t(factor) >= h->factors.size()) return SHAMPOO4_ERR_INVALID_ARG;
+  if (off_u) *off_u = h->factors[factor].dbg_u;
+  if (off_q) *off_q = h->factors[factor].dbg_q;
+  return SHAMPOO4_OK;
+}
+
+extern "C" shampoo4_status shampoo4_debug_wait_limit(shampoo4_handle h, uint64_t ns) {
+  if (!h) return SHAMPOO4_ERR_INVALID_ARG;
+  h->wait_ns = ns;
   return SHAMPOO4_OK;
 }
 

@@ -46,8 +46,11 @@ struct TcGemmDesc {
 // Tile width N of the kernel instance: 256 (TF32), 128 (split), or 64
 // (split, narrow products).
 int tc_block_n(int split);
+// wait_ns: how long each pipeline wait may take before the CTA gives up
+// (SHAMPOO4_FLAG_TIMEOUT); 0 means the default of 2 s, which is also the cap.
 shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split, int bn,
-                               const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st);
+                               const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st,
+                               uint64_t wait_ns = 0);
 // Encode a 2-D fp32 tensor map (rows x cols, leading dimension ld elements),
 // box 32 (contiguous) x box_rows, zero fill out of bounds; 128-byte swizzle,
 // with 32-byte atoms for an operand read MN-major.

@@ -230,6 +230,39 @@ shampoo4_status shampoo4_debug_q_offset(shampoo4_handle h, int32_t factor, size_
  * tests and diagnostics. */
 shampoo4_status shampoo4_debug_s_offset(shampoo4_handle h, int32_t factor, size_t* off_s);
 
+/* Debug capture, for tests and diagnostics: the boundaries between the
+ * refresh's stages.  ("4-bit Shampoo for Memory-Efficient Network Training",
+ * abstract: the dequantized eigenvector matrix is rectified, then refined;
+ * the refinement is one subspace step, Y = (S + eps I) U, Y = QR.)
+ *
+ * shampoo4_debug_capture_bytes gives the size of the capture buffer: two
+ * fp32 d x d matrices per factor, each 256-byte aligned.
+ * shampoo4_debug_capture registers a caller-owned device buffer of that size
+ * (256-byte aligned; NULL unregisters).  The handle must then be bound again
+ * (shampoo4_bind, reset = 0 keeps the state), because the refresh programs
+ * carry the buffer's addresses.  While one is registered, every
+ * refresh_roots also copies, for each factor it refreshes, the rectified
+ * basis that enters the subspace step (after dequantization and Bjorck; the
+ * identity on a first refresh) and the orthonormal Q that is then
+ * requantized.  The buffer must stay allocated until it is unregistered and
+ * the handle bound again, or destroyed.  Without one, the copies are not
+ * launched.  shampoo4_debug_capture_layout gives the byte offsets of a
+ * factor's two row-major matrices in the buffer. */
+shampoo4_status shampoo4_debug_capture_bytes(shampoo4_handle h, size_t* bytes);
+shampoo4_status shampoo4_debug_capture(shampoo4_handle h, void* d_buf);
+shampoo4_status shampoo4_debug_capture_layout(shampoo4_handle h, int32_t factor, size_t* off_u,
+                                              size_t* off_q);
+
+/* Diagnostic: the time limit of the tensor-core products' pipeline waits
+ * (a CTA waiting for a free stage, for loaded operands or for its finished
+ * accumulator).  On expiry a CTA raises SHAMPOO4_FLAG_TIMEOUT, issues
+ * nothing more, waits (up to 2 s) for the loads and MMAs it already issued,
+ * frees its tensor memory and exits; the call's outputs are then undefined,
+ * the handle and the CUDA context stay usable.  ns = 0 restores the default
+ * of 2 s, which is also the largest limit.  Used by the tests to exercise
+ * that return path; it takes effect at the next launch. */
+shampoo4_status shampoo4_debug_wait_limit(shampoo4_handle h, uint64_t ns);
+
 /* Refresh sharding: the rank that refreshes a factor, and the state byte
  * range [*off, *off + *bytes) holding the codes, scales and eigenvalues of
  * every factor that rank refreshes (the same on every rank's handle). */
@@ -309,8 +342,10 @@ shampoo4_status quant4_tables(float codebook[16], float thresholds[15]);
  * Scratch is a fixed 1 MiB + 4 KiB device array inside the library (one per
  * device); every call resets what must start at zero.  Calls that overlap
  * (different streams or unordered host threads) share it and race: order
- * them.  The first call on a device looks the array up and may load the
- * module; make it before any stream capture.  Everything is enqueued on
+ * them.  Every call looks up the array's address in the current device's
+ * context (cudaGetSymbolAddress: no allocation, and right again after a
+ * context is destroyed and recreated).  The first call on a device may load
+ * the module; make it before any stream capture.  Everything is enqueued on
  * `stream`; nothing is allocated or freed. */
 shampoo4_status shampoo4_update_stats_noalloc(float* d_L, float* d_R, const float* d_G, int32_t m,
                                               int32_t n, int64_t ldg, float beta, uint32_t* d_flags,

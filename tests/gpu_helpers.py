@@ -48,32 +48,120 @@ def basis_root(Q, lam, eps):
     return (Q * mu[None, :]) @ Q.T
 
 
-def refresh_errors(sh, orc, eps):
-    """After sh.refresh_roots() and orc.refresh_roots() from the same incoming
-    state: per factor (d, ||Q^T Q - I||_F/sqrt(d), lambda excess, root excess),
-    with the requantized codes checked bit-exact against the oracle quantizer
-    applied to the library's own Q.  The lambda and root excesses are taken
-    over the fp32-accurate arithmetic's resolution, as in the stage tests:
-    about 16 u lambda_max for lambda and u kappa for the basis-invariant root
-    (u = 2^-21), nothing pinned beyond u32 kappa >= 1."""
-    out = []
-    for f in range(sh.nfactors):
-        d = orc.factors[f].d
-        Qg = sh.debug_q(f).cpu().numpy().astype(np.float64)
-        g = gpu_factor(sh, f)
-        oc, os_ = O.quantize(Qg.astype(np.float32).ravel())
-        assert np.array_equal(g.codes, oc) and np.array_equal(g.scales, os_), f
-        orth = float(np.linalg.norm(Qg.T @ Qg - np.eye(d)) / np.sqrt(d))
-        Qo, lo = orc.factors[f].q_last, orc.factors[f].lam.astype(np.float64)
-        lg = g.lam.astype(np.float64)
-        big = lo > 1e3 * eps
-        slack = 16 * 2.0 ** -21 * lo.max()
-        excess = np.maximum(np.abs(lg - lo) - slack, 0.0)
-        lam_err = float(np.max(excess[big] / lo[big])) if big.any() else 0.0
-        kappa = (lo.max() + eps) / (lo.min() + eps)
-        root_err = rel_fro(basis_root(Qg, lo, eps), basis_root(Qo, lo, eps))
-        root_err = max(root_err - 2.0 ** -21 * kappa, 0.0)
-        if 6e-8 * kappa >= 1.0:
-            root_err = 0.0
-        out.append((d, orth, lam_err, root_err))
-    return out
+# Unit roundoff of the fp32-accurate (3xTF32) products that the subspace
+# step, the QR and the Rayleigh quotients run on.
+U21 = 2.0 ** -21
+# The refresh gates allow the stage tolerance plus this multiple of the
+# oracle's own spread (the "band" below).
+BAND_FACTOR = 4.0
+
+
+def _oracle_spread(S, U, eps, Qo, lo, big, seeds=3):
+    """The oracle's own sensitivity at this input: the largest change of
+    lambda_i (relative, over lambda_i > 1e3 eps) and of the basis-invariant
+    root when S and U carry independent relative perturbations of 2^-21 --
+    the rounding any fp32-accurate arithmetic leaves in the subspace
+    product, the QR and the Rayleigh product.  Rank-deficient or
+    ill-conditioned statistics make the last columns of the QR inside S's
+    range, and the eigen-directions next to eps, sensitive far beyond 2^-21;
+    this measures by how much, for this very factor."""
+    S = np.asarray(S, np.float64)
+    U = np.asarray(U, np.float64)
+    band_lam = band_root = 0.0
+    ref = basis_root(Qo, lo, eps)
+    for seed in range(seeds):
+        rng = np.random.default_rng(9000 + seed)
+        E = rng.standard_normal(S.shape)
+        Sp = S * (1.0 + U21 * (E + E.T) / np.sqrt(2.0))
+        Up = U * (1.0 + U21 * rng.standard_normal(U.shape))
+        Qp, lp = O.subspace_step(Sp, Up, eps)
+        if big.any():
+            band_lam = max(band_lam, float(np.max(np.abs(lp - lo)[big] / lo[big])))
+        band_root = max(band_root, rel_fro(basis_root(Qp, lo, eps), ref))
+    return band_lam, band_root
+
+
+def staged_refresh_check(sh, f, incoming, eps, bjorck_iters, tol, end_to_end=True):
+    """Factor f's last refresh against the oracle, stage by stage, from the
+    library's own incoming state (``incoming``: the factor as read before the
+    refresh, has_basis set as the library had it).  Needs a handle made with
+    debug=True (the capture of the rectified basis and of Q).
+
+    Stage 1, dequantize + Bjorck: the library's rectified basis against
+    oracle.bjorck(oracle.dequantize(codes)) -- relative Frobenius <= tol
+    (the identity, exactly, on a first refresh).
+    Stage 2, subspace step + QR + Rayleigh quotients, fed the library's own
+    rectified basis: lambda_i (relative, lambda_i > 1e3 eps) and the
+    basis-invariant root Q diag((lambda_o + eps)^-1/4) Q^T (relative
+    Frobenius) each within tol + BAND_FACTOR x the oracle's own spread.
+    Stage 3, requantization: codes and scales bit-exact with the oracle's
+    quantizer applied to the library's Q.
+    Also, not gated: the same lambda and root errors against the oracle's
+    whole fp64 refresh from the incoming codes (fp64 Bjorck), which adds the
+    sensitivity of stage 2 to the TF32 Bjorck's rounding.
+
+    Returns a dict of the raw errors, the bands and the verdicts."""
+    d = incoming.d
+    Ug = sh.debug_rectified(f).cpu().numpy().astype(np.float64)
+    Qg = sh.debug_q(f).cpu().numpy().astype(np.float64)
+    g = gpu_factor(sh, f)
+    rec = {"factor": f, "d": d}
+    # stage 1
+    if incoming.has_basis:
+        U0 = O.dequantize(incoming.codes, incoming.scales, d * d).reshape(d, d).astype(np.float64)
+        Uo = O.bjorck(U0, bjorck_iters)
+        rec["bjorck"] = rel_fro(Ug, Uo)
+        rec["bjorck_ok"] = rec["bjorck"] <= tol
+    else:
+        rec["bjorck"] = float(np.max(np.abs(Ug - np.eye(d))))
+        rec["bjorck_ok"] = rec["bjorck"] == 0.0
+    # stage 2, from the library's rectified basis
+    Qo, lo = O.subspace_step(incoming.S, Ug, eps)
+    lg = g.lam.astype(np.float64)
+    big = lo > 1e3 * eps
+    rec["lam"] = float(np.max(np.abs(lg - lo)[big] / lo[big])) if big.any() else 0.0
+    rec["root"] = rel_fro(basis_root(Qg, lo, eps), basis_root(Qo, lo, eps))
+    rec["band_lam"], rec["band_root"] = _oracle_spread(incoming.S, Ug, eps, Qo, lo, big)
+    rec["lam_ok"] = rec["lam"] <= tol + BAND_FACTOR * rec["band_lam"]
+    rec["root_ok"] = rec["root"] <= tol + BAND_FACTOR * rec["band_root"]
+    rec["banded"] = bool(BAND_FACTOR * max(rec["band_lam"], rec["band_root"]) > tol)
+    rec["orth"] = float(np.linalg.norm(Qg.T @ Qg - np.eye(d)) / np.sqrt(d))
+    # stage 3
+    oc, os_ = O.quantize(Qg.astype(np.float32).ravel())
+    rec["codes_ok"] = bool(np.array_equal(g.codes, oc) and np.array_equal(g.scales, os_))
+    if end_to_end:
+        e = O.Factor(d, incoming.S, codes=incoming.codes, scales=incoming.scales, lam=incoming.lam,
+                     has_basis=incoming.has_basis)
+        O.refresh_factor(e, eps, bjorck_iters)
+        le = e.lam.astype(np.float64)
+        bige = le > 1e3 * eps
+        rec["e2e_lam"] = float(np.max(np.abs(lg - le)[bige] / le[bige])) if bige.any() else 0.0
+        rec["e2e_root"] = rel_fro(basis_root(Qg, le, eps), basis_root(e.q_last, le, eps))
+    rec["ok"] = bool(rec["bjorck_ok"] and rec["lam_ok"] and rec["root_ok"] and rec["codes_ok"])
+    return rec
+
+
+def format_record(tag, r):
+    s = (f"{tag} factor {r['factor']} d={r['d']}: bjorck {r['bjorck']:.2e} lambda {r['lam']:.2e} "
+         f"(band {r['band_lam']:.2e}) root {r['root']:.2e} (band {r['band_root']:.2e}) orth {r['orth']:.2e}")
+    if "e2e_lam" in r:
+        s += f" | whole fp64 refresh: lambda {r['e2e_lam']:.2e} root {r['e2e_root']:.2e}"
+    return s + ("" if r["ok"] else "  FAIL")
+
+
+def staged_refresh_all(sh, incoming, eps, bjorck_iters, tol, tag, end_to_end=True):
+    """staged_refresh_check over the factors in ``incoming`` (factor index ->
+    incoming Factor, has_basis set); prints one line per factor and how many
+    needed the band, and asserts every verdict.  Returns the records."""
+    recs = []
+    for f in sorted(incoming):
+        r = staged_refresh_check(sh, f, incoming[f], eps, bjorck_iters, tol, end_to_end)
+        print(format_record(tag, r))
+        recs.append(r)
+    nb = sum(r["banded"] for r in recs)
+    print(f"{tag}: {len(recs)} factors checked, {nb} with BAND_FACTOR x band above the tolerance; "
+          f"worst bjorck {max(r['bjorck'] for r in recs):.2e} lambda {max(r['lam'] for r in recs):.2e} "
+          f"root {max(r['root'] for r in recs):.2e}")
+    bad = [r["factor"] for r in recs if not r["ok"]]
+    assert not bad, f"{tag}: factors {bad} outside the staged refresh gates"
+    return recs

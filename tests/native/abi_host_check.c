@@ -76,6 +76,20 @@ int main(void) {
   CHECK(shampoo4_owner_span(h, 0, &soff, &sbytes) == SHAMPOO4_OK && soff == 0 && sbytes > 0);
   CHECK(shampoo4_owner_span(h, 1, &soff, &sbytes) == SHAMPOO4_ERR_INVALID_ARG);
 
+  /* debug capture: two fp32 d x d matrices per factor, 256-byte aligned,
+     disjoint; a misaligned buffer is refused */
+  size_t dbytes = 0;
+  CHECK(shampoo4_debug_capture_bytes(h, &dbytes) == SHAMPOO4_OK && dbytes % 256 == 0);
+  for (int32_t f = 0; f < nfactors; ++f) {
+    size_t ou = 1, oq = 1;
+    int32_t d;
+    CHECK(shampoo4_factor_layout(h, f, NULL, NULL, NULL, NULL, &d) == SHAMPOO4_OK);
+    CHECK(shampoo4_debug_capture_layout(h, f, &ou, &oq) == SHAMPOO4_OK);
+    CHECK(ou % 256 == 0 && oq % 256 == 0 && ou + 4 * (size_t)d * (size_t)d <= oq);
+    CHECK(oq + 4 * (size_t)d * (size_t)d <= dbytes);
+  }
+  CHECK(shampoo4_debug_capture(h, (void*)(uintptr_t)0x1010) == SHAMPOO4_ERR_INVALID_ARG);
+
   /* calls that need bound buffers are refused before touching a device */
   CHECK(shampoo4_refresh_roots(h, NULL) == SHAMPOO4_ERR_NOT_READY);
   shampoo4_destroy(h);

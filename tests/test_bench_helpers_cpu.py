@@ -49,6 +49,7 @@ def test_every_library_stage_has_a_bound():
 
 def test_traffic_is_reported_only_for_the_captured_gemm_source(monkeypatch):
     n = 1 << 20
+    monkeypatch.setattr(bench, "TRAFFIC_SOURCE_SHA", bench.gemm_source_sha())
     assert bench.stage_traffic("qr_gram", n) == pytest.approx(bench.TRAFFIC_PER_ELEMENT["qr_gram"] * n)
     assert bench.stage_traffic("roots", n) is None                    # no capture covers it
     monkeypatch.setattr(bench, "TRAFFIC_SOURCE_SHA", "0" * 16)
@@ -73,3 +74,37 @@ def test_clock_summary_reports_throttle_reasons():
     s = c.summary()
     assert s["sm_mhz"] == 1850.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
     assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
+
+
+def test_step_roofline_follows_the_work_model_by_hand():
+    """The headline fraction can be rebuilt by hand from ms_per_step: one
+    1024 x 1024 tile refreshed every step, TF32 mode.  Statistics 2mn(m+n) =
+    4 d^3, precondition 2(m^3 + n^3) + 2mn(m+n) = 8 d^3, Bjorck 2 x 20 d^3
+    at the TF32 rate; subspace + QR + Rayleigh 2 x (2 + 8/3 + 2) d^3 at a
+    third of it."""
+    d = 1024.0
+    single, triple = bench.step_work([(1024, 1024)], 5, 1, "tf32")
+    assert single == pytest.approx((4 + 8 + 40) * d ** 3)
+    assert triple == pytest.approx(2 * (2 + 8 / 3 + 2) * d ** 3)
+    tf32 = 1400.0 * 1.1 / 2.25 * 1e12
+    ideal = single / tf32 + triple / (tf32 / 3)
+    r = bench.formula_roofline((single, triple), 0.010, _pk(), "measured", "step")
+    assert r["frac"] == pytest.approx(ideal / 0.010)
+    assert r["achieved"] == pytest.approx((single + triple) / 0.010 / 1e12)
+    assert r["achieved"] / r["peak"] == pytest.approx(r["frac"])
+    # a refresh interval T amortizes only the refresh terms
+    s10, t10 = bench.step_work([(1024, 1024)], 5, 10, "tf32")
+    assert s10 == pytest.approx((12 + 4) * d ** 3) and t10 == pytest.approx(triple / 10)
+    # FP32 mode: every product at the 3xTF32 rate
+    s32, t32 = bench.step_work([(1024, 1024)], 5, 1, "fp32")
+    assert s32 == 0 and t32 == pytest.approx(single + triple)
+
+
+def test_cpu_sample_takes_every_ragged_tile_then_seeded_full_ones():
+    w = bench.workload_shapes(5)
+    blocks, sample = bench.cpu_tile_sample(w, 48)
+    ragged = [k for k, b in enumerate(blocks) if b.m < 1024 or b.n < 1024]
+    assert len(blocks) == 480 and len(ragged) == 32 and len(sample) == 48
+    assert set(ragged) <= set(sample)
+    assert sample == sorted(set(sample))
+    assert bench.cpu_tile_sample(w, 48)[1] == sample              # seeded

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 from oracle import shampoo4_oracle as O
-from gpu_helpers import basis_root, cuda_f32, gpu_factor, oracle_from_gpu, rel_fro
+from gpu_helpers import cuda_f32, gpu_factor, oracle_from_gpu, rel_fro, staged_refresh_all
 
 pytestmark = pytest.mark.gpu
 
@@ -64,18 +64,24 @@ def test_update_stats(which, precision):
 @pytest.mark.parametrize("precision", ["tf32", "fp32"])
 @pytest.mark.parametrize("which", list(SHAPE_SETS))
 def test_refresh_and_precondition(which, precision):
+    """Every factor's refresh, stage by stage from the library's incoming
+    state (gpu_helpers.staged_refresh_check): Bjorck, then the subspace
+    step / QR / Rayleigh quotients fed the library's rectified basis, then
+    the requantized codes; then the preconditioned update from the library's
+    refreshed state."""
     shapes = SHAPE_SETS[which]
-    sh = _mk(shapes, precision)
+    sh = _mk(shapes, precision, debug=True)
     eps = float(np.float32(1e-6))
-    report = []
     for rnd in range(2):                       # first refresh (U = I), then a warm one
         for step in range(2):
             gs = _grads(shapes, 200 if which in FIXED_GRADIENT else 200 + 10 * rnd + step,
                         GRAD_SCALE.get(which, 1.0))
             sh.update_stats([cuda_f32(g) for g in gs])
         torch.cuda.synchronize()
-        orc = oracle_from_gpu(sh, shapes, has_basis=(rnd > 0))
-        orc.refresh_roots()
+        incoming = {}
+        for f in range(sh.nfactors):
+            incoming[f] = gpu_factor(sh, f)
+            incoming[f].has_basis = rnd > 0
         sh.refresh_roots()
         torch.cuda.synchronize()
         flags = sh.status_flags()
@@ -84,43 +90,8 @@ def test_refresh_and_precondition(which, precision):
         # fp64 redo, which is reported but is not an error
         allowed = 0x10 if which == "ragged" else 0
         assert flags & ~allowed == 0, flags
-        for f in range(sh.nfactors):
-            d = orc.factors[f].d
-            Qg = sh.debug_q(f).cpu().numpy().astype(np.float64)
-            g = gpu_factor(sh, f)
-            # (i) requantized codes: bit-exact with the oracle quantizer on the GPU's Q
-            oc, os_ = O.quantize(Qg.astype(np.float32).ravel())
-            assert np.array_equal(g.codes, oc) and np.array_equal(g.scales, os_)
-            # (ii) orthonormality of the GPU's Q
-            orth = np.linalg.norm(Qg.T @ Qg - np.eye(d)) / np.sqrt(d)
-            assert orth <= 1e-5, orth
-            # (iii) eigenvalues and (iv) basis-invariant root against the oracle
-            Qo, lo = orc.factors[f].q_last, orc.factors[f].lam.astype(np.float64)
-            lg = g.lam.astype(np.float64)
-            # lambda_i = q_i^T S q_i comes from an fp32-accurate product S Q
-            # (3xTF32: each product carries a relative error of about
-            # u = 2^-21), so its error is absolute, about u * lambda_max, on
-            # top of the stage tolerance: the excess over that bound is
-            # reported relative to lambda_i.
-            big = lo > 1e3 * eps
-            slack = 16 * 2.0 ** -21 * lo.max()
-            excess = np.maximum(np.abs(lg - lo) - slack, 0.0)
-            lam_err = np.max(excess[big] / lo[big]) if big.any() else 0.0
-            # The basis-invariant root is only determined to the arithmetic's
-            # resolution: the subspace product carries an absolute error of
-            # about u * lambda_max per column (u = 2^-21 for the fp32-accurate
-            # products), so the eigen-directions of the smallest eigenvalues,
-            # which dominate the root, move by about u * kappa(S + eps I).
-            # The excess over that is what is held to the stage tolerance;
-            # beyond u32 * kappa >= 1 (rank-deficient statistics with a large
-            # lambda_max / eps) nothing is pinned and the root is compared
-            # only through the preconditioned update below.
-            kappa = (lo.max() + eps) / (lo.min() + eps)
-            root_err = rel_fro(basis_root(Qg, lo, eps), basis_root(Qo, lo, eps))
-            root_err = max(root_err - 2.0 ** -21 * kappa, 0.0)
-            if 6e-8 * kappa >= 1.0:
-                root_err = 0.0
-            report.append((rnd, f, d, orth, lam_err, root_err, kappa))
+        recs = staged_refresh_all(sh, incoming, eps, 5, TOL[precision], f"refresh {which} {precision} round {rnd}")
+        assert max(r["orth"] for r in recs) <= 1e-5
         # precondition with the GPU's state injected into the oracle
         orc2 = oracle_from_gpu(sh, shapes, has_basis=True)
         gs = _grads(shapes, 300 + rnd)
@@ -129,14 +100,8 @@ def test_refresh_and_precondition(which, precision):
         want = orc2.precondition(gs)
         for o, w in zip(out, want):
             e = rel_fro(o.cpu().numpy(), w)
-            report.append((rnd, "D", w.shape, e))
+            print(f"refresh {which} {precision} round {rnd}: update {w.shape} {e:.2e}")
             assert e <= TOL[precision], e
-    for r in report:
-        print("refresh", which, precision, r)
-    worst_lam = max(r[4] for r in report if len(r) == 7)
-    worst_root = max(r[5] for r in report if len(r) == 7)
-    print(f"refresh {which} {precision}: worst lambda {worst_lam:.3e} root {worst_root:.3e}")
-    assert worst_lam <= TOL[precision] and worst_root <= TOL[precision]
 
 
 def test_precondition_before_refresh_is_not_ready():

@@ -2,16 +2,17 @@
 distributions: one 128x128 weight; one 1024x1024 layer with a fixed rank-16
 term; the 53 ResNet-50 convolutions with Student-t gradients; a 12-block
 d = 768 transformer stack.  Two steps (a cold refresh, then a warm one):
-every factor's Q is checked for orthonormality on the GPU, sampled factors
-against the oracle's refresh from the same incoming state, sampled tiles of
-the preconditioned update against the oracle from the library's state.
+every factor's Q is checked for orthonormality on the GPU, sampled factors'
+refreshes stage by stage against the oracle from the same incoming state
+(gpu_helpers.staged_refresh_check), sampled tiles of the preconditioned
+update against the oracle from the library's state.
 Collected last: the longest GPU tests."""
 import numpy as np
 import pytest
 import torch
 
 from oracle import shampoo4_oracle as O
-from gpu_helpers import basis_root, gpu_factor, rel_fro
+from gpu_helpers import gpu_factor, rel_fro, staged_refresh_all
 
 pytestmark = pytest.mark.gpu
 
@@ -44,7 +45,7 @@ def test_workload_sampled(wid):
     w = WORKLOADS[wid]
     shapes = list(w.shapes)
     sh = api.Shampoo4(shapes, beta=w.beta, eps=w.eps, max_block=w.max_block, bjorck_iters=w.bjorck_iters,
-                      precision="tf32")
+                      precision="tf32", debug=True)
     eps = float(np.float32(w.eps))
     g_host = {s: [gradient(w, i, s) for i in range(len(shapes))] for s in (1, 2, 3)}
     dev = lambda s: [torch.from_numpy(g).cuda() for g in g_host[s]]
@@ -71,22 +72,8 @@ def test_workload_sampled(wid):
     assert worst <= 1e-5
 
     for f in picks:
-        fac = before[f]
-        fac.has_basis = True
-        O.refresh_factor(fac, eps, w.bjorck_iters)
-        g = gpu_factor(sh, f)
-        Qg = sh.debug_q(f).cpu().numpy().astype(np.float64)
-        oc, os_ = O.quantize(Qg.astype(np.float32).ravel())
-        assert np.array_equal(g.codes, oc) and np.array_equal(g.scales, os_), f
-        lo, lg = fac.lam.astype(np.float64), g.lam.astype(np.float64)
-        big = lo > 1e3 * eps
-        slack = 16 * 2.0 ** -21 * lo.max()
-        lam_err = np.max(np.maximum(np.abs(lg - lo) - slack, 0.0)[big] / lo[big]) if big.any() else 0.0
-        kappa = (lo.max() + eps) / (lo.min() + eps)
-        root_err = rel_fro(basis_root(Qg, lo, eps), basis_root(fac.q_last, lo, eps))
-        root_err = max(root_err - 2.0 ** -21 * kappa, 0.0) if 6e-8 * kappa < 1.0 else 0.0
-        print(f"workload {wid} factor {f} d={fac.d}: lambda {lam_err:.2e} root {root_err:.2e} kappa {kappa:.2e}")
-        assert lam_err <= TOL_TF32 and root_err <= TOL_TF32, f
+        before[f].has_basis = True
+    staged_refresh_all(sh, before, eps, w.bjorck_iters, TOL_TF32, f"workload {wid}")
 
     out = sh.precondition(dev(3))
     torch.cuda.synchronize()

@@ -79,6 +79,33 @@ def test_noalloc_nonfinite_gradient_leaves_state():
     assert not torch.equal(L, L1)
 
 
+@pytest.mark.gpu
+def test_noalloc_calls_allocate_no_device_memory():
+    """The point of the entry point: after a first call has loaded the
+    module, further calls -- other shapes included -- leave the device's free
+    memory and torch's allocator exactly where they were."""
+    import torch
+    from bit_quantized_shampoo_b200 import api
+
+    bufs = {}
+    for m, n in ((64, 96), (512, 512), (1024, 256), (300, 17)):
+        g = torch.from_numpy(_grads((m, n), 90 + m)[0]).cuda()
+        bufs[(m, n)] = (torch.zeros(m, m, device="cuda"), torch.zeros(n, n, device="cuda"), g)
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L, R, G = bufs[(64, 96)]
+    api.update_stats_noalloc(L, R, G, 0.9, flags=flags)          # warm-up: module load
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    alloc0 = torch.cuda.memory_stats().get("allocated_bytes.all.current", 0)
+    for _ in range(3):
+        for L, R, G in bufs.values():
+            api.update_stats_noalloc(L, R, G, 0.9, flags=flags)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_stats().get("allocated_bytes.all.current", 0) == alloc0
+    assert int(flags.item()) == 0
+
+
 def test_noalloc_rejects_before_touching_the_device():
     """Size and argument checks return before any CUDA call, so they run
     without a GPU; the pointers are never dereferenced."""
