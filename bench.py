@@ -70,6 +70,8 @@ def parse():
                          "default sharded refresh, where each rank refreshes 1/N of the factors (by cost) and "
                          "the ranks exchange codes, scales and eigenvalues (one NCCL broadcast per rank)")
     ap.add_argument("--no-configs", action="store_true", help="skip timing the four smaller workloads")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip timing the codebook and root-method variants on the transformer layer stack")
     ap.add_argument("--cpu-tiles", type=int, default=48,
                     help="tiles of the CPU baseline's sample: every ragged tile, then seeded full ones")
     ap.add_argument("--shapes", default=None, help="comma-separated RxC list replacing the workload's shapes")
@@ -154,6 +156,7 @@ STAGE_BOUND = {
     "qr_potrf": "latency", "qr_inverse": "latency", "rayleigh": "hbm", "requant": "hbm", "precond_dequant": "hbm",
     "basis": "hbm", "stats_scan": "hbm", "refresh_scan": "hbm", "qr_convert": "hbm", "precond_mu": "hbm",
     "stats_dequant": "hbm", "stats_rebuild": "tf32", "tables": "latency",
+    "newton_elt": "hbm", "newton_gemm": "3xtf32",
 }
 
 
@@ -428,6 +431,47 @@ def measure_config(wid, dev, args, pk, pk_src, world):
            "roofline": formula_roofline(step_work(dims, w.bjorck_iters, T, args.precision), ms / 1e3, pk, pk_src,
                                         f"step at T = {T}, algorithmic flops of the work model"),
            "workspace_bytes": sh.workspace_bytes, "state_bytes": sh.state_bytes}
+    del sh, sets, out
+    return res
+
+
+def measure_variant(wid, dev, args, pk, pk_src, world, **kw):
+    """Step (refresh every step) and refresh-call times of one handle variant
+    (codebook, root method) on a workload; CUDA events on the launching
+    stream, max over ranks."""
+    import torch
+    from bit_quantized_shampoo_b200 import api
+    from bit_quantized_shampoo_b200.workloads import WORKLOADS, gradient
+    w = WORKLOADS[wid]
+    shapes = list(w.shapes)
+    sh = api.Shampoo4(shapes, beta=w.beta, eps=w.eps, max_block=w.max_block, bjorck_iters=w.bjorck_iters,
+                      precision=args.precision, device=dev, **kw)
+    sets = [[torch.from_numpy(gradient(w, i, 1 + s)).to(dev) for i in range(len(shapes))] for s in range(2)]
+    out = [torch.empty(s, dtype=torch.float32, device=dev) for s in shapes]
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        sh.update_stats(sets[i % 2])
+        sh.refresh_roots()
+        sh.precondition(sets[i % 2], out=out)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    reps = 5
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    ev[0].record(stream)
+    for i in range(reps):
+        step(i)
+    ev[1].record(stream)
+    for _ in range(reps):
+        sh.refresh_roots()
+    ev[2].record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(ev[0].elapsed_time(ev[1]), dev) / reps
+    rms = max_over_ranks(ev[1].elapsed_time(ev[2]), dev) / reps
+    res = {"ms_per_step": ms, "refresh_ms": rms, "root_refreshes_per_s": world * sh.nfactors * 1e3 / rms,
+           "state_bytes": sh.state_bytes, "status_flags": sh.status_flags()}
     del sh, sets, out
     return res
 
@@ -728,6 +772,16 @@ def main():
         line["configs"] = {}
         for wid in (1, 2, 3, 4):
             line["configs"][f"c{wid}"] = measure_config(wid, dev, args, pk, pk_src, world)
+            torch.cuda.empty_cache()
+
+    # the alternatives the 4-bit Shampoo abstract compares against, on the
+    # transformer layer stack with a refresh every step
+    if not args.no_variants and args.shapes is None and args.workload == 5:
+        torch.cuda.empty_cache()
+        line["variants"] = {"workload": "transformer stack, 12 blocks of d=768, refresh every step"}
+        for name, kw in (("eigen_linear_square", {}), ("eigen_dynamic_tree", {"codebook": "dynamic_tree"}),
+                         ("newton_fp32_root", {"root": "newton"}), ("newton_4bit_root", {"root": "newton_q4"})):
+            line["variants"][name] = measure_variant(4, dev, args, pk, pk_src, world, **kw)
             torch.cuda.empty_cache()
 
     if rank == 0 and world == 1 and not args.no_cpu:

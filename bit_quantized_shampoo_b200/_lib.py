@@ -30,12 +30,18 @@ GRAFT_SGD = 0
 GRAFT_ADAM = 1
 PREC_TF32 = 0
 PREC_FP32 = 1
+CODEBOOK_LINEAR_SQUARE = 0
+CODEBOOK_DYNAMIC_TREE = 1
+ROOT_EIGEN = 0
+ROOT_NEWTON = 1
+ROOT_NEWTON_Q4 = 2
 
 
 class Config(C.Structure):
     _fields_ = [("beta", C.c_float), ("eps", C.c_float), ("max_block", C.c_int32),
                 ("quant_block", C.c_int32), ("bjorck_iters", C.c_int32), ("precision", C.c_int32),
-                ("compressed_stats", C.c_int32), ("refresh_rank", C.c_int32), ("refresh_world", C.c_int32)]
+                ("compressed_stats", C.c_int32), ("refresh_rank", C.c_int32), ("refresh_world", C.c_int32),
+                ("codebook", C.c_int32), ("root_method", C.c_int32), ("newton_iters", C.c_int32)]
 
 
 class GraftConfig(C.Structure):
@@ -79,6 +85,12 @@ _SIGS = {
     "quant4_unpack": [C.POINTER(C.c_void_p), C.POINTER(C.c_void_p), c_i64_p, C.c_int32,
                       C.POINTER(C.c_void_p), C.c_void_p],
     "quant4_tables": [c_f32_p, c_f32_p],
+    "quant4_pack_ex": [C.POINTER(C.c_void_p), c_i64_p, C.c_int32, C.POINTER(C.c_void_p),
+                       C.POINTER(C.c_void_p), C.c_int32, C.c_void_p],
+    "quant4_unpack_ex": [C.POINTER(C.c_void_p), C.POINTER(C.c_void_p), c_i64_p, C.c_int32,
+                         C.POINTER(C.c_void_p), C.c_int32, C.c_void_p],
+    "quant4_tables_ex": [C.c_int32, c_f32_p, c_f32_p],
+    "shampoo4_root_offset": [C.c_void_p, C.c_int32, c_size_p],
     "shampoo4_update_stats_noalloc": [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_int32, C.c_int64,
                                       C.c_float, C.c_void_p, C.c_void_p],
     "shampoo4_graft_state_bytes": [C.c_void_p, C.c_int32, c_size_p],

@@ -34,13 +34,18 @@ class Shampoo4:
 
     def __init__(self, shapes, beta=0.95, eps=1e-6, max_block=1024, bjorck_iters=5,
                  precision="tf32", device=None, reset=True, compressed=False, refresh_rank=0, refresh_world=1,
-                 debug=False):
+                 debug=False, codebook="linear_square", root="eigen", newton_iters=0):
         self.shapes = [(int(r), int(c)) for r, c in shapes]
         self.compressed = bool(compressed)
         self.refresh_rank, self.refresh_world = int(refresh_rank), int(refresh_world)
+        self.codebook = _codebook(codebook)
+        roots = {"eigen": L.ROOT_EIGEN, "newton": L.ROOT_NEWTON, "newton_q4": L.ROOT_NEWTON_Q4}
+        if root not in roots:
+            raise ValueError(f"root must be one of {sorted(roots)}")
+        self.root_method = roots[root]
         cfg = L.Config(beta, eps, max_block, 64, bjorck_iters,
                        L.PREC_FP32 if precision == "fp32" else L.PREC_TF32, 1 if compressed else 0,
-                       self.refresh_rank, self.refresh_world)
+                       self.refresh_rank, self.refresh_world, self.codebook, self.root_method, int(newton_iters))
         params = (L.Param * len(self.shapes))(*[L.Param(r, c) for r, c in self.shapes])
         h = C.c_void_p()
         L.call("shampoo4_init", C.byref(cfg), params, len(self.shapes), C.byref(h))
@@ -182,6 +187,14 @@ class Shampoo4:
         lam = st[ol.value:ol.value + 4 * d].view(torch.float32)
         return S, codes, scales, lam
 
+    def root_view(self, f):
+        """Root method "newton": the factor's fp32 root P from the last
+        refresh, as a view into the state buffer."""
+        off = C.c_size_t()
+        L.call("shampoo4_root_offset", self._h, f, C.byref(off))
+        d = self._dim(f)
+        return self.state[off.value:off.value + 4 * d * d].view(torch.float32).view(d, d)
+
     def _dim(self, f):
         d = C.c_int32()
         L.call("shampoo4_factor_layout", self._h, f, None, None, None, None, C.byref(d))
@@ -240,7 +253,14 @@ def _graft_kind(kind):
     return kinds[kind]
 
 
-def quant4_pack(xs, codes=None, scales=None, stream=None):
+def _codebook(codebook):
+    books = {"linear_square": L.CODEBOOK_LINEAR_SQUARE, "dynamic_tree": L.CODEBOOK_DYNAMIC_TREE}
+    if codebook not in books:
+        raise ValueError(f"codebook must be one of {sorted(books)}")
+    return books[codebook]
+
+
+def quant4_pack(xs, codes=None, scales=None, stream=None, codebook="linear_square"):
     """Quantize a list of fp32 CUDA tensors (flattened)."""
     xs = [x.contiguous() for x in xs]
     ns = [x.numel() for x in xs]
@@ -250,18 +270,18 @@ def quant4_pack(xs, codes=None, scales=None, stream=None):
         codes = [torch.empty((n + 1) // 2, dtype=torch.uint8, device=x.device) for x, n in zip(xs, ns)]
     if scales is None:
         scales = [torch.empty((n + 63) // 64, dtype=torch.float32, device=x.device) for x, n in zip(xs, ns)]
-    L.call("quant4_pack", L.ptr_array([x.data_ptr() for x in xs]), L.i64_array(ns), len(xs),
+    L.call("quant4_pack_ex", L.ptr_array([x.data_ptr() for x in xs]), L.i64_array(ns), len(xs),
            L.ptr_array([c.data_ptr() for c in codes]), L.ptr_array([s.data_ptr() for s in scales]),
-           _stream(stream))
+           _codebook(codebook), _stream(stream))
     return codes, scales
 
 
-def quant4_unpack(codes, scales, ns, out=None, stream=None):
+def quant4_unpack(codes, scales, ns, out=None, stream=None, codebook="linear_square"):
     if out is None:
         out = [torch.empty(n, dtype=torch.float32, device=c.device) for c, n in zip(codes, ns)]
-    L.call("quant4_unpack", L.ptr_array([c.data_ptr() for c in codes]),
+    L.call("quant4_unpack_ex", L.ptr_array([c.data_ptr() for c in codes]),
            L.ptr_array([s.data_ptr() for s in scales]), L.i64_array(ns), len(codes),
-           L.ptr_array([o.data_ptr() for o in out]), _stream(stream))
+           L.ptr_array([o.data_ptr() for o in out]), _codebook(codebook), _stream(stream))
     return out
 
 
@@ -284,8 +304,8 @@ def update_stats_noalloc(L_, R_, G, beta, flags=None, stream=None):
            C.c_void_p(G.data_ptr()), m, n, ldg, float(beta), fp, _stream(stream))
 
 
-def quant4_tables():
+def quant4_tables(codebook="linear_square"):
     cb = (C.c_float * 16)()
     th = (C.c_float * 15)()
-    L.call("quant4_tables", cb, th)
+    L.call("quant4_tables_ex", _codebook(codebook), cb, th)
     return list(cb), list(th)

@@ -19,16 +19,39 @@
 
 namespace s4 {
 
-// ---- linear square codebook ("4-bit Shampoo ...", abstract) -------------
-// Level j is sgn(y) y^2 for y = (2j - 15)/15, evaluated in double as
-// ((2j-15)|2j-15|) / 225; threshold k is the fp32 rounding of the double
-// midpoint of levels k and k+1.  Everything is a compile-time constant.
-__host__ __device__ constexpr double level_f64(int j) {
-  return double((2 * j - 15) * ((2 * j - 15) < 0 ? -(2 * j - 15) : (2 * j - 15))) / 225.0;
+// ---- 4-bit codebooks -------------------------------------------------------
+// kCodebookLinearSquare ("4-bit Shampoo ...", abstract: linear square
+// quantization): level j is sgn(y) y^2 for y = (2j - 15)/15, evaluated in
+// double as ((2j-15)|2j-15|) / 225.
+// kCodebookDynamicTree (the abstract's alternative, read as Dettmers' 2016
+// dynamic tree data type restricted to 4 bits): a sign, then in the three
+// remaining bits a run of E zeros (the decimal exponent), an indicator 1 and
+// k = 2 - E fraction bits i, magnitude 10^-E (0.1 + 0.9 (i + 1) / 2^k); the
+// pattern 000 is zero.  In the 16-level order (ascending) the three bits p
+// of level 8 + p hold +magnitude(p) and level 7 - p holds -magnitude(p), so
+// levels 7 and 8 are both zero.  Evaluated in double as the integer ratio
+// (2^k + 9 (i + 1)) / (10^(E+1) 2^k).
+// Threshold k of either codebook is the fp32 rounding of the double
+// midpoint of levels k and k+1.
+enum { kCodebookLinearSquare = 0, kCodebookDynamicTree = 1, kCodebookCount = 2 };
+
+__host__ __device__ constexpr double dyn_tree_magnitude(int p) {
+  if (p == 0) return 0.0;
+  const int e = p >= 4 ? 0 : (p >= 2 ? 1 : 2);       // zeros before the indicator bit
+  const int k = 2 - e;                                // fraction bits after it
+  const int i = p & ((1 << k) - 1);
+  double den = double(1 << k) * 10.0;
+  for (int q = 0; q < e; ++q) den *= 10.0;
+  return double((1 << k) + 9 * (i + 1)) / den;
 }
-__host__ __device__ constexpr float level_f32(int j) { return float(level_f64(j)); }
-__host__ __device__ constexpr float threshold_f32(int k) {
-  return float((level_f64(k) + level_f64(k + 1)) / 2.0);
+__host__ __device__ constexpr double level_f64(int cb, int j) {
+  return cb == kCodebookDynamicTree
+             ? (j >= 8 ? dyn_tree_magnitude(j - 8) : -dyn_tree_magnitude(7 - j))
+             : double((2 * j - 15) * ((2 * j - 15) < 0 ? -(2 * j - 15) : (2 * j - 15))) / 225.0;
+}
+__host__ __device__ constexpr float level_f32(int cb, int j) { return float(level_f64(cb, j)); }
+__host__ __device__ constexpr float threshold_f32(int cb, int k) {
+  return float((level_f64(cb, k) + level_f64(cb, k + 1)) / 2.0);
 }
 
 constexpr int kQuantBlock = 64;

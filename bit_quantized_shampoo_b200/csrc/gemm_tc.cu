@@ -63,8 +63,32 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait with an explicit bound on how long the hardware may suspend the
+// thread inside the instruction (its suspendTimeHint, in ns).
+__device__ __forceinline__ bool mbar_try_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait: false after about limit_ns without the phase completing.
+// try_wait may suspend the thread until the phase completes, so a limit
+// below the 2 s default (a diagnostic) is also passed as the suspend hint:
+// otherwise a short wait would simply be absorbed inside the instruction.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitNs) {
+  if (limit_ns < kWaitNs) {
+    const uint32_t hint = limit_ns < 1000000ull ? uint32_t(limit_ns) : 1000000u;
+    const uint64_t t0 = now_ns();
+    for (;;) {
+      if (mbar_try_hint(bar, parity, hint)) return true;
+      if (now_ns() - t0 > limit_ns) return false;
+    }
+  }
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = now_ns();
   for (;;) {

@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(256) k_basis(const BasisDesc* __restrict__ des
   const int d = g.d, r = blockIdx.x;
   if (r >= d) return;                                      // CTA-uniform
   __shared__ float level[16];
-  if (threadIdx.x < 16) level[threadIdx.x] = level_f32(threadIdx.x);
+  if (threadIdx.x < 16) level[threadIdx.x] = level_f32(g.codebook, threadIdx.x);
   __syncthreads();
   const int c0 = threadIdx.x * 4;
   if (c0 >= d) return;
@@ -697,6 +697,84 @@ shampoo4_status launch_copy(const CopyDesc* d_desc, int count, int64_t max_elems
   const int chunks = int((max_elems + kConvertChunk - 1) / kConvertChunk);
   const int64_t items = int64_t(count) * chunks;
   k_copy<<<unsigned(items < kWorkCtas ? items : kWorkCtas), 256, 0, st>>>(d_desc, count, chunks);
+  S4_CUDA(cudaGetLastError());
+  return SHAMPOO4_OK;
+}
+
+// ---- coupled Newton inverse fourth root: norm and elementwise steps ---------
+__global__ void __launch_bounds__(512) k_newton_norm(const NewtonNormDesc* __restrict__ descs) {
+  const NewtonNormDesc& g = descs[blockIdx.x];
+  if (g.skip && *g.skip) return;
+  const int d = g.d;
+  const int64_t n = int64_t(d) * d;
+  double t = 0.0;
+  for (int64_t e = threadIdx.x; e < n; e += blockDim.x) {
+    const int64_t r = e / d, c = e - r * d;
+    const double a = double(g.S[e]) + (r == c ? double(g.eps) : 0.0);
+    t = fma(a, a, t);
+  }
+  __shared__ double part[512];
+  part[threadIdx.x] = t;
+  __syncthreads();
+  for (int w = 256; w > 0; w >>= 1) {
+    if (int(threadIdx.x) < w) part[threadIdx.x] += part[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double c = sqrt(part[0]);
+    g.sc[0] = float(1.0 / c);
+    g.sc[1] = float(1.0 / sqrt(sqrt(c)));
+  }
+}
+
+shampoo4_status launch_newton_norm(const NewtonNormDesc* d_desc, int count, cudaStream_t st) {
+  if (count <= 0) return SHAMPOO4_OK;
+  k_newton_norm<<<count, 512, 0, st>>>(d_desc);
+  S4_CUDA(cudaGetLastError());
+  return SHAMPOO4_OK;
+}
+
+__global__ void __launch_bounds__(256) k_newton_elt(const NewtonEltDesc* __restrict__ descs, int count, int chunks) {
+  for (int w = blockIdx.x; w < count * chunks; w += gridDim.x) {
+    const NewtonEltDesc& g = descs[w / chunks];
+    const int d = g.d;
+    const int64_t n = int64_t(d) * d;
+    const int64_t lo = int64_t(w % chunks) * kConvertChunk;
+    if (lo >= n || (g.skip && *g.skip)) continue;
+    const int64_t hi = lo + kConvertChunk < n ? lo + kConvertChunk : n;
+    const double inv_c = double(g.sc[0]);
+    const float root_c = g.sc[1];
+    for (int64_t e = lo + threadIdx.x; e < hi; e += blockDim.x) {
+      const int64_t r = e / d, c = e - r * d;
+      const bool diag = r == c;
+      if (g.mode == kNewtonFinal) {
+        g.m[e] = g.in[e] * root_c;
+        continue;
+      }
+      float mv;
+      if (g.mode == kNewtonInit) {
+        mv = float((double(g.in[e]) + (diag ? double(g.eps) : 0.0)) * inv_c);
+        g.m[e] = mv;
+        put_split(mv, g.mh, g.ml, e);
+      } else {
+        mv = g.in[e];
+      }
+      const float fv = (diag ? 1.25f : 0.0f) - 0.25f * mv;
+      if (g.f) g.f[e] = fv;
+      put_split(fv, g.fh, g.fl, e);
+      if (g.x) {
+        g.x[e] = fv;
+        put_split(fv, g.xh, g.xl, e);
+      }
+    }
+  }
+}
+
+shampoo4_status launch_newton_elt(const NewtonEltDesc* d_desc, int count, int64_t max_elems, cudaStream_t st) {
+  if (count <= 0 || max_elems <= 0) return SHAMPOO4_OK;
+  const int chunks = int((max_elems + kConvertChunk - 1) / kConvertChunk);
+  const int64_t items = int64_t(count) * chunks;
+  k_newton_elt<<<unsigned(items < kWorkCtas ? items : kWorkCtas), 256, 0, st>>>(d_desc, count, chunks);
   S4_CUDA(cudaGetLastError());
   return SHAMPOO4_OK;
 }

@@ -91,6 +91,7 @@ struct BasisDesc {
   float* Vh; float* Vl;
   int32_t d;
   int32_t identity;
+  int32_t codebook;
 };
 
 // lambda_i = max(sum_r Q[r,i] T[r,i], 0), T = S Q; written only if *skip==0.
@@ -176,6 +177,34 @@ struct ConvertDesc {
   const uint32_t* skip;       // optional
 };
 
+
+// Coupled Newton inverse fourth root ("Shampoo -- Second-Order Optimizer",
+// "Computing the inverse fourth root"), A = S + eps I:
+//   norm:  c = ||A||_F in fp64; sc[0] = 1/c, sc[1] = c^(-1/4) (fp32)
+//   INIT:  M = A / c (fp32 master + TF32 split), F = 1.25 I - 0.25 M
+//          (split), X = F (fp32 + split): the first iteration's X = I F
+//   STEP:  F = 1.25 I - 0.25 M from the fp32 M (split)
+//   FINAL: P = sc[1] X (fp32)
+// Splits are written when the pointers are set; everything is skipped for
+// a factor with *skip != 0.
+struct NewtonNormDesc {
+  const float* S;
+  float* sc;
+  int32_t d; float eps;
+  const uint32_t* skip;
+};
+enum { kNewtonInit = 0, kNewtonStep = 1, kNewtonFinal = 2 };
+struct NewtonEltDesc {
+  const float* in;
+  const float* sc;
+  float* m; float* mh; float* ml;      // INIT: M; FINAL: P (m only)
+  float* f;                            // INIT, STEP: F in fp32 (CUDA-core factors)
+  float* fh; float* fl;                // INIT, STEP: F as a TF32 split (tensor-core factors)
+  float* x; float* xh; float* xl;      // INIT: X = F
+  int32_t d; int32_t mode;
+  float eps; int32_t pad_;
+  const uint32_t* skip;
+};
 
 // dst[0, n) = src[0, n): the debug capture of a refresh's intermediate
 // matrices into a caller buffer.
@@ -316,6 +345,8 @@ shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max
                                const uint32_t* guard = nullptr);
 shampoo4_status launch_gate(const GateDesc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_copy(const CopyDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
+shampoo4_status launch_newton_norm(const NewtonNormDesc* d_desc, int count, cudaStream_t st);
+shampoo4_status launch_newton_elt(const NewtonEltDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_inv128(const Inv128Desc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaStream_t st);
 shampoo4_status launch_rowdiag(const RowDiagDesc* d_desc, int count, int max_d, cudaStream_t st);
@@ -325,8 +356,10 @@ shampoo4_status launch_rowdiag(const RowDiagDesc* d_desc, int count, int max_d, 
 // kernels issued (one per batch of up to 64 non-empty tensors).
 shampoo4_status launch_pack(const float* const* x, const int64_t* n, int32_t count,
                             uint8_t* const* codes, float* const* scales, cudaStream_t st,
-                            const uint32_t* const* skip = nullptr, int* launched = nullptr);
+                            const uint32_t* const* skip = nullptr, int* launched = nullptr,
+                            int codebook = kCodebookLinearSquare);
 shampoo4_status launch_unpack(const uint8_t* const* codes, const float* const* scales,
-                              const int64_t* n, int32_t count, float* const* x, cudaStream_t st);
+                              const int64_t* n, int32_t count, float* const* x, cudaStream_t st,
+                              int codebook = kCodebookLinearSquare);
 
 }  // namespace s4

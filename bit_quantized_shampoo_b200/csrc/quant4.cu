@@ -1,18 +1,22 @@
 // Stand-alone 4-bit codec: quant4_pack / quant4_unpack over batches of fp32
 // tensors ("4-bit Shampoo for Memory-Efficient Network Training", abstract:
-// block-wise linear square quantization).
+// block-wise linear square quantization; the dynamic tree map is the
+// alternative codebook).
 //
-// Memory-bound.  One CTA of 256 threads covers 4096 consecutive elements of
-// one tensor (64 quantization blocks); each thread owns two groups of 8
-// elements (two 32-byte loads in flight), 8 consecutive lanes own one block.
+// Memory-bound.  One CTA of 256 threads covers 16384 consecutive elements of
+// one tensor (256 quantization blocks); each thread owns four groups of 8
+// elements and issues all four groups' loads (128 bytes) before it computes
+// any of them, so that enough reads are in flight to cover DRAM latency
+// while the warp spends its issue slots on the quantization arithmetic.  8
+// consecutive lanes own one block.
 #include "quant4.cuh"
 #include "plan.h"
 
 namespace s4 {
 
 constexpr int kCodecThreads = 256;
-constexpr int kCodecGroupsPerThread = 2;
-constexpr int kCodecEltsPerCta = kCodecThreads * 8 * kCodecGroupsPerThread;   // 4096
+constexpr int kCodecGroupsPerThread = 4;
+constexpr int kCodecEltsPerCta = kCodecThreads * 8 * kCodecGroupsPerThread;   // 16384
 constexpr int kCodecMaxBatch = 64;
 
 struct PackTensor {
@@ -27,6 +31,7 @@ struct PackTensor {
 };
 struct PackBatch {
   int32_t count;
+  int32_t codebook;
   PackTensor t[kCodecMaxBatch];
 };
 
@@ -41,6 +46,7 @@ struct UnpackTensor {
 };
 struct UnpackBatch {
   int32_t count;
+  int32_t codebook;
   UnpackTensor t[kCodecMaxBatch];
 };
 
@@ -54,11 +60,10 @@ __device__ __forceinline__ int find_tensor(const B& b, int64_t cta) {
   return lo;
 }
 
-// Quantize the 8 elements starting at element e0 of tensor t (all lanes of
-// the warp call this together; lanes past the end contribute zeros).
-__device__ __forceinline__ void pack_group(const PackTensor& t, int64_t e0, const float* thr) {
-  float v[8];
-  uint32_t valid = 0;
+// The 8 elements starting at element e0 of tensor t into v (zeros past the
+// end; valid marks the elements that exist).
+__device__ __forceinline__ void load_group(const PackTensor& t, int64_t e0, float (&v)[8], uint32_t& valid) {
+  valid = 0;
   if (t.vec_x && e0 + 8 <= t.n) {
     const float4* p = reinterpret_cast<const float4*>(t.x + e0);
     float4 a = __ldg(p), b = __ldg(p + 1);
@@ -73,6 +78,12 @@ __device__ __forceinline__ void pack_group(const PackTensor& t, int64_t e0, cons
       valid |= ok ? (1u << e) : 0u;
     }
   }
+}
+
+// Quantize one loaded group (all lanes of the warp call this together) and
+// store its codes and, from the block's first lane, its scale.
+__device__ __forceinline__ void pack_group(const PackTensor& t, int64_t e0, const float (&v)[8], uint32_t valid,
+                                           const float* thr) {
   float s;
   uint32_t packed = quantize8(v, valid, thr, &s);
   if ((threadIdx.x & 7) == 0 && e0 < t.n) t.scales[e0 / kQuantBlock] = s;
@@ -91,15 +102,23 @@ __device__ __forceinline__ void pack_group(const PackTensor& t, int64_t e0, cons
 __global__ void __launch_bounds__(kCodecThreads)
 k_quant4_pack(const __grid_constant__ PackBatch b) {
   __shared__ CodecSmem sm;
-  codec_smem_init(sm);
-  __syncthreads();
+  codec_smem_init(sm, b.codebook);
   const PackTensor& t = b.t[find_tensor(b, blockIdx.x)];
-  if (t.skip && *t.skip) return;
-  int64_t e_base = (int64_t(blockIdx.x) - t.cta_begin) * kCodecEltsPerCta;
+  const int64_t e_base = (int64_t(blockIdx.x) - t.cta_begin) * kCodecEltsPerCta;
+  const bool skip = t.skip && *t.skip;
+  float v[kCodecGroupsPerThread][8];
+  uint32_t valid[kCodecGroupsPerThread];
 #pragma unroll
   for (int g = 0; g < kCodecGroupsPerThread; ++g) {
-    int64_t e0 = e_base + (int64_t(g) * kCodecThreads + threadIdx.x) * 8;
-    pack_group(t, e0, sm.thr);
+    const int64_t e0 = e_base + (int64_t(g) * kCodecThreads + threadIdx.x) * 8;
+    load_group(t, skip ? t.n : e0, v[g], valid[g]);
+  }
+  __syncthreads();                                      // the tables
+  if (skip) return;                                     // CTA-uniform
+#pragma unroll
+  for (int g = 0; g < kCodecGroupsPerThread; ++g) {
+    const int64_t e0 = e_base + (int64_t(g) * kCodecThreads + threadIdx.x) * 8;
+    pack_group(t, e0, v[g], valid[g], sm.thr);
   }
 }
 
@@ -134,7 +153,7 @@ __device__ __forceinline__ void unpack_group(const UnpackTensor& t, int64_t e0, 
 __global__ void __launch_bounds__(kCodecThreads)
 k_quant4_unpack(const __grid_constant__ UnpackBatch b) {
   __shared__ CodecSmem sm;
-  codec_smem_init(sm);
+  codec_smem_init(sm, b.codebook);
   __syncthreads();
   const UnpackTensor& t = b.t[find_tensor(b, blockIdx.x)];
   int64_t e_base = (int64_t(blockIdx.x) - t.cta_begin) * kCodecEltsPerCta;
@@ -148,11 +167,13 @@ k_quant4_unpack(const __grid_constant__ UnpackBatch b) {
 // Host launchers, shared with the optimizer's own requantization.
 shampoo4_status launch_pack(const float* const* x, const int64_t* n, int32_t count,
                             uint8_t* const* codes, float* const* scales, cudaStream_t st,
-                            const uint32_t* const* skip, int* launched) {
+                            const uint32_t* const* skip, int* launched, int codebook) {
   if (launched) *launched = 0;
+  if (codebook < 0 || codebook >= kCodebookCount) return SHAMPOO4_ERR_INVALID_ARG;
   for (int32_t base = 0; base < count; base += kCodecMaxBatch) {
     PackBatch b;
     b.count = 0;
+    b.codebook = codebook;
     int64_t ctas = 0;
     for (int32_t i = base; i < count && i < base + kCodecMaxBatch; ++i) {
       if (n[i] == 0) continue;
@@ -174,10 +195,12 @@ shampoo4_status launch_pack(const float* const* x, const int64_t* n, int32_t cou
 }
 
 shampoo4_status launch_unpack(const uint8_t* const* codes, const float* const* scales,
-                              const int64_t* n, int32_t count, float* const* x, cudaStream_t st) {
+                              const int64_t* n, int32_t count, float* const* x, cudaStream_t st, int codebook) {
+  if (codebook < 0 || codebook >= kCodebookCount) return SHAMPOO4_ERR_INVALID_ARG;
   for (int32_t base = 0; base < count; base += kCodecMaxBatch) {
     UnpackBatch b;
     b.count = 0;
+    b.codebook = codebook;
     int64_t ctas = 0;
     for (int32_t i = base; i < count && i < base + kCodecMaxBatch; ++i) {
       if (n[i] == 0) continue;
@@ -213,9 +236,10 @@ static shampoo4_status check_codec_args(const void* const* a, const void* const*
   return SHAMPOO4_OK;
 }
 
-extern "C" shampoo4_status quant4_pack(const float* const* d_x, const int64_t* n, int32_t count,
-                                       uint8_t* const* d_codes, float* const* d_scales,
-                                       shampoo4_stream_t stream) {
+extern "C" shampoo4_status quant4_pack_ex(const float* const* d_x, const int64_t* n, int32_t count,
+                                          uint8_t* const* d_codes, float* const* d_scales, int32_t codebook,
+                                          shampoo4_stream_t stream) {
+  if (codebook < 0 || codebook >= s4::kCodebookCount) return SHAMPOO4_ERR_INVALID_ARG;
   S4_TRY(check_codec_args(reinterpret_cast<const void* const*>(d_x),
                           reinterpret_cast<const void* const*>(d_codes),
                           reinterpret_cast<const void* const*>(d_scales), n, count));
@@ -223,12 +247,14 @@ extern "C" shampoo4_status quant4_pack(const float* const* d_x, const int64_t* n
     if (n[i] > 0 && (!s4::aligned(d_x[i], 4) || !s4::aligned(d_scales[i], 4)))
       return SHAMPOO4_ERR_INVALID_ARG;
   if (count == 0) return SHAMPOO4_OK;
-  return s4::launch_pack(d_x, n, count, d_codes, d_scales, reinterpret_cast<cudaStream_t>(stream));
+  return s4::launch_pack(d_x, n, count, d_codes, d_scales, reinterpret_cast<cudaStream_t>(stream), nullptr,
+                         nullptr, codebook);
 }
 
-extern "C" shampoo4_status quant4_unpack(const uint8_t* const* d_codes, const float* const* d_scales,
-                                         const int64_t* n, int32_t count, float* const* d_x,
-                                         shampoo4_stream_t stream) {
+extern "C" shampoo4_status quant4_unpack_ex(const uint8_t* const* d_codes, const float* const* d_scales,
+                                            const int64_t* n, int32_t count, float* const* d_x, int32_t codebook,
+                                            shampoo4_stream_t stream) {
+  if (codebook < 0 || codebook >= s4::kCodebookCount) return SHAMPOO4_ERR_INVALID_ARG;
   S4_TRY(check_codec_args(reinterpret_cast<const void* const*>(d_codes),
                           reinterpret_cast<const void* const*>(d_scales),
                           reinterpret_cast<const void* const*>(d_x), n, count));
@@ -236,12 +262,28 @@ extern "C" shampoo4_status quant4_unpack(const uint8_t* const* d_codes, const fl
     if (n[i] > 0 && (!s4::aligned(d_x[i], 4) || !s4::aligned(d_scales[i], 4)))
       return SHAMPOO4_ERR_INVALID_ARG;
   if (count == 0) return SHAMPOO4_OK;
-  return s4::launch_unpack(d_codes, d_scales, n, count, d_x, reinterpret_cast<cudaStream_t>(stream));
+  return s4::launch_unpack(d_codes, d_scales, n, count, d_x, reinterpret_cast<cudaStream_t>(stream), codebook);
+}
+
+extern "C" shampoo4_status quant4_pack(const float* const* d_x, const int64_t* n, int32_t count,
+                                       uint8_t* const* d_codes, float* const* d_scales,
+                                       shampoo4_stream_t stream) {
+  return quant4_pack_ex(d_x, n, count, d_codes, d_scales, s4::kCodebookLinearSquare, stream);
+}
+
+extern "C" shampoo4_status quant4_unpack(const uint8_t* const* d_codes, const float* const* d_scales,
+                                         const int64_t* n, int32_t count, float* const* d_x,
+                                         shampoo4_stream_t stream) {
+  return quant4_unpack_ex(d_codes, d_scales, n, count, d_x, s4::kCodebookLinearSquare, stream);
+}
+
+extern "C" shampoo4_status quant4_tables_ex(int32_t codebook, float levels[16], float thresholds[15]) {
+  if (!levels || !thresholds || codebook < 0 || codebook >= s4::kCodebookCount) return SHAMPOO4_ERR_INVALID_ARG;
+  for (int j = 0; j < 16; ++j) levels[j] = s4::level_f32(codebook, j);
+  for (int k = 0; k < 15; ++k) thresholds[k] = s4::threshold_f32(codebook, k);
+  return SHAMPOO4_OK;
 }
 
 extern "C" shampoo4_status quant4_tables(float codebook[16], float thresholds[15]) {
-  if (!codebook || !thresholds) return SHAMPOO4_ERR_INVALID_ARG;
-  for (int j = 0; j < 16; ++j) codebook[j] = s4::level_f32(j);
-  for (int k = 0; k < 15; ++k) thresholds[k] = s4::threshold_f32(k);
-  return SHAMPOO4_OK;
+  return quant4_tables_ex(s4::kCodebookLinearSquare, codebook, thresholds);
 }

@@ -1,6 +1,7 @@
-// Device-side pieces of the block-wise linear square 4-bit codec
-// ("4-bit Shampoo for Memory-Efficient Network Training", abstract: linear
-// square quantization, block-wise, of the eigenvector matrix).
+// Device-side pieces of the block-wise 4-bit codec ("4-bit Shampoo for
+// Memory-Efficient Network Training", abstract: linear square quantization,
+// block-wise, of the eigenvector matrix; the dynamic tree map is the
+// alternative it compares against).
 //
 // Layout: a block is 64 consecutive elements; 8 consecutive lanes of a warp
 // own one block, 8 elements each, so the block's absmax is a 3-step
@@ -10,17 +11,18 @@
 
 namespace s4 {
 
-// Thresholds t_0..t_14 in shared memory (indexed by a per-lane position).
+// Thresholds t_0..t_14 (t_15 = +Inf) and the 16 levels of one codebook, in
+// shared memory.
 struct CodecSmem {
   float thr[16];
   float level[16];
 };
 
-__device__ __forceinline__ void codec_smem_init(CodecSmem& sm) {
+__device__ __forceinline__ void codec_smem_init(CodecSmem& sm, int codebook) {
   if (threadIdx.x < 16) {
     int j = threadIdx.x;
-    sm.level[j] = level_f32(j);
-    sm.thr[j] = j < 15 ? threshold_f32(j) : __int_as_float(0x7f800000);
+    sm.level[j] = level_f32(codebook, j);
+    sm.thr[j] = j < 15 ? threshold_f32(codebook, j) : __int_as_float(0x7f800000);
   }
 }
 
@@ -49,28 +51,30 @@ __device__ __forceinline__ float div_rn_shared(float x, float s, float r) {
   return fmaf(e, r, q0);
 }
 
+// Absmax of the 8 values a lane owns, as the bits of |x| with the sign
+// cleared: as unsigned integers these order NaN above +Inf above every
+// finite magnitude, so one integer max tracks the absmax and whether the
+// block holds a NaN (bits > 0x7f800000) or an infinity (== 0x7f800000).
+__device__ __forceinline__ uint32_t absmax_bits8(const float (&v)[8]) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m = max(m, __float_as_uint(v[e]) & 0x7fffffffu);
+  return m;
+}
+
 // Quantize 8 values owned by this lane; the 8 lanes of the block are the
 // aligned 8-lane segment of the warp that contains this lane.  All 32 lanes
 // of the warp must call it together.  Returns the 8 codes packed as 4 bytes
-// (element 0 in the low nibble of byte 0) and the block scale in *scale.
-// Lanes whose elements lie past the end pass zeros and a valid mask of 0
-// for those elements; their codes are forced to 0.
+// (element 0 in the low nibble of byte 0) and the block scale in *scale:
+// the absmax, NaN (canonical) if the block holds a NaN, +Inf if it holds an
+// infinity and no NaN.  Lanes whose elements lie past the end pass zeros and
+// a valid mask of 0 for those elements; their codes are forced to 0.
 __device__ __forceinline__ uint32_t quantize8(const float (&v)[8], uint32_t valid_mask,
                                               const float* thr, float* scale) {
-  float m = 0.0f;
-  uint32_t has_nan = 0;
+  uint32_t m = absmax_bits8(v);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    float a = fabsf(v[e]);
-    has_nan |= (a != a) ? 1u : 0u;
-    m = fmaxf(m, a);                 // fmaxf ignores NaN; tracked separately
-  }
-#pragma unroll
-  for (int off = 4; off >= 1; off >>= 1) {
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    has_nan |= __shfl_xor_sync(0xffffffffu, has_nan, off);
-  }
-  float s = has_nan ? __int_as_float(0x7fc00000) : m;
+  for (int off = 4; off >= 1; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+  const float s = m > 0x7f800000u ? __int_as_float(0x7fc00000) : __uint_as_float(m);
   *scale = s;
   uint32_t packed = 0;
   if (s == 0.0f) {

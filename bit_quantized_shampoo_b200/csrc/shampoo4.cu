@@ -30,7 +30,7 @@ using namespace s4;
 namespace {
 
 enum class Kind { GemmF32, GemmF64, Potrf, Trsm, Basis, Rayleigh, Mu, Scan, Convert, Pack, Shift, GemmTC, GemmTCSplit,
-                  GemmTCSplit64, PotrfF, ShiftF, Gate, Diag, RowDiag, Inv128, Copy };
+                  GemmTCSplit64, PotrfF, ShiftF, Gate, Diag, RowDiag, Inv128, Copy, NewtonNorm, NewtonElt };
 
 struct Launch {
   Kind kind;
@@ -66,6 +66,7 @@ struct FactorPlan {
   int32_t block, side, d;
   bool tc;
   size_t st_S, st_codes, st_scales, st_lam;
+  size_t st_P;                           // root method NEWTON: the fp32 root in the state
   size_t ws_S;                           // compressed statistics: S lives here
   size_t ws_mu;
   size_t ws_W64, ws_Q64, ws_U, ws_T, ws_Y;
@@ -79,6 +80,7 @@ struct FactorPlan {
 };
 
 constexpr size_t kAlign = 256;
+constexpr int kDefaultNewtonIters = 32;
 constexpr int kPanelW = 64;     // Cholesky panel width (64 x 64 diagonal blocks)
 constexpr int kSolveW = 128;    // solve panel width (128 x 128 inverse blocks)
 
@@ -264,6 +266,7 @@ shampoo4_status plan(shampoo4_ctx* h) {
       f.st_codes = take(st, (dd + 1) / 2);
       f.st_scales = take(st, 4 * ((dd + kQuantBlock - 1) / kQuantBlock));
       f.st_lam = take(st, 4 * size_t(f.d));
+      f.st_P = h->cfg.root_method == SHAMPOO4_ROOT_NEWTON ? take(st, 4 * dd) : SIZE_MAX;
     }
     h->span_bytes[r] = st - h->span_off[r];
   }
@@ -545,6 +548,7 @@ void build_stats_into(Builder& b, std::vector<Launch>& prog, bool rebuild) {
       sum_dd += double(d) * d;
       BasisDesc x{};
       x.codes = b.sb(f.st_codes); x.scales = b.sf(f.st_scales); x.d = d; x.identity = 0;
+      x.codebook = h->cfg.codebook;
       if (f.tc) {
         // V = U diag(sqrt(lambda)) -> X[1] split; S = V V^T.  The same
         // rounded V on both sides keeps S positive semidefinite (up to the
@@ -943,7 +947,214 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
   }
 }
 
+// Refresh by the coupled Newton iteration (root methods NEWTON and
+// NEWTON_Q4; "Shampoo -- Second-Order Optimizer", "Computing the inverse
+// fourth root"): P = (S + eps I)^(-1/4) from the fp32 statistic with
+// matrix products only.  A = S + eps I, c = ||A||_F, M = A / c, X = I; then
+// newton_iters times F = (5 I - M) / 4, X <- X F, M <- F^4 M (F^4 as
+// (F F)(F F)); P = X c^(-1/4).  Every product is fp32-accurate (3xTF32 on
+// the tensor cores, fp32 on the CUDA cores): with TF32 products the
+// iteration drifts off and diverges on condition numbers above about 1e5.
+// The first iteration's X = I F is F itself (written by the INIT step).
+// Buffers (per factor, from the eigen refresh's workspace): X in the two
+// triplets X[0], X[1]; M in Z and (W, Th, Tl); F in (Sh, Sl); F^2 and F^4
+// in the fp64 fallback regions, each as two fp32 d x d arrays.  A factor
+// whose statistic holds NaN/Inf keeps its previous root.
+void build_refresh_newton(Builder& b, std::vector<Launch>& prog) {
+  shampoo4_ctx* h = b.h;
+  const size_t nf = h->factors.size();
+  const int iters = h->cfg.newton_iters;
+  const bool q4 = h->cfg.root_method == SHAMPOO4_ROOT_NEWTON_Q4;
+  int dmax = 0;
+  int64_t emax = 0;
+  double sum_dd = 0;
+  for (auto& f : h->factors) {
+    dmax = std::max(dmax, f.d);
+    emax = std::max<int64_t>(emax, int64_t(f.d) * f.d);
+    sum_dd += double(f.d) * f.d;
+  }
+  {  // non-finite statistic -> keep the previous root
+    std::vector<ScanDesc> scan;
+    for (size_t i = 0; i < nf; ++i) {
+      const FactorPlan& f = h->factors[i];
+      ScanDesc sd{};
+      sd.X = b.S(f); sd.ld = f.d; sd.rows = sd.cols = f.d;
+      sd.ref.tab = -1;
+      sd.flag = b.fail(i);
+      sd.bit = SHAMPOO4_FLAG_NONFINITE_STATE;
+      scan.push_back(sd);
+    }
+    b.tag = SHAMPOO4_STAGE_REFRESH_SCAN;
+    b.emit(prog, Kind::Scan, scan, dmax, 0, 4.0 * sum_dd);
+  }
+  struct Bufs {
+    float *xm[2], *xh[2], *xl[2], *mm[2], *mh[2], *ml[2];
+    float *fm, *fh, *fl, *f2h, *f2l, *f4h, *f4l, *sc;
+  };
+  std::vector<Bufs> nb(nf);
+  for (size_t i = 0; i < nf; ++i) {
+    const FactorPlan& f = h->factors[i];
+    const size_t dd = size_t(f.d) * f.d;
+    Bufs& u = nb[i];
+    std::memset(&u, 0, sizeof(u));
+    u.sc = b.wf(f.ws_mu);
+    float* w64 = reinterpret_cast<float*>(b.wd(f.ws_W64));
+    float* q64 = reinterpret_cast<float*>(b.wd(f.ws_Q64));
+    if (f.tc) {
+      for (int k = 0; k < 2; ++k) {
+        u.xm[k] = b.wf(f.ws_Xm[k]); u.xh[k] = b.wf(f.ws_Xh[k]); u.xl[k] = b.wf(f.ws_Xl[k]);
+      }
+      u.mm[0] = b.wf(f.ws_Zm); u.mh[0] = b.wf(f.ws_Zh); u.ml[0] = b.wf(f.ws_Zl);
+      u.mm[1] = b.wf(f.ws_W); u.mh[1] = b.wf(f.ws_Th); u.ml[1] = b.wf(f.ws_Tl);
+      u.fh = b.wf(f.ws_Sh); u.fl = b.wf(f.ws_Sl);
+      u.f2h = w64; u.f2l = w64 + dd;
+      u.f4h = q64; u.f4l = q64 + dd;
+    } else {                                     // fp32 matrices only
+      u.xm[0] = b.wf(f.ws_U); u.xm[1] = b.wf(f.ws_T);
+      u.mm[0] = b.wf(f.ws_Y); u.mm[1] = w64;
+      u.fm = w64 + dd;
+      u.f2h = q64; u.f4h = q64 + dd;
+    }
+  }
+  {
+    std::vector<NewtonNormDesc> nd;
+    std::vector<NewtonEltDesc> el;
+    for (size_t i = 0; i < nf; ++i) {
+      const FactorPlan& f = h->factors[i];
+      const Bufs& u = nb[i];
+      nd.push_back({b.S(f), u.sc, f.d, h->cfg.eps, b.fail(i)});
+      NewtonEltDesc e{};
+      e.in = b.S(f); e.sc = u.sc; e.d = f.d; e.mode = kNewtonInit; e.eps = h->cfg.eps; e.skip = b.fail(i);
+      e.m = u.mm[0]; e.mh = u.mh[0]; e.ml = u.ml[0];
+      e.f = u.fm; e.fh = u.fh; e.fl = u.fl;
+      e.x = u.xm[0]; e.xh = u.xh[0]; e.xl = u.xl[0];
+      el.push_back(e);
+    }
+    b.tag = SHAMPOO4_STAGE_NEWTON_ELT;
+    b.emit(prog, Kind::NewtonNorm, nd, 0, 0, 4.0 * sum_dd);
+    b.emit(prog, Kind::NewtonElt, el, emax, 0, 20.0 * sum_dd);
+  }
+  int cx = 0, cm = 0;
+  // C = A B for every factor: fp32-accurate on the tensor cores (split
+  // operands) or on the CUDA cores; outputs as given (fp32, split)
+  auto products = [&](auto pick) {
+    std::vector<TcGemmDesc> t;
+    std::vector<GemmF32Desc> g;
+    for (size_t i = 0; i < nf; ++i) {
+      const FactorPlan& f = h->factors[i];
+      const int d = f.d;
+      float *ah, *al, *bh, *bl, *cm_, *ch, *cl;
+      pick(nb[i], ah, al, bh, bl, cm_, ch, cl);
+      if (f.tc) {
+        TcGemmDesc x = gemmtc(d, d, d, 1.0f, 0.0f);
+        x.a = b.operand(ah, al, d, d, true, false, true);
+        x.b = b.operand(bh, bl, d, d, false, false, true, kSquareBN);
+        x.C = cm_; x.ldc = d;
+        x.Chi = ch; x.Clo = cl; x.ldh = d;
+        x.skip = b.fail(i);
+        t.push_back(x);
+      } else {
+        GemmF32Desc x = gemm32(d, d, d, 0, 0, kModeFP32, 1.0f, 0.0f);
+        x.A = ah; x.lda = d;
+        x.B = bh; x.ldb = d;
+        x.C = cm_; x.ldc = d;
+        x.skip = b.fail(i);
+        g.push_back(x);
+      }
+    }
+    b.tag = SHAMPOO4_STAGE_NEWTON_GEMM;
+    emit_gemmtc(b, prog, t, true, kSquareBN);
+    emit_gemm32(b, prog, g);
+  };
+  for (int it = 1; it <= iters; ++it) {
+    if (it > 1) {                                            // X <- X F
+      const int o = cx ^ 1;
+      products([&](const Bufs& u, float*& ah, float*& al, float*& bh, float*& bl, float*& c, float*& ch,
+                   float*& cl) {
+        ah = u.xh[cx] ? u.xh[cx] : u.xm[cx]; al = u.xl[cx];
+        bh = u.fh ? u.fh : u.fm; bl = u.fl;
+        c = u.xm[o]; ch = u.xh[o]; cl = u.xl[o];
+      });
+      cx = o;
+    }
+    products([&](const Bufs& u, float*& ah, float*& al, float*& bh, float*& bl, float*& c, float*& ch,
+                 float*& cl) {                                // F^2 = F F
+      ah = bh = u.fh ? u.fh : u.fm; al = bl = u.fl;
+      if (u.f2l) { c = nullptr; ch = u.f2h; cl = u.f2l; } else { c = u.f2h; ch = cl = nullptr; }
+    });
+    products([&](const Bufs& u, float*& ah, float*& al, float*& bh, float*& bl, float*& c, float*& ch,
+                 float*& cl) {                                // F^4 = F^2 F^2
+      ah = bh = u.f2h; al = bl = u.f2l;
+      if (u.f4l) { c = nullptr; ch = u.f4h; cl = u.f4l; } else { c = u.f4h; ch = cl = nullptr; }
+    });
+    {
+      const int o = cm ^ 1;
+      products([&](const Bufs& u, float*& ah, float*& al, float*& bh, float*& bl, float*& c, float*& ch,
+                   float*& cl) {                              // M <- F^4 M
+        ah = u.f4h; al = u.f4l;
+        bh = u.mh[cm] ? u.mh[cm] : u.mm[cm]; bl = u.ml[cm];
+        c = u.mm[o]; ch = u.mh[o]; cl = u.ml[o];
+      });
+      cm = o;
+    }
+    if (it < iters) {                                         // F = 1.25 I - 0.25 M
+      std::vector<NewtonEltDesc> el;
+      for (size_t i = 0; i < nf; ++i) {
+        const FactorPlan& f = h->factors[i];
+        const Bufs& u = nb[i];
+        NewtonEltDesc e{};
+        e.in = u.mm[cm]; e.sc = u.sc; e.d = f.d; e.mode = kNewtonStep; e.skip = b.fail(i);
+        e.f = u.fm; e.fh = u.fh; e.fl = u.fl;
+        el.push_back(e);
+      }
+      b.tag = SHAMPOO4_STAGE_NEWTON_ELT;
+      b.emit(prog, Kind::NewtonElt, el, emax, 0, 12.0 * sum_dd);
+    }
+  }
+  // P = c^(-1/4) X: into the state (NEWTON) or a free workspace matrix to
+  // be quantized (NEWTON_Q4)
+  std::vector<float*> P(nf);
+  {
+    std::vector<NewtonEltDesc> el;
+    std::vector<CopyDesc> cp;
+    for (size_t i = 0; i < nf; ++i) {
+      const FactorPlan& f = h->factors[i];
+      const Bufs& u = nb[i];
+      P[i] = q4 ? u.mm[cm ^ 1] : b.sf(f.st_P);
+      NewtonEltDesc e{};
+      e.in = u.xm[cx]; e.sc = u.sc; e.d = f.d; e.mode = kNewtonFinal; e.skip = b.fail(i);
+      e.m = P[i];
+      el.push_back(e);
+      cp.push_back({P[i], b.dbg(f.dbg_q), int64_t(f.d) * f.d});
+    }
+    b.tag = SHAMPOO4_STAGE_NEWTON_ELT;
+    b.emit(prog, Kind::NewtonElt, el, emax, 0, 8.0 * sum_dd);
+    b.tag = SHAMPOO4_STAGE_QR_CONVERT;
+    b.emit(prog, Kind::Copy, cp, emax, 0, 8.0 * sum_dd);
+  }
+  if (q4) {  // quantize the root itself
+    Launch L{};
+    L.kind = Kind::Pack;
+    L.tag = SHAMPOO4_STAGE_REQUANT;
+    for (size_t i = 0; i < nf; ++i) {
+      const FactorPlan& f = h->factors[i];
+      L.px.push_back(P[i]);
+      L.pn.push_back(int64_t(f.d) * f.d);
+      L.pcodes.push_back(b.sb(f.st_codes));
+      L.pscales.push_back(b.sf(f.st_scales));
+      L.pskip.push_back(b.fail(i));
+      L.bytes += 4.5625 * double(f.d) * f.d;
+    }
+    L.count = int(nf);
+    prog.push_back(std::move(L));
+  }
+}
+
 void build_refresh_owned(Builder& b, std::vector<Launch>& prog, bool first) {
+  if (b.h->cfg.root_method != SHAMPOO4_ROOT_EIGEN) {
+    build_refresh_newton(b, prog);
+    return;
+  }
   shampoo4_ctx* h = b.h;
   const size_t nf = h->factors.size();
   const bool split = split_of(h->cfg);
@@ -985,6 +1196,7 @@ void build_refresh_owned(Builder& b, std::vector<Launch>& prog, bool first) {
       BasisDesc x{};
       x.codes = b.sb(f.st_codes); x.scales = b.sf(f.st_scales);
       x.d = f.d; x.identity = first ? 1 : 0;
+      x.codebook = h->cfg.codebook;
       // TF32 Björck reads only U's hi part (and rewrites lo at its last
       // step); without Björck steps the fp32-accurate subspace product
       // reads both parts
@@ -1260,12 +1472,40 @@ void build_precondition(Builder& b) {
   std::vector<RowDiagDesc> rdiag;              // exact diagonal of the fp32-accurate roots
   std::vector<float*> Pm(nf);                  // fp32 root of each factor
   double bytes_bd = 0;
+  const bool newton = h->cfg.root_method != SHAMPOO4_ROOT_EIGEN;
+  std::vector<ScanDesc> psplit;                // NEWTON: TF32 split of the stored root
   for (size_t i = 0; i < nf; ++i) {
     const FactorPlan& f = h->factors[i];
     const int d = f.d;
-    mu.push_back({b.sf(f.st_lam), b.wf(f.ws_mu), d, 0});
     BasisDesc x{};
     x.codes = b.sb(f.st_codes); x.scales = b.sf(f.st_scales); x.d = d; x.identity = 0;
+    x.codebook = h->cfg.codebook;
+    if (newton) {
+      // the root from the refresh: fp32 in the state (NEWTON), or its 4-bit
+      // codes (NEWTON_Q4); tensor-core factors also need its TF32 split in
+      // Th/Tl, and the fp32 copy feeds a tile that is not a tensor-core tile
+      const bool tile_tc = h->blocks[f.block].tc;
+      if (h->cfg.root_method == SHAMPOO4_ROOT_NEWTON) {
+        Pm[i] = b.sf(f.st_P);
+        if (f.tc) {
+          ScanDesc sd{};
+          sd.X = b.sf(f.st_P); sd.ld = d; sd.rows = sd.cols = d;
+          sd.ref.tab = -1;
+          sd.flag = b.tcbad(i);                 // scratch word; bit 0 raises nothing
+          sd.oh = b.wf(f.ws_Th); sd.ol = split ? b.wf(f.ws_Tl) : nullptr;
+          psplit.push_back(sd);
+          bytes_bd += (4.0 + (split ? 8.0 : 4.0)) * double(d) * d;
+        }
+      } else {
+        x.U = f.tc ? (tile_tc ? nullptr : b.wf(f.ws_Xm[1])) : b.wf(f.ws_U);
+        if (f.tc) { x.Uh = b.wf(f.ws_Th); x.Ul = split ? b.wf(f.ws_Tl) : nullptr; }
+        Pm[i] = f.tc ? b.wf(f.ws_Xm[1]) : b.wf(f.ws_U);
+        bd.push_back(x);
+        bytes_bd += (0.5625 + 4.0 + (split ? 8.0 : 4.0)) * double(d) * d;
+      }
+      continue;
+    }
+    mu.push_back({b.sf(f.st_lam), b.wf(f.ws_mu), d, 0});
     if (f.tc) {
       // U -> X[0] split, U diag(mu) -> X[1] split; P = (U mu) U^T -> Th/Tl (+ fp32 in X[1].m)
       x.Uh = b.wf(f.ws_Xh[0]); x.Ul = split ? b.wf(f.ws_Xl[0]) : nullptr;
@@ -1303,6 +1543,7 @@ void build_precondition(Builder& b) {
   b.emit(h->prog_precond, Kind::Mu, mu, dmax);
   b.tag = SHAMPOO4_STAGE_PRECOND_DEQUANT;
   b.emit(h->prog_precond, Kind::Basis, bd, emax, 0, bytes_bd);
+  b.emit(h->prog_precond, Kind::Scan, psplit, dmax, 0, bytes_bd);
   b.tag = SHAMPOO4_STAGE_ROOTS;
   emit_gemmtc(b, h->prog_precond, troots, split);
   b.emit(h->prog_precond, Kind::RowDiag, rdiag, dmax, 0, 16.0 * sum_dd);
@@ -1429,12 +1670,18 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
       case Kind::Convert:
         S4_TRY(launch_convert(static_cast<const ConvertDesc*>(d), L.count, L.extent, st, guard));
         break;
+      case Kind::NewtonNorm:
+        S4_TRY(launch_newton_norm(static_cast<const NewtonNormDesc*>(d), L.count, st));
+        break;
+      case Kind::NewtonElt:
+        S4_TRY(launch_newton_elt(static_cast<const NewtonEltDesc*>(d), L.count, L.extent, st));
+        break;
       case Kind::Copy:
         if (h->d_dbg) S4_TRY(launch_copy(static_cast<const CopyDesc*>(d), L.count, L.extent, st));
         break;
       case Kind::Pack:
         S4_TRY(launch_pack(L.px.data(), L.pn.data(), L.count, L.pcodes.data(), L.pscales.data(), st,
-                           L.pskip.data(), &rec.kernels));
+                           L.pskip.data(), &rec.kernels, h->cfg.codebook));
         break;
     }
     if (h->timing) {
@@ -1541,6 +1788,13 @@ extern "C" shampoo4_status shampoo4_init(const shampoo4_config* cfg, const shamp
     return SHAMPOO4_ERR_INVALID_ARG;
   if (cfg->compressed_stats != 0 && cfg->compressed_stats != 1) return SHAMPOO4_ERR_INVALID_ARG;
   if (cfg->refresh_world < 0 || cfg->refresh_world > 4096) return SHAMPOO4_ERR_INVALID_ARG;
+  if (cfg->codebook != SHAMPOO4_CODEBOOK_LINEAR_SQUARE && cfg->codebook != SHAMPOO4_CODEBOOK_DYNAMIC_TREE)
+    return SHAMPOO4_ERR_INVALID_ARG;
+  if (cfg->root_method != SHAMPOO4_ROOT_EIGEN && cfg->root_method != SHAMPOO4_ROOT_NEWTON &&
+      cfg->root_method != SHAMPOO4_ROOT_NEWTON_Q4)
+    return SHAMPOO4_ERR_INVALID_ARG;
+  if (cfg->root_method != SHAMPOO4_ROOT_EIGEN && cfg->compressed_stats) return SHAMPOO4_ERR_INVALID_ARG;
+  if (cfg->newton_iters < 0 || cfg->newton_iters > 100) return SHAMPOO4_ERR_INVALID_ARG;
   if (cfg->refresh_world > 1 && (cfg->refresh_rank < 0 || cfg->refresh_rank >= cfg->refresh_world))
     return SHAMPOO4_ERR_INVALID_ARG;
   for (int32_t i = 0; i < nparams; ++i)
@@ -1550,6 +1804,7 @@ extern "C" shampoo4_status shampoo4_init(const shampoo4_config* cfg, const shamp
   shampoo4_ctx* h = new (std::nothrow) shampoo4_ctx();
   if (!h) return SHAMPOO4_ERR_INVALID_ARG;
   h->cfg = *cfg;
+  if (h->cfg.newton_iters == 0) h->cfg.newton_iters = kDefaultNewtonIters;
   h->params.assign(params, params + nparams);
   h->world = cfg->refresh_world > 1 ? cfg->refresh_world : 1;
   h->rank = h->world > 1 ? cfg->refresh_rank : 0;
@@ -1739,8 +1994,17 @@ extern "C" shampoo4_status shampoo4_factor_layout(shampoo4_handle h, int32_t fac
   return SHAMPOO4_OK;
 }
 
+extern "C" shampoo4_status shampoo4_root_offset(shampoo4_handle h, int32_t factor, size_t* off_P) {
+  if (!h || !off_P || factor < 0 || size_t(factor) >= h->factors.size()) return SHAMPOO4_ERR_INVALID_ARG;
+  if (h->cfg.root_method != SHAMPOO4_ROOT_NEWTON || h->factors[factor].st_P == SIZE_MAX)
+    return SHAMPOO4_ERR_INVALID_ARG;
+  *off_P = h->factors[factor].st_P;
+  return SHAMPOO4_OK;
+}
+
 extern "C" shampoo4_status shampoo4_debug_q_offset(shampoo4_handle h, int32_t factor, size_t* off_q) {
   if (!h || !off_q || factor < 0 || size_t(factor) >= h->factors.size()) return SHAMPOO4_ERR_INVALID_ARG;
+  if (h->cfg.root_method != SHAMPOO4_ROOT_EIGEN) return SHAMPOO4_ERR_INVALID_ARG;
   if (!h->bound) return SHAMPOO4_ERR_NOT_READY;
   *off_q = h->last_refresh_first ? h->factors[factor].ws_q_first : h->factors[factor].ws_q_next;
   return SHAMPOO4_OK;
@@ -1821,7 +2085,8 @@ extern "C" const char* shampoo4_stage_name(int32_t stage) {
       "stats_scan", "stats_gemm", "refresh_scan", "basis", "bjorck_gram", "bjorck_update",
       "subspace", "qr_gram", "qr_potrf", "qr_trsm_panel", "qr_syrk", "qr_solve_update",
       "qr_solve_panel", "qr_convert", "rayleigh_gemm", "rayleigh", "requant", "precond_dequant",
-      "precond_mu", "roots", "apply_left", "apply_right", "qr_inverse", "stats_dequant", "stats_rebuild", "tables"};
+      "precond_mu", "roots", "apply_left", "apply_right", "qr_inverse", "stats_dequant", "stats_rebuild", "tables",
+      "newton_elt", "newton_gemm"};
   if (stage < 0 || stage >= SHAMPOO4_STAGE_COUNT) return "unknown";
   return names[stage];
 }

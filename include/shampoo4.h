@@ -123,7 +123,44 @@ typedef struct {
                             rank) before precondition, which covers every
                             tile.  0 <= refresh_rank < refresh_world.       */
   int32_t refresh_world; /* 0 or 1: one rank refreshes every factor.        */
+  int32_t codebook;      /* shampoo4_codebook of the 4-bit state            */
+  int32_t root_method;   /* shampoo4_root_method                            */
+  int32_t newton_iters;  /* coupled Newton iterations per refresh (root
+                            methods NEWTON*), 1..100; 0 selects 32          */
 } shampoo4_config;
+
+/* The 4-bit codebook ("4-bit Shampoo for Memory-Efficient Network
+ * Training", abstract: linear square quantization, compared there with
+ * dynamic tree quantization).
+ *  LINEAR_SQUARE: 16 levels sgn(y) y^2, y = (2j - 15)/15, no exact zero.
+ *  DYNAMIC_TREE: Dettmers' (2016) dynamic tree data type restricted to 4
+ *   bits: a sign, then in the other three bits a run of E zeros (a decimal
+ *   exponent), an indicator 1 and k = 2 - E fraction bits i, magnitude
+ *   10^-E (0.1 + 0.9 (i + 1) / 2^k); 000 is zero.  Magnitudes 0, 0.01,
+ *   0.055, 0.1, 0.325, 0.55, 0.775, 1; levels 7 and 8 are both zero.
+ * Either way threshold k is the fp32 rounding of the midpoint of levels k
+ * and k+1 (in double), and a code is the number of thresholds strictly
+ * below v = x / absmax. */
+typedef enum { SHAMPOO4_CODEBOOK_LINEAR_SQUARE = 0, SHAMPOO4_CODEBOOK_DYNAMIC_TREE = 1 } shampoo4_codebook;
+
+/* How each factor's inverse fourth root is obtained.
+ *  EIGEN (the 4-bit Shampoo method): the 4-bit state is the eigenvector
+ *   matrix U with eigenvalues lambda; refresh_roots refines U (dequantize,
+ *   Bjorck, one subspace step) and precondition forms
+ *   P = U diag((lambda + eps)^-1/4) U^T from the codes.
+ *  NEWTON: refresh_roots computes P = (S + eps I)^-1/4 from the fp32
+ *   statistic by the coupled Newton iteration of "Shampoo -- Second-Order
+ *   Optimizer", "Computing the inverse fourth root" (c = ||S + eps I||_F,
+ *   M = (S + eps I)/c, X = I; newton_iters times F = (5 I - M)/4, X <- X F,
+ *   M <- F^4 M; P = X c^-1/4), with fp32-accurate tensor-core products, and
+ *   stores P in fp32 in the state (4 d^2 bytes per factor, a 32-bit root
+ *   cache); precondition applies it.
+ *  NEWTON_Q4: the same root, stored block-wise in 4 bits with the codebook
+ *   above -- quantizing the preconditioner itself, the alternative the
+ *   4-bit Shampoo abstract argues against (its codes and scales take the
+ *   place of U's).
+ * The NEWTON methods need the fp32 statistic (compressed_stats = 0). */
+typedef enum { SHAMPOO4_ROOT_EIGEN = 0, SHAMPOO4_ROOT_NEWTON = 1, SHAMPOO4_ROOT_NEWTON_Q4 = 2 } shampoo4_root_method;
 
 typedef struct { int64_t rows, cols; } shampoo4_param;   /* 2-D weights only;
                             reshape convolutions to out x (in*kh*kw)        */
@@ -219,6 +256,11 @@ shampoo4_status shampoo4_factor_layout(shampoo4_handle h, int32_t factor, size_t
                                        size_t* off_codes, size_t* off_scales,
                                        size_t* off_lambda, int32_t* dim);
 
+/* Root method NEWTON: byte offset inside the state of the factor's fp32
+ * d x d root P = (S + eps I)^-1/4 from the last refresh_roots.
+ * ERR_INVALID_ARG for the other root methods. */
+shampoo4_status shampoo4_root_offset(shampoo4_handle h, int32_t factor, size_t* off_P);
+
 /* Byte offset inside the workspace of the fp32 d x d orthonormal Q that the
  * last refresh quantized for this factor (valid until the next call that uses
  * the workspace).  For tests and diagnostics. */
@@ -244,7 +286,8 @@ shampoo4_status shampoo4_debug_s_offset(shampoo4_handle h, int32_t factor, size_
  * refresh_roots also copies, for each factor it refreshes, the rectified
  * basis that enters the subspace step (after dequantization and Bjorck; the
  * identity on a first refresh) and the orthonormal Q that is then
- * requantized.  The buffer must stay allocated until it is unregistered and
+ * requantized (root methods NEWTON*: the root P in the second slot; the
+ * first is not written).  The buffer must stay allocated until it is unregistered and
  * the handle bound again, or destroyed.  Without one, the copies are not
  * launched.  shampoo4_debug_capture_layout gives the byte offsets of a
  * factor's two row-major matrices in the buffer. */
@@ -279,7 +322,8 @@ typedef enum {
   SHAMPOO4_STAGE_RAYLEIGH, SHAMPOO4_STAGE_REQUANT, SHAMPOO4_STAGE_PRECOND_DEQUANT,
   SHAMPOO4_STAGE_PRECOND_MU, SHAMPOO4_STAGE_ROOTS, SHAMPOO4_STAGE_APPLY_LEFT,
   SHAMPOO4_STAGE_APPLY_RIGHT, SHAMPOO4_STAGE_QR_INVERSE, SHAMPOO4_STAGE_STATS_DEQUANT,
-  SHAMPOO4_STAGE_STATS_REBUILD, SHAMPOO4_STAGE_TABLES, SHAMPOO4_STAGE_COUNT
+  SHAMPOO4_STAGE_STATS_REBUILD, SHAMPOO4_STAGE_TABLES, SHAMPOO4_STAGE_NEWTON_ELT,
+  SHAMPOO4_STAGE_NEWTON_GEMM, SHAMPOO4_STAGE_COUNT
 } shampoo4_stage;
 
 /* Launch timing, for diagnostics and roofline figures.  While enabled, every
@@ -322,6 +366,17 @@ shampoo4_status quant4_unpack(const uint8_t* const* d_codes, const float* const*
 
 /* The 16 codebook levels and 15 thresholds the codec uses (host copy). */
 shampoo4_status quant4_tables(float codebook[16], float thresholds[15]);
+
+/* quant4_pack / quant4_unpack / quant4_tables with a shampoo4_codebook
+ * (the plain names use SHAMPOO4_CODEBOOK_LINEAR_SQUARE); an unknown
+ * codebook returns SHAMPOO4_ERR_INVALID_ARG. */
+shampoo4_status quant4_pack_ex(const float* const* d_x, const int64_t* n, int32_t count,
+                               uint8_t* const* d_codes, float* const* d_scales, int32_t codebook,
+                               shampoo4_stream_t stream);
+shampoo4_status quant4_unpack_ex(const uint8_t* const* d_codes, const float* const* d_scales,
+                                 const int64_t* n, int32_t count, float* const* d_x, int32_t codebook,
+                                 shampoo4_stream_t stream);
+shampoo4_status quant4_tables_ex(int32_t codebook, float levels[16], float thresholds[15]);
 
 /* Statistics update of ONE tile with no handle, no workspace and no device
  * allocation (no counterpart in the 4-bit Shampoo paper: an interface for

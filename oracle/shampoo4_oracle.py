@@ -32,6 +32,14 @@ fp32 only where the state is stored in fp32.
 Readings where the pages are silent (all repeated in the design notes):
   codebook    cb_j = sgn(y_j) y_j^2, y_j = -1 + 2j/15, j = 0..15 (16 levels,
               no exact zero); thresholds are the fp32-rounded midpoints.
+              The dynamic tree alternative the abstract names: Dettmers'
+              dynamic tree data type restricted to 4 bits (sign, decimal
+              exponent as a run of zeros, indicator bit, linear fraction
+              over [0.1, 1] at the upper bin edges; 000 is zero).
+  Newton root the coupled Newton iteration of "Computing the inverse fourth
+              root" with c = ||A||_F and a fixed iteration count, as a root
+              method in place of the eigen form; its root is kept in fp32, or
+              quantized block-wise (quantizing the preconditioner itself).
   scale       per 64-element block of the row-major flattening, fp32 absmax.
   code        number of thresholds strictly below v = fp32(x / absmax); a
               zero block gets code 7 everywhere; NaN in a block gives a NaN
@@ -49,31 +57,62 @@ import math
 import numpy as np
 
 QUANT_BLOCK = 64
+LINEAR_SQUARE = 0
+DYNAMIC_TREE = 1
 
 
 # --------------------------------------------------------------------------
-# Linear square 4-bit codec ("4-bit Shampoo ...", abstract: linear square
-# quantization of the eigenvector matrix, block-wise).
+# Block-wise 4-bit codec ("4-bit Shampoo ...", abstract: linear square
+# quantization of the eigenvector matrix, block-wise, which it finds
+# slightly better than dynamic tree quantization).
 # --------------------------------------------------------------------------
 
-def codebook_f64() -> np.ndarray:
-    """cb_j = sgn(y_j) * y_j^2 with y_j = (2j - 15)/15, j = 0..15, in fp64."""
-    j = np.arange(16, dtype=np.float64)
-    y = 2.0 * j - 15.0
-    return (y * np.abs(y)) / 225.0
+def _dynamic_tree_magnitude(bits: int) -> float:
+    """The 4-bit reading of the dynamic tree data type (Dettmers, "8-bit
+    approximations for parallelism in deep learning", 2016): after the sign,
+    the three bits hold a run of E zeros (the decimal exponent), an
+    indicator 1, and the k = 2 - E bits left over as a linear fraction i;
+    the value is 10^-E (0.1 + 0.9 (i + 1) / 2^k), and 000 (no indicator) is
+    zero.  The fraction takes the upper edge of each of the 2^k equal bins
+    of [0.1, 1], so the largest magnitude is 1 (absmax-normalized blocks
+    keep their absmax exactly, as the linear square map's end levels do).
+    Returns the magnitude as the fp64 rounding of the exact rational."""
+    from fractions import Fraction
+    b = [(bits >> 2) & 1, (bits >> 1) & 1, bits & 1]
+    if 1 not in b:
+        return 0.0
+    e = b.index(1)                     # zeros before the indicator
+    k = 2 - e                          # fraction bits after it
+    i = bits & ((1 << k) - 1)
+    return float(Fraction(10) ** -e * (Fraction(1, 10) + Fraction(9, 10) * Fraction(i + 1, 2 ** k)))
 
 
-def codebook_f32() -> np.ndarray:
-    return codebook_f64().astype(np.float32)
+def codebook_f64(codebook: int = LINEAR_SQUARE) -> np.ndarray:
+    """The 16 levels in ascending order, fp64.
+    LINEAR_SQUARE: cb_j = sgn(y_j) * y_j^2 with y_j = (2j - 15)/15.
+    DYNAMIC_TREE: level 8 + p is +magnitude(p), level 7 - p is
+    -magnitude(p), for the 3-bit patterns p (so levels 7 and 8 are zero)."""
+    if codebook == LINEAR_SQUARE:
+        j = np.arange(16, dtype=np.float64)
+        y = 2.0 * j - 15.0
+        return (y * np.abs(y)) / 225.0
+    if codebook == DYNAMIC_TREE:
+        mag = [_dynamic_tree_magnitude(p) for p in range(8)]
+        return np.array([-mag[7 - j] for j in range(8)] + [mag[p] for p in range(8)], np.float64)
+    raise ValueError(f"unknown codebook {codebook}")
 
 
-def thresholds_f32() -> np.ndarray:
+def codebook_f32(codebook: int = LINEAR_SQUARE) -> np.ndarray:
+    return codebook_f64(codebook).astype(np.float32)
+
+
+def thresholds_f32(codebook: int = LINEAR_SQUARE) -> np.ndarray:
     """t_k = fp32(midpoint of cb_k and cb_{k+1}) for k = 0..14."""
-    cb = codebook_f64()
+    cb = codebook_f64(codebook)
     return ((cb[:-1] + cb[1:]) / 2.0).astype(np.float32)
 
 
-def quantize(x: np.ndarray, block: int = QUANT_BLOCK):
+def quantize(x: np.ndarray, block: int = QUANT_BLOCK, codebook: int = LINEAR_SQUARE):
     """Quantize a flat fp32 vector to (packed codes uint8, scales fp32).
 
     Returns ceil(n/2) code bytes and ceil(n/block) scales.
@@ -87,7 +126,7 @@ def quantize(x: np.ndarray, block: int = QUANT_BLOCK):
     scales = np.abs(xb).max(axis=1) if nb else np.zeros(0, np.float32)
     # numpy's max already returns NaN for a block holding a NaN and +Inf for
     # one holding +-Inf (and no NaN).
-    thr = thresholds_f32()
+    thr = thresholds_f32(codebook)
     with np.errstate(divide="ignore", invalid="ignore"):
         v = (xb / scales[:, None]).astype(np.float32)    # one IEEE fp32 division
     codes = np.zeros(xb.shape, dtype=np.uint8)
@@ -115,10 +154,10 @@ def unpack_nibbles(packed: np.ndarray, n: int) -> np.ndarray:
 
 
 def dequantize(packed: np.ndarray, scales: np.ndarray, n: int,
-               block: int = QUANT_BLOCK) -> np.ndarray:
+               block: int = QUANT_BLOCK, codebook: int = LINEAR_SQUARE) -> np.ndarray:
     """x_i = fp32(cb_code(i)) * scale(i // block), one fp32 multiply."""
     codes = unpack_nibbles(packed, n)
-    cb = codebook_f32()
+    cb = codebook_f32(codebook)
     s = np.repeat(np.asarray(scales, dtype=np.float32), block)[:n]
     return (cb[codes] * s).astype(np.float32)
 
@@ -170,7 +209,8 @@ def ema_stats(S: np.ndarray, Gb: np.ndarray, beta: float, side: str) -> np.ndarr
     return s.astype(np.float32)
 
 
-def compressed_stats(f: "Factor", Gb: np.ndarray, beta: float, side: str) -> np.ndarray:
+def compressed_stats(f: "Factor", Gb: np.ndarray, beta: float, side: str,
+                     codebook: int = LINEAR_SQUARE) -> np.ndarray:
     """The statistic update when S is kept only as its 4-bit eigenbasis and
     eigenvalues ("4-bit Shampoo ...", abstract: the preconditioner is stored
     through its quantized eigenvector matrix): the previous statistic is
@@ -183,7 +223,7 @@ def compressed_stats(f: "Factor", Gb: np.ndarray, beta: float, side: str) -> np.
     g = np.asarray(Gb, dtype=np.float64)
     stored = np.zeros((f.d, f.d))
     if f.has_basis:
-        U = dequantize(f.codes, f.scales, f.d * f.d).reshape(f.d, f.d).astype(np.float64)
+        U = dequantize(f.codes, f.scales, f.d * f.d, codebook=codebook).reshape(f.d, f.d).astype(np.float64)
         lam = np.asarray(f.lam, np.float64)
         stored = (U * lam[None, :]) @ U.T
     if not np.all(np.isfinite(g)):
@@ -266,21 +306,28 @@ class Factor:
     U64: np.ndarray | None = None         # quant=off: fp64 basis
     has_basis: bool = False
     q_last: np.ndarray | None = None      # pre-quantization Q of last refresh
+    P: np.ndarray | None = None           # NEWTON: the fp32 root
 
 
-def refresh_factor(f: Factor, eps: float, bjorck_iters: int, quant: bool = True) -> None:
+ROOT_EIGEN = 0
+ROOT_NEWTON = 1
+ROOT_NEWTON_Q4 = 2
+
+
+def refresh_factor(f: Factor, eps: float, bjorck_iters: int, quant: bool = True,
+                   codebook: int = LINEAR_SQUARE) -> None:
     d = f.d
     if not f.has_basis:
         U = np.eye(d)
     elif quant:
-        U = dequantize(f.codes, f.scales, d * d).reshape(d, d).astype(np.float64)
+        U = dequantize(f.codes, f.scales, d * d, codebook=codebook).reshape(d, d).astype(np.float64)
         U = bjorck(U, bjorck_iters)
     else:
         U = f.U64
     Q, lam = subspace_step(f.S, U, eps)
     f.q_last = Q
     if quant:
-        f.codes, f.scales = quantize(Q.astype(np.float32).ravel())
+        f.codes, f.scales = quantize(Q.astype(np.float32).ravel(), codebook=codebook)
         f.lam = lam.astype(np.float32)
     else:
         f.U64 = Q
@@ -288,9 +335,31 @@ def refresh_factor(f: Factor, eps: float, bjorck_iters: int, quant: bool = True)
     f.has_basis = True
 
 
-def factor_root(f: Factor, eps: float, quant: bool = True) -> np.ndarray:
+def refresh_factor_newton(f: Factor, eps: float, iters: int, quantize_root: bool,
+                          codebook: int = LINEAR_SQUARE) -> None:
+    """The root by the coupled Newton iteration ("Computing the inverse
+    fourth root"), P = (S + eps I)^(-1/4), kept in fp32 -- or, with
+    quantize_root, quantized block-wise to 4 bits: quantizing the
+    preconditioner itself, the alternative the 4-bit Shampoo abstract argues
+    against."""
+    A = np.asarray(f.S, np.float64) + eps * np.eye(f.d)
+    P = newton_inverse_root(A, 4, iters)
+    f.q_last = P
+    if quantize_root:
+        f.codes, f.scales = quantize(P.astype(np.float32).ravel(), codebook=codebook)
+    else:
+        f.P = P.astype(np.float32)
+    f.has_basis = True
+
+
+def factor_root(f: Factor, eps: float, quant: bool = True, codebook: int = LINEAR_SQUARE,
+                root_method: int = ROOT_EIGEN) -> np.ndarray:
+    if root_method == ROOT_NEWTON:
+        return np.asarray(f.P, np.float64)
+    if root_method == ROOT_NEWTON_Q4:
+        return dequantize(f.codes, f.scales, f.d * f.d, codebook=codebook).reshape(f.d, f.d).astype(np.float64)
     if quant:
-        U = dequantize(f.codes, f.scales, f.d * f.d).reshape(f.d, f.d)
+        U = dequantize(f.codes, f.scales, f.d * f.d, codebook=codebook).reshape(f.d, f.d)
         return root_from_basis(U, f.lam, eps)
     return root_from_basis(f.U64, f.lam, eps)
 
@@ -299,15 +368,21 @@ class Shampoo4Oracle:
     """The whole preconditioner step over a list of 2-D parameters."""
 
     def __init__(self, shapes, beta=0.95, eps=1e-6, bjorck_iters=5,
-                 max_block=1024, quant=True, compressed=False):
+                 max_block=1024, quant=True, compressed=False, codebook=LINEAR_SQUARE,
+                 root_method=ROOT_EIGEN, newton_iters=32):
         self.shapes = [tuple(s) for s in shapes]
         self.beta = float(beta)
         self.eps = float(eps)
         self.bjorck_iters = int(bjorck_iters)
         self.quant = bool(quant)
         self.compressed = bool(compressed)
+        self.codebook = int(codebook)
+        self.root_method = int(root_method)
+        self.newton_iters = int(newton_iters)
         if self.compressed and not self.quant:
             raise ValueError("compressed statistics need the 4-bit basis")
+        if self.root_method != ROOT_EIGEN and self.compressed:
+            raise ValueError("the Newton root needs the fp32 statistic")
         self.blocks = partition(self.shapes, max_block)
         self.factors: list[Factor] = []
         for b in self.blocks:
@@ -323,23 +398,27 @@ class Shampoo4Oracle:
             g = self.block_view(grads, k)
             fl, fr = self.factors[2 * k], self.factors[2 * k + 1]
             if self.compressed:
-                fl.S = compressed_stats(fl, g, self.beta, "L")
-                fr.S = compressed_stats(fr, g, self.beta, "R")
+                fl.S = compressed_stats(fl, g, self.beta, "L", self.codebook)
+                fr.S = compressed_stats(fr, g, self.beta, "R", self.codebook)
             else:
                 fl.S = ema_stats(fl.S, g, self.beta, "L")
                 fr.S = ema_stats(fr.S, g, self.beta, "R")
 
     def refresh_roots(self) -> None:
         for f in self.factors:
-            refresh_factor(f, self.eps, self.bjorck_iters, self.quant)
+            if self.root_method == ROOT_EIGEN:
+                refresh_factor(f, self.eps, self.bjorck_iters, self.quant, self.codebook)
+            else:
+                refresh_factor_newton(f, self.eps, self.newton_iters, self.root_method == ROOT_NEWTON_Q4,
+                                      self.codebook)
 
     def precondition(self, grads) -> list[np.ndarray]:
         if not all(f.has_basis for f in self.factors):
             raise RuntimeError("precondition before the first refresh")
         out = [np.zeros(s, np.float32) for s in self.shapes]
         for k, b in enumerate(self.blocks):
-            PL = factor_root(self.factors[2 * k], self.eps, self.quant)
-            PR = factor_root(self.factors[2 * k + 1], self.eps, self.quant)
+            PL = factor_root(self.factors[2 * k], self.eps, self.quant, self.codebook, self.root_method)
+            PR = factor_root(self.factors[2 * k + 1], self.eps, self.quant, self.codebook, self.root_method)
             d = apply_roots(PL, self.block_view(grads, k), PR)
             out[b.param][b.r0:b.r0 + b.m, b.c0:b.c0 + b.n] = d.astype(np.float32)
         return out

@@ -34,7 +34,8 @@ def gpu_factor(sh, f: int) -> O.Factor:
 def oracle_from_gpu(sh, shapes, has_basis: bool) -> O.Shampoo4Oracle:
     cfg = sh.config
     orc = O.Shampoo4Oracle(shapes, beta=float(np.float32(cfg.beta)), eps=float(np.float32(cfg.eps)),
-                           bjorck_iters=cfg.bjorck_iters, max_block=cfg.max_block)
+                           bjorck_iters=cfg.bjorck_iters, max_block=cfg.max_block, codebook=cfg.codebook,
+                           root_method=cfg.root_method, newton_iters=cfg.newton_iters or 32)
     for f in range(len(orc.factors)):
         g = gpu_factor(sh, f)
         g.has_basis = has_basis
@@ -81,7 +82,7 @@ def _oracle_spread(S, U, eps, Qo, lo, big, seeds=3):
     return band_lam, band_root
 
 
-def staged_refresh_check(sh, f, incoming, eps, bjorck_iters, tol, end_to_end=True):
+def staged_refresh_check(sh, f, incoming, eps, bjorck_iters, tol, end_to_end=True, codebook=O.LINEAR_SQUARE):
     """Factor f's last refresh against the oracle, stage by stage, from the
     library's own incoming state (``incoming``: the factor as read before the
     refresh, has_basis set as the library had it).  Needs a handle made with
@@ -108,7 +109,7 @@ def staged_refresh_check(sh, f, incoming, eps, bjorck_iters, tol, end_to_end=Tru
     rec = {"factor": f, "d": d}
     # stage 1
     if incoming.has_basis:
-        U0 = O.dequantize(incoming.codes, incoming.scales, d * d).reshape(d, d).astype(np.float64)
+        U0 = O.dequantize(incoming.codes, incoming.scales, d * d, codebook=codebook).reshape(d, d).astype(np.float64)
         Uo = O.bjorck(U0, bjorck_iters)
         rec["bjorck"] = rel_fro(Ug, Uo)
         rec["bjorck_ok"] = rec["bjorck"] <= tol
@@ -127,12 +128,12 @@ def staged_refresh_check(sh, f, incoming, eps, bjorck_iters, tol, end_to_end=Tru
     rec["banded"] = bool(BAND_FACTOR * max(rec["band_lam"], rec["band_root"]) > tol)
     rec["orth"] = float(np.linalg.norm(Qg.T @ Qg - np.eye(d)) / np.sqrt(d))
     # stage 3
-    oc, os_ = O.quantize(Qg.astype(np.float32).ravel())
+    oc, os_ = O.quantize(Qg.astype(np.float32).ravel(), codebook=codebook)
     rec["codes_ok"] = bool(np.array_equal(g.codes, oc) and np.array_equal(g.scales, os_))
     if end_to_end:
         e = O.Factor(d, incoming.S, codes=incoming.codes, scales=incoming.scales, lam=incoming.lam,
                      has_basis=incoming.has_basis)
-        O.refresh_factor(e, eps, bjorck_iters)
+        O.refresh_factor(e, eps, bjorck_iters, codebook=codebook)
         le = e.lam.astype(np.float64)
         bige = le > 1e3 * eps
         rec["e2e_lam"] = float(np.max(np.abs(lg - le)[bige] / le[bige])) if bige.any() else 0.0
@@ -149,13 +150,13 @@ def format_record(tag, r):
     return s + ("" if r["ok"] else "  FAIL")
 
 
-def staged_refresh_all(sh, incoming, eps, bjorck_iters, tol, tag, end_to_end=True):
+def staged_refresh_all(sh, incoming, eps, bjorck_iters, tol, tag, end_to_end=True, codebook=O.LINEAR_SQUARE):
     """staged_refresh_check over the factors in ``incoming`` (factor index ->
     incoming Factor, has_basis set); prints one line per factor and how many
     needed the band, and asserts every verdict.  Returns the records."""
     recs = []
     for f in sorted(incoming):
-        r = staged_refresh_check(sh, f, incoming[f], eps, bjorck_iters, tol, end_to_end)
+        r = staged_refresh_check(sh, f, incoming[f], eps, bjorck_iters, tol, end_to_end, codebook)
         print(format_record(tag, r))
         recs.append(r)
     nb = sum(r["banded"] for r in recs)

@@ -37,6 +37,45 @@ def test_codec_tables_match_the_oracle_definition():
     assert np.array_equal(np.array(th, np.float32), O.thresholds_f32())
 
 
+def test_dynamic_tree_tables_match_the_oracle_definition():
+    cb = (C.c_float * 16)()
+    th = (C.c_float * 15)()
+    L.call("quant4_tables_ex", L.CODEBOOK_DYNAMIC_TREE, cb, th)
+    assert np.array_equal(np.array(cb, np.float32), O.codebook_f32(O.DYNAMIC_TREE))
+    assert np.array_equal(np.array(th, np.float32), O.thresholds_f32(O.DYNAMIC_TREE))
+    assert L.lib().quant4_tables_ex(7, cb, th) == 1
+
+
+def test_codebook_and_root_method_configs():
+    params = (L.Param * 1)(L.Param(64, 96))
+
+    def init(**kw):
+        cfg = L.Config(0.95, 1e-6, 1024, 64, 5, 0, kw.get("compressed", 0), 0, 1, kw.get("codebook", 0),
+                       kw.get("root", 0), kw.get("iters", 0))
+        h = C.c_void_p()
+        st = L.lib().shampoo4_init(C.byref(cfg), params, 1, C.byref(h))
+        return st, h
+    for kw in ({"codebook": 2}, {"root": 3}, {"root": 1, "compressed": 1}, {"root": 2, "iters": 101},
+               {"iters": -1}):
+        st, h = init(**kw)
+        assert st == 1 and not h.value, kw
+    st, h = init(codebook=1, root=2, iters=20)
+    assert st == 0
+    off = C.c_size_t()
+    assert L.lib().shampoo4_root_offset(h, 0, C.byref(off)) == 1          # no fp32 root kept
+    L.lib().shampoo4_destroy(h)
+    st, h = init(root=1)
+    assert st == 0
+    sizes = []
+    for f in range(2):
+        L.call("shampoo4_root_offset", h, f, C.byref(off))
+        sizes.append(off.value)
+    stb = C.c_size_t()
+    L.call("shampoo4_sizes", h, C.byref(stb), None)
+    assert sizes[0] % 256 == 0 and sizes[0] + 4 * 64 * 64 <= sizes[1] and sizes[1] + 4 * 96 * 96 <= stb.value
+    L.lib().shampoo4_destroy(h)
+
+
 def _init(shapes, **kw):
     cfg = L.Config(kw.get("beta", 0.95), kw.get("eps", 1e-6), kw.get("max_block", 1024), kw.get("qb", 64),
                    kw.get("bj", 5), kw.get("prec", 0), kw.get("compressed", 0))

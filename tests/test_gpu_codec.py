@@ -1,5 +1,5 @@
 """quant4_pack / quant4_unpack on the GPU against the oracle codec: codes and
-scales bit for bit."""
+scales bit for bit, for both codebooks (linear square and dynamic tree)."""
 import numpy as np
 import pytest
 import torch
@@ -15,41 +15,48 @@ def _api():
     return api
 
 
-def _check(xs):
+BOOKS = {"linear_square": O.LINEAR_SQUARE, "dynamic_tree": O.DYNAMIC_TREE}
+
+
+def _check(xs, book="linear_square"):
     api = _api()
+    cbk = BOOKS[book]
     tx = [cuda_f32(x) for x in xs]
-    codes, scales = api.quant4_pack(tx)
+    codes, scales = api.quant4_pack(tx, codebook=book)
     torch.cuda.synchronize()
     for x, c, s in zip(xs, codes, scales):
-        oc, os_ = O.quantize(x)
+        oc, os_ = O.quantize(x, codebook=cbk)
         gc, gs = c.cpu().numpy(), s.cpu().numpy()
         assert np.array_equal(gc, oc), (x.size, np.nonzero(gc != oc)[0][:8])
         assert np.array_equal(gs.view(np.uint32), os_.view(np.uint32)) or \
             np.array_equal(np.isnan(gs), np.isnan(os_)) and np.array_equal(gs[~np.isnan(gs)], os_[~np.isnan(os_)])
-    back = api.quant4_unpack(codes, scales, [x.size for x in xs])
+    back = api.quant4_unpack(codes, scales, [x.size for x in xs], codebook=book)
     torch.cuda.synchronize()
     for x, c, s, b in zip(xs, codes, scales, back):
-        ref = O.dequantize(c.cpu().numpy(), s.cpu().numpy(), x.size)
+        ref = O.dequantize(c.cpu().numpy(), s.cpu().numpy(), x.size, codebook=cbk)
         got = b.cpu().numpy()
         assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)) or \
             (np.array_equal(np.isnan(got), np.isnan(ref)) and np.array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)]))
 
 
-def test_ragged_sizes_one_batch():
+@pytest.mark.parametrize("book", list(BOOKS))
+def test_ragged_sizes_one_batch(book):
     rng = np.random.default_rng(11)
-    sizes = [1, 2, 7, 8, 63, 64, 65, 127, 128, 4095, 4096, 4097, 8193, 100003, 1 << 18]
-    _check([rng.standard_normal(n).astype(np.float32) for n in sizes])
+    sizes = [1, 2, 7, 8, 63, 64, 65, 127, 128, 4095, 4096, 4097, 8193, 16383, 16384, 16385, 100003, 1 << 18]
+    _check([rng.standard_normal(n).astype(np.float32) for n in sizes], book)
 
 
-def test_eigenvector_shaped_inputs():
+@pytest.mark.parametrize("book", list(BOOKS))
+def test_eigenvector_shaped_inputs(book):
     from bit_quantized_shampoo_b200.workloads import u_like
     xs = [u_like(d, 100 + d)[0].ravel() for d in (64, 147, 576, 768, 1024)]
-    _check(xs)
+    _check(xs, book)
 
 
-def test_special_values():
+@pytest.mark.parametrize("book", list(BOOKS))
+def test_special_values(book):
     rng = np.random.default_rng(12)
-    t = O.thresholds_f32()
+    t = O.thresholds_f32(BOOKS[book])
     blocks = []
     blocks.append(np.zeros(64, np.float32))                                   # zero block
     blocks.append((rng.standard_normal(64) * 1e-39).astype(np.float32))      # subnormal scale
@@ -63,18 +70,19 @@ def test_special_values():
     b = np.ones(64, np.float32); b[4] = np.inf; b[7] = -np.inf; blocks.append(b)
     b = (rng.standard_normal(64) * 3e38).astype(np.float32); blocks.append(b)   # near overflow
     b = (rng.standard_normal(64)).astype(np.float32) * np.float32(2.0 ** -126); blocks.append(b)
-    _check([np.concatenate(blocks).astype(np.float32)])
-    _check(blocks)
+    _check([np.concatenate(blocks).astype(np.float32)], book)
+    _check(blocks, book)
 
 
-def test_shared_divisor_division_matches_ieee_over_exponent_range():
+@pytest.mark.parametrize("book", list(BOOKS))
+def test_shared_divisor_division_matches_ieee_over_exponent_range(book):
     rng = np.random.default_rng(13)
     xs = []
     for e in range(-140, 120, 7):
         x = rng.standard_normal(64 * 97).astype(np.float32) * np.float32(2.0 ** e)
         m = rng.integers(-60, 1, size=x.size).astype(np.float32)
         xs.append((x * np.exp2(m)).astype(np.float32))
-    _check(xs)
+    _check(xs, book)
 
 
 def test_misaligned_pointers():

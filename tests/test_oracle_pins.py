@@ -599,3 +599,187 @@ def test_cost_model_reproduces_the_pages_figures():
         assert abs(got[k] - v) <= tol * abs(v) + 1e-12, (k, got[k], v)
     # the per-step term is the sum of its four parts
     assert C.step_flops(300, 70) == C.stats_flops(300, 70) + C.apply_flops(300, 70)
+
+
+# ------------------------------------------- dynamic tree codebook (f3)
+
+def test_dynamic_tree_codebook_follows_its_bit_layout():
+    """The 4-bit dynamic tree map: symmetric, both middle levels zero, and
+    for each decimal exponent E (zeros before the indicator bit) the 2^(2-E)
+    magnitudes lie in (0.1, 1] x 10^-E on an equally spaced grid of step
+    0.9 x 10^-E / 2^(2-E) ending at 10^-E.  Every pattern is decoded here
+    from its bits as a string, independently of the oracle's arithmetic."""
+    cb = O.codebook_f64(O.DYNAMIC_TREE)
+    assert cb.size == 16 and np.all(np.diff(cb) >= 0)
+    assert np.array_equal(cb, -cb[::-1])
+    assert cb[7] == 0.0 and cb[8] == 0.0 and cb[15] == 1.0
+    pos = cb[8:]
+    for p in range(8):
+        bits = format(p, "03b")
+        if "1" not in bits:
+            assert pos[p] == 0.0
+            continue
+        e = bits.index("1")
+        frac = bits[e + 1:]
+        k = len(frac)
+        i = int(frac, 2) if frac else 0
+        lo, hi = 0.1 * 10.0 ** -e, 10.0 ** -e
+        assert lo < pos[p] <= hi * (1 + 1e-15)
+        step = 0.9 * 10.0 ** -e / 2 ** k
+        assert abs(pos[p] - (hi - (2 ** k - 1 - i) * step)) <= 1e-15
+    t = O.thresholds_f32(O.DYNAMIC_TREE)
+    assert t[7] == 0.0 and np.all(np.diff(t) >= 0)
+
+
+def test_dynamic_tree_count_rule_is_nearest_level():
+    """Brute force around every threshold of the dynamic tree map (2^10 fp32
+    neighbours each): the count rule picks the nearest level, measured with
+    exact rational distances to the levels of the bit-layout definition,
+    the lower one on an exact tie -- except between an fp32 threshold and
+    the exact midpoint it rounds (inclusive of the threshold), where the
+    fp32 threshold decides by definition.  Every level also round-trips
+    exactly at absmax 2^k.  (The linear square map has its own exact test
+    above.)"""
+    from fractions import Fraction
+    cbk = O.DYNAMIC_TREE
+    cb = O.codebook_f64(cbk)
+    t = O.thresholds_f32(cbk)
+
+    def level(j):                       # exact rational from the bit layout
+        p = j - 8 if j >= 8 else 7 - j
+        bits = format(p, "03b")
+        if "1" not in bits:
+            return Fraction(0)
+        e = bits.index("1")
+        k = 2 - e
+        i = int(bits[e + 1:], 2) if k else 0
+        m = Fraction(1, 10 ** e) * (Fraction(1, 10) + Fraction(9, 10) * Fraction(i + 1, 2 ** k))
+        return m if j >= 8 else -m
+    lv = [level(j) for j in range(16)]
+    assert np.array_equal(np.array([float(x) for x in lv]), cb)
+    vals = []
+    for tk in t:
+        b = np.array([tk], np.float32).view(np.uint32)[0].astype(np.int64)
+        if tk == 0.0:
+            mag = np.arange(0, 512).astype(np.uint32).view(np.float32)
+            vals += [mag, -mag]
+        else:
+            vals.append((b + np.arange(-512, 512)).astype(np.uint32).view(np.float32))
+    v = np.unique(np.concatenate(vals).astype(np.float32))
+    v = v[np.abs(v) <= 1.0]
+    nblk = (v.size + 62) // 63
+    x = np.zeros(nblk * 64, np.float32)
+    x.reshape(nblk, 64)[:, 0] = 1.0
+    flat = x.reshape(nblk, 64)[:, 1:].ravel()
+    flat[:v.size] = v
+    x.reshape(nblk, 64)[:, 1:] = flat.reshape(nblk, 63)
+    codes, scales = O.quantize(x, codebook=cbk)
+    got = O.unpack_nibbles(codes, x.size).reshape(nblk, 64)[:, 1:].ravel()[:v.size]
+    mids = [(lv[k] + lv[k + 1]) / 2 for k in range(15)]
+    checked = 0
+    for vi, ci in zip(v.tolist(), got.tolist()):
+        fv = Fraction(vi)
+        if any(Fraction(float(tk)) != mk and min(Fraction(float(tk)), mk) <= fv <= max(Fraction(float(tk)), mk)
+               for tk, mk in zip(t, mids)):
+            continue
+        dist = [abs(fv - L) for L in lv]
+        nearest = dist.index(min(dist))                  # first = lower on ties
+        assert lv[ci] == lv[nearest], (vi, ci, nearest)
+        checked += 1
+    assert checked > 0.9 * v.size
+    for k in (-7, 0, 3):
+        j = np.tile(np.arange(16), 8)
+        j[::64] = 15
+        xs = (O.codebook_f32(cbk)[j] * np.float32(2.0 ** k)).astype(np.float32)
+        c2, s2 = O.quantize(xs, codebook=cbk)
+        assert np.array_equal(O.dequantize(c2, s2, xs.size, codebook=cbk), xs)
+
+
+def test_dynamic_tree_error_bound():
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal(64 * 101 + 7).astype(np.float32)
+    codes, scales = O.quantize(x, codebook=O.DYNAMIC_TREE)
+    xr = O.dequantize(codes, scales, x.size, codebook=O.DYNAMIC_TREE)
+    half_gap = np.max(np.diff(O.codebook_f64(O.DYNAMIC_TREE))) / 2     # (0.325 - 0.1) / 2
+    assert abs(half_gap - 0.1125) < 1e-15
+    s = np.repeat(scales, 64)[:x.size].astype(np.float64)
+    assert np.all(np.abs(x.astype(np.float64) - xr) <= half_gap * s * (1 + 1e-6) + 1e-30)
+
+
+# --------------------------------------------- Newton root method (f4)
+
+def test_newton_root_method_matches_the_lapack_root_through_the_step():
+    """Root method NEWTON: the refresh's P is (S + eps I)^(-1/4) and the
+    update is P_L G P_R -- checked against roots built from LAPACK eigh of
+    S + eps I (an independent route), through the oracle's whole step."""
+    rng = np.random.default_rng(31)
+    shapes = [(24, 40)]
+    orc = O.Shampoo4Oracle(shapes, eps=1e-4, root_method=O.ROOT_NEWTON, newton_iters=40)
+    gs = [rng.standard_normal(shapes[0]).astype(np.float32) for _ in range(3)]
+    for t, g in enumerate(gs, 1):
+        D = orc.step(t, [g], refresh_every=1)[0]
+
+    def eig_root(S, eps):
+        w, V = np.linalg.eigh(np.asarray(S, np.float64) + eps * np.eye(S.shape[0]))
+        return (V * w ** -0.25) @ V.T
+    PL, PR = (eig_root(f.S, orc.eps) for f in orc.factors)
+    for f, P in zip(orc.factors, (PL, PR)):
+        assert np.linalg.norm(f.P - P) <= 1e-6 * np.linalg.norm(P)        # P stored in fp32
+    want = PL @ gs[-1].astype(np.float64) @ PR
+    assert np.linalg.norm(D - want) <= 2e-6 * np.linalg.norm(want)
+
+
+def test_newton_root_of_a_diagonal_statistic_and_the_quantized_root():
+    """A diagonal S gives P = diag((s + eps)^-1/4) (Newton keeps diagonal
+    iterates diagonal).  With NEWTON_Q4 each 64-element quantization block is
+    one row of P: its absmax is the diagonal entry, which takes the top
+    level and decodes exactly to the fp32 scale, and every other entry is
+    an exact zero, which the count rule sends to code 7 -- level -1/225 of
+    the linear square map (it has no zero), so it decodes to -scale/225."""
+    d, eps = 64, 1e-6
+    s = np.geomspace(1.0, 1e-3, d).astype(np.float32)
+    want = (s.astype(np.float64) + eps) ** -0.25
+    orc = O.Shampoo4Oracle([(d, d)], eps=eps, root_method=O.ROOT_NEWTON, newton_iters=40)
+    f = orc.factors[0]
+    f.S = np.diag(s).astype(np.float32)
+    O.refresh_factor_newton(f, eps, 40, False)
+    P = O.factor_root(f, eps, root_method=O.ROOT_NEWTON)
+    assert np.count_nonzero(P - np.diag(np.diag(P))) == 0
+    assert np.allclose(np.diag(P), want, rtol=1e-6, atol=0)
+    fq = O.Factor(d, f.S.copy())
+    O.refresh_factor_newton(fq, eps, 40, True)
+    Pq = O.factor_root(fq, eps, root_method=O.ROOT_NEWTON_Q4)
+    sc = fq.scales.astype(np.float64)
+    assert np.array_equal(np.diag(Pq), sc)
+    off = Pq - np.diag(np.diag(Pq))
+    expect_off = (np.float32(-1.0 / 225.0) * fq.scales.astype(np.float32))[:, None] * (1 - np.eye(d))
+    assert np.array_equal(off, expect_off.astype(np.float32).astype(np.float64))
+    assert np.allclose(sc, want, rtol=1e-6, atol=0)
+
+
+def test_the_abstracts_two_comparisons_on_both_codebooks():
+    """"4-bit Shampoo ...", abstract: quantizing the eigenvector matrix beats
+    quantizing the preconditioner itself, and linear square quantization is
+    (slightly) better than dynamic tree quantization.  On statistics with a
+    decaying spectrum (kappa = 1e4), the inverse-root error (relative
+    Frobenius) of: eigenvectors in 4 bits + Bjorck, for each codebook, and
+    the root itself in 4 bits, for each codebook.  The first comparison is
+    asserted; the codebook comparison is reported (the dynamic tree map is
+    a reading of a method the pages only name)."""
+    rng = np.random.default_rng(43)
+    d, eps = 64, 1e-6
+    errs = {k: [] for k in ("U_ls", "U_dt", "P_ls", "P_dt")}
+    for trial in range(4):
+        V = random_orthogonal(d, rng)
+        lam = np.geomspace(1.0, 1e-4, d) * rng.uniform(0.5, 2.0)
+        P = (V * (lam + eps)[None, :] ** -0.25) @ V.T
+        rel = lambda X: np.linalg.norm(X - P) / np.linalg.norm(P)
+        for cbk, tag in ((O.LINEAR_SQUARE, "ls"), (O.DYNAMIC_TREE, "dt")):
+            c, sc = O.quantize(V.astype(np.float32).ravel(), codebook=cbk)
+            Uq = O.dequantize(c, sc, d * d, codebook=cbk).reshape(d, d).astype(np.float64)
+            errs["U_" + tag].append(rel(O.root_from_basis(O.bjorck(Uq, 5), lam, eps)))
+            c2, sc2 = O.quantize(P.astype(np.float32).ravel(), codebook=cbk)
+            errs["P_" + tag].append(rel(O.dequantize(c2, sc2, d * d, codebook=cbk).reshape(d, d)))
+    mean = {k: float(np.mean(v)) for k, v in errs.items()}
+    print("inverse-root error, mean of 4:", {k: f"{v:.3e}" for k, v in mean.items()})
+    assert max(mean["U_ls"], mean["U_dt"]) < min(mean["P_ls"], mean["P_dt"])
