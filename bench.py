@@ -516,17 +516,27 @@ def main():
 
     counter = [0]
 
-    def one_step(g, out):
+    refresh_ev = []                 # (start, end) CUDA events around each timed refresh
+
+    def one_step(g, out, ev=None):
         sh.update_stats(g)
+        if ev is not None:
+            ev[0].record(stream)
         sh.refresh_roots()
+        if ev is not None:
+            ev[1].record(stream)
         if shard:
             sh.exchange_roots()
         sh.precondition(g, out=out)
 
-    def step():
+    def step(timed=False):
         g = dev_sets[counter[0] % nsets]
         counter[0] += 1
-        one_step(g, dev_out)
+        ev = None
+        if timed:
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            refresh_ev.append(ev)
+        one_step(g, dev_out, ev)
 
     for _ in range(args.warmup):
         step()
@@ -540,7 +550,7 @@ def main():
         torch.cuda.nvtx.range_push("timed")
         e0.record(stream)
         for _ in range(args.steps):
-            step()
+            step(timed=True)
         e1.record(stream)
         torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
@@ -584,10 +594,14 @@ def main():
     refresh_stages = ("refresh_scan", "basis", "bjorck_gram", "bjorck_update", "subspace", "qr_gram", "qr_potrf",
                       "qr_trsm_panel", "qr_syrk", "qr_solve_update", "qr_solve_panel", "qr_convert", "qr_inverse",
                       "rayleigh_gemm", "rayleigh", "requant")
-    refresh_ms = sum(stages[k]["ms"] for k in refresh_stages if k in stages)
+    # the refresh call itself, between CUDA events on the caller's stream
+    # (its parts run concurrently on the handle's streams, so summed stage
+    # times would overstate it)
+    refresh_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in refresh_ev), dev) / args.steps
+    stage_sum = sum(stages[k]["ms"] for k in refresh_stages if k in stages)
     others = [formula_roofline(refresh_work(dims, w.bjorck_iters, args.precision), refresh_ms / 1e3, pk, pk_src,
-                               "refresh of every factor (a3-a8), algorithmic flops of the work model; time = sum of "
-                               "its stages' launch times")]
+                               "refresh of every factor (a3-a8), algorithmic flops of the work model; time = the "
+                               "refresh call between CUDA events on the caller's stream")]
     # per stage: the flops each launch's descriptors carry (the implementation's
     # products, which exceed the work model's count for the QR)
     ranked = sorted(stages, key=lambda k: -stages[k]["ms"])
@@ -607,6 +621,7 @@ def main():
             "config": {"workload": w.name, "tiles": sh.nblocks, "factors": sh.nfactors,
                        "steps_per_refresh": 1,
                        "refresh_ms_per_step": refresh_ms,
+                       "refresh_stage_busy_ms": stage_sum,
                        "statistics": "compressed (4-bit eigenbasis + eigenvalues)" if args.compressed else "fp32",
                        "parallelism": (f"refresh sharded over {world} ranks + NCCL span broadcasts" if shard
                                        else f"{world} independent replica(s)"),
@@ -619,6 +634,24 @@ def main():
             "gpu_launches": launches,
             "clocks": clocks, "roofline": roof, "rooflines_other": others,
             "stages_ms": {k: round(v["ms"], 4) for k, v in sorted(stages.items(), key=lambda kv: -kv[1]["ms"])}}
+
+    # the same refresh as one launch sequence on the caller's stream (the
+    # handle's default splits it in two concurrent parts): the split's gain
+    if not shard:
+        L.call("shampoo4_debug_refresh_parts", sh._h, 1)
+        sh.bind(reset=False)
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize()
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        for _ in range(3):
+            sh.refresh_roots()
+        r1.record(stream)
+        torch.cuda.synchronize()
+        line["config"]["refresh_ms_one_part"] = r0.elapsed_time(r1) / 3
+        L.call("shampoo4_debug_refresh_parts", sh._h, 2)
+        sh.bind(reset=False)
 
     # end to end through the public API with host buffers: every step copies
     # its gradients in from pinned host memory and its update out to pinned

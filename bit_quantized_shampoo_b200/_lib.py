@@ -78,6 +78,7 @@ _SIGS = {
     "shampoo4_debug_capture": [C.c_void_p, C.c_void_p],
     "shampoo4_debug_capture_layout": [C.c_void_p, C.c_int32, c_size_p, c_size_p],
     "shampoo4_debug_wait_limit": [C.c_void_p, C.c_uint64],
+    "shampoo4_debug_refresh_parts": [C.c_void_p, C.c_int32],
     "shampoo4_factor_owner": [C.c_void_p, C.c_int32, c_i32_p],
     "shampoo4_owner_span": [C.c_void_p, C.c_int32, c_size_p, c_size_p],
     "quant4_pack": [C.POINTER(C.c_void_p), c_i64_p, C.c_int32, C.POINTER(C.c_void_p),

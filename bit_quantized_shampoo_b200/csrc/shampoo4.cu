@@ -103,7 +103,16 @@ struct shampoo4_ctx {
   uint64_t wait_ns = 0;                  // tensor-core pipeline wait limit (0: the kernel's default)
   size_t ws_desc = 0, ws_desc_bytes = 0;
   // programs
-  std::vector<Launch> prog_stats, prog_stats_first, prog_refresh_first, prog_refresh, prog_precond;
+  std::vector<Launch> prog_stats, prog_stats_first, prog_precond;
+  // the refresh, split into parts of about equal d^3 cost whose programs run
+  // concurrently on the handle's own streams (forked from and joined back to
+  // the caller's stream); one part runs on the caller's stream itself
+  static constexpr int kMaxParts = 2;
+  int refresh_parts = kMaxParts;           // requested (shampoo4_debug_refresh_parts)
+  int nparts = 1;                          // built
+  std::vector<Launch> prog_refresh_first[kMaxParts], prog_refresh[kMaxParts];
+  cudaStream_t part_stream[kMaxParts] = {};
+  cudaEvent_t part_fork = nullptr, part_join[kMaxParts] = {};
   std::vector<uint8_t> arena;            // host image of the descriptor region
   std::vector<CUtensorMap> maps;         // host image of the tensor-map region
   // bound buffers
@@ -393,13 +402,18 @@ struct Builder {
   // the factor's statistic: in the state, or (compressed statistics) in the
   // workspace
   float* S(const FactorPlan& f) const { return f.st_S == SIZE_MAX ? wf(f.ws_S) : sf(f.st_S); }
-  uint32_t* fail(size_t fi) const { return wu(h->ws_fail) + fi; }
-  uint32_t* tcbad(size_t fi) const { return wu(h->ws_tcbad) + fi; }
-  uint32_t* tcgood(size_t fi) const { return wu(h->ws_tcgood) + fi; }
+  // Per-factor scratch words are indexed by the factor's index in the
+  // handle; while a program is built over a subset of the factors (a rank's
+  // share, a part of the refresh), gmap maps the subset's positions to it.
+  const std::vector<size_t>* gmap = nullptr;
+  size_t gi(size_t i) const { return gmap ? (*gmap)[i] : i; }
+  uint32_t* fail(size_t fi) const { return wu(h->ws_fail) + gi(fi); }
+  uint32_t* tcbad(size_t fi) const { return wu(h->ws_tcbad) + gi(fi); }
+  uint32_t* tcgood(size_t fi) const { return wu(h->ws_tcgood) + gi(fi); }
   unsigned long long* devsq(size_t fi) const {
-    return reinterpret_cast<unsigned long long*>(ws + h->ws_devsq) + fi;
+    return reinterpret_cast<unsigned long long*>(ws + h->ws_devsq) + gi(fi);
   }
-  uint32_t* skip3(size_t fi) const { return wu(h->ws_skip3) + fi; }
+  uint32_t* skip3(size_t fi) const { return wu(h->ws_skip3) + gi(fi); }
   uint32_t* gflags() const { return wu(h->ws_flags); }
   float* dbg(size_t off) const { return h->d_dbg ? reinterpret_cast<float*>(h->d_dbg + off) : nullptr; }
 
@@ -1425,32 +1439,50 @@ void build_refresh_owned(Builder& b, std::vector<Launch>& prog, bool first) {
   }
 }
 
-// The refresh programs cover this rank's factors only: they are built over
-// the owned subset (per-factor scratch words are indexed within it), and the
-// offsets the builder assigns to the subset are copied back.
-void build_refresh(Builder& b, std::vector<Launch>& prog, bool first) {
+// The refresh programs cover this rank's factors only, split into up to
+// nparts parts balanced by d^3 cost (longest first, each to the lighter
+// part; each part keeps the factors' order).  Each part's program is built
+// over its subset of the factors (per-factor scratch words keep the
+// factors' own indices, through Builder::gmap), and the workspace offsets
+// the builder assigns are copied back.
+void build_refresh(Builder& b, std::vector<Launch>* progs, bool first) {
   shampoo4_ctx* h = b.h;
-  if (h->world <= 1) {
-    build_refresh_owned(b, prog, first);
-    return;
-  }
-  std::vector<size_t> idx;
-  std::vector<FactorPlan> mine;
+  std::vector<size_t> owned;
   for (size_t i = 0; i < h->factors.size(); ++i)
-    if (h->owner[i] == h->rank) {
-      idx.push_back(i);
-      mine.push_back(h->factors[i]);
+    if (h->owner[i] == h->rank) owned.push_back(i);
+  const int nparts = owned.size() >= 2 ? h->refresh_parts : 1;
+  std::vector<std::vector<size_t>> parts(nparts);
+  {
+    std::vector<size_t> order = owned;
+    auto cost = [&](size_t i) { return double(h->factors[i].d) * h->factors[i].d * h->factors[i].d; };
+    std::stable_sort(order.begin(), order.end(), [&](size_t a, size_t c) { return cost(a) > cost(c); });
+    std::vector<double> load(nparts, 0.0);
+    for (size_t i : order) {
+      int p = 0;
+      for (int q = 1; q < nparts; ++q)
+        if (load[q] < load[p]) p = q;
+      parts[p].push_back(i);
+      load[p] += cost(i);
     }
-  if (mine.empty()) return;
-  std::vector<FactorPlan> all;
-  all.swap(h->factors);
-  h->factors = mine;
-  build_refresh_owned(b, prog, first);
-  for (size_t j = 0; j < idx.size(); ++j) {
-    all[idx[j]].ws_q_first = h->factors[j].ws_q_first;
-    all[idx[j]].ws_q_next = h->factors[j].ws_q_next;
+    for (auto& v : parts) std::sort(v.begin(), v.end());
   }
-  h->factors.swap(all);
+  h->nparts = nparts;
+  for (int p = 0; p < nparts; ++p) {
+    if (parts[p].empty()) continue;
+    std::vector<FactorPlan> sub;
+    for (size_t i : parts[p]) sub.push_back(h->factors[i]);
+    std::vector<FactorPlan> all;
+    all.swap(h->factors);
+    h->factors = sub;
+    b.gmap = &parts[p];
+    build_refresh_owned(b, progs[p], first);
+    b.gmap = nullptr;
+    for (size_t j = 0; j < parts[p].size(); ++j) {
+      all[parts[p][j]].ws_q_first = h->factors[j].ws_q_first;
+      all[parts[p][j]].ws_q_next = h->factors[j].ws_q_next;
+    }
+    h->factors.swap(all);
+  }
 }
 
 void build_precondition(Builder& b) {
@@ -1563,7 +1595,11 @@ void build_precondition(Builder& b) {
       tleft.push_back(l);
       TcGemmDesc r = gemmtc(bp.m, bp.n, bp.n, 1.0f, 0.0f);       // D = B P_R
       r.a = b.operand(b.wf(bp.ws_Bh), b.wf(bp.ws_Bl), bp.m, bp.n, true, false, split);
-      r.b = b.operand(b.wf(fr.ws_Th), b.wf(fr.ws_Tl), bp.n, bp.n, false, true, split);  // P_R symmetric
+      // P_R is symmetric for the eigen and fp32 Newton roots, read K-major as
+      // P_R^T; a root quantized itself (NEWTON_Q4: blocks run along rows) is
+      // not, and is read as stored
+      const bool sym = h->cfg.root_method != SHAMPOO4_ROOT_NEWTON_Q4;
+      r.b = b.operand(b.wf(fr.ws_Th), b.wf(fr.ws_Tl), bp.n, bp.n, false, sym, split);
       r.c_ref = {1, bp.param, bp.r0, bp.c0};
       tright.push_back(r);
     } else {
@@ -1822,8 +1858,8 @@ extern "C" shampoo4_status shampoo4_init(const shampoo4_config* cfg, const shamp
   h->ws_desc = align_up(h->ws_maps + h->ws_nmaps * sizeof(CUtensorMap), kAlign);
   h->ws_desc_bytes = align_up(h->arena.size(), kAlign);
   h->ws_bytes = h->ws_desc + h->ws_desc_bytes;
-  h->prog_stats.clear(); h->prog_stats_first.clear(); h->prog_refresh_first.clear(); h->prog_refresh.clear();
-  h->prog_precond.clear();
+  h->prog_stats.clear(); h->prog_stats_first.clear(); h->prog_precond.clear();
+  for (int p = 0; p < shampoo4_ctx::kMaxParts; ++p) { h->prog_refresh_first[p].clear(); h->prog_refresh[p].clear(); }
   h->arena.clear();
   h->maps.clear();
   *out = h;
@@ -1853,12 +1889,19 @@ extern "C" shampoo4_status shampoo4_bind(shampoo4_handle h, void* d_state, void*
     S4_CUDA(cudaHostAlloc(&h->gtab_pinned, sizeof(PtrEntry) * 3 * h->params.size() + 64, cudaHostAllocDefault));
     S4_CUDA(cudaEventCreateWithFlags(&h->gtab_event, cudaEventDisableTiming));
   }
+  if (!h->part_fork) {
+    S4_CUDA(cudaEventCreateWithFlags(&h->part_fork, cudaEventDisableTiming));
+    for (int p = 0; p < shampoo4_ctx::kMaxParts; ++p) {
+      S4_CUDA(cudaStreamCreateWithFlags(&h->part_stream[p], cudaStreamNonBlocking));
+      S4_CUDA(cudaEventCreateWithFlags(&h->part_join[p], cudaEventDisableTiming));
+    }
+  }
   if (h->tab_event_pending) S4_CUDA(cudaEventSynchronize(h->tab_event));
   if (h->gtab_event_pending) S4_CUDA(cudaEventSynchronize(h->gtab_event));
   h->d_state = static_cast<uint8_t*>(d_state);
   h->d_ws = static_cast<uint8_t*>(d_workspace);
-  h->prog_stats.clear(); h->prog_stats_first.clear(); h->prog_refresh_first.clear(); h->prog_refresh.clear();
-  h->prog_precond.clear();
+  h->prog_stats.clear(); h->prog_stats_first.clear(); h->prog_precond.clear();
+  for (int p = 0; p < shampoo4_ctx::kMaxParts; ++p) { h->prog_refresh_first[p].clear(); h->prog_refresh[p].clear(); }
   h->arena.clear();
   h->maps.clear();
   Builder b{h, h->arena, h->d_ws, h->d_state, true};
@@ -1867,7 +1910,10 @@ extern "C" shampoo4_status shampoo4_bind(shampoo4_handle h, void* d_state, void*
   build_refresh(b, h->prog_refresh, false);
   build_precondition(b);
   if (b.err != SHAMPOO4_OK) return b.err;
-  if (align_up(h->arena.size(), kAlign) != h->ws_desc_bytes || h->maps.size() != h->ws_nmaps)
+  // init sized both regions with the most refresh parts; fewer parts need
+  // no more room (each launch's descriptor array is 256-byte aligned, so a
+  // split launch takes at least what the whole one did)
+  if (align_up(h->arena.size(), kAlign) > h->ws_desc_bytes || h->maps.size() > h->ws_nmaps)
     return SHAMPOO4_ERR_WORKSPACE;
   S4_CUDA(cudaMemsetAsync(h->d_ws, 0, h->ws_maps, st));
   if (!h->maps.empty())
@@ -1921,7 +1967,19 @@ extern "C" shampoo4_status shampoo4_refresh_roots(shampoo4_handle h, shampoo4_st
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_devsq, 0, 8 * h->factors.size(), st));
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_fbany, h->any_simt ? 1 : 0, 4, st));
   const bool first = !h->has_basis;
-  S4_TRY(run(h, first ? h->prog_refresh_first : h->prog_refresh, st));
+  std::vector<Launch>* progs = first ? h->prog_refresh_first : h->prog_refresh;
+  if (h->nparts == 1) {
+    S4_TRY(run(h, progs[0], st));
+  } else {
+    // fork the parts onto the handle's streams and join them back
+    S4_CUDA(cudaEventRecord(h->part_fork, st));
+    for (int p = 0; p < h->nparts; ++p) {
+      S4_CUDA(cudaStreamWaitEvent(h->part_stream[p], h->part_fork, 0));
+      S4_TRY(run(h, progs[p], h->part_stream[p]));
+      S4_CUDA(cudaEventRecord(h->part_join[p], h->part_stream[p]));
+    }
+    for (int p = 0; p < h->nparts; ++p) S4_CUDA(cudaStreamWaitEvent(st, h->part_join[p], 0));
+  }
   h->last_refresh_first = first;
   h->has_basis = true;
   h->stats_pending = false;
@@ -2049,6 +2107,13 @@ extern "C" shampoo4_status shampoo4_debug_capture_layout(shampoo4_handle h, int3
   if (!h || factor < 0 || size_t(factor) >= h->factors.size()) return SHAMPOO4_ERR_INVALID_ARG;
   if (off_u) *off_u = h->factors[factor].dbg_u;
   if (off_q) *off_q = h->factors[factor].dbg_q;
+  return SHAMPOO4_OK;
+}
+
+extern "C" shampoo4_status shampoo4_debug_refresh_parts(shampoo4_handle h, int32_t parts) {
+  if (!h || parts < 1 || parts > shampoo4_ctx::kMaxParts) return SHAMPOO4_ERR_INVALID_ARG;
+  h->refresh_parts = parts;
+  h->bound = false;                       // the programs are rebuilt by the next bind
   return SHAMPOO4_OK;
 }
 
@@ -2216,6 +2281,14 @@ extern "C" void shampoo4_destroy(shampoo4_handle h) {
   }
   if (h->gtab_pinned) cudaFreeHost(h->gtab_pinned);
   if (h->flags_pinned) cudaFreeHost(h->flags_pinned);
+  for (int p = 0; p < shampoo4_ctx::kMaxParts; ++p) {
+    if (h->part_stream[p]) {
+      cudaStreamSynchronize(h->part_stream[p]);
+      cudaStreamDestroy(h->part_stream[p]);
+    }
+    if (h->part_join[p]) cudaEventDestroy(h->part_join[p]);
+  }
+  if (h->part_fork) cudaEventDestroy(h->part_fork);
   delete h;
 }
 

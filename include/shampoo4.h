@@ -296,6 +296,15 @@ shampoo4_status shampoo4_debug_capture(shampoo4_handle h, void* d_buf);
 shampoo4_status shampoo4_debug_capture_layout(shampoo4_handle h, int32_t factor, size_t* off_u,
                                               size_t* off_q);
 
+/* Diagnostic: how many parts the refresh is split into (1 or 2; default 2).
+ * The factors are dealt to the parts by d^3 cost, and the parts' launch
+ * sequences run concurrently on the handle's own CUDA streams, forked from
+ * and joined back to the caller's stream (so a graph captured on the
+ * caller's stream captures them too).  Each factor's arithmetic does not
+ * depend on the split.  Takes effect at the next shampoo4_bind (reset = 0
+ * keeps the state). */
+shampoo4_status shampoo4_debug_refresh_parts(shampoo4_handle h, int32_t parts);
+
 /* Diagnostic: the time limit of the tensor-core products' pipeline waits
  * (a CTA waiting for a free stage, for loaded operands or for its finished
  * accumulator).  On expiry a CTA raises SHAMPOO4_FLAG_TIMEOUT, issues

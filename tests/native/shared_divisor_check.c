@@ -2,7 +2,9 @@
  * r = RN(1/s) and q0 = RN(x r), Markstein's correction q = RN(q0 + e r),
  * e = x - s q0 (exact under FMA), must equal the IEEE quotient RN(x / s)
  * for every normal s and |x| <= s, except where the kernel takes the plain
- * division (|x| or |q0| below 2^-100).  Prints "mismatches N" and exits 1
+ * division (|x| or |q0| below 2^-100); and, for scales in [2^-60, 1], that
+ * the same sequence without that test still gives the code IEEE division
+ * gives.  Prints "mismatches N" and exits 1
  * on any mismatch.  Build: cc -O2 -mfma -ffp-contract=off ... -lm */
 #include <math.h>
 #include <stdint.h>
@@ -47,6 +49,35 @@ int main(int argc, char** argv) {
       ++tested;
       if (memcmp(&q, &ref, 4)) ++bad;
     }
+  /* Blocks with a scale in [2^-60, 1] take the division without the guard
+   * (no per-element test).  There: for |x| >= 2^-100 the quotient must be
+   * the IEEE one bit for bit; below, it must be tiny (under 2^-30, far below
+   * the smallest nonzero threshold magnitude of either codebook, 0.005) with
+   * the sign the IEEE quotient has, +0 and -0 counting as not positive: the
+   * code then depends on that sign alone. */
+  long bad_tiny = 0, tested_tiny = 0;
+  for (long it = 0; it < n; ++it) {
+    float s = bits((uint32_t)(67 + rnd() % 60) << 23 | (rnd() & 0x7fffff));     /* 2^-60 .. 2^-1 */
+    if (rnd() % 8 == 0) s = 1.0f;
+    uint32_t xb = rnd();
+    float x = bits(xb);
+    if (!isfinite(x)) continue;
+    if (rnd() & 1) x = bits((xb & 0x80000000u) | (rnd() % (27u << 23)));      /* below 2^-100 */
+    if (fabsf(x) > s) continue;
+    float r = 1.0f / s;
+    float q0 = x * r;
+    float q = fmaf(fmaf(-q0, s, x), r, q0);
+    float ref = x / s;
+    if (fabsf(x) >= 0x1p-100f) {
+      ++tested;
+      if (memcmp(&q, &ref, 4)) ++bad;
+    } else {
+      ++tested_tiny;
+      if (!(fabsf(q) < 0x1p-30f && fabsf(ref) < 0x1p-30f && ((q > 0.0f) == (ref > 0.0f)))) ++bad_tiny;
+    }
+  }
+  printf("unguarded: tiny tested %ld bad %ld\n", tested_tiny, bad_tiny);
+  bad += bad_tiny;
   printf("tested %ld mismatches %ld\n", tested, bad);
   return bad ? 1 : 0;
 }

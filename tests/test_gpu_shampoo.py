@@ -129,3 +129,35 @@ def test_nonfinite_gradient_leaves_statistics_unchanged():
     after = [sh.factor_views(f)[0].cpu().numpy() for f in range(sh.nfactors)]
     assert np.array_equal(after[0], before[0]) and np.array_equal(after[1], before[1])
     assert not np.array_equal(after[2], before[2])        # the clean parameter still updated
+
+
+@pytest.mark.parametrize("precision", ["tf32", "fp32"])
+def test_refresh_parts_are_bit_identical_to_one_part(precision):
+    """The refresh split into two parts on the handle's own streams computes
+    exactly what one launch sequence over all factors computes: every
+    factor's codes, scales, eigenvalues and captured Q bit for bit, over a
+    cold and a warm refresh, with CUDA-core and tensor-core factors."""
+    from bit_quantized_shampoo_b200 import _lib as L
+    shapes = [(200, 130), (256, 512), (1024, 768), (96, 576)]
+    runs = []
+    for parts in (1, 2):
+        sh = _mk(shapes, precision, debug=True)
+        L.call("shampoo4_debug_refresh_parts", sh._h, parts)
+        sh.bind(reset=True)
+        got = []
+        for rnd in range(2):
+            for step in range(2):
+                sh.update_stats([cuda_f32(g) for g in _grads(shapes, 400 + 10 * rnd + step)])
+            sh.refresh_roots()
+            torch.cuda.synchronize()
+            snap = []
+            for f in range(sh.nfactors):
+                _, c, s, lam = sh.factor_views(f)
+                snap.append((c.cpu().numpy().copy(), s.cpu().numpy().copy(), lam.cpu().numpy().copy(),
+                             sh.debug_q(f).cpu().numpy().copy()))
+            got.append(snap)
+        runs.append(got)
+    for rnd in range(2):
+        for f, (a, b) in enumerate(zip(runs[0][rnd], runs[1][rnd])):
+            for x, y in zip(a, b):
+                assert np.array_equal(x.view(np.uint8), y.view(np.uint8)), (rnd, f)

@@ -1,0 +1,110 @@
+"""Teacher-forced trajectories on the four smaller workloads, at each one's
+own step count and refresh interval (one 128x128 weight: 10 steps, a
+refresh every step; the 1024x1024 layer with its rank-16 term: 100 steps,
+every 10th; the ResNet-50 convolutions and the d = 768 transformer stack:
+20 steps, every 10th).  Every step checks, from the library's own incoming
+state: the statistics update (sampled factors), the refresh stage by stage
+when one runs (gpu_helpers.staged_refresh_check, sampled factors), and the
+preconditioned update (sampled tiles; on the long trajectories, on refresh
+steps and the last step).  Alongside, a free-running oracle
+steps the same seeded gradients from its own state; its distance to the
+library -- the fraction of differing 4-bit codes and the relative update
+error -- is printed, not gated: codes are a discontinuous function of the
+basis, so two correct runs part ways at the first flipped code."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import shampoo4_oracle as O
+from gpu_helpers import gpu_factor, rel_fro, staged_refresh_all
+
+pytestmark = pytest.mark.gpu
+
+TOL_TF32 = 2e-3
+
+
+def _picks(sh, limit):
+    dims = [sh.block_info(k)[3:5] for k in range(sh.nblocks)]
+    tiles = {0, sh.nblocks - 1, max(range(sh.nblocks), key=lambda k: max(dims[k])),
+             min(range(sh.nblocks), key=lambda k: min(dims[k]))}
+    return sorted(tiles)[:limit]
+
+
+@pytest.mark.parametrize("wid", [1, 2, 3, 4])
+def test_teacher_forced_trajectory(wid):
+    from bit_quantized_shampoo_b200 import api
+    from bit_quantized_shampoo_b200.workloads import WORKLOADS, gradient
+
+    w = WORKLOADS[wid]
+    shapes = list(w.shapes)
+    T = w.refresh_every
+    sh = api.Shampoo4(shapes, beta=w.beta, eps=w.eps, max_block=w.max_block, bjorck_iters=w.bjorck_iters,
+                      precision="tf32", debug=True)
+    beta, eps = float(np.float32(w.beta)), float(np.float32(w.eps))
+    tiles = _picks(sh, 4)
+    facs = sorted({f for k in tiles for f in (2 * k, 2 * k + 1)})
+    free = O.Shampoo4Oracle(shapes, beta=beta, eps=eps, bjorck_iters=w.bjorck_iters, max_block=w.max_block)
+    blocks = free.blocks
+    worst = {"stats": 0.0, "update": 0.0}
+    for t in range(1, w.steps + 1):
+        g_host = [gradient(w, i, t) for i in range(len(shapes))]
+        G = [torch.from_numpy(g).cuda() for g in g_host]
+        before = {f: gpu_factor(sh, f) for f in facs}
+        sh.update_stats(G)
+        torch.cuda.synchronize()
+        for f in facs:                               # statistics from the incoming S
+            b = blocks[f // 2]
+            Gb = g_host[b.param][b.r0:b.r0 + b.m, b.c0:b.c0 + b.n]
+            want = O.ema_stats(before[f].S, Gb, beta, "L" if f % 2 == 0 else "R")
+            e = rel_fro(sh.factor_views(f)[0].cpu().numpy(), want)
+            worst["stats"] = max(worst["stats"], e)
+            assert e <= TOL_TF32, (t, f, e)
+        if (t - 1) % T == 0:
+            incoming = {}
+            for f in facs:
+                incoming[f] = gpu_factor(sh, f)
+                incoming[f].has_basis = t > 1
+            sh.refresh_roots()
+            torch.cuda.synchronize()
+            assert sh.status_flags() & ~0x10 == 0
+            staged_refresh_all(sh, incoming, eps, w.bjorck_iters, TOL_TF32, f"workload {wid} step {t}",
+                               end_to_end=False)
+        out = sh.precondition(G)
+        torch.cuda.synchronize()
+        # the update from the library's state: every step of the short
+        # trajectories; on refresh steps and the last step of the long ones
+        # (the CPU oracle's roots dominate the test's time)
+        check_update = w.steps <= 10 or (t - 1) % T == 0 or t == w.steps
+        for k in (tiles if check_update else []):
+            b = blocks[k]
+            Gb = g_host[b.param][b.r0:b.r0 + b.m, b.c0:b.c0 + b.n]
+            want = O.apply_roots(O.factor_root(gpu_factor(sh, 2 * k), eps), Gb,
+                                 O.factor_root(gpu_factor(sh, 2 * k + 1), eps))
+            e = rel_fro(out[b.param][b.r0:b.r0 + b.m, b.c0:b.c0 + b.n].cpu().numpy(), want)
+            worst["update"] = max(worst["update"], e)
+            assert e <= TOL_TF32, (t, k, e)
+        # the free-running oracle on the same gradients, sampled tiles only
+        for k in tiles:
+            b = blocks[k]
+            Gb = g_host[b.param][b.r0:b.r0 + b.m, b.c0:b.c0 + b.n]
+            for f, side in ((2 * k, "L"), (2 * k + 1, "R")):
+                free.factors[f].S = O.ema_stats(free.factors[f].S, Gb, beta, side)
+                if (t - 1) % T == 0:
+                    O.refresh_factor(free.factors[f], eps, w.bjorck_iters)
+        if (t - 1) % T == 0 or t == w.steps:
+            mism, drift = [], []
+            for k in tiles:
+                b = blocks[k]
+                Gb = g_host[b.param][b.r0:b.r0 + b.m, b.c0:b.c0 + b.n]
+                for f in (2 * k, 2 * k + 1):
+                    a = O.unpack_nibbles(free.factors[f].codes, free.factors[f].d ** 2)
+                    c = O.unpack_nibbles(gpu_factor(sh, f).codes, free.factors[f].d ** 2)
+                    mism.append(float(np.mean(a != c)))
+                Df = O.apply_roots(O.factor_root(free.factors[2 * k], eps), Gb,
+                                   O.factor_root(free.factors[2 * k + 1], eps))
+                drift.append(rel_fro(out[b.param][b.r0:b.r0 + b.m, b.c0:b.c0 + b.n].cpu().numpy(), Df))
+            print(f"workload {wid} step {t}: free-running oracle vs library: codes differing "
+                  f"{np.mean(mism):.3%} (worst factor {max(mism):.3%}), update rel. error "
+                  f"{np.mean(drift):.2e} (worst tile {max(drift):.2e})")
+    print(f"workload {wid}: {w.steps} steps, refresh every {T}: worst stats {worst['stats']:.2e}, "
+          f"worst update {worst['update']:.2e}")
