@@ -41,7 +41,8 @@ class Config(C.Structure):
     _fields_ = [("beta", C.c_float), ("eps", C.c_float), ("max_block", C.c_int32),
                 ("quant_block", C.c_int32), ("bjorck_iters", C.c_int32), ("precision", C.c_int32),
                 ("compressed_stats", C.c_int32), ("refresh_rank", C.c_int32), ("refresh_world", C.c_int32),
-                ("codebook", C.c_int32), ("root_method", C.c_int32), ("newton_iters", C.c_int32)]
+                ("codebook", C.c_int32), ("root_method", C.c_int32), ("newton_iters", C.c_int32),
+                ("group_tiles", C.c_int32)]
 
 
 class GraftConfig(C.Structure):

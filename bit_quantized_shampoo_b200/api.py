@@ -34,7 +34,7 @@ class Shampoo4:
 
     def __init__(self, shapes, beta=0.95, eps=1e-6, max_block=1024, bjorck_iters=5,
                  precision="tf32", device=None, reset=True, compressed=False, refresh_rank=0, refresh_world=1,
-                 debug=False, codebook="linear_square", root="eigen", newton_iters=0):
+                 debug=False, codebook="linear_square", root="eigen", newton_iters=0, group_tiles=0):
         self.shapes = [(int(r), int(c)) for r, c in shapes]
         self.compressed = bool(compressed)
         self.refresh_rank, self.refresh_world = int(refresh_rank), int(refresh_world)
@@ -45,7 +45,8 @@ class Shampoo4:
         self.root_method = roots[root]
         cfg = L.Config(beta, eps, max_block, 64, bjorck_iters,
                        L.PREC_FP32 if precision == "fp32" else L.PREC_TF32, 1 if compressed else 0,
-                       self.refresh_rank, self.refresh_world, self.codebook, self.root_method, int(newton_iters))
+                       self.refresh_rank, self.refresh_world, self.codebook, self.root_method, int(newton_iters),
+                       int(group_tiles))
         params = (L.Param * len(self.shapes))(*[L.Param(r, c) for r, c in self.shapes])
         h = C.c_void_p()
         L.call("shampoo4_init", C.byref(cfg), params, len(self.shapes), C.byref(h))
@@ -210,7 +211,11 @@ class Shampoo4:
             L.call("shampoo4_debug_capture_layout", self._h, f, None, C.byref(off))
             return self.debug_buffer[off.value:off.value + 4 * d * d].view(torch.float32).view(d, d)
         off = C.c_size_t()
-        L.call("shampoo4_debug_q_offset", self._h, f, C.byref(off))
+        st = L.lib().shampoo4_debug_q_offset(self._h, f, C.byref(off))
+        if st == 6:
+            raise RuntimeError("debug_q: with several tile groups the workspace copy of Q does not survive the "
+                               "refresh; make the handle with debug=True")
+        L.check("shampoo4_debug_q_offset", st)
         return self.workspace[off.value:off.value + 4 * d * d].view(torch.float32).view(d, d)
 
     def debug_rectified(self, f):

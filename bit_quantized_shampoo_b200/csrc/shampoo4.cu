@@ -48,6 +48,20 @@ struct Launch {
   std::vector<const uint32_t*> pskip;
 };
 
+// The launches of one API call: one or more sequences, each run in order
+// on a lane: -1 is the caller's stream, p >= 0 the handle's stream p
+// (forked from and joined back to the caller's stream).
+struct Program {
+  std::vector<std::vector<Launch>> seq;
+  std::vector<int> lane;
+  void clear() { seq.clear(); lane.clear(); }
+  std::vector<Launch>& add(int l) {
+    seq.emplace_back();
+    lane.push_back(l);
+    return seq.back();
+  }
+};
+
 struct BlockPlan {
   int32_t param;
   int64_t r0, c0;
@@ -81,6 +95,9 @@ struct FactorPlan {
 
 constexpr size_t kAlign = 256;
 constexpr int kDefaultNewtonIters = 32;
+// automatic grouping: the largest run of consecutive tiles whose call
+// scratch fits in this many bytes (two such slots are allocated)
+constexpr size_t kGroupBytes = size_t(8) << 30;
 constexpr int kPanelW = 64;     // Cholesky panel width (64 x 64 diagonal blocks)
 constexpr int kSolveW = 128;    // solve panel width (128 x 128 inverse blocks)
 
@@ -96,6 +113,7 @@ struct shampoo4_ctx {
   size_t ws_flags = 0, ws_tabs = 0, ws_fail = 0, ws_bflag = 0, ws_maps = 0, ws_nmaps = 0;
   size_t ws_tcbad = 0, ws_tcgood = 0, ws_devsq = 0, ws_skip3 = 0, ws_fbany = 0;
   bool any_simt = false;                 // some factor always takes the fp64 QR
+  std::vector<int32_t> group_begin;      // tile groups: [group_begin[g], group_begin[g+1])
   // optional debug capture (shampoo4_debug_capture): every refresh copies
   // each refreshed factor's rectified basis and pre-quantization Q here
   uint8_t* d_dbg = nullptr;
@@ -103,14 +121,13 @@ struct shampoo4_ctx {
   uint64_t wait_ns = 0;                  // tensor-core pipeline wait limit (0: the kernel's default)
   size_t ws_desc = 0, ws_desc_bytes = 0;
   // programs
-  std::vector<Launch> prog_stats, prog_stats_first, prog_precond;
-  // the refresh, split into parts of about equal d^3 cost whose programs run
-  // concurrently on the handle's own streams (forked from and joined back to
-  // the caller's stream); one part runs on the caller's stream itself
+  // With one tile group, statistics and precondition run on the caller's
+  // stream and the refresh is split into parts of about equal d^3 cost that
+  // run concurrently on the handle's streams; with several groups, every
+  // call runs group g on the handle's stream g mod 2.
+  Program prog_stats, prog_stats_first, prog_refresh_first, prog_refresh, prog_precond;
   static constexpr int kMaxParts = 2;
   int refresh_parts = kMaxParts;           // requested (shampoo4_debug_refresh_parts)
-  int nparts = 1;                          // built
-  std::vector<Launch> prog_refresh_first[kMaxParts], prog_refresh[kMaxParts];
   cudaStream_t part_stream[kMaxParts] = {};
   cudaEvent_t part_fork = nullptr, part_join[kMaxParts] = {};
   std::vector<uint8_t> arena;            // host image of the descriptor region
@@ -304,54 +321,110 @@ shampoo4_status plan(shampoo4_ctx* h) {
   h->ws_skip3 = take(ws, 4 * h->factors.size());
   h->ws_fbany = take(ws, 4);
   h->ws_bflag = take(ws, 4 * h->blocks.size());
-  for (FactorPlan& f : h->factors) {
-    size_t dd = size_t(f.d) * f.d;
-    f.ws_S = (h->cfg.compressed_stats && h->owner[&f - h->factors.data()] == h->rank) ? take(ws, 4 * dd) : SIZE_MAX;
+  // persistent per factor: the rebuilt statistic (compressed statistics,
+  // valid from update_stats to refresh_roots) and the root weights
+  for (size_t i = 0; i < h->factors.size(); ++i) {
+    FactorPlan& f = h->factors[i];
+    const size_t dd = size_t(f.d) * f.d;
+    f.ws_S = (h->cfg.compressed_stats && h->owner[i] == h->rank) ? take(ws, 4 * dd) : SIZE_MAX;
     f.ws_mu = take(ws, 4 * size_t(f.d));
+  }
+  // Scratch of one call: the refresh's matrices per factor, the split
+  // gradient and apply intermediate per tile.  The tiles are cut into
+  // groups of consecutive tiles; group g's scratch lives in slot g mod 2,
+  // so groups that share a slot run one after another on the same stream
+  // and the workspace holds the scratch of two groups, not of every tile.
+  auto factor_scratch = [&](FactorPlan& f, size_t& cur) {
+    const size_t dd = size_t(f.d) * f.d;
     if (f.tc) {
       for (int i = 0; i < 2; ++i) {
-        f.ws_Xm[i] = take(ws, 4 * dd);
-        f.ws_Xh[i] = take(ws, 4 * dd);
-        f.ws_Xl[i] = take(ws, 4 * dd);
+        f.ws_Xm[i] = take(cur, 4 * dd);
+        f.ws_Xh[i] = take(cur, 4 * dd);
+        f.ws_Xl[i] = take(cur, 4 * dd);
       }
-      f.ws_Th = take(ws, 4 * dd);
-      f.ws_Tl = take(ws, 4 * dd);
-      f.ws_Sh = take(ws, 4 * dd);
-      f.ws_Sl = take(ws, 4 * dd);
-      f.ws_W = take(ws, 4 * dd);
-      f.ws_Zm = take(ws, 4 * dd);
-      f.ws_Zh = take(ws, 4 * dd);
-      f.ws_Zl = take(ws, 4 * dd);
+      f.ws_Th = take(cur, 4 * dd);
+      f.ws_Tl = take(cur, 4 * dd);
+      f.ws_Sh = take(cur, 4 * dd);
+      f.ws_Sl = take(cur, 4 * dd);
+      f.ws_W = take(cur, 4 * dd);
+      f.ws_Zm = take(cur, 4 * dd);
+      f.ws_Zh = take(cur, 4 * dd);
+      f.ws_Zl = take(cur, 4 * dd);
       // the inverse blocks are written 64 x 64 (zero-padded): rows up to a
       // multiple of 64
       const size_t dpad = align_up(size_t(f.d), kPanelW);
-      f.ws_Ih = take(ws, 4 * dpad * kPanelW);
-      f.ws_Il = take(ws, 4 * dpad * kPanelW);
+      f.ws_Ih = take(cur, 4 * dpad * kPanelW);
+      f.ws_Il = take(cur, 4 * dpad * kPanelW);
       const size_t dpad2 = align_up(size_t(f.d), kSolveW);
-      f.ws_Jh = take(ws, 4 * dpad2 * kSolveW);
-      f.ws_Jl = take(ws, 4 * dpad2 * kSolveW);
-      f.ws_Ph = take(ws, 4 * size_t(f.d) * kSolveW);
-      f.ws_Pl = take(ws, 4 * size_t(f.d) * kSolveW);
-      f.ws_W64 = take(ws, 8 * dd);            // fp64 fallback of the QR
-      f.ws_Q64 = take(ws, 8 * dd);
+      f.ws_Jh = take(cur, 4 * dpad2 * kSolveW);
+      f.ws_Jl = take(cur, 4 * dpad2 * kSolveW);
+      f.ws_Ph = take(cur, 4 * size_t(f.d) * kSolveW);
+      f.ws_Pl = take(cur, 4 * size_t(f.d) * kSolveW);
+      f.ws_W64 = take(cur, 8 * dd);            // fp64 fallback of the QR
+      f.ws_Q64 = take(cur, 8 * dd);
     } else {
-      f.ws_W64 = take(ws, 8 * dd);
-      f.ws_Q64 = take(ws, 8 * dd);
-      f.ws_U = take(ws, 4 * dd);
-      f.ws_T = take(ws, 4 * dd);
-      f.ws_Y = take(ws, 4 * dd);
+      f.ws_W64 = take(cur, 8 * dd);
+      f.ws_Q64 = take(cur, 8 * dd);
+      f.ws_U = take(cur, 4 * dd);
+      f.ws_T = take(cur, 4 * dd);
+      f.ws_Y = take(cur, 4 * dd);
     }
-  }
-  for (BlockPlan& b : h->blocks) {
-    size_t mn = size_t(b.m) * b.n;
+  };
+  auto tile_scratch = [&](BlockPlan& b, size_t& cur) {
+    const size_t mn = size_t(b.m) * b.n;
     if (!b.tc) {
-      b.ws_tmp = take(ws, 4 * mn);
-      continue;
+      b.ws_tmp = take(cur, 4 * mn);
+      return;
     }
-    b.ws_Gh = take(ws, 4 * mn);
-    b.ws_Gl = take(ws, 4 * mn);
-    b.ws_Bh = take(ws, 4 * mn);
-    b.ws_Bl = take(ws, 4 * mn);
+    b.ws_Gh = take(cur, 4 * mn);
+    b.ws_Gl = take(cur, 4 * mn);
+    b.ws_Bh = take(cur, 4 * mn);
+    b.ws_Bl = take(cur, 4 * mn);
+  };
+  auto group_bytes = [&](size_t k0, size_t k1) {
+    size_t cur = 0;
+    for (size_t k = k0; k < k1; ++k) {
+      FactorPlan a = h->factors[2 * k], c = h->factors[2 * k + 1];
+      BlockPlan t = h->blocks[k];
+      factor_scratch(a, cur);
+      factor_scratch(c, cur);
+      tile_scratch(t, cur);
+    }
+    return align_up(cur, kAlign);
+  };
+  // groups: group_tiles tiles each, or (0) as many as keep a group's scratch
+  // within kGroupBytes; one group when the refresh is sharded over ranks
+  const size_t nb = h->blocks.size();
+  h->group_begin.assign(1, 0);
+  if (h->world > 1 || h->cfg.group_tiles >= int64_t(nb)) {
+    h->group_begin.push_back(int32_t(nb));
+  } else if (h->cfg.group_tiles > 0) {
+    for (size_t k = h->cfg.group_tiles; k < nb; k += h->cfg.group_tiles) h->group_begin.push_back(int32_t(k));
+    h->group_begin.push_back(int32_t(nb));
+  } else {
+    size_t k0 = 0;
+    for (size_t k = 0; k < nb; ++k)
+      if (k > k0 && group_bytes(k0, k + 1) > kGroupBytes) {
+        h->group_begin.push_back(int32_t(k));
+        k0 = k;
+      }
+    h->group_begin.push_back(int32_t(nb));
+  }
+  const int ngroups = int(h->group_begin.size()) - 1;
+  const int nslots = ngroups > 1 ? 2 : 1;
+  for (int sl = 0; sl < nslots; ++sl) {
+    const size_t base = align_up(ws, kAlign);
+    size_t extent = 0;
+    for (int g = sl; g < ngroups; g += nslots) {
+      size_t cur = base;
+      for (int32_t k = h->group_begin[g]; k < h->group_begin[g + 1]; ++k) {
+        factor_scratch(h->factors[2 * k], cur);
+        factor_scratch(h->factors[2 * k + 1], cur);
+        tile_scratch(h->blocks[k], cur);
+      }
+      extent = std::max(extent, cur - base);
+    }
+    ws = base + extent;
   }
   plan_graft(h, ws);
   h->ws_maps = align_up(ws, kAlign);
@@ -406,7 +479,9 @@ struct Builder {
   // handle; while a program is built over a subset of the factors (a rank's
   // share, a part of the refresh), gmap maps the subset's positions to it.
   const std::vector<size_t>* gmap = nullptr;
+  const std::vector<size_t>* bmap = nullptr;    // the same for tiles
   size_t gi(size_t i) const { return gmap ? (*gmap)[i] : i; }
+  uint32_t* bflag(size_t k) const { return wu(h->ws_bflag) + (bmap ? (*bmap)[k] : k); }
   uint32_t* fail(size_t fi) const { return wu(h->ws_fail) + gi(fi); }
   uint32_t* tcbad(size_t fi) const { return wu(h->ws_tcbad) + gi(fi); }
   uint32_t* tcgood(size_t fi) const { return wu(h->ws_tcgood) + gi(fi); }
@@ -520,7 +595,7 @@ void build_grad_copy(Builder& b, std::vector<Launch>& prog, int tag, bool with_f
     ScanDesc s{};
     s.rows = bp.m; s.cols = bp.n;
     s.ref = {0, bp.param, bp.r0, bp.c0};
-    s.flag = b.wu(h->ws_bflag) + k;
+    s.flag = b.bflag(k);
     s.bit = with_flags ? SHAMPOO4_FLAG_NONFINITE_GRAD : 0u;
     if (bp.tc) {
       s.oh = b.wf(bp.ws_Gh);
@@ -608,7 +683,7 @@ void build_stats_into(Builder& b, std::vector<Launch>& prog, bool rebuild) {
   const float beta = (compressed && !rebuild) ? 0.0f : h->cfg.beta;
   for (size_t k = 0; k < h->blocks.size(); ++k) {
     const BlockPlan& bp = h->blocks[k];
-    uint32_t* skip = b.wu(h->ws_bflag) + k;
+    uint32_t* skip = b.bflag(k);
     for (int side = 0; side < 2; ++side) {
       if (h->owner[2 * k + side] != h->rank) continue;
       const FactorPlan& f = h->factors[2 * k + side];
@@ -644,10 +719,70 @@ void build_stats_into(Builder& b, std::vector<Launch>& prog, bool rebuild) {
   emit_gemm32(b, prog, g);
 }
 
+// Swaps one tile group in for the builders: tiles k0..k1-1 become local
+// tiles 0.., their factors local factors 2(k - k0) + side, and gmap/bmap
+// give the builders the handle-wide indices of the per-factor scratch words
+// and tile flags.  The handle's lists come back on destruction, with the
+// workspace offsets the builders assigned.
+struct GroupScope {
+  shampoo4_ctx* h;
+  Builder& b;
+  std::vector<BlockPlan> blocks;
+  std::vector<FactorPlan> factors;
+  std::vector<int32_t> owner;
+  std::vector<size_t> fmap, bmap;
+  GroupScope(Builder& bb, int32_t k0, int32_t k1) : h(bb.h), b(bb) {
+    std::vector<BlockPlan> lb;
+    std::vector<FactorPlan> lf;
+    std::vector<int32_t> lo;
+    for (int32_t k = k0; k < k1; ++k) {
+      lb.push_back(h->blocks[k]);
+      bmap.push_back(size_t(k));
+      for (int side = 0; side < 2; ++side) {
+        FactorPlan f = h->factors[2 * k + side];
+        f.block = k - k0;
+        lf.push_back(f);
+        fmap.push_back(size_t(2 * k + side));
+        lo.push_back(h->owner[2 * k + side]);
+      }
+    }
+    blocks.swap(h->blocks);
+    factors.swap(h->factors);
+    owner.swap(h->owner);
+    h->blocks.swap(lb);
+    h->factors.swap(lf);
+    h->owner.swap(lo);
+    b.gmap = &fmap;
+    b.bmap = &bmap;
+  }
+  ~GroupScope() {
+    for (size_t j = 0; j < fmap.size(); ++j) {
+      factors[fmap[j]].ws_q_first = h->factors[j].ws_q_first;
+      factors[fmap[j]].ws_q_next = h->factors[j].ws_q_next;
+    }
+    h->blocks.swap(blocks);
+    h->factors.swap(factors);
+    h->owner.swap(owner);
+    b.gmap = nullptr;
+    b.bmap = nullptr;
+  }
+};
+
+int ngroups(const shampoo4_ctx* h) { return int(h->group_begin.size()) - 1; }
+
 void build_stats(Builder& b) {
   shampoo4_ctx* h = b.h;
-  build_stats_into(b, h->prog_stats, true);
-  if (h->cfg.compressed_stats) build_stats_into(b, h->prog_stats_first, false);
+  const int ng = ngroups(h);
+  for (int g = 0; g < ng; ++g) {
+    if (ng == 1) {
+      build_stats_into(b, h->prog_stats.add(-1), true);
+      if (h->cfg.compressed_stats) build_stats_into(b, h->prog_stats_first.add(-1), false);
+      break;
+    }
+    GroupScope scope(b, h->group_begin[g], h->group_begin[g + 1]);
+    build_stats_into(b, h->prog_stats.add(g % 2), true);
+    if (h->cfg.compressed_stats) build_stats_into(b, h->prog_stats_first.add(g % 2), false);
+  }
 }
 
 // fp64 Cholesky-QR pass over the factors with use[i]: X (fp32, d x d) -> Q
@@ -1445,8 +1580,16 @@ void build_refresh_owned(Builder& b, std::vector<Launch>& prog, bool first) {
 // over its subset of the factors (per-factor scratch words keep the
 // factors' own indices, through Builder::gmap), and the workspace offsets
 // the builder assigns are copied back.
-void build_refresh(Builder& b, std::vector<Launch>* progs, bool first) {
+void build_refresh(Builder& b, Program& prog, bool first) {
   shampoo4_ctx* h = b.h;
+  const int ng = ngroups(h);
+  if (ng > 1) {
+    for (int g = 0; g < ng; ++g) {
+      GroupScope scope(b, h->group_begin[g], h->group_begin[g + 1]);
+      build_refresh_owned(b, prog.add(g % 2), first);
+    }
+    return;
+  }
   std::vector<size_t> owned;
   for (size_t i = 0; i < h->factors.size(); ++i)
     if (h->owner[i] == h->rank) owned.push_back(i);
@@ -1466,7 +1609,6 @@ void build_refresh(Builder& b, std::vector<Launch>* progs, bool first) {
     }
     for (auto& v : parts) std::sort(v.begin(), v.end());
   }
-  h->nparts = nparts;
   for (int p = 0; p < nparts; ++p) {
     if (parts[p].empty()) continue;
     std::vector<FactorPlan> sub;
@@ -1475,7 +1617,7 @@ void build_refresh(Builder& b, std::vector<Launch>* progs, bool first) {
     all.swap(h->factors);
     h->factors = sub;
     b.gmap = &parts[p];
-    build_refresh_owned(b, progs[p], first);
+    build_refresh_owned(b, prog.add(nparts == 1 ? -1 : p), first);
     b.gmap = nullptr;
     for (size_t j = 0; j < parts[p].size(); ++j) {
       all[parts[p][j]].ws_q_first = h->factors[j].ws_q_first;
@@ -1485,7 +1627,7 @@ void build_refresh(Builder& b, std::vector<Launch>* progs, bool first) {
   }
 }
 
-void build_precondition(Builder& b) {
+void build_precondition_into(Builder& b, std::vector<Launch>& prog) {
   shampoo4_ctx* h = b.h;
   const size_t nf = h->factors.size();
   const bool split = split_of(h->cfg);
@@ -1572,15 +1714,15 @@ void build_precondition(Builder& b) {
     bd.push_back(x);
   }
   b.tag = SHAMPOO4_STAGE_PRECOND_MU;
-  b.emit(h->prog_precond, Kind::Mu, mu, dmax);
+  b.emit(prog, Kind::Mu, mu, dmax);
   b.tag = SHAMPOO4_STAGE_PRECOND_DEQUANT;
-  b.emit(h->prog_precond, Kind::Basis, bd, emax, 0, bytes_bd);
-  b.emit(h->prog_precond, Kind::Scan, psplit, dmax, 0, bytes_bd);
+  b.emit(prog, Kind::Basis, bd, emax, 0, bytes_bd);
+  b.emit(prog, Kind::Scan, psplit, dmax, 0, bytes_bd);
   b.tag = SHAMPOO4_STAGE_ROOTS;
-  emit_gemmtc(b, h->prog_precond, troots, split);
-  b.emit(h->prog_precond, Kind::RowDiag, rdiag, dmax, 0, 16.0 * sum_dd);
-  emit_gemm32(b, h->prog_precond, roots);
-  build_grad_copy(b, h->prog_precond, SHAMPOO4_STAGE_STATS_SCAN, false);
+  emit_gemmtc(b, prog, troots, split);
+  b.emit(prog, Kind::RowDiag, rdiag, dmax, 0, 16.0 * sum_dd);
+  emit_gemm32(b, prog, roots);
+  build_grad_copy(b, prog, SHAMPOO4_STAGE_STATS_SCAN, false);
   std::vector<GemmF32Desc> left, right;
   std::vector<TcGemmDesc> tleft, tright;
   for (size_t k = 0; k < h->blocks.size(); ++k) {
@@ -1617,11 +1759,24 @@ void build_precondition(Builder& b) {
     }
   }
   b.tag = SHAMPOO4_STAGE_APPLY_LEFT;
-  emit_gemmtc(b, h->prog_precond, tleft, split);
-  emit_gemm32(b, h->prog_precond, left);
+  emit_gemmtc(b, prog, tleft, split);
+  emit_gemm32(b, prog, left);
   b.tag = SHAMPOO4_STAGE_APPLY_RIGHT;
-  emit_gemmtc(b, h->prog_precond, tright, split);
-  emit_gemm32(b, h->prog_precond, right);
+  emit_gemmtc(b, prog, tright, split);
+  emit_gemm32(b, prog, right);
+}
+
+void build_precondition(Builder& b) {
+  shampoo4_ctx* h = b.h;
+  const int ng = ngroups(h);
+  if (ng == 1) {
+    build_precondition_into(b, h->prog_precond.add(-1));
+    return;
+  }
+  for (int g = 0; g < ng; ++g) {
+    GroupScope scope(b, h->group_begin[g], h->group_begin[g + 1]);
+    build_precondition_into(b, h->prog_precond.add(g % 2));
+  }
 }
 
 cudaEvent_t take_event(shampoo4_ctx* h) {
@@ -1728,6 +1883,30 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
   return SHAMPOO4_OK;
 }
 
+// Run one call's program: its sequences on their lanes, the handle's
+// streams forked from the caller's stream and joined back to it.
+shampoo4_status run_program(shampoo4_ctx* h, const Program& P, cudaStream_t st) {
+  bool used[shampoo4_ctx::kMaxParts] = {};
+  bool fork = false;
+  for (int l : P.lane)
+    if (l >= 0) used[l] = fork = true;
+  if (!fork) {
+    for (const auto& q : P.seq) S4_TRY(run(h, q, st));
+    return SHAMPOO4_OK;
+  }
+  S4_CUDA(cudaEventRecord(h->part_fork, st));
+  for (int p = 0; p < shampoo4_ctx::kMaxParts; ++p)
+    if (used[p]) S4_CUDA(cudaStreamWaitEvent(h->part_stream[p], h->part_fork, 0));
+  for (size_t i = 0; i < P.seq.size(); ++i)
+    S4_TRY(run(h, P.seq[i], P.lane[i] < 0 ? st : h->part_stream[P.lane[i]]));
+  for (int p = 0; p < shampoo4_ctx::kMaxParts; ++p)
+    if (used[p]) {
+      S4_CUDA(cudaEventRecord(h->part_join[p], h->part_stream[p]));
+      S4_CUDA(cudaStreamWaitEvent(st, h->part_join[p], 0));
+    }
+  return SHAMPOO4_OK;
+}
+
 shampoo4_status collect_timing(shampoo4_ctx* h) {
   for (auto& r : h->recs) {
     S4_CUDA(cudaEventSynchronize(r.e1));
@@ -1831,6 +2010,7 @@ extern "C" shampoo4_status shampoo4_init(const shampoo4_config* cfg, const shamp
     return SHAMPOO4_ERR_INVALID_ARG;
   if (cfg->root_method != SHAMPOO4_ROOT_EIGEN && cfg->compressed_stats) return SHAMPOO4_ERR_INVALID_ARG;
   if (cfg->newton_iters < 0 || cfg->newton_iters > 100) return SHAMPOO4_ERR_INVALID_ARG;
+  if (cfg->group_tiles < 0) return SHAMPOO4_ERR_INVALID_ARG;
   if (cfg->refresh_world > 1 && (cfg->refresh_rank < 0 || cfg->refresh_rank >= cfg->refresh_world))
     return SHAMPOO4_ERR_INVALID_ARG;
   for (int32_t i = 0; i < nparams; ++i)
@@ -1859,7 +2039,7 @@ extern "C" shampoo4_status shampoo4_init(const shampoo4_config* cfg, const shamp
   h->ws_desc_bytes = align_up(h->arena.size(), kAlign);
   h->ws_bytes = h->ws_desc + h->ws_desc_bytes;
   h->prog_stats.clear(); h->prog_stats_first.clear(); h->prog_precond.clear();
-  for (int p = 0; p < shampoo4_ctx::kMaxParts; ++p) { h->prog_refresh_first[p].clear(); h->prog_refresh[p].clear(); }
+  h->prog_refresh_first.clear(); h->prog_refresh.clear();
   h->arena.clear();
   h->maps.clear();
   *out = h;
@@ -1901,7 +2081,7 @@ extern "C" shampoo4_status shampoo4_bind(shampoo4_handle h, void* d_state, void*
   h->d_state = static_cast<uint8_t*>(d_state);
   h->d_ws = static_cast<uint8_t*>(d_workspace);
   h->prog_stats.clear(); h->prog_stats_first.clear(); h->prog_precond.clear();
-  for (int p = 0; p < shampoo4_ctx::kMaxParts; ++p) { h->prog_refresh_first[p].clear(); h->prog_refresh[p].clear(); }
+  h->prog_refresh_first.clear(); h->prog_refresh.clear();
   h->arena.clear();
   h->maps.clear();
   Builder b{h, h->arena, h->d_ws, h->d_state, true};
@@ -1951,7 +2131,7 @@ extern "C" shampoo4_status shampoo4_update_stats(shampoo4_handle h, const float*
   S4_TRY(set_tables(h, d_grads, ld, nullptr, nullptr, st));
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_bflag, 0, 4 * h->blocks.size(), st));
   const bool rebuild = !h->cfg.compressed_stats || h->has_basis;
-  S4_TRY(run(h, rebuild ? h->prog_stats : h->prog_stats_first, st));
+  S4_TRY(run_program(h, rebuild ? h->prog_stats : h->prog_stats_first, st));
   h->stats_pending = h->cfg.compressed_stats != 0;
   return SHAMPOO4_OK;
 }
@@ -1967,19 +2147,7 @@ extern "C" shampoo4_status shampoo4_refresh_roots(shampoo4_handle h, shampoo4_st
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_devsq, 0, 8 * h->factors.size(), st));
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_fbany, h->any_simt ? 1 : 0, 4, st));
   const bool first = !h->has_basis;
-  std::vector<Launch>* progs = first ? h->prog_refresh_first : h->prog_refresh;
-  if (h->nparts == 1) {
-    S4_TRY(run(h, progs[0], st));
-  } else {
-    // fork the parts onto the handle's streams and join them back
-    S4_CUDA(cudaEventRecord(h->part_fork, st));
-    for (int p = 0; p < h->nparts; ++p) {
-      S4_CUDA(cudaStreamWaitEvent(h->part_stream[p], h->part_fork, 0));
-      S4_TRY(run(h, progs[p], h->part_stream[p]));
-      S4_CUDA(cudaEventRecord(h->part_join[p], h->part_stream[p]));
-    }
-    for (int p = 0; p < h->nparts; ++p) S4_CUDA(cudaStreamWaitEvent(st, h->part_join[p], 0));
-  }
+  S4_TRY(run_program(h, first ? h->prog_refresh_first : h->prog_refresh, st));
   h->last_refresh_first = first;
   h->has_basis = true;
   h->stats_pending = false;
@@ -2005,7 +2173,7 @@ extern "C" shampoo4_status shampoo4_precondition(shampoo4_handle h, const float*
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   S4_TRY(set_tables(h, d_grads, ld, d_out, ld_out, st));
-  return run(h, h->prog_precond, st);
+  return run_program(h, h->prog_precond, st);
 }
 
 extern "C" shampoo4_status shampoo4_get_status_flags(shampoo4_handle h, uint32_t* flags,
@@ -2063,6 +2231,7 @@ extern "C" shampoo4_status shampoo4_root_offset(shampoo4_handle h, int32_t facto
 extern "C" shampoo4_status shampoo4_debug_q_offset(shampoo4_handle h, int32_t factor, size_t* off_q) {
   if (!h || !off_q || factor < 0 || size_t(factor) >= h->factors.size()) return SHAMPOO4_ERR_INVALID_ARG;
   if (h->cfg.root_method != SHAMPOO4_ROOT_EIGEN) return SHAMPOO4_ERR_INVALID_ARG;
+  if (ngroups(h) > 1) return SHAMPOO4_ERR_UNSUPPORTED;    // a later group reuses the scratch
   if (!h->bound) return SHAMPOO4_ERR_NOT_READY;
   *off_q = h->last_refresh_first ? h->factors[factor].ws_q_first : h->factors[factor].ws_q_next;
   return SHAMPOO4_OK;

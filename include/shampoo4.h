@@ -127,6 +127,17 @@ typedef struct {
   int32_t root_method;   /* shampoo4_root_method                            */
   int32_t newton_iters;  /* coupled Newton iterations per refresh (root
                             methods NEWTON*), 1..100; 0 selects 32          */
+  int32_t group_tiles;   /* tiles per group of the calls' scratch.  The
+                            workspace holds the per-call scratch (the
+                            refresh's matrices per factor, the split gradient
+                            per tile) of two groups of consecutive tiles,
+                            which the calls process in turn on two CUDA
+                            streams of the handle, not of every tile at once.
+                            0: as many tiles per group as keep a group's
+                            scratch within 8 GiB; >= the tile count: one
+                            group (the largest workspace).  With
+                            refresh_world > 1 there is one group.  Results do
+                            not depend on the grouping.                     */
 } shampoo4_config;
 
 /* The 4-bit codebook ("4-bit Shampoo for Memory-Efficient Network
@@ -263,7 +274,9 @@ shampoo4_status shampoo4_root_offset(shampoo4_handle h, int32_t factor, size_t* 
 
 /* Byte offset inside the workspace of the fp32 d x d orthonormal Q that the
  * last refresh quantized for this factor (valid until the next call that uses
- * the workspace).  For tests and diagnostics. */
+ * the workspace).  Root method EIGEN and one tile group only (with several,
+ * a later group reuses the scratch: ERR_UNSUPPORTED; shampoo4_debug_capture
+ * works either way).  For tests and diagnostics. */
 shampoo4_status shampoo4_debug_q_offset(shampoo4_handle h, int32_t factor, size_t* off_q);
 
 /* With compressed_stats: byte offset inside the workspace of the fp32 d x d

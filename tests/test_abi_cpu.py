@@ -76,6 +76,33 @@ def test_codebook_and_root_method_configs():
     L.lib().shampoo4_destroy(h)
 
 
+def test_tile_groups_bound_the_workspace():
+    """The calls' scratch is held for two groups of consecutive tiles, not
+    for every tile: on the Llama layer set one group needs 81.9 GB, the
+    automatic grouping (at most 8 GiB of scratch per group) about a fifth
+    of it, and 16 tiles per group less than one and a half times the 4.5 GB
+    state.  A negative group size is refused."""
+    w = WORKLOADS[5]
+    params = (L.Param * len(w.shapes))(*[L.Param(r, c) for r, c in w.shapes])
+    sizes = {}
+    for gt in (100000, 0, 16, 1):
+        cfg = L.Config(0.95, 1e-6, 1024, 64, 5, 0, 0, 0, 1, 0, 0, 0, gt)
+        h = C.c_void_p()
+        L.call("shampoo4_init", C.byref(cfg), params, len(w.shapes), C.byref(h))
+        st, ws = C.c_size_t(), C.c_size_t()
+        L.call("shampoo4_sizes", h, C.byref(st), C.byref(ws))
+        sizes[gt] = (st.value, ws.value)
+        L.lib().shampoo4_destroy(h)
+    state = sizes[0][0]
+    assert sizes[100000][1] > 80e9
+    assert sizes[0][1] < 0.25 * sizes[100000][1]
+    assert sizes[16][1] < 1.5 * state
+    assert sizes[1][1] < sizes[16][1] < sizes[0][1]
+    cfg = L.Config(0.95, 1e-6, 1024, 64, 5, 0, 0, 0, 1, 0, 0, 0, -1)
+    h = C.c_void_p()
+    assert L.lib().shampoo4_init(C.byref(cfg), params, len(w.shapes), C.byref(h)) == 1
+
+
 def _init(shapes, **kw):
     cfg = L.Config(kw.get("beta", 0.95), kw.get("eps", 1e-6), kw.get("max_block", 1024), kw.get("qb", 64),
                    kw.get("bj", 5), kw.get("prec", 0), kw.get("compressed", 0))

@@ -161,3 +161,37 @@ def test_refresh_parts_are_bit_identical_to_one_part(precision):
         for f, (a, b) in enumerate(zip(runs[0][rnd], runs[1][rnd])):
             for x, y in zip(a, b):
                 assert np.array_equal(x.view(np.uint8), y.view(np.uint8)), (rnd, f)
+
+
+@pytest.mark.parametrize("compressed", [False, True])
+def test_tile_groups_give_the_same_results(compressed):
+    """Grouping the tiles (the calls' scratch held for two groups at a time,
+    the groups run in turn on the handle's two streams) changes no result:
+    statistics, codes, scales, eigenvalues, captured Q and the
+    preconditioned update are bit for bit those of one group, over a cold
+    and a warm refresh."""
+    shapes = [(200, 130), (256, 512), (1024, 768), (96, 576), (300, 260)]
+    runs = []
+    for gt in (100000, 1, 2):
+        sh = _mk(shapes, "tf32", debug=True, group_tiles=gt, compressed=compressed)
+        got = []
+        for rnd in range(2):
+            gs = _grads(shapes, 450 + rnd)
+            sh.update_stats([cuda_f32(g) for g in gs])
+            sh.refresh_roots()
+            out = sh.precondition([cuda_f32(g) for g in gs])
+            torch.cuda.synchronize()
+            assert sh.status_flags() & ~0x10 == 0
+            snap = [o.cpu().numpy().copy() for o in out]
+            for f in range(sh.nfactors):
+                S, c, s, lam = sh.factor_views(f)
+                snap += [c.cpu().numpy().copy(), s.cpu().numpy().copy(), lam.cpu().numpy().copy(),
+                         sh.debug_q(f).cpu().numpy().copy()]
+                if not compressed:
+                    snap.append(S.cpu().numpy().copy())
+            got.append(snap)
+        runs.append(got)
+    for other in runs[1:]:
+        for rnd in range(2):
+            for i, (x, y) in enumerate(zip(runs[0][rnd], other[rnd])):
+                assert np.array_equal(x.view(np.uint8), y.view(np.uint8)), (rnd, i)
