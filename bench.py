@@ -798,9 +798,34 @@ def main():
                          "status_flags": sh.status_flags()}
         del weights, gstate
 
+    # bounded workspace layouts of the same step: 48 and 16 tiles per group
+    # (the default here is one group, the largest workspace and the fastest)
+    layouts_ok = not args.no_configs and args.shapes is None and args.workload == 5 and not shard
+    if layouts_ok:
+        del sh
+        torch.cuda.empty_cache()
+        line["layouts"] = {}
+        for name, gt in (("48_tiles_per_group", 48), ("16_tiles_per_group", 16)):
+            lay = api.Shampoo4(shapes, beta=w.beta, eps=w.eps, max_block=w.max_block, bjorck_iters=w.bjorck_iters,
+                               precision=args.precision, device=dev, group_tiles=gt)
+            for i in range(3):
+                lay.update_stats(dev_sets[i % nsets]); lay.refresh_roots(); lay.precondition(dev_sets[i % nsets], out=dev_out)
+            torch.cuda.synchronize()
+            l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            l0.record(stream)
+            for i in range(3):
+                lay.update_stats(dev_sets[i % nsets]); lay.refresh_roots(); lay.precondition(dev_sets[i % nsets], out=dev_out)
+            l1.record(stream)
+            torch.cuda.synchronize()
+            line["layouts"][name] = {"group_tiles": gt, "workspace_bytes": lay.workspace_bytes,
+                                     "ms_per_step": max_over_ranks(l0.elapsed_time(l1), dev) / 3}
+            del lay
+            torch.cuda.empty_cache()
+
     # the four smaller workloads, each at its own refresh interval
     if not args.no_configs and args.shapes is None and args.workload == 5:
-        del sh
+        if not layouts_ok:
+            del sh
         torch.cuda.empty_cache()
         line["configs"] = {}
         for wid in (1, 2, 3, 4):

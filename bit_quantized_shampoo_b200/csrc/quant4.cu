@@ -3,20 +3,21 @@
 // block-wise linear square quantization; the dynamic tree map is the
 // alternative codebook).
 //
-// Memory-bound.  One CTA of 256 threads covers 16384 consecutive elements of
-// one tensor (256 quantization blocks); each thread owns four groups of 8
-// elements and issues all four groups' loads (128 bytes) before it computes
-// any of them, so that enough reads are in flight to cover DRAM latency
-// while the warp spends its issue slots on the quantization arithmetic.  8
-// consecutive lanes own one block.
+// Memory-bound.  One CTA of 256 threads covers 8192 consecutive elements of
+// one tensor (128 quantization blocks); each thread owns two groups of 8
+// elements and issues both groups' loads before it computes either.  8
+// consecutive lanes own one block.  (Measured on a 1 GiB tensor: four
+// groups per thread, persistent grid-stride loops with the next group's
+// loads in flight, and immediate-operand threshold searches were all
+// slower; their register use costs more occupancy than they save.)
 #include "quant4.cuh"
 #include "plan.h"
 
 namespace s4 {
 
 constexpr int kCodecThreads = 256;
-constexpr int kCodecGroupsPerThread = 4;
-constexpr int kCodecEltsPerCta = kCodecThreads * 8 * kCodecGroupsPerThread;   // 16384
+constexpr int kCodecGroupsPerThread = 2;
+constexpr int kCodecEltsPerCta = kCodecThreads * 8 * kCodecGroupsPerThread;   // 8192
 constexpr int kCodecMaxBatch = 64;
 
 struct PackTensor {

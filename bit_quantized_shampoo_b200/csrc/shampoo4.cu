@@ -95,8 +95,11 @@ struct FactorPlan {
 
 constexpr size_t kAlign = 256;
 constexpr int kDefaultNewtonIters = 32;
-// automatic grouping: the largest run of consecutive tiles whose call
-// scratch fits in this many bytes (two such slots are allocated)
+// automatic grouping: one group while the whole call scratch fits in
+// kOneGroupBytes (every launch then covers every factor, which the
+// latency-bound steps of the QR chain need), else runs of consecutive tiles
+// whose scratch fits in kGroupBytes (two such slots are allocated)
+constexpr size_t kOneGroupBytes = size_t(96) << 30;
 constexpr size_t kGroupBytes = size_t(8) << 30;
 constexpr int kPanelW = 64;     // Cholesky panel width (64 x 64 diagonal blocks)
 constexpr int kSolveW = 128;    // solve panel width (128 x 128 inverse blocks)
@@ -400,6 +403,8 @@ shampoo4_status plan(shampoo4_ctx* h) {
     h->group_begin.push_back(int32_t(nb));
   } else if (h->cfg.group_tiles > 0) {
     for (size_t k = h->cfg.group_tiles; k < nb; k += h->cfg.group_tiles) h->group_begin.push_back(int32_t(k));
+    h->group_begin.push_back(int32_t(nb));
+  } else if (group_bytes(0, nb) <= kOneGroupBytes) {
     h->group_begin.push_back(int32_t(nb));
   } else {
     size_t k0 = 0;

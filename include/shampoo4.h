@@ -133,9 +133,12 @@ typedef struct {
                             per tile) of two groups of consecutive tiles,
                             which the calls process in turn on two CUDA
                             streams of the handle, not of every tile at once.
-                            0: as many tiles per group as keep a group's
-                            scratch within 8 GiB; >= the tile count: one
-                            group (the largest workspace).  With
+                            0: one group while the whole scratch fits in
+                            96 GiB, else as many tiles per group as keep a
+                            group's scratch within 8 GiB; >= the tile count:
+                            one group.  One group is the fastest (every
+                            launch covers every factor; the QR chain's
+                            latency-bound steps need that) and the largest.  With
                             refresh_world > 1 there is one group.  Results do
                             not depend on the grouping.                     */
 } shampoo4_config;

@@ -166,3 +166,28 @@ def staged_refresh_all(sh, incoming, eps, bjorck_iters, tol, tag, end_to_end=Tru
     bad = [r["factor"] for r in recs if not r["ok"]]
     assert not bad, f"{tag}: factors {bad} outside the staged refresh gates"
     return recs
+
+
+def update_band(fl, fr, G, eps, seeds=2):
+    """The oracle's own spread of the preconditioned update D = P_L G P_R
+    (roots from the factors' codes and eigenvalues) when every operand of
+    the TF32 products -- U diag(mu), U, G and the intermediate P_L G --
+    carries an independent relative perturbation of the size of TF32
+    round-to-nearest (uniform in +-2^-11).  A root that leans on the
+    eigen-directions next to eps (the first refresh of a statistic, or a
+    rank-deficient one) amplifies that rounding through cancellation in
+    P_L G P_R."""
+    def root(f, rng):
+        U = O.dequantize(f.codes, f.scales, f.d * f.d).reshape(f.d, f.d).astype(np.float64)
+        mu = (np.asarray(f.lam, np.float64) + eps) ** -0.25
+        jit = lambda X: X * (1.0 + 2.0 ** -11 * rng.uniform(-1, 1, X.shape))
+        return jit(U * mu[None, :]) @ jit(U).T
+    ref = O.apply_roots(O.factor_root(fl, eps), G, O.factor_root(fr, eps))
+    band = 0.0
+    for seed in range(seeds):
+        rng = np.random.default_rng(7000 + seed)
+        PL, PR = root(fl, rng), root(fr, rng)
+        jit = lambda X: X * (1.0 + 2.0 ** -11 * rng.uniform(-1, 1, X.shape))
+        B = jit(jit(PL) @ jit(np.asarray(G, np.float64)))
+        band = max(band, rel_fro(B @ jit(PR), ref))
+    return band

@@ -78,14 +78,15 @@ def test_codebook_and_root_method_configs():
 
 def test_tile_groups_bound_the_workspace():
     """The calls' scratch is held for two groups of consecutive tiles, not
-    for every tile: on the Llama layer set one group needs 81.9 GB, the
-    automatic grouping (at most 8 GiB of scratch per group) about a fifth
+    for every tile: on the Llama layer set one group (what the automatic
+    rule picks below 96 GiB) needs 81.9 GB, 48 tiles per group about a fifth
     of it, and 16 tiles per group less than one and a half times the 4.5 GB
-    state.  A negative group size is refused."""
+    state; the Llama set twice over exceeds 96 GiB in one group, and the
+    automatic rule groups it.  A negative group size is refused."""
     w = WORKLOADS[5]
     params = (L.Param * len(w.shapes))(*[L.Param(r, c) for r, c in w.shapes])
     sizes = {}
-    for gt in (100000, 0, 16, 1):
+    for gt in (100000, 0, 48, 16, 1):
         cfg = L.Config(0.95, 1e-6, 1024, 64, 5, 0, 0, 0, 1, 0, 0, 0, gt)
         h = C.c_void_p()
         L.call("shampoo4_init", C.byref(cfg), params, len(w.shapes), C.byref(h))
@@ -94,10 +95,19 @@ def test_tile_groups_bound_the_workspace():
         sizes[gt] = (st.value, ws.value)
         L.lib().shampoo4_destroy(h)
     state = sizes[0][0]
-    assert sizes[100000][1] > 80e9
-    assert sizes[0][1] < 0.25 * sizes[100000][1]
+    assert sizes[100000][1] > 80e9 and sizes[0][1] == sizes[100000][1]
+    assert sizes[48][1] < 0.25 * sizes[100000][1]
     assert sizes[16][1] < 1.5 * state
-    assert sizes[1][1] < sizes[16][1] < sizes[0][1]
+    assert sizes[1][1] < sizes[16][1] < sizes[48][1]
+    twice = list(w.shapes) * 2
+    p2 = (L.Param * len(twice))(*[L.Param(r, c) for r, c in twice])
+    cfg = L.Config(0.95, 1e-6, 1024, 64, 5, 0, 0, 0, 1, 0, 0, 0, 0)
+    h = C.c_void_p()
+    L.call("shampoo4_init", C.byref(cfg), p2, len(twice), C.byref(h))
+    ws = C.c_size_t()
+    L.call("shampoo4_sizes", h, None, C.byref(ws))
+    assert ws.value < 20e9                      # grouped: two slots of at most 8 GiB
+    L.lib().shampoo4_destroy(h)
     cfg = L.Config(0.95, 1e-6, 1024, 64, 5, 0, 0, 0, 1, 0, 0, 0, -1)
     h = C.c_void_p()
     assert L.lib().shampoo4_init(C.byref(cfg), params, len(w.shapes), C.byref(h)) == 1
