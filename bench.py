@@ -541,7 +541,6 @@ def main():
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    L.call("shampoo4_timing_enable", sh._h, 1)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -562,7 +561,14 @@ def main():
     # one step together
     value = args.steps / (ms / 1e3) if shard else job_rate(world, args.steps, ms)
 
-    # per-stage times measured live over the timed region
+    # per-stage times: the library's launch timing (an event pair around
+    # every launch) over separate steps after the timed region, so that the
+    # timed steps carry no instrumentation
+    tsteps = max(1, min(3, args.steps))
+    L.call("shampoo4_timing_enable", sh._h, 1)
+    for _ in range(tsteps):
+        step()
+    torch.cuda.synchronize()
     stages = {}
     launches = 0
     s = 0
@@ -574,9 +580,9 @@ def main():
         L.call("shampoo4_timing_read", sh._h, s, C.byref(t_ms), C.byref(n), C.byref(fl), C.byref(by))
         s += 1
         if n.value:
-            stages[name] = {"ms": t_ms.value / args.steps, "launches": n.value // args.steps,
-                            "flops": fl.value / args.steps, "bytes": by.value / args.steps}
-            launches += n.value
+            stages[name] = {"ms": t_ms.value / tsteps, "launches": n.value // tsteps,
+                            "flops": fl.value / tsteps, "bytes": by.value / tsteps}
+            launches += n.value // tsteps
     L.call("shampoo4_timing_enable", sh._h, 0)
     status = sh.status_flags()
 
@@ -631,14 +637,15 @@ def main():
                               f"of fp32 statistics; L2 is 0.126 GB)")},
             "root_refreshes_per_s": value * sh.nfactors,
             "status_flags": status,
-            "gpu_launches": launches,
+            "gpu_launches": launches * args.steps,
             "clocks": clocks, "roofline": roof, "rooflines_other": others,
-            "stages_ms": {k: round(v["ms"], 4) for k, v in sorted(stages.items(), key=lambda kv: -kv[1]["ms"])}}
+            "stages_ms": {k: round(v["ms"], 4) for k, v in sorted(stages.items(), key=lambda kv: -kv[1]["ms"])},
+            "stages_note": f"launch durations per step over {tsteps} step(s) after the timed region"}
 
-    # the same refresh as one launch sequence on the caller's stream (the
-    # handle's default splits it in two concurrent parts): the split's gain
+    # the same refresh split into two cost-balanced parts on the handle's
+    # two streams (the default is one launch sequence)
     if not shard:
-        L.call("shampoo4_debug_refresh_parts", sh._h, 1)
+        L.call("shampoo4_debug_refresh_parts", sh._h, 2)
         sh.bind(reset=False)
         for _ in range(2):
             step()
@@ -649,8 +656,8 @@ def main():
             sh.refresh_roots()
         r1.record(stream)
         torch.cuda.synchronize()
-        line["config"]["refresh_ms_one_part"] = r0.elapsed_time(r1) / 3
-        L.call("shampoo4_debug_refresh_parts", sh._h, 2)
+        line["config"]["refresh_ms_two_parts"] = r0.elapsed_time(r1) / 3
+        L.call("shampoo4_debug_refresh_parts", sh._h, 1)
         sh.bind(reset=False)
 
     # end to end through the public API with host buffers: every step copies

@@ -84,9 +84,9 @@ __device__ __forceinline__ void load_group(const PackTensor& t, int64_t e0, floa
 // Quantize one loaded group (all lanes of the warp call this together) and
 // store its codes and, from the block's first lane, its scale.
 __device__ __forceinline__ void pack_group(const PackTensor& t, int64_t e0, const float (&v)[8], uint32_t valid,
-                                           const float* thr) {
+                                           const float2* bucket) {
   float s;
-  uint32_t packed = quantize8(v, valid, thr, &s);
+  uint32_t packed = quantize8(v, valid, bucket, &s);
   if ((threadIdx.x & 7) == 0 && e0 < t.n) t.scales[e0 / kQuantBlock] = s;
   if (valid == 0) return;
   int64_t byte0 = e0 >> 1;
@@ -119,7 +119,7 @@ k_quant4_pack(const __grid_constant__ PackBatch b) {
 #pragma unroll
   for (int g = 0; g < kCodecGroupsPerThread; ++g) {
     const int64_t e0 = e_base + (int64_t(g) * kCodecThreads + threadIdx.x) * 8;
-    pack_group(t, e0, v[g], valid[g], sm.thr);
+    pack_group(t, e0, v[g], valid[g], sm.bucket);
   }
 }
 

@@ -11,29 +11,64 @@
 
 namespace s4 {
 
-// Thresholds t_0..t_14 (t_15 = +Inf) and the 16 levels of one codebook, in
-// shared memory.
+// The code decision by buckets.  Both codebooks are symmetric (t_7 = 0,
+// t_14-k = -t_k), so with a = |v| the count of thresholds below v is
+//   v > 0:  8 + #{j >= 8 : a > t_j}          v <= 0 (or NaN):  7 - #{j >= 8 : a >= t_j}
+// and for a in [0, 1] the positive thresholds are found by bucket: the
+// bits of a above bit 20 (exponent and three mantissa bits) index 64
+// buckets over [2^-8, 1), each holding at most one positive threshold of
+// either codebook.  Bucket i stores (t, n): that threshold (NaN if none)
+// and the number of positive thresholds below the bucket, so
+//   #{a > t_j} = n + (a > t),   #{a >= t_j} = n + (a >= t).
+// Entry 0 takes everything below 2^-8 (no threshold there: n = 0), entry 65
+// everything from 1 up, infinities and NaN (n = 7, t = NaN), which gives
+// 15 for +Inf, 0 for -Inf and NaN, as the count rule does.  Checked against
+// the count rule on every fp32 value in [-1, 1] of both codebooks.
+constexpr uint32_t kBucketBase = 0x3B8u;        // bits(2^-8) >> 20
+constexpr int kBuckets = 66;
+
+// Thresholds t_0..t_14 (t_15 = +Inf), the 16 levels of one codebook and
+// the bucket table, in shared memory.
 struct CodecSmem {
   float thr[16];
   float level[16];
+  float2 bucket[kBuckets];                      // (t, the bits of the integer n)
 };
 
+// Fill the tables (threads 0..65 of the block); the caller synchronizes.
 __device__ __forceinline__ void codec_smem_init(CodecSmem& sm, int codebook) {
-  if (threadIdx.x < 16) {
-    int j = threadIdx.x;
+  const int j = threadIdx.x;
+  if (j < 16) {
     sm.level[j] = level_f32(codebook, j);
     sm.thr[j] = j < 15 ? threshold_f32(codebook, j) : __int_as_float(0x7f800000);
   }
+  if (j < kBuckets) {
+    float t = __int_as_float(0x7fc00000);
+    int n = 7;
+    if (j == 0) {
+      n = 0;
+    } else if (j < kBuckets - 1) {
+      const float lo = __uint_as_float((kBucketBase + j - 1) << 20);
+      const float hi = __uint_as_float((kBucketBase + j) << 20);
+      n = 0;
+      for (int k = 8; k < 15; ++k) {
+        const float tk = threshold_f32(codebook, k);
+        if (tk < lo) ++n;
+        else if (tk < hi) t = tk;
+      }
+    }
+    sm.bucket[j] = make_float2(t, __int_as_float(n));
+  }
 }
 
-// code = number of thresholds strictly below v (t sorted ascending), by a
-// 4-step binary search.  NaN compares false everywhere and gives 0.
-__device__ __forceinline__ uint32_t code_of(float v, const float* thr) {
-  uint32_t c = (v > thr[7]) ? 8u : 0u;
-  c += (v > thr[c + 3]) ? 4u : 0u;
-  c += (v > thr[c + 1]) ? 2u : 0u;
-  c += (v > thr[c]) ? 1u : 0u;
-  return c;
+// code = number of thresholds t_k strictly below v, by the buckets above.
+__device__ __forceinline__ uint32_t code_bucket(float v, const float2* bucket) {
+  const uint32_t ab = __float_as_uint(v) & 0x7fffffffu;
+  const uint32_t i = min(max(ab >> 20, kBucketBase - 1u), kBucketBase + 64u) - (kBucketBase - 1u);
+  const float2 e = bucket[i];
+  const float a = __uint_as_float(ab);
+  const int n = __float_as_int(e.y);
+  return v > 0.0f ? uint32_t(8 + n + (a > e.x ? 1 : 0)) : uint32_t(7 - n - (a >= e.x ? 1 : 0));
 }
 
 // IEEE round-to-nearest x / s for a block that shares one divisor s.
@@ -70,7 +105,7 @@ __device__ __forceinline__ uint32_t absmax_bits8(const float (&v)[8]) {
 // infinity and no NaN.  Lanes whose elements lie past the end pass zeros and
 // a valid mask of 0 for those elements; their codes are forced to 0.
 __device__ __forceinline__ uint32_t quantize8(const float (&v)[8], uint32_t valid_mask,
-                                              const float* thr, float* scale) {
+                                              const float2* bucket, float* scale) {
   uint32_t m = absmax_bits8(v);
 #pragma unroll
   for (int off = 4; off >= 1; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
@@ -90,7 +125,7 @@ __device__ __forceinline__ uint32_t quantize8(const float (&v)[8], uint32_t vali
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     float q = fast ? div_rn_shared(v[e], s, r) : __fdiv_rn(v[e], s);
-    uint32_t c = code_of(q, thr);
+    uint32_t c = code_bucket(q, bucket);
     c = ((valid_mask >> e) & 1u) ? c : 0u;
     packed |= c << (4 * e);
   }

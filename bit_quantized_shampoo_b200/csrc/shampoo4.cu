@@ -130,7 +130,7 @@ struct shampoo4_ctx {
   // call runs group g on the handle's stream g mod 2.
   Program prog_stats, prog_stats_first, prog_refresh_first, prog_refresh, prog_precond;
   static constexpr int kMaxParts = 2;
-  int refresh_parts = kMaxParts;           // requested (shampoo4_debug_refresh_parts)
+  int refresh_parts = 1;                   // requested (shampoo4_debug_refresh_parts)
   cudaStream_t part_stream[kMaxParts] = {};
   cudaEvent_t part_fork = nullptr, part_join[kMaxParts] = {};
   std::vector<uint8_t> arena;            // host image of the descriptor region
@@ -956,40 +956,54 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
   {
     // Gram W = X^T X (lower triangle: fp32 into W, its TF32 split into
     // Th/Tl), optional shift
-    std::vector<TcGemmDesc> g;
+    // The gated pass first runs a Gram that only sums its deviation from I
+    // (no outputs: on warm refreshes every factor passes the gate, so the
+    // matrices would never be read), then the Gram with outputs for the
+    // factors the gate sends through the pass.
+    std::vector<TcGemmDesc> g, gg;
     std::vector<ShiftDescF> sd;
     std::vector<GateDesc> gd;
-    std::vector<DiagDesc> dg;
+    std::vector<DiagDesc> dg, dgg;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
       if (!f.tc) continue;
       const int d = f.d;
       TcGemmDesc w = gemmtc(d, d, d, 1.0f, 0.0f);
+      w.a = b.operand(X[i].h, X[i].l, d, d, true, true, true);
+      w.b = b.operand(X[i].h, X[i].l, d, d, false, false, true, kSquareBN);
+      w.symmetric = 2;
+      w.skip = b.tcbad(i);
       if (gated) {
-        w.devsq = b.devsq(i);
+        TcGemmDesc dev = w;                                           // deviation only
+        dev.devsq = b.devsq(i);
+        gg.push_back(dev);
+        dgg.push_back({X[i].m, b.wf(f.ws_W), d, d, 0, b.devsq(i), b.tcbad(i)});
         const double tol = kLastPassTol * std::sqrt(double(d));        // on ||Q^T Q - I||_F / sqrt(d)
         const double thr = std::min(tol * tol * d * double(kDevFineUnit), 0x1p62);
         gd.push_back({b.devsq(i), b.tcbad(i), b.skip3(i), static_cast<unsigned long long>(thr)});
+        w.skip = b.skip3(i);
       }
-      w.a = b.operand(X[i].h, X[i].l, d, d, true, true, true);
-      w.b = b.operand(X[i].h, X[i].l, d, d, false, false, true, kSquareBN);
       // only the lower triangles of W and of its TF32 split are ever read
       // (Cholesky blocks, panel updates, and the first panel's L21 product,
       // which takes W21 from the split): no mirror stores
       w.C = b.wf(f.ws_W); w.ldc = d;
       w.Chi = b.wf(f.ws_Th); w.Clo = b.wf(f.ws_Tl); w.ldh = d;
-      w.symmetric = 2;
-      w.skip = b.tcbad(i);
       g.push_back(w);
-      dg.push_back({X[i].m, b.wf(f.ws_W), d, d, 0, gated ? b.devsq(i) : nullptr, b.tcbad(i)});
+      dg.push_back({X[i].m, b.wf(f.ws_W), d, d, 0, nullptr, gated ? b.skip3(i) : b.tcbad(i)});
       if (shifted) sd.push_back({b.wf(f.ws_W), d, d, kTcShift * float(d), b.tcbad(i)});
+    }
+    auto elems = [](const std::vector<DiagDesc>& v) { double s = 0; for (auto& x : v) s += double(x.d) * x.d; return s; };
+    if (gated) {
+      b.tag = SHAMPOO4_STAGE_QR_GRAM;
+      emit_gemmtc(b, prog, gg, true, kSquareBN);
+      b.emit(prog, Kind::Diag, dgg, dmax, 0, 4.0 * elems(dgg));
+      b.tag = SHAMPOO4_STAGE_QR_CONVERT;
+      b.emit(prog, Kind::Gate, gd, 0);
     }
     b.tag = SHAMPOO4_STAGE_QR_GRAM;
     emit_gemmtc(b, prog, g, true, kSquareBN);
-    b.emit(prog, Kind::Diag, dg, dmax, 0, 4.0 * [&] { double s = 0; for (auto& x : dg) s += double(x.d) * x.d; return s; }());
+    b.emit(prog, Kind::Diag, dg, dmax, 0, 4.0 * elems(dg));
     b.emit(prog, Kind::ShiftF, sd, 0);
-    b.tag = SHAMPOO4_STAGE_QR_CONVERT;
-    b.emit(prog, Kind::Gate, gd, 0);
   }
   // the rest of the pass: skipped for a broken-down factor, and for a
   // factor the gate passed

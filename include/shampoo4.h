@@ -312,8 +312,9 @@ shampoo4_status shampoo4_debug_capture(shampoo4_handle h, void* d_buf);
 shampoo4_status shampoo4_debug_capture_layout(shampoo4_handle h, int32_t factor, size_t* off_u,
                                               size_t* off_q);
 
-/* Diagnostic: how many parts the refresh is split into (1 or 2; default 2).
- * The factors are dealt to the parts by d^3 cost, and the parts' launch
+/* Diagnostic: how many parts the refresh of a one-group handle is split
+ * into (1 or 2; default 1: on the Llama layer set two parts measured no
+ * faster).  The factors are dealt to the parts by d^3 cost, and the parts' launch
  * sequences run concurrently on the handle's own CUDA streams, forked from
  * and joined back to the caller's stream (so a graph captured on the
  * caller's stream captures them too).  Each factor's arithmetic does not
