@@ -33,6 +33,7 @@ struct PackTensor {
 struct PackBatch {
   int32_t count;
   int32_t codebook;
+  CodecTables tables;
   PackTensor t[kCodecMaxBatch];
 };
 
@@ -48,8 +49,16 @@ struct UnpackTensor {
 struct UnpackBatch {
   int32_t count;
   int32_t codebook;
+  CodecTables tables;
   UnpackTensor t[kCodecMaxBatch];
 };
+
+// The tables of each codebook, built once on the host.
+const CodecTables& host_tables(int codebook) {
+  static const CodecTables t[kCodebookCount] = {make_codec_tables(kCodebookLinearSquare),
+                                               make_codec_tables(kCodebookDynamicTree)};
+  return t[codebook];
+}
 
 template <class B>
 __device__ __forceinline__ int find_tensor(const B& b, int64_t cta) {
@@ -103,7 +112,7 @@ __device__ __forceinline__ void pack_group(const PackTensor& t, int64_t e0, cons
 __global__ void __launch_bounds__(kCodecThreads)
 k_quant4_pack(const __grid_constant__ PackBatch b) {
   __shared__ CodecSmem sm;
-  codec_smem_init(sm, b.codebook);
+  codec_smem_init(sm, b.tables);
   const PackTensor& t = b.t[find_tensor(b, blockIdx.x)];
   const int64_t e_base = (int64_t(blockIdx.x) - t.cta_begin) * kCodecEltsPerCta;
   const bool skip = t.skip && *t.skip;
@@ -154,7 +163,7 @@ __device__ __forceinline__ void unpack_group(const UnpackTensor& t, int64_t e0, 
 __global__ void __launch_bounds__(kCodecThreads)
 k_quant4_unpack(const __grid_constant__ UnpackBatch b) {
   __shared__ CodecSmem sm;
-  codec_smem_init(sm, b.codebook);
+  codec_smem_init(sm, b.tables);
   __syncthreads();
   const UnpackTensor& t = b.t[find_tensor(b, blockIdx.x)];
   int64_t e_base = (int64_t(blockIdx.x) - t.cta_begin) * kCodecEltsPerCta;
@@ -175,6 +184,7 @@ shampoo4_status launch_pack(const float* const* x, const int64_t* n, int32_t cou
     PackBatch b;
     b.count = 0;
     b.codebook = codebook;
+    b.tables = host_tables(codebook);
     int64_t ctas = 0;
     for (int32_t i = base; i < count && i < base + kCodecMaxBatch; ++i) {
       if (n[i] == 0) continue;
@@ -202,6 +212,7 @@ shampoo4_status launch_unpack(const uint8_t* const* codes, const float* const* s
     UnpackBatch b;
     b.count = 0;
     b.codebook = codebook;
+    b.tables = host_tables(codebook);
     int64_t ctas = 0;
     for (int32_t i = base; i < count && i < base + kCodecMaxBatch; ++i) {
       if (n[i] == 0) continue;

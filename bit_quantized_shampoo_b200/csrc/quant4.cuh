@@ -7,6 +7,7 @@
 // own one block, 8 elements each, so the block's absmax is a 3-step
 // xor-shuffle inside each 8-lane segment.
 #pragma once
+#include <string.h>
 #include "common.cuh"
 
 namespace s4 {
@@ -27,29 +28,32 @@ namespace s4 {
 constexpr uint32_t kBucketBase = 0x3B8u;        // bits(2^-8) >> 20
 constexpr int kBuckets = 66;
 
-// Thresholds t_0..t_14 (t_15 = +Inf), the 16 levels of one codebook and
-// the bucket table, in shared memory.
-struct CodecSmem {
-  float thr[16];
+// The tables of one codebook: its 16 levels, the bucket table above, and
+// the 15 thresholds (t_15 = +Inf).  Built once on the host
+// (codec_tables), passed in the launch parameters and copied to shared
+// memory by each CTA.
+struct CodecTables {
   float level[16];
+  float thr[16];
   float2 bucket[kBuckets];                      // (t, the bits of the integer n)
 };
 
-// Fill the tables (threads 0..65 of the block); the caller synchronizes.
-__device__ __forceinline__ void codec_smem_init(CodecSmem& sm, int codebook) {
-  const int j = threadIdx.x;
-  if (j < 16) {
-    sm.level[j] = level_f32(codebook, j);
-    sm.thr[j] = j < 15 ? threshold_f32(codebook, j) : __int_as_float(0x7f800000);
+__host__ __device__ inline CodecTables make_codec_tables(int codebook) {
+  CodecTables c{};
+  for (int j = 0; j < 16; ++j) {
+    c.level[j] = level_f32(codebook, j);
+    c.thr[j] = j < 15 ? threshold_f32(codebook, j) : __builtin_huge_valf();
   }
-  if (j < kBuckets) {
-    float t = __int_as_float(0x7fc00000);
+  for (int j = 0; j < kBuckets; ++j) {
+    float t = __builtin_nanf("");
     int n = 7;
     if (j == 0) {
       n = 0;
     } else if (j < kBuckets - 1) {
-      const float lo = __uint_as_float((kBucketBase + j - 1) << 20);
-      const float hi = __uint_as_float((kBucketBase + j) << 20);
+      const uint32_t lo_bits = (kBucketBase + j - 1) << 20, hi_bits = (kBucketBase + j) << 20;
+      float lo, hi;
+      memcpy(&lo, &lo_bits, 4);
+      memcpy(&hi, &hi_bits, 4);
       n = 0;
       for (int k = 8; k < 15; ++k) {
         const float tk = threshold_f32(codebook, k);
@@ -57,8 +61,21 @@ __device__ __forceinline__ void codec_smem_init(CodecSmem& sm, int codebook) {
         else if (tk < hi) t = tk;
       }
     }
-    sm.bucket[j] = make_float2(t, __int_as_float(n));
+    float nb;
+    memcpy(&nb, &n, 4);
+    c.bucket[j] = make_float2(t, nb);
   }
+  return c;
+}
+
+using CodecSmem = CodecTables;
+
+// Copy the tables (a CodecTables in the launch parameters) to shared
+// memory; the caller synchronizes.
+__device__ __forceinline__ void codec_smem_init(CodecSmem& sm, const CodecTables& src) {
+  const uint32_t* a = reinterpret_cast<const uint32_t*>(&src);
+  uint32_t* b = reinterpret_cast<uint32_t*>(&sm);
+  for (int i = threadIdx.x; i < int(sizeof(CodecTables) / 4); i += blockDim.x) b[i] = a[i];
 }
 
 // code = number of thresholds t_k strictly below v, by the buckets above.

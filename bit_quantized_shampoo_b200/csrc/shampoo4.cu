@@ -2048,11 +2048,15 @@ extern "C" shampoo4_status shampoo4_init(const shampoo4_config* cfg, const shamp
   // Tensor-map and descriptor bytes: build the programs once against a null
   // base (maps counted, not encoded) to size both regions; bind rebuilds
   // them with the real addresses.
+  // (sized with the most refresh parts: a split program never needs less)
   Builder b{h, h->arena, nullptr, nullptr, false};
+  const int parts = h->refresh_parts;
+  h->refresh_parts = shampoo4_ctx::kMaxParts;
   build_stats(b);
   build_refresh(b, h->prog_refresh_first, true);
   build_refresh(b, h->prog_refresh, false);
   build_precondition(b);
+  h->refresh_parts = parts;
   h->ws_nmaps = h->maps.size();
   h->ws_desc = align_up(h->ws_maps + h->ws_nmaps * sizeof(CUtensorMap), kAlign);
   h->ws_desc_bytes = align_up(h->arena.size(), kAlign);
