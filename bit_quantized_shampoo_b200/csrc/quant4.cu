@@ -3,13 +3,17 @@
 // block-wise linear square quantization; the dynamic tree map is the
 // alternative codebook).
 //
-// Memory-bound.  One CTA of 256 threads covers 8192 consecutive elements of
-// one tensor (128 quantization blocks); each thread owns two groups of 8
+// Memory-bound.  One CTA of 256 threads covers 4096 consecutive elements of
+// one tensor (64 quantization blocks); each thread owns two groups of 8
 // elements and issues both groups' loads before it computes either.  8
-// consecutive lanes own one block.  (Measured on a 1 GiB tensor: four
-// groups per thread, persistent grid-stride loops with the next group's
-// loads in flight, and immediate-operand threshold searches were all
-// slower; their register use costs more occupancy than they save.)
+// consecutive lanes own one block.  A warp whose blocks all have a scale in
+// [2^-60, 1] and no missing elements takes the code decision by signed
+// buckets: one byte per bucket in shared memory (broadcast-friendly, almost
+// free of bank conflicts) and the threshold by a shuffle from the lane that
+// holds it; any other warp takes the general decision (quantize8).
+// (Measured on a 1 GiB tensor: four groups per thread and persistent
+// grid-stride loops were slower; a float2 table of 129 to 513 entries lost
+// to bank conflicts.)
 #include "quant4.cuh"
 #include "plan.h"
 
@@ -17,7 +21,7 @@ namespace s4 {
 
 constexpr int kCodecThreads = 256;
 constexpr int kCodecGroupsPerThread = 2;
-constexpr int kCodecEltsPerCta = kCodecThreads * 8 * kCodecGroupsPerThread;   // 8192
+constexpr int kCodecEltsPerCta = kCodecThreads * 8 * kCodecGroupsPerThread;   // 4096
 constexpr int kCodecMaxBatch = 64;
 
 struct PackTensor {
@@ -34,6 +38,7 @@ struct PackBatch {
   int32_t count;
   int32_t codebook;
   CodecTables tables;
+  SignedBuckets sb;
   PackTensor t[kCodecMaxBatch];
 };
 
@@ -57,6 +62,11 @@ struct UnpackBatch {
 const CodecTables& host_tables(int codebook) {
   static const CodecTables t[kCodebookCount] = {make_codec_tables(kCodebookLinearSquare),
                                                make_codec_tables(kCodebookDynamicTree)};
+  return t[codebook];
+}
+const SignedBuckets& host_signed_buckets(int codebook) {
+  static const SignedBuckets t[kCodebookCount] = {make_signed_buckets(kCodebookLinearSquare),
+                                                 make_signed_buckets(kCodebookDynamicTree)};
   return t[codebook];
 }
 
@@ -91,12 +101,22 @@ __device__ __forceinline__ void load_group(const PackTensor& t, int64_t e0, floa
 }
 
 // Quantize one loaded group (all lanes of the warp call this together) and
-// store its codes and, from the block's first lane, its scale.
+// store its codes and, from the block's first lane, its scale.  FULL: the
+// group lies inside the tensor, x is 16-byte and codes 4-byte aligned.
+template <int SHIFT, bool FULL>
 __device__ __forceinline__ void pack_group(const PackTensor& t, int64_t e0, const float (&v)[8], uint32_t valid,
-                                           const float2* bucket) {
-  float s;
-  uint32_t packed = quantize8(v, valid, bucket, &s);
-  if ((threadIdx.x & 7) == 0 && e0 < t.n) t.scales[e0 / kQuantBlock] = s;
+                                           const uint8_t* below, float t_lane, const float2* bucket) {
+  float s = block_absmax_nan(v);
+  uint32_t packed;
+  if (__all_sync(0xffffffffu, (FULL || valid == 0xffu) && s >= 0x1p-60f && s <= 1.0f))   // warp-uniform
+    packed = quantize8_signed<SHIFT>(v, s, below, t_lane);
+  else
+    packed = quantize8(v, FULL ? 0xffu : valid, bucket, &s);
+  if ((threadIdx.x & 7) == 0 && (FULL || e0 < t.n)) t.scales[e0 / kQuantBlock] = s;
+  if (FULL) {
+    *reinterpret_cast<uint32_t*>(t.codes + (e0 >> 1)) = packed;
+    return;
+  }
   if (valid == 0) return;
   int64_t byte0 = e0 >> 1;
   if (t.vec_codes && valid == 0xffu) {
@@ -109,27 +129,53 @@ __device__ __forceinline__ void pack_group(const PackTensor& t, int64_t e0, cons
   }
 }
 
-__global__ void __launch_bounds__(kCodecThreads)
-k_quant4_pack(const __grid_constant__ PackBatch b) {
-  __shared__ CodecSmem sm;
-  codec_smem_init(sm, b.tables);
-  const PackTensor& t = b.t[find_tensor(b, blockIdx.x)];
-  const int64_t e_base = (int64_t(blockIdx.x) - t.cta_begin) * kCodecEltsPerCta;
-  const bool skip = t.skip && *t.skip;
+template <int SHIFT, bool FULL>
+__device__ __forceinline__ void pack_cta(const PackTensor& t, int64_t e_base, bool skip, const uint8_t* below,
+                                         float t_lane, const float2* bucket) {
   float v[kCodecGroupsPerThread][8];
   uint32_t valid[kCodecGroupsPerThread];
 #pragma unroll
   for (int g = 0; g < kCodecGroupsPerThread; ++g) {
     const int64_t e0 = e_base + (int64_t(g) * kCodecThreads + threadIdx.x) * 8;
-    load_group(t, skip ? t.n : e0, v[g], valid[g]);
+    if (FULL) {
+      const float4* p = reinterpret_cast<const float4*>(t.x + e0);
+      const float4 a = __ldg(p), c = __ldg(p + 1);
+      v[g][0] = a.x; v[g][1] = a.y; v[g][2] = a.z; v[g][3] = a.w;
+      v[g][4] = c.x; v[g][5] = c.y; v[g][6] = c.z; v[g][7] = c.w;
+      valid[g] = 0xffu;
+    } else {
+      load_group(t, skip ? t.n : e0, v[g], valid[g]);
+    }
   }
-  __syncthreads();                                      // the tables
+  __syncthreads();                                      // the bucket bytes
   if (skip) return;                                     // CTA-uniform
 #pragma unroll
   for (int g = 0; g < kCodecGroupsPerThread; ++g) {
     const int64_t e0 = e_base + (int64_t(g) * kCodecThreads + threadIdx.x) * 8;
-    pack_group(t, e0, v[g], valid[g], sm.bucket);
+    pack_group<SHIFT, FULL>(t, e0, v[g], valid[g], below, t_lane, bucket);
   }
+}
+
+// SHIFT = signed_bucket_shift(b.codebook).  The general decision reads its
+// bucket table from the launch parameters (rare: ragged ends, scales
+// outside [2^-60, 1], NaN and infinities).  A CTA whose 4096 elements all
+// lie inside an aligned tensor takes the unchecked loads and stores.
+template <int SHIFT>
+__global__ void __launch_bounds__(kCodecThreads)
+k_quant4_pack(const __grid_constant__ PackBatch b) {
+  constexpr int kWords = (signed_bucket_count(SHIFT) + 3) / 4;
+  __shared__ uint32_t below[kWords];
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(b.sb.below);
+  for (int i = threadIdx.x; i < kWords; i += kCodecThreads) below[i] = src[i];
+  const float t_lane = b.tables.thr[threadIdx.x & 15];
+  const PackTensor t = b.t[find_tensor(b, blockIdx.x)];
+  const int64_t e_base = (int64_t(blockIdx.x) - t.cta_begin) * kCodecEltsPerCta;
+  const bool skip = t.skip && *t.skip;
+  const uint8_t* bl = reinterpret_cast<const uint8_t*>(below);
+  if (!skip && t.vec_x && t.vec_codes && e_base + kCodecEltsPerCta <= t.n)
+    pack_cta<SHIFT, true>(t, e_base, false, bl, t_lane, b.tables.bucket);
+  else
+    pack_cta<SHIFT, false>(t, e_base, skip, bl, t_lane, b.tables.bucket);
 }
 
 __device__ __forceinline__ void unpack_group(const UnpackTensor& t, int64_t e0, const float* level) {
@@ -185,6 +231,8 @@ shampoo4_status launch_pack(const float* const* x, const int64_t* n, int32_t cou
     b.count = 0;
     b.codebook = codebook;
     b.tables = host_tables(codebook);
+    b.sb = host_signed_buckets(codebook);
+    if (!b.sb.ok) return SHAMPOO4_ERR_INVALID_ARG;           // no codebook in use has such a bucket
     int64_t ctas = 0;
     for (int32_t i = base; i < count && i < base + kCodecMaxBatch; ++i) {
       if (n[i] == 0) continue;
@@ -198,7 +246,8 @@ shampoo4_status launch_pack(const float* const* x, const int64_t* n, int32_t cou
     }
     if (b.count == 0) continue;
     if (ctas > 0x7fffffffLL) return SHAMPOO4_ERR_INVALID_ARG;
-    k_quant4_pack<<<unsigned(ctas), kCodecThreads, 0, st>>>(b);
+    if (b.sb.shift == 14) k_quant4_pack<14><<<unsigned(ctas), kCodecThreads, 0, st>>>(b);
+    else k_quant4_pack<16><<<unsigned(ctas), kCodecThreads, 0, st>>>(b);
     S4_CUDA(cudaGetLastError());
     if (launched) ++*launched;
   }

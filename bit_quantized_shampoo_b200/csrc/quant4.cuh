@@ -68,6 +68,54 @@ __host__ __device__ inline CodecTables make_codec_tables(int codebook) {
   return c;
 }
 
+// The code decision of the common case, by signed buckets.  For q in
+// [-1, 1], qb = RN(q + 3) lies in [2, 4]; its bits above bit SHIFT index
+// uniform buckets of width 2^(SHIFT - 22) (129 for SHIFT = 16, 513 for 14),
+// monotone in q, each holding at most one threshold of the codebook.  With
+// c0 = the number of thresholds in lower buckets (one byte per bucket), the
+// thresholds are sorted, so the only one that can lie in q's bucket is
+// t_c0, and
+//   code = #{k : q > t_k} = c0 + (q > t_c0),   t_15 = +Inf,
+// exactly, whatever the rounding of q + 3 (only its monotonicity is used).
+// The width must stay below the smallest gap between thresholds: 0.022 for
+// linear square (SHIFT 16: 2^-6), 0.005 for the dynamic tree (SHIFT 14:
+// 2^-8).  make_signed_buckets reports a bucket with two thresholds.
+__host__ __device__ constexpr int signed_bucket_shift(int codebook) {
+  return codebook == kCodebookDynamicTree ? 14 : 16;
+}
+__host__ __device__ constexpr int signed_bucket_count(int shift) {
+  return int((0x40800000u >> shift) - (0x40000000u >> shift)) + 1;
+}
+constexpr int kSignedBucketBytes = 516;         // signed_bucket_count(14), padded to words
+struct SignedBuckets {
+  uint8_t below[kSignedBucketBytes];            // c0 of each bucket
+  int32_t shift;
+  int32_t ok;                                   // 0 if some bucket holds two thresholds
+};
+
+__host__ __device__ inline uint32_t signed_bucket_of(float q, int shift) {
+  const float qb = q + 3.0f;
+  uint32_t b;
+  memcpy(&b, &qb, 4);
+  return (b >> shift) - (0x40000000u >> shift);
+}
+
+__host__ __device__ inline SignedBuckets make_signed_buckets(int codebook) {
+  SignedBuckets sb{};
+  sb.shift = signed_bucket_shift(codebook);
+  sb.ok = 1;
+  uint32_t kb[15];
+  for (int j = 0; j < 15; ++j) kb[j] = signed_bucket_of(threshold_f32(codebook, j), sb.shift);
+  for (int j = 1; j < 15; ++j)
+    if (kb[j] == kb[j - 1]) sb.ok = 0;
+  for (int k = 0; k < signed_bucket_count(sb.shift); ++k) {
+    int c0 = 0;
+    for (int j = 0; j < 15; ++j) c0 += kb[j] < uint32_t(k) ? 1 : 0;
+    sb.below[k] = uint8_t(c0);
+  }
+  return sb;
+}
+
 using CodecSmem = CodecTables;
 
 // Copy the tables (a CodecTables in the launch parameters) to shared
@@ -145,6 +193,54 @@ __device__ __forceinline__ uint32_t quantize8(const float (&v)[8], uint32_t vali
     uint32_t c = code_bucket(q, bucket);
     c = ((valid_mask >> e) & 1u) ? c : 0u;
     packed |= c << (4 * e);
+  }
+  return packed;
+}
+
+// max(|a|, |b|, |c|), NaN if any operand is NaN.
+__device__ __forceinline__ float absmax3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
+  return d;
+}
+__device__ __forceinline__ float max2_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+// The absmax of the block (the aligned 8-lane segment's 64 values) as a
+// float: NaN if the block holds a NaN.  All 32 lanes call it together.
+__device__ __forceinline__ float block_absmax_nan(const float (&v)[8]) {
+  float m = max2_nan(absmax3_nan(v[0], v[1], v[2]), absmax3_nan(v[3], v[4], v[5]));
+  m = max2_nan(m, max2_nan(fabsf(v[6]), fabsf(v[7])));
+#pragma unroll
+  for (int off = 4; off >= 1; off >>= 1) m = max2_nan(m, __shfl_xor_sync(0xffffffffu, m, off));
+  return m;
+}
+
+// Quantize 8 values of a block with scale s in [2^-60, 1] (so |q| <= 1 and
+// no NaN), all elements valid.  below: the signed-bucket bytes in shared
+// memory; t_lane: threshold t_(lane mod 16) of the codebook (t_15 = +Inf)
+// held by each lane, fetched by a shuffle.  All 32 lanes call it together.
+// The quotient is Markstein's sequence without the small-operand test: for
+// |x| >= 2^-100 it is the IEEE quotient, below that a quotient under 2^-30
+// with the IEEE quotient's sign (+0 and -0 both counting as not positive),
+// and the code of such a quotient depends on its sign alone.
+template <int SHIFT>
+__device__ __forceinline__ uint32_t quantize8_signed(const float (&v)[8], float s, const uint8_t* below,
+                                                     float t_lane) {
+  constexpr uint32_t off = 0x40000000u >> SHIFT;
+  const float r = __frcp_rn(s);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float q0 = v[e] * r;
+    const float q = fmaf(fmaf(-q0, s, v[e]), r, q0);
+    const float qb = q + 3.0f;
+    const uint32_t c0 = below[(__float_as_uint(qb) >> SHIFT) - off];
+    const float t = __shfl_sync(0xffffffffu, t_lane, int(c0));
+    packed += (c0 + (q > t ? 1u : 0u)) << (4 * e);
   }
   return packed;
 }

@@ -64,3 +64,53 @@ def test_bucket_rule_equals_the_count_rule(cbk):
     v = np.concatenate(vals).astype(np.float32)
     v = np.concatenate([v, -v, np.float32([np.nan, -np.nan, np.inf, -np.inf, 0.0, -0.0, 1.0, -1.0])])
     assert np.array_equal(_bucket_codes(v, nb, tb), _rule(v, t))
+
+
+# ---- the signed buckets of the common case (quant4.cuh, quantize8_signed) --
+#
+# For q in [-1, 1]: qb = float32(q + 3) in [2, 4]; bucket k = (bits(qb) >>
+# SHIFT) - (bits(2.0) >> SHIFT); c0[k] = the number of thresholds whose own
+# bucket is below k; code = c0 + (q > t[c0]) with t[15] = +Inf.  SHIFT is
+# 16 for linear square and 14 for the dynamic tree.  (Run once over all
+# 2.1e9 fp32 values of [-1, 1] for both codebooks: no mismatch.)
+
+SHIFTS = {O.LINEAR_SQUARE: 16, O.DYNAMIC_TREE: 14}
+
+
+def _signed_bucket(q, shift):
+    qb = (q.astype(np.float32) + np.float32(3.0)).astype(np.float32)
+    return (qb.view(np.uint32) >> shift).astype(np.int64) - (0x40000000 >> shift)
+
+
+def _signed_codes(q, t, shift):
+    kb = _signed_bucket(t, shift)
+    assert np.all(np.diff(kb) > 0), "two thresholds share a bucket"
+    count = (0x40800000 >> shift) - (0x40000000 >> shift) + 1
+    c0 = np.array([int(np.sum(kb < k)) for k in range(count)], np.int64)
+    t16 = np.concatenate([t, np.float32([np.inf])]).astype(np.float32)
+    c = c0[_signed_bucket(q, shift)]
+    return c + (q > t16[c])
+
+
+@pytest.mark.parametrize("cbk", [O.LINEAR_SQUARE, O.DYNAMIC_TREE])
+def test_signed_bucket_rule_equals_the_count_rule(cbk):
+    shift = SHIFTS[cbk]
+    t = O.thresholds_f32(cbk)
+    # the bucket width stays below the smallest gap between thresholds
+    assert 2.0 ** (shift - 22) < np.min(np.diff(t.astype(np.float64)))
+    vals = []
+    for tk in t:                                   # every pattern near each threshold
+        b = int(np.float32(tk).view(np.uint32))
+        vals.append((b + np.arange(-65536, 65536)).astype(np.uint32).view(np.float32))
+    off = 0x40000000 >> shift
+    count = (0x40800000 >> shift) - off + 1
+    for k in range(count + 1):                     # values on both sides of each bucket edge
+        edge = np.uint32((off + k) << shift).view(np.float32) - np.float32(3.0)
+        vals.append(np.float32(edge) + np.arange(-2000, 2000, dtype=np.float32) * np.float32(2.0 ** -24))
+    rng = np.random.default_rng(5)
+    vals.append(rng.uniform(-1, 1, 4 << 20).astype(np.float32))
+    vals.append(np.float32([0.0, -0.0, 1.0, -1.0, 1e-38, -1e-38, 1e-45, -1e-45, 2.0 ** -30, -(2.0 ** -30)]))
+    q = np.concatenate(vals).astype(np.float32)
+    q = q[np.abs(q) <= 1]
+    q = np.concatenate([q, -q])
+    assert np.array_equal(_signed_codes(q, t, shift), _rule(q, t))

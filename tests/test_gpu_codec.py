@@ -85,6 +85,51 @@ def test_shared_divisor_division_matches_ieee_over_exponent_range(book):
     _check(xs, book)
 
 
+@pytest.mark.parametrize("book", list(BOOKS))
+def test_signed_bucket_path(book):
+    """Whole warps (4 blocks of 64) with scales in [2^-60, 1] and no ragged
+    end take the signed-bucket decision; one block out of range sends its
+    warp to the general one.  Ties: thresholds times a power-of-two scale
+    equal to the block's absmax."""
+    rng = np.random.default_rng(16)
+    t = O.thresholds_f32(BOOKS[book])
+    xs = []
+    for s in (1.0, 0.5, 2.0 ** -20, 2.0 ** -60, 2.0 ** -59, 0.7, 0.999999):
+        x = (rng.uniform(-1, 1, 64 * 4 * 33) * s).astype(np.float32)
+        x[::64] = np.float32(s)                               # absmax exactly s
+        xs.append(x)
+    for p in (0, -3, -40, -60):
+        s = np.float32(2.0 ** p)
+        blk = np.concatenate([t * s, -t * s, [s], np.zeros(64 - 31)]).astype(np.float32)[:64]
+        xs.append(np.tile(blk, 4 * 9))
+    x = (rng.uniform(-1, 1, 64 * 4 * 16) * 0.3).astype(np.float32)
+    x[64 * 4 * 5 + 17] = 1.5                                  # one warp to the general path
+    x[64 * 4 * 9 + 3] = np.float32(2.0 ** -61)                # below 2^-60: general path
+    x[64 * 4 * 9 + 4:64 * 4 * 9 + 64] = 0.0
+    x[64 * 4 * 9:64 * 4 * 9 + 3] = 0.0
+    xs.append(x)
+    _check(xs, book)
+    _check([np.concatenate(xs)], book)
+
+
+@pytest.mark.parametrize("book", list(BOOKS))
+def test_large_tensor_unit_scale_sampled(book):
+    """512 MiB with block scales below 1 (the signed-bucket path), sampled."""
+    api = _api()
+    n = (1 << 27) + 37
+    g = torch.Generator(device="cuda").manual_seed(6)
+    x = torch.randn(n, device="cuda", generator=g) * 0.125
+    codes, scales = api.quant4_pack([x], codebook=book)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(17)
+    nb = (n + 63) // 64
+    for b in list(rng.integers(0, nb, 64)) + [nb - 1]:
+        lo, hi = 64 * int(b), min(64 * int(b) + 64, n)
+        oc, os_ = O.quantize(x[lo:hi].cpu().numpy(), codebook=BOOKS[book])
+        assert scales[0][int(b)].item() == os_[0]
+        assert np.array_equal(codes[0][lo // 2:(hi + 1) // 2].cpu().numpy(), oc)
+
+
 def test_misaligned_pointers():
     api = _api()
     rng = np.random.default_rng(14)
