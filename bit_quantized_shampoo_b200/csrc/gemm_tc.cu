@@ -449,8 +449,9 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmDesc& g, const PtrEntr
 template <int BN, bool SPLIT, int STAGES>
 __global__ void __launch_bounds__(192, STAGES <= 2 ? 2 : 1)
 k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, int nparams,
-          uint32_t* __restrict__ gflags, uint64_t wait_ns) {
+          uint32_t* __restrict__ gflags, uint64_t wait_ns, const uint32_t* __restrict__ guard) {
   using Cfg = TcCfg<BN, SPLIT, STAGES>;
+  if (guard && *guard == 0u) return;                      // no problem of the launch runs
   const TcGemmDesc& g = descs[blockIdx.y];
   const int tiles_n = (g.N + BN - 1) / BN;
   const int tiles_m = (g.M + kBM - 1) / kBM;
@@ -580,9 +581,400 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
   }
 }
 
+// ---------------------------------------------------------------------------
+// Persistent form (the fp32-accurate 128-wide instance).  One CTA per SM
+// walks the batch's running tiles (tile t, t + gridDim.x, ...).  The
+// operand ring runs on across tiles, so the next tile's loads start while
+// this one's MMAs finish.  The epilogue reads a finished tile's four
+// accumulators into registers (each lane one row of 128 columns, the
+// partial sums added with round-to-nearest), hands tensor memory back to
+// the MMA warp at once, and writes the outputs from registers while the
+// next tile's main loop runs.  Each epilogue warp has one staging block of
+// 32 rows, used in turn for the Cin chunk and for the transposed output
+// rows.
+template <int BN, bool SPLIT, int STAGES>
+struct PersCfg {
+  using Base = TcCfg<BN, SPLIT, STAGES>;
+  static constexpr int kPitch = 36;
+  static constexpr int kRowBuf = 32 * kPitch * 4;       // one staging block per epilogue warp
+  static constexpr int kSmem = Base::kStage * STAGES + 4 * kRowBuf + 1024;
+  static_assert(kSmem <= 227 * 1024, "persistent GEMM fits in shared memory");
+};
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__host__ __device__ __forceinline__ int tiles_in_row(int symmetric, int N, int bn, int tm) {
+  const int tiles_n = (N + bn - 1) / bn;
+  if (!symmetric) return tiles_n;
+  const int c = ((tm + 1) * kBM + bn - 1) / bn;            // tn * bn < (tm + 1) * kBM
+  return c < tiles_n ? c : tiles_n;
+}
+
+// Running tile t of the batch (tc_assign_tiles numbered them): problem p
+// (a cursor that only moves forward, as t does), tile origin (m0, n0);
+// false when the problem is skipped.  Every role walks the same tiles.
+template <int BN>
+__device__ __forceinline__ bool pers_tile(const TcGemmDesc* __restrict__ descs, int count, int64_t t, int& p,
+                                          int& m0, int& n0) {
+  while (p + 1 < count && descs[p + 1].tile_begin <= t) ++p;
+  const TcGemmDesc& g = descs[p];
+  int x = int(t - g.tile_begin);
+  const int tiles_m = (g.M + kBM - 1) / kBM;
+  int tm = 0;
+  for (; tm < tiles_m; ++tm) {
+    const int c = tiles_in_row(g.symmetric, g.N, BN, tm);
+    if (x < c) break;
+    x -= c;
+  }
+  m0 = tm * kBM;
+  n0 = x * BN;
+  return !(g.skip && *g.skip);
+}
+
+// Outputs of one tile from the accumulator values in registers (lane l of
+// epilogue warp q holds row m0 + 32 q + l, columns n0 + 32 i + j in
+// v[i][j]).  Same outputs and rounding as epilogue_tile.
+template <int BN>
+__device__ __forceinline__ void epilogue_regs(const TcGemmDesc& g, const PtrEntry* __restrict__ tabs, int nparams,
+                                              int m0, int n0, float (&v)[BN / 32][32], int q, int lane,
+                                              uint8_t* wbuf) {
+  constexpr int kPitch = 36, kChunks = BN / 32;
+  EpiArgs e;
+  e.load(g, tabs, nparams);
+  const int rbase = m0 + 32 * q;
+  const int row = rbase + lane;
+  const bool row_ok = row < e.M;
+  const int nrows = min(32, e.M - rbase);
+  const int ncols = min(BN, e.N - n0);
+  const int nchunks = ncols > 0 ? (ncols + 31) / 32 : 0;
+  if (nrows <= 0) return;
+  const bool cin_bulk = e.beta != 0.0f &&
+                        ((reinterpret_cast<uintptr_t>(e.Cin) | uintptr_t(e.ldcin * 4)) & 15) == 0 &&
+                        (e.N & 3) == 0;
+  const bool out_bulk = ((reinterpret_cast<uintptr_t>(e.C) | uintptr_t(e.ldc * 4) |
+                          reinterpret_cast<uintptr_t>(e.Chi) | reinterpret_cast<uintptr_t>(e.Clo) |
+                          uintptr_t(e.ldh * 4)) & 15) == 0 &&
+                        (e.N & 3) == 0;
+  const uint32_t wsm = smem_u32(wbuf);
+  float* stage = reinterpret_cast<float*>(wbuf);
+  const int sr = lane >> 3, sc = 4 * (lane & 7);
+  unsigned long long dev_fine = 0;
+#pragma unroll
+  for (int i = 0; i < kChunks; ++i) {
+    if (i >= nchunks) break;
+    const int cb = n0 + 32 * i;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[i][j] *= e.alpha;
+    if (e.beta != 0.0f) {
+      if (cin_bulk) {
+        // Cin chunk into the staging block, 4 full 128-byte rows per warp
+        // instruction (lane l: rows 4 t + l / 8, columns 4 (l % 8))
+        __syncwarp();                                   // previous reads of the block done
+        if (cb + sc < e.N) {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int rr = 4 * t + sr;
+            if (rbase + rr < e.M)
+              cp_async16(wsm + uint32_t((rr * kPitch + sc) * 4), e.Cin + int64_t(rbase + rr) * e.ldcin + cb + sc);
+          }
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncwarp();
+        if (row_ok) {
+          const float4* src = reinterpret_cast<const float4*>(stage + lane * kPitch);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            if (cb + 4 * t < e.N) {
+              const float4 x = src[t];
+              v[i][4 * t + 0] = fmaf(e.beta, x.x, v[i][4 * t + 0]);
+              v[i][4 * t + 1] = fmaf(e.beta, x.y, v[i][4 * t + 1]);
+              v[i][4 * t + 2] = fmaf(e.beta, x.z, v[i][4 * t + 2]);
+              v[i][4 * t + 3] = fmaf(e.beta, x.w, v[i][4 * t + 3]);
+            }
+          }
+        }
+      } else if (row_ok) {
+        const float* src = e.Cin + int64_t(row) * e.ldcin + cb;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (cb + j < e.N) v[i][j] = fmaf(e.beta, __ldg(src + j), v[i][j]);
+      }
+    }
+    if (e.devsq && row_ok) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int c = cb + j;
+        if (c >= e.N || c == row || (e.symmetric && c > row)) continue;
+        const float sq = v[i][j] * v[i][j];
+        const unsigned long long w = (e.symmetric && c < row) ? 2ull : 1ull;
+        dev_fine += w * static_cast<unsigned long long>(fminf(sq, kDevFineClamp) * kDevFineUnit);
+      }
+    }
+    const bool below = !e.symmetric || cb + 31 < rbase;   // whole chunk left of every row
+    if (out_bulk && below) {
+      const bool col_ok = cb + sc < e.N;
+#pragma unroll 1
+      for (int o = 0; o < 3; ++o) {
+        float* out = o == 0 ? e.C : (o == 1 ? e.Chi : e.Clo);
+        if (!out) continue;                             // warp-uniform
+        const int64_t ld = o == 0 ? e.ldc : e.ldh;
+        __syncwarp();                                   // previous reads of the block done
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          float4 x = make_float4(v[i][4 * t], v[i][4 * t + 1], v[i][4 * t + 2], v[i][4 * t + 3]);
+          if (o == 1 || (o == 0 && e.out_round)) {
+            x = make_float4(rn_tf32(x.x), rn_tf32(x.y), rn_tf32(x.z), rn_tf32(x.w));
+          } else if (o == 2) {
+            x = make_float4(rn_tf32(x.x - rn_tf32(x.x)), rn_tf32(x.y - rn_tf32(x.y)),
+                            rn_tf32(x.z - rn_tf32(x.z)), rn_tf32(x.w - rn_tf32(x.w)));
+          }
+          *reinterpret_cast<float4*>(stage + lane * kPitch + 4 * t) = x;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int rr = 4 * t + sr;
+          if (rbase + rr < e.M && col_ok)
+            *reinterpret_cast<float4*>(out + int64_t(rbase + rr) * ld + cb + sc) =
+                *reinterpret_cast<const float4*>(stage + rr * kPitch + sc);
+        }
+      }
+    } else if (row_ok) {
+      if (out_bulk) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int c = cb + 4 * t;
+          if (c >= e.N) break;
+          if (!e.symmetric || c + 3 <= row) {
+            e.put4(int64_t(row), c, v[i][4 * t + 0], v[i][4 * t + 1], v[i][4 * t + 2], v[i][4 * t + 3]);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (c + u <= row) e.put(int64_t(row), c + u, v[i][4 * t + u]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int c = cb + j;
+          if (c < e.N && (!e.symmetric || c <= row)) e.put(int64_t(row), c, v[i][j]);
+        }
+      }
+    }
+    if (e.symmetric == 1 && cb < rbase + 32) {          // mirror of the strictly-lower part
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int c = cb + j;
+        if (row_ok && c < e.N && c < row) e.put(int64_t(c), row, v[i][j]);
+      }
+    }
+  }
+  if (e.devsq) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dev_fine += __shfl_xor_sync(0xffffffffu, dev_fine, o);
+    if (lane == 0 && dev_fine) atomicAdd(e.devsq, dev_fine);
+  }
+  __syncwarp();                                         // the block is free for the next tile
+}
+
+template <int BN, bool SPLIT, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, const PtrEntry* __restrict__ tabs,
+               int nparams, uint32_t* __restrict__ gflags, uint64_t wait_ns, const uint32_t* __restrict__ guard) {
+  using Cfg = TcCfg<BN, SPLIT, STAGES>;
+  if (guard && *guard == 0u) return;                      // no problem of the launch runs
+  using PCfg = PersCfg<BN, SPLIT, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* staging = smem + Cfg::kStage * STAGES;
+  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES], acc_full, acc_empty;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&acc_full, 1);
+    mbar_init(&acc_empty, 4);                           // one arrival per epilogue warp
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                 "r"(Cfg::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = tmem_slot;
+  int p = 0;                                                // each role's problem cursor
+
+  if (warp == 0) {
+    if (lane == 0) {                                        // ---- TMA producer
+      uint32_t it = 0;                                      // k-blocks issued, over all tiles
+      int last_p = -1;
+      for (int64_t t = blockIdx.x; t < total && !*(volatile int*)&abort_flag; t += gridDim.x) {
+        int m0, n0;
+        if (!pers_tile<BN>(descs, count, t, p, m0, n0)) continue;
+        const TcOperand ga = descs[p].a, gb = descs[p].b;   // registers (see k_gemm_tc)
+        const int kblocks = (descs[p].K + kBK - 1) / kBK;
+        if (p != last_p) {
+          asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(ga.hi)) : "memory");
+          asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(gb.hi)) : "memory");
+          if (SPLIT) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(ga.lo)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(gb.lo)) : "memory");
+          }
+          last_p = p;
+        }
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (it >= STAGES && !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, wait_ns)) {
+            atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+            abort_flag = 1;
+            break;
+          }
+          if (*(volatile int*)&abort_flag) break;
+          const uint32_t st = smem_u32(smem + s * Cfg::kStage);
+          mbar_expect_tx(&full_bar[s], Cfg::kStage);
+          const int k0 = kb * kBK;
+          load_operand(ga.hi, ga, kBM, m0, k0, st, &full_bar[s]);
+          load_operand(gb.hi, gb, BN, n0, k0, st + Cfg::kATile, &full_bar[s]);
+          if (SPLIT) {
+            load_operand(ga.lo, ga, kBM, m0, k0, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+            load_operand(gb.lo, gb, BN, n0, k0, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+          }
+        }
+      }
+      // the loads issued last land before the CTA exits (earlier ones were
+      // consumed by MMAs before their stages were refilled)
+      for (uint32_t k = it > uint32_t(STAGES) ? it - STAGES : 0; k < it; ++k)
+        if (!mbar_wait(&full_bar[k % STAGES], (k / STAGES) & 1, kWaitNs)) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {                                        // ---- MMA issuer
+      uint32_t it = 0, ntiles = 0;
+      for (int64_t t = blockIdx.x; t < total && !*(volatile int*)&abort_flag; t += gridDim.x) {
+        int m0, n0;
+        if (!pers_tile<BN>(descs, count, t, p, m0, n0)) continue;
+        const TcOperand ga = descs[p].a, gb = descs[p].b;
+        const int kblocks = (descs[p].K + kBK - 1) / kBK;
+        const uint32_t idesc = idesc_tf32(kBM, BN, ga.mn_major, gb.mn_major);
+        // the epilogue has read the previous tile's accumulators
+        if (ntiles > 0 && !mbar_wait(&acc_empty, (ntiles - 1) & 1, wait_ns)) {
+          atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+          abort_flag = 1;
+          break;
+        }
+        fence_after_sync();
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full_bar[s], (it / STAGES) & 1, wait_ns)) {
+            atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+            abort_flag = 1;
+            ok = false;
+            break;
+          }
+          if (*(volatile int*)&abort_flag) { ok = false; break; }
+          fence_after_sync();
+          const uint32_t st = smem_u32(smem + s * Cfg::kStage);
+          const uint32_t a_hi = st, b_hi = st + Cfg::kATile;
+          const uint32_t a_lo = st + Cfg::kATile + Cfg::kBTile, b_lo = a_lo + Cfg::kATile;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 8; ++kk) {
+            const uint32_t acc = (kb >= Cfg::kAcc || kk != 0) ? 1u : 0u;
+            const uint32_t dt = tmem + uint32_t((kb % Cfg::kAcc) * BN);
+            mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(gb, b_hi, kk), idesc, acc);
+            if (SPLIT) {
+              mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(gb, b_lo, kk), idesc, 1);
+              mma_tf32(dt, operand_desc(ga, a_lo, kk), operand_desc(gb, b_hi, kk), idesc, 1);
+            }
+          }
+          mma_commit(&empty_bar[s]);
+        }
+        mma_commit(&acc_full);                              // this tile's accumulators complete
+        ++ntiles;
+        if (!ok) break;
+      }
+      // every MMA issued completes before tensor memory is freed
+      if (ntiles > 0 && !mbar_wait(&acc_full, (ntiles - 1) & 1, kWaitNs)) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+    }
+  } else {                                                  // ---- epilogue, warps 2..5
+    const int q = warp & 3;
+    uint8_t* wbuf = staging + q * PCfg::kRowBuf;
+    uint32_t ntiles = 0;
+    for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+      int m0, n0;
+      if (!pers_tile<BN>(descs, count, t, p, m0, n0)) continue;
+      const bool ok = mbar_wait(&acc_full, ntiles & 1, wait_ns);
+      if (!ok) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
+      if (!ok || *(volatile int*)&abort_flag) break;
+      fence_after_sync();
+      const int kblocks = (descs[p].K + kBK - 1) / kBK;
+      const int nacc = kblocks < Cfg::kAcc ? kblocks : Cfg::kAcc;
+      float v[BN / 32][32];
+#pragma unroll
+      for (int i = 0; i < BN / 32; ++i) {
+        uint32_t r[32];
+        tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(32 * i), r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[i][j] = __uint_as_float(r[j]);
+        for (int a = 1; a < nacc; ++a) {                    // the other accumulators, added with RN
+          tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(a * BN + 32 * i), r);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[i][j] += __uint_as_float(r[j]);
+        }
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty);               // tensor memory free for the next tile
+      ++ntiles;
+      epilogue_regs<BN>(descs[p], tabs, nparams, m0, n0, v, q, lane, wbuf);
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(Cfg::kTmemCols)
+                 : "memory");
+  }
+}
+
+template <int BN, bool SPLIT, int STAGES>
+shampoo4_status launch_tc_pers(const TcGemmDesc* d_desc, int count, int64_t total, const PtrEntry* tabs,
+                               int nparams, uint32_t* gflags, uint64_t wait_ns, cudaStream_t st,
+                               const uint32_t* guard) {
+  using PCfg = PersCfg<BN, SPLIT, STAGES>;
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    S4_CUDA(cudaGetDevice(&dev));
+    S4_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    S4_CUDA(cudaFuncSetAttribute(k_gemm_tc_pers<BN, SPLIT, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 PCfg::kSmem));
+  }
+  if (total <= 0) return SHAMPOO4_OK;
+  const int grid = int(total < sms ? total : sms);
+  k_gemm_tc_pers<BN, SPLIT, STAGES><<<grid, 192, PCfg::kSmem, st>>>(d_desc, count, total, tabs, nparams, gflags,
+                                                                     wait_ns, guard);
+  S4_CUDA(cudaGetLastError());
+  return SHAMPOO4_OK;
+}
+
 template <int BN, bool SPLIT, int STAGES>
 shampoo4_status launch_tc_impl(const TcGemmDesc* d_desc, int count, int max_tiles, const PtrEntry* tabs,
-                               int nparams, uint32_t* gflags, uint64_t wait_ns, cudaStream_t st) {
+                               int nparams, uint32_t* gflags, uint64_t wait_ns, cudaStream_t st,
+                               const uint32_t* guard) {
   using Cfg = TcCfg<BN, SPLIT, STAGES>;
   static bool configured = false;
   if (!configured) {
@@ -593,7 +985,7 @@ shampoo4_status launch_tc_impl(const TcGemmDesc* d_desc, int count, int max_tile
   for (int base = 0; base < count; base += 65535) {
     const int c = count - base < 65535 ? count - base : 65535;
     k_gemm_tc<BN, SPLIT, STAGES><<<dim3(unsigned(max_tiles), unsigned(c)), 192, Cfg::kSmem, st>>>(
-        d_desc + base, tabs, nparams, gflags, wait_ns);
+        d_desc + base, tabs, nparams, gflags, wait_ns, guard);
     S4_CUDA(cudaGetLastError());
   }
   return SHAMPOO4_OK;
@@ -603,23 +995,49 @@ shampoo4_status launch_tc_impl(const TcGemmDesc* d_desc, int count, int max_tile
 
 int tc_block_n(int split) { return split ? 128 : 256; }
 
+// The 128-wide fp32-accurate instance runs in its persistent form (0: one
+// tile per CTA, for comparisons).
+int tc_persistent = 1;
+
+int tc_tiles_in_row(const TcGemmDesc& g, int bn, int tm) { return tiles_in_row(g.symmetric, g.N, bn, tm); }
+
+int64_t tc_assign_tiles(TcGemmDesc* v, int count, int bn) {
+  int64_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    v[i].tile_begin = int32_t(total);
+    const int tiles_m = (v[i].M + kBM - 1) / kBM;
+    for (int tm = 0; tm < tiles_m; ++tm) total += tiles_in_row(v[i].symmetric, v[i].N, bn, tm);
+  }
+  return total;
+}
+
 shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split, int bn,
                                const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st,
-                               uint64_t wait_ns) {
+                               uint64_t wait_ns, int64_t total_tiles, const uint32_t* guard) {
   if (count <= 0 || max_tiles <= 0) return SHAMPOO4_OK;
   if (wait_ns == 0 || wait_ns > kWaitNs) wait_ns = kWaitNs;
-  // One tile per CTA.  TF32: two 2-stage CTAs per SM, so one tile's
-  // epilogue overlaps the other's main loop.  (A persistent form with two
-  // TMEM accumulator sets and eight epilogue warps was measured against it:
-  // faster on single-output products, slower on the symmetric and
-  // multi-output products this library runs.)  Split mode: one 3-stage CTA
-  // per SM with 128-wide tiles (four accumulators fill TMEM), or two 2-stage
-  // CTAs per SM with 64-wide tiles for the narrow panel updates, where the
-  // MMA issue rate of a 64-wide instruction makes a second issuing CTA per
-  // SM worth more than overlap.
-  if (!split) return launch_tc_impl<256, false, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, wait_ns, st);
-  if (bn == 64) return launch_tc_impl<64, true, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, wait_ns, st);
-  return launch_tc_impl<128, true, 3>(d_desc, count, max_tiles, tabs, nparams, gflags, wait_ns, st);
+  // TF32: one tile per CTA, two 2-stage CTAs per SM, so one tile's
+  // epilogue overlaps the other's main loop.  (Persistent forms were
+  // measured against it on 960 products of 1024 x 1024 x 1024 and lost: two
+  // 256-column accumulators drained by four epilogue warps, 1.3x slower with
+  // three outputs and 2.2x on mirrored symmetric products; 128-wide tiles
+  // with the register epilogue, 1.2x to 5.9x slower.  A TF32 tile's main
+  // loop is too short to hide four warps' epilogue.)  Split mode, 128 wide:
+  // the persistent register form (1.35x to 1.47x faster than one tile per
+  // CTA: the main loop of three products per K step hides the epilogue),
+  // or one tile per CTA when no tile numbering is given; 64 wide (the
+  // narrow panel updates): two 2-stage CTAs per SM, where the MMA issue rate
+  // of a 64-wide instruction makes a second issuing CTA per SM worth more
+  // than overlap (its persistent register form was 1.4x to 2.1x slower on
+  // the panel shapes, K = 64 to 512).
+  const bool pers = total_tiles >= 0 && total_tiles < 0x7fffffffLL;
+  if (!split)
+    return launch_tc_impl<256, false, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, wait_ns, st, guard);
+  if (bn == 64)
+    return launch_tc_impl<64, true, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, wait_ns, st, guard);
+  if (pers && tc_persistent)
+    return launch_tc_pers<128, true, 3>(d_desc, count, total_tiles, tabs, nparams, gflags, wait_ns, st, guard);
+  return launch_tc_impl<128, true, 3>(d_desc, count, max_tiles, tabs, nparams, gflags, wait_ns, st, guard);
 }
 
 // ---------------------------------------------------------------- host side

@@ -353,7 +353,9 @@ constexpr int kPotrfFSmem = 2 * kPanel * (kPanel + 1) * 8;
 // suffices; the square roots and divisions are applied once at the end.
 // Padding beyond jb is the identity in the factorization and zero in the
 // written inverse.
-__global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ descs) {
+__global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ descs,
+                                                 const uint32_t* __restrict__ guard) {
+  if (guard && *guard == 0u) return;                      // no factor needs this launch
   const PotrfDescF& g = descs[blockIdx.x];
   const int jb = g.jb;
   if (jb <= 0 || *g.fail || (g.skip && *g.skip)) return;
@@ -442,14 +444,14 @@ __global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ 
   }
 }
 
-shampoo4_status launch_potrf_f(const PotrfDescF* d_desc, int count, cudaStream_t st) {
+shampoo4_status launch_potrf_f(const PotrfDescF* d_desc, int count, cudaStream_t st, const uint32_t* guard) {
   if (count <= 0) return SHAMPOO4_OK;
   static bool configured = false;
   if (!configured) {
     S4_CUDA(cudaFuncSetAttribute(k_potrf_f, cudaFuncAttributeMaxDynamicSharedMemorySize, kPotrfFSmem));
     configured = true;
   }
-  k_potrf_f<<<count, 256, kPotrfFSmem, st>>>(d_desc);
+  k_potrf_f<<<count, 256, kPotrfFSmem, st>>>(d_desc, guard);
   S4_CUDA(cudaGetLastError());
   return SHAMPOO4_OK;
 }
@@ -464,7 +466,8 @@ __global__ void __launch_bounds__(256) k_shift_f(const ShiftDescF* __restrict__ 
 }
 
 // ---- exact Gram diagonal ------------------------------------------------------
-__global__ void __launch_bounds__(256) k_diag(const DiagDesc* __restrict__ descs) {
+__global__ void __launch_bounds__(256) k_diag(const DiagDesc* __restrict__ descs, const uint32_t* __restrict__ guard) {
+  if (guard && *guard == 0u) return;
   const DiagDesc& g = descs[blockIdx.y];
   if (g.skip && *g.skip) return;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -492,11 +495,11 @@ __global__ void __launch_bounds__(256) k_diag(const DiagDesc* __restrict__ descs
   }
 }
 
-shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaStream_t st) {
+shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaStream_t st, const uint32_t* guard) {
   if (count <= 0 || max_d <= 0) return SHAMPOO4_OK;
   for (int base = 0; base < count; base += 65535) {
     const int c = count - base < 65535 ? count - base : 65535;
-    k_diag<<<dim3(unsigned((max_d + 255) / 256), unsigned(c)), 256, 0, st>>>(d_desc + base);
+    k_diag<<<dim3(unsigned((max_d + 255) / 256), unsigned(c)), 256, 0, st>>>(d_desc + base, guard);
     S4_CUDA(cudaGetLastError());
   }
   return SHAMPOO4_OK;
@@ -541,7 +544,9 @@ shampoo4_status launch_rowdiag(const RowDiagDesc* d_desc, int count, int max_d, 
 // then A^-1's space takes B^-1 and C's space takes -B^-1 T.
 constexpr int kInvSmem = 3 * 64 * 65 * 8;
 
-__global__ void __launch_bounds__(256) k_inv128(const Inv128Desc* __restrict__ descs) {
+__global__ void __launch_bounds__(256) k_inv128(const Inv128Desc* __restrict__ descs,
+                                                const uint32_t* __restrict__ guard) {
+  if (guard && *guard == 0u) return;
   const Inv128Desc& g = descs[blockIdx.x];
   if (g.skip && *g.skip) return;
   extern __shared__ double sm_inv[];
@@ -619,14 +624,14 @@ __global__ void __launch_bounds__(256) k_inv128(const Inv128Desc* __restrict__ d
   }
 }
 
-shampoo4_status launch_inv128(const Inv128Desc* d_desc, int count, cudaStream_t st) {
+shampoo4_status launch_inv128(const Inv128Desc* d_desc, int count, cudaStream_t st, const uint32_t* guard) {
   if (count <= 0) return SHAMPOO4_OK;
   static bool configured = false;
   if (!configured) {
     S4_CUDA(cudaFuncSetAttribute(k_inv128, cudaFuncAttributeMaxDynamicSharedMemorySize, kInvSmem));
     configured = true;
   }
-  k_inv128<<<count, 256, kInvSmem, st>>>(d_desc);
+  k_inv128<<<count, 256, kInvSmem, st>>>(d_desc, guard);
   S4_CUDA(cudaGetLastError());
   return SHAMPOO4_OK;
 }
@@ -636,7 +641,9 @@ __global__ void __launch_bounds__(256) k_gate(const GateDesc* __restrict__ descs
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= count) return;
   const GateDesc& g = descs[i];
-  *g.out = (*g.bad != 0u || *g.devsq <= g.thr) ? 1u : 0u;
+  const uint32_t skip = (*g.bad != 0u || *g.devsq <= g.thr) ? 1u : 0u;
+  *g.out = skip;
+  if (!skip && g.any) *g.any = 1u;
 }
 
 shampoo4_status launch_gate(const GateDesc* d_desc, int count, cudaStream_t st) {

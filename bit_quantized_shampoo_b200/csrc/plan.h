@@ -271,6 +271,7 @@ struct GateDesc {
   const uint32_t* bad;
   uint32_t* out;
   unsigned long long thr;
+  uint32_t* any;       // optional: set to 1 when this factor goes through the pass
 };
 
 
@@ -339,7 +340,9 @@ shampoo4_status launch_scan(const ScanDesc* d_desc, int count, int64_t max_rows,
                             const PtrEntry* tabs, int nparams, uint32_t* flags, cudaStream_t st);
 shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st,
                              const uint32_t* guard = nullptr);
-shampoo4_status launch_potrf_f(const PotrfDescF* d_desc, int count, cudaStream_t st);
+// guard (optional, as for the fp64 launches): the whole launch is skipped
+// when *guard == 0.
+shampoo4_status launch_potrf_f(const PotrfDescF* d_desc, int count, cudaStream_t st, const uint32_t* guard = nullptr);
 shampoo4_status launch_shift_f(const ShiftDescF* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st,
                                const uint32_t* guard = nullptr);
@@ -347,8 +350,9 @@ shampoo4_status launch_gate(const GateDesc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_copy(const CopyDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_newton_norm(const NewtonNormDesc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_newton_elt(const NewtonEltDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
-shampoo4_status launch_inv128(const Inv128Desc* d_desc, int count, cudaStream_t st);
-shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaStream_t st);
+shampoo4_status launch_inv128(const Inv128Desc* d_desc, int count, cudaStream_t st, const uint32_t* guard = nullptr);
+shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaStream_t st,
+                            const uint32_t* guard = nullptr);
 shampoo4_status launch_rowdiag(const RowDiagDesc* d_desc, int count, int max_d, cudaStream_t st);
 
 // Codec launchers (quant4.cu).  `skip` (optional, per tensor) suppresses a

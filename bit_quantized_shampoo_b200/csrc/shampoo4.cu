@@ -40,6 +40,7 @@ struct Launch {
   int64_t extent;      // max tiles / rows / elements, per kind
   double flops = 0, bytes = 0;   // algorithmic work of the launch
   size_t guard_off = SIZE_MAX;   // workspace word gating the whole launch (fp64 QR passes)
+  int64_t tiles = -1;            // tensor-core products: the batch's running tiles
   // Pack launches carry host-side tensor lists instead of descriptors.
   std::vector<const float*> px;
   std::vector<int64_t> pn;
@@ -115,6 +116,7 @@ struct shampoo4_ctx {
   // workspace regions
   size_t ws_flags = 0, ws_tabs = 0, ws_fail = 0, ws_bflag = 0, ws_maps = 0, ws_nmaps = 0;
   size_t ws_tcbad = 0, ws_tcgood = 0, ws_devsq = 0, ws_skip3 = 0, ws_fbany = 0;
+  size_t ws_p3any = 0;                   // some factor goes through the gated last QR pass
   bool any_simt = false;                 // some factor always takes the fp64 QR
   std::vector<int32_t> group_begin;      // tile groups: [group_begin[g], group_begin[g+1])
   // optional debug capture (shampoo4_debug_capture): every refresh copies
@@ -323,6 +325,7 @@ shampoo4_status plan(shampoo4_ctx* h) {
   h->ws_devsq = take(ws, 8 * h->factors.size());
   h->ws_skip3 = take(ws, 4 * h->factors.size());
   h->ws_fbany = take(ws, 4);
+  h->ws_p3any = take(ws, 4);
   h->ws_bflag = take(ws, 4 * h->blocks.size());
   // persistent per factor: the rebuilt statistic (compressed statistics,
   // valid from update_stats to refresh_roots) and the root weights
@@ -581,7 +584,11 @@ void emit_gemmtc(Builder& b, std::vector<Launch>& prog, const std::vector<TcGemm
     mt = std::max(mt, ((g.M + 127) / 128) * ((g.N + bn - 1) / bn));
     fl += product_flops(g.M, g.N, g.K, g.symmetric);
   }
-  b.emit(prog, !split ? Kind::GemmTC : (bn == 64 ? Kind::GemmTCSplit64 : Kind::GemmTCSplit), v, mt, fl);
+  if (v.empty()) return;
+  std::vector<TcGemmDesc> w = v;
+  const int64_t total = tc_assign_tiles(w.data(), int(w.size()), bn);
+  b.emit(prog, !split ? Kind::GemmTC : (bn == 64 ? Kind::GemmTCSplit64 : Kind::GemmTCSplit), w, mt, fl);
+  prog.back().tiles = total;
 }
 
 int mode_of(const shampoo4_config& c) { return c.precision == SHAMPOO4_PREC_FP32 ? kModeFP32 : kModeTF32; }
@@ -980,7 +987,7 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
         dgg.push_back({X[i].m, b.wf(f.ws_W), d, d, 0, b.devsq(i), b.tcbad(i)});
         const double tol = kLastPassTol * std::sqrt(double(d));        // on ||Q^T Q - I||_F / sqrt(d)
         const double thr = std::min(tol * tol * d * double(kDevFineUnit), 0x1p62);
-        gd.push_back({b.devsq(i), b.tcbad(i), b.skip3(i), static_cast<unsigned long long>(thr)});
+        gd.push_back({b.devsq(i), b.tcbad(i), b.skip3(i), static_cast<unsigned long long>(thr), b.wu(h->ws_p3any)});
         w.skip = b.skip3(i);
       }
       // only the lower triangles of W and of its TF32 split are ever read
@@ -999,6 +1006,8 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
       b.emit(prog, Kind::Diag, dgg, dmax, 0, 4.0 * elems(dgg));
       b.tag = SHAMPOO4_STAGE_QR_CONVERT;
       b.emit(prog, Kind::Gate, gd, 0);
+      // the rest of the pass runs only if some factor goes through it
+      b.guard = h->ws_p3any;
     }
     b.tag = SHAMPOO4_STAGE_QR_GRAM;
     emit_gemmtc(b, prog, g, true, kSquareBN);
@@ -1113,6 +1122,7 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
     b.tag = SHAMPOO4_STAGE_QR_SOLVE_PANEL;
     emit_gemmtc(b, prog, qp, true, 64);
   }
+  if (gated) b.guard = SIZE_MAX;
 }
 
 // Refresh by the coupled Newton iteration (root methods NEWTON and
@@ -1854,10 +1864,10 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
       case Kind::GemmTCSplit64:
         S4_TRY(launch_gemm_tc(static_cast<const TcGemmDesc*>(d), L.count, int(L.extent),
                               L.kind == Kind::GemmTC ? 0 : 1, L.kind == Kind::GemmTCSplit64 ? 64 : 0, tabs, np,
-                              gflags, st, h->wait_ns));
+                              gflags, st, h->wait_ns, L.tiles, guard));
         break;
       case Kind::PotrfF:
-        S4_TRY(launch_potrf_f(static_cast<const PotrfDescF*>(d), L.count, st));
+        S4_TRY(launch_potrf_f(static_cast<const PotrfDescF*>(d), L.count, st, guard));
         break;
       case Kind::ShiftF:
         S4_TRY(launch_shift_f(static_cast<const ShiftDescF*>(d), L.count, st));
@@ -1866,10 +1876,10 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
         S4_TRY(launch_gate(static_cast<const GateDesc*>(d), L.count, st));
         break;
       case Kind::Diag:
-        S4_TRY(launch_diag(static_cast<const DiagDesc*>(d), L.count, int(L.extent), st));
+        S4_TRY(launch_diag(static_cast<const DiagDesc*>(d), L.count, int(L.extent), st, guard));
         break;
       case Kind::Inv128:
-        S4_TRY(launch_inv128(static_cast<const Inv128Desc*>(d), L.count, st));
+        S4_TRY(launch_inv128(static_cast<const Inv128Desc*>(d), L.count, st, guard));
         break;
       case Kind::RowDiag:
         S4_TRY(launch_rowdiag(static_cast<const RowDiagDesc*>(d), L.count, int(L.extent), st));
@@ -2169,6 +2179,7 @@ extern "C" shampoo4_status shampoo4_refresh_roots(shampoo4_handle h, shampoo4_st
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_tcgood, 1, 4 * h->factors.size(), st));
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_devsq, 0, 8 * h->factors.size(), st));
   S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_fbany, h->any_simt ? 1 : 0, 4, st));
+  S4_CUDA(cudaMemsetAsync(h->d_ws + h->ws_p3any, 0, 4, st));
   const bool first = !h->has_basis;
   S4_TRY(run_program(h, first ? h->prog_refresh_first : h->prog_refresh, st));
   h->last_refresh_first = first;

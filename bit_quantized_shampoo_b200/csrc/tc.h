@@ -29,7 +29,9 @@ struct TcGemmDesc {
   int32_t M, N, K;
   int32_t symmetric;
   int32_t out_round;
-  int32_t pad_;
+  // index of the problem's first tile in the batch's list of tiles that
+  // run (tc_assign_tiles); read by the persistent kernel only
+  int32_t tile_begin;
   float alpha, beta;
   TcOperand a, b;
   float* C; int64_t ldc;
@@ -48,9 +50,19 @@ struct TcGemmDesc {
 int tc_block_n(int split);
 // wait_ns: how long each pipeline wait may take before the CTA gives up
 // (SHAMPOO4_FLAG_TIMEOUT); 0 means the default of 2 s, which is also the cap.
+// total_tiles: the batch's number of running tiles from tc_assign_tiles on
+// the same descriptors; without it (-1) every instance runs one tile per CTA.
+// guard (optional): the whole launch is skipped when *guard == 0.
 shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split, int bn,
                                const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st,
-                               uint64_t wait_ns = 0);
+                               uint64_t wait_ns = 0, int64_t total_tiles = -1, const uint32_t* guard = nullptr);
+// Tiles of one problem that run for tile width bn: all, or for a symmetric
+// product those touching the lower triangle (row block tm runs column
+// blocks tn with tn * bn < (tm + 1) * 128).
+int tc_tiles_in_row(const TcGemmDesc& g, int bn, int tm);
+// Number the running tiles of a batch: sets tile_begin of each descriptor,
+// returns the total.
+int64_t tc_assign_tiles(TcGemmDesc* v, int count, int bn);
 // Encode a 2-D fp32 tensor map (rows x cols, leading dimension ld elements),
 // box 32 (contiguous) x box_rows, zero fill out of bounds; 128-byte swizzle,
 // with 32-byte atoms for an operand read MN-major.
