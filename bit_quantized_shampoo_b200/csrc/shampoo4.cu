@@ -1412,11 +1412,16 @@ void build_refresh_owned(Builder& b, std::vector<Launch>& prog, bool first) {
         TcGemmDesc u = gemmtc(d, d, d, -0.5f, 1.5f);         // U' = 1.5 U - 0.5 U T
         u.a = b.operand(b.wf(f.ws_Xh[c]), b.wf(f.ws_Xl[c]), d, d, true, false, split);
         u.b = b.operand(b.wf(f.ws_Th), b.wf(f.ws_Tl), d, d, false, true, split);   // T symmetric
-        u.Cin = b.wf(f.ws_Xm[c]); u.ldcin = d;
-        u.C = b.wf(f.ws_Xm[o]); u.ldc = d;
+        // With TF32 products the iterates are TF32 numbers between steps:
+        // a step after the first takes 1.5 U from U's TF32 value, and only
+        // the last step writes fp32 U (the products' own TF32 rounding
+        // already limits the iteration to that precision).
+        const bool last = it + 1 == iters;
+        u.Cin = (split || it == 0) ? b.wf(f.ws_Xm[c]) : b.wf(f.ws_Xh[c]); u.ldcin = d;
+        u.C = (split || last) ? b.wf(f.ws_Xm[o]) : nullptr; u.ldc = d;
         // U's lo part feeds the next Björck products only when fp32-accurate;
         // the last one always feeds the fp32-accurate subspace product
-        u.Chi = b.wf(f.ws_Xh[o]); u.Clo = (split || it + 1 == iters) ? b.wf(f.ws_Xl[o]) : nullptr; u.ldh = d;
+        u.Chi = b.wf(f.ws_Xh[o]); u.Clo = (split || last) ? b.wf(f.ws_Xl[o]) : nullptr; u.ldh = d;
         tupd.push_back(u);
         cur[i] = o;
       } else {
