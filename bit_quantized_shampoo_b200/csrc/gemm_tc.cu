@@ -204,6 +204,13 @@ __device__ __forceinline__ void load_operand(const CUtensorMap* map, const TcOpe
   }
 }
 
+// The B operand of K block k0 of an output tile at column n0: as given, or,
+// past the stored tiles of a symmetric operand (bt maps), its transpose
+// read MN-major.
+__device__ __forceinline__ bool b_transposed(const CUtensorMap* bt_hi, int k0, int n0, int bn) {
+  return bt_hi != nullptr && k0 >= n0 + bn;
+}
+
 __device__ __forceinline__ uint64_t operand_desc(const TcOperand& op, uint32_t base, int kk) {
   // K-major (128 B swizzle): rows of 128 B, 8-row groups 1024 B apart; a K
   // step of 8 is 32 B along the row.
@@ -222,7 +229,8 @@ struct EpiArgs {
   unsigned long long* devsq;
 
   __device__ __forceinline__ void load(const TcGemmDesc& g, const PtrEntry* tabs, int nparams) {
-    M = g.M; N = g.N; symmetric = g.symmetric; out_round = g.out_round;
+    M = g.M; N = g.N; out_round = g.out_round;
+    symmetric = g.symmetric == 3 ? 0 : g.symmetric;      // mode 3 writes its tiles in full
     alpha = g.alpha; beta = g.beta;
     C = g.C; ldc = g.ldc;
     if (g.c_ref.tab >= 0) {
@@ -501,6 +509,10 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(ga.lo)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(gb.lo)) : "memory");
       }
+      const CUtensorMap* bt_hi = g.bt_hi;
+      const CUtensorMap* bt_lo = g.bt_lo;
+      TcOperand gt = gb;                                    // transposed reads of B
+      gt.hi = bt_hi; gt.lo = bt_lo; gt.mn_major = 1;
       int issued = 0;
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % Cfg::kStages;
@@ -513,11 +525,13 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
         const uint32_t st = smem_u32(smem + s * Cfg::kStage);
         mbar_expect_tx(&full_bar[s], Cfg::kStage);
         const int k0 = kb * kBK;
+        const bool tr = b_transposed(bt_hi, k0, n0, BN);
+        const TcOperand& ob = tr ? gt : gb;
         load_operand(ga.hi, ga, kBM, m0, k0, st, &full_bar[s]);
-        load_operand(gb.hi, gb, BN, n0, k0, st + Cfg::kATile, &full_bar[s]);
+        load_operand(ob.hi, ob, BN, n0, k0, st + Cfg::kATile, &full_bar[s]);
         if (SPLIT) {
           load_operand(ga.lo, ga, kBM, m0, k0, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
-          load_operand(gb.lo, gb, BN, n0, k0, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+          load_operand(ob.lo, ob, BN, n0, k0, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
         }
         issued = kb + 1;
       }
@@ -532,7 +546,11 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
   } else if (warp == 1) {
     if (lane == 0) {                                        // ---- MMA issuer
       const TcOperand ga = g.a, gb = g.b;                   // registers, as in the producer
-      const uint32_t idesc = idesc_tf32(kBM, BN, ga.mn_major, gb.mn_major);
+      const CUtensorMap* bt_hi = g.bt_hi;
+      TcOperand gt = gb;
+      gt.mn_major = 1;
+      const uint32_t idesc_n = idesc_tf32(kBM, BN, ga.mn_major, gb.mn_major);
+      const uint32_t idesc_t = idesc_tf32(kBM, BN, ga.mn_major, 1);
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % Cfg::kStages;
         if (!mbar_wait(&full_bar[s], (kb / Cfg::kStages) & 1, wait_ns)) {
@@ -545,15 +563,18 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
         const uint32_t st = smem_u32(smem + s * Cfg::kStage);
         const uint32_t a_hi = st, b_hi = st + Cfg::kATile;
         const uint32_t a_lo = st + Cfg::kATile + Cfg::kBTile, b_lo = a_lo + Cfg::kATile;
+        const bool tr = b_transposed(bt_hi, kb * kBK, n0, BN);
+        const TcOperand& ob = tr ? gt : gb;
+        const uint32_t idesc = tr ? idesc_t : idesc_n;
 #pragma unroll
         for (int kk = 0; kk < kBK / 8; ++kk) {
           // first MMA into accumulator kb mod kAcc overwrites it
           const uint32_t acc = (kb >= Cfg::kAcc || kk != 0) ? 1u : 0u;
           const uint32_t dt = tmem + uint32_t((kb % Cfg::kAcc) * BN);
-          mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(gb, b_hi, kk), idesc, acc);
+          mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(ob, b_hi, kk), idesc, acc);
           if (SPLIT) {
-            mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(gb, b_lo, kk), idesc, 1);
-            mma_tf32(dt, operand_desc(ga, a_lo, kk), operand_desc(gb, b_hi, kk), idesc, 1);
+            mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(ob, b_lo, kk), idesc, 1);
+            mma_tf32(dt, operand_desc(ga, a_lo, kk), operand_desc(ob, b_hi, kk), idesc, 1);
           }
         }
         mma_commit(&empty_bar[s]);                          // stage free once these MMAs finish
@@ -825,6 +846,9 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
         int m0, n0;
         if (!pers_tile<BN>(descs, count, t, p, m0, n0)) continue;
         const TcOperand ga = descs[p].a, gb = descs[p].b;   // registers (see k_gemm_tc)
+        const CUtensorMap* bt_hi = descs[p].bt_hi;
+        TcOperand gt = gb;                                  // transposed reads of B
+        gt.hi = bt_hi; gt.lo = descs[p].bt_lo; gt.mn_major = 1;
         const int kblocks = (descs[p].K + kBK - 1) / kBK;
         if (p != last_p) {
           asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(ga.hi)) : "memory");
@@ -846,11 +870,13 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
           const uint32_t st = smem_u32(smem + s * Cfg::kStage);
           mbar_expect_tx(&full_bar[s], Cfg::kStage);
           const int k0 = kb * kBK;
+          const bool tr = b_transposed(bt_hi, k0, n0, BN);
+          const TcOperand& ob = tr ? gt : gb;
           load_operand(ga.hi, ga, kBM, m0, k0, st, &full_bar[s]);
-          load_operand(gb.hi, gb, BN, n0, k0, st + Cfg::kATile, &full_bar[s]);
+          load_operand(ob.hi, ob, BN, n0, k0, st + Cfg::kATile, &full_bar[s]);
           if (SPLIT) {
             load_operand(ga.lo, ga, kBM, m0, k0, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
-            load_operand(gb.lo, gb, BN, n0, k0, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+            load_operand(ob.lo, ob, BN, n0, k0, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
           }
         }
       }
@@ -866,8 +892,12 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
         int m0, n0;
         if (!pers_tile<BN>(descs, count, t, p, m0, n0)) continue;
         const TcOperand ga = descs[p].a, gb = descs[p].b;
+        const CUtensorMap* bt_hi = descs[p].bt_hi;
+        TcOperand gt = gb;
+        gt.mn_major = 1;
         const int kblocks = (descs[p].K + kBK - 1) / kBK;
-        const uint32_t idesc = idesc_tf32(kBM, BN, ga.mn_major, gb.mn_major);
+        const uint32_t idesc_n = idesc_tf32(kBM, BN, ga.mn_major, gb.mn_major);
+        const uint32_t idesc_t = idesc_tf32(kBM, BN, ga.mn_major, 1);
         // the epilogue has read the previous tile's accumulators
         if (ntiles > 0 && !mbar_wait(&acc_empty, (ntiles - 1) & 1, wait_ns)) {
           atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
@@ -889,14 +919,17 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
           const uint32_t st = smem_u32(smem + s * Cfg::kStage);
           const uint32_t a_hi = st, b_hi = st + Cfg::kATile;
           const uint32_t a_lo = st + Cfg::kATile + Cfg::kBTile, b_lo = a_lo + Cfg::kATile;
+          const bool tr = b_transposed(bt_hi, kb * kBK, n0, BN);
+          const TcOperand& ob = tr ? gt : gb;
+          const uint32_t idesc = tr ? idesc_t : idesc_n;
 #pragma unroll
           for (int kk = 0; kk < kBK / 8; ++kk) {
             const uint32_t acc = (kb >= Cfg::kAcc || kk != 0) ? 1u : 0u;
             const uint32_t dt = tmem + uint32_t((kb % Cfg::kAcc) * BN);
-            mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(gb, b_hi, kk), idesc, acc);
+            mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(ob, b_hi, kk), idesc, acc);
             if (SPLIT) {
-              mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(gb, b_lo, kk), idesc, 1);
-              mma_tf32(dt, operand_desc(ga, a_lo, kk), operand_desc(gb, b_hi, kk), idesc, 1);
+              mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(ob, b_lo, kk), idesc, 1);
+              mma_tf32(dt, operand_desc(ga, a_lo, kk), operand_desc(ob, b_hi, kk), idesc, 1);
             }
           }
           mma_commit(&empty_bar[s]);

@@ -1402,16 +1402,18 @@ void build_refresh_owned(Builder& b, std::vector<Launch>& prog, bool first) {
         TcGemmDesc g = gemmtc(d, d, d, 1.0f, 0.0f);          // T = U^T U
         g.a = b.operand(b.wf(f.ws_Xh[c]), b.wf(f.ws_Xl[c]), d, d, true, true, split);
         g.b = b.operand(b.wf(f.ws_Xh[c]), b.wf(f.ws_Xl[c]), d, d, false, false, split);
-        // the update reads T's lo part only when fp32-accurate.  T is an
-        // internal product: computed as a full (non-symmetric) product,
-        // which is faster than the lower tiles plus mirror stores of a
-        // symmetric one (measured 3.9 against 4.8 ms on 960 products of
-        // 1024^3); its two triangles may then differ in the last bit.
+        // the update reads T's lo part only when fp32-accurate.  T is
+        // symmetric: only the tiles touching the lower triangle are computed,
+        // written in full (mode 3; no mirror stores), and the update reads
+        // the K blocks beyond them from their transposes.
+        g.symmetric = 3;
         g.Chi = b.wf(f.ws_Th); g.Clo = split ? b.wf(f.ws_Tl) : nullptr; g.ldh = d;
         tgram.push_back(g);
         TcGemmDesc u = gemmtc(d, d, d, -0.5f, 1.5f);         // U' = 1.5 U - 0.5 U T
         u.a = b.operand(b.wf(f.ws_Xh[c]), b.wf(f.ws_Xl[c]), d, d, true, false, split);
         u.b = b.operand(b.wf(f.ws_Th), b.wf(f.ws_Tl), d, d, false, true, split);   // T symmetric
+        u.bt_hi = b.map(b.wf(f.ws_Th), d, d, 32, 1);
+        u.bt_lo = split ? b.map(b.wf(f.ws_Tl), d, d, 32, 1) : nullptr;
         // With TF32 products the iterates are TF32 numbers between steps:
         // a step after the first takes 1.5 U from U's TF32 value, and only
         // the last step writes fp32 U (the products' own TF32 rounding

@@ -23,8 +23,15 @@ struct TcOperand {
 // Chi = RN(v), Clo = RN(v - Chi) with leading dimension ldh.  symmetric:
 // only tiles touching the lower triangle run; 1: every element below the
 // diagonal is also written to its mirror position; 2: only the lower
-// triangle (diagonal included) is written.  skip: problem skipped
-// when *skip != 0.  c_ref: C taken from the per-call pointer tables.
+// triangle (diagonal included) is written; 3: the running tiles are
+// written in full (a symmetric matrix stored by those tiles, read back
+// through bt_hi/bt_lo).  skip: problem skipped when *skip != 0.  c_ref: C
+// taken from the per-call pointer tables.
+//
+// bt_hi/bt_lo (optional): op(B) is a symmetric matrix stored only in the
+// tiles of a symmetric-mode-3 product of this tile width, and b reads it
+// K-major (op(B)[k, n] = X[n, k]).  K blocks at or beyond n0 + BN, outside
+// the stored tiles, read X[k, n] instead through these MN-major maps of X.
 struct TcGemmDesc {
   int32_t M, N, K;
   int32_t symmetric;
@@ -43,6 +50,8 @@ struct TcGemmDesc {
   // when symmetric) of the deviation sum of plan.h; the diagonal's share
   // comes from the diagonal kernel
   unsigned long long* devsq;
+  const CUtensorMap* bt_hi;
+  const CUtensorMap* bt_lo;
 };
 
 // Tile width N of the kernel instance: 256 (TF32), 128 (split), or 64
