@@ -341,18 +341,29 @@ shampoo4_status launch_shift(const ShiftDesc* d_desc, int count, cudaStream_t st
 }
 
 // ---- fp32-storage Cholesky panel (fp64 inside) ------------------------------
-// Factor the jb x jb diagonal block, then (if requested) invert the factor:
-// thread c forms column c of L^-1 by forward substitution.
-constexpr int kPotrfFSmem = 2 * kPanel * (kPanel + 1) * 8;
+// Factor the jb x jb diagonal block, then (if requested) invert the factor.
+// Shared memory: the factor and the inverse as fp64 64 x 65 arrays (for the
+// coalesced write-out and the inverse's column reads) and two
+// double-buffered 64-vectors.
+constexpr int kPotrfFSmem = (2 * kPanel * (kPanel + 1) + 4 * kPanel) * 8;
 
-// One 64 x 64 block per CTA, fp64 in shared memory, 256 threads as a
-// 16 x 16 grid (thread (ty, tx) owns rows ty + 16 i and columns tx + 16 j).
-// Both loops keep columns (or rows) unscaled while they are read -- the
-// LDL^T form: A[r][s] -= A[r][c] A[s][c] / A[c][c] -- so that a step reads
-// only values no thread writes in that step, and one barrier per step
-// suffices; the square roots and divisions are applied once at the end.
-// Padding beyond jb is the identity in the factorization and zero in the
-// written inverse.
+// One 64 x 64 block per CTA, fp64, 256 threads as a 16 x 16 grid: thread
+// (ty, tx) holds rows ty + 16 i and columns tx + 16 j (i, j < 4) of the
+// factor and of the inverse in registers.  The factorization keeps columns
+// unscaled while they are read -- the LDL^T form: A[r][s] -= A[r][c]
+// A[s][c] / A[c][c] -- and the inverse X = U^-1 of the unit-lower factor
+// (U[r][k] = A[r][k] / A[k][k]) runs by rows, right-looking, in the same
+// sweep: step c needs column c of A and row c of X, both final by then.
+// Their owners publish them to double-buffered shared vectors, so one
+// barrier per step suffices, and the two sequential chains are one.  The
+// square roots and divisions are applied once at the end: L = U D^1/2,
+// L^-1 = D^-1/2 U^-1.  Padding beyond jb is the identity in the
+// factorization and zero in the written inverse.
+template <int N>
+__device__ __forceinline__ double pick4(const double (&v)[N], int j) {
+  return j == 0 ? v[0] : (j == 1 ? v[1] : (j == 2 ? v[2] : v[3]));
+}
+
 __global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ descs,
                                                  const uint32_t* __restrict__ guard) {
   if (guard && *guard == 0u) return;                      // no factor needs this launch
@@ -362,21 +373,44 @@ __global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ 
   extern __shared__ double sm_potrf[];
   double (*A)[kPanel + 1] = reinterpret_cast<double (*)[kPanel + 1]>(sm_potrf);
   double (*X)[kPanel + 1] = reinterpret_cast<double (*)[kPanel + 1]>(sm_potrf + kPanel * (kPanel + 1));
+  double (*vec)[kPanel] = reinterpret_cast<double (*)[kPanel]>(sm_potrf + 2 * kPanel * (kPanel + 1));
   __shared__ int bad;
   const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
-  for (int r = t >> 6; r < kPanel; r += 4) {
-    const int c = t & 63;
-    A[r][c] = (r < jb && c <= r) ? double(g.A[int64_t(r) * g.ld + c]) : (r == c ? 1.0 : 0.0);
-    X[r][c] = (r == c) ? 1.0 : 0.0;
+  double a[4][4], x[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = ty + 16 * i;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = tx + 16 * j;
+      a[i][j] = (r < jb && c <= r) ? double(g.A[int64_t(r) * g.ld + c]) : (r == c ? 1.0 : 0.0);
+      x[i][j] = r == c ? 1.0 : 0.0;
+    }
   }
   if (t == 0) bad = 0;
-  __syncthreads();
-  // factorization: after step c, A[c][c] is the pivot d_c and column c
-  // below it holds L[:, c] sqrt(d_c)
+  // step c: after it, A[c][c] is the pivot d_c, column c below it holds
+  // L[:, c] sqrt(d_c), and rows > c of X have taken column c of U
   for (int c = 0; c < jb; ++c) {
-    double p = A[c][c];
-    if (!(p > double(g.min_pivot)) || !isfinite(p)) {
-      if (t == 0) bad = 1;
+    double* col = vec[c & 1];
+    double* row = vec[2 + (c & 1)];
+    if (tx == (c & 15)) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        double v[4] = {a[i][0], a[i][1], a[i][2], a[i][3]};
+        col[ty + 16 * i] = pick4(v, c >> 4);
+      }
+    }
+    if (ty == (c & 15)) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        double v[4] = {x[0][j], x[1][j], x[2][j], x[3][j]};
+        row[tx + 16 * j] = pick4(v, c >> 4);
+      }
+    }
+    __syncthreads();
+    double p = col[c];
+    if (!(p > double(g.min_pivot)) || !isfinite(p)) {      // breakdown: a pivot of 1 keeps
+      if (t == 0) bad = 1;                                  // everything below finite
       p = 1.0;
     }
     const double ip = 1.0 / p;
@@ -384,38 +418,29 @@ __global__ void __launch_bounds__(256) k_potrf_f(const PotrfDescF* __restrict__ 
     for (int i = 0; i < 4; ++i) {
       const int r = ty + 16 * i;
       if (r <= c || r >= jb) continue;
-      const double arc = A[r][c] * ip;
+      const double arc = col[r] * ip;                       // also U[r][c]
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const int s2 = tx + 16 * jj;
-        if (s2 > c && s2 <= r) A[r][s2] = fma(-arc, A[s2][c], A[r][s2]);
+        if (s2 > c && s2 <= r) a[i][jj] = fma(-arc, col[s2], a[i][jj]);
+        if (s2 <= c) x[i][jj] = fma(-arc, row[s2], x[i][jj]);
       }
     }
-    __syncthreads();
   }
-  // pivots: breakdown leaves 1 so that nothing below is NaN
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      A[ty + 16 * i][tx + 16 * j] = a[i][j];
+      X[ty + 16 * i][tx + 16 * j] = x[i][j];
+    }
+  __syncthreads();
+  // pivots of the write-out: a breakdown's 1, as in the sweep
   for (int c = t; c < kPanel; c += blockDim.x) {
     const double p = A[c][c];
     if (c < jb && (!(p > double(g.min_pivot)) || !isfinite(p))) A[c][c] = 1.0;
   }
   __syncthreads();
-  // inverse of the unit-lower factor U (U[r][k] = A[r][k] / d_k, r > k):
-  // X <- U^-1 by rows, right-looking; then L^-1 = D^-1/2 U^-1
-  for (int k = 0; k < jb; ++k) {
-    const double ik = 1.0 / A[k][k];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = ty + 16 * i;
-      if (r <= k || r >= jb) continue;
-      const double urk = A[r][k] * ik;
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int c2 = tx + 16 * jj;
-        if (c2 <= k) X[r][c2] = fma(-urk, X[k][c2], X[r][c2]);
-      }
-    }
-    __syncthreads();
-  }
   // write L = U D^1/2 (fp32 + split) and L^-1 = D^-1/2 U^-1 (split, zero
   // outside jb x jb)
   for (int r = t >> 6; r < kPanel; r += 4) {
