@@ -47,7 +47,7 @@ class Config(C.Structure):
 
 class GraftConfig(C.Structure):
     _fields_ = [("kind", C.c_int32), ("beta1", C.c_float), ("beta2", C.c_float),
-                ("adam_eps", C.c_float), ("graft_eps", C.c_float)]
+                ("adam_eps", C.c_float), ("graft_eps", C.c_float), ("dir_norms", C.c_int32)]
 
 
 class Param(C.Structure):

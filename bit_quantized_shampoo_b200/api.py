@@ -120,10 +120,12 @@ class Shampoo4:
                 state[ov.value:ov.value + n].view(torch.float32).view(r, c))
 
     def graft_update(self, state, step, lr, grads, dirs, weights, kind="adam", beta1=0.9, beta2=0.999,
-                     adam_eps=1e-8, graft_eps=1e-16, stream=None):
+                     adam_eps=1e-8, graft_eps=1e-16, dir_norms=False, stream=None):
         """W <- W - lr * ||d_graft|| / (||D|| + graft_eps) * D per tile, in place
-        on ``weights``; ``dirs`` is this step's precondition output."""
-        cfg = L.GraftConfig(_graft_kind(kind), beta1, beta2, adam_eps, graft_eps)
+        on ``weights``; ``dirs`` is this step's precondition output.
+        dir_norms: take ||D|| as the last precondition recorded it (``dirs``
+        must be that call's output, unmodified), so D is read once."""
+        cfg = L.GraftConfig(_graft_kind(kind), beta1, beta2, adam_eps, graft_eps, 1 if dir_norms else 0)
         p, ld = self._ptrs(grads, "grads")
         q, ldq = self._ptrs(dirs, "dirs")
         w, ldw = self._ptrs(weights, "weights")

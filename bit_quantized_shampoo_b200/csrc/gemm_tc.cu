@@ -227,6 +227,7 @@ struct EpiArgs {
   float* Chi; float* Clo; int64_t ldh;
   const float* Cin; int64_t ldcin;
   unsigned long long* devsq;
+  double* sumsq;
 
   __device__ __forceinline__ void load(const TcGemmDesc& g, const PtrEntry* tabs, int nparams) {
     M = g.M; N = g.N; out_round = g.out_round;
@@ -241,6 +242,41 @@ struct EpiArgs {
     Chi = g.Chi; Clo = g.Clo; ldh = g.ldh;
     Cin = g.Cin; ldcin = g.ldcin;
     devsq = g.devsq;
+    sumsq = C ? g.sumsq : nullptr;
+  }
+  // Sum of squares of the C values of one lane's row segment (columns
+  // cb .. cb + 31 below N; the symmetric triangle as written).  A full
+  // segment of a plain product sums in fp32 (eight chains of four fused
+  // multiply-adds, then pairwise: within 7 units of fp32 rounding of the
+  // segment's sum), the rest in fp64.
+  __device__ __forceinline__ double seg_sumsq(const float (&v)[32], int64_t row, int cb) const {
+    if (cb + 32 <= N && !symmetric && !out_round) {
+      float s[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) s[k] = v[k] * v[k];
+#pragma unroll
+      for (int j = 8; j < 32; j += 8)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s[k] = fmaf(v[j + k], v[j + k], s[k]);
+      return double(((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7])));
+    }
+    double acc = 0.0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int c = cb + j;
+      if (c < N && (!symmetric || c <= row)) {
+        const double x = double(out_round ? rn_tf32(v[j]) : v[j]);
+        acc = fma(x, x, acc);
+      }
+    }
+    return acc;
+  }
+  // The warp's share of the tile's sum of squares into its slot.
+  __device__ __forceinline__ void put_sumsq(double acc, int m0, int n0, int bn, int q, int lane) const {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    const int tiles_n = (N + bn - 1) / bn;
+    if (lane == 0) sumsq[4 * ((m0 / 128) * tiles_n + n0 / bn) + q] = acc;
   }
   // One element to every requested output: C (optionally TF32-rounded) and
   // the TF32 split (Chi, Clo).
@@ -307,6 +343,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmDesc& g, const PtrEntr
   const uint32_t wsm = smem_u32(wbuf);
   const uint32_t my_row = uint32_t(lane * Cfg::kPitch * 4);
   unsigned long long dev_fine = 0;                      // deviation sum, plan.h units
+  double ss_acc = 0.0;                                  // sum of squares of C (sumsq)
   // Cin chunk i into buffer i & 1 with 16-byte cp.async pieces, four
   // full 128-byte rows per warp instruction: lane l copies rows
   // 4 t + l / 8 (t < 8), columns 4 (l % 8).  One group per chunk.
@@ -377,6 +414,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmDesc& g, const PtrEntr
           dev_fine += w * static_cast<unsigned long long>(fminf(q, kDevFineClamp) * kDevFineUnit);
         }
       }
+      if (e.sumsq && row_ok) ss_acc += e.seg_sumsq(v, row, cb);
       // row segment: columns cb.. of this lane's row (only col <= row
       // when the product is symmetric)
       const bool below = !e.symmetric || cb + 31 < rbase;   // whole chunk left of every row
@@ -452,6 +490,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmDesc& g, const PtrEntr
     }
     cp_async_wait<0>();                                 // nothing in flight into the buffers
   }
+  if (e.sumsq && i_lo == 0) e.put_sumsq(ss_acc, m0, n0, BN, q, lane);   // every warp of the tile, once
 }
 
 template <int BN, bool SPLIT, int STAGES>
@@ -656,7 +695,9 @@ __device__ __forceinline__ bool pers_tile(const TcGemmDesc* __restrict__ descs, 
 
 // Outputs of one tile from the accumulator values in registers (lane l of
 // epilogue warp q holds row m0 + 32 q + l, columns n0 + 32 i + j in
-// v[i][j]).  Same outputs and rounding as epilogue_tile.
+// v[i][j]).  Same outputs and rounding as epilogue_tile, except the sum of
+// squares (sumsq), which only the one-tile-per-CTA kernels record: in this
+// epilogue, at the register limit, it cost the QR solve products 8%.
 template <int BN>
 __device__ __forceinline__ void epilogue_regs(const TcGemmDesc& g, const PtrEntry* __restrict__ tabs, int nparams,
                                               int m0, int n0, float (&v)[BN / 32][32], int q, int lane,

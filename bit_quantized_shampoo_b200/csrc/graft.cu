@@ -10,6 +10,8 @@
 // Both passes are HBM-bound elementwise sweeps:
 //   k_graft_norms  reads G, D (and m, v), writes m, v, and one fp64 pair of
 //                  partial sums (sum d_graft^2, sum D^2) per band of rows;
+//                  with recorded norms (dir_norms) a tensor-core tile's sum
+//                  D^2 comes from the apply's epilogue and D is not read;
 //   k_graft_apply  sums its tile's partials in a fixed order (the result is
 //                  independent of scheduling), then W <- W - r D with one
 //                  fused multiply-add per element, r rounded to fp32 once.
@@ -47,11 +49,11 @@ __device__ __forceinline__ void block_sum2(double& x, double& y) {
   }
 }
 
-template <bool kAdam>
-__global__ void __launch_bounds__(kGraftThreads) k_graft_norms(const GraftArgs a) {
-  const GraftItem it = a.items[blockIdx.x];
-  double sg = 0.0, sd = 0.0;
-  if (a.bflag[it.block] == 0u) {
+// Moments and the item's partial sums; kReadD: D's sum of squares from D
+// itself (else it was recorded by the apply and is added in k_graft_apply).
+template <bool kAdam, bool kReadD>
+__device__ __forceinline__ void graft_norms_item(const GraftArgs& a, const GraftItem& it, double& sg, double& sd) {
+  {
     const PtrEntry eg = a.tabs[it.param], ed = a.tabs[a.nparams + it.param];
     const float* G = eg.ptr + it.r0 * eg.ld + it.c0;
     const float* D = ed.ptr + it.r0 * ed.ld + it.c0;
@@ -68,7 +70,7 @@ __global__ void __launch_bounds__(kGraftThreads) k_graft_norms(const GraftArgs a
       for (int e = threadIdx.x; e < n4; e += kGraftThreads) {
         const int r = e / c4n, c = (e - r * c4n) * 4;
         const float4 g = *reinterpret_cast<const float4*>(G + r * eg.ld + c);
-        const float4 d = *reinterpret_cast<const float4*>(D + r * ed.ld + c);
+        const float4 d = kReadD ? *reinterpret_cast<const float4*>(D + r * ed.ld + c) : make_float4(0.f, 0.f, 0.f, 0.f);
         float4 m = make_float4(0.f, 0.f, 0.f, 0.f), v = m;
         if (kAdam) {
           m = *reinterpret_cast<const float4*>(M + r * it.state_ld + c);
@@ -88,7 +90,7 @@ __global__ void __launch_bounds__(kGraftThreads) k_graft_norms(const GraftArgs a
     } else {
       for (int r = 0; r < it.rows; ++r)
         for (int c = threadIdx.x; c < it.cols; c += kGraftThreads) {
-          const float g = G[r * eg.ld + c], d = D[r * ed.ld + c];
+          const float g = G[r * eg.ld + c], d = kReadD ? D[r * ed.ld + c] : 0.0f;
           float m = 0.f, v = 0.f;
           if (kAdam) { m = M[r * it.state_ld + c]; v = V[r * it.state_ld + c]; }
           const float q = graft_dir<kAdam>(a, g, m, v);
@@ -97,6 +99,16 @@ __global__ void __launch_bounds__(kGraftThreads) k_graft_norms(const GraftArgs a
           sd += double(d) * d;
         }
     }
+  }
+}
+
+template <bool kAdam>
+__global__ void __launch_bounds__(kGraftThreads) k_graft_norms(const GraftArgs a) {
+  const GraftItem it = a.items[blockIdx.x];
+  double sg = 0.0, sd = 0.0;
+  if (a.bflag[it.block] == 0u) {
+    if (a.use_dsq && it.dsq_n > 0) graft_norms_item<kAdam, false>(a, it, sg, sd);
+    else graft_norms_item<kAdam, true>(a, it, sg, sd);
   }
   block_sum2(sg, sd);
   if (threadIdx.x == 0) {
@@ -116,6 +128,8 @@ __global__ void __launch_bounds__(kGraftThreads) k_graft_apply(const GraftArgs a
       sg += a.parts[2 * int64_t(it.part0 + i)];
       sd += a.parts[2 * int64_t(it.part0 + i) + 1];
     }
+    if (a.use_dsq && it.dsq_n > 0)                          // D's norm as the apply recorded it
+      for (int i = 0; i < it.dsq_n; ++i) sd += a.dsq[it.dsq_off + i];
     const double den = sqrt(sd) + a.graft_eps;
     const double r = den > 0.0 ? a.lr * (sqrt(sg) / den) : 0.0;
     const float rf = float(r);

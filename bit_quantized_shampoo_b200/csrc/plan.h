@@ -291,6 +291,8 @@ struct GraftItem {
   int32_t part0, nparts;       // the tile's first item and its item count
   int64_t m_off, v_off;        // element offsets of the band origin's moments
   int64_t state_ld;            // moments are dense per parameter: ld = cols
+  int64_t dsq_off;             // the tile's recorded sums of squares of D
+  int32_t dsq_n, pad_;         // (0: none; a CUDA-core tile)
 };
 
 struct GraftArgs {
@@ -304,6 +306,8 @@ struct GraftArgs {
   double* parts;               // 2 * nitems
   uint32_t* flags;             // status word
   int32_t kind;
+  const double* dsq;           // recorded sums of squares of D (use_dsq)
+  int32_t use_dsq;
   float beta1, beta2, omb1, omb2;       // omb = 1 - beta, in fp32
   float c1, c2;                         // 1 / (1 - beta^t)
   float adam_eps;

@@ -70,6 +70,8 @@ struct BlockPlan {
   bool tc;
   size_t ws_Gh, ws_Gl, ws_Bh, ws_Bl;   // tensor-core path: G split, apply intermediate split
   size_t ws_tmp;                       // CUDA-core path: apply intermediate
+  int64_t dsq_off = 0;                 // tensor-core path: the apply's recorded sums of squares
+  int32_t dsq_n = 0;                   // of D (4 per output tile), in the ws_dsq array
 };
 
 // Per-factor workspace.  Tensor-core factors: fp32/TF32-split triplets
@@ -170,6 +172,8 @@ struct shampoo4_ctx {
   // grafted weight update: bands of tile rows, the moments' layout, and a
   // per-call pointer table of its own (gradients, directions, weights)
   std::vector<GraftItem> graft_items;
+  size_t ws_dsq = 0;                     // sums of squares of D recorded by the apply
+  bool dsq_valid = false;                // a precondition has recorded them
   std::vector<size_t> graft_off_m, graft_off_v;   // bytes, per parameter
   size_t graft_state_bytes = 0;
   size_t ws_gtab = 0, ws_gitems = 0, ws_gparts = 0;
@@ -214,6 +218,18 @@ void plan_graft(shampoo4_ctx* h, size_t& ws) {
     h->graft_off_v[p] = take(gs, 4 * elems);
   }
   h->graft_state_bytes = align_up(gs, kAlign);
+  // the apply's recorded sums of squares: 4 per output tile of a
+  // tensor-core tile's D = B P_R, in TF32 mode (the fp32-accurate apply runs
+  // the persistent kernel, which does not record them)
+  int64_t nd = 0;
+  const bool record = h->cfg.precision != SHAMPOO4_PREC_FP32;
+  const int bn = tc_block_n(0);
+  for (auto& b : h->blocks) {
+    b.dsq_off = nd;
+    b.dsq_n = (b.tc && record) ? 4 * ((b.m + 127) / 128) * ((b.n + bn - 1) / bn) : 0;
+    nd += b.dsq_n;
+  }
+  h->ws_dsq = take(ws, 8 * size_t(std::max<int64_t>(nd, 1)));
   for (size_t k = 0; k < h->blocks.size(); ++k) {
     const BlockPlan& b = h->blocks[k];
     const int64_t cols = h->params[b.param].cols;
@@ -234,6 +250,8 @@ void plan_graft(shampoo4_ctx* h, size_t& ws) {
       it.m_off = int64_t(h->graft_off_m[b.param] / 4) + e;
       it.v_off = int64_t(h->graft_off_v[b.param] / 4) + e;
       it.state_ld = cols;
+      it.dsq_off = b.dsq_off;
+      it.dsq_n = b.dsq_n;
       h->graft_items.push_back(it);
     }
   }
@@ -1779,6 +1797,7 @@ void build_precondition_into(Builder& b, std::vector<Launch>& prog) {
       const bool sym = h->cfg.root_method != SHAMPOO4_ROOT_NEWTON_Q4;
       r.b = b.operand(b.wf(fr.ws_Th), b.wf(fr.ws_Tl), bp.n, bp.n, false, sym, split);
       r.c_ref = {1, bp.param, bp.r0, bp.c0};
+      r.sumsq = bp.dsq_n ? b.wd(h->ws_dsq) + bp.dsq_off : nullptr;   // ||D||^2 for the grafted update
       tright.push_back(r);
     } else {
       float* tmp = b.wf(bp.ws_tmp);
@@ -2214,7 +2233,9 @@ extern "C" shampoo4_status shampoo4_precondition(shampoo4_handle h, const float*
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   S4_TRY(set_tables(h, d_grads, ld, d_out, ld_out, st));
-  return run_program(h, h->prog_precond, st);
+  S4_TRY(run_program(h, h->prog_precond, st));
+  h->dsq_valid = true;                  // the apply recorded ||D||^2 per tile
+  return SHAMPOO4_OK;
 }
 
 extern "C" shampoo4_status shampoo4_get_status_flags(shampoo4_handle h, uint32_t* flags,
@@ -2373,6 +2394,7 @@ namespace {
 bool graft_config_ok(const shampoo4_graft_config* c) {
   if (!c) return false;
   if (c->kind != SHAMPOO4_GRAFT_SGD && c->kind != SHAMPOO4_GRAFT_ADAM) return false;
+  if (c->dir_norms != 0 && c->dir_norms != 1) return false;
   if (!(c->graft_eps >= 0.0f) || !std::isfinite(c->graft_eps)) return false;
   if (c->kind == SHAMPOO4_GRAFT_ADAM) {
     if (!(c->beta1 >= 0.0f && c->beta1 < 1.0f) || !(c->beta2 >= 0.0f && c->beta2 < 1.0f)) return false;
@@ -2473,6 +2495,11 @@ extern "C" shampoo4_status shampoo4_graft_update(shampoo4_handle h, const shampo
   a.adam_eps = cfg->adam_eps;
   a.lr = double(lr);
   a.graft_eps = double(cfg->graft_eps);
+  if (cfg->dir_norms) {
+    if (!h->dsq_valid) return SHAMPOO4_ERR_NOT_READY;
+    a.use_dsq = 1;
+    a.dsq = reinterpret_cast<const double*>(h->d_ws + h->ws_dsq);
+  }
   return launch_graft(a, st);
 }
 

@@ -52,6 +52,12 @@ struct TcGemmDesc {
   unsigned long long* devsq;
   const CUtensorMap* bt_hi;
   const CUtensorMap* bt_lo;
+  // optional (TF32 and 64-wide instances; the persistent 128-wide one
+  // ignores it): the sum of squares (fp64) of the values each epilogue warp
+  // writes to C, at sumsq[4 * (tile_row * tiles_n + tile_col) + warp]
+  // (tiles_n = ceil(N / tile width)); every running tile writes its four
+  // slots, so the sum over them, in any fixed order, is ||C||_F^2
+  double* sumsq;
 };
 
 // Tile width N of the kernel instance: 256 (TF32), 128 (split), or 64

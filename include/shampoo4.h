@@ -455,6 +455,16 @@ typedef struct {
   float beta1, beta2;    /* Adam moment decays, in [0, 1) (ignored for SGD)   */
   float adam_eps;        /* Adam's denominator epsilon, >= 0                  */
   float graft_eps;       /* epsilon of the norm ratio, >= 0                   */
+  int32_t dir_norms;     /* 0: ||D_b|| from d_dirs.  1: from the last
+                            shampoo4_precondition on this handle, whose
+                            tensor-core apply records each tile's sum of
+                            squares as it writes D (fp32 sums of 32-element
+                            row segments, added in fp64, then summed here in
+                            a fixed order), so D is read once; d_dirs must
+                            then be that call's output, unmodified.  Tiles on
+                            the CUDA-core path, and every tile in FP32
+                            precision, still read D.  Before any
+                            precondition: SHAMPOO4_ERR_NOT_READY.            */
 } shampoo4_graft_config;
 
 /* Bytes of grafting state the caller provides for this handle's parameters:

@@ -32,9 +32,9 @@ def _rng_list(shapes, seed, scale):
     return [(r.standard_normal(s) * scale).astype(np.float32) for s in shapes]
 
 
-def _run(kind, shapes, max_block, steps=3, lr=1e-2, nan_tile=None):
+def _run(kind, shapes, max_block, steps=3, lr=1e-2, nan_tile=None, dir_norms=False, precision="tf32"):
     from bit_quantized_shampoo_b200 import api
-    sh = api.Shampoo4(shapes, max_block=max_block, precision="tf32")
+    sh = api.Shampoo4(shapes, max_block=max_block, precision=precision)
     go = GO.GraftOracle(shapes, kind=GO.GRAFT_ADAM if kind == "adam" else GO.GRAFT_SGD,
                         max_block=max_block)
     state = sh.graft_state(kind)
@@ -53,7 +53,7 @@ def _run(kind, shapes, max_block, steps=3, lr=1e-2, nan_tile=None):
         torch.cuda.synchronize()
         w_before = [w.cpu().numpy() for w in W]
         d_host = [d.cpu().numpy() for d in D]
-        sh.graft_update(state, t, lr, G, D, W, kind=kind)
+        sh.graft_update(state, t, lr, G, D, W, kind=kind, dir_norms=dir_norms)
         torch.cuda.synchronize()
         want = go.step(t, lr, g_host, d_host, w_before)
         got = [w.cpu().numpy() for w in W]
@@ -66,11 +66,14 @@ def _run(kind, shapes, max_block, steps=3, lr=1e-2, nan_tile=None):
     return sh, go, results
 
 
+@pytest.mark.parametrize("dir_norms", [False, True])
 @pytest.mark.parametrize("kind", ["sgd", "adam"])
 @pytest.mark.parametrize("case", sorted(CASES))
-def test_graft_update_matches_oracle(kind, case):
+def test_graft_update_matches_oracle(kind, case, dir_norms):
+    # dir_norms: ||D_b|| as the apply recorded it while writing D (the
+    # oracle still takes it from D itself)
     shapes, max_block = CASES[case]
-    sh, go, results = _run(kind, shapes, max_block)
+    sh, go, results = _run(kind, shapes, max_block, dir_norms=dir_norms)
     for t, (before, want, got) in enumerate(results, 1):
         for p in range(len(shapes)):
             step_o = want[p].astype(np.float64) - before[p]
@@ -82,6 +85,29 @@ def test_graft_update_matches_oracle(kind, case):
     # fp64 (an informational flag); nothing else may be raised
     from bit_quantized_shampoo_b200 import _lib
     assert sh.status_flags() & ~_lib.FLAG_QR_FALLBACK == 0
+
+
+def test_graft_recorded_norms_fp32_path():
+    # the fp32-accurate apply (persistent 3xTF32 kernel) records no ||D||^2:
+    # with dir_norms the update reads D for every tile
+    shapes, max_block = [(1100, 704), (64, 48)], 512
+    sh, go, results = _run("adam", shapes, max_block, steps=2, dir_norms=True, precision="fp32")
+    for t, (before, want, got) in enumerate(results, 1):
+        for p in range(len(shapes)):
+            e = rel_fro(got[p].astype(np.float64) - before[p], want[p].astype(np.float64) - before[p])
+            print(f"fp32 recorded norms t={t} param {p}: step {e:.2e}")
+            assert e <= TOL_STEP, (t, p)
+
+
+def test_graft_recorded_norms_need_a_precondition():
+    from bit_quantized_shampoo_b200 import api, _lib
+    shapes = [(128, 96)]
+    sh = api.Shampoo4(shapes, max_block=128, precision="tf32")
+    G = [cuda_f32(x) for x in _rng_list(shapes, 3, 1.0)]
+    W = [torch.zeros(shapes[0], dtype=torch.float32, device="cuda")]
+    sh.update_stats(G)
+    with pytest.raises(_lib.Shampoo4Error):
+        sh.graft_update(None, 1, 0.1, G, G, W, kind="sgd", dir_norms=True)
 
 
 def test_graft_step_norm_per_tile_on_the_gpu():
