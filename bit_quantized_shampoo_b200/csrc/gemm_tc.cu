@@ -210,6 +210,12 @@ __device__ __forceinline__ void load_operand(const CUtensorMap* map, const TcOpe
 __device__ __forceinline__ bool b_transposed(const CUtensorMap* bt_hi, int k0, int n0, int bn) {
   return bt_hi != nullptr && k0 >= n0 + bn;
 }
+// The same for the A operand of an output tile at row m0: the stored tiles
+// of the symmetric operand (width bn) cover K block k0 of rows m0.. when
+// its bn-wide block starts below m0 + 128.
+__device__ __forceinline__ bool a_transposed(const CUtensorMap* at_hi, int k0, int m0, int bn) {
+  return at_hi != nullptr && (k0 / bn) * bn >= m0 + kBM;
+}
 
 __device__ __forceinline__ uint64_t operand_desc(const TcOperand& op, uint32_t base, int kk) {
   // K-major (128 B swizzle): rows of 128 B, 8-row groups 1024 B apart; a K
@@ -552,6 +558,9 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
       const CUtensorMap* bt_lo = g.bt_lo;
       TcOperand gt = gb;                                    // transposed reads of B
       gt.hi = bt_hi; gt.lo = bt_lo; gt.mn_major = 1;
+      const CUtensorMap* at_hi = g.at_hi;
+      TcOperand gat = ga;                                   // transposed reads of A
+      gat.hi = at_hi; gat.lo = g.at_lo; gat.mn_major = 1;
       int issued = 0;
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % Cfg::kStages;
@@ -566,10 +575,11 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
         const int k0 = kb * kBK;
         const bool tr = b_transposed(bt_hi, k0, n0, BN);
         const TcOperand& ob = tr ? gt : gb;
-        load_operand(ga.hi, ga, kBM, m0, k0, st, &full_bar[s]);
+        const TcOperand& oa = a_transposed(at_hi, k0, m0, BN) ? gat : ga;
+        load_operand(oa.hi, oa, kBM, m0, k0, st, &full_bar[s]);
         load_operand(ob.hi, ob, BN, n0, k0, st + Cfg::kATile, &full_bar[s]);
         if (SPLIT) {
-          load_operand(ga.lo, ga, kBM, m0, k0, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+          load_operand(oa.lo, oa, kBM, m0, k0, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
           load_operand(ob.lo, ob, BN, n0, k0, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
         }
         issued = kb + 1;
@@ -586,10 +596,10 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
     if (lane == 0) {                                        // ---- MMA issuer
       const TcOperand ga = g.a, gb = g.b;                   // registers, as in the producer
       const CUtensorMap* bt_hi = g.bt_hi;
-      TcOperand gt = gb;
+      const CUtensorMap* at_hi = g.at_hi;
+      TcOperand gt = gb, gat = ga;
       gt.mn_major = 1;
-      const uint32_t idesc_n = idesc_tf32(kBM, BN, ga.mn_major, gb.mn_major);
-      const uint32_t idesc_t = idesc_tf32(kBM, BN, ga.mn_major, 1);
+      gat.mn_major = 1;
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % Cfg::kStages;
         if (!mbar_wait(&full_bar[s], (kb / Cfg::kStages) & 1, wait_ns)) {
@@ -602,18 +612,18 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
         const uint32_t st = smem_u32(smem + s * Cfg::kStage);
         const uint32_t a_hi = st, b_hi = st + Cfg::kATile;
         const uint32_t a_lo = st + Cfg::kATile + Cfg::kBTile, b_lo = a_lo + Cfg::kATile;
-        const bool tr = b_transposed(bt_hi, kb * kBK, n0, BN);
-        const TcOperand& ob = tr ? gt : gb;
-        const uint32_t idesc = tr ? idesc_t : idesc_n;
+        const TcOperand& ob = b_transposed(bt_hi, kb * kBK, n0, BN) ? gt : gb;
+        const TcOperand& oa = a_transposed(at_hi, kb * kBK, m0, BN) ? gat : ga;
+        const uint32_t idesc = idesc_tf32(kBM, BN, oa.mn_major, ob.mn_major);
 #pragma unroll
         for (int kk = 0; kk < kBK / 8; ++kk) {
           // first MMA into accumulator kb mod kAcc overwrites it
           const uint32_t acc = (kb >= Cfg::kAcc || kk != 0) ? 1u : 0u;
           const uint32_t dt = tmem + uint32_t((kb % Cfg::kAcc) * BN);
-          mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(ob, b_hi, kk), idesc, acc);
+          mma_tf32(dt, operand_desc(oa, a_hi, kk), operand_desc(ob, b_hi, kk), idesc, acc);
           if (SPLIT) {
-            mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(ob, b_lo, kk), idesc, 1);
-            mma_tf32(dt, operand_desc(ga, a_lo, kk), operand_desc(ob, b_hi, kk), idesc, 1);
+            mma_tf32(dt, operand_desc(oa, a_hi, kk), operand_desc(ob, b_lo, kk), idesc, 1);
+            mma_tf32(dt, operand_desc(oa, a_lo, kk), operand_desc(ob, b_hi, kk), idesc, 1);
           }
         }
         mma_commit(&empty_bar[s]);                          // stage free once these MMAs finish
@@ -890,6 +900,9 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
         const CUtensorMap* bt_hi = descs[p].bt_hi;
         TcOperand gt = gb;                                  // transposed reads of B
         gt.hi = bt_hi; gt.lo = descs[p].bt_lo; gt.mn_major = 1;
+        const CUtensorMap* at_hi = descs[p].at_hi;
+        TcOperand gat = ga;                                 // transposed reads of A
+        gat.hi = at_hi; gat.lo = descs[p].at_lo; gat.mn_major = 1;
         const int kblocks = (descs[p].K + kBK - 1) / kBK;
         if (p != last_p) {
           asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(ga.hi)) : "memory");
@@ -913,10 +926,11 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
           const int k0 = kb * kBK;
           const bool tr = b_transposed(bt_hi, k0, n0, BN);
           const TcOperand& ob = tr ? gt : gb;
-          load_operand(ga.hi, ga, kBM, m0, k0, st, &full_bar[s]);
+          const TcOperand& oa = a_transposed(at_hi, k0, m0, BN) ? gat : ga;
+          load_operand(oa.hi, oa, kBM, m0, k0, st, &full_bar[s]);
           load_operand(ob.hi, ob, BN, n0, k0, st + Cfg::kATile, &full_bar[s]);
           if (SPLIT) {
-            load_operand(ga.lo, ga, kBM, m0, k0, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+            load_operand(oa.lo, oa, kBM, m0, k0, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
             load_operand(ob.lo, ob, BN, n0, k0, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
           }
         }
@@ -934,11 +948,11 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
         if (!pers_tile<BN>(descs, count, t, p, m0, n0)) continue;
         const TcOperand ga = descs[p].a, gb = descs[p].b;
         const CUtensorMap* bt_hi = descs[p].bt_hi;
-        TcOperand gt = gb;
+        const CUtensorMap* at_hi = descs[p].at_hi;
+        TcOperand gt = gb, gat = ga;
         gt.mn_major = 1;
+        gat.mn_major = 1;
         const int kblocks = (descs[p].K + kBK - 1) / kBK;
-        const uint32_t idesc_n = idesc_tf32(kBM, BN, ga.mn_major, gb.mn_major);
-        const uint32_t idesc_t = idesc_tf32(kBM, BN, ga.mn_major, 1);
         // the epilogue has read the previous tile's accumulators
         if (ntiles > 0 && !mbar_wait(&acc_empty, (ntiles - 1) & 1, wait_ns)) {
           atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
@@ -960,17 +974,17 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
           const uint32_t st = smem_u32(smem + s * Cfg::kStage);
           const uint32_t a_hi = st, b_hi = st + Cfg::kATile;
           const uint32_t a_lo = st + Cfg::kATile + Cfg::kBTile, b_lo = a_lo + Cfg::kATile;
-          const bool tr = b_transposed(bt_hi, kb * kBK, n0, BN);
-          const TcOperand& ob = tr ? gt : gb;
-          const uint32_t idesc = tr ? idesc_t : idesc_n;
+          const TcOperand& ob = b_transposed(bt_hi, kb * kBK, n0, BN) ? gt : gb;
+          const TcOperand& oa = a_transposed(at_hi, kb * kBK, m0, BN) ? gat : ga;
+          const uint32_t idesc = idesc_tf32(kBM, BN, oa.mn_major, ob.mn_major);
 #pragma unroll
           for (int kk = 0; kk < kBK / 8; ++kk) {
             const uint32_t acc = (kb >= Cfg::kAcc || kk != 0) ? 1u : 0u;
             const uint32_t dt = tmem + uint32_t((kb % Cfg::kAcc) * BN);
-            mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(ob, b_hi, kk), idesc, acc);
+            mma_tf32(dt, operand_desc(oa, a_hi, kk), operand_desc(ob, b_hi, kk), idesc, acc);
             if (SPLIT) {
-              mma_tf32(dt, operand_desc(ga, a_hi, kk), operand_desc(ob, b_lo, kk), idesc, 1);
-              mma_tf32(dt, operand_desc(ga, a_lo, kk), operand_desc(ob, b_hi, kk), idesc, 1);
+              mma_tf32(dt, operand_desc(oa, a_hi, kk), operand_desc(ob, b_lo, kk), idesc, 1);
+              mma_tf32(dt, operand_desc(oa, a_lo, kk), operand_desc(ob, b_hi, kk), idesc, 1);
             }
           }
           mma_commit(&empty_bar[s]);

@@ -1742,10 +1742,13 @@ void build_precondition_into(Builder& b, std::vector<Launch>& prog) {
       TcGemmDesc g = gemmtc(d, d, d, 1.0f, 0.0f);
       g.a = b.operand(b.wf(f.ws_Xh[1]), b.wf(f.ws_Xl[1]), d, d, true, false, split);
       g.b = b.operand(b.wf(f.ws_Xh[0]), b.wf(f.ws_Xl[0]), d, d, false, true, split);
-      // P is internal: a full product (faster than lower tiles plus mirror
-      // stores); its fp32 copy only feeds the CUDA-core apply of a tile
-      // that is not a tensor-core tile
+      // P is symmetric: for a tensor-core tile only the tiles touching its
+      // lower triangle are computed, written in full (mode 3), and the
+      // applies read the K blocks beyond them from their transposes.  Its
+      // fp32 copy feeds only the CUDA-core apply of a tile that is not a
+      // tensor-core tile, which reads all of it (a full product then).
       float* pm = h->blocks[f.block].tc ? nullptr : b.wf(f.ws_Xm[1]);
+      if (!pm) g.symmetric = 3;
       g.C = pm; g.ldc = d;
       g.Chi = b.wf(f.ws_Th); g.Clo = split ? b.wf(f.ws_Tl) : nullptr; g.ldh = d;
       troots.push_back(g);
@@ -1786,6 +1789,10 @@ void build_precondition_into(Builder& b, std::vector<Launch>& prog) {
     if (bp.tc) {
       TcGemmDesc l = gemmtc(bp.m, bp.n, bp.m, 1.0f, 0.0f);       // B = P_L G
       l.a = b.operand(b.wf(fl.ws_Th), b.wf(fl.ws_Tl), bp.m, bp.m, true, false, split);
+      if (!newton) {                                              // P_L stored by its lower tiles
+        l.at_hi = b.map(b.wf(fl.ws_Th), bp.m, bp.m, 32, 1);
+        l.at_lo = split ? b.map(b.wf(fl.ws_Tl), bp.m, bp.m, 32, 1) : nullptr;
+      }
       l.b = b.operand(b.wf(bp.ws_Gh), b.wf(bp.ws_Gl), bp.m, bp.n, false, false, split);
       l.Chi = b.wf(bp.ws_Bh); l.Clo = split ? b.wf(bp.ws_Bl) : nullptr; l.ldh = bp.n;
       tleft.push_back(l);
@@ -1796,6 +1803,10 @@ void build_precondition_into(Builder& b, std::vector<Launch>& prog) {
       // not, and is read as stored
       const bool sym = h->cfg.root_method != SHAMPOO4_ROOT_NEWTON_Q4;
       r.b = b.operand(b.wf(fr.ws_Th), b.wf(fr.ws_Tl), bp.n, bp.n, false, sym, split);
+      if (!newton) {                                              // P_R stored by its lower tiles
+        r.bt_hi = b.map(b.wf(fr.ws_Th), bp.n, bp.n, 32, 1);
+        r.bt_lo = split ? b.map(b.wf(fr.ws_Tl), bp.n, bp.n, 32, 1) : nullptr;
+      }
       r.c_ref = {1, bp.param, bp.r0, bp.c0};
       r.sumsq = bp.dsq_n ? b.wd(h->ws_dsq) + bp.dsq_off : nullptr;   // ||D||^2 for the grafted update
       tright.push_back(r);

@@ -32,6 +32,9 @@ struct TcOperand {
 // tiles of a symmetric-mode-3 product of this tile width, and b reads it
 // K-major (op(B)[k, n] = X[n, k]).  K blocks at or beyond n0 + BN, outside
 // the stored tiles, read X[k, n] instead through these MN-major maps of X.
+// at_hi/at_lo (optional): the same for op(A) = X read K-major: K blocks
+// whose BN-wide block starts at or beyond m0 + 128 read X[k, m] through
+// these MN-major maps.
 struct TcGemmDesc {
   int32_t M, N, K;
   int32_t symmetric;
@@ -52,6 +55,8 @@ struct TcGemmDesc {
   unsigned long long* devsq;
   const CUtensorMap* bt_hi;
   const CUtensorMap* bt_lo;
+  const CUtensorMap* at_hi;
+  const CUtensorMap* at_lo;
   // optional (TF32 and 64-wide instances; the persistent 128-wide one
   // ignores it): the sum of squares (fp64) of the values each epilogue warp
   // writes to C, at sumsq[4 * (tile_row * tiles_n + tile_col) + warp]
