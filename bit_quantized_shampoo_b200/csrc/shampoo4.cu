@@ -1397,12 +1397,17 @@ void build_refresh_owned(Builder& b, std::vector<Launch>& prog, bool first) {
       // step); without Björck steps the fp32-accurate subspace product
       // reads both parts
       if (f.tc) {
-        x.U = b.wf(f.ws_Xm[0]); x.Uh = b.wf(f.ws_Xh[0]);
+        // with TF32 Björck steps the dequantized U is read only through its
+        // TF32 value (the products' operand and the first step's 1.5 U): no
+        // fp32 copy is written
+        const bool tf32_bjorck = !split && !first && h->cfg.bjorck_iters > 0;
+        x.U = tf32_bjorck ? nullptr : b.wf(f.ws_Xm[0]); x.Uh = b.wf(f.ws_Xh[0]);
         x.Ul = (split || first || h->cfg.bjorck_iters == 0) ? b.wf(f.ws_Xl[0]) : nullptr;
       }
       else x.U = b.wf(f.ws_U);
       bd.push_back(x);
-      bytes += (first ? 0.0 : 0.5625) * double(f.d) * f.d + (f.tc ? 12.0 : 4.0) * double(f.d) * f.d;
+      bytes += (first ? 0.0 : 0.5625) * double(f.d) * f.d +
+               4.0 * ((x.U ? 1 : 0) + (x.Uh ? 1 : 0) + (x.Ul ? 1 : 0)) * double(f.d) * f.d;
     }
     b.tag = SHAMPOO4_STAGE_BASIS;
     b.emit(prog, Kind::Basis, bd, emax, 0, bytes);
@@ -1433,11 +1438,12 @@ void build_refresh_owned(Builder& b, std::vector<Launch>& prog, bool first) {
         u.bt_hi = b.map(b.wf(f.ws_Th), d, d, 32, 1);
         u.bt_lo = split ? b.map(b.wf(f.ws_Tl), d, d, 32, 1) : nullptr;
         // With TF32 products the iterates are TF32 numbers between steps:
-        // a step after the first takes 1.5 U from U's TF32 value, and only
-        // the last step writes fp32 U (the products' own TF32 rounding
-        // already limits the iteration to that precision).
+        // every step takes 1.5 U from U's TF32 value (the first from the
+        // dequantized U's), and only the last step writes fp32 U (the
+        // products' own TF32 rounding already limits the iteration to that
+        // precision).
         const bool last = it + 1 == iters;
-        u.Cin = (split || it == 0) ? b.wf(f.ws_Xm[c]) : b.wf(f.ws_Xh[c]); u.ldcin = d;
+        u.Cin = split ? b.wf(f.ws_Xm[c]) : b.wf(f.ws_Xh[c]); u.ldcin = d;
         u.C = (split || last) ? b.wf(f.ws_Xm[o]) : nullptr; u.ldc = d;
         // U's lo part feeds the next Björck products only when fp32-accurate;
         // the last one always feeds the fp32-accurate subspace product
