@@ -107,76 +107,110 @@ shampoo4_status launch_trsm(const TrsmDesc* d_desc, int count, int max_rows, cud
 }
 
 // ---- U = dequant(codes, scales) or I ------------------------------------
-// One CTA per row, each thread four consecutive columns: one 16-bit load of
-// codes, one scale (a 64-element block never splits a group of four), and
-// 16-byte stores of every output, so each warp writes 512 contiguous bytes.
-// Rows whose length is not a multiple of 4 take the element-wise path.
+// The matrix is walked as a flat array: each thread takes groups of 8
+// consecutive elements (4 code bytes, one scale, two 16-byte stores per
+// output), kBasisGroups groups per thread with all loads issued first.
+// A group that a row boundary splits (d not a multiple of 8) takes the
+// per-element path.
+constexpr int kBasisGroups = 2;
+constexpr int kBasisEltsPerCta = 256 * 8 * kBasisGroups;
+
+__device__ __forceinline__ void basis_put8(const BasisDesc& g, int64_t e0, int c0, const float (&v)[8]) {
+  if (g.U) {
+    float4* p = reinterpret_cast<float4*>(g.U + e0);
+    p[0] = make_float4(v[0], v[1], v[2], v[3]);
+    p[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+  if (g.Uh) {
+    float h[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) h[k] = tf32_rn(v[k]);
+    float4* ph = reinterpret_cast<float4*>(g.Uh + e0);
+    ph[0] = make_float4(h[0], h[1], h[2], h[3]);
+    ph[1] = make_float4(h[4], h[5], h[6], h[7]);
+    if (g.Ul) {
+      float4* pl = reinterpret_cast<float4*>(g.Ul + e0);
+      pl[0] = make_float4(tf32_rn(v[0] - h[0]), tf32_rn(v[1] - h[1]), tf32_rn(v[2] - h[2]), tf32_rn(v[3] - h[3]));
+      pl[1] = make_float4(tf32_rn(v[4] - h[4]), tf32_rn(v[5] - h[5]), tf32_rn(v[6] - h[6]), tf32_rn(v[7] - h[7]));
+    }
+  }
+  if (g.Vh) {
+    const float4 m0 = *reinterpret_cast<const float4*>(g.mu + c0);
+    const float4 m1 = *reinterpret_cast<const float4*>(g.mu + c0 + 4);
+    const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+    float w[8], h[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) { w[k] = v[k] * mm[k]; h[k] = tf32_rn(w[k]); }
+    float4* ph = reinterpret_cast<float4*>(g.Vh + e0);
+    ph[0] = make_float4(h[0], h[1], h[2], h[3]);
+    ph[1] = make_float4(h[4], h[5], h[6], h[7]);
+    if (g.Vl) {
+      float4* pl = reinterpret_cast<float4*>(g.Vl + e0);
+      pl[0] = make_float4(tf32_rn(w[0] - h[0]), tf32_rn(w[1] - h[1]), tf32_rn(w[2] - h[2]), tf32_rn(w[3] - h[3]));
+      pl[1] = make_float4(tf32_rn(w[4] - h[4]), tf32_rn(w[5] - h[5]), tf32_rn(w[6] - h[6]), tf32_rn(w[7] - h[7]));
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) k_basis(const BasisDesc* __restrict__ descs) {
   const BasisDesc& g = descs[blockIdx.y];
-  const int d = g.d, r = blockIdx.x;
-  if (r >= d) return;                                      // CTA-uniform
+  const int d = g.d;
+  const int64_t n = int64_t(d) * d;
+  const int64_t base = int64_t(blockIdx.x) * kBasisEltsPerCta;
+  if (base >= n) return;                                   // CTA-uniform
   __shared__ float level[16];
   if (threadIdx.x < 16) level[threadIdx.x] = level_f32(g.codebook, threadIdx.x);
-  __syncthreads();
-  const int c0 = threadIdx.x * 4;
-  if (c0 >= d) return;
-  const int64_t e0 = int64_t(r) * d + c0;
-  if ((d & 3) == 0) {
-    float v[4];
-    if (g.identity) {
+  const bool vec = (d & 7) == 0;
+  uint32_t packed[kBasisGroups];
+  float sc[kBasisGroups];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) v[k] = (r == c0 + k) ? 1.0f : 0.0f;
-    } else {
-      const uint32_t packed = *reinterpret_cast<const uint16_t*>(g.codes + (e0 >> 1));
-      const float sc = g.scales[e0 / kQuantBlock];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) v[k] = level[(packed >> (4 * k)) & 15u] * sc;
+  for (int q = 0; q < kBasisGroups; ++q) {                 // loads first
+    const int64_t e0 = base + (int64_t(q) * 256 + threadIdx.x) * 8;
+    packed[q] = 0;
+    sc[q] = 0.0f;
+    if (vec && !g.identity && e0 < n) {
+      packed[q] = *reinterpret_cast<const uint32_t*>(g.codes + (e0 >> 1));
+      sc[q] = g.scales[e0 / kQuantBlock];
     }
-    if (g.U) *reinterpret_cast<float4*>(g.U + e0) = make_float4(v[0], v[1], v[2], v[3]);
-    if (g.Uh) {
-      const float4 h = make_float4(tf32_rn(v[0]), tf32_rn(v[1]), tf32_rn(v[2]), tf32_rn(v[3]));
-      *reinterpret_cast<float4*>(g.Uh + e0) = h;
-      if (g.Ul)
-        *reinterpret_cast<float4*>(g.Ul + e0) =
-            make_float4(tf32_rn(v[0] - h.x), tf32_rn(v[1] - h.y), tf32_rn(v[2] - h.z), tf32_rn(v[3] - h.w));
-    }
-    if (g.Vh) {
-      const float4 m = *reinterpret_cast<const float4*>(g.mu + c0);
-      const float w0 = v[0] * m.x, w1 = v[1] * m.y, w2 = v[2] * m.z, w3 = v[3] * m.w;
-      const float4 h = make_float4(tf32_rn(w0), tf32_rn(w1), tf32_rn(w2), tf32_rn(w3));
-      *reinterpret_cast<float4*>(g.Vh + e0) = h;
-      if (g.Vl)
-        *reinterpret_cast<float4*>(g.Vl + e0) =
-            make_float4(tf32_rn(w0 - h.x), tf32_rn(w1 - h.y), tf32_rn(w2 - h.z), tf32_rn(w3 - h.w));
-    }
-    return;
   }
+  __syncthreads();                                          // the level table
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int c = c0 + k;
-    if (c >= d) break;
-    const int64_t e = e0 + k;
-    float x;
-    if (g.identity) {
-      x = (r == c) ? 1.0f : 0.0f;
-    } else {
-      const uint32_t byte = g.codes[e >> 1];
-      x = level[(e & 1) ? (byte >> 4) : (byte & 15u)] * g.scales[e / kQuantBlock];
+  for (int q = 0; q < kBasisGroups; ++q) {
+    const int64_t e0 = base + (int64_t(q) * 256 + threadIdx.x) * 8;
+    if (e0 >= n) continue;
+    const int r = int(e0 / d), c0 = int(e0 - int64_t(r) * d);
+    if (vec) {
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        v[k] = g.identity ? ((r == c0 + k) ? 1.0f : 0.0f) : level[(packed[q] >> (4 * k)) & 15u] * sc[q];
+      basis_put8(g, e0, c0, v);
+      continue;
     }
-    if (g.U) g.U[e] = x;
-    put_split(x, g.Uh, g.Ul, e);
-    if (g.Vh) put_split(x * g.mu[c], g.Vh, g.Vl, e);
+    for (int k = 0; k < 8 && e0 + k < n; ++k) {            // d not a multiple of 8
+      const int64_t e = e0 + k;
+      const int rr = int(e / d), c = int(e - int64_t(rr) * d);
+      float x;
+      if (g.identity) {
+        x = (rr == c) ? 1.0f : 0.0f;
+      } else {
+        const uint32_t byte = g.codes[e >> 1];
+        x = level[(e & 1) ? (byte >> 4) : (byte & 15u)] * g.scales[e / kQuantBlock];
+      }
+      if (g.U) g.U[e] = x;
+      put_split(x, g.Uh, g.Ul, e);
+      if (g.Vh) put_split(x * g.mu[c], g.Vh, g.Vl, e);
+    }
   }
 }
 
 shampoo4_status launch_basis(const BasisDesc* d_desc, int count, int64_t max_elems, cudaStream_t st) {
   if (count <= 0 || max_elems <= 0) return SHAMPOO4_OK;
-  int64_t max_d = 1;
-  while (max_d * max_d < max_elems) ++max_d;               // extent is the largest d * d
-  if (max_d > 1024) return SHAMPOO4_ERR_INVALID_ARG;
+  const int64_t ctas = (max_elems + kBasisEltsPerCta - 1) / kBasisEltsPerCta;
+  if (ctas > 0x7fffffffLL) return SHAMPOO4_ERR_INVALID_ARG;
   for (int base = 0; base < count; base += 65535) {
     int c = count - base < 65535 ? count - base : 65535;
-    k_basis<<<dim3(unsigned(max_d), c), 256, 0, st>>>(d_desc + base);
+    k_basis<<<dim3(unsigned(ctas), c), 256, 0, st>>>(d_desc + base);
     S4_CUDA(cudaGetLastError());
   }
   return SHAMPOO4_OK;
