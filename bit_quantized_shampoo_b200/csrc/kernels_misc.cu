@@ -217,22 +217,38 @@ shampoo4_status launch_basis(const BasisDesc* d_desc, int count, int64_t max_ele
 }
 
 // ---- lambda_i = max(q_i . (S q)_i, 0) -----------------------------------
+// One CTA per strip of 32 columns: warp w sums rows w, w + 8, ... of its
+// lane's column in fp64 (coalesced 128-byte rows of Q and T), and the
+// eight partial sums are added in warp order, so the result does not
+// depend on scheduling.
 __global__ void __launch_bounds__(256) k_rayleigh(const RayleighDesc* __restrict__ descs) {
   const RayleighDesc& g = descs[blockIdx.y];
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= g.d) return;
+  const int c0 = blockIdx.x * 32;
+  if (c0 >= g.d) return;                                   // CTA-uniform
   if (g.skip && *g.skip) return;
+  __shared__ double part[8][32];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, i = c0 + lane;
   double acc = 0.0;
-  for (int r = 0; r < g.d; ++r)
-    acc += double(g.Q[int64_t(r) * g.d + i]) * double(g.T[int64_t(r) * g.d + i]);
-  g.lam[i] = float(acc > 0.0 ? acc : 0.0);
+  if (i < g.d) {
+#pragma unroll 4
+    for (int r = w; r < g.d; r += 8)
+      acc = fma(double(g.Q[int64_t(r) * g.d + i]), double(g.T[int64_t(r) * g.d + i]), acc);
+  }
+  part[w][lane] = acc;
+  __syncthreads();
+  if (w == 0 && i < g.d) {
+    double s = 0.0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) s += part[k][lane];
+    g.lam[i] = float(s > 0.0 ? s : 0.0);
+  }
 }
 
 shampoo4_status launch_rayleigh(const RayleighDesc* d_desc, int count, int max_d, cudaStream_t st) {
   if (count <= 0 || max_d <= 0) return SHAMPOO4_OK;
   for (int base = 0; base < count; base += 65535) {
     int c = count - base < 65535 ? count - base : 65535;
-    k_rayleigh<<<dim3((max_d + 255) / 256, c), 256, 0, st>>>(d_desc + base);
+    k_rayleigh<<<dim3((max_d + 31) / 32, c), 256, 0, st>>>(d_desc + base);
     S4_CUDA(cudaGetLastError());
   }
   return SHAMPOO4_OK;
@@ -302,12 +318,14 @@ k_scan(const ScanDesc* __restrict__ descs, const PtrEntry* __restrict__ tabs, in
   if (vec) {
     // 16-byte pieces over the whole matrix, four independent pieces in
     // flight per thread
+    // rows x cols / 4 pieces fit in 32 bits (a tile is at most 1024 x 1024,
+    // a statistic 1024 x 1024): 32-bit index arithmetic
     const int c4n = g.cols >> 2;
-    const int64_t n4 = int64_t(g.rows) * c4n;
-    const int64_t step = int64_t(gridDim.x) * blockDim.x;
+    const int n4 = g.rows * c4n;
+    const int step = int(gridDim.x) * int(blockDim.x);
 #pragma unroll 4
-    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n4; e += step) {
-      const int r = int(e / c4n), c = int(e - int64_t(r) * c4n) * 4;
+    for (int e = int(blockIdx.x) * int(blockDim.x) + int(threadIdx.x); e < n4; e += step) {
+      const int r = e / c4n, c = (e - r * c4n) * 4;
       const float4 v = *reinterpret_cast<const float4*>(X + int64_t(r) * ld + c);
       bad |= !isfinite(v.x) || !isfinite(v.y) || !isfinite(v.z) || !isfinite(v.w);
       if (g.oh) {
