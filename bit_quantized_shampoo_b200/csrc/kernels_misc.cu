@@ -543,43 +543,32 @@ __global__ void __launch_bounds__(256) k_shift_f(const ShiftDescF* __restrict__ 
 }
 
 // ---- exact Gram diagonal ------------------------------------------------------
-// One CTA per strip of 32 columns: warp w sums the squares of rows w,
-// w + 8, ... of its lane's column in fp64 (coalesced 128-byte rows), and the
-// eight partial sums are added pairwise in a fixed order.
 __global__ void __launch_bounds__(256) k_diag(const DiagDesc* __restrict__ descs, const uint32_t* __restrict__ guard) {
   if (guard && *guard == 0u) return;
   const DiagDesc& g = descs[blockIdx.y];
-  const int c0 = blockIdx.x * 32;
-  if (c0 >= g.d) return;                                   // CTA-uniform
   if (g.skip && *g.skip) return;
-  __shared__ double part[8][32];
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, i = c0 + lane;
-  double acc = 0.0;
-  if (i < g.d) {
-    const float* x = g.X + i;
-#pragma unroll 4
-    for (int k = w; k < g.d; k += 8) {
-      const double a = x[int64_t(k) * g.d];
-      acc = fma(a, a, acc);
-    }
-  }
-  part[w][lane] = acc;
-  __syncthreads();
-  if (w != 0) return;                                      // warp-uniform
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
   unsigned long long t = 0;
   if (i < g.d) {
-    const double s = ((part[0][lane] + part[1][lane]) + (part[2][lane] + part[3][lane])) +
-                     ((part[4][lane] + part[5][lane]) + (part[6][lane] + part[7][lane]));
-    const float wv = float(s);
-    g.W[int64_t(i) * g.ldw + i] = wv;
+    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+    const float* x = g.X + i;
+    int k = 0;
+    for (; k + 4 <= g.d; k += 4) {
+      const double a = x[int64_t(k) * g.d], b = x[int64_t(k + 1) * g.d];
+      const double c = x[int64_t(k + 2) * g.d], e = x[int64_t(k + 3) * g.d];
+      s0 = fma(a, a, s0); s1 = fma(b, b, s1); s2 = fma(c, c, s2); s3 = fma(e, e, s3);
+    }
+    for (; k < g.d; ++k) { const double a = x[int64_t(k) * g.d]; s0 = fma(a, a, s0); }
+    const float w = float((s0 + s1) + (s2 + s3));
+    g.W[int64_t(i) * g.ldw + i] = w;
     if (g.devsq) {
-      const float q = (wv - 1.0f) * (wv - 1.0f);
+      const float q = (w - 1.0f) * (w - 1.0f);
       t = static_cast<unsigned long long>(fminf(q, kDevFineClamp) * kDevFineUnit);
     }
   }
   if (g.devsq) {
     for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    if (lane == 0 && t) atomicAdd(g.devsq, t);
+    if ((threadIdx.x & 31) == 0 && t) atomicAdd(g.devsq, t);
   }
 }
 
@@ -587,7 +576,7 @@ shampoo4_status launch_diag(const DiagDesc* d_desc, int count, int max_d, cudaSt
   if (count <= 0 || max_d <= 0) return SHAMPOO4_OK;
   for (int base = 0; base < count; base += 65535) {
     const int c = count - base < 65535 ? count - base : 65535;
-    k_diag<<<dim3(unsigned((max_d + 31) / 32), unsigned(c)), 256, 0, st>>>(d_desc + base, guard);
+    k_diag<<<dim3(unsigned((max_d + 255) / 256), unsigned(c)), 256, 0, st>>>(d_desc + base, guard);
     S4_CUDA(cudaGetLastError());
   }
   return SHAMPOO4_OK;
