@@ -633,12 +633,26 @@ __global__ void __launch_bounds__(256) k_inv128(const Inv128Desc* __restrict__ d
   const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
   const int n1 = min(64, g.d - g.j), n2 = max(0, min(64, g.d - g.j - 64));
   auto out = [&](int r, int c, double v) { put_split(float(v), g.jh, g.jl, int64_t(g.j + r) * 128 + c); };
-  for (int r = t >> 6; r < 64; r += 4) {
-    const int c = t & 63;
-    const int64_t a = int64_t(g.j + r) * 64 + c;
-    Xi[r][c] = double(g.ih[a]) + double(g.il[a]);
-    const int64_t o = int64_t(g.j + 64 + r) * g.d + g.j + c;
-    Cm[r][c] = (r < n2 && c < n1) ? double(g.oh[o]) + double(g.ol[o]) : 0.0;
+  {
+    // every load in flight before the stores (16 rows per thread)
+    float xh[16], xl[16], ch[16], cl[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int r = (t >> 6) + 4 * q, c = t & 63;
+      const int64_t a = int64_t(g.j + r) * 64 + c;
+      xh[q] = g.ih[a];
+      xl[q] = g.il[a];
+      const bool in = r < n2 && c < n1;
+      const int64_t o = int64_t(g.j + 64 + r) * g.d + g.j + c;
+      ch[q] = in ? g.oh[o] : 0.0f;
+      cl[q] = in ? g.ol[o] : 0.0f;
+    }
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int r = (t >> 6) + 4 * q, c = t & 63;
+      Xi[r][c] = double(xh[q]) + double(xl[q]);
+      Cm[r][c] = double(ch[q]) + double(cl[q]);
+    }
   }
   __syncthreads();
   // T = C A^-1 (thread (ty, tx): rows ty + 16 i, columns tx + 16 k)
@@ -666,10 +680,17 @@ __global__ void __launch_bounds__(256) k_inv128(const Inv128Desc* __restrict__ d
     out(r, c, (c < 64 && r < n1 && c < n1) ? Xi[r][c] : 0.0);
   }
   __syncthreads();
-  for (int r = t >> 6; r < 64; r += 4) {
-    const int c = t & 63;
-    const int64_t b = int64_t(g.j + 64 + r) * 64 + c;
-    Xi[r][c] = n2 > 0 ? double(g.ih[b]) + double(g.il[b]) : 0.0;
+  {
+    float bh[16], bl[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int r = (t >> 6) + 4 * q, c = t & 63;
+      const int64_t b = int64_t(g.j + 64 + r) * 64 + c;
+      bh[q] = n2 > 0 ? g.ih[b] : 0.0f;
+      bl[q] = n2 > 0 ? g.il[b] : 0.0f;
+    }
+#pragma unroll
+    for (int q = 0; q < 16; ++q) Xi[(t >> 6) + 4 * q][t & 63] = double(bh[q]) + double(bl[q]);
   }
   __syncthreads();
   // M = -B^-1 T into Cm
