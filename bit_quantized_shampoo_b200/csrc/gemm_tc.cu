@@ -216,13 +216,16 @@ __device__ __forceinline__ bool b_transposed(const CUtensorMap* bt_hi, int k0, i
 __device__ __forceinline__ bool a_transposed(const CUtensorMap* at_hi, int k0, int m0, int bn) {
   return at_hi != nullptr && (k0 / bn) * bn >= m0 + kBM;
 }
+// First K index read through the second operand pair (a2, b2), or one past
+// any K when the product has none.
+__device__ __forceinline__ int second_pair_k(const TcGemmDesc& g) { return g.a2.hi ? g.ksplit : 0x7fffffff; }
 
-__device__ __forceinline__ uint64_t operand_desc(const TcOperand& op, uint32_t base, int kk) {
+__device__ __forceinline__ uint64_t operand_desc(int mn_major, uint32_t base, int kk) {
   // K-major (128 B swizzle): rows of 128 B, 8-row groups 1024 B apart; a K
   // step of 8 is 32 B along the row.
   // MN-major (128 B swizzle, 32 B atoms): 32-wide MN groups 4096 B apart,
   // 4-row K groups 512 B apart; a K step of 8 rows is 1024 B.
-  return op.mn_major ? smem_desc(base + kk * 1024, 4096, 512, 1) : smem_desc(base + kk * 32, 16, 1024, 2);
+  return mn_major ? smem_desc(base + kk * 1024, 4096, 512, 1) : smem_desc(base + kk * 32, 16, 1024, 2);
 }
 
 // Output fields of one problem, held in registers by the epilogue warps.
@@ -561,6 +564,8 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
       const CUtensorMap* at_hi = g.at_hi;
       TcOperand gat = ga;                                   // transposed reads of A
       gat.hi = at_hi; gat.lo = g.at_lo; gat.mn_major = 1;
+      const int ks = second_pair_k(g);
+      const TcOperand ga2 = g.a2, gb2 = g.b2;
       int issued = 0;
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % Cfg::kStages;
@@ -573,14 +578,16 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
         const uint32_t st = smem_u32(smem + s * Cfg::kStage);
         mbar_expect_tx(&full_bar[s], Cfg::kStage);
         const int k0 = kb * kBK;
-        const bool tr = b_transposed(bt_hi, k0, n0, BN);
-        const TcOperand& ob = tr ? gt : gb;
-        const TcOperand& oa = a_transposed(at_hi, k0, m0, BN) ? gat : ga;
-        load_operand(oa.hi, oa, kBM, m0, k0, st, &full_bar[s]);
-        load_operand(ob.hi, ob, BN, n0, k0, st + Cfg::kATile, &full_bar[s]);
+        const bool sec = k0 >= ks;
+        const int kc = sec ? k0 - ks : k0;
+        TcOperand oa = a_transposed(at_hi, k0, m0, BN) ? gat : ga;   // by value: stays in registers
+        TcOperand ob = b_transposed(bt_hi, k0, n0, BN) ? gt : gb;
+        if (sec) { oa = ga2; ob = gb2; }
+        load_operand(oa.hi, oa, kBM, m0, kc, st, &full_bar[s]);
+        load_operand(ob.hi, ob, BN, n0, kc, st + Cfg::kATile, &full_bar[s]);
         if (SPLIT) {
-          load_operand(oa.lo, oa, kBM, m0, k0, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
-          load_operand(ob.lo, ob, BN, n0, k0, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+          load_operand(oa.lo, oa, kBM, m0, kc, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+          load_operand(ob.lo, ob, BN, n0, kc, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
         }
         issued = kb + 1;
       }
@@ -594,12 +601,12 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
     }
   } else if (warp == 1) {
     if (lane == 0) {                                        // ---- MMA issuer
-      const TcOperand ga = g.a, gb = g.b;                   // registers, as in the producer
+      // register copies, as in the producer; the MMA needs only each K
+      // block's operand layouts
       const CUtensorMap* bt_hi = g.bt_hi;
       const CUtensorMap* at_hi = g.at_hi;
-      TcOperand gt = gb, gat = ga;
-      gt.mn_major = 1;
-      gat.mn_major = 1;
+      const int ks = second_pair_k(g);
+      const TcOperand ga = g.a, gb = g.b, ga2 = g.a2, gb2 = g.b2;
       for (int kb = 0; kb < kblocks; ++kb) {
         const int s = kb % Cfg::kStages;
         if (!mbar_wait(&full_bar[s], (kb / Cfg::kStages) & 1, wait_ns)) {
@@ -612,18 +619,19 @@ k_gemm_tc(const TcGemmDesc* __restrict__ descs, const PtrEntry* __restrict__ tab
         const uint32_t st = smem_u32(smem + s * Cfg::kStage);
         const uint32_t a_hi = st, b_hi = st + Cfg::kATile;
         const uint32_t a_lo = st + Cfg::kATile + Cfg::kBTile, b_lo = a_lo + Cfg::kATile;
-        const TcOperand& ob = b_transposed(bt_hi, kb * kBK, n0, BN) ? gt : gb;
-        const TcOperand& oa = a_transposed(at_hi, kb * kBK, m0, BN) ? gat : ga;
-        const uint32_t idesc = idesc_tf32(kBM, BN, oa.mn_major, ob.mn_major);
+        const bool sec = kb * kBK >= ks;
+        const int amn = sec ? ga2.mn_major : (a_transposed(at_hi, kb * kBK, m0, BN) ? 1 : ga.mn_major);
+        const int bmn = sec ? gb2.mn_major : (b_transposed(bt_hi, kb * kBK, n0, BN) ? 1 : gb.mn_major);
+        const uint32_t idesc = idesc_tf32(kBM, BN, amn, bmn);
 #pragma unroll
         for (int kk = 0; kk < kBK / 8; ++kk) {
           // first MMA into accumulator kb mod kAcc overwrites it
           const uint32_t acc = (kb >= Cfg::kAcc || kk != 0) ? 1u : 0u;
           const uint32_t dt = tmem + uint32_t((kb % Cfg::kAcc) * BN);
-          mma_tf32(dt, operand_desc(oa, a_hi, kk), operand_desc(ob, b_hi, kk), idesc, acc);
+          mma_tf32(dt, operand_desc(amn, a_hi, kk), operand_desc(bmn, b_hi, kk), idesc, acc);
           if (SPLIT) {
-            mma_tf32(dt, operand_desc(oa, a_hi, kk), operand_desc(ob, b_lo, kk), idesc, 1);
-            mma_tf32(dt, operand_desc(oa, a_lo, kk), operand_desc(ob, b_hi, kk), idesc, 1);
+            mma_tf32(dt, operand_desc(amn, a_hi, kk), operand_desc(bmn, b_lo, kk), idesc, 1);
+            mma_tf32(dt, operand_desc(amn, a_lo, kk), operand_desc(bmn, b_hi, kk), idesc, 1);
           }
         }
         mma_commit(&empty_bar[s]);                          // stage free once these MMAs finish
@@ -685,9 +693,20 @@ __host__ __device__ __forceinline__ int tiles_in_row(int symmetric, int N, int b
 // Running tile t of the batch (tc_assign_tiles numbered them): problem p
 // (a cursor that only moves forward, as t does), tile origin (m0, n0);
 // false when the problem is skipped.  Every role walks the same tiles.
+// With the batch's tile list the lookup is one load; without it the cursor
+// walks the problems, one dependent load per problem passed, which on a
+// batch of many small problems costs microseconds per tile.
 template <int BN>
-__device__ __forceinline__ bool pers_tile(const TcGemmDesc* __restrict__ descs, int count, int64_t t, int& p,
-                                          int& m0, int& n0) {
+__device__ __forceinline__ bool pers_tile(const TcGemmDesc* __restrict__ descs, int count,
+                                          const uint64_t* __restrict__ list, int64_t t, int& p, int& m0, int& n0) {
+  if (list) {
+    const uint64_t e = list[t];
+    p = int(uint32_t(e));
+    m0 = int((e >> 32) & 0xffffu) * kBM;
+    n0 = int(e >> 48) * BN;
+    const uint32_t* skip = descs[p].skip;
+    return !(skip && *skip);
+  }
   while (p + 1 < count && descs[p + 1].tile_begin <= t) ++p;
   const TcGemmDesc& g = descs[p];
   int x = int(t - g.tile_begin);
@@ -855,7 +874,8 @@ __device__ __forceinline__ void epilogue_regs(const TcGemmDesc& g, const PtrEntr
 template <int BN, bool SPLIT, int STAGES>
 __global__ void __launch_bounds__(192, 1)
 k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, const PtrEntry* __restrict__ tabs,
-               int nparams, uint32_t* __restrict__ gflags, uint64_t wait_ns, const uint32_t* __restrict__ guard) {
+               int nparams, uint32_t* __restrict__ gflags, uint64_t wait_ns, const uint32_t* __restrict__ guard,
+               const uint64_t* __restrict__ tile_list) {
   using Cfg = TcCfg<BN, SPLIT, STAGES>;
   if (guard && *guard == 0u) return;                      // no problem of the launch runs
   using PCfg = PersCfg<BN, SPLIT, STAGES>;
@@ -895,7 +915,7 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
       int last_p = -1;
       for (int64_t t = blockIdx.x; t < total && !*(volatile int*)&abort_flag; t += gridDim.x) {
         int m0, n0;
-        if (!pers_tile<BN>(descs, count, t, p, m0, n0)) continue;
+        if (!pers_tile<BN>(descs, count, tile_list, t, p, m0, n0)) continue;
         const TcOperand ga = descs[p].a, gb = descs[p].b;   // registers (see k_gemm_tc)
         const CUtensorMap* bt_hi = descs[p].bt_hi;
         TcOperand gt = gb;                                  // transposed reads of B
@@ -903,6 +923,8 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
         const CUtensorMap* at_hi = descs[p].at_hi;
         TcOperand gat = ga;                                 // transposed reads of A
         gat.hi = at_hi; gat.lo = descs[p].at_lo; gat.mn_major = 1;
+        const int ks = second_pair_k(descs[p]);
+        const TcOperand ga2 = descs[p].a2, gb2 = descs[p].b2;
         const int kblocks = (descs[p].K + kBK - 1) / kBK;
         if (p != last_p) {
           asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(ga.hi)) : "memory");
@@ -924,14 +946,16 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
           const uint32_t st = smem_u32(smem + s * Cfg::kStage);
           mbar_expect_tx(&full_bar[s], Cfg::kStage);
           const int k0 = kb * kBK;
-          const bool tr = b_transposed(bt_hi, k0, n0, BN);
-          const TcOperand& ob = tr ? gt : gb;
-          const TcOperand& oa = a_transposed(at_hi, k0, m0, BN) ? gat : ga;
-          load_operand(oa.hi, oa, kBM, m0, k0, st, &full_bar[s]);
-          load_operand(ob.hi, ob, BN, n0, k0, st + Cfg::kATile, &full_bar[s]);
+          const bool sec = k0 >= ks;
+          const int kc = sec ? k0 - ks : k0;
+          TcOperand oa = a_transposed(at_hi, k0, m0, BN) ? gat : ga;   // by value: stays in registers
+          TcOperand ob = b_transposed(bt_hi, k0, n0, BN) ? gt : gb;
+          if (sec) { oa = ga2; ob = gb2; }
+          load_operand(oa.hi, oa, kBM, m0, kc, st, &full_bar[s]);
+          load_operand(ob.hi, ob, BN, n0, kc, st + Cfg::kATile, &full_bar[s]);
           if (SPLIT) {
-            load_operand(oa.lo, oa, kBM, m0, k0, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
-            load_operand(ob.lo, ob, BN, n0, k0, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+            load_operand(oa.lo, oa, kBM, m0, kc, st + Cfg::kATile + Cfg::kBTile, &full_bar[s]);
+            load_operand(ob.lo, ob, BN, n0, kc, st + 2 * Cfg::kATile + Cfg::kBTile, &full_bar[s]);
           }
         }
       }
@@ -945,13 +969,11 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
       uint32_t it = 0, ntiles = 0;
       for (int64_t t = blockIdx.x; t < total && !*(volatile int*)&abort_flag; t += gridDim.x) {
         int m0, n0;
-        if (!pers_tile<BN>(descs, count, t, p, m0, n0)) continue;
-        const TcOperand ga = descs[p].a, gb = descs[p].b;
+        if (!pers_tile<BN>(descs, count, tile_list, t, p, m0, n0)) continue;
         const CUtensorMap* bt_hi = descs[p].bt_hi;
         const CUtensorMap* at_hi = descs[p].at_hi;
-        TcOperand gt = gb, gat = ga;
-        gt.mn_major = 1;
-        gat.mn_major = 1;
+        const int ks = second_pair_k(descs[p]);
+        const TcOperand ga = descs[p].a, gb = descs[p].b, ga2 = descs[p].a2, gb2 = descs[p].b2;
         const int kblocks = (descs[p].K + kBK - 1) / kBK;
         // the epilogue has read the previous tile's accumulators
         if (ntiles > 0 && !mbar_wait(&acc_empty, (ntiles - 1) & 1, wait_ns)) {
@@ -974,17 +996,18 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
           const uint32_t st = smem_u32(smem + s * Cfg::kStage);
           const uint32_t a_hi = st, b_hi = st + Cfg::kATile;
           const uint32_t a_lo = st + Cfg::kATile + Cfg::kBTile, b_lo = a_lo + Cfg::kATile;
-          const TcOperand& ob = b_transposed(bt_hi, kb * kBK, n0, BN) ? gt : gb;
-          const TcOperand& oa = a_transposed(at_hi, kb * kBK, m0, BN) ? gat : ga;
-          const uint32_t idesc = idesc_tf32(kBM, BN, oa.mn_major, ob.mn_major);
+          const bool sec = kb * kBK >= ks;
+          const int amn = sec ? ga2.mn_major : (a_transposed(at_hi, kb * kBK, m0, BN) ? 1 : ga.mn_major);
+          const int bmn = sec ? gb2.mn_major : (b_transposed(bt_hi, kb * kBK, n0, BN) ? 1 : gb.mn_major);
+          const uint32_t idesc = idesc_tf32(kBM, BN, amn, bmn);
 #pragma unroll
           for (int kk = 0; kk < kBK / 8; ++kk) {
             const uint32_t acc = (kb >= Cfg::kAcc || kk != 0) ? 1u : 0u;
             const uint32_t dt = tmem + uint32_t((kb % Cfg::kAcc) * BN);
-            mma_tf32(dt, operand_desc(oa, a_hi, kk), operand_desc(ob, b_hi, kk), idesc, acc);
+            mma_tf32(dt, operand_desc(amn, a_hi, kk), operand_desc(bmn, b_hi, kk), idesc, acc);
             if (SPLIT) {
-              mma_tf32(dt, operand_desc(oa, a_hi, kk), operand_desc(ob, b_lo, kk), idesc, 1);
-              mma_tf32(dt, operand_desc(oa, a_lo, kk), operand_desc(ob, b_hi, kk), idesc, 1);
+              mma_tf32(dt, operand_desc(amn, a_hi, kk), operand_desc(bmn, b_lo, kk), idesc, 1);
+              mma_tf32(dt, operand_desc(amn, a_lo, kk), operand_desc(bmn, b_hi, kk), idesc, 1);
             }
           }
           mma_commit(&empty_bar[s]);
@@ -1002,7 +1025,7 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
     uint32_t ntiles = 0;
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
       int m0, n0;
-      if (!pers_tile<BN>(descs, count, t, p, m0, n0)) continue;
+      if (!pers_tile<BN>(descs, count, tile_list, t, p, m0, n0)) continue;
       const bool ok = mbar_wait(&acc_full, ntiles & 1, wait_ns);
       if (!ok) atomicOr(gflags, SHAMPOO4_FLAG_TIMEOUT);
       if (!ok || *(volatile int*)&abort_flag) break;
@@ -1041,7 +1064,7 @@ k_gemm_tc_pers(const TcGemmDesc* __restrict__ descs, int count, int64_t total, c
 template <int BN, bool SPLIT, int STAGES>
 shampoo4_status launch_tc_pers(const TcGemmDesc* d_desc, int count, int64_t total, const PtrEntry* tabs,
                                int nparams, uint32_t* gflags, uint64_t wait_ns, cudaStream_t st,
-                               const uint32_t* guard) {
+                               const uint32_t* guard, const uint64_t* tile_list) {
   using PCfg = PersCfg<BN, SPLIT, STAGES>;
   static int sms = 0;
   if (!sms) {
@@ -1054,7 +1077,7 @@ shampoo4_status launch_tc_pers(const TcGemmDesc* d_desc, int count, int64_t tota
   if (total <= 0) return SHAMPOO4_OK;
   const int grid = int(total < sms ? total : sms);
   k_gemm_tc_pers<BN, SPLIT, STAGES><<<grid, 192, PCfg::kSmem, st>>>(d_desc, count, total, tabs, nparams, gflags,
-                                                                     wait_ns, guard);
+                                                                     wait_ns, guard, tile_list);
   S4_CUDA(cudaGetLastError());
   return SHAMPOO4_OK;
 }
@@ -1089,19 +1112,26 @@ int tc_persistent = 1;
 
 int tc_tiles_in_row(const TcGemmDesc& g, int bn, int tm) { return tiles_in_row(g.symmetric, g.N, bn, tm); }
 
-int64_t tc_assign_tiles(TcGemmDesc* v, int count, int bn) {
+int64_t tc_assign_tiles(TcGemmDesc* v, int count, int bn, std::vector<uint64_t>* list) {
   int64_t total = 0;
   for (int i = 0; i < count; ++i) {
     v[i].tile_begin = int32_t(total);
     const int tiles_m = (v[i].M + kBM - 1) / kBM;
-    for (int tm = 0; tm < tiles_m; ++tm) total += tiles_in_row(v[i].symmetric, v[i].N, bn, tm);
+    for (int tm = 0; tm < tiles_m; ++tm) {
+      const int c = tiles_in_row(v[i].symmetric, v[i].N, bn, tm);
+      if (list)
+        for (int tn = 0; tn < c; ++tn)
+          list->push_back(uint64_t(uint32_t(i)) | (uint64_t(uint32_t(tm)) << 32) | (uint64_t(uint32_t(tn)) << 48));
+      total += c;
+    }
   }
   return total;
 }
 
 shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split, int bn,
                                const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st,
-                               uint64_t wait_ns, int64_t total_tiles, const uint32_t* guard) {
+                               uint64_t wait_ns, int64_t total_tiles, const uint32_t* guard,
+                               const uint64_t* tile_list) {
   if (count <= 0 || max_tiles <= 0) return SHAMPOO4_OK;
   if (wait_ns == 0 || wait_ns > kWaitNs) wait_ns = kWaitNs;
   // TF32: one tile per CTA, two 2-stage CTAs per SM, so one tile's
@@ -1124,7 +1154,8 @@ shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tile
   if (bn == 64)
     return launch_tc_impl<64, true, 2>(d_desc, count, max_tiles, tabs, nparams, gflags, wait_ns, st, guard);
   if (pers && tc_persistent)
-    return launch_tc_pers<128, true, 3>(d_desc, count, total_tiles, tabs, nparams, gflags, wait_ns, st, guard);
+    return launch_tc_pers<128, true, 3>(d_desc, count, total_tiles, tabs, nparams, gflags, wait_ns, st, guard,
+                                        tile_list);
   return launch_tc_impl<128, true, 3>(d_desc, count, max_tiles, tabs, nparams, gflags, wait_ns, st, guard);
 }
 

@@ -41,6 +41,7 @@ struct Launch {
   double flops = 0, bytes = 0;   // algorithmic work of the launch
   size_t guard_off = SIZE_MAX;   // workspace word gating the whole launch (fp64 QR passes)
   int64_t tiles = -1;            // tensor-core products: the batch's running tiles
+  size_t list_off = SIZE_MAX;    // persistent products: byte offset of the tile list
   // Pack launches carry host-side tensor lists instead of descriptors.
   std::vector<const float*> px;
   std::vector<int64_t> pn;
@@ -91,7 +92,6 @@ struct FactorPlan {
   size_t ws_Zm, ws_Zh, ws_Zl;
   size_t ws_Ih, ws_Il;                   // 64 x 64 inverse diagonal blocks of L (rows to a multiple of 64)
   size_t ws_Jh, ws_Jl;                   // 128 x 128 inverse diagonal blocks (rows to a multiple of 128)
-  size_t ws_Ph, ws_Pl;                   // d x 128: solve panel temporary
   size_t ws_q_first, ws_q_next;
   size_t dbg_u, dbg_q;                   // debug capture: offsets of the rectified U and of Q
 };
@@ -382,8 +382,6 @@ shampoo4_status plan(shampoo4_ctx* h) {
       const size_t dpad2 = align_up(size_t(f.d), kSolveW);
       f.ws_Jh = take(cur, 4 * dpad2 * kSolveW);
       f.ws_Jl = take(cur, 4 * dpad2 * kSolveW);
-      f.ws_Ph = take(cur, 4 * size_t(f.d) * kSolveW);
-      f.ws_Pl = take(cur, 4 * size_t(f.d) * kSolveW);
       f.ws_W64 = take(cur, 8 * dd);            // fp64 fallback of the QR
       f.ws_Q64 = take(cur, 8 * dd);
     } else {
@@ -604,9 +602,14 @@ void emit_gemmtc(Builder& b, std::vector<Launch>& prog, const std::vector<TcGemm
   }
   if (v.empty()) return;
   std::vector<TcGemmDesc> w = v;
-  const int64_t total = tc_assign_tiles(w.data(), int(w.size()), bn);
+  // the 128-wide split instance runs persistent CTAs, which look their
+  // tiles up in the list
+  const bool pers = split && bn == 128;
+  std::vector<uint64_t> list;
+  const int64_t total = tc_assign_tiles(w.data(), int(w.size()), bn, pers ? &list : nullptr);
   b.emit(prog, !split ? Kind::GemmTC : (bn == 64 ? Kind::GemmTCSplit64 : Kind::GemmTCSplit), w, mt, fl);
   prog.back().tiles = total;
+  if (pers && !list.empty()) prog.back().list_off = b.put(list);
 }
 
 int mode_of(const shampoo4_config& c) { return c.precision == SHAMPOO4_PREC_FP32 ? kModeFP32 : kModeTF32; }
@@ -1087,58 +1090,69 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
     b.tag = SHAMPOO4_STAGE_QR_TRSM_PANEL;
     emit_gemmtc(b, prog, l21, true, 64);
   }
-  // Solve Q L^T = X by 128-wide column panels, through the 128 x 128
-  // inverse diagonal blocks assembled from the 64 x 64 ones (k_inv128):
-  //   T = X[:, J] - Q[:, <J] L[J, <J]^T      tensor cores, TF32 split into P
-  //   Q[:, J] = T L[J, J]^-T                  tensor cores
-  // 128-wide products keep the MMA at its 128-column rate (a 64-column
-  // instruction pays about the same issue time for half the work), and the
-  // solve takes half as many steps.
+  // Solve Q L^T = X by 128-wide column panels J, one product each:
+  //   Q[:, J] = (X[:, J] - Q[:, <J] L[J, <J]^T) L[J, J]^-T
+  //           = Q[:, <J] H[J, <J]^T + X[:, J] L[J, J]^-T,
+  // with H[J, <J] = -L[J, J]^-1 L[J, <J].  The 128 x 128 inverse diagonal
+  // blocks are assembled from the 64 x 64 ones (k_inv128); the block rows
+  // of H are one batched product written over L's split (each output tile
+  // reads exactly the L tile it replaces, and nothing later reads L).  The
+  // panel product takes K blocks below j from Q and H, and the last one
+  // from X and L[J, J]^-1 (the second operand pair): no intermediate panel
+  // goes through memory, and the 128-wide MMA runs at its full rate.
   {
     std::vector<Inv128Desc> iv;
+    std::vector<TcGemmDesc> hv;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
       if (!f.tc) continue;
-      for (int j = 0; j < f.d; j += kSolveW)
+      const int d = f.d, dp = int(align_up(size_t(d), kSolveW));
+      for (int j = 0; j < d; j += kSolveW) {
         iv.push_back({b.wf(f.ws_Ih), b.wf(f.ws_Il), b.wf(f.ws_Th), b.wf(f.ws_Tl), b.wf(f.ws_Jh), b.wf(f.ws_Jl),
-                      f.d, j, skip_of(i)});
+                      d, j, skip_of(i)});
+        if (j == 0) continue;
+        const int jb = std::min(kSolveW, d - j);
+        TcGemmDesc g = gemmtc(jb, j, jb, -1.0f, 0.0f);               // H[J, <J]
+        g.a = b.operand(b.wf(f.ws_Jh), b.wf(f.ws_Jl), dp, kSolveW, true, false, true);
+        g.a.row0 = j;
+        g.b = b.operand(b.wf(f.ws_Th), b.wf(f.ws_Tl), d, d, false, false, true);
+        g.b.row0 = j;
+        g.Chi = b.wf(f.ws_Th) + int64_t(j) * d; g.Clo = b.wf(f.ws_Tl) + int64_t(j) * d; g.ldh = d;
+        g.skip = skip_of(i);
+        hv.push_back(g);
+      }
     }
     b.tag = SHAMPOO4_STAGE_QR_INVERSE;
     b.emit(prog, Kind::Inv128, iv, 0);
+    emit_gemmtc(b, prog, hv, true, kSolveW);
   }
   for (int j = 0; j < dmax; j += kSolveW) {
-    std::vector<TcGemmDesc> up, qp;
+    std::vector<TcGemmDesc> qp;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
       if (!f.tc || j >= f.d) continue;
       const int d = f.d, jb = std::min(kSolveW, d - j);
-      TcGemmDesc q = gemmtc(d, jb, jb, 1.0f, 0.0f);
+      TcGemmDesc q = gemmtc(d, jb, j + jb, 1.0f, 0.0f);
+      TcOperand xa = b.operand(X[i].h, X[i].l, d, d, true, false, true);          // X[:, J]
+      xa.col0 = j;
+      TcOperand jinv = b.operand(b.wf(f.ws_Jh), b.wf(f.ws_Jl), int(align_up(size_t(d), kSolveW)), kSolveW, false,
+                                 true, true, kSolveW);                                 // L[J, J]^-T
+      jinv.row0 = j;
       if (j > 0) {
-        TcGemmDesc u = gemmtc(d, jb, j, -1.0f, 1.0f);
-        u.a = b.operand(Q[i].h, Q[i].l, d, d, true, false, true);
-        u.b = b.operand(b.wf(f.ws_Th), b.wf(f.ws_Tl), d, d, false, true, true, kSolveW);
-        u.b.row0 = j;
-        u.Chi = b.wf(f.ws_Ph); u.Clo = b.wf(f.ws_Pl); u.ldh = kSolveW;
-        u.Cin = X[i].m + j; u.ldcin = d;
-        u.skip = skip_of(i);
-        up.push_back(u);
-        q.a = b.operand(b.wf(f.ws_Ph), b.wf(f.ws_Pl), d, kSolveW, true, false, true);
+        q.a = b.operand(Q[i].h, Q[i].l, d, d, true, false, true);                    // Q[:, <J]
+        q.b = b.operand(b.wf(f.ws_Th), b.wf(f.ws_Tl), d, d, false, true, true, kSolveW);
+        q.b.row0 = j;                                                                 // H[J, <J]^T
+        q.a2 = xa; q.b2 = jinv; q.ksplit = j;
       } else {
-        q.a = b.operand(X[i].h, X[i].l, d, d, true, false, true);   // T = X[:, 0:jb]
+        q.a = xa; q.b = jinv;
       }
-      q.b = b.operand(b.wf(f.ws_Jh), b.wf(f.ws_Jl), int(align_up(size_t(d), kSolveW)), kSolveW, false, true, true,
-                      64);
-      q.b.row0 = j;
       q.C = Q[i].m + j; q.ldc = d;
       q.Chi = Q[i].h + j; q.Clo = Q[i].l + j; q.ldh = d;
       q.skip = skip_of(i);
       qp.push_back(q);
     }
     b.tag = SHAMPOO4_STAGE_QR_SOLVE_UPDATE;
-    emit_gemmtc(b, prog, up, true, kSolveW);
-    // the panel product is short (K <= 128): 64-wide tiles, two CTAs per SM
-    b.tag = SHAMPOO4_STAGE_QR_SOLVE_PANEL;
-    emit_gemmtc(b, prog, qp, true, 64);
+    emit_gemmtc(b, prog, qp, true, kSolveW);
   }
   if (gated) b.guard = SIZE_MAX;
 }
@@ -1907,7 +1921,10 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
       case Kind::GemmTCSplit64:
         S4_TRY(launch_gemm_tc(static_cast<const TcGemmDesc*>(d), L.count, int(L.extent),
                               L.kind == Kind::GemmTC ? 0 : 1, L.kind == Kind::GemmTCSplit64 ? 64 : 0, tabs, np,
-                              gflags, st, h->wait_ns, L.tiles, guard));
+                              gflags, st, h->wait_ns, L.tiles, guard,
+                              L.list_off == SIZE_MAX ? nullptr
+                                                     : reinterpret_cast<const uint64_t*>(h->d_ws + h->ws_desc +
+                                                                                         L.list_off)));
         break;
       case Kind::PotrfF:
         S4_TRY(launch_potrf_f(static_cast<const PotrfDescF*>(d), L.count, st, guard));

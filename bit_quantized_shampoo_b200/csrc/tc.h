@@ -1,6 +1,7 @@
 // Descriptors of the tensor-core GEMM (gemm_tc.cu).
 #pragma once
 #include <cuda.h>
+#include <vector>
 #include "plan.h"
 
 namespace s4 {
@@ -63,6 +64,14 @@ struct TcGemmDesc {
   // (tiles_n = ceil(N / tile width)); every running tile writes its four
   // slots, so the sum over them, in any fixed order, is ||C||_F^2
   double* sumsq;
+  // optional second operand pair (split mode, 128-wide tiles): K blocks at
+  // or beyond ksplit (a multiple of 32) read op(A) through a2 and op(B)
+  // through b2, at K coordinate k - ksplit, so that C = [A1 A2] [B1; B2]
+  // for pieces stored apart.  Unused when a2.hi is null; when set, a and b
+  // must hold valid maps too (ksplit > 0).
+  TcOperand a2, b2;
+  int32_t ksplit;
+  int32_t pad2_;
 };
 
 // Tile width N of the kernel instance: 256 (TF32), 128 (split), or 64
@@ -73,16 +82,22 @@ int tc_block_n(int split);
 // total_tiles: the batch's number of running tiles from tc_assign_tiles on
 // the same descriptors; without it (-1) every instance runs one tile per CTA.
 // guard (optional): the whole launch is skipped when *guard == 0.
+// tile_list (optional, persistent instance): entry t names running tile t
+// of the batch, packed as problem | tile row << 32 | tile column << 48
+// (tc_assign_tiles writes it), so that a CTA finds its tile with one load
+// instead of walking the problem list.
 shampoo4_status launch_gemm_tc(const TcGemmDesc* d_desc, int count, int max_tiles, int split, int bn,
                                const PtrEntry* tabs, int nparams, uint32_t* gflags, cudaStream_t st,
-                               uint64_t wait_ns = 0, int64_t total_tiles = -1, const uint32_t* guard = nullptr);
+                               uint64_t wait_ns = 0, int64_t total_tiles = -1, const uint32_t* guard = nullptr,
+                               const uint64_t* tile_list = nullptr);
 // Tiles of one problem that run for tile width bn: all, or for a symmetric
 // product those touching the lower triangle (row block tm runs column
 // blocks tn with tn * bn < (tm + 1) * 128).
 int tc_tiles_in_row(const TcGemmDesc& g, int bn, int tm);
 // Number the running tiles of a batch: sets tile_begin of each descriptor,
-// returns the total.
-int64_t tc_assign_tiles(TcGemmDesc* v, int count, int bn);
+// returns the total; with list, also appends each running tile's packed
+// entry (problem | tile row << 32 | tile column << 48) in that order.
+int64_t tc_assign_tiles(TcGemmDesc* v, int count, int bn, std::vector<uint64_t>* list = nullptr);
 // Encode a 2-D fp32 tensor map (rows x cols, leading dimension ld elements),
 // box 32 (contiguous) x box_rows, zero fill out of bounds; 128-byte swizzle,
 // with 32-byte atoms for an operand read MN-major.
