@@ -235,7 +235,6 @@ struct EpiArgs {
   float* C; int64_t ldc;
   float* Chi; float* Clo; int64_t ldh;
   const float* Cin; int64_t ldcin;
-  unsigned long long* devsq;
   double* sumsq;
 
   __device__ __forceinline__ void load(const TcGemmDesc& g, const PtrEntry* tabs, int nparams) {
@@ -250,7 +249,6 @@ struct EpiArgs {
     }
     Chi = g.Chi; Clo = g.Clo; ldh = g.ldh;
     Cin = g.Cin; ldcin = g.ldcin;
-    devsq = g.devsq;
     sumsq = C ? g.sumsq : nullptr;
   }
   // Sum of squares of the C values of one lane's row segment (columns
@@ -351,7 +349,6 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmDesc& g, const PtrEntr
   const bool out_vec = out_bulk;                        // same alignment conditions
   const uint32_t wsm = smem_u32(wbuf);
   const uint32_t my_row = uint32_t(lane * Cfg::kPitch * 4);
-  unsigned long long dev_fine = 0;                      // deviation sum, plan.h units
   double ss_acc = 0.0;                                  // sum of squares of C (sumsq)
   // Cin chunk i into buffer i & 1 with 16-byte cp.async pieces, four
   // full 128-byte rows per warp instruction: lane l copies rows
@@ -411,16 +408,6 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmDesc& g, const PtrEntr
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             if (cb + j < e.N) v[j] = fmaf(e.beta, __ldg(src + j), v[j]);
-        }
-      }
-      if (e.devsq && row_ok) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int c = cb + j;
-          if (c >= e.N || c == row || (e.symmetric && c > row)) continue;
-          const float q = v[j] * v[j];
-          const unsigned long long w = (e.symmetric && c < row) ? 2ull : 1ull;
-          dev_fine += w * static_cast<unsigned long long>(fminf(q, kDevFineClamp) * kDevFineUnit);
         }
       }
       if (e.sumsq && row_ok) ss_acc += e.seg_sumsq(v, row, cb);
@@ -491,11 +478,6 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmDesc& g, const PtrEntr
           if (row_ok && c < e.N && c < row) e.put(int64_t(c), row, v[j]);
         }
       }
-    }
-    if (e.devsq) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) dev_fine += __shfl_xor_sync(0xffffffffu, dev_fine, o);
-      if (lane == 0 && dev_fine) atomicAdd(e.devsq, dev_fine);
     }
     cp_async_wait<0>();                                 // nothing in flight into the buffers
   }
@@ -751,7 +733,6 @@ __device__ __forceinline__ void epilogue_regs(const TcGemmDesc& g, const PtrEntr
   const uint32_t wsm = smem_u32(wbuf);
   float* stage = reinterpret_cast<float*>(wbuf);
   const int sr = lane >> 3, sc = 4 * (lane & 7);
-  unsigned long long dev_fine = 0;
 #pragma unroll
   for (int i = 0; i < kChunks; ++i) {
     if (i >= nchunks) break;
@@ -792,16 +773,6 @@ __device__ __forceinline__ void epilogue_regs(const TcGemmDesc& g, const PtrEntr
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           if (cb + j < e.N) v[i][j] = fmaf(e.beta, __ldg(src + j), v[i][j]);
-      }
-    }
-    if (e.devsq && row_ok) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int c = cb + j;
-        if (c >= e.N || c == row || (e.symmetric && c > row)) continue;
-        const float sq = v[i][j] * v[i][j];
-        const unsigned long long w = (e.symmetric && c < row) ? 2ull : 1ull;
-        dev_fine += w * static_cast<unsigned long long>(fminf(sq, kDevFineClamp) * kDevFineUnit);
       }
     }
     const bool below = !e.symmetric || cb + 31 < rbase;   // whole chunk left of every row
@@ -862,11 +833,6 @@ __device__ __forceinline__ void epilogue_regs(const TcGemmDesc& g, const PtrEntr
         if (row_ok && c < e.N && c < row) e.put(int64_t(c), row, v[i][j]);
       }
     }
-  }
-  if (e.devsq) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) dev_fine += __shfl_xor_sync(0xffffffffu, dev_fine, o);
-    if (lane == 0 && dev_fine) atomicAdd(e.devsq, dev_fine);
   }
   __syncwarp();                                         // the block is free for the next tile
 }

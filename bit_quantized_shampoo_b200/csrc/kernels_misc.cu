@@ -548,7 +548,6 @@ __global__ void __launch_bounds__(256) k_diag(const DiagDesc* __restrict__ descs
   const DiagDesc& g = descs[blockIdx.y];
   if (g.skip && *g.skip) return;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  unsigned long long t = 0;
   if (i < g.d) {
     double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
     const float* x = g.X + i;
@@ -559,16 +558,7 @@ __global__ void __launch_bounds__(256) k_diag(const DiagDesc* __restrict__ descs
       s0 = fma(a, a, s0); s1 = fma(b, b, s1); s2 = fma(c, c, s2); s3 = fma(e, e, s3);
     }
     for (; k < g.d; ++k) { const double a = x[int64_t(k) * g.d]; s0 = fma(a, a, s0); }
-    const float w = float((s0 + s1) + (s2 + s3));
-    g.W[int64_t(i) * g.ldw + i] = w;
-    if (g.devsq) {
-      const float q = (w - 1.0f) * (w - 1.0f);
-      t = static_cast<unsigned long long>(fminf(q, kDevFineClamp) * kDevFineUnit);
-    }
-  }
-  if (g.devsq) {
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    if ((threadIdx.x & 31) == 0 && t) atomicAdd(g.devsq, t);
+    g.W[int64_t(i) * g.ldw + i] = float((s0 + s1) + (s2 + s3));
   }
 }
 
@@ -731,6 +721,109 @@ shampoo4_status launch_inv128(const Inv128Desc* d_desc, int count, cudaStream_t 
   }
   k_inv128<<<count, 256, kInvSmem, st>>>(d_desc, guard);
   S4_CUDA(cudaGetLastError());
+  return SHAMPOO4_OK;
+}
+
+// ---- orthogonality sketch ------------------------------------------------------
+// Sign bits of columns 16 m .. 16 m + 15: the lowbias32 integer mixer
+// (C. Wellons, "Prospecting for Hash Functions", 2018) of m.
+__device__ __forceinline__ uint32_t sketch_signs(uint32_t m) {
+  uint32_t x = m + 0x9e3779b9u;
+  x ^= x >> 16;
+  x *= 0x7feb352du;
+  x ^= x >> 15;
+  x *= 0x846ca68bu;
+  x ^= x >> 16;
+  return x;
+}
+
+__device__ __forceinline__ double signed_by(float v, uint32_t bit) {
+  return double(__uint_as_float(__float_as_uint(v) ^ (bit << 31)));
+}
+
+// Pass one: row r of Z = Q Omega, z_j = sum over columns c = j (mod 16) of
+// +-Q[r][c] (exact fp32 values, fp64 sums).
+__global__ void __launch_bounds__(128) k_sketch_z(const SketchDesc* __restrict__ descs) {
+  const SketchDesc& g = descs[blockIdx.y];
+  const int d = g.d;
+  const int r = blockIdx.x * 128 + threadIdx.x;
+  if (r >= d || (g.skip && *g.skip)) return;
+  const float* q = g.Q + int64_t(r) * d;
+  double z[kSketchCols];
+#pragma unroll
+  for (int j = 0; j < kSketchCols; ++j) z[j] = 0.0;
+  for (int c0 = 0; c0 < d; c0 += 16) {
+    const uint32_t s = sketch_signs(uint32_t(c0 >> 4));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (c0 + 4 * u < d) {                                 // d % 4 == 0
+        const float4 v = *reinterpret_cast<const float4*>(q + c0 + 4 * u);
+        z[4 * u + 0] += signed_by(v.x, (s >> (4 * u + 0)) & 1u);
+        z[4 * u + 1] += signed_by(v.y, (s >> (4 * u + 1)) & 1u);
+        z[4 * u + 2] += signed_by(v.z, (s >> (4 * u + 2)) & 1u);
+        z[4 * u + 3] += signed_by(v.w, (s >> (4 * u + 3)) & 1u);
+      }
+    }
+  }
+  double* zr = g.Z + int64_t(r) * kSketchCols;
+#pragma unroll
+  for (int j = 0; j < kSketchCols; ++j) zr[j] = z[j];
+}
+
+// Pass two: column c of Q^T Z - Omega, its squares clamped and summed as
+// integers (order-independent), one atomic per warp.
+__global__ void __launch_bounds__(128) k_sketch_r(const SketchDesc* __restrict__ descs) {
+  const SketchDesc& g = descs[blockIdx.y];
+  const int d = g.d;
+  if (int(blockIdx.x) * 128 >= d || (g.skip && *g.skip)) return;   // CTA-uniform
+  __shared__ double zs[32][kSketchCols];
+  const int c = blockIdx.x * 128 + threadIdx.x;
+  const bool ok = c < d;
+  double y[kSketchCols];
+#pragma unroll
+  for (int j = 0; j < kSketchCols; ++j) y[j] = 0.0;
+  for (int r0 = 0; r0 < d; r0 += 32) {
+    const int nr = min(32, d - r0);
+    __syncthreads();                                        // previous rows consumed
+    for (int e = threadIdx.x; e < nr * kSketchCols; e += 128)
+      zs[e / kSketchCols][e % kSketchCols] = g.Z[int64_t(r0) * kSketchCols + e];
+    __syncthreads();
+    if (ok) {
+      const float* qc = g.Q + int64_t(r0) * d + c;
+#pragma unroll 4
+      for (int rr = 0; rr < nr; ++rr) {
+        const double qv = double(qc[int64_t(rr) * d]);
+#pragma unroll
+        for (int j = 0; j < kSketchCols; ++j) y[j] = fma(qv, zs[rr][j], y[j]);
+      }
+    }
+  }
+  unsigned long long t = 0;
+  if (ok) {
+    const uint32_t bit = (sketch_signs(uint32_t(c >> 4)) >> (c & 15)) & 1u;
+#pragma unroll
+    for (int j = 0; j < kSketchCols; ++j) {
+      const double w = j == (c & 15) ? (bit ? -1.0 : 1.0) : 0.0;
+      const double e = y[j] - w;
+      const double sq = fmin(e * e, double(kDevFineClamp));
+      t += static_cast<unsigned long long>(sq * double(kDevFineUnit));
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  if ((threadIdx.x & 31) == 0 && t) atomicAdd(g.devsq, t);
+}
+
+shampoo4_status launch_sketch(const SketchDesc* d_desc, int count, int max_d, int pass, cudaStream_t st) {
+  if (count <= 0 || max_d <= 0) return SHAMPOO4_OK;
+  for (int base = 0; base < count; base += 65535) {
+    const int c = count - base < 65535 ? count - base : 65535;
+    const dim3 grid(unsigned((max_d + 127) / 128), unsigned(c));
+    if (pass == 0)
+      k_sketch_z<<<grid, 128, 0, st>>>(d_desc + base);
+    else
+      k_sketch_r<<<grid, 128, 0, st>>>(d_desc + base);
+    S4_CUDA(cudaGetLastError());
+  }
   return SHAMPOO4_OK;
 }
 

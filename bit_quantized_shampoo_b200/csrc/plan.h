@@ -218,14 +218,11 @@ struct CopyDesc {
 // W_ii <- sum_k X[k, i]^2 (fp64 sums, one thread per column, rounded once
 // to fp32) for i < d, X row-major d x d.  The tensor cores' accumulation
 // truncates, so a Gram's diagonal -- a sum of positive terms -- comes out
-// low by about 1e-8 K relative; this restores it.  devsq (optional, two
-// words): adds the diagonal's share of sum (W_ij - delta_ij)^2, as the GEMM
-// epilogue does for the off-diagonal part (see kDevFineUnit).
+// low by about 1e-8 K relative; this restores it.
 struct DiagDesc {
   const float* X;
   float* W; int64_t ldw;
   int32_t d; int32_t pad_;
-  unsigned long long* devsq;
   const uint32_t* skip;
 };
 
@@ -243,8 +240,9 @@ struct RowDiagDesc {
   float* C; float* Chi; float* Clo;
 };
 
-// Deviation sum sum_ij min((W_ij - delta_ij)^2, 2^-20) of a Gram, in units
-// of 2^-60: an exact integer sum, independent of the order of additions.
+// Deviation sums (the orthogonality sketch below) clamp each square at
+// 2^-20 and add in units of 2^-60: an exact integer sum, independent of the
+// order of additions.
 constexpr float kDevFineClamp = 0x1p-20f, kDevFineUnit = 0x1p60f;
 
 // Inverse of a 128 x 128 lower-triangular diagonal block of L from the
@@ -263,9 +261,28 @@ struct Inv128Desc {
   const uint32_t* skip;
 };
 
-// Decision before the last Cholesky-QR pass of a factor, from the Gram of
-// its input Q: out = 1 (skip the pass) when *bad != 0 or *devsq <= thr (Q
-// already orthonormal to the arithmetic's floor), else 0.
+// Orthogonality sketch of a factor's Q (d x d fp32, row-major, d % 4 == 0),
+// two fp64 passes.  Omega (d x 16) holds one sign per row: Omega[c][c mod
+// 16] = -1 or +1 from bit c mod 16 of the lowbias32 integer mixer of c / 16,
+// zero elsewhere.  Pass one: Z = Q Omega (Z row-major d x 16, fp64).  Pass
+// two: devsq += sum_cj min((Q^T Z - Omega)_cj^2, 2^-20), in units of 2^-60.
+// (Q^T Z - Omega) = E Omega with E = Q^T Q - I, and for independent signs
+// E ||E Omega||_F^2 = ||E||_F^2: the sum estimates the Gram deviation that
+// the gate compares, without the Gram.  One thread per row (pass one) or
+// column (pass two), 128 per CTA.
+constexpr int kSketchCols = 16;
+struct SketchDesc {
+  const float* Q;
+  double* Z;                    // d x 16 scratch
+  unsigned long long* devsq;
+  int32_t d; int32_t pad_;
+  const uint32_t* skip;
+};
+
+// Decision before the last Cholesky-QR pass of a factor, from the deviation
+// of its input Q from orthonormal (the sketch above): out = 1 (skip the
+// pass) when *bad != 0 or *devsq <= thr (Q already orthonormal to the
+// arithmetic's floor), else 0.
 struct GateDesc {
   const unsigned long long* devsq;
   const uint32_t* bad;
@@ -351,6 +368,7 @@ shampoo4_status launch_shift_f(const ShiftDescF* d_desc, int count, cudaStream_t
 shampoo4_status launch_convert(const ConvertDesc* d_desc, int count, int64_t max_elems, cudaStream_t st,
                                const uint32_t* guard = nullptr);
 shampoo4_status launch_gate(const GateDesc* d_desc, int count, cudaStream_t st);
+shampoo4_status launch_sketch(const SketchDesc* d_desc, int count, int max_d, int pass, cudaStream_t st);
 shampoo4_status launch_copy(const CopyDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);
 shampoo4_status launch_newton_norm(const NewtonNormDesc* d_desc, int count, cudaStream_t st);
 shampoo4_status launch_newton_elt(const NewtonEltDesc* d_desc, int count, int64_t max_elems, cudaStream_t st);

@@ -30,7 +30,8 @@ using namespace s4;
 namespace {
 
 enum class Kind { GemmF32, GemmF64, Potrf, Trsm, Basis, Rayleigh, Mu, Scan, Convert, Pack, Shift, GemmTC, GemmTCSplit,
-                  GemmTCSplit64, PotrfF, ShiftF, Gate, Diag, RowDiag, Inv128, Copy, NewtonNorm, NewtonElt };
+                  GemmTCSplit64, PotrfF, ShiftF, Gate, Diag, RowDiag, Inv128, Copy, NewtonNorm, NewtonElt,
+                  SketchZ, SketchR };
 
 struct Launch {
   Kind kind;
@@ -90,6 +91,7 @@ struct FactorPlan {
   size_t ws_W64, ws_Q64, ws_U, ws_T, ws_Y;
   size_t ws_Xm[2], ws_Xh[2], ws_Xl[2], ws_Th, ws_Tl, ws_Sh, ws_Sl, ws_W;
   size_t ws_Zm, ws_Zh, ws_Zl;
+  size_t ws_sketch;                      // d x 16 fp64: the last QR pass's orthogonality sketch
   size_t ws_Ih, ws_Il;                   // 64 x 64 inverse diagonal blocks of L (rows to a multiple of 64)
   size_t ws_Jh, ws_Jl;                   // 128 x 128 inverse diagonal blocks (rows to a multiple of 128)
   size_t ws_q_first, ws_q_next;
@@ -374,6 +376,7 @@ shampoo4_status plan(shampoo4_ctx* h) {
       f.ws_Zm = take(cur, 4 * dd);
       f.ws_Zh = take(cur, 4 * dd);
       f.ws_Zl = take(cur, 4 * dd);
+      f.ws_sketch = take(cur, 8 * size_t(kSketchCols) * f.d);
       // the inverse blocks are written 64 x 64 (zero-padded): rows up to a
       // multiple of 64
       const size_t dpad = align_up(size_t(f.d), kPanelW);
@@ -984,14 +987,16 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
   {
     // Gram W = X^T X (lower triangle: fp32 into W, its TF32 split into
     // Th/Tl), optional shift
-    // The gated pass first runs a Gram that only sums its deviation from I
-    // (no outputs: on warm refreshes every factor passes the gate, so the
-    // matrices would never be read), then the Gram with outputs for the
-    // factors the gate sends through the pass.
-    std::vector<TcGemmDesc> g, gg;
+    // The gated pass first measures how far its input is from orthonormal
+    // by a two-pass fp64 sketch of ||Q^T Q - I||_F (no Gram: on warm
+    // refreshes every factor passes the gate, and a Gram's matrices would
+    // never be read), then runs the Gram with outputs for the factors the
+    // gate sends through the pass.
+    std::vector<TcGemmDesc> g;
     std::vector<ShiftDescF> sd;
     std::vector<GateDesc> gd;
-    std::vector<DiagDesc> dg, dgg;
+    std::vector<DiagDesc> dg;
+    std::vector<SketchDesc> sk;
     for (size_t i = 0; i < nf; ++i) {
       const FactorPlan& f = h->factors[i];
       if (!f.tc) continue;
@@ -1002,10 +1007,7 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
       w.symmetric = 2;
       w.skip = b.tcbad(i);
       if (gated) {
-        TcGemmDesc dev = w;                                           // deviation only
-        dev.devsq = b.devsq(i);
-        gg.push_back(dev);
-        dgg.push_back({X[i].m, b.wf(f.ws_W), d, d, 0, b.devsq(i), b.tcbad(i)});
+        sk.push_back({X[i].m, b.wd(f.ws_sketch), b.devsq(i), d, 0, b.tcbad(i)});
         const double tol = kLastPassTol * std::sqrt(double(d));        // on ||Q^T Q - I||_F / sqrt(d)
         const double thr = std::min(tol * tol * d * double(kDevFineUnit), 0x1p62);
         gd.push_back({b.devsq(i), b.tcbad(i), b.skip3(i), static_cast<unsigned long long>(thr), b.wu(h->ws_p3any)});
@@ -1017,14 +1019,16 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
       w.C = b.wf(f.ws_W); w.ldc = d;
       w.Chi = b.wf(f.ws_Th); w.Clo = b.wf(f.ws_Tl); w.ldh = d;
       g.push_back(w);
-      dg.push_back({X[i].m, b.wf(f.ws_W), d, d, 0, nullptr, gated ? b.skip3(i) : b.tcbad(i)});
+      dg.push_back({X[i].m, b.wf(f.ws_W), d, d, 0, gated ? b.skip3(i) : b.tcbad(i)});
       if (shifted) sd.push_back({b.wf(f.ws_W), d, d, kTcShift * float(d), b.tcbad(i)});
     }
     auto elems = [](const std::vector<DiagDesc>& v) { double s = 0; for (auto& x : v) s += double(x.d) * x.d; return s; };
     if (gated) {
       b.tag = SHAMPOO4_STAGE_QR_GRAM;
-      emit_gemmtc(b, prog, gg, true, kSquareBN);
-      b.emit(prog, Kind::Diag, dgg, dmax, 0, 4.0 * elems(dgg));
+      double sk_elems = 0;
+      for (auto& x : sk) sk_elems += double(x.d) * x.d;
+      b.emit(prog, Kind::SketchZ, sk, dmax, 2.0 * sk_elems, 4.0 * sk_elems);
+      b.emit(prog, Kind::SketchR, sk, dmax, 2.0 * kSketchCols * sk_elems, 4.0 * sk_elems);
       b.tag = SHAMPOO4_STAGE_QR_CONVERT;
       b.emit(prog, Kind::Gate, gd, 0);
       // the rest of the pass runs only if some factor goes through it
@@ -1937,6 +1941,11 @@ shampoo4_status run(shampoo4_ctx* h, const std::vector<Launch>& prog, cudaStream
         break;
       case Kind::Diag:
         S4_TRY(launch_diag(static_cast<const DiagDesc*>(d), L.count, int(L.extent), st, guard));
+        break;
+      case Kind::SketchZ:
+      case Kind::SketchR:
+        S4_TRY(launch_sketch(static_cast<const SketchDesc*>(d), L.count, int(L.extent),
+                             L.kind == Kind::SketchZ ? 0 : 1, st));
         break;
       case Kind::Inv128:
         S4_TRY(launch_inv128(static_cast<const Inv128Desc*>(d), L.count, st, guard));

@@ -50,10 +50,6 @@ struct TcGemmDesc {
   const float* Cin; int64_t ldcin;
   const uint32_t* skip;
   OperandRef c_ref;
-  // optional: the off-diagonal share (strictly-lower elements counted twice
-  // when symmetric) of the deviation sum of plan.h; the diagonal's share
-  // comes from the diagonal kernel
-  unsigned long long* devsq;
   const CUtensorMap* bt_hi;
   const CUtensorMap* bt_lo;
   const CUtensorMap* at_hi;
