@@ -166,9 +166,9 @@ STAGE_BOUND = {
 # factors of the same kind moves the same bytes per element.  Valid only for
 # the GEMM source it was taken on: the figure is dropped (traffic = null) when
 # gemm_tc.cu or tc.h has changed since.
-TRAFFIC_SOURCE_SHA = "40af43b2b2540035"
-TRAFFIC_PER_ELEMENT = {"stats_gemm": 6.610, "bjorck_gram": 5.434, "bjorck_update": 10.704,
-                       "subspace": 32.668, "qr_gram": 13.148}
+TRAFFIC_SOURCE_SHA = "6c7fb2eaf26f9bd9"
+TRAFFIC_PER_ELEMENT = {"stats_gemm": 6.589, "bjorck_gram": 5.469, "bjorck_update": 10.482,
+                       "subspace": 32.758, "qr_gram": 13.184}
 
 
 def gemm_source_sha():

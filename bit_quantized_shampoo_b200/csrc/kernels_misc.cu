@@ -789,12 +789,20 @@ __global__ void __launch_bounds__(128) k_sketch_r(const SketchDesc* __restrict__
       zs[e / kSketchCols][e % kSketchCols] = g.Z[int64_t(r0) * kSketchCols + e];
     __syncthreads();
     if (ok) {
+      // eight rows' loads in flight before their products (the pass is
+      // bound by the latency of these column reads otherwise)
       const float* qc = g.Q + int64_t(r0) * d + c;
-#pragma unroll 4
-      for (int rr = 0; rr < nr; ++rr) {
-        const double qv = double(qc[int64_t(rr) * d]);
+      for (int rr = 0; rr < nr; rr += 8) {
+        float qv[8];
 #pragma unroll
-        for (int j = 0; j < kSketchCols; ++j) y[j] = fma(qv, zs[rr][j], y[j]);
+        for (int u = 0; u < 8; ++u) qv[u] = rr + u < nr ? qc[int64_t(rr + u) * d] : 0.0f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (rr + u >= nr) break;                          // rows past nr hold no staged Z
+          const double qd = double(qv[u]);
+#pragma unroll
+          for (int j = 0; j < kSketchCols; ++j) y[j] = fma(qd, zs[rr + u][j], y[j]);
+        }
       }
     }
   }
