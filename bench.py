@@ -167,8 +167,11 @@ STAGE_BOUND = {
 # the GEMM source it was taken on: the figure is dropped (traffic = null) when
 # gemm_tc.cu or tc.h has changed since.
 TRAFFIC_SOURCE_SHA = "6c7fb2eaf26f9bd9"
+# (The QR Gram stage is left out: its first-pass Gram runs in TF32 since
+# that capture, and the fp32-accurate second-pass Gram moves 13.18 B per
+# element, so no single per-launch figure describes the stage.)
 TRAFFIC_PER_ELEMENT = {"stats_gemm": 6.589, "bjorck_gram": 5.469, "bjorck_update": 10.482,
-                       "subspace": 32.758, "qr_gram": 13.184}
+                       "subspace": 32.758}
 
 
 def gemm_source_sha():

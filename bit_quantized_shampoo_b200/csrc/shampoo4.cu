@@ -952,13 +952,23 @@ void build_cholqr_pass(Builder& b, std::vector<Launch>& prog, const std::vector<
 // pass succeeds when that is below about 1e3.  Factors beyond that break
 // down in a Cholesky panel and are redone in fp64 from the intact Y.
 //
+// The first pass only preconditions: with any triangular L1, Q0 = X L1^-T
+// and the later passes' factors give Y = Q R with R = L3^T L2^T L1^T, so
+// the final Q does not depend on how well L1 factors X^T X, as long as the
+// solve uses that same L1 accurately.  Its Gram therefore runs in TF32
+// (operands rounded once, fp32 accumulation, exact diagonal): in the
+// equilibrated frame that errs by about 2^-11 sqrt(2 / 3d) per off-diagonal
+// element, some 8e-4 in 2-norm at d = 1024, well under the shift; what the
+// shift leaves of Q0's orthogonality dominates either way.  Its Cholesky,
+// its solve and the later passes stay fp32-accurate.
+//
 // A warm subspace step (U from the previous refresh) has Y = (S + eps I) U
 // with nearly orthogonal columns of very different lengths: X D^-1 is close
 // to orthonormal, and two passes already reach the orthogonality floor of
 // this arithmetic (||Q^T Q - I||_F / sqrt(d) near 1.1e-7 sqrt(d), set by
 // the unbiased rounding of the off-diagonal sums).  So the third pass is
-// gated per factor: its Gram also measures ||Q^T Q - I||_F of the second
-// pass's output; its Cholesky and solve run only when that exceeds
+// gated per factor: a two-pass fp64 sketch estimates ||Q^T Q - I||_F of the
+// second pass's output; its Cholesky and solve run only when that exceeds
 // kLastPassTol sqrt(d) * sqrt(d) (a cold first refresh needs them).  In that
 // pass a Cholesky pivot at or below kLastPassPivot -- a column of the
 // (unit-column) input nearly in the span of the previous ones, so that the
@@ -984,6 +994,7 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
   int dmax = 0;
   for (auto& f : h->factors) if (f.tc) dmax = std::max(dmax, f.d);
   if (dmax == 0) return;
+  const bool tf32_gram = shifted;          // the first pass only preconditions (above)
   {
     // Gram W = X^T X (lower triangle: fp32 into W, its TF32 split into
     // Th/Tl), optional shift
@@ -1002,8 +1013,9 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
       if (!f.tc) continue;
       const int d = f.d;
       TcGemmDesc w = gemmtc(d, d, d, 1.0f, 0.0f);
-      w.a = b.operand(X[i].h, X[i].l, d, d, true, true, true);
-      w.b = b.operand(X[i].h, X[i].l, d, d, false, false, true, kSquareBN);
+      w.a = b.operand(X[i].h, tf32_gram ? nullptr : X[i].l, d, d, true, true, !tf32_gram);
+      w.b = b.operand(X[i].h, tf32_gram ? nullptr : X[i].l, d, d, false, false, !tf32_gram,
+                      tf32_gram ? 0 : kSquareBN);
       w.symmetric = 2;
       w.skip = b.tcbad(i);
       if (gated) {
@@ -1035,7 +1047,7 @@ void build_cholqr_tc(Builder& b, std::vector<Launch>& prog, const std::vector<Tr
       b.guard = h->ws_p3any;
     }
     b.tag = SHAMPOO4_STAGE_QR_GRAM;
-    emit_gemmtc(b, prog, g, true, kSquareBN);
+    emit_gemmtc(b, prog, g, !tf32_gram, tf32_gram ? 0 : kSquareBN);
     b.emit(prog, Kind::Diag, dg, dmax, 0, 4.0 * elems(dg));
     b.emit(prog, Kind::ShiftF, sd, 0);
   }

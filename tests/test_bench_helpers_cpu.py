@@ -50,10 +50,11 @@ def test_every_library_stage_has_a_bound():
 def test_traffic_is_reported_only_for_the_captured_gemm_source(monkeypatch):
     n = 1 << 20
     monkeypatch.setattr(bench, "TRAFFIC_SOURCE_SHA", bench.gemm_source_sha())
-    assert bench.stage_traffic("qr_gram", n) == pytest.approx(bench.TRAFFIC_PER_ELEMENT["qr_gram"] * n)
+    assert bench.stage_traffic("subspace", n) == pytest.approx(bench.TRAFFIC_PER_ELEMENT["subspace"] * n)
     assert bench.stage_traffic("roots", n) is None                    # no capture covers it
+    assert bench.stage_traffic("qr_gram", n) is None                  # two kinds of launch, no one figure
     monkeypatch.setattr(bench, "TRAFFIC_SOURCE_SHA", "0" * 16)
-    assert bench.stage_traffic("qr_gram", n) is None                  # source changed since the capture
+    assert bench.stage_traffic("subspace", n) is None                 # source changed since the capture
 
 
 def test_measured_peaks_are_read_else_the_fallback():
