@@ -410,6 +410,7 @@ def measure_config(wid, dev, args, pk, pk_src, world):
         step()
     cycles = max(1, (20 + T - 1) // T) if T > 1 else 20
     torch.cuda.synchronize()
+    warmup_flags = sh.status_flags()         # the cold first refresh's, cleared
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(cycles * T):
@@ -430,7 +431,7 @@ def measure_config(wid, dev, args, pk, pk_src, world):
     res = {"workload": w.name, "tiles": sh.nblocks, "factors": sh.nfactors, "refresh_every": T,
            "steps_timed": cycles * T, "ms_per_step": ms, "us_per_step": ms * 1e3,
            "steps_per_s": world * 1e3 / ms, "refresh_ms": rms, "root_refreshes_per_s": world * sh.nfactors * 1e3 / rms,
-           "status_flags": sh.status_flags(),
+           "status_flags": sh.status_flags(), "warmup_status_flags": warmup_flags,
            "roofline": formula_roofline(step_work(dims, w.bjorck_iters, T, args.precision), ms / 1e3, pk, pk_src,
                                         f"step at T = {T}, algorithmic flops of the work model"),
            "workspace_bytes": sh.workspace_bytes, "state_bytes": sh.state_bytes}
@@ -461,6 +462,7 @@ def measure_variant(wid, dev, args, pk, pk_src, world, **kw):
     for i in range(3):
         step(i)
     torch.cuda.synchronize()
+    warmup_flags = sh.status_flags()         # the cold first refresh's, cleared
     reps = 5
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     ev[0].record(stream)
@@ -474,7 +476,7 @@ def measure_variant(wid, dev, args, pk, pk_src, world, **kw):
     ms = max_over_ranks(ev[0].elapsed_time(ev[1]), dev) / reps
     rms = max_over_ranks(ev[1].elapsed_time(ev[2]), dev) / reps
     res = {"ms_per_step": ms, "refresh_ms": rms, "root_refreshes_per_s": world * sh.nfactors * 1e3 / rms,
-           "state_bytes": sh.state_bytes, "status_flags": sh.status_flags()}
+           "state_bytes": sh.state_bytes, "status_flags": sh.status_flags(), "warmup_status_flags": warmup_flags}
     del sh, sets, out
     return res
 
@@ -544,6 +546,10 @@ def main():
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    # the latched flags of the warm-up (its first refresh is the cold one,
+    # from U = I) are read and cleared here, so the line's status_flags
+    # describe the steps after it
+    warmup_flags = sh.status_flags()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -639,7 +645,7 @@ def main():
                        "l2": (f"inputs larger than L2 ({g_bytes / 1e9:.2f} GB of G, {stat_bytes / 1e9:.2f} GB "
                               f"of fp32 statistics; L2 is 0.126 GB)")},
             "root_refreshes_per_s": value * sh.nfactors,
-            "status_flags": status,
+            "status_flags": status, "warmup_status_flags": warmup_flags,
             "gpu_launches": launches * args.steps,
             "clocks": clocks, "roofline": roof, "rooflines_other": others,
             "stages_ms": {k: round(v["ms"], 4) for k, v in sorted(stages.items(), key=lambda kv: -kv[1]["ms"])},
